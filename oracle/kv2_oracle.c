@@ -1,0 +1,651 @@
+/*
+ * kv2_oracle.c — plain, slow CPU oracle of the 2-bit KV-cache path.
+ *
+ * TEST INFRASTRUCTURE ONLY. Only the tests, the smoke check and the benchmark's
+ * CPU-baseline leg may load this file's library; the product path never does.
+ * It shares no code, header or table with the CUDA library.
+ *
+ * Source of the method: "QuantWM: Training-Free 2-bit KV Cache Quantization for
+ * Stable Video World Models" (besthub.dev article), sections
+ *   "1. Quantization Sensitivity-Aware Clustering (QSAC)" and
+ *   "2. Principal Subspace Attention Compensation (PSAC)".
+ * The pages leave the exact formulas open; every reading taken here is the one
+ * written out below and in the design notes (codec, ranking score, perturbation
+ * estimate, coefficient precision, sign and order of eigenvectors).
+ *
+ * Precision: quantizer decisions (centroid choice, INT2 codes, fp16 scale and
+ * zero) are taken in fp32 in the stated operation order, using fmaf only where
+ * stated (compile with -ffp-contract=off). Eigen-decomposition and attention are
+ * fp64. 16-bit float conversions are written from the IEEE 754 definition.
+ *
+ * Parity pins (tests/test_oracle_*.py): rounding functions vs numpy/torch casts
+ * and directed-rounding brackets; codec invariants and per-element brute force;
+ * QSAC vs brute-force argmin (candidates = M) and vs plain nearest centre
+ * (candidates = 1, unit weights); PSAC r = d and r = 0 closed forms; Jacobi vs
+ * numpy.linalg.eigh; attention vs a two-pass softmax and a centroid-only closed
+ * form. Parity unpinned: whether the perturbation estimate is the authors' exact
+ * heuristic (the pages print no worked example).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define GROUP 32
+
+/* ------------------------------------------------------------------------ */
+/* IEEE 754 binary16 / bfloat16                                             */
+/* ------------------------------------------------------------------------ */
+
+enum { RND_NEAREST_EVEN = 0, RND_DOWN = 1, RND_UP = 2 };
+
+/* Round a finite or infinite double to a binary format with `man` fraction
+ * bits, minimum normal exponent `emin` and largest finite value `maxf`, under
+ * the given rounding mode. Returns the rounded value as a double (exact). */
+static double round_to_format(double x, int man, int emin, double maxf, int mode)
+{
+    if (isnan(x)) return x;
+    int neg = signbit(x) != 0;
+    double a = fabs(x);
+    if (isinf(a)) return x;
+    if (a == 0.0) return x;
+    int e2;
+    frexp(a, &e2);                 /* a in [2^(e2-1), 2^e2) */
+    int e = e2 - 1;                /* floor(log2 a) */
+    if (e < emin) e = emin;        /* subnormal range shares the emin quantum */
+    double quantum = ldexp(1.0, e - man);
+    double n = a / quantum;        /* exact: division by a power of two */
+    double k;
+    if (mode == RND_NEAREST_EVEN) {
+        double f = floor(n), rem = n - f;
+        if (rem > 0.5) k = f + 1.0;
+        else if (rem < 0.5) k = f;
+        else k = (fmod(f, 2.0) == 0.0) ? f : f + 1.0;
+    } else {
+        /* magnitude toward zero for (down, positive) and (up, negative) */
+        int toward_zero = (mode == RND_DOWN) ? !neg : neg;
+        k = toward_zero ? floor(n) : ceil(n);
+    }
+    double r = k * quantum;
+    if (r > maxf) {
+        int toward_zero = (mode == RND_NEAREST_EVEN) ? 0 : ((mode == RND_DOWN) ? !neg : neg);
+        r = toward_zero ? maxf : INFINITY;
+    }
+    return neg ? -r : r;
+}
+
+static const double F16_MAX = 65504.0;
+
+static uint16_t f16_encode_exact(double r)
+{
+    /* r is already representable in binary16 (or +-inf / nan) */
+    uint16_t sign = signbit(r) ? 0x8000u : 0u;
+    double a = fabs(r);
+    if (isnan(r)) return 0x7e00u;
+    if (isinf(a)) return (uint16_t)(sign | 0x7c00u);
+    if (a == 0.0) return sign;
+    if (a < ldexp(1.0, -14)) return (uint16_t)(sign | (uint16_t)(a / ldexp(1.0, -24)));
+    int e2;
+    frexp(a, &e2);
+    int e = e2 - 1;
+    uint16_t mant = (uint16_t)(a / ldexp(1.0, e - 10) - 1024.0);
+    return (uint16_t)(sign | ((uint16_t)(e + 15) << 10) | mant);
+}
+
+uint16_t or_f16_from_f32(float x, int mode)
+{
+    return f16_encode_exact(round_to_format((double)x, 10, -14, F16_MAX, mode));
+}
+
+float or_f32_from_f16(uint16_t h)
+{
+    int neg = (h >> 15) & 1, e = (h >> 10) & 0x1f, m = h & 0x3ff;
+    double v;
+    if (e == 0) v = ldexp((double)m, -24);
+    else if (e == 31) v = m ? NAN : INFINITY;
+    else v = ldexp((double)(m | 0x400), e - 25);
+    return (float)(neg ? -v : v);
+}
+
+float or_f32_from_bf16(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+uint16_t or_bf16_from_f32(float x)
+{
+    if (isnan(x)) return 0x7fc0u;
+    double bmax = ldexp(2.0 - ldexp(1.0, -7), 127);
+    float r = (float)round_to_format((double)x, 7, -126, bmax, RND_NEAREST_EVEN);
+    uint32_t u;
+    memcpy(&u, &r, 4);
+    return (uint16_t)(u >> 16);
+}
+
+/* ------------------------------------------------------------------------ */
+/* INT2 group codec                                                          */
+/*   QuantWM article, "1. QSAC": the centre-relative residual is quantized to  */
+/*   2 bits; the cache stores an fp16 scale and an fp16 zero per group of 32    */
+/*   channels (asymmetric INT2). Reading taken: zero = the group minimum       */
+/*   rounded down to fp16, scale = (max - zero)/3 rounded up to fp16, so that  */
+/*   [zero, zero + 3 scale] covers the group; codes round half to even.        */
+/* ------------------------------------------------------------------------ */
+
+static void codec_params(const float* x, int n, uint16_t* s_bits, uint16_t* z_bits)
+{
+    float mn = x[0], mx = x[0];
+    for (int i = 1; i < n; ++i) {
+        if (x[i] < mn) mn = x[i];
+        if (x[i] > mx) mx = x[i];
+    }
+    uint16_t zb = or_f16_from_f32(mn, RND_DOWN);
+    float z = or_f32_from_f16(zb);
+    float range = mx - z;              /* fp32, round to nearest */
+    float q = range / 3.0f;            /* fp32 correctly rounded division */
+    *z_bits = zb;
+    *s_bits = or_f16_from_f32(q, RND_UP);
+}
+
+static uint32_t codec_code(float x, float s, float z)
+{
+    if (s == 0.0f) return 0u;
+    float t = (x - z) / s;             /* fp32 subtraction, fp32 division */
+    float c = rintf(t);                /* round half to even */
+    if (c < 0.0f) c = 0.0f;
+    if (c > 3.0f) c = 3.0f;
+    return (uint32_t)c;
+}
+
+static float codec_dequant(uint32_t code, float s, float z)
+{
+    return fmaf((float)code, s, z);
+}
+
+/* exported for the tests: one group of n values */
+void or_codec_group(const float* x, int n, uint16_t* s_bits, uint16_t* z_bits,
+                    uint8_t* codes, float* deq)
+{
+    codec_params(x, n, s_bits, z_bits);
+    float s = or_f32_from_f16(*s_bits), z = or_f32_from_f16(*z_bits);
+    for (int i = 0; i < n; ++i) {
+        codes[i] = (uint8_t)codec_code(x[i], s, z);
+        if (deq) deq[i] = codec_dequant(codes[i], s, z);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* PSAC basis fit (article section "2. PSAC": historical Query energy          */
+/* concentrates in a few principal directions; QSAC's sensitivity weights are  */
+/* the per-channel Query energy).                                              */
+/*   S = (1/N) sum q q^T over the N = n*G history queries of the KV head's     */
+/*   query-head group (uncentred second moment), w_c = S_cc, W_g = sum of w_c   */
+/*   over the group's channels (fp32, ascending c), P = top-r eigenvectors of S */
+/*   (eigenvalues descending, each vector's largest-magnitude entry positive).  */
+/* ------------------------------------------------------------------------ */
+
+/* cyclic Jacobi eigen-decomposition of a symmetric n x n matrix A (destroyed);
+ * eigenvalues on return in A's diagonal, eigenvectors in the columns of V */
+static void jacobi_eigen(double* A, double* V, int n)
+{
+    for (int i = 0; i < n; ++i)
+        for (int j = 0; j < n; ++j) V[i * n + j] = (i == j) ? 1.0 : 0.0;
+    double total = 0.0;
+    for (int i = 0; i < n * n; ++i) total += A[i] * A[i];
+    for (int sweep = 0; sweep < 100; ++sweep) {
+        double off = 0.0;
+        for (int p = 0; p < n; ++p)
+            for (int q = p + 1; q < n; ++q) off += 2.0 * A[p * n + q] * A[p * n + q];
+        if (off <= 1e-28 * total || off == 0.0) break;
+        for (int p = 0; p < n - 1; ++p) {
+            for (int q = p + 1; q < n; ++q) {
+                double apq = A[p * n + q];
+                if (apq == 0.0) continue;
+                double app = A[p * n + p], aqq = A[q * n + q];
+                double theta = (aqq - app) / (2.0 * apq);
+                double t = (theta >= 0.0 ? 1.0 : -1.0) / (fabs(theta) + sqrt(theta * theta + 1.0));
+                double c = 1.0 / sqrt(t * t + 1.0), s = t * c;
+                /* A <- J^T A J with J the rotation in the (p, q) plane */
+                for (int k = 0; k < n; ++k) {
+                    double akp = A[k * n + p], akq = A[k * n + q];
+                    A[k * n + p] = c * akp - s * akq;
+                    A[k * n + q] = s * akp + c * akq;
+                }
+                for (int k = 0; k < n; ++k) {
+                    double apk = A[p * n + k], aqk = A[q * n + k];
+                    A[p * n + k] = c * apk - s * aqk;
+                    A[q * n + k] = s * apk + c * aqk;
+                }
+                for (int k = 0; k < n; ++k) {
+                    double vkp = V[k * n + p], vkq = V[k * n + q];
+                    V[k * n + p] = c * vkp - s * vkq;
+                    V[k * n + q] = s * vkp + c * vkq;
+                }
+            }
+        }
+    }
+}
+
+int or_fit(const uint16_t* Qh, int n, int Hq, int Hkv, int d, int r,
+           float* P, float* w, float* Wg, double* evals, double* energy)
+{
+    if (Hkv <= 0 || Hq % Hkv || d % GROUP || r < 0 || r > d || n <= 0) return 1;
+    int G = Hq / Hkv, ng = d / GROUP;
+    double* S = (double*)calloc((size_t)d * d, sizeof(double));
+    double* Vec = (double*)malloc((size_t)d * d * sizeof(double));
+    double* lam = (double*)malloc((size_t)d * sizeof(double));
+    int* order = (int*)malloc((size_t)d * sizeof(int));
+    double* q = (double*)malloc((size_t)d * sizeof(double));
+    for (int h = 0; h < Hkv; ++h) {
+        memset(S, 0, (size_t)d * d * sizeof(double));
+        for (int t = 0; t < n; ++t)
+            for (int g = 0; g < G; ++g) {
+                const uint16_t* qr = Qh + ((size_t)t * Hq + (size_t)h * G + g) * d;
+                for (int c = 0; c < d; ++c) q[c] = or_f32_from_bf16(qr[c]);
+                for (int a = 0; a < d; ++a)
+                    for (int b = 0; b < d; ++b) S[a * d + b] += q[a] * q[b];
+            }
+        double N = (double)n * G;
+        for (int i = 0; i < d * d; ++i) S[i] /= N;
+        for (int c = 0; c < d; ++c) w[(size_t)h * d + c] = (float)S[c * d + c];
+        for (int g = 0; g < ng; ++g) {
+            float acc = 0.0f;
+            for (int c = g * GROUP; c < (g + 1) * GROUP; ++c) acc = acc + w[(size_t)h * d + c];
+            Wg[(size_t)h * ng + g] = acc;
+        }
+        jacobi_eigen(S, Vec, d);
+        for (int i = 0; i < d; ++i) { lam[i] = S[i * d + i]; order[i] = i; }
+        /* eigenvalues descending; equal values keep the lower index first */
+        for (int i = 1; i < d; ++i) {
+            int o = order[i], j = i - 1;
+            while (j >= 0 && lam[order[j]] < lam[o]) { order[j + 1] = order[j]; --j; }
+            order[j + 1] = o;
+        }
+        double tot = 0.0, top = 0.0;
+        for (int i = 0; i < d; ++i) tot += lam[i];
+        for (int i = 0; i < r; ++i) top += lam[order[i]];
+        if (energy) energy[h] = tot > 0.0 ? top / tot : 0.0;
+        if (evals)
+            for (int i = 0; i < d; ++i) evals[(size_t)h * d + i] = lam[order[i]];
+        for (int i = 0; i < r; ++i) {
+            int col = order[i];
+            int arg = 0;
+            for (int c = 1; c < d; ++c)
+                if (fabs(Vec[c * d + col]) > fabs(Vec[arg * d + col])) arg = c;
+            double sg = Vec[arg * d + col] < 0.0 ? -1.0 : 1.0;
+            for (int c = 0; c < d; ++c)
+                P[((size_t)h * d + c) * r + i] = (float)(sg * Vec[c * d + col]);
+        }
+    }
+    free(S); free(Vec); free(lam); free(order); free(q);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* QSAC + INT2 packing + PSAC coefficients for appended tokens.               */
+/*   Ranking (article "1. QSAC": candidates by a Query-sensitivity-weighted    */
+/*   distance): D_j = sum_c w_c (k_c - mu_jc)^2. The key's own weighted norm   */
+/*   sum_c w_c k_c^2 is the same for every j, so the ranking score is          */
+/*       score_j = nrm_j - 2 dot_j,                                            */
+/*       nrm_j = sum_c (w_c mu_jc) mu_jc,   dot_j = sum_c (w_c k_c) mu_jc,     */
+/*   each sum an fp32 fmaf chain over ascending c starting from 0, the         */
+/*   products w_c mu_jc and w_c k_c rounded to fp32 first, and                 */
+/*   score_j = fmaf(-2, dot_j, nrm_j). Candidates: the C smallest (score, j).  */
+/*   Choice (same section: estimated perturbation from the residual group's    */
+/*   dynamic range and its sensitivity): E_j = sum_g (W_g s_g) s_g, an fp32     */
+/*   fmaf chain over ascending g with s_g the group's fp16 scale; the least E  */
+/*   wins, ties to the earlier candidate.                                      */
+/*   PSAC coefficients (article "2. PSAC"): a_i = sum_c P_ci e_c with          */
+/*   e = residual - dequantized residual, an fp32 fmaf chain over ascending c, */
+/*   stored as fp16 (round to nearest even).                                   */
+/* Layouts: K, V bf16 [B][n_new][Hkv][d]; centroids fp16 [Hkv][M][d];          */
+/* P [Hkv][d][r]; w [Hkv][d]; Wg [Hkv][d/32]; packed streams as in the         */
+/* library: [B][Hkv][cap][...].                                              */
+/* ------------------------------------------------------------------------ */
+
+static uint32_t pack_word(const uint32_t* codes16)
+{
+    uint32_t w = 0;
+    for (int i = 0; i < 16; ++i) w |= (codes16[i] & 3u) << (2 * i);
+    return w;
+}
+
+static void quantize_row(const float* x, int d, uint32_t* code_words, uint32_t* sz, float* deq)
+{
+    uint32_t codes[16];
+    for (int g = 0; g < d / GROUP; ++g) {
+        uint16_t sb, zb;
+        codec_params(x + g * GROUP, GROUP, &sb, &zb);
+        float s = or_f32_from_f16(sb), z = or_f32_from_f16(zb);
+        sz[g] = (uint32_t)sb | ((uint32_t)zb << 16);
+        for (int half = 0; half < 2; ++half) {
+            for (int i = 0; i < 16; ++i) {
+                int c = g * GROUP + half * 16 + i;
+                codes[i] = codec_code(x[c], s, z);
+                if (deq) deq[c] = codec_dequant(codes[i], s, z);
+            }
+            code_words[(g * GROUP + half * 16) / 16] = pack_word(codes);
+        }
+    }
+}
+
+int or_quantize(int B, int Hkv, int d, int M, int r, int cap,
+                const uint16_t* K, const uint16_t* V, int n_new, int pos, int C,
+                const uint16_t* cent, const float* P, const float* w, const float* Wg,
+                uint32_t* k_code, uint32_t* v_code, uint32_t* k_sz, uint32_t* v_sz,
+                void* cidx, uint16_t* psac,
+                int32_t* cand_out, float* score_out, float* E_out)
+{
+    if (d % GROUP || C < 1 || C > M || pos < 0 || pos + n_new > cap) return 1;
+    int ng = d / GROUP, nw = d / 16;
+    float* mu = (float*)malloc((size_t)M * d * sizeof(float));
+    float* nrm = (float*)malloc((size_t)M * sizeof(float));
+    float* score = (float*)malloc((size_t)M * sizeof(float));
+    int* cand = (int*)malloc((size_t)C * sizeof(int));
+    float* k = (float*)malloc((size_t)d * sizeof(float));
+    float* wk = (float*)malloc((size_t)d * sizeof(float));
+    float* x = (float*)malloc((size_t)d * sizeof(float));
+    float* deq = (float*)malloc((size_t)d * sizeof(float));
+    float* xbest = (float*)malloc((size_t)d * sizeof(float));
+    uint32_t* cw = (uint32_t*)malloc((size_t)nw * sizeof(uint32_t));
+    uint32_t* szr = (uint32_t*)malloc((size_t)ng * sizeof(uint32_t));
+    char* used = (char*)malloc((size_t)M);
+    for (int h = 0; h < Hkv; ++h) {
+        const float* wh = w + (size_t)h * d;
+        for (int j = 0; j < M; ++j) {
+            float acc = 0.0f;
+            for (int c = 0; c < d; ++c) {
+                float m = or_f32_from_f16(cent[((size_t)h * M + j) * d + c]);
+                mu[(size_t)j * d + c] = m;
+                float wm = wh[c] * m;
+                acc = fmaf(wm, m, acc);
+            }
+            nrm[j] = acc;
+        }
+        for (int b = 0; b < B; ++b) {
+            for (int t = 0; t < n_new; ++t) {
+                size_t in = (((size_t)b * n_new + t) * Hkv + h) * d;
+                size_t slot = ((size_t)b * Hkv + h) * cap + (size_t)(pos + t);
+                size_t dbg = (((size_t)b * n_new + t) * Hkv + h);
+                for (int c = 0; c < d; ++c) {
+                    k[c] = or_f32_from_bf16(K[in + c]);
+                    wk[c] = wh[c] * k[c];
+                }
+                /* ranking */
+                for (int j = 0; j < M; ++j) {
+                    float dot = 0.0f;
+                    const float* m = mu + (size_t)j * d;
+                    for (int c = 0; c < d; ++c) dot = fmaf(wk[c], m[c], dot);
+                    score[j] = fmaf(-2.0f, dot, nrm[j]);
+                }
+                memset(used, 0, (size_t)M);
+                for (int i = 0; i < C; ++i) {
+                    int best = -1;
+                    for (int j = 0; j < M; ++j) {
+                        if (used[j]) continue;
+                        if (best < 0 || score[j] < score[best]) best = j;
+                    }
+                    used[best] = 1;
+                    cand[i] = best;
+                    if (cand_out) cand_out[dbg * C + i] = best;
+                    if (score_out) score_out[dbg * C + i] = score[best];
+                }
+                /* choice by estimated perturbation */
+                int chosen = -1;
+                float bestE = 0.0f;
+                for (int i = 0; i < C; ++i) {
+                    int j = cand[i];
+                    const float* m = mu + (size_t)j * d;
+                    for (int c = 0; c < d; ++c) x[c] = k[c] - m[c];
+                    float E = 0.0f;
+                    for (int g = 0; g < ng; ++g) {
+                        uint16_t sb, zb;
+                        codec_params(x + g * GROUP, GROUP, &sb, &zb);
+                        float s = or_f32_from_f16(sb);
+                        float ws = Wg[(size_t)h * ng + g] * s;
+                        E = fmaf(ws, s, E);
+                    }
+                    if (E_out) E_out[dbg * C + i] = E;
+                    if (chosen < 0 || E < bestE) {
+                        chosen = j;
+                        bestE = E;
+                        memcpy(xbest, x, (size_t)d * sizeof(float));
+                    }
+                }
+                /* residual codes, scales, zeros */
+                quantize_row(xbest, d, cw, szr, deq);
+                memcpy(k_code + slot * nw, cw, (size_t)nw * 4);
+                memcpy(k_sz + slot * ng, szr, (size_t)ng * 4);
+                if (M <= 256) ((uint8_t*)cidx)[slot] = (uint8_t)chosen;
+                else ((uint16_t*)cidx)[slot] = (uint16_t)chosen;
+                /* PSAC coefficients of the key's quantization error */
+                for (int i = 0; i < r; ++i) {
+                    float a = 0.0f;
+                    for (int c = 0; c < d; ++c) {
+                        float e = xbest[c] - deq[c];
+                        a = fmaf(P[((size_t)h * d + c) * r + i], e, a);
+                    }
+                    psac[slot * (size_t)r + i] = or_f16_from_f32(a, RND_NEAREST_EVEN);
+                }
+                /* values: same codec, no centre */
+                for (int c = 0; c < d; ++c) x[c] = or_f32_from_bf16(V[in + c]);
+                quantize_row(x, d, cw, szr, NULL);
+                memcpy(v_code + slot * nw, cw, (size_t)nw * 4);
+                memcpy(v_sz + slot * ng, szr, (size_t)ng * 4);
+            }
+        }
+    }
+    free(mu); free(nrm); free(score); free(cand); free(k); free(wk); free(x);
+    free(deq); free(xbest); free(cw); free(szr); free(used);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Attention over the packed cache (fp64).                                    */
+/*   logit_t = scale * (q . khat_t + (q P) . a_t), khat_t = mu_idx + deq_t:    */
+/*   the PSAC term is the Key compensation of article "2. PSAC" applied to the */
+/*   score, q.(khat + P a) = q.khat + (qP).a. Softmax in two passes.           */
+/*   Decode: dequantized values are exact (mu + code s + z in fp64), matching   */
+/*   a kernel that never rounds them. Chunk: the kernel's operand precision:   */
+/*   khat = bf16(fp32(fmaf(code, s, z) + mu)), vhat = fp16(fmaf(code, s, z)),  */
+/*   u = qP as fp16, self keys bf16, self values as fp16.                      */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    int B, Hkv, d, M, r, cap;
+    const uint32_t *k_code, *v_code, *k_sz, *v_sz;
+    const void* cidx;
+    const uint16_t *psac, *cent;
+    const float* P;
+} or_cache;
+
+static int cache_idx(const or_cache* c, size_t slot)
+{
+    return c->M <= 256 ? ((const uint8_t*)c->cidx)[slot] : ((const uint16_t*)c->cidx)[slot];
+}
+
+static uint32_t code_at(const uint32_t* words, int ch)
+{
+    return (words[ch / 16] >> (2 * (ch % 16))) & 3u;
+}
+
+/* exact dequantized key/value rows of one token (decode precision) */
+static void dequant_exact(const or_cache* c, size_t slot, double* kh, double* vh)
+{
+    int d = c->d, ng = d / GROUP;
+    const uint32_t* kw = c->k_code + slot * (d / 16);
+    const uint32_t* vw = c->v_code + slot * (d / 16);
+    int j = cache_idx(c, slot);
+    int h = (int)((slot / (size_t)c->cap) % (size_t)c->Hkv);
+    for (int g = 0; g < ng; ++g) {
+        uint32_t ks = c->k_sz[slot * ng + g], vs = c->v_sz[slot * ng + g];
+        double s = or_f32_from_f16((uint16_t)(ks & 0xffff)), z = or_f32_from_f16((uint16_t)(ks >> 16));
+        double sv = or_f32_from_f16((uint16_t)(vs & 0xffff)), zv = or_f32_from_f16((uint16_t)(vs >> 16));
+        for (int ch = g * GROUP; ch < (g + 1) * GROUP; ++ch) {
+            double m = or_f32_from_f16(c->cent[((size_t)h * c->M + j) * d + ch]);
+            kh[ch] = m + (double)code_at(kw, ch) * s + z;
+            vh[ch] = (double)code_at(vw, ch) * sv + zv;
+        }
+    }
+}
+
+/* operand-precision dequantized rows (chunk kernel precision) */
+static void dequant_operand(const or_cache* c, size_t slot, double* kh, double* vh)
+{
+    int d = c->d, ng = d / GROUP;
+    const uint32_t* kw = c->k_code + slot * (d / 16);
+    const uint32_t* vw = c->v_code + slot * (d / 16);
+    int j = cache_idx(c, slot);
+    int h = (int)((slot / (size_t)c->cap) % (size_t)c->Hkv);
+    for (int g = 0; g < ng; ++g) {
+        uint32_t ks = c->k_sz[slot * ng + g], vs = c->v_sz[slot * ng + g];
+        float s = or_f32_from_f16((uint16_t)(ks & 0xffff)), z = or_f32_from_f16((uint16_t)(ks >> 16));
+        float sv = or_f32_from_f16((uint16_t)(vs & 0xffff)), zv = or_f32_from_f16((uint16_t)(vs >> 16));
+        for (int ch = g * GROUP; ch < (g + 1) * GROUP; ++ch) {
+            float m = or_f32_from_f16(c->cent[((size_t)h * c->M + j) * d + ch]);
+            float kd = fmaf((float)code_at(kw, ch), s, z);
+            float k32 = kd + m;
+            kh[ch] = or_f32_from_bf16(or_bf16_from_f32(k32));
+            float vd = fmaf((float)code_at(vw, ch), sv, zv);
+            vh[ch] = or_f32_from_f16(or_f16_from_f32(vd, RND_NEAREST_EVEN));
+        }
+    }
+}
+
+/* softmax-weighted sum over n keys given logits and value rows */
+static void softmax_combine(const double* logit, const double* vals, int n, int d, double* out)
+{
+    for (int c = 0; c < d; ++c) out[c] = 0.0;
+    if (n == 0) return;
+    double m = logit[0];
+    for (int i = 1; i < n; ++i) if (logit[i] > m) m = logit[i];
+    double l = 0.0;
+    for (int i = 0; i < n; ++i) l += exp(logit[i] - m);
+    for (int i = 0; i < n; ++i) {
+        double p = exp(logit[i] - m) / l;
+        for (int c = 0; c < d; ++c) out[c] += p * vals[(size_t)i * d + c];
+    }
+}
+
+int or_decode(int B, int Hkv, int d, int M, int r, int cap,
+              const uint32_t* k_code, const uint32_t* v_code, const uint32_t* k_sz,
+              const uint32_t* v_sz, const void* cidx, const uint16_t* psac,
+              const uint16_t* cent, const float* P,
+              int len, const uint16_t* Q, int Hq, double sm_scale, double* out)
+{
+    if (Hq % Hkv || len < 0 || len > cap) return 1;
+    or_cache c = {B, Hkv, d, M, r, cap, k_code, v_code, k_sz, v_sz, cidx, psac, cent, P};
+    int G = Hq / Hkv;
+    double* logit = (double*)malloc(((size_t)len + 1) * sizeof(double));
+    double* vals = (double*)malloc(((size_t)len + 1) * d * sizeof(double));
+    double* kh = (double*)malloc((size_t)d * sizeof(double));
+    double* q = (double*)malloc((size_t)d * sizeof(double));
+    double* u = (double*)malloc(((size_t)r + 1) * sizeof(double));
+    for (int b = 0; b < B; ++b)
+        for (int hq = 0; hq < Hq; ++hq) {
+            int h = hq / G;
+            const uint16_t* qr = Q + ((size_t)b * Hq + hq) * d;
+            for (int ch = 0; ch < d; ++ch) q[ch] = or_f32_from_bf16(qr[ch]);
+            for (int i = 0; i < r; ++i) {
+                u[i] = 0.0;
+                for (int ch = 0; ch < d; ++ch) u[i] += q[ch] * (double)P[((size_t)h * d + ch) * r + i];
+            }
+            for (int t = 0; t < len; ++t) {
+                size_t slot = ((size_t)b * Hkv + h) * cap + t;
+                dequant_exact(&c, slot, kh, vals + (size_t)t * d);
+                double acc = 0.0;
+                for (int ch = 0; ch < d; ++ch) acc += q[ch] * kh[ch];
+                for (int i = 0; i < r; ++i)
+                    acc += u[i] * (double)or_f32_from_f16(psac[slot * r + i]);
+                logit[t] = acc * sm_scale;
+            }
+            softmax_combine(logit, vals, len, d, out + ((size_t)b * Hq + hq) * d);
+        }
+    free(logit); free(vals); free(kh); free(q); free(u);
+    return 0;
+}
+
+/* Chunk attention for a list of query rows. Q bf16 [B][Nq][Hq][d]; Kself, Vself
+ * bf16 [B][Nq][Hkv][d]; query i of frame i / frame_tokens sees every cached
+ * token and the self tokens of frames <= its own. rows[k] = (b, i, hq) triples;
+ * out [nrows][d]. */
+int or_chunk(int B, int Hkv, int d, int M, int r, int cap,
+             const uint32_t* k_code, const uint32_t* v_code, const uint32_t* k_sz,
+             const uint32_t* v_sz, const void* cidx, const uint16_t* psac,
+             const uint16_t* cent, const float* P, int len,
+             const uint16_t* Q, int Hq, int Nq, const uint16_t* Kself, const uint16_t* Vself,
+             int frame_tokens, double sm_scale, const int32_t* rows, int nrows, double* out)
+{
+    if (Hq % Hkv || len < 0 || len > cap || frame_tokens <= 0) return 1;
+    or_cache c = {B, Hkv, d, M, r, cap, k_code, v_code, k_sz, v_sz, cidx, psac, cent, P};
+    int G = Hq / Hkv;
+    size_t nmax = (size_t)len + (size_t)Nq + 1;
+    double* logit = (double*)malloc(nmax * sizeof(double));
+    double* vals = (double*)malloc(nmax * d * sizeof(double));
+    double* kh = (double*)malloc((size_t)d * sizeof(double));
+    double* q = (double*)malloc((size_t)d * sizeof(double));
+    double* u = (double*)malloc(((size_t)r + 1) * sizeof(double));
+    for (int k = 0; k < nrows; ++k) {
+        int b = rows[3 * k], i = rows[3 * k + 1], hq = rows[3 * k + 2];
+        int h = hq / G;
+        const uint16_t* qr = Q + (((size_t)b * Nq + i) * Hq + hq) * d;
+        for (int ch = 0; ch < d; ++ch) q[ch] = or_f32_from_bf16(qr[ch]);
+        for (int a = 0; a < r; ++a) {
+            double acc = 0.0;
+            for (int ch = 0; ch < d; ++ch) acc += q[ch] * (double)P[((size_t)h * d + ch) * r + a];
+            u[a] = or_f32_from_f16(or_f16_from_f32((float)acc, RND_NEAREST_EVEN));
+        }
+        size_t n = 0;
+        for (int t = 0; t < len; ++t, ++n) {
+            size_t slot = ((size_t)b * Hkv + h) * cap + t;
+            dequant_operand(&c, slot, kh, vals + n * d);
+            double acc = 0.0;
+            for (int ch = 0; ch < d; ++ch) acc += q[ch] * kh[ch];
+            for (int a = 0; a < r; ++a) acc += u[a] * (double)or_f32_from_f16(psac[slot * r + a]);
+            logit[n] = acc * sm_scale;
+        }
+        int fi = i / frame_tokens;
+        for (int j = 0; j < Nq && j / frame_tokens <= fi; ++j, ++n) {
+            const uint16_t* kr = Kself + (((size_t)b * Nq + j) * Hkv + h) * d;
+            const uint16_t* vr = Vself + (((size_t)b * Nq + j) * Hkv + h) * d;
+            double acc = 0.0;
+            for (int ch = 0; ch < d; ++ch) {
+                acc += q[ch] * (double)or_f32_from_bf16(kr[ch]);
+                vals[n * d + ch] = or_f32_from_f16(or_f16_from_f32(or_f32_from_bf16(vr[ch]), RND_NEAREST_EVEN));
+            }
+            logit[n] = acc * sm_scale;
+        }
+        softmax_combine(logit, vals, (int)n, d, out + (size_t)k * d);
+    }
+    free(logit); free(vals); free(kh); free(q); free(u);
+    return 0;
+}
+
+/* Decode logits of one query against the packed cache (fp64), for tests of the
+ * PSAC and centroid closed forms. q fp64 [d]; out [len]. */
+int or_decode_logits(int Hkv, int d, int M, int r, int cap, int b, int h,
+                     const uint32_t* k_code, const uint32_t* k_sz, const void* cidx,
+                     const uint16_t* psac, const uint16_t* cent, const float* P,
+                     int len, const double* q, double* out)
+{
+    or_cache c = {b + 1, Hkv, d, M, r, cap, k_code, k_code, k_sz, k_sz, cidx, psac, cent, P};
+    double* kh = (double*)malloc((size_t)d * sizeof(double));
+    double* vh = (double*)malloc((size_t)d * sizeof(double));
+    double* u = (double*)malloc(((size_t)r + 1) * sizeof(double));
+    for (int i = 0; i < r; ++i) {
+        u[i] = 0.0;
+        for (int ch = 0; ch < d; ++ch) u[i] += q[ch] * (double)P[((size_t)h * d + ch) * r + i];
+    }
+    for (int t = 0; t < len; ++t) {
+        size_t slot = ((size_t)b * Hkv + h) * cap + t;
+        dequant_exact(&c, slot, kh, vh);
+        double acc = 0.0;
+        for (int ch = 0; ch < d; ++ch) acc += q[ch] * kh[ch];
+        for (int i = 0; i < r; ++i) acc += u[i] * (double)or_f32_from_f16(psac[slot * r + i]);
+        out[t] = acc;
+    }
+    free(kh); free(vh); free(u);
+    return 0;
+}
