@@ -1,0 +1,364 @@
+"""Benchmark of the 2-bit KV-cache hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Headline workload (one GPU, replicas only for N > 1): LLM-style decode, batch 8,
+32 query / 8 KV heads, d=128, 32,768 cached tokens per sequence, M=64 centroids,
+QSAC candidates 4, PSAC rank 8, bf16 output. One step = quantize/append of the
+new token of every sequence + decode attention over the packed cache (prep,
+split-K, combine). ``value`` = packed-cache bytes read per step / step time
+(GB/s); inputs already resident in HBM; the packed cache (237 MB) is larger
+than L2, so successive steps re-read it from HBM.
+
+Extra sections of the same JSON line: ``quantize`` (4,680 new tokens x 40
+heads, M=256, C=8, r=8: tokens/s and GB/s), ``fit`` (PSAC basis fit) and
+``chunk`` (video-world-model chunk attention, TFLOP/s) when available.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+BYTES_PER_TOKEN_HEAD = lambda d, r, M: 2 * (d // 16) * 4 + 2 * (d // 32) * 4 + (1 if M <= 256 else 2) + 2 * r
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region."""
+
+    def __init__(self, index=0):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------
+
+def setup_decode(torch, kv2, s: wl.Spec):
+    """Packed cache of the LLM decode workload built on the GPU by the library:
+    fit on the history queries, quantize/append of the 32,768-token prefix."""
+    w = wl.make(s.name, with_chunk=False)
+    dev = torch.device("cuda")
+    Qh = torch.from_numpy(w.Qhist.view(np.int16)).to(dev)
+    P, wt, Wg, en = kv2.kv2_fit_psac_basis(Qh, s.H_kv, s.r)
+    cache = kv2.Cache(s.B, s.H_kv, s.d, s.M, s.r, s.capacity, torch.from_numpy(w.centroids.view(np.int16)))
+    cache.set_fit(P, wt, Wg)
+    K = torch.from_numpy(np.ascontiguousarray(w.K[:, :s.T]).view(np.int16)).to(dev)
+    V = torch.from_numpy(np.ascontiguousarray(w.V[:, :s.T]).view(np.int16)).to(dev)
+    kv2.kv2_quantize_append(cache, K, V, 0, s.C)
+    del K, V
+    new_k = torch.from_numpy(np.ascontiguousarray(w.K[:, s.T:s.T + 1]).view(np.int16)).to(dev)
+    new_v = torch.from_numpy(np.ascontiguousarray(w.V[:, s.T:s.T + 1]).view(np.int16)).to(dev)
+    Q = torch.from_numpy(w.Qdec.view(np.int16)).to(dev)
+    torch.cuda.synchronize()
+    return w, cache, new_k, new_v, Q, Qh
+
+
+def run_gpu(args, rank, world):
+    import torch
+    import bit_kv_cache_centroid_b200 as kv2
+    torch.cuda.set_device(rank % max(torch.cuda.device_count(), 1))
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+        dist = dist_mod
+    s = wl.spec("llm_decode")
+    w, cache, new_k, new_v, Q, Qh = setup_decode(torch, kv2, s)
+    length = s.T + 1
+    scale = 1.0 / math.sqrt(s.d)
+    out = torch.empty((s.B, s.H_q, s.d), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(kv2.kv2_decode_workspace_size(cache, s.H_q, length), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        kv2.kv2_quantize_append(cache, new_k, new_v, s.T, s.C)
+        kv2.kv2_attention_decode(cache, length, Q, scale, out_dtype=kv2.KV2_OUT_BF16, out=out, ws=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    dec_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        time.sleep(0.3)
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            kv2.kv2_quantize_append(cache, new_k, new_v, s.T, s.C)
+            dec_ev[i][0].record(stream)
+            kv2.kv2_attention_decode(cache, length, Q, scale, out_dtype=kv2.KV2_OUT_BF16, out=out, ws=ws)
+            dec_ev[i][1].record(stream)
+            ev[i][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        time.sleep(0.2)
+    total_ms = t0.elapsed_time(t1)
+    if dist:
+        tt = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_step = total_ms / args.steps
+    dec_ms = statistics.mean(a.elapsed_time(b) for a, b in dec_ev)
+    bytes_step = length * s.B * s.H_kv * BYTES_PER_TOKEN_HEAD(s.d, s.r, s.M)
+    value = bytes_step * world / (ms_step * 1e-3) / 1e9
+
+    # ---- end to end through host buffers (pinned), copies inside the timed region
+    hk = new_k.cpu().pin_memory()
+    hv = new_v.cpu().pin_memory()
+    hq = Q.cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dk, dv, dq = torch.empty_like(new_k), torch.empty_like(new_v), torch.empty_like(Q)
+
+    def e2e_step():
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dq.copy_(hq, non_blocking=True)
+        kv2.kv2_quantize_append(cache, dk, dv, s.T, s.C)
+        kv2.kv2_attention_decode(cache, length, dq, scale, out_dtype=kv2.KV2_OUT_BF16, out=out, ws=ws)
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b) / args.steps
+    h2d = hk.numel() * 2 + hv.numel() * 2 + hq.numel() * 2
+    d2h = hout.numel() * 2
+
+    pk, src = peaks()
+    achieved = bytes_step / (dec_ms * 1e-3) / 1e9
+    result = {
+        "metric": "2-bit KV attention: packed-cache GB/s (% of HBM peak); quantize tokens/s",
+        "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "u2+f32", "data": "synthetic",
+        "config": {"workload": "llm_decode: B=8, H_q=32, H_kv=8, d=128, T=32768 cached, M=64, C=4, r=8, "
+                               "bf16 out; step = append 1 token/seq + decode",
+                   "global_batch": s.B * world, "seq_len": length, "parallelism": f"replicas x{world}",
+                   "l2": "packed cache 237 MB > 126 MB L2 (no flush)"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": None,
+                     "kernel": "kv2_attention_decode (prep + split-K + combine)",
+                     "peak_source": src, "decode_ms": round(dec_ms, 5)},
+        "e2e": {"value": round(bytes_step / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if not args.skip_extras and rank == 0:
+        result.update(extras(torch, kv2, args, pk))
+    if rank == 0 and not args.no_cpu:
+        result["cpu_baseline"] = cpu_baseline(args, budget_s=args.cpu_seconds)
+    return result
+
+
+def extras(torch, kv2, args, pk):
+    """Quantize/append throughput and fit time (same JSON line)."""
+    out = {}
+    s = wl.spec("quant_append")
+    w = wl.make("quant_append", T=wl.FRAME_TOKENS, with_chunk=False)
+    dev = torch.device("cuda")
+    Qh = torch.from_numpy(w.Qhist.view(np.int16)).to(dev)
+    cap = (s.capacity + 15) // 16 * 16
+    cache = kv2.Cache(s.B, s.H_kv, s.d, s.M, s.r, cap, torch.from_numpy(w.centroids.view(np.int16)))
+    P, wt, Wg, en = kv2.kv2_fit_psac_basis(Qh, s.H_kv, s.r)
+    cache.set_fit(P, wt, Wg)
+    K = torch.from_numpy(np.ascontiguousarray(w.K_new).view(np.int16)).to(dev)
+    V = torch.from_numpy(np.ascontiguousarray(w.V_new).view(np.int16)).to(dev)
+    for _ in range(3):
+        kv2.kv2_quantize_append(cache, K, V, s.T, s.C)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = max(5, args.steps // 2)
+    a.record()
+    for _ in range(n):
+        kv2.kv2_quantize_append(cache, K, V, s.T, s.C)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / n
+    toks = s.n_new * s.B
+    rd = K.numel() * 2 * 2
+    wr = toks * s.H_kv * BYTES_PER_TOKEN_HEAD(s.d, s.r, s.M)
+    fma = toks * s.H_kv * s.M * s.d
+    out["quantize"] = {"workload": "quant_append: 4680 new tokens x 40 heads, d=128, M=256, C=8, r=8",
+                       "ms": round(ms, 4), "tokens_per_s": round(toks / (ms * 1e-3), 1),
+                       "token_heads_per_s": round(toks * s.H_kv / (ms * 1e-3), 1),
+                       "GBps": round((rd + wr) / (ms * 1e-3) / 1e9, 2),
+                       "hbm_frac": round((rd + wr) / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+                       "ranking_TFMAps": round(fma / (ms * 1e-3) / 1e12, 3)}
+    a.record()
+    for _ in range(3):
+        kv2.kv2_fit_psac_basis(Qh, s.H_kv, s.r)
+    b.record()
+    torch.cuda.synchronize()
+    out["fit"] = {"workload": "40 heads x 512 history queries, d=128, r=8", "ms": round(a.elapsed_time(b) / 3, 3)}
+    return out
+
+
+# ----------------------------------------------------------------------------
+# CPU: the oracle as it stands
+# ----------------------------------------------------------------------------
+
+def cpu_baseline(args, budget_s=15.0):
+    """Oracle decode (fp64, single thread) on whole sequences of the LLM decode
+    workload until ~budget_s of CPU time; GB/s of packed cache attended."""
+    import oracle
+    oracle.build()
+    s = wl.spec("llm_decode")
+    pc = wl.random_packed_cache(s.with_(B=1), T=s.T + 1)
+    rng = np.random.default_rng(5)
+    P = np.zeros((s.H_kv, s.d, s.r), np.float32)
+    for h in range(s.H_kv):
+        q, _ = np.linalg.qr(rng.standard_normal((s.d, s.d)))
+        P[h] = q[:, :s.r]
+    Q = wl.bf16_bits(rng.standard_normal((1, s.H_q, s.d)).astype(np.float32))
+    seqs, t = 0, 0.0
+    while t < budget_s and seqs < 64:
+        t0 = time.perf_counter()
+        oracle.decode(pc, P, s.T + 1, Q, 1.0 / math.sqrt(s.d))
+        t += time.perf_counter() - t0
+        seqs += 1
+    bytes_ = seqs * (s.T + 1) * s.H_kv * BYTES_PER_TOKEN_HEAD(s.d, s.r, s.M)
+    return {"value": round(bytes_ / t / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{seqs} sequence(s) x 8 KV heads x 32 query heads x 32,769 tokens (oracle decode, fp64)",
+            "seconds": round(t, 2)}
+
+
+def run_reference(args):
+    r = cpu_baseline(args, budget_s=max(2.0, args.cpu_seconds / max(args.steps, 1)))
+    ms = (r["seconds"] * 1e3)
+    return {"impl": "reference",
+            "metric": "2-bit KV attention: packed-cache GB/s (% of HBM peak); quantize tokens/s",
+            "value": r["value"], "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "llm_decode: B=8, H_q=32, H_kv=8, d=128, T=32768 cached, M=64, C=4, r=8",
+                       "global_batch": 8, "seq_len": 32769, "parallelism": "none (CPU oracle)"},
+            "cpu_baseline": r,
+            "e2e": {"value": r["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="libkv2")
+    ap.add_argument("--skip-extras", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--only", choices=["decode", "quantize"], default=None,
+                    help="run one section only (for profiler captures)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if args.only == "quantize":
+        import torch
+        import bit_kv_cache_centroid_b200 as kv2
+        print(json.dumps(extras(torch, kv2, args, peaks()[0])), flush=True)
+        return
+    if args.only == "decode":
+        args.skip_extras, args.no_cpu = True, True
+    res = run_gpu(args, rank, world)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

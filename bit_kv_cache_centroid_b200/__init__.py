@@ -1,0 +1,219 @@
+"""Thin Python binding of libkv2 (include/kv2.h): argument marshalling only.
+
+Every step of the path runs in the CUDA library; this module passes device
+pointers (``tensor.data_ptr()``) and the current CUDA stream. PyTorch is used
+for device memory and streams only. If ``libkv2.so`` is missing or fails to
+load, importing the binding raises: there is no CPU fallback.
+
+Names follow the C ABI: ``kv2_fit_psac_basis``, ``kv2_quantize_append``,
+``kv2_attention_decode``, ``kv2_attention_chunk`` and the workspace-size
+queries. ``Cache`` owns the device buffers of one packed cache and builds the
+``kv2_cache`` descriptor.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkv2.so")
+
+KV2_OK = 0
+KV2_OUT_F32 = 0
+KV2_OUT_BF16 = 1
+GROUP = 32
+STATUS = {0: "KV2_OK", 1: "KV2_ERR_INVALID_ARG", 2: "KV2_ERR_UNSUPPORTED", 3: "KV2_ERR_CAPACITY",
+          4: "KV2_ERR_CUDA", 5: "KV2_ERR_TIMEOUT", 6: "KV2_ERR_WORKSPACE"}
+
+
+class Kv2Error(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{STATUS.get(status, status)}: {detail}")
+        self.status = status
+
+
+class kv2_cache(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H_kv", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("M", ctypes.c_int32), ("r", ctypes.c_int32), ("capacity", ctypes.c_int32),
+                ("k_code", ctypes.c_void_p), ("v_code", ctypes.c_void_p),
+                ("k_sz", ctypes.c_void_p), ("v_sz", ctypes.c_void_p),
+                ("cidx", ctypes.c_void_p), ("psac", ctypes.c_void_p),
+                ("centroids", ctypes.c_void_p), ("P", ctypes.c_void_p),
+                ("w", ctypes.c_void_p), ("Wg", ctypes.c_void_p)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libkv2.so not built ({LIB_PATH}); run python -m bit_kv_cache_centroid_b200.build")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    L.kv2_status_string.restype = ctypes.c_char_p
+    L.kv2_status_string.argtypes = [I]
+    L.kv2_last_error.restype = ctypes.c_char_p
+    L.kv2_version.restype = I
+    L.kv2_fit_workspace_size.restype = S
+    L.kv2_fit_workspace_size.argtypes = [I, I]
+    L.kv2_fit_psac_basis.restype = I
+    L.kv2_fit_psac_basis.argtypes = [P, I, I, I, I, I, P, P, P, P, P, S, P]
+    L.kv2_quantize_append.restype = I
+    L.kv2_quantize_append.argtypes = [ctypes.POINTER(kv2_cache), P, P, I, I, I, P]
+    L.kv2_decode_workspace_size.restype = S
+    L.kv2_decode_workspace_size.argtypes = [ctypes.POINTER(kv2_cache), I, I]
+    L.kv2_attention_decode.restype = I
+    L.kv2_attention_decode.argtypes = [ctypes.POINTER(kv2_cache), I, P, I, ctypes.c_float, P, I, P, S, P]
+    L.kv2_chunk_workspace_size.restype = S
+    L.kv2_chunk_workspace_size.argtypes = [ctypes.POINTER(kv2_cache), I, I]
+    L.kv2_attention_chunk.restype = I
+    L.kv2_attention_chunk.argtypes = [ctypes.POINTER(kv2_cache), I, P, I, I, P, P, I,
+                                      ctypes.c_float, P, I, P, S, P]
+    return L
+
+
+lib = _load()
+EXPORTS = ["kv2_status_string", "kv2_last_error", "kv2_version", "kv2_fit_workspace_size",
+           "kv2_fit_psac_basis", "kv2_quantize_append", "kv2_decode_workspace_size",
+           "kv2_attention_decode", "kv2_chunk_workspace_size", "kv2_attention_chunk"]
+
+
+def _check(status: int):
+    if status != KV2_OK:
+        raise Kv2Error(status, lib.kv2_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class Cache:
+    """Device buffers of one packed cache (layout of include/kv2.h) plus the
+    read-only centroid table and fitted statistics it points to."""
+
+    def __init__(self, B, H_kv, d, M, r, capacity, centroids, device="cuda"):
+        if capacity % 16:
+            raise ValueError("capacity must be a multiple of 16")
+        self.B, self.H_kv, self.d, self.M, self.r, self.capacity = B, H_kv, d, M, r, capacity
+        sh = (B, H_kv, capacity)
+        u32 = torch.int32
+        self.k_code = torch.zeros(sh + (d // 16,), dtype=u32, device=device)
+        self.v_code = torch.zeros(sh + (d // 16,), dtype=u32, device=device)
+        self.k_sz = torch.zeros(sh + (d // GROUP,), dtype=u32, device=device)
+        self.v_sz = torch.zeros(sh + (d // GROUP,), dtype=u32, device=device)
+        self.cidx = torch.zeros(sh, dtype=torch.uint8 if M <= 256 else torch.int16, device=device)
+        self.psac = torch.zeros(sh + (max(r, 1),), dtype=torch.int16, device=device)
+        self.centroids = torch.as_tensor(centroids).to(device=device, dtype=torch.int16).contiguous()
+        self.P = torch.zeros((H_kv, d, max(r, 1)), dtype=torch.float32, device=device)
+        self.w = torch.ones((H_kv, d), dtype=torch.float32, device=device)
+        self.Wg = torch.full((H_kv, d // GROUP), float(GROUP), dtype=torch.float32, device=device)
+        self.energy = torch.zeros(H_kv, dtype=torch.float32, device=device)
+
+    def desc(self) -> kv2_cache:
+        return kv2_cache(self.B, self.H_kv, self.d, self.M, self.r, self.capacity,
+                         self.k_code.data_ptr(), self.v_code.data_ptr(), self.k_sz.data_ptr(),
+                         self.v_sz.data_ptr(), self.cidx.data_ptr(),
+                         self.psac.data_ptr() if self.r else 0, self.centroids.data_ptr(),
+                         self.P.data_ptr(), self.w.data_ptr(), self.Wg.data_ptr())
+
+    def set_fit(self, P, w, Wg):
+        if self.r:
+            self.P.copy_(torch.as_tensor(P).reshape(self.H_kv, self.d, self.r))
+        self.w.copy_(torch.as_tensor(w).reshape(self.H_kv, self.d))
+        self.Wg.copy_(torch.as_tensor(Wg).reshape(self.H_kv, self.d // GROUP))
+
+    def load_packed(self, pc):
+        """Copy a host packed cache (numpy arrays, library layout) in."""
+        for name in ("k_code", "v_code", "k_sz", "v_sz"):
+            getattr(self, name).copy_(torch.from_numpy(getattr(pc, name).view("int32")))
+        self.cidx.copy_(torch.from_numpy(pc.cidx.view("uint8" if self.M <= 256 else "int16")))
+        if self.r:
+            self.psac.copy_(torch.from_numpy(pc.psac.view("int16")))
+
+    def to_host(self):
+        """Host numpy copies of the packed streams (library layout)."""
+        out = {n: getattr(self, n).cpu().numpy().view("uint32") for n in ("k_code", "v_code", "k_sz", "v_sz")}
+        out["cidx"] = self.cidx.cpu().numpy().view("uint8" if self.M <= 256 else "uint16")
+        out["psac"] = self.psac.cpu().numpy().view("uint16")[..., :self.r]
+        return out
+
+
+# ----------------------------------------------------------------------------
+# entry points (same names as the C ABI)
+# ----------------------------------------------------------------------------
+
+def kv2_fit_workspace_size(H_kv: int, d: int) -> int:
+    return int(lib.kv2_fit_workspace_size(H_kv, d))
+
+
+def kv2_fit_psac_basis(Qhist: torch.Tensor, H_kv: int, r: int, P=None, w=None, Wg=None,
+                       energy=None, ws=None, stream=None):
+    """Qhist bf16 [n][H_q][d] (device) -> (P [H_kv][d][r], w [H_kv][d], Wg, energy)."""
+    n, H_q, d = Qhist.shape
+    dev = Qhist.device
+    P = torch.empty((H_kv, d, max(r, 1)), dtype=torch.float32, device=dev) if P is None else P
+    w = torch.empty((H_kv, d), dtype=torch.float32, device=dev) if w is None else w
+    Wg = torch.empty((H_kv, d // GROUP), dtype=torch.float32, device=dev) if Wg is None else Wg
+    energy = torch.empty(H_kv, dtype=torch.float32, device=dev) if energy is None else energy
+    need = kv2_fit_workspace_size(H_kv, d)
+    ws = torch.empty(need, dtype=torch.uint8, device=dev) if ws is None else ws
+    _check(lib.kv2_fit_psac_basis(_ptr(Qhist), n, H_q, H_kv, d, r, _ptr(P), _ptr(w), _ptr(Wg),
+                                  _ptr(energy), _ptr(ws), ws.numel(), _stream(stream)))
+    return P[:, :, :r], w, Wg, energy
+
+
+def kv2_quantize_append(cache: Cache, K: torch.Tensor, V: torch.Tensor, pos: int,
+                        candidates: int, stream=None):
+    """K, V bf16 [B][n_new][H_kv][d] (device) -> written into cache slots [pos, pos+n_new)."""
+    d = cache.desc()
+    n_new = K.shape[1]
+    _check(lib.kv2_quantize_append(ctypes.byref(d), _ptr(K), _ptr(V), n_new, pos, candidates,
+                                   _stream(stream)))
+
+
+def kv2_decode_workspace_size(cache: Cache, H_q: int, length: int) -> int:
+    d = cache.desc()
+    return int(lib.kv2_decode_workspace_size(ctypes.byref(d), H_q, length))
+
+
+def kv2_attention_decode(cache: Cache, length: int, Q: torch.Tensor, sm_scale: float,
+                         out_dtype: int = KV2_OUT_F32, out=None, ws=None, stream=None):
+    """Q bf16 [B][H_q][d] -> out [B][H_q][d] (fp32 or bf16)."""
+    B, H_q, dd = Q.shape
+    if out is None:
+        out = torch.empty((B, H_q, dd), dtype=torch.float32 if out_dtype == KV2_OUT_F32 else torch.bfloat16,
+                          device=Q.device)
+    if ws is None:
+        ws = torch.empty(max(kv2_decode_workspace_size(cache, H_q, length), 16), dtype=torch.uint8,
+                         device=Q.device)
+    d = cache.desc()
+    _check(lib.kv2_attention_decode(ctypes.byref(d), length, _ptr(Q), H_q, float(sm_scale), _ptr(out),
+                                    out_dtype, _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def kv2_chunk_workspace_size(cache: Cache, H_q: int, Nq: int) -> int:
+    d = cache.desc()
+    return int(lib.kv2_chunk_workspace_size(ctypes.byref(d), H_q, Nq))
+
+
+def kv2_attention_chunk(cache: Cache, length: int, Q: torch.Tensor, Kself: torch.Tensor,
+                        Vself: torch.Tensor, frame_tokens: int, sm_scale: float,
+                        out_dtype: int = KV2_OUT_F32, out=None, ws=None, stream=None):
+    """Q bf16 [B][Nq][H_q][d], Kself/Vself bf16 [B][Nq][H_kv][d] -> out [B][Nq][H_q][d]."""
+    B, Nq, H_q, dd = Q.shape
+    if out is None:
+        out = torch.empty((B, Nq, H_q, dd), dtype=torch.float32 if out_dtype == KV2_OUT_F32 else torch.bfloat16,
+                          device=Q.device)
+    if ws is None:
+        ws = torch.empty(max(kv2_chunk_workspace_size(cache, H_q, Nq), 16), dtype=torch.uint8,
+                         device=Q.device)
+    d = cache.desc()
+    _check(lib.kv2_attention_chunk(ctypes.byref(d), length, _ptr(Q), H_q, Nq, _ptr(Kself), _ptr(Vself),
+                                   frame_tokens, float(sm_scale), _ptr(out), out_dtype, _ptr(ws),
+                                   ws.numel(), _stream(stream)))
+    return out

@@ -1,0 +1,174 @@
+// api.cu — extern "C" entry points of libkv2 (declared in include/kv2.h):
+// argument validation, workspace sizing and kernel dispatch. The library never
+// allocates device memory; every buffer is the caller's.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "internal.h"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+kv2_status fail(kv2_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+kv2_status ok() {
+  g_last_error[0] = '\0';
+  return KV2_OK;
+}
+
+kv2_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return ok();
+  return fail(KV2_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape and pointer checks common to every call that reads the cache.
+kv2_status check_cache(const kv2_cache* c, bool need_cache_streams, bool need_fit) {
+  if (!c) return fail(KV2_ERR_INVALID_ARG, "cache descriptor is NULL");
+  if (c->B <= 0 || c->H_kv <= 0 || c->capacity < 0 || c->M <= 0 || c->r < 0)
+    return fail(KV2_ERR_INVALID_ARG, "cache sizes must be positive (B=%d H_kv=%d M=%d r=%d cap=%d)",
+                c->B, c->H_kv, c->M, c->r, c->capacity);
+  if (c->d != 64 && c->d != 128) return fail(KV2_ERR_UNSUPPORTED, "head dim d=%d (supported: 64, 128)", c->d);
+  if (c->M > kv2::kMaxCentroids) return fail(KV2_ERR_UNSUPPORTED, "M=%d centroids (max 512)", c->M);
+  if (c->r > c->d || (c->r & 1)) return fail(KV2_ERR_UNSUPPORTED, "PSAC rank r=%d (even, <= d)", c->r);
+  if (c->capacity % 16) return fail(KV2_ERR_UNSUPPORTED, "capacity %d is not a multiple of 16", c->capacity);
+  if (!c->centroids || !aligned16(c->centroids))
+    return fail(KV2_ERR_INVALID_ARG, "centroids must be a non-NULL 16-byte aligned pointer");
+  if (need_cache_streams) {
+    const void* ptrs[] = {c->k_code, c->v_code, c->k_sz, c->v_sz, c->cidx};
+    for (const void* p : ptrs)
+      if (!p || !aligned16(p)) return fail(KV2_ERR_INVALID_ARG, "cache stream pointer NULL or not 16-byte aligned");
+    if (c->r && (!c->psac || !aligned16(c->psac)))
+      return fail(KV2_ERR_INVALID_ARG, "psac pointer NULL or not 16-byte aligned");
+  }
+  if (need_fit) {
+    if (!c->w || !c->Wg || !aligned16(c->w) || !aligned16(c->Wg))
+      return fail(KV2_ERR_INVALID_ARG, "w / Wg pointers NULL or not 16-byte aligned");
+  }
+  if (c->r && (!c->P || !aligned16(c->P))) return fail(KV2_ERR_INVALID_ARG, "P pointer NULL or not 16-byte aligned");
+  return KV2_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kv2_status_string(kv2_status s) {
+  switch (s) {
+    case KV2_OK: return "KV2_OK";
+    case KV2_ERR_INVALID_ARG: return "KV2_ERR_INVALID_ARG";
+    case KV2_ERR_UNSUPPORTED: return "KV2_ERR_UNSUPPORTED";
+    case KV2_ERR_CAPACITY: return "KV2_ERR_CAPACITY";
+    case KV2_ERR_CUDA: return "KV2_ERR_CUDA";
+    case KV2_ERR_TIMEOUT: return "KV2_ERR_TIMEOUT";
+    case KV2_ERR_WORKSPACE: return "KV2_ERR_WORKSPACE";
+  }
+  return "KV2_ERR_UNKNOWN";
+}
+
+const char* kv2_last_error(void) { return g_last_error; }
+
+int kv2_version(void) { return 100; }
+
+size_t kv2_fit_workspace_size(int H_kv, int d) {
+  if (H_kv <= 0 || (d != 64 && d != 128)) return 0;
+  return kv2::fit_workspace_bytes(H_kv, d);
+}
+
+kv2_status kv2_fit_psac_basis(const uint16_t* Qhist, int n, int H_q, int H_kv, int d, int r,
+                              float* P, float* w, float* Wg, float* energy, void* ws,
+                              size_t ws_bytes, void* stream) {
+  if (n <= 0 || H_q <= 0 || H_kv <= 0 || r < 0) return fail(KV2_ERR_INVALID_ARG, "fit: sizes must be positive");
+  if (H_q % H_kv) return fail(KV2_ERR_UNSUPPORTED, "fit: H_q=%d not a multiple of H_kv=%d", H_q, H_kv);
+  if (d != 64 && d != 128) return fail(KV2_ERR_UNSUPPORTED, "fit: head dim d=%d (supported: 64, 128)", d);
+  if (r > d) return fail(KV2_ERR_UNSUPPORTED, "fit: r=%d > d=%d", r, d);
+  if (!Qhist || !w || !Wg || !ws || (r && !P)) return fail(KV2_ERR_INVALID_ARG, "fit: NULL pointer");
+  if (!aligned16(Qhist) || !aligned16(ws)) return fail(KV2_ERR_INVALID_ARG, "fit: misaligned pointer");
+  if (ws_bytes < kv2::fit_workspace_bytes(H_kv, d))
+    return fail(KV2_ERR_WORKSPACE, "fit: workspace %zu < %zu bytes", ws_bytes, kv2::fit_workspace_bytes(H_kv, d));
+  kv2::FitArgs a{Qhist, n, H_q, H_kv, d, r, P, w, Wg, energy, ws};
+  return cuda_status(kv2::launch_fit(a, static_cast<cudaStream_t>(stream)), "fit launch");
+}
+
+kv2_status kv2_quantize_append(const kv2_cache* c, const uint16_t* K, const uint16_t* V, int n_new,
+                               int pos, int candidates, void* stream) {
+  kv2_status st = check_cache(c, true, true);
+  if (st != KV2_OK) return st;
+  if (n_new < 0) return fail(KV2_ERR_INVALID_ARG, "quantize: n_new=%d < 0", n_new);
+  if (pos < 0 || pos > c->capacity - n_new)
+    return fail(KV2_ERR_CAPACITY, "quantize: slots [%d, %d) exceed capacity %d", pos, pos + n_new, c->capacity);
+  if (candidates < 1 || candidates > c->M)
+    return fail(KV2_ERR_INVALID_ARG, "quantize: candidates=%d outside 1..M=%d", candidates, c->M);
+  if (n_new == 0) return ok();
+  if (!K || !V || !aligned16(K) || !aligned16(V))
+    return fail(KV2_ERR_INVALID_ARG, "quantize: K / V NULL or not 16-byte aligned");
+  kv2::QuantizeArgs a{K, V, c->B, c->H_kv, c->d, c->M, c->r, c->capacity, n_new, pos, candidates,
+                      c->centroids, c->P, c->w, c->Wg, c->k_code, c->v_code, c->k_sz, c->v_sz,
+                      c->cidx, c->psac};
+  return cuda_status(kv2::launch_quantize(a, static_cast<cudaStream_t>(stream)), "quantize launch");
+}
+
+size_t kv2_decode_workspace_size(const kv2_cache* c, int H_q, int len) {
+  if (!c || H_q <= 0 || c->H_kv <= 0 || H_q % c->H_kv || len < 0) return 0;
+  if (check_cache(c, false, false) != KV2_OK) return 0;
+  return kv2::decode_workspace_bytes(*c, H_q, len);
+}
+
+kv2_status kv2_attention_decode(const kv2_cache* c, int len, const uint16_t* Q, int H_q, float sm_scale,
+                                void* out, int out_dtype, void* ws, size_t ws_bytes, void* stream) {
+  kv2_status st = check_cache(c, true, false);
+  if (st != KV2_OK) return st;
+  if (H_q <= 0 || H_q % c->H_kv) return fail(KV2_ERR_UNSUPPORTED, "decode: H_q=%d not a multiple of H_kv=%d", H_q, c->H_kv);
+  const int G = H_q / c->H_kv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return fail(KV2_ERR_UNSUPPORTED, "decode: H_q/H_kv=%d (supported 1, 2, 4, 8)", G);
+  if (len < 0 || len > c->capacity) return fail(KV2_ERR_CAPACITY, "decode: len=%d outside 0..capacity=%d", len, c->capacity);
+  if (out_dtype != KV2_OUT_F32 && out_dtype != KV2_OUT_BF16) return fail(KV2_ERR_INVALID_ARG, "decode: out_dtype=%d", out_dtype);
+  if (!Q || !out || !ws || !aligned16(Q) || !aligned16(out) || !aligned16(ws))
+    return fail(KV2_ERR_INVALID_ARG, "decode: Q / out / ws NULL or not 16-byte aligned");
+  const size_t need = kv2::decode_workspace_bytes(*c, H_q, len);
+  if (ws_bytes < need) return fail(KV2_ERR_WORKSPACE, "decode: workspace %zu < %zu bytes", ws_bytes, need);
+  kv2::DecodeArgs a{c, len, H_q, Q, sm_scale, out, out_dtype, ws, ws_bytes};
+  return cuda_status(kv2::launch_decode(a, static_cast<cudaStream_t>(stream)), "decode launch");
+}
+
+size_t kv2_chunk_workspace_size(const kv2_cache* c, int H_q, int Nq) {
+  if (!c || H_q <= 0 || c->H_kv <= 0 || H_q % c->H_kv || Nq < 0) return 0;
+  if (check_cache(c, false, false) != KV2_OK) return 0;
+  return kv2::chunk_workspace_bytes(*c, H_q, Nq);
+}
+
+kv2_status kv2_attention_chunk(const kv2_cache* c, int len, const uint16_t* Q, int H_q, int Nq,
+                               const uint16_t* Kself, const uint16_t* Vself, int frame_tokens,
+                               float sm_scale, void* out, int out_dtype, void* ws, size_t ws_bytes,
+                               void* stream) {
+  kv2_status st = check_cache(c, true, false);
+  if (st != KV2_OK) return st;
+  if (c->d != 128) return fail(KV2_ERR_UNSUPPORTED, "chunk: head dim d=%d (supported: 128)", c->d);
+  if (c->r != 0 && c->r != 8 && c->r != 16) return fail(KV2_ERR_UNSUPPORTED, "chunk: r=%d (supported 0, 8, 16)", c->r);
+  if (H_q <= 0 || H_q % c->H_kv) return fail(KV2_ERR_UNSUPPORTED, "chunk: H_q=%d not a multiple of H_kv=%d", H_q, c->H_kv);
+  if (Nq < 0 || frame_tokens <= 0) return fail(KV2_ERR_INVALID_ARG, "chunk: Nq=%d frame_tokens=%d", Nq, frame_tokens);
+  if (len < 0 || len > c->capacity) return fail(KV2_ERR_CAPACITY, "chunk: len=%d outside 0..capacity=%d", len, c->capacity);
+  if (out_dtype != KV2_OUT_F32 && out_dtype != KV2_OUT_BF16) return fail(KV2_ERR_INVALID_ARG, "chunk: out_dtype=%d", out_dtype);
+  if (Nq == 0) return ok();
+  if (!Q || !Kself || !Vself || !out || !ws)
+    return fail(KV2_ERR_INVALID_ARG, "chunk: NULL pointer");
+  if (!aligned16(Q) || !aligned16(Kself) || !aligned16(Vself) || !aligned16(out) || !aligned16(ws))
+    return fail(KV2_ERR_INVALID_ARG, "chunk: pointer not 16-byte aligned");
+  const size_t need = kv2::chunk_workspace_bytes(*c, H_q, Nq);
+  if (ws_bytes < need) return fail(KV2_ERR_WORKSPACE, "chunk: workspace %zu < %zu bytes", ws_bytes, need);
+  kv2::ChunkArgs a{c, len, H_q, Nq, frame_tokens, Q, Kself, Vself, sm_scale, out, out_dtype, ws, ws_bytes, nullptr};
+  cudaError_t e = kv2::launch_chunk(a, static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported) return fail(KV2_ERR_UNSUPPORTED, "chunk: kernel not available");
+  return cuda_status(e, "chunk launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,58 @@
+// Device helpers shared by the libkv2 kernels.
+#pragma once
+
+#include <cstdint>
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+namespace kv2 {
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+__device__ __forceinline__ float f16_to_f32(uint16_t h) {
+  return __half2float(__ushort_as_half(h));
+}
+
+// fp32 -> fp16 bit patterns with an explicit rounding direction.
+__device__ __forceinline__ uint16_t f16_rd(float x) { return __half_as_ushort(__float2half_rd(x)); }
+__device__ __forceinline__ uint16_t f16_ru(float x) { return __half_as_ushort(__float2half_ru(x)); }
+__device__ __forceinline__ uint16_t f16_rn(float x) { return __half_as_ushort(__float2half_rn(x)); }
+
+// Order-preserving map of an fp32 value to uint32 (for packed argmin keys).
+__device__ __forceinline__ uint32_t float_order(float f) {
+  uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// INT2 group codec, shared by the quantizer's decision and encoding stages.
+// zero = round-down of the minimum, scale = round-up of (max - zero)/3.
+struct GroupParams {
+  uint16_t s_bits, z_bits;
+  float s, z;
+};
+
+__device__ __forceinline__ GroupParams group_params(float mn, float mx) {
+  GroupParams p;
+  p.z_bits = f16_rd(mn);
+  p.z = f16_to_f32(p.z_bits);
+  float q = __fdiv_rn(__fsub_rn(mx, p.z), 3.0f);
+  p.s_bits = f16_ru(q);
+  p.s = f16_to_f32(p.s_bits);
+  return p;
+}
+
+__device__ __forceinline__ uint32_t group_code(float x, const GroupParams& p) {
+  if (p.s == 0.0f) return 0u;
+  float c = rintf(__fdiv_rn(__fsub_rn(x, p.z), p.s));
+  c = fminf(fmaxf(c, 0.0f), 3.0f);
+  return static_cast<uint32_t>(c);
+}
+
+__device__ __forceinline__ float group_dequant(uint32_t code, const GroupParams& p) {
+  return __fmaf_rn(static_cast<float>(code), p.s, p.z);
+}
+
+}  // namespace kv2

@@ -1,0 +1,79 @@
+// Internal declarations shared by the host entry points and the kernel files
+// of libkv2. Nothing here is part of the C ABI (see include/kv2.h).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "kv2.h"
+
+namespace kv2 {
+
+constexpr int kGroup = 32;          // channels per quantization group
+constexpr int kMaxCentroids = 512;  // centroid ids fit in u16 above 256
+
+// Arguments of one quantize/append call (validated by the host entry point).
+struct QuantizeArgs {
+  const uint16_t* K;   // bf16 [B][n_new][H][d]
+  const uint16_t* V;
+  int B, H, d, M, r, cap, n_new, pos, C;
+  const uint16_t* cent;  // fp16 [H][M][d]
+  const float* P;        // [H][d][r]
+  const float* w;        // [H][d]
+  const float* Wg;       // [H][d/32]
+  uint32_t* k_code;
+  uint32_t* v_code;
+  uint32_t* k_sz;
+  uint32_t* v_sz;
+  void* cidx;
+  uint16_t* psac;
+};
+cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s);
+
+// Decode attention.
+struct DecodeArgs {
+  const kv2_cache* c;   // host copy of the descriptor
+  int len, H_q;
+  const uint16_t* Q;    // bf16 [B][H_q][d]
+  float sm_scale;
+  void* out;
+  int out_dtype;
+  void* ws;
+  size_t ws_bytes;
+};
+size_t decode_workspace_bytes(const kv2_cache& c, int H_q, int len);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+
+// PSAC basis fit.
+struct FitArgs {
+  const uint16_t* Qhist;  // bf16 [n][H_q][d]
+  int n, H_q, H_kv, d, r;
+  float* P;
+  float* w;
+  float* Wg;
+  float* energy;
+  void* ws;
+};
+size_t fit_workspace_bytes(int H_kv, int d);
+cudaError_t launch_fit(const FitArgs& a, cudaStream_t s);
+
+// Chunk attention (tcgen05).
+struct ChunkArgs {
+  const kv2_cache* c;
+  int len, H_q, Nq, frame_tokens;
+  const uint16_t* Q;      // bf16 [B][Nq][H_q][d]
+  const uint16_t* Kself;  // bf16 [B][Nq][H_kv][d]
+  const uint16_t* Vself;
+  float sm_scale;
+  void* out;
+  int out_dtype;
+  void* ws;
+  size_t ws_bytes;
+  int* err_flag;          // device word for bounded-wait timeouts (in ws)
+};
+size_t chunk_workspace_bytes(const kv2_cache& c, int H_q, int Nq);
+cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t s);
+
+}  // namespace kv2

@@ -1,0 +1,193 @@
+/*
+ * kv2.h — C ABI of libkv2: a training-free 2-bit KV cache with
+ * sensitivity-aware centroids (QSAC) and principal-subspace compensation
+ * (PSAC), and attention that reads the packed cache directly, for NVIDIA B200
+ * (sm_100a).
+ *
+ * Method: "QuantWM: Training-Free 2-bit KV Cache Quantization for Stable Video
+ * World Models" (besthub.dev article), sections "1. Quantization
+ * Sensitivity-Aware Clustering (QSAC)" and "2. Principal Subspace Attention
+ * Compensation (PSAC)". The principle of unpacking a 2-bit cache inside the
+ * attention kernel, so that no dense fp16 cache is ever built, is the one the
+ * OmniKVQuant page ("OmniKVQuant: KV Cache Quantization for Omni-LLMs",
+ * abstract) states for its decode kernel.
+ *
+ * Conventions for every entry point:
+ *  - All data pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates or frees device memory. Pointers must be 16-byte aligned.
+ *  - 16-bit floats travel as uint16_t bit patterns: bf16 for keys, values and
+ *    queries; fp16 for centroid tables, scales, zeros and PSAC coefficients.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream). Work is
+ *    enqueued asynchronously; argument errors are returned synchronously
+ *    before anything is enqueued; a failed launch returns KV2_ERR_CUDA.
+ *  - Supported shapes: head dim d in {64, 128}; quantization groups of 32
+ *    channels; 1 <= M <= 512 centroids per KV head (ids stored as u8 when
+ *    M <= 256, else u16); 0 <= r <= d PSAC rank (r a multiple of 8 for the
+ *    chunk kernel, r <= 16 there); H_q a multiple of H_kv. Anything else
+ *    returns KV2_ERR_UNSUPPORTED.
+ *  - Input magnitudes: keys, values and centroid-relative residuals must stay
+ *    within +-60000 (fp16 range of the stored zero and scale); larger inputs
+ *    give unspecified codes. NaN inputs propagate to the affected outputs.
+ *  - Dense tensors use the token-major layout [batch][token][head][d].
+ */
+#ifndef KV2_H
+#define KV2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kv2_status {
+  KV2_OK = 0,
+  KV2_ERR_INVALID_ARG = 1,  /* null or misaligned pointer, negative size      */
+  KV2_ERR_UNSUPPORTED = 2,  /* shape outside the supported set (see above)   */
+  KV2_ERR_CAPACITY = 3,     /* pos + n_new > capacity, or len > capacity     */
+  KV2_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed          */
+  KV2_ERR_TIMEOUT = 5,      /* a bounded device-side wait ran out            */
+  KV2_ERR_WORKSPACE = 6     /* workspace smaller than the *_workspace_size() */
+} kv2_status;
+
+enum { KV2_OUT_F32 = 0, KV2_OUT_BF16 = 1 };
+
+/*
+ * Packed cache of one layer (caller-owned device memory). Per (batch b,
+ * KV head h) every stream is contiguous along tokens, slot = (b*H_kv + h)*capacity + t:
+ *   k_code, v_code : uint32 [B][H_kv][capacity][d/16]; channel c of a token is
+ *                    in word c/16 at bits 2(c%16)..2(c%16)+1 (INT2 codes 0..3)
+ *   k_sz, v_sz     : uint32 [B][H_kv][capacity][d/32]; per 32-channel group,
+ *                    low half = fp16 scale s, high half = fp16 zero z; the
+ *                    dequantized value of code q is fmaf(q, s, z)
+ *   cidx           : centroid id per token, uint8 (M <= 256) or uint16 [B][H_kv][capacity]
+ *   psac           : fp16 [B][H_kv][capacity][r] PSAC coefficients a = P^T e
+ *   centroids      : fp16 [H_kv][M][d] (read-only; shared by the batch)
+ *   P, w, Wg       : fp32 [H_kv][d][r] basis, [H_kv][d] channel sensitivities,
+ *                    [H_kv][d/32] group sensitivities, as written by
+ *                    kv2_fit_psac_basis (read-only)
+ * A key is reconstructed as centroid[cidx] + fmaf(code, s, z) (+ P a for the
+ * logit correction), a value as fmaf(code, s, z).
+ */
+typedef struct kv2_cache {
+  int32_t B, H_kv, d, M, r, capacity;
+  uint32_t* k_code;
+  uint32_t* v_code;
+  uint32_t* k_sz;
+  uint32_t* v_sz;
+  void* cidx;
+  uint16_t* psac;
+  const uint16_t* centroids;
+  const float* P;
+  const float* w;
+  const float* Wg;
+} kv2_cache;
+
+/* Human-readable name of a status. Never NULL. */
+const char* kv2_status_string(kv2_status s);
+
+/* Detail of the last error returned on the calling host thread ("" if none). */
+const char* kv2_last_error(void);
+
+/* Library ABI version (major*100 + minor). */
+int kv2_version(void);
+
+/*
+ * Workspace for kv2_fit_psac_basis, in bytes: 2*H_kv*d*d*8 (fp64 Gram
+ * matrices and eigenvector accumulators). Returns 0 for unsupported shapes.
+ */
+size_t kv2_fit_workspace_size(int H_kv, int d);
+
+/*
+ * kv2_fit_psac_basis — Query statistics of article section "2. PSAC"
+ * (historical Query energy concentrates in a few principal directions) and
+ * the sensitivity weights of "1. QSAC".
+ * Qhist  : bf16 [n][H_q][d] history (calibration) queries. For KV head h the
+ *          statistics pool the n*G vectors of its query heads h*G..h*G+G-1
+ *          (G = H_q/H_kv).
+ * Outputs (fp32, device): S = (1/(n*G)) sum q q^T (uncentred second moment),
+ *   w[h][c] = S_cc; Wg[h][g] = sum of w over group g's 32 channels;
+ *   P[h][c][i] = i-th eigenvector of S by decreasing eigenvalue (i < r), sign
+ *   fixed so its largest-magnitude entry is positive; energy[h] (may be NULL)
+ *   = share of trace(S) in the top r eigenvalues.
+ * Method on the device: fp64 Gram accumulation, cyclic Jacobi in fp64.
+ * ws: device workspace of kv2_fit_workspace_size(H_kv, d) bytes.
+ */
+kv2_status kv2_fit_psac_basis(const uint16_t* Qhist, int n, int H_q, int H_kv, int d,
+                              int r, float* P, float* w, float* Wg, float* energy,
+                              void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * kv2_quantize_append — QSAC centroid assignment, INT2 residual/value
+ * packing and PSAC coefficients for n_new new tokens of every (batch, KV
+ * head), written to slots [pos, pos + n_new) (article "1. QSAC", "2. PSAC").
+ * K, V   : bf16 [B][n_new][H_kv][d].
+ * candidates (C, 1..M): the C centres of smallest ranking score
+ *   score_j = nrm_j - 2 sum_c (w_c k_c) mu_jc   (= weighted squared distance
+ *   minus the key's own weighted norm), ties to the lower id, are kept; the one
+ *   whose residual gives the least E_j = sum_g W_g s_g^2 (s_g the group's fp16
+ *   scale) is chosen, ties to the better-ranked. C = 1 with w = 1 is the plain
+ *   nearest-centre (QVG) assignment.
+ * Codec per group of 32 (residual k - mu for keys, v for values): zero =
+ *   fp16 round-down of the minimum, scale = fp16 round-up of (max - zero)/3,
+ *   code = clamp(round-half-even((x - zero)/scale), 0, 3) (0 when scale = 0).
+ * PSAC: a_i = sum_c P_ci (x_c - fmaf(code_c, s, z)), rounded to fp16.
+ * All quantizer decisions are taken in fp32 in the order stated in the oracle
+ * and are reproducible bit for bit. Tokens outside [pos, pos+n_new) are never
+ * read or written; concurrent calls on overlapping slots race.
+ * Errors: KV2_ERR_CAPACITY if pos < 0 or pos + n_new > capacity.
+ */
+kv2_status kv2_quantize_append(const kv2_cache* cache, const uint16_t* K, const uint16_t* V,
+                               int n_new, int pos, int candidates, void* stream);
+
+/*
+ * Workspace for kv2_attention_decode, in bytes (per-query-head centroid
+ * logits qmu[M], q P, and the split-K partials). Returns 0 for unsupported
+ * shapes.
+ */
+size_t kv2_decode_workspace_size(const kv2_cache* cache, int H_q, int len);
+
+/*
+ * kv2_attention_decode — one query token per sequence against the first
+ * `len` cached tokens of every (batch, KV head), reading the packed cache
+ * directly: logit_t = sm_scale * (q.mu[cidx_t] + sum_g (s_g sum_{c in g} q_c
+ * code_c + z_g sum_{c in g} q_c) + (qP).a_t); online softmax; values
+ * dequantized in registers. Split-K over the sequence, then a log-sum-exp
+ * merge. fp32 arithmetic throughout.
+ * Q   : bf16 [B][H_q][d]; out: [B][H_q][d], fp32 (KV2_OUT_F32) or bf16
+ *       (KV2_OUT_BF16, round to nearest even). len = 0 writes zeros.
+ * ws  : device workspace of kv2_decode_workspace_size(cache, H_q, len) bytes.
+ */
+kv2_status kv2_attention_decode(const kv2_cache* cache, int len, const uint16_t* Q, int H_q,
+                                float sm_scale, void* out, int out_dtype,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Workspace for kv2_attention_chunk, in bytes (fp16 q P per query). Returns 0
+ * for unsupported shapes.
+ */
+size_t kv2_chunk_workspace_size(const kv2_cache* cache, int H_q, int Nq);
+
+/*
+ * kv2_attention_chunk — Nq queries per (batch, query head) of a video-world-
+ * model chunk against the whole packed cache (first `len` tokens) plus the
+ * chunk's own dense keys/values, block-causal by latent frame: query i sees
+ * every cached token and the self tokens j with j/frame_tokens <= i/frame_tokens.
+ * Tensor cores (tcgen05, accumulators in TMEM): packed key tiles are
+ * dequantized to bf16 centroid + residual in shared memory, the PSAC term
+ * (qP).a enters as fp16 extra contraction columns, value tiles and
+ * probabilities are fp16, accumulation fp32.
+ * Q     : bf16 [B][Nq][H_q][d]; Kself, Vself: bf16 [B][Nq][H_kv][d];
+ * out   : [B][Nq][H_q][d] fp32 or bf16. Requires d = 128.
+ * ws    : device workspace of kv2_chunk_workspace_size(cache, H_q, Nq) bytes.
+ */
+kv2_status kv2_attention_chunk(const kv2_cache* cache, int len, const uint16_t* Q, int H_q,
+                               int Nq, const uint16_t* Kself, const uint16_t* Vself,
+                               int frame_tokens, float sm_scale, void* out, int out_dtype,
+                               void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KV2_H */

@@ -1,0 +1,132 @@
+"""GPU parity of kv2_attention_decode against the fp64 oracle on the same
+packed cache: max-abs 2e-3 and relative L2 1e-3 (fp32 output), and the bf16
+output against the bf16 rounding of the oracle at the same thresholds."""
+import numpy as np
+import pytest
+import torch
+
+import workloads as wl
+from helpers import assert_attention_close, bf16_round, gpu_cache_like, host_cache, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _decode_both(orc, pc, P, length, Q, scale, out_dtype=0):
+    import bit_kv_cache_centroid_b200 as kv2
+    ref = orc.decode(pc, P, length, Q, scale)
+    gc = gpu_cache_like(pc)
+    if pc.r:
+        gc.P.copy_(torch.from_numpy(np.ascontiguousarray(P)))
+    out = kv2.kv2_attention_decode(gc, length, to_dev(Q, torch.int16), scale, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy(), ref
+
+
+def _basis(s, seed):
+    rng = np.random.default_rng(seed)
+    P = np.zeros((s.H_kv, s.d, max(s.r, 0)), np.float32)
+    for h in range(s.H_kv):
+        q, _ = np.linalg.qr(rng.standard_normal((s.d, s.d)))
+        P[h] = q[:, :s.r]
+    return P
+
+
+def test_tiny_oracle_quantized_cache(orc):
+    w = wl.make("tiny")
+    s = w.spec
+    f = orc.fit(w.Qhist, s.H_kv, s.r)
+    pc = host_cache(s, w.centroids)
+    orc.quantize(pc, w.K[:, :s.T], w.V[:, :s.T], 0, s.C, f.P, f.w, f.Wg)
+    scale = 1.0 / np.sqrt(s.d)
+    got, ref = _decode_both(orc, pc, f.P, s.T, w.Qdec, scale)
+    assert_attention_close(got, ref, what="tiny f32")
+    got16, _ = _decode_both(orc, pc, f.P, s.T, w.Qdec, scale, out_dtype=1)
+    assert_attention_close(got16, bf16_round(ref), what="tiny bf16")
+
+
+@pytest.mark.parametrize("d,G,M,r,T,length", [
+    (128, 4, 64, 8, 1200, 1),          # one token
+    (128, 4, 64, 8, 1200, 127),        # under one tile
+    (128, 4, 64, 8, 1200, 129),        # one tile + 1
+    (128, 1, 512, 16, 5200, 5137),     # MHA, u16 ids, rank 16, many tiles + ragged tail
+    (128, 2, 256, 0, 3000, 2999),      # no PSAC
+    (128, 8, 64, 8, 2100, 2049),       # 8 query heads per KV head
+    (64, 4, 16, 8, 900, 899),          # d = 64
+])
+def test_random_packed_caches(orc, d, G, M, r, T, length):
+    s = wl.spec("tiny", d=d, H_kv=2, H_q=2 * G, M=M, r=r, T=T, B=2)
+    pc = wl.random_packed_cache(s, T=T, seed=d + G + M + r)
+    P = _basis(s, 3)
+    rng = np.random.default_rng(T)
+    Q = wl.bf16_bits(rng.standard_normal((s.B, s.H_q, d)).astype(np.float32) * 1.5)
+    got, ref = _decode_both(orc, pc, P, length, Q, 1.0 / np.sqrt(d))
+    assert_attention_close(got, ref, what=f"d{d} G{G} M{M} r{r} len{length}")
+
+
+def test_empty_cache_gives_zeros(orc):
+    s = wl.spec("tiny", T=64)
+    pc = wl.random_packed_cache(s, T=64)
+    Q = wl.bf16_bits(np.ones((1, s.H_q, s.d), np.float32))
+    got, ref = _decode_both(orc, pc, _basis(s, 1), 0, Q, 0.125)
+    assert np.all(got == 0.0) and np.all(ref == 0.0)
+
+
+def test_peaked_attention(orc):
+    """A query aligned with one cached key: the softmax is nearly one-hot, so
+    errors in the logits would show directly in the output."""
+    s = wl.spec("tiny", d=128, H_q=4, H_kv=4, M=64, r=8, T=600)
+    pc = wl.random_packed_cache(s, T=600, seed=5)
+    P = _basis(s, 2)
+    rng = np.random.default_rng(1)
+    Q = wl.bf16_bits(rng.standard_normal((1, 4, 128)).astype(np.float32) * 6.0)
+    got, ref = _decode_both(orc, pc, P, 600, Q, 1.0 / np.sqrt(128))
+    assert_attention_close(got, ref, what="peaked")
+
+
+@pytest.mark.slow
+def test_llm_decode_full_size_sampled(orc):
+    """The LLM decode workload (batch 8, 32/8 heads, d=128, 32,768 cached
+    tokens, M=64, r=8) in the launch configuration the benchmark times; the
+    oracle recomputes the outputs of two sequences."""
+    import bit_kv_cache_centroid_b200 as kv2
+    s = wl.spec("llm_decode")
+    pc = wl.random_packed_cache(s, T=s.T)
+    P = _basis(s, 7)
+    rng = np.random.default_rng(2)
+    Q = wl.bf16_bits(rng.standard_normal((s.B, s.H_q, s.d)).astype(np.float32))
+    gc = gpu_cache_like(pc)
+    gc.P.copy_(torch.from_numpy(P))
+    scale = 1.0 / np.sqrt(s.d)
+    out = kv2.kv2_attention_decode(gc, s.T, to_dev(Q, torch.int16), scale, out_dtype=kv2.KV2_OUT_BF16)
+    out32 = kv2.kv2_attention_decode(gc, s.T, to_dev(Q, torch.int16), scale)
+    torch.cuda.synchronize()
+    for b in (0, s.B - 1):
+        sub = wl.PackedCache(1, s.H_kv, s.d, s.M, s.r, pc.capacity, pc.k_code[b:b + 1], pc.v_code[b:b + 1],
+                             pc.k_sz[b:b + 1], pc.v_sz[b:b + 1], pc.cidx[b:b + 1], pc.psac[b:b + 1],
+                             pc.centroids)
+        ref = orc.decode(sub, P, s.T, Q[b:b + 1], scale)
+        assert_attention_close(out32[b:b + 1].cpu().numpy(), ref, what=f"llm f32 b{b}")
+        assert_attention_close(out[b:b + 1].float().cpu().numpy(), bf16_round(ref), what=f"llm bf16 b{b}")
+
+
+@pytest.mark.slow
+def test_long_horizon_decode_full_size_sampled(orc):
+    """Long-horizon memory: 187,200 cached tokens (120 latent frames, frames
+    30/60/90 revisiting frame 0), 40 heads, M=512, r=16, one query per head;
+    the oracle recomputes 4 heads."""
+    import bit_kv_cache_centroid_b200 as kv2
+    s = wl.spec("long_horizon")
+    pc = wl.random_packed_cache(s, T=s.T, revisit_every=30)
+    P = _basis(s, 9)
+    rng = np.random.default_rng(3)
+    Q = wl.bf16_bits(rng.standard_normal((1, s.H_q, s.d)).astype(np.float32))
+    gc = gpu_cache_like(pc)
+    gc.P.copy_(torch.from_numpy(P))
+    scale = 1.0 / np.sqrt(s.d)
+    out = kv2.kv2_attention_decode(gc, s.T, to_dev(Q, torch.int16), scale).cpu().numpy()
+    heads = [0, 13, 27, 39]
+    sub = wl.PackedCache(1, len(heads), s.d, s.M, s.r, pc.capacity, pc.k_code[:, heads], pc.v_code[:, heads],
+                         pc.k_sz[:, heads], pc.v_sz[:, heads], pc.cidx[:, heads], pc.psac[:, heads],
+                         pc.centroids[heads])
+    ref = orc.decode(sub, P[heads], s.T, Q[:, heads], scale)
+    assert_attention_close(out[:, heads], ref, what="long-horizon decode")

@@ -1,0 +1,123 @@
+"""GPU parity of kv2_quantize_append against the oracle (same seeded inputs,
+same fitted statistics): centroid ids, INT2 code words and packed bytes
+bit-exact; fp16 scales, zeros and PSAC coefficients within 1 fp16 ulp."""
+import numpy as np
+import pytest
+import torch
+
+import workloads as wl
+from helpers import f16_ulp_diff, gpu_cache_like, host_cache, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _compare(pc_ref, got, slots=None, what=""):
+    """slots: (b, h, t) index arrays to compare, else everything."""
+    def sel(a):
+        return a if slots is None else a[slots]
+    for name in ("k_code", "v_code"):
+        np.testing.assert_array_equal(sel(got[name]), sel(getattr(pc_ref, name)), err_msg=f"{what} {name}")
+    np.testing.assert_array_equal(sel(got["cidx"]), sel(pc_ref.cidx), err_msg=f"{what} cidx")
+    for name in ("k_sz", "v_sz"):
+        a, b = sel(got[name]), sel(getattr(pc_ref, name))
+        for half in (0, 16):
+            d = f16_ulp_diff((a >> half) & 0xFFFF, (b >> half) & 0xFFFF)
+            assert d.max() <= 1, f"{what} {name} differs by {d.max()} ulp"
+    if pc_ref.r:
+        d = f16_ulp_diff(sel(got["psac"]), sel(pc_ref.psac[..., :pc_ref.r]))
+        assert d.max() <= 1, f"{what} psac differs by {d.max()} ulp"
+    exact = {n: float(np.mean(sel(got[n]) == sel(getattr(pc_ref, n)))) for n in ("k_sz", "v_sz")}
+    return exact
+
+
+def _run(orc, s: wl.Spec, pos=0, n_tok=None, C=None, unit_w=False, seed=None):
+    w = wl.make(s.name, seed=seed, **{k: getattr(s, k) for k in
+                                      ("B", "H_q", "H_kv", "d", "M", "r", "T", "n_new", "n_hist", "Nq")})
+    s = w.spec
+    C = s.C if C is None else C
+    n_tok = s.T if n_tok is None else n_tok
+    f = orc.fit(w.Qhist, s.H_kv, s.r)
+    if unit_w:
+        f.w[:] = 1.0
+        f.Wg[:] = 32.0
+    cap = (pos + n_tok + 15) // 16 * 16 + 16
+    ref = host_cache(s, w.centroids, capacity=cap)
+    K = np.ascontiguousarray(w.K[:, :n_tok])
+    V = np.ascontiguousarray(w.V[:, :n_tok])
+    orc.quantize(ref, K, V, pos, C, f.P, f.w, f.Wg)
+    import bit_kv_cache_centroid_b200 as kv2
+    gc = gpu_cache_like(host_cache(s, w.centroids, capacity=cap), fit=f)
+    kv2.kv2_quantize_append(gc, to_dev(K, torch.int16), to_dev(V, torch.int16), pos, C)
+    torch.cuda.synchronize()
+    return ref, gc.to_host()
+
+
+def test_tiny_bit_exact(orc):
+    ref, got = _run(orc, wl.spec("tiny"))
+    exact = _compare(ref, got, what="tiny")
+    assert exact["k_sz"] == 1.0 and exact["v_sz"] == 1.0
+
+
+@pytest.mark.parametrize("M,C,r,B,n_tok,pos", [
+    (64, 4, 8, 2, 203, 5),       # LLM-like table, ragged token count, unaligned position
+    (256, 8, 8, 1, 150, 37),     # video table: several key tiles + a ragged tail
+    (512, 8, 16, 1, 77, 0),      # long-horizon table (u16 ids), rank 16
+    (100, 3, 0, 1, 65, 16),      # M not a multiple of 32, no PSAC
+    (256, 256, 8, 1, 40, 0),     # candidates = M: brute-force choice
+    (33, 1, 16, 2, 70, 3),       # candidates = 1
+])
+def test_mid_sizes_bit_exact(orc, M, C, r, B, n_tok, pos):
+    s = wl.spec("tiny", d=128, H_q=4, H_kv=2, M=M, r=r, B=B, T=n_tok, n_new=1, n_hist=64, Nq=0)
+    ref, got = _run(orc, s, pos=pos, n_tok=n_tok, C=C)
+    _compare(ref, got, what=f"M{M} C{C} r{r}")
+
+
+def test_nearest_centre_mode(orc):
+    """candidates = 1 with unit weights: plain nearest-centre assignment."""
+    s = wl.spec("tiny", d=64, M=16, r=8)
+    ref, got = _run(orc, s, C=1, unit_w=True)
+    _compare(ref, got, what="qvg")
+
+
+def test_video_keys_bit_exact(orc):
+    """Video-law keys (smooth fields, outlier channels) at d=128, M=256, C=8."""
+    s = wl.spec("quant_append", H_q=2, H_kv=2, T=320, n_new=1, n_hist=128, Nq=0, frame_tokens=160)
+    ref, got = _run(orc, s, n_tok=300)
+    _compare(ref, got, what="video")
+
+
+@pytest.mark.slow
+def test_quant_append_full_size_sampled(orc):
+    """The full quantize/append workload (4,680 new tokens x 40 heads appended
+    at 37,440, M=256, C=8, r=8) in the launch configuration the benchmark
+    times; the oracle recomputes a sample of 24 tokens x 40 heads."""
+    import bit_kv_cache_centroid_b200 as kv2
+    s = wl.spec("quant_append")
+    w = wl.make("quant_append")
+    f = orc.fit(w.Qhist, s.H_kv, s.r)
+    cap = (s.capacity + 15) // 16 * 16
+    gc = gpu_cache_like(host_cache(s, w.centroids, capacity=cap), fit=f)
+    K = np.ascontiguousarray(w.K_new)
+    V = np.ascontiguousarray(w.V_new)
+    kv2.kv2_quantize_append(gc, to_dev(K, torch.int16), to_dev(V, torch.int16), s.T, s.C)
+    torch.cuda.synchronize()
+    got = gc.to_host()
+    rng = np.random.default_rng(11)
+    toks = np.sort(rng.choice(s.n_new, 24, replace=False))
+    toks[-1] = s.n_new - 1                       # include the ragged last tile
+    ref = host_cache(s, w.centroids, capacity=cap)
+    # the oracle appends the sampled tokens at their own slots one by one
+    for t in toks:
+        orc.quantize(ref, K[:, t:t + 1], V[:, t:t + 1], s.T + int(t), s.C, f.P, f.w, f.Wg)
+    bb, hh, tt = np.meshgrid(np.arange(s.B), np.arange(s.H_kv), s.T + toks, indexing="ij")
+    _compare(ref, got, slots=(bb.ravel(), hh.ravel(), tt.ravel()), what="quant_append full")
+
+
+def test_capacity_overflow_rejected():
+    import bit_kv_cache_centroid_b200 as kv2
+    s = wl.spec("tiny")
+    c = kv2.Cache(1, 2, 64, 16, 8, 32, torch.zeros(2, 16, 64, dtype=torch.int16))
+    K = torch.zeros(1, 8, 2, 64, dtype=torch.int16, device="cuda")
+    with pytest.raises(kv2.Kv2Error) as e:
+        kv2.kv2_quantize_append(c, K, K, 30, 1)
+    assert e.value.status == 3

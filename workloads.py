@@ -336,7 +336,7 @@ class PackedCache:
 
     @staticmethod
     def empty(B, H_kv, d, M, r, capacity, centroids):
-        cap = capacity
+        cap = (capacity + 15) // 16 * 16          # the library wants capacity % 16 == 0
         return PackedCache(
             B, H_kv, d, M, r, cap,
             np.zeros((B, H_kv, cap, d // 16), np.uint32),
@@ -360,7 +360,7 @@ def random_packed_cache(s: Spec, T: int | None = None, seed: int | None = None,
     so that retrieval targets recur (long-horizon workload)."""
     T = s.T if T is None else T
     rng = np.random.default_rng((s.seed if seed is None else seed) + 1000)
-    cap = max(s.capacity, T)
+    cap = (max(s.capacity, T) + 15) // 16 * 16
     if centroids is None:
         centroids = f16_bits(rng.standard_normal((s.H_kv, s.M, s.d)).astype(np.float32))
     pc = PackedCache.empty(s.B, s.H_kv, s.d, s.M, s.r, cap, centroids)
