@@ -71,7 +71,24 @@ def _load():
     return L
 
 
-lib = _load()
+_lib = None
+
+
+def _get_lib():
+    global _lib
+    if _lib is None:
+        _lib = _load()
+    return _lib
+
+
+def __getattr__(name):
+    # ``lib`` is loaded on first use so that the build step can import this
+    # package before libkv2.so exists; any use without the library raises.
+    if name == "lib":
+        return _get_lib()
+    raise AttributeError(name)
+
+
 EXPORTS = ["kv2_status_string", "kv2_last_error", "kv2_version", "kv2_fit_workspace_size",
            "kv2_fit_psac_basis", "kv2_quantize_append", "kv2_decode_workspace_size",
            "kv2_attention_decode", "kv2_chunk_workspace_size", "kv2_attention_chunk"]
@@ -79,7 +96,7 @@ EXPORTS = ["kv2_status_string", "kv2_last_error", "kv2_version", "kv2_fit_worksp
 
 def _check(status: int):
     if status != KV2_OK:
-        raise Kv2Error(status, lib.kv2_last_error().decode())
+        raise Kv2Error(status, _get_lib().kv2_last_error().decode())
 
 
 def _ptr(t):
@@ -147,7 +164,7 @@ class Cache:
 # ----------------------------------------------------------------------------
 
 def kv2_fit_workspace_size(H_kv: int, d: int) -> int:
-    return int(lib.kv2_fit_workspace_size(H_kv, d))
+    return int(_get_lib().kv2_fit_workspace_size(H_kv, d))
 
 
 def kv2_fit_psac_basis(Qhist: torch.Tensor, H_kv: int, r: int, P=None, w=None, Wg=None,
@@ -161,7 +178,7 @@ def kv2_fit_psac_basis(Qhist: torch.Tensor, H_kv: int, r: int, P=None, w=None, W
     energy = torch.empty(H_kv, dtype=torch.float32, device=dev) if energy is None else energy
     need = kv2_fit_workspace_size(H_kv, d)
     ws = torch.empty(need, dtype=torch.uint8, device=dev) if ws is None else ws
-    _check(lib.kv2_fit_psac_basis(_ptr(Qhist), n, H_q, H_kv, d, r, _ptr(P), _ptr(w), _ptr(Wg),
+    _check(_get_lib().kv2_fit_psac_basis(_ptr(Qhist), n, H_q, H_kv, d, r, _ptr(P), _ptr(w), _ptr(Wg),
                                   _ptr(energy), _ptr(ws), ws.numel(), _stream(stream)))
     return P[:, :, :r], w, Wg, energy
 
@@ -171,13 +188,13 @@ def kv2_quantize_append(cache: Cache, K: torch.Tensor, V: torch.Tensor, pos: int
     """K, V bf16 [B][n_new][H_kv][d] (device) -> written into cache slots [pos, pos+n_new)."""
     d = cache.desc()
     n_new = K.shape[1]
-    _check(lib.kv2_quantize_append(ctypes.byref(d), _ptr(K), _ptr(V), n_new, pos, candidates,
+    _check(_get_lib().kv2_quantize_append(ctypes.byref(d), _ptr(K), _ptr(V), n_new, pos, candidates,
                                    _stream(stream)))
 
 
 def kv2_decode_workspace_size(cache: Cache, H_q: int, length: int) -> int:
     d = cache.desc()
-    return int(lib.kv2_decode_workspace_size(ctypes.byref(d), H_q, length))
+    return int(_get_lib().kv2_decode_workspace_size(ctypes.byref(d), H_q, length))
 
 
 def kv2_attention_decode(cache: Cache, length: int, Q: torch.Tensor, sm_scale: float,
@@ -191,14 +208,14 @@ def kv2_attention_decode(cache: Cache, length: int, Q: torch.Tensor, sm_scale: f
         ws = torch.empty(max(kv2_decode_workspace_size(cache, H_q, length), 16), dtype=torch.uint8,
                          device=Q.device)
     d = cache.desc()
-    _check(lib.kv2_attention_decode(ctypes.byref(d), length, _ptr(Q), H_q, float(sm_scale), _ptr(out),
+    _check(_get_lib().kv2_attention_decode(ctypes.byref(d), length, _ptr(Q), H_q, float(sm_scale), _ptr(out),
                                     out_dtype, _ptr(ws), ws.numel(), _stream(stream)))
     return out
 
 
 def kv2_chunk_workspace_size(cache: Cache, H_q: int, Nq: int) -> int:
     d = cache.desc()
-    return int(lib.kv2_chunk_workspace_size(ctypes.byref(d), H_q, Nq))
+    return int(_get_lib().kv2_chunk_workspace_size(ctypes.byref(d), H_q, Nq))
 
 
 def kv2_attention_chunk(cache: Cache, length: int, Q: torch.Tensor, Kself: torch.Tensor,
@@ -213,7 +230,7 @@ def kv2_attention_chunk(cache: Cache, length: int, Q: torch.Tensor, Kself: torch
         ws = torch.empty(max(kv2_chunk_workspace_size(cache, H_q, Nq), 16), dtype=torch.uint8,
                          device=Q.device)
     d = cache.desc()
-    _check(lib.kv2_attention_chunk(ctypes.byref(d), length, _ptr(Q), H_q, Nq, _ptr(Kself), _ptr(Vself),
+    _check(_get_lib().kv2_attention_chunk(ctypes.byref(d), length, _ptr(Q), H_q, Nq, _ptr(Kself), _ptr(Vself),
                                    frame_tokens, float(sm_scale), _ptr(out), out_dtype, _ptr(ws),
                                    ws.numel(), _stream(stream)))
     return out
