@@ -60,6 +60,16 @@ kv2_status check_cache(const kv2_cache* c, bool need_cache_streams, bool need_fi
 
 }  // namespace
 
+namespace kv2 {
+kv2_status set_last_error(kv2_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+}  // namespace kv2
+
 extern "C" {
 
 const char* kv2_status_string(kv2_status s) {

@@ -76,4 +76,7 @@ struct ChunkArgs {
 size_t chunk_workspace_bytes(const kv2_cache& c, int H_q, int Nq);
 cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t s);
 
+// Records the detail returned by kv2_last_error() on this thread; returns st.
+kv2_status set_last_error(kv2_status st, const char* fmt, ...);
+
 }  // namespace kv2

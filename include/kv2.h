@@ -163,6 +163,28 @@ kv2_status kv2_attention_decode(const kv2_cache* cache, int len, const uint16_t*
                                 void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * kv2_attention_decode_noalloc — the same computation and arguments as
+ * kv2_attention_decode, minus the workspace: the scratch lives in a fixed
+ * 8 MiB array inside the library, so the caller allocates nothing. It serves
+ * callers that may not allocate device memory themselves (a plugin inside a
+ * framework that owns the allocator, a serving loop where cudaMalloc would
+ * synchronize the device). The paper has no counterpart; it is a convenience
+ * of this library.
+ *  - Shapes whose kv2_decode_workspace_size exceeds 8 MiB (8388608 bytes) are
+ *    rejected with KV2_ERR_WORKSPACE.
+ *  - Every GPU that loads the library holds the 8 MiB array until exit.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) and caches it; make that first call before any
+ *    stream capture.
+ *  - All calls share the array and it keeps the last call's contents: calls
+ *    that overlap on the GPU race on it and must be serialized by the caller.
+ *  - No cudaMalloc, cudaFree or other allocating call is made.
+ */
+kv2_status kv2_attention_decode_noalloc(const kv2_cache* cache, int len, const uint16_t* Q,
+                                        int H_q, float sm_scale, void* out, int out_dtype,
+                                        void* stream);
+
+/*
  * Workspace for kv2_attention_chunk, in bytes (fp16 q P per query). Returns 0
  * for unsupported shapes.
  */
