@@ -267,6 +267,7 @@ def extras(torch, kv2, args, pk):
                        "GBps": round((rd + wr) / (ms * 1e-3) / 1e9, 2),
                        "hbm_frac": round((rd + wr) / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
                        "ranking_TFMAps": round(fma / (ms * 1e-3) / 1e12, 3)}
+    out["chunk"] = chunk_section(torch, kv2, args, pk)
     a.record()
     for _ in range(3):
         kv2.kv2_fit_psac_basis(Qh, s.H_kv, s.r)
@@ -274,6 +275,59 @@ def extras(torch, kv2, args, pk):
     torch.cuda.synchronize()
     out["fit"] = {"workload": "40 heads x 512 history queries, d=128, r=8", "ms": round(a.elapsed_time(b) / 3, 3)}
     return out
+
+
+def chunk_flops(s: wl.Spec, length: int) -> float:
+    """Algorithmic FLOPs of one chunk call: 4 d per (query, visible key) for
+    Q K^T and P V, plus 2 x 16 per (query, cached key) for the PSAC columns."""
+    F = s.frame_tokens
+    f = np.arange(s.Nq) // F
+    self_seen = np.minimum((f + 1) * F, s.Nq).astype(np.float64)
+    per_head = (4.0 * s.d * (length + self_seen) + (2.0 * 16 * length if s.r else 0.0)).sum()
+    return float(per_head * s.H_q * s.B)
+
+
+def chunk_section(torch, kv2, args, pk):
+    """Video world-model chunk attention: 40 heads, 37,440 cached tokens, 4,680
+    queries (3 latent frames), block-causal by frame, M=256, r=8 (packed cache
+    drawn directly in the packed format)."""
+    s = wl.spec("video_chunk")
+    pc = wl.random_packed_cache(s, T=s.T)
+    cache = kv2.Cache(s.B, s.H_kv, s.d, s.M, s.r, pc.capacity, torch.from_numpy(pc.centroids.view(np.int16)))
+    cache.load_packed(pc)
+    rng = np.random.default_rng(3)
+    P = np.zeros((s.H_kv, s.d, s.r), np.float32)
+    for h in range(s.H_kv):
+        q, _ = np.linalg.qr(rng.standard_normal((s.d, s.d)))
+        P[h] = q[:, :s.r]
+    cache.P.copy_(torch.from_numpy(P))
+    dev = lambda x: torch.from_numpy(wl.bf16_bits(x).view(np.int16)).cuda()
+    Q = dev(rng.standard_normal((1, s.Nq, s.H_q, s.d)).astype(np.float32))
+    Ks = dev(rng.standard_normal((1, s.Nq, s.H_kv, s.d)).astype(np.float32))
+    Vs = dev(rng.standard_normal((1, s.Nq, s.H_kv, s.d)).astype(np.float32))
+    out = torch.empty((1, s.Nq, s.H_q, s.d), dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(kv2.kv2_chunk_workspace_size(cache, s.H_q, s.Nq), dtype=torch.uint8, device="cuda")
+    scale = 1.0 / math.sqrt(s.d)
+    run = lambda: kv2.kv2_attention_chunk(cache, s.T, Q, Ks, Vs, s.frame_tokens, scale,
+                                          out_dtype=kv2.KV2_OUT_BF16, out=out, ws=ws)
+    for _ in range(2):
+        run()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = 3
+    a.record()
+    for _ in range(n):
+        run()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / n
+    fl = chunk_flops(s, s.T)
+    tf = fl / (ms * 1e-3) / 1e12
+    return {"workload": "video_chunk: 40 heads, d=128, 37,440 cached + 4,680 queries (3 frames), "
+                        "block-causal, M=256, r=8, bf16 out",
+            "ms": round(ms, 3), "tflop": round(fl / 1e12, 4), "TFLOPs": round(tf, 1),
+            "tensor_frac": round(tf / pk["bf16_tflops"], 4), "peak_tflops": pk["bf16_tflops"],
+            "timeout_flag": int(ws[:4].view(torch.int32).item())}
 
 
 # ----------------------------------------------------------------------------
@@ -328,7 +382,7 @@ def main():
     ap.add_argument("--skip-extras", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--only", choices=["decode", "quantize"], default=None,
+    ap.add_argument("--only", choices=["decode", "quantize", "chunk"], default=None,
                     help="run one section only (for profiler captures)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -348,6 +402,11 @@ def main():
         import torch
         import bit_kv_cache_centroid_b200 as kv2
         print(json.dumps(extras(torch, kv2, args, peaks()[0])), flush=True)
+        return
+    if args.only == "chunk":
+        import torch
+        import bit_kv_cache_centroid_b200 as kv2
+        print(json.dumps(chunk_section(torch, kv2, args, peaks()[0])), flush=True)
         return
     if args.only == "decode":
         args.skip_extras, args.no_cpu = True, True

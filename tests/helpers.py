@@ -24,6 +24,25 @@ def assert_attention_close(got, ref, max_abs=2e-3, rel=1e-3, what=""):
     return err, r
 
 
+def assert_bf16_attention_close(got, ref, max_abs=2e-3, rel=1e-3, what=""):
+    """A bf16 output is the kernel's fp32 result rounded to bf16: within the fp32
+    tolerance of the oracle plus half a bf16 ulp of the value (the output's own
+    rounding, which can fall on the other side of a rounding boundary than the
+    rounding of the oracle), and within the relative-L2 tolerance of the bf16
+    rounding of the oracle."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    a = np.abs(ref)
+    ulp = np.where(a > 0, 2.0 ** (np.floor(np.log2(np.maximum(a, 1e-38))) - 7), 2.0 ** -133)
+    err = np.abs(got - ref)
+    bad = err > max_abs + 0.5 * ulp
+    r = rel_l2(got, bf16_round(ref))
+    assert not bad.any() and r <= rel, \
+        f"{what}: {int(bad.sum())} elements beyond max-abs {max_abs} + ulp/2 (worst {err.max():.3e}); rel-L2 {r:.3e}"
+    return float(err.max()), r
+
+
 def bf16_round(x):
     """fp64/fp32 -> bf16 -> fp32 (round to nearest even) via torch."""
     import torch

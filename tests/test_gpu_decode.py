@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import workloads as wl
-from helpers import assert_attention_close, bf16_round, gpu_cache_like, host_cache, to_dev
+from helpers import assert_attention_close, assert_bf16_attention_close, bf16_round, gpu_cache_like, host_cache, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -41,7 +41,7 @@ def test_tiny_oracle_quantized_cache(orc):
     got, ref = _decode_both(orc, pc, f.P, s.T, w.Qdec, scale)
     assert_attention_close(got, ref, what="tiny f32")
     got16, _ = _decode_both(orc, pc, f.P, s.T, w.Qdec, scale, out_dtype=1)
-    assert_attention_close(got16, bf16_round(ref), what="tiny bf16")
+    assert_bf16_attention_close(got16, ref, what="tiny bf16")
 
 
 @pytest.mark.parametrize("d,G,M,r,T,length", [
@@ -106,7 +106,7 @@ def test_llm_decode_full_size_sampled(orc):
                              pc.centroids)
         ref = orc.decode(sub, P, s.T, Q[b:b + 1], scale)
         assert_attention_close(out32[b:b + 1].cpu().numpy(), ref, what=f"llm f32 b{b}")
-        assert_attention_close(out[b:b + 1].float().cpu().numpy(), bf16_round(ref), what=f"llm bf16 b{b}")
+        assert_bf16_attention_close(out[b:b + 1].float().cpu().numpy(), ref, what=f"llm bf16 b{b}")
 
 
 @pytest.mark.slow
