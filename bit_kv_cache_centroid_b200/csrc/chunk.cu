@@ -11,17 +11,27 @@
 //   S  = Q . Khat^T           bf16 x bf16, Khat = bf16(fmaf(code, s, z) + mu[idx])
 //      + U . A^T              fp16 x fp16, U = fp16(q P), A = the stored fp16
 //                             PSAC coefficients (K = 16 extra contraction columns)
-//   O  = P . Vhat             fp16 x fp16, Vhat = fp16(fmaf(code, s, z)), P = fp16
+//   O += P . Vhat             fp16 x fp16, Vhat = fp16(fmaf(code, s, z)), P = fp16
 //
-// Packed key/value tiles are dequantized into shared memory in the canonical
-// 128-byte-swizzled layouts the MMA descriptors describe; no dense cache is
-// kept anywhere. One CTA handles 128 queries of one (batch, query head); TMEM
-// holds S (128 columns) and the tile's P.V (128 columns); the softmax keeps
-// the running max / sum / output in registers (thread = query row = TMEM lane).
+// One CTA (17 warps) serves two 128-query tiles of one (batch, query head);
+// every dequantized key/value tile feeds both. Warp roles:
+//   warps 0-3, 4-7  softmax of query tile 0 / 1 (thread = query row = TMEM lane):
+//                   S from TMEM, online softmax, P written back into the S
+//                   columns as fp16 pairs, O rescaled in TMEM when a row max grows;
+//   warps 8-15      producer (two threads per key row, 64 channels each):
+//                   packed key/value tiles -> 128-byte-swizzled bf16 Khat /
+//                   fp16 Vhat / fp16 PSAC tiles in a 2-stage ring;
+//   warp 16         issues the MMAs (one thread) and owns the TMEM allocation.
+// TMEM (512 columns): S0, S1, O0, O1. The PV MMA reads P straight from TMEM.
+// mbarriers: kv_full/kv_empty (ring), s_full, p_full, o_done (per query tile).
+// A commit covers every earlier MMA of the issuing thread, so "S of tile j
+// done" also means "P.V of tile j-1 done": the softmax may then overwrite P
+// and rescale O.
 //
-// Every mbarrier wait is bounded by a clock-cycle budget; a wait that runs out
-// records 1 in the first word of the workspace and the CTA waits (bounded) for
-// its MMAs in flight, frees its TMEM and returns.
+// Every wait is bounded by an SM-clock budget; on expiry the waiting thread
+// raises a CTA-wide abort flag that ends every other wait, the kernel records
+// 1 in the workspace's first word, waits (bounded) for its MMAs in flight,
+// frees its TMEM and returns.
 #include <cfloat>
 #include <cstdlib>
 
@@ -31,23 +41,30 @@
 namespace kv2 {
 namespace {
 
-constexpr int kRows = 128;       // queries per CTA (= TMEM lanes)
-constexpr int kKeys = 128;       // keys per tile
+constexpr int kRows = 128;        // queries per query tile (= TMEM lanes)
+constexpr int kKeys = 128;        // keys per tile
 constexpr int kD = 128;
-constexpr int kThreads = 128;
+constexpr int kThreads = 544;     // 17 warps
+constexpr int kProdWarp0 = 8, kProdThreads = 256, kMmaWarp = 16;
 
 // shared-memory map (offsets from a 1024-byte aligned base)
-constexpr uint32_t OFF_Q = 0;            // Q    [2 k-chunks][128 rows][128 B], SW128, K-major
-constexpr uint32_t OFF_K = 32768;        // Khat [2 k-chunks][128 keys][128 B], SW128, K-major
-constexpr uint32_t OFF_V = 65536;        // Vhat [2 n-blocks][128 keys][128 B], SW128, MN-major
-constexpr uint32_t OFF_P = 98304;        // P    [2 k-chunks][128 rows][128 B], SW128, K-major
-constexpr uint32_t OFF_U = 131072;       // U    [16 row groups][2 k-chunks][8 rows][16 B]
-constexpr uint32_t OFF_A = 135168;       // A    [16 key groups][2 k-chunks][8 keys][16 B]
-constexpr uint32_t OFF_BAR = 139264;     // mbarriers + TMEM address
-constexpr uint32_t SMEM_USED = OFF_BAR + 64;
+constexpr uint32_t OFF_Q0 = 0;           // Q tile 0 [2 k-chunks][128 rows][128 B], SW128, K-major
+constexpr uint32_t OFF_Q1 = 32768;       // Q tile 1
+constexpr uint32_t OFF_U0 = 65536;       // U = fp16(qP) tile 0 [16 row groups][2][8 rows][16 B]
+constexpr uint32_t OFF_U1 = 69632;       // U tile 1
+constexpr uint32_t OFF_STAGE = 73728;    // 2 stages of STAGE_BYTES
+constexpr uint32_t ST_K = 0;             // Khat [2 k-chunks][128 keys][128 B], SW128, K-major
+constexpr uint32_t ST_V = 32768;         // Vhat [2 n-blocks][128 keys][128 B], SW128, MN-major
+constexpr uint32_t ST_A = 65536;         // A    [16 key groups][2][8 keys][16 B]
+constexpr uint32_t STAGE_BYTES = 69632;
+constexpr uint32_t OFF_BAR = OFF_STAGE + 2 * STAGE_BYTES;   // 212992
+constexpr uint32_t SMEM_USED = OFF_BAR + 128;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;
+// barrier slots (8 bytes each) from OFF_BAR
+constexpr uint32_t B_KV_FULL = 0, B_KV_EMPTY = 16, B_S_FULL = 32, B_P_FULL = 48, B_O_DONE = 64, B_FINAL = 80,
+                   B_NEVER = 88, B_TMEM_SLOT = 96, B_ABORT = 100;
 
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemCols = 512;
 
 // ---------------------------------------------------------------------------
 // PTX wrappers (sm_100a)
@@ -81,6 +98,19 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
+// A operand from TMEM (K-major: lane = row, each 32-bit column = 2 fp16 values)
+__device__ __forceinline__ void mma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                : "memory");
@@ -93,21 +123,38 @@ __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t phase) {
+// try_wait suspends the calling thread (it issues nothing) until the phase
+// completes or a hardware time limit passes; either way control comes back.
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t phase) {
   uint32_t done;
   asm volatile(
-      "{\n\t.reg .pred P1;\n\tmbarrier.test_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
+      "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
       "selp.b32 %0, 1, 0, P1;\n\t}\n"
       : "=r"(done)
       : "r"(bar), "r"(phase)
       : "memory");
   return done != 0;
 }
-// Bounded wait: spins until the phase completes or `budget` SM clock cycles pass.
+// Bounded wait: until the phase completes or `budget` SM clock cycles pass.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase, unsigned long long budget) {
   const unsigned long long t0 = clock64();
-  while (!mbar_test(bar, phase)) {
+  while (!mbar_try(bar, phase)) {
     if (clock64() - t0 > budget) return false;
+  }
+  return true;
+}
+
+// Bounded wait that also gives up as soon as another role raised the abort
+// flag; a wait that runs out raises it.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint32_t bar, uint32_t phase, unsigned long long budget,
+                                                   volatile int* abort) {
+  const unsigned long long t0 = clock64();
+  while (!mbar_try(bar, phase)) {
+    if (*abort) return false;
+    if (clock64() - t0 > budget) {
+      *abort = 1;
+      return false;
+    }
   }
   return true;
 }
@@ -153,6 +200,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 // byte offset of 16-byte chunk `c16` (0..15) of row `row` in a [2][128][128 B]
 // 128-byte-swizzled operand tile (K-major: chunks along K; MN-major: along N)
 __device__ __forceinline__ uint32_t sw128_off(int row, int c16) {
@@ -164,12 +221,27 @@ __device__ __forceinline__ uint32_t nosw_off(int row, int c) {
   return uint32_t((row >> 3) * 256 + c * 128 + (row & 7) * 16);
 }
 
+// two fp32 -> packed bf16x2 / f16x2 (one paired conversion, round to nearest even)
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  return uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(a))) |
-         (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(b))) << 16);
+  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&v);
 }
 __device__ __forceinline__ uint32_t pack_f16(float a, float b) {
-  return uint32_t(__half_as_ushort(__float2half_rn(a))) | (uint32_t(__half_as_ushort(__float2half_rn(b))) << 16);
+  const __half2 v = __floats2half2_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// 2^x on the MUFU unit (relative error ~2^-22; P is rounded to fp16 after)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Code of bit position 2j of a 16-bit code field as a float times 4^j, exact:
+// (w & (3 << 2j)) | 0x4B000000 is the float 2^23 + code * 4^j.
+__device__ __forceinline__ float code_x4j(uint32_t w, int j) {
+  return __uint_as_float((w & (3u << (2 * j))) | 0x4B000000u) - 8388608.0f;
 }
 
 struct ChunkParams {
@@ -195,73 +267,99 @@ struct ChunkParams {
 // ---------------------------------------------------------------------------
 // operand producers (thread = one row)
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void zero_rows(uint8_t* tile, int row) {
-#pragma unroll
-  for (int c = 0; c < 16; ++c) *reinterpret_cast<uint4*>(tile + sw128_off(row, c)) = make_uint4(0, 0, 0, 0);
+
+// Packed fields of half a cached token row (channels 64*half .. 64*half+63),
+// loaded one tile ahead of their use.
+struct RawHalf {
+  uint4 kw, vw;       // 4 code words each
+  uint2 ksz, vsz;     // 2 groups: fp16 scale | fp16 zero << 16
+  uint4 a0, a1;       // PSAC coefficients (half 0 only)
+  int idx;            // centroid id
+};
+
+__device__ __forceinline__ void load_raw_half(const ChunkParams& p, size_t slot, int half, RawHalf& r) {
+  r.kw = *reinterpret_cast<const uint4*>(p.k_code + slot * 8 + half * 4);
+  r.vw = *reinterpret_cast<const uint4*>(p.v_code + slot * 8 + half * 4);
+  r.ksz = *reinterpret_cast<const uint2*>(p.k_sz + slot * 4 + half * 2);
+  r.vsz = *reinterpret_cast<const uint2*>(p.v_sz + slot * 4 + half * 2);
+  r.idx = (p.M <= 256) ? int(static_cast<const uint8_t*>(p.cidx)[slot])
+                       : int(static_cast<const uint16_t*>(p.cidx)[slot]);
+  r.a0 = make_uint4(0, 0, 0, 0);
+  r.a1 = make_uint4(0, 0, 0, 0);
+  if (half == 0 && p.r >= 8) r.a0 = *reinterpret_cast<const uint4*>(p.psac + slot * p.r);
+  if (half == 0 && p.r >= 16) r.a1 = *reinterpret_cast<const uint4*>(p.psac + slot * p.r + 8);
 }
 
-// cached token -> Khat (bf16) row, PSAC row, Vhat (fp16) row
-__device__ void dequant_cache_row(const ChunkParams& p, size_t slot, int h, int row, uint8_t* smem) {
-  const uint4* kw4 = reinterpret_cast<const uint4*>(p.k_code + slot * 8);
-  const uint4* vw4 = reinterpret_cast<const uint4*>(p.v_code + slot * 8);
-  const uint4 k0 = kw4[0], k1 = kw4[1], v0 = vw4[0], v1 = vw4[1];
-  const uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-  const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-  const uint4 ks = *reinterpret_cast<const uint4*>(p.k_sz + slot * 4);
-  const uint4 vs = *reinterpret_cast<const uint4*>(p.v_sz + slot * 4);
-  const uint32_t ksz[4] = {ks.x, ks.y, ks.z, ks.w};
-  const uint32_t vsz[4] = {vs.x, vs.y, vs.z, vs.w};
-  const int idx = (p.M <= 256) ? int(static_cast<const uint8_t*>(p.cidx)[slot])
-                               : int(static_cast<const uint16_t*>(p.cidx)[slot]);
-  const uint4* mu = reinterpret_cast<const uint4*>(p.cent + (size_t(h) * p.M + min(idx, p.M - 1)) * kD);
+// half a Khat (bf16) row and half a Vhat (fp16) row from the packed fields and
+// the centroid half-row m4; half 0 also writes the PSAC row
+__device__ void dequant_cache_half(const RawHalf& r, const uint4 (&m4)[8], int row, int half, uint8_t* stage) {
+  const uint32_t kw[4] = {r.kw.x, r.kw.y, r.kw.z, r.kw.w};
+  const uint32_t vw[4] = {r.vw.x, r.vw.y, r.vw.z, r.vw.w};
+  const uint32_t ksz[2] = {r.ksz.x, r.ksz.y};
+  const uint32_t vsz[2] = {r.vsz.x, r.vsz.y};
+  // fmaf(code, s, z) with the code read as code * 4^j: the scale carries 4^-j
+  // (exact power-of-two scaling), so the product and its single rounding are
+  // those of fmaf(code, s, z).
 #pragma unroll
-  for (int c16 = 0; c16 < 16; ++c16) {              // 8 channels per chunk
-    const int g = c16 >> 2;
-    const float ksc = __half2float(__ushort_as_half(uint16_t(ksz[g] & 0xffff)));
+  for (int g = 0; g < 2; ++g) {
+    const float ks = __half2float(__ushort_as_half(uint16_t(ksz[g] & 0xffff)));
+    const float vs = __half2float(__ushort_as_half(uint16_t(vsz[g] & 0xffff)));
     const float kz = __half2float(__ushort_as_half(uint16_t(ksz[g] >> 16)));
-    const float vsc = __half2float(__ushort_as_half(uint16_t(vsz[g] & 0xffff)));
     const float vz = __half2float(__ushort_as_half(uint16_t(vsz[g] >> 16)));
-    const uint4 m4 = __ldg(mu + c16);
-    const __half2* mh = reinterpret_cast<const __half2*>(&m4);
-    const uint32_t kword = kw[c16 >> 1] >> ((c16 & 1) * 16);
-    const uint32_t vword = vw[c16 >> 1] >> ((c16 & 1) * 16);
-    uint32_t kb[4], vb[4];
+    float ksc[8], vsc[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 m = __half22float2(mh[i]);
-      const float c0 = float((kword >> (4 * i)) & 3u), c1 = float((kword >> (4 * i + 2)) & 3u);
-      const float k0f = __fadd_rn(__fmaf_rn(c0, ksc, kz), m.x);
-      const float k1f = __fadd_rn(__fmaf_rn(c1, ksc, kz), m.y);
-      kb[i] = pack_bf16(k0f, k1f);
-      const float d0 = float((vword >> (4 * i)) & 3u), d1 = float((vword >> (4 * i + 2)) & 3u);
-      vb[i] = pack_f16(__fmaf_rn(d0, vsc, vz), __fmaf_rn(d1, vsc, vz));
+    for (int j = 0; j < 8; ++j) {
+      ksc[j] = ks * __uint_as_float(uint32_t(127 - 2 * j) << 23);
+      vsc[j] = vs * __uint_as_float(uint32_t(127 - 2 * j) << 23);
     }
-    *reinterpret_cast<uint4*>(smem + OFF_K + sw128_off(row, c16)) = make_uint4(kb[0], kb[1], kb[2], kb[3]);
-    *reinterpret_cast<uint4*>(smem + OFF_V + sw128_off(row, c16)) = make_uint4(vb[0], vb[1], vb[2], vb[3]);
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {                // 8 channels per chunk
+      const int c16 = half * 8 + g * 4 + cc;         // chunk index within the row
+      const int lc = g * 4 + cc;                      // chunk index within this half
+      const __half2* mh = reinterpret_cast<const __half2*>(&m4[lc]);
+      const uint32_t kword = (kw[lc >> 1] >> ((lc & 1) * 16)) & 0xffffu;
+      const uint32_t vword = (vw[lc >> 1] >> ((lc & 1) * 16)) & 0xffffu;
+      uint32_t kb[4], vb[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 m = __half22float2(mh[i]);
+        const float k0f = __fadd_rn(__fmaf_rn(code_x4j(kword, 2 * i), ksc[2 * i], kz), m.x);
+        const float k1f = __fadd_rn(__fmaf_rn(code_x4j(kword, 2 * i + 1), ksc[2 * i + 1], kz), m.y);
+        kb[i] = pack_bf16(k0f, k1f);
+        vb[i] = pack_f16(__fmaf_rn(code_x4j(vword, 2 * i), vsc[2 * i], vz),
+                         __fmaf_rn(code_x4j(vword, 2 * i + 1), vsc[2 * i + 1], vz));
+      }
+      *reinterpret_cast<uint4*>(stage + ST_K + sw128_off(row, c16)) = make_uint4(kb[0], kb[1], kb[2], kb[3]);
+      *reinterpret_cast<uint4*>(stage + ST_V + sw128_off(row, c16)) = make_uint4(vb[0], vb[1], vb[2], vb[3]);
+    }
   }
-  // PSAC coefficients: r (0, 8 or 16) fp16 values, zero-padded to 16
-  uint4 a0 = make_uint4(0, 0, 0, 0), a1 = make_uint4(0, 0, 0, 0);
-  if (p.r >= 8) a0 = *reinterpret_cast<const uint4*>(p.psac + slot * p.r);
-  if (p.r >= 16) a1 = *reinterpret_cast<const uint4*>(p.psac + slot * p.r + 8);
-  *reinterpret_cast<uint4*>(smem + OFF_A + nosw_off(row, 0)) = a0;
-  *reinterpret_cast<uint4*>(smem + OFF_A + nosw_off(row, 1)) = a1;
+  if (half == 0) {
+    *reinterpret_cast<uint4*>(stage + ST_A + nosw_off(row, 0)) = r.a0;
+    *reinterpret_cast<uint4*>(stage + ST_A + nosw_off(row, 1)) = r.a1;
+  }
 }
 
-// chunk token -> Khat row (bf16 copy), Vhat row (bf16 -> fp16)
-__device__ void copy_self_row(const ChunkParams& p, const uint16_t* krow, const uint16_t* vrow, int row,
-                              uint8_t* smem) {
-  const uint4* k4 = reinterpret_cast<const uint4*>(krow);
-  const uint4* v4 = reinterpret_cast<const uint4*>(vrow);
+// chunk token -> half a Khat row (bf16 copy) and half a Vhat row (bf16 -> fp16)
+__device__ void copy_self_half(const uint16_t* krow, const uint16_t* vrow, int row, int half, uint8_t* stage) {
+  const uint4* k4 = reinterpret_cast<const uint4*>(krow) + half * 8;
+  const uint4* v4 = reinterpret_cast<const uint4*>(vrow) + half * 8;
 #pragma unroll
-  for (int c16 = 0; c16 < 16; ++c16) {
-    *reinterpret_cast<uint4*>(smem + OFF_K + sw128_off(row, c16)) = __ldg(k4 + c16);
-    const uint4 v = __ldg(v4 + c16);
+  for (int c = 0; c < 8; ++c) {
+    const int c16 = half * 8 + c;
+    *reinterpret_cast<uint4*>(stage + ST_K + sw128_off(row, c16)) = __ldg(k4 + c);
+    const uint4 v = __ldg(v4 + c);
     const uint32_t u[4] = {v.x, v.y, v.z, v.w};
     uint32_t o[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) o[i] = pack_f16(__uint_as_float(u[i] << 16), __uint_as_float(u[i] & 0xffff0000u));
-    *reinterpret_cast<uint4*>(smem + OFF_V + sw128_off(row, c16)) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(stage + ST_V + sw128_off(row, c16)) = make_uint4(o[0], o[1], o[2], o[3]);
   }
+}
+
+__device__ __forceinline__ void zero_half(uint8_t* tile, int row, int half) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    *reinterpret_cast<uint4*>(tile + sw128_off(row, half * 8 + c)) = make_uint4(0, 0, 0, 0);
 }
 
 // ---------------------------------------------------------------------------
@@ -269,28 +367,36 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
-  const uint32_t bar_s = sb + OFF_BAR, bar_o = sb + OFF_BAR + 8, bar_never = sb + OFF_BAR + 16;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 32);
-  volatile int* s_fail = reinterpret_cast<volatile int*>(smem + OFF_BAR + 40);
+  const uint32_t bar = sb + OFF_BAR;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + B_TMEM_SLOT);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + OFF_BAR + B_ABORT);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qt = blockIdx.x, hq = blockIdx.y, b = blockIdx.z;
   const int G = p.H_q / p.H_kv, h = hq / G;
-  const int q0 = qt * kRows;
-  const int qi = q0 + tid;                  // this thread's query (row, TMEM lane)
-  const bool q_ok = qi < p.Nq;
+  const int q0 = qt * 2 * kRows;
 
   if (tid == 0) {
-    mbar_init(bar_s, 1);
-    mbar_init(bar_o, 1);
-    mbar_init(bar_never, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar + B_KV_FULL + 8 * i, kProdThreads);   // one arrival per producer thread
+      mbar_init(bar + B_KV_EMPTY + 8 * i, 1);         // MMA commit
+      mbar_init(bar + B_S_FULL + 8 * i, 1);           // MMA commit
+      mbar_init(bar + B_P_FULL + 8 * i, kRows);       // one arrival per softmax thread
+      mbar_init(bar + B_O_DONE + 8 * i, 1);           // MMA commit
+    }
+    mbar_init(bar + B_FINAL, 1);
+    mbar_init(bar + B_NEVER, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    *s_fail = 0;
+    *abort = 0;
   }
-  if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+  if (warp == kMmaWarp) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
 
-  // ---- Q tile (bf16, SW128 K-major) and U = fp16(q P) (no swizzle, K = 16)
-  {
+  // ---- Q tiles (bf16, SW128 K-major) and U = fp16(q P) (no swizzle, K = 16)
+  if (warp < 8) {
+    const int x = warp >> 2, row = tid - x * kRows;
+    const int qi = q0 + x * kRows + row;
+    const bool q_ok = qi < p.Nq;
+    uint8_t* qtile = smem + (x ? OFF_Q1 : OFF_Q0);
     float u[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) u[j] = 0.0f;
@@ -299,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
 #pragma unroll 1
     for (int c16 = 0; c16 < 16; ++c16) {
       const uint4 v = q_ok ? __ldg(src + c16) : make_uint4(0, 0, 0, 0);
-      *reinterpret_cast<uint4*>(smem + OFF_Q + sw128_off(tid, c16)) = v;
+      *reinterpret_cast<uint4*>(qtile + sw128_off(row, c16)) = v;
       if (p.r > 0) {
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -315,176 +421,240 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
     uint32_t uw[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) uw[j] = pack_f16(u[2 * j], u[2 * j + 1]);
-    *reinterpret_cast<uint4*>(smem + OFF_U + nosw_off(tid, 0)) = make_uint4(uw[0], uw[1], uw[2], uw[3]);
-    *reinterpret_cast<uint4*>(smem + OFF_U + nosw_off(tid, 1)) = make_uint4(uw[4], uw[5], uw[6], uw[7]);
+    uint8_t* utile = smem + (x ? OFF_U1 : OFF_U0);
+    *reinterpret_cast<uint4*>(utile + nosw_off(row, 0)) = make_uint4(uw[0], uw[1], uw[2], uw[3]);
+    *reinterpret_cast<uint4*>(utile + nosw_off(row, 1)) = make_uint4(uw[4], uw[5], uw[6], uw[7]);
   }
   fence_proxy_async();
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tO = tmem + kKeys;
-  const uint32_t lane_base = uint32_t(warp * 32) << 16;
 
   const int n_cache = (p.len + kKeys - 1) / kKeys;
-  const int last_q = min(q0 + kRows, p.Nq) - 1;
+  const int last_q = min(q0 + 2 * kRows, p.Nq) - 1;
   const int self_len = min(p.Nq, (last_q / p.F + 1) * p.F);
   const int n_self = (self_len + kKeys - 1) / kKeys;
-  const int my_self_lim = min(self_len, (min(qi, p.Nq - 1) / p.F + 1) * p.F);
-
-  float m_run = -INFINITY, l_run = 0.0f;
-  uint32_t phase = 0;
-  bool failed = false;
-  int pending = 0;     // MMA group committed and not yet waited for: 1 = S, 2 = O
   const int n_tiles = n_cache + n_self;
 
-  for (int j = 0; j < n_tiles; ++j) {
-    const bool cache = j < n_cache;
-    const int k0 = cache ? j * kKeys : (j - n_cache) * kKeys;
-    const int kvalid = cache ? min(kKeys, p.len - k0) : min(kKeys, self_len - k0);
-    // ---- produce Khat, A, Vhat rows (the previous tile's MMAs have completed)
-    const int key = k0 + tid;
-    if (tid < kvalid) {
-      if (cache) {
-        dequant_cache_row(p, (size_t(b) * p.H_kv + h) * p.cap + key, h, tid, smem);
+  if (warp == kMmaWarp) {
+    // ================= MMA issue (one thread) =================
+    for (int j = 0; j < n_tiles; ++j) {
+      const int s = j & 1;
+      const uint32_t use = uint32_t(j >> 1);
+      const bool cache = j < n_cache;
+      if (p.force_timeout && j == 0 && !mbar_wait_or_abort(bar + B_NEVER, 0, p.budget, abort)) break;
+      if (!mbar_wait_or_abort(bar + B_KV_FULL + 8 * s, use & 1, p.budget, abort)) break;
+      fence_after_sync();
+      const uint32_t st = sb + OFF_STAGE + s * STAGE_BYTES;
+      bool ok = true;
+      for (int x = 0; x < 2 && ok; ++x) {
+        if (j > 0 && !mbar_wait_or_abort(bar + B_O_DONE + 8 * x, (j - 1) & 1, p.budget, abort)) { ok = false; break; }
+        fence_after_sync();
+        if (lane == 0) {
+          const uint32_t tS = tmem + x * kKeys;
+          const uint32_t qb = sb + (x ? OFF_Q1 : OFF_Q0);
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_f16(tS, make_sdesc(qb + off, 16, 1024, kLayoutSW128),
+                    make_sdesc(st + ST_K + off, 16, 1024, kLayoutSW128), IDESC_QK, kk > 0);
+          }
+          if (cache && p.r > 0)
+            mma_f16(tS, make_sdesc(sb + (x ? OFF_U1 : OFF_U0), 128, 256, kLayoutNone),
+                    make_sdesc(st + ST_A, 128, 256, kLayoutNone), IDESC_UA, 1);
+          mma_commit(bar + B_S_FULL + 8 * x);
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      for (int x = 0; x < 2 && ok; ++x) {
+        if (!mbar_wait_or_abort(bar + B_P_FULL + 8 * x, j & 1, p.budget, abort)) { ok = false; break; }
+        fence_after_sync();
+        if (lane == 0) {
+          const uint32_t tP = tmem + x * kKeys, tO = tmem + 2 * kKeys + x * kD;
+#pragma unroll
+          for (int kk = 0; kk < kKeys / 16; ++kk)
+            mma_f16_tmem_a(tO, tP + kk * 8, make_sdesc(st + ST_V + kk * 2048, 16384, 1024, kLayoutSW128), IDESC_PV,
+                           (j > 0 || kk > 0));
+          mma_commit(bar + B_O_DONE + 8 * x);
+          if (x == 1) mma_commit(bar + B_KV_EMPTY + 8 * s);   // stage free once every MMA on it is done
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+    }
+  } else if (warp >= kProdWarp0) {
+    // ================= producer: packed tiles -> operand tiles =================
+    // The packed fields of cached tile j+1 are loaded while tile j is
+    // dequantized; the centroid half-row is fetched as soon as its id is known.
+    const int pt = tid - kProdWarp0 * 32;
+    const int row = pt >> 1, half = pt & 1;
+    const size_t slot0 = (size_t(b) * p.H_kv + h) * p.cap;
+    const uint4* cent4 = reinterpret_cast<const uint4*>(p.cent) + size_t(h) * p.M * (kD / 8) + half * 8;
+    RawHalf raw;
+    bool raw_ok = (n_cache > 0) && row < min(kKeys, p.len);
+    if (raw_ok) load_raw_half(p, slot0 + row, half, raw);
+    for (int j = 0; j < n_tiles; ++j) {
+      const int s = j & 1;
+      const uint32_t use = uint32_t(j >> 1);
+      const bool cache = j < n_cache;
+      const int k0 = cache ? j * kKeys : (j - n_cache) * kKeys;
+      const int kvalid = cache ? min(kKeys, p.len - k0) : min(kKeys, self_len - k0);
+      uint4 m4[8];
+      if (cache && raw_ok) {
+        const uint4* mu = cent4 + size_t(min(raw.idx, p.M - 1)) * (kD / 8);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) m4[c] = __ldg(mu + c);
+      }
+      RawHalf next;
+      const int jn = j + 1;
+      const bool next_ok = jn < n_cache && row < min(kKeys, p.len - jn * kKeys);
+      if (next_ok) load_raw_half(p, slot0 + size_t(jn) * kKeys + row, half, next);
+      if (use >= 1 && !mbar_wait_or_abort(bar + B_KV_EMPTY + 8 * s, (use - 1) & 1, p.budget, abort)) break;
+      uint8_t* stage = smem + OFF_STAGE + s * STAGE_BYTES;
+      if (row < kvalid) {
+        if (cache) {
+          dequant_cache_half(raw, m4, row, half, stage);
+        } else {
+          const size_t srow = (size_t(b) * p.Nq + k0 + row) * p.H_kv + h;
+          copy_self_half(p.Ks + srow * kD, p.Vs + srow * kD, row, half, stage);
+        }
       } else {
-        const size_t srow = (size_t(b) * p.Nq + key) * p.H_kv + h;
-        copy_self_row(p, p.Ks + srow * kD, p.Vs + srow * kD, tid, smem);
+        zero_half(stage + ST_K, row, half);
+        zero_half(stage + ST_V, row, half);
+        if (half == 0) {
+          *reinterpret_cast<uint4*>(stage + ST_A + nosw_off(row, 0)) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(stage + ST_A + nosw_off(row, 1)) = make_uint4(0, 0, 0, 0);
+        }
       }
-    } else {
-      zero_rows(smem + OFF_K, tid);
-      zero_rows(smem + OFF_V, tid);
-      *reinterpret_cast<uint4*>(smem + OFF_A + nosw_off(tid, 0)) = make_uint4(0, 0, 0, 0);
-      *reinterpret_cast<uint4*>(smem + OFF_A + nosw_off(tid, 1)) = make_uint4(0, 0, 0, 0);
+      fence_proxy_async();
+      mbar_arrive(bar + B_KV_FULL + 8 * s);
+      raw = next;
+      raw_ok = next_ok;
     }
-    fence_proxy_async();
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    // ---- S = Q Khat^T (+ U A^T)
-    if (tid == 0) {
+  } else {
+    // ================= softmax of query tile x =================
+    const int x = warp >> 2, row = tid - x * kRows;
+    const int qi = q0 + x * kRows + row;
+    const bool q_ok = qi < p.Nq;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + x * kKeys + lane_base, tO = tmem + 2 * kKeys + x * kD + lane_base;
+    const int my_self_lim = min(self_len, (min(qi, p.Nq - 1) / p.F + 1) * p.F);
+    float m_run = -INFINITY, l_run = 0.0f;
+    bool done = true;
+    for (int j = 0; j < n_tiles; ++j) {
+      if (!mbar_wait_or_abort(bar + B_S_FULL + 8 * x, j & 1, p.budget, abort)) { done = false; break; }
+      fence_after_sync();
+      const bool cache = j < n_cache;
+      const int k0 = cache ? j * kKeys : (j - n_cache) * kKeys;
+      const int lim = cache ? min(kKeys, p.len - k0) : (my_self_lim - k0);
+      const bool full = __all_sync(0xffffffffu, lim >= kKeys);   // no masked key in the warp's rows
+      // row max and row sum with 8 independent partial accumulators (short
+      // dependency chains on the critical S -> softmax -> P.V path)
+      float mpart[8];
 #pragma unroll
-      for (int kk = 0; kk < kD / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-        mma_f16(tS, make_sdesc(sb + OFF_Q + off, 16, 1024, kLayoutSW128),
-                make_sdesc(sb + OFF_K + off, 16, 1024, kLayoutSW128), IDESC_QK, kk > 0);
+      for (int i = 0; i < 8; ++i) mpart[i] = -INFINITY;
+#pragma unroll 1
+      for (int c0 = 0; c0 < kKeys; c0 += 32) {
+        float v[32];
+        tmem_ld32(tS + c0, v);
+        if (full) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) mpart[i & 7] = fmaxf(mpart[i & 7], v[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c0 + i < lim) mpart[i & 7] = fmaxf(mpart[i & 7], v[i]);
+        }
       }
-      if (cache && p.r > 0)
-        mma_f16(tS, make_sdesc(sb + OFF_U, 128, 256, kLayoutNone), make_sdesc(sb + OFF_A, 128, 256, kLayoutNone),
-                IDESC_UA, 1);
-      mma_commit(bar_s);
-    }
-    pending = 1;
-    if (p.force_timeout && !mbar_wait(bar_never, 0, p.budget)) *s_fail = 1;
-    if (!*s_fail && !mbar_wait(bar_s, phase, p.budget)) *s_fail = 1;
-    __syncthreads();
-    if (*s_fail) { failed = true; break; }
-    pending = 0;
-    fence_after_sync();
-
-    // ---- softmax of this row over the tile; P (fp16) to shared memory
-    const int lim = cache ? kvalid : (my_self_lim - k0);
-    float mt = -INFINITY;
+      const float mt = fmaxf(fmaxf(fmaxf(mpart[0], mpart[1]), fmaxf(mpart[2], mpart[3])),
+                             fmaxf(fmaxf(mpart[4], mpart[5]), fmaxf(mpart[6], mpart[7])));
+      const float m_new = fmaxf(m_run, mt * p.scale_log2);
+      const float alpha = (m_new == -INFINITY) ? 1.0f : ex2(m_run - m_new);
+      float spart[8];
 #pragma unroll
-    for (int c0 = 0; c0 < kKeys; c0 += 32) {
-      float v[32];
-      tmem_ld32(tS + lane_base + c0, v);
+      for (int i = 0; i < 8; ++i) spart[i] = 0.0f;
+#pragma unroll 1
+      for (int c0 = 0; c0 < kKeys; c0 += 32) {
+        float v[32];
+        tmem_ld32(tS + c0, v);
+        uint32_t pw[16];
+        if (full) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (c0 + i < lim) mt = fmaxf(mt, v[i]);
-    }
-    const float m_new = fmaxf(m_run, mt * p.scale_log2);
-    const float alpha = (m_new == -INFINITY) ? 1.0f : exp2f(m_run - m_new);
-    float lsum = 0.0f;
+          for (int i = 0; i < 32; i += 2) {
+            const float p0 = ex2(fmaf(v[i], p.scale_log2, -m_new));
+            const float p1 = ex2(fmaf(v[i + 1], p.scale_log2, -m_new));
+            spart[i & 7] += p0;
+            spart[(i + 1) & 7] += p1;
+            pw[i / 2] = pack_f16(p0, p1);
+          }
+        } else {
 #pragma unroll
-    for (int c0 = 0; c0 < kKeys; c0 += 32) {
-      float v[32];
-      tmem_ld32(tS + lane_base + c0, v);
-      uint32_t pw[16];
-#pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        const float p0 = (c0 + i < lim) ? exp2f(fmaf(v[i], p.scale_log2, -m_new)) : 0.0f;
-        const float p1 = (c0 + i + 1 < lim) ? exp2f(fmaf(v[i + 1], p.scale_log2, -m_new)) : 0.0f;
-        lsum += p0 + p1;
-        pw[i / 2] = pack_f16(p0, p1);
+          for (int i = 0; i < 32; i += 2) {
+            const float p0 = (c0 + i < lim) ? ex2(fmaf(v[i], p.scale_log2, -m_new)) : 0.0f;
+            const float p1 = (c0 + i + 1 < lim) ? ex2(fmaf(v[i + 1], p.scale_log2, -m_new)) : 0.0f;
+            spart[i & 7] += p0;
+            spart[(i + 1) & 7] += p1;
+            pw[i / 2] = pack_f16(p0, p1);
+          }
+        }
+        tmem_st16(tS + c0 / 2, pw);       // P over S columns already read
       }
+      const float lsum = ((spart[0] + spart[1]) + (spart[2] + spart[3])) + ((spart[4] + spart[5]) + (spart[6] + spart[7]));
+      l_run = l_run * alpha + lsum;
+      m_run = m_new;
+      if (__any_sync(0xffffffffu, j > 0 && alpha != 1.0f)) {   // warp-wide TMEM access
+#pragma unroll 1
+        for (int c0 = 0; c0 < kD; c0 += 32) {
+          float v[32];
+          tmem_ld32(tO + c0, v);
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4*>(smem + OFF_P + sw128_off(tid, c0 / 8 + q)) =
-            make_uint4(pw[4 * q], pw[4 * q + 1], pw[4 * q + 2], pw[4 * q + 3]);
+          for (int i = 0; i < 32; ++i) v[i] *= alpha;
+          tmem_st32(tO + c0, v);
+        }
+      }
+      fence_before_sync();
+      mbar_arrive(bar + B_P_FULL + 8 * x);
     }
-    l_run = l_run * alpha + lsum;
-    m_run = m_new;
-    // ---- rescale the running output in TMEM when a row's max grew. The TMEM
-    // load/store are .sync.aligned warp instructions: the whole warp executes
-    // them when any of its rows needs it (alpha is 1 for the others).
-    if (__any_sync(0xffffffffu, j > 0 && alpha != 1.0f)) {
-#pragma unroll
+    if (done && mbar_wait_or_abort(bar + B_O_DONE + 8 * x, (n_tiles - 1) & 1, p.budget, abort)) {
+      fence_after_sync();
+      const float inv = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
+      const size_t obase = ((size_t(b) * p.Nq + min(qi, p.Nq - 1)) * p.H_q + hq) * kD;
+#pragma unroll 1
       for (int c0 = 0; c0 < kD; c0 += 32) {
         float v[32];
-        tmem_ld32(tO + lane_base + c0, v);
+        tmem_ld32(tO + c0, v);            // every lane: warp-wide TMEM load
+        if (!q_ok) continue;
+        if (p.out_dtype == KV2_OUT_F32) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + obase + c0);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] *= alpha;
-        tmem_st32(tO + lane_base + c0, v);
+          for (int i = 0; i < 32; i += 4) dst[i / 4] = make_float4(v[i] * inv, v[i + 1] * inv, v[i + 2] * inv, v[i + 3] * inv);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + obase + c0);
+#pragma unroll
+          for (int i = 0; i < 32; i += 8)
+            dst[i / 8] = make_uint4(pack_bf16(v[i] * inv, v[i + 1] * inv), pack_bf16(v[i + 2] * inv, v[i + 3] * inv),
+                                    pack_bf16(v[i + 4] * inv, v[i + 5] * inv), pack_bf16(v[i + 6] * inv, v[i + 7] * inv));
+        }
       }
     }
-    fence_proxy_async();
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    // ---- O += P Vhat
-    if (tid == 0) {
-#pragma unroll
-      for (int kk = 0; kk < kKeys / 16; ++kk) {
-        mma_f16(tO, make_sdesc(sb + OFF_P + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kLayoutSW128),
-                make_sdesc(sb + OFF_V + kk * 2048, 16384, 1024, kLayoutSW128), IDESC_PV, (j > 0 || kk > 0));
-      }
-      mma_commit(bar_o);
-    }
-    pending = 2;
-    if (!mbar_wait(bar_o, phase, p.budget)) *s_fail = 1;
-    __syncthreads();
-    if (*s_fail) { failed = true; break; }
-    pending = 0;
-    fence_after_sync();
-    phase ^= 1u;
   }
 
-  if (failed) {
-    if (tid == 0) atomicExch(p.err, 1);
-    // wait (bounded) for the MMA group still in flight before freeing TMEM
-    if (pending == 1) mbar_wait(bar_s, phase, 1ull << 32);
-    if (pending == 2) mbar_wait(bar_o, phase, 1ull << 32);
-  } else {
-    // every lane runs the (warp-wide) TMEM loads; only valid rows store
-    const float inv = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
-    const size_t obase = ((size_t(b) * p.Nq + min(qi, p.Nq - 1)) * p.H_q + hq) * kD;
-#pragma unroll
-    for (int c0 = 0; c0 < kD; c0 += 32) {
-      float v[32];
-      if (n_tiles > 0) {
-        tmem_ld32(tO + lane_base + c0, v);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = 0.0f;
-      }
-      if (!q_ok) continue;
-      if (p.out_dtype == KV2_OUT_F32) {
-        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + obase + c0);
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) dst[i / 4] = make_float4(v[i] * inv, v[i + 1] * inv, v[i + 2] * inv, v[i + 3] * inv);
-      } else {
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + obase + c0);
-#pragma unroll
-        for (int i = 0; i < 32; i += 8)
-          dst[i / 8] = make_uint4(pack_bf16(v[i] * inv, v[i + 1] * inv), pack_bf16(v[i + 2] * inv, v[i + 3] * inv),
-                                  pack_bf16(v[i + 4] * inv, v[i + 5] * inv), pack_bf16(v[i + 6] * inv, v[i + 7] * inv));
-      }
-    }
-  }
   fence_before_sync();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kMmaWarp) {
+    if (*abort) {
+      if (lane == 0) {
+        atomicExch(p.err, 1);
+        mma_commit(bar + B_FINAL);                       // wait (bounded) for MMAs in flight
+      }
+      __syncwarp();
+      mbar_wait(bar + B_FINAL, 0, 1ull << 32);
+    }
+    fence_after_sync();
+    tmem_dealloc(tmem, kTmemCols);
+  }
 }
 
 unsigned long long env_budget() {
@@ -514,7 +684,7 @@ cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(chunk_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SMEM_ALLOC));
   if (e != cudaSuccess) return e;
-  dim3 grid((a.Nq + kRows - 1) / kRows, a.H_q, c.B);
+  dim3 grid((a.Nq + 2 * kRows - 1) / (2 * kRows), a.H_q, c.B);
   chunk_attn_kernel<<<grid, kThreads, SMEM_ALLOC, s>>>(p);
   return cudaGetLastError();
 }

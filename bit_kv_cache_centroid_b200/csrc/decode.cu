@@ -25,7 +25,10 @@
 //   decode_combine log-sum-exp merge of the splits.
 // Codes become floats without integer->float conversions: for channel i of a
 // 32-bit code word, (word & (3 << 2i)) | 0x4B000000 is the float 2^23 + code*4^i;
-// subtracting 2^23 leaves code*4^i exactly, and q carries the factor 4^-i.
+// subtracting 2^23 leaves code*4^i exactly, and q carries the factor 4^-i
+// (channels 10..15 use the word shifted right by 12, so the exponent stays
+// below 10). Two channels are extracted at once into an fp32 pair with 64-bit
+// logic on a duplicated word, then consumed by packed f32x2 arithmetic.
 #include <cfloat>
 
 #include "common.cuh"
@@ -38,15 +41,9 @@ constexpr int kTile = 128;        // tokens per tile
 constexpr int kThreads = 128;     // one thread per token in the logit phase
 constexpr float kLog2e = 1.4426950408889634f;
 
-// power-of-4 exponent carried by channel i (0..15) of a code word
-__host__ __device__ constexpr int code_exp(int i) { return i <= 10 ? i : i - 6; }
-
-__device__ __forceinline__ float code_val(uint32_t word, int i) {
-  // code * 4^code_exp(i), exact
-  const uint32_t src = (i <= 10) ? word : (word >> 12);
-  const int sh = 2 * code_exp(i);
-  return __uint_as_float((src & (3u << sh)) | 0x4B000000u) - 8388608.0f;
-}
+// power-of-4 exponent carried by channel i (0..15) of a code word: channels
+// 0..9 are read in place, channels 10..15 from the word shifted right by 12
+__host__ __device__ constexpr int code_exp(int i) { return i < 10 ? i : i - 6; }
 
 struct PrepLayout {
   int D, M, r, NG, stride;
@@ -119,6 +116,61 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
 
+// Packed fp32 pairs (Blackwell f32x2 arithmetic): one instruction, two lanes.
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 pack2u(uint32_t lo, uint32_t hi) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+__device__ __forceinline__ f32x2 pack2(float lo, float hi) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 unpack2(f32x2 v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ f32x2 ffma2(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f32x2 fsub2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f32x2 fmul2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// {w, w} and {w >> 12, w >> 12}: the two 64-bit sources of a code word's pairs
+struct WordPair {
+  f32x2 lo, hi;
+};
+__device__ __forceinline__ WordPair word_pair(uint32_t w) {
+  const uint32_t wh = w >> 12;
+  return WordPair{pack2u(w, w), pack2u(wh, wh)};
+}
+// codes of channels (2k, 2k+1) of a code word as {code*4^e(2k), code*4^e(2k+1)}
+__device__ __forceinline__ f32x2 code_pair(const WordPair& wp, int k) {
+  const int c0 = 2 * k, c1 = 2 * k + 1;
+  const f32x2 src = (c0 < 10) ? wp.lo : wp.hi;            // pairs never straddle channel 10
+  const unsigned long long mask =
+      (static_cast<unsigned long long>(3u << (2 * code_exp(c1))) << 32) | (3u << (2 * code_exp(c0)));
+  f32x2 bits;
+  asm("{\n\t.reg .b64 t;\n\tand.b64 t, %1, %2;\n\tor.b64 %0, t, 0x4B0000004B000000;\n\t}\n"
+      : "=l"(bits) : "l"(src), "l"(mask));
+  return fsub2(bits, 0x4B0000004B000000ull);
+}
+
+constexpr int kStages = 3;
+
 template <int D, int G, bool U16>
 struct DCfg {
   static constexpr int NG = D / 32;
@@ -134,11 +186,17 @@ struct DCfg {
   static constexpr int vs_off = ks_off + kTile * NG * 4;
   static constexpr int ix_off = vs_off + kTile * NG * 4;
   static constexpr int ps_off = ix_off + kTile * IDXB;
-  static constexpr int red_bytes = TS * G * D * 4;   // final value reduction
-  __host__ __device__ static int stage_bytes(int r) { return ps_off + kTile * r * 2; }
-  __host__ __device__ static int tables_off(int r) {
-    const int two = 2 * stage_bytes(r);
-    return two > red_bytes ? two : red_bytes;
+  // tables after the stages
+  static constexpr int qs_bytes = D * G * 4;                  // q' as [D/2][G] pairs
+  static constexpr int pw_bytes = kTile * NG * G * 4;          // p s_v per (token, group, head)
+  static constexpr int red_bytes = (TS * G * D + kThreads * G * NG) * 4;   // final reduction
+  __host__ __device__ static int stage_bytes(int r) { return (ps_off + kTile * r * 2 + 15) & ~15; }
+  __host__ __device__ static int stages_bytes(int r) {
+    const int st = kStages * stage_bytes(r);
+    return st > red_bytes ? st : red_bytes;
+  }
+  __host__ __device__ static int tables_bytes(int M, int r) {
+    return qs_bytes + pw_bytes + (G * M + G * r + G * NG + 4 * G + 4) * 4;
   }
 };
 
@@ -149,15 +207,13 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int r = p.r, M = p.M;
   const int stage = Cfg::stage_bytes(r);
-  unsigned char* st[2] = {smem, smem + stage};
-  float* qs = reinterpret_cast<float*>(smem + Cfg::tables_off(r));   // [D][G]  q'
-  float* mus = qs + D * G;                                  // [G][M]
-  float* us = mus + G * M;                                  // [G][r]
-  float* sgs = us + G * r;                                  // [G][NG]
-  float* ps = sgs + G * NG;                                 // [G][kTile] probabilities
-  float* red = ps + G * kTile;                              // [4 warps][G] reductions
-  float* mrun = red + 4 * G;                                // [G] running max
-  float* alpha_s = mrun + G;                                // [G]
+  unsigned char* tables = smem + Cfg::stages_bytes(r);
+  f32x2* qs2 = reinterpret_cast<f32x2*>(tables);                              // [D/2][G]
+  float* pw_s = reinterpret_cast<float*>(tables + Cfg::qs_bytes);               // [kTile][NG][G]
+  float* mus = pw_s + kTile * NG * G;                                           // [G][M]
+  float* us = mus + G * M;                                                      // [G][r]
+  float* sgs = us + G * r;                                                      // [G][NG]
+  float* red = sgs + G * NG;                                                    // [4 warps][G]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int split = blockIdx.x, bh = blockIdx.y;
@@ -168,132 +224,116 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
   const int t_end = min(p.len, t_begin + p.tiles_per_split * kTile);
   const int ntiles = (t_end > t_begin) ? (t_end - t_begin + kTile - 1) / kTile : 0;
 
-  // query-side tables of the G query heads
-  for (int i = tid; i < G * D; i += kThreads) {
-    const int g = i / D, c = i % D;
-    qs[c * G + g] = p.prep[size_t(b * p.H_q + h * G + g) * L.stride + L.q_off() + c];
-  }
-  for (int i = tid; i < G * M; i += kThreads) {
-    const int g = i / M, j = i % M;
-    mus[i] = p.prep[size_t(b * p.H_q + h * G + g) * L.stride + L.mu_off() + j];
-  }
-  for (int i = tid; i < G * r; i += kThreads) {
-    const int g = i / r, k = i % r;
-    us[i] = p.prep[size_t(b * p.H_q + h * G + g) * L.stride + L.u_off() + k];
-  }
-  for (int i = tid; i < G * NG; i += kThreads) {
-    const int g = i / NG, k = i % NG;
-    sgs[i] = p.prep[size_t(b * p.H_q + h * G + g) * L.stride + L.sig_off() + k];
-  }
-  if (tid < G) mrun[tid] = -FLT_MAX;
-
-  auto issue = [&](int tile, unsigned char* dst) {
-    const int t0 = t_begin + tile * kTile;
-    const int n = min(kTile, t_end - t0);
-    const int n16 = (n + 15) & ~15;                      // within capacity (cap % 16 == 0)
-    const size_t s0 = base_slot + t0;
-    auto copy = [&](int off, const void* src, int bytes_per_tok) {
-      const int chunks = n16 * bytes_per_tok / 16;
-      const char* g = static_cast<const char*>(src) + s0 * bytes_per_tok;
-      for (int i = tid; i < chunks; i += kThreads) cp_async16(dst + off + i * 16, g + i * 16);
-    };
-    copy(Cfg::kc_off, p.k_code, NW * 4);
-    copy(Cfg::vc_off, p.v_code, NW * 4);
-    copy(Cfg::ks_off, p.k_sz, NG * 4);
-    copy(Cfg::vs_off, p.v_sz, NG * 4);
-    copy(Cfg::ix_off, p.cidx, Cfg::IDXB);
-    if (r) copy(Cfg::ps_off, p.psac, r * 2);
+  auto issue = [&](int tile) {
+    if (tile < ntiles) {
+      unsigned char* dst = smem + (tile % kStages) * stage;
+      const int t0 = t_begin + tile * kTile;
+      const int n16 = (min(kTile, t_end - t0) + 15) & ~15;   // within capacity (cap % 16 == 0)
+      const size_t s0 = base_slot + t0;
+      auto copy = [&](int off, const void* src, int bytes_per_tok) {
+        const int chunks = n16 * bytes_per_tok / 16;
+        const char* g = static_cast<const char*>(src) + s0 * bytes_per_tok;
+        for (int i = tid; i < chunks; i += kThreads) cp_async16(dst + off + i * 16, g + i * 16);
+      };
+      copy(Cfg::kc_off, p.k_code, NW * 4);
+      copy(Cfg::vc_off, p.v_code, NW * 4);
+      copy(Cfg::ks_off, p.k_sz, NG * 4);
+      copy(Cfg::vs_off, p.v_sz, NG * 4);
+      copy(Cfg::ix_off, p.cidx, Cfg::IDXB);
+      if (r) copy(Cfg::ps_off, p.psac, r * 2);
+    }
+    cp_async_commit();
   };
+  issue(0);
+  issue(1);
 
-  // value accumulators: CH channels x G heads, scaled by 4^code_exp per channel
-  const int cb = tid % CB, ts = tid / CB;
-  float acc[G][CH];
-  float pz[G];
+  // query-side tables of the G query heads sharing this KV head
+  const float* prep_h = p.prep + size_t(b * p.H_q + h * G) * L.stride;
+  for (int i = tid; i < G * (D / 2); i += kThreads) {
+    const int g = i % G, c2 = i / G;
+    const float* q = prep_h + size_t(g) * L.stride + L.q_off();
+    qs2[c2 * G + g] = pack2(q[2 * c2], q[2 * c2 + 1]);
+  }
+  for (int i = tid; i < G * M; i += kThreads) mus[i] = prep_h[size_t(i / M) * L.stride + L.mu_off() + i % M];
+  for (int i = tid; i < G * r; i += kThreads) us[i] = prep_h[size_t(i / r) * L.stride + L.u_off() + i % r];
+  for (int i = tid; i < G * NG; i += kThreads) sgs[i] = prep_h[size_t(i / NG) * L.stride + L.sig_off() + i % NG];
+
+  // per-thread state; the running max is identical in every thread
+  float m_run[G], lsum[G], pz[G][NG];
+  f32x2 oacc[G][CH / 2];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    pz[g] = 0.0f;
+    m_run[g] = -FLT_MAX;
+    lsum[g] = 0.0f;
 #pragma unroll
-    for (int c = 0; c < CH; ++c) acc[g][c] = 0.0f;
+    for (int k = 0; k < NG; ++k) pz[g][k] = 0.0f;
+#pragma unroll
+    for (int c = 0; c < CH / 2; ++c) oacc[g][c] = 0ull;
   }
-  float lsum[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) lsum[g] = 0.0f;
-
-  if (ntiles > 0) issue(0, st[0]);
-  cp_async_commit();
-  __syncthreads();
+  const int cb = tid % CB, ts = tid / CB;
+  const int vword = (cb * CH) / 16, vsub = ((cb * CH) % 16) / 2, vgrp = (cb * CH) / 32;
 
   for (int tile = 0; tile < ntiles; ++tile) {
-    unsigned char* cur = st[tile & 1];
-    if (tile + 1 < ntiles) issue(tile + 1, st[(tile + 1) & 1]);
-    cp_async_commit();
     cp_async_wait<1>();
-    __syncthreads();
+    __syncthreads();          // tile data ready; every thread is done with tile - 1
+    issue(tile + 2);          // into the stage tile - 1 used
+    const unsigned char* cur = smem + (tile % kStages) * stage;
+    const int n = min(kTile, t_end - (t_begin + tile * kTile));
+    const int t = tid;                                 // logit phase: thread = token
 
-    const int t0 = t_begin + tile * kTile;
-    const int n = min(kTile, t_end - t0);
-
-    // ---- logits: thread = token, all G heads
+    // ---- logits of the G query heads
     float lg[G];
     {
-      const int t = tid;
+      int idx;
+      if constexpr (U16) idx = reinterpret_cast<const uint16_t*>(cur + Cfg::ix_off)[t];
+      else idx = cur[Cfg::ix_off + t];
+      idx = min(idx, M - 1);
+#pragma unroll
+      for (int g = 0; g < G; ++g) lg[g] = mus[g * M + idx];
       const uint32_t* kw = reinterpret_cast<const uint32_t*>(cur + Cfg::kc_off) + t * NW;
       const uint32_t* ksz = reinterpret_cast<const uint32_t*>(cur + Cfg::ks_off) + t * NG;
-      float dot[G][NG];
 #pragma unroll
-      for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int k = 0; k < NG; ++k) dot[g][k] = 0.0f;
-#pragma unroll
-      for (int w4 = 0; w4 < NW; w4 += 4) {
-        const uint4 wv = *reinterpret_cast<const uint4*>(kw + w4);
+      for (int grp = 0; grp < NG; grp += 2) {          // two groups' chains interleaved
+        const uint4 wv = *reinterpret_cast<const uint4*>(kw + 2 * grp);
         const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+        f32x2 dacc[2][G];
 #pragma unroll
-        for (int ww = 0; ww < 4; ++ww) {
-          const int w = w4 + ww, grp = w / 2;
+        for (int u = 0; u < 2; ++u)
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float f = code_val(words[ww], i);
-            const float* qc = qs + (w * 16 + i) * G;
-            if constexpr (G == 4) {
-              const float4 q4 = *reinterpret_cast<const float4*>(qc);
-              dot[0][grp] = fmaf(q4.x, f, dot[0][grp]);
-              dot[1][grp] = fmaf(q4.y, f, dot[1][grp]);
-              dot[2][grp] = fmaf(q4.z, f, dot[2][grp]);
-              dot[3][grp] = fmaf(q4.w, f, dot[3][grp]);
-            } else {
+          for (int g = 0; g < G; ++g) dacc[u][g] = 0ull;
 #pragma unroll
-              for (int g = 0; g < G; ++g) dot[g][grp] = fmaf(qc[g], f, dot[g][grp]);
+        for (int ww = 0; ww < 2; ++ww) {
+          const WordPair wp0 = word_pair(words[ww]), wp1 = word_pair(words[2 + ww]);
+          const f32x2* q0 = qs2 + (grp * 2 + ww) * 8 * G;
+          const f32x2* q1 = qs2 + (grp * 2 + 2 + ww) * 8 * G;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const f32x2 c0 = code_pair(wp0, k), c1 = code_pair(wp1, k);
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+              dacc[0][g] = ffma2(q0[k * G + g], c0, dacc[0][g]);
+              dacc[1][g] = ffma2(q1[k * G + g], c1, dacc[1][g]);
             }
           }
         }
-      }
-      int idx;
-      if constexpr (U16) idx = reinterpret_cast<const uint16_t*>(cur + Cfg::ix_off)[t];
-      else idx = (cur + Cfg::ix_off)[t];
-      idx = min(idx, M - 1);
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float l = mus[g * M + idx];
-#pragma unroll
-        for (int k = 0; k < NG; ++k) {
-          const uint32_t sz = ksz[k];
+        for (int u = 0; u < 2; ++u) {
+          const uint32_t sz = ksz[grp + u];
           const float s = __half2float(__ushort_as_half(uint16_t(sz & 0xffff)));
           const float z = __half2float(__ushort_as_half(uint16_t(sz >> 16)));
-          l = fmaf(s, dot[g][k], l);
-          l = fmaf(z, sgs[g * NG + k], l);
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float2 d2 = unpack2(dacc[u][g]);
+            lg[g] = fmaf(s, d2.x + d2.y, fmaf(z, sgs[g * NG + grp + u], lg[g]));
+          }
         }
-        lg[g] = l;
       }
       if (r) {
         const __half2* a2 = reinterpret_cast<const __half2*>(cur + Cfg::ps_off) + t * (r / 2);
         for (int k = 0; k < r / 2; ++k) {
           const float2 a = __half22float2(a2[k]);
 #pragma unroll
-          for (int g = 0; g < G; ++g) {
-            lg[g] = fmaf(us[g * r + 2 * k], a.x, lg[g]);
-            lg[g] = fmaf(us[g * r + 2 * k + 1], a.y, lg[g]);
-          }
+          for (int g = 0; g < G; ++g) lg[g] = fmaf(us[g * r + 2 * k], a.x, fmaf(us[g * r + 2 * k + 1], a.y, lg[g]));
         }
       }
       if (t >= n) {
@@ -301,7 +341,7 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
         for (int g = 0; g < G; ++g) lg[g] = -FLT_MAX;
       }
     }
-    // ---- tile max per head, new running max, probabilities
+    // ---- tile max per head (block-wide), new running max
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       float m = lg[g];
@@ -310,83 +350,105 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
       if (lane == 0) red[warp * G + g] = m;
     }
     __syncthreads();
-    if (tid < G) {
-      const float m_old = mrun[tid];
-      const float m_new = fmaxf(m_old, fmaxf(fmaxf(red[tid], red[G + tid]), fmaxf(red[2 * G + tid], red[3 * G + tid])));
-      alpha_s[tid] = exp2f(m_old - m_new);
-      mrun[tid] = m_new;
-    }
-    __syncthreads();
+    float alpha[G];
+    bool rescale = false;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      const float pr = (tid < n) ? exp2f(lg[g] - mrun[g]) : 0.0f;
-      ps[g * kTile + tid] = pr;
-      const float al = alpha_s[g];
-      lsum[g] = lsum[g] * al + pr;        // per-thread partial sums, rescaled alike
+      const float tmax = fmaxf(fmaxf(red[g], red[G + g]), fmaxf(red[2 * G + g], red[3 * G + g]));
+      const float m_new = fmaxf(m_run[g], tmax);
+      alpha[g] = exp2f(m_run[g] - m_new);
+      rescale |= (m_new != m_run[g]);
+      m_run[g] = m_new;
+    }
+    if (rescale) {                                   // uniform across the CTA
 #pragma unroll
-      for (int c = 0; c < CH; ++c) acc[g][c] *= al;
-      pz[g] *= al;
+      for (int g = 0; g < G; ++g) {
+        const f32x2 a2 = pack2(alpha[g], alpha[g]);
+        lsum[g] *= alpha[g];
+#pragma unroll
+        for (int k = 0; k < NG; ++k) pz[g][k] *= alpha[g];
+#pragma unroll
+        for (int c = 0; c < CH / 2; ++c) oacc[g][c] = fmul2(oacc[g][c], a2);
+      }
+    }
+    // ---- probabilities; p s_v per (group, head) for the value phase; sum p z_v
+    {
+      const uint32_t* vsz = reinterpret_cast<const uint32_t*>(cur + Cfg::vs_off) + t * NG;
+      float pr[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        pr[g] = (t < n) ? exp2f(lg[g] - m_run[g]) : 0.0f;
+        lsum[g] += pr[g];
+      }
+#pragma unroll
+      for (int grp = 0; grp < NG; ++grp) {
+        const uint32_t sz = vsz[grp];
+        const float s = (t < n) ? __half2float(__ushort_as_half(uint16_t(sz & 0xffff))) : 0.0f;
+        const float z = (t < n) ? __half2float(__ushort_as_half(uint16_t(sz >> 16))) : 0.0f;
+        float* dst = pw_s + (t * NG + grp) * G;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          dst[g] = pr[g] * s;
+          pz[g][grp] = fmaf(pr[g], z, pz[g][grp]);
+        }
+      }
     }
     __syncthreads();
 
     // ---- values: thread = (channel block, token slice)
     {
       const uint32_t* vw = reinterpret_cast<const uint32_t*>(cur + Cfg::vc_off);
-      const uint32_t* vsz = reinterpret_cast<const uint32_t*>(cur + Cfg::vs_off);
-      const int c0 = cb * CH;
-      const int word = c0 / 16, sub = c0 % 16, grp = c0 / 32;
-      for (int t = ts; t < n; t += TS) {
-        const uint32_t wv = vw[t * NW + word];
-        const uint32_t sz = vsz[t * NG + grp];
-        const float s = __half2float(__ushort_as_half(uint16_t(sz & 0xffff)));
-        const float z = __half2float(__ushort_as_half(uint16_t(sz >> 16)));
-        float pw[G];
+      for (int tt = ts; tt < n; tt += TS) {
+        const WordPair wp = word_pair(vw[tt * NW + vword]);
+        const float* pws = pw_s + (tt * NG + vgrp) * G;
+        f32x2 pw[G];
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float pr = ps[g * kTile + t];
-          pw[g] = pr * s;
-          pz[g] = fmaf(pr, z, pz[g]);
-        }
+        for (int g = 0; g < G; ++g) pw[g] = pack2(pws[g], pws[g]);
 #pragma unroll
-        for (int c = 0; c < CH; ++c) {
-          const float f = code_val(wv, sub + c);
+        for (int k = 0; k < CH / 2; ++k) {
+          const f32x2 cpair = code_pair(wp, vsub + k);
 #pragma unroll
-          for (int g = 0; g < G; ++g) acc[g][c] = fmaf(pw[g], f, acc[g][c]);
+          for (int g = 0; g < G; ++g) oacc[g][k] = ffma2(pw[g], cpair, oacc[g][k]);
         }
       }
     }
-    __syncthreads();
+    // no barrier here: the next tile's first barrier orders these reads before
+    // the copy into this stage and before the next writes of pw_s
   }
   cp_async_wait<0>();
-
-  // ---- reduce: probabilities' sum over threads, value partials over token slices
-  float* rbuf = reinterpret_cast<float*>(smem);      // reuse the stage buffers
   __syncthreads();
+
+  // ---- reduce: value partials over token slices, p z_v and p sums over threads
+  float* rbuf = reinterpret_cast<float*>(smem);            // [TS][G][D], then [kThreads][G][NG]
+  float* zbuf = rbuf + TS * G * D;
 #pragma unroll
   for (int g = 0; g < G; ++g) {
+#pragma unroll
+    for (int k = 0; k < CH / 2; ++k) {
+      const float2 v = unpack2(oacc[g][k]);
+      const int c = cb * CH + 2 * k;
+      rbuf[(ts * G + g) * D + c] = ldexpf(v.x, -2 * code_exp(c % 16));
+      rbuf[(ts * G + g) * D + c + 1] = ldexpf(v.y, -2 * code_exp((c + 1) % 16));
+    }
+#pragma unroll
+    for (int k = 0; k < NG; ++k) zbuf[(tid * G + g) * NG + k] = pz[g][k];
     float l = lsum[g];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
     if (lane == 0) red[warp * G + g] = l;
   }
-  // value partials: [TS][G][D], then the zero term per group (only channel block's group)
-#pragma unroll
-  for (int g = 0; g < G; ++g)
-#pragma unroll
-    for (int c = 0; c < CH; ++c) {
-      const int ch = cb * CH + c;
-      rbuf[(ts * G + g) * D + ch] = ldexpf(acc[g][c], -2 * code_exp(ch % 16)) + pz[g];
-    }
   __syncthreads();
   float* dst = p.part + (size_t(bh) * p.splits + split) * G * (D + 2);
   for (int i = tid; i < G * D; i += kThreads) {
-    const int g = i / D, ch = i % D;
+    const int g = i / D, c = i % D;
     float o = 0.0f;
-    for (int k = 0; k < TS; ++k) o += rbuf[(k * G + g) * D + ch];
-    dst[g * (D + 2) + ch] = o;
+    for (int k = 0; k < TS; ++k) o += rbuf[(k * G + g) * D + c];
+    float z = 0.0f;
+    for (int k = 0; k < kThreads; ++k) z += zbuf[(k * G + g) * NG + c / 32];
+    dst[g * (D + 2) + c] = o + z;
   }
   if (tid < G) {
-    dst[tid * (D + 2) + D] = mrun[tid];
+    dst[tid * (D + 2) + D] = m_run[tid];
     dst[tid * (D + 2) + D + 1] = red[tid] + red[G + tid] + red[2 * G + tid] + red[3 * G + tid];
   }
 }
@@ -420,13 +482,14 @@ __global__ void decode_combine(const float* __restrict__ part, int H_q, int H_kv
 }
 
 template <int D, int G, bool U16>
-cudaError_t launch_split(const SplitParams& sp, int B, cudaStream_t s) {
+size_t split_smem(int M, int r) {
   using Cfg = DCfg<D, G, U16>;
-  const int stage = Cfg::stage_bytes(sp.r);
-  const size_t tables = (size_t(D) * G + size_t(G) * sp.M + size_t(G) * sp.r + G * Cfg::NG +
-                         size_t(G) * kTile + 4 * G + 2 * G) * 4;
-  (void)stage;
-  const size_t smem = size_t(Cfg::tables_off(sp.r)) + tables;
+  return size_t(Cfg::stages_bytes(r)) + size_t(Cfg::tables_bytes(M, r));
+}
+
+template <int D, int G, bool U16>
+cudaError_t launch_split(const SplitParams& sp, int B, cudaStream_t s) {
+  const size_t smem = split_smem<D, G, U16>(sp.M, sp.r);
   auto kern = decode_split<D, G, U16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
@@ -446,6 +509,30 @@ cudaError_t launch_g(int G, const SplitParams& sp, int B, cudaStream_t s) {
   }
 }
 
+// resident split CTAs per SM for this shape (occupancy query; 4 if unknown)
+template <int D, int G, bool U16>
+int ctas_per_sm_t(int M, int r) {
+  const size_t smem = split_smem<D, G, U16>(M, r);
+  auto kern = decode_split<D, G, U16>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess) return 4;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, smem) != cudaSuccess || n <= 0) return 4;
+  return n;
+}
+template <int D, bool U16>
+int ctas_per_sm_g(int G, int M, int r) {
+  switch (G) {
+    case 1: return ctas_per_sm_t<D, 1, U16>(M, r);
+    case 2: return ctas_per_sm_t<D, 2, U16>(M, r);
+    case 4: return ctas_per_sm_t<D, 4, U16>(M, r);
+    default: return ctas_per_sm_t<D, 8, U16>(M, r);
+  }
+}
+int ctas_per_sm(const kv2_cache& c, int G) {
+  if (c.d == 64) return c.M > 256 ? ctas_per_sm_g<64, true>(G, c.M, c.r) : ctas_per_sm_g<64, false>(G, c.M, c.r);
+  return c.M > 256 ? ctas_per_sm_g<128, true>(G, c.M, c.r) : ctas_per_sm_g<128, false>(G, c.M, c.r);
+}
+
 int sm_count() {
   static int n = 0;
   if (n == 0) {
@@ -457,10 +544,13 @@ int sm_count() {
   return n;
 }
 
-void plan_splits(const kv2_cache& c, int len, int* splits, int* tiles_per_split) {
+// Splits along the sequence: as many CTAs as fit in one wave (resident CTAs
+// per SM x SMs), each covering a whole number of 128-token tiles.
+void plan_splits(const kv2_cache& c, int H_q, int len, int* splits, int* tiles_per_split) {
   const int tiles = (len + kTile - 1) / kTile;
   const int pairs = c.B * c.H_kv;
-  int want = (sm_count() * 4 + pairs - 1) / pairs;
+  const int slots = sm_count() * ctas_per_sm(c, H_q / c.H_kv);
+  int want = slots / pairs;
   want = want < 1 ? 1 : want;
   int tps = (tiles + want - 1) / want;
   tps = tps < 1 ? 1 : tps;
@@ -472,7 +562,7 @@ void plan_splits(const kv2_cache& c, int len, int* splits, int* tiles_per_split)
 
 size_t decode_workspace_bytes(const kv2_cache& c, int H_q, int len) {
   int splits, tps;
-  plan_splits(c, len, &splits, &tps);
+  plan_splits(c, H_q, len, &splits, &tps);
   const PrepLayout L(c.d, c.M, c.r);
   const size_t prep = size_t(c.B) * H_q * L.stride * 4;
   const size_t part = size_t(c.B) * c.H_kv * splits * (H_q / c.H_kv) * (c.d + 2) * 4;
@@ -482,7 +572,7 @@ size_t decode_workspace_bytes(const kv2_cache& c, int H_q, int len) {
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   const kv2_cache& c = *a.c;
   int splits, tps;
-  plan_splits(c, a.len, &splits, &tps);
+  plan_splits(c, a.H_q, a.len, &splits, &tps);
   const PrepLayout L(c.d, c.M, c.r);
   float* prep = static_cast<float*>(a.ws);
   const size_t prep_bytes = (size_t(c.B) * a.H_q * L.stride * 4 + 255) & ~size_t(255);
