@@ -175,6 +175,7 @@ def run_gpu(args, rank, world):
         total_ms = float(tt.item())
     ms_step = total_ms / args.steps
     dec_ms = statistics.mean(a.elapsed_time(b) for a, b in dec_ev)
+    app_ms = statistics.mean(ev[i][0].elapsed_time(dec_ev[i][0]) for i in range(args.steps))
     bytes_step = length * s.B * s.H_kv * BYTES_PER_TOKEN_HEAD(s.d, s.r, s.M)
     value = bytes_step * world / (ms_step * 1e-3) / 1e9
 
@@ -223,7 +224,8 @@ def run_gpu(args, rank, world):
                      "peak_source": src, "decode_ms": round(dec_ms, 5)},
         "e2e": {"value": round(bytes_step / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
-        "gpu_launches": 4 * args.steps,
+        "step_ms": {"append": round(app_ms, 5), "decode": round(dec_ms, 5)},
+        "gpu_launches": 3 * args.steps,
         "clocks": clk.summary(),
     }
     if not args.skip_extras and rank == 0:

@@ -14,13 +14,14 @@
 //   out     = sum_t softmax_t * (code_t s_t + z_t)
 //
 // Three kernels:
-//   decode_prep   per query head: q' (q scaled, with a per-channel power-of-4
-//                 factor matching the code extraction), q.mu_j for every centre,
-//                 u = qP, per-group sums of q;
-//   decode_split  grid (splits, B*H_kv): streams 128-token tiles of every packed
-//                 stream with cp.async (double-buffered), one thread per token for
-//                 the logits of the G query heads sharing the KV head (so each
-//                 byte is read once per KV head), online softmax, values
+//   decode_split  grid (splits, B*H_kv): first the query-side tables of the G
+//                 query heads sharing the KV head (q scaled, with a per-channel
+//                 power-of-4 factor matching the code extraction; q.mu_j for
+//                 every centre; u = qP; per-group sums of q), built while the
+//                 first tile is in flight; then it streams 128-token tiles of
+//                 every packed stream with cp.async (double-buffered), one
+//                 thread per token for the logits of the G query heads (so
+//                 each byte is read once per KV head), online softmax, values
 //                 accumulated as sum_t (p_t s_t) code_t + sum_t p_t z_t;
 //   decode_combine log-sum-exp merge of the splits.
 // Codes become floats without integer->float conversions: for channel i of a
@@ -45,56 +46,6 @@ constexpr float kLog2e = 1.4426950408889634f;
 // 0..9 are read in place, channels 10..15 from the word shifted right by 12
 __host__ __device__ constexpr int code_exp(int i) { return i < 10 ? i : i - 6; }
 
-struct PrepLayout {
-  int D, M, r, NG, stride;
-  __host__ __device__ PrepLayout(int d, int m, int rr) : D(d), M(m), r(rr), NG(d / 32) {
-    stride = (D + M + r + NG + 3) & ~3;
-  }
-  __host__ __device__ int q_off() const { return 0; }
-  __host__ __device__ int mu_off() const { return D; }
-  __host__ __device__ int u_off() const { return D + M; }
-  __host__ __device__ int sig_off() const { return D + M + r; }
-};
-
-// ---------------------------------------------------------------------------
-__global__ void decode_prep(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ cent,
-                            const float* __restrict__ P, int H_q, int H_kv, int D, int M, int r,
-                            float scale, float* __restrict__ prep) {
-  const int bq = blockIdx.x;                 // b * H_q + hq
-  const int hq = bq % H_q;
-  const int h = hq / (H_q / H_kv);
-  const PrepLayout L(D, M, r);
-  float* out = prep + size_t(bq) * L.stride;
-  __shared__ float q_s[128];
-  for (int c = threadIdx.x; c < D; c += blockDim.x) {
-    const float q = bf16_to_f32(Q[size_t(bq) * D + c]) * scale;
-    q_s[c] = q;
-    out[L.q_off() + c] = ldexpf(q, -2 * code_exp(c % 16));
-  }
-  __syncthreads();
-  const __half* ch = reinterpret_cast<const __half*>(cent) + size_t(h) * M * D;
-  for (int j = threadIdx.x; j < M; j += blockDim.x) {
-    float acc = 0.0f;
-    const __half2* row = reinterpret_cast<const __half2*>(ch + size_t(j) * D);
-    for (int c = 0; c < D / 2; ++c) {
-      const float2 m = __half22float2(row[c]);
-      acc = fmaf(q_s[2 * c], m.x, acc);
-      acc = fmaf(q_s[2 * c + 1], m.y, acc);
-    }
-    out[L.mu_off() + j] = acc;
-  }
-  for (int i = threadIdx.x; i < r; i += blockDim.x) {
-    float acc = 0.0f;
-    for (int c = 0; c < D; ++c) acc = fmaf(q_s[c], P[(size_t(h) * D + c) * r + i], acc);
-    out[L.u_off() + i] = acc;
-  }
-  for (int g = threadIdx.x; g < D / 32; g += blockDim.x) {
-    float acc = 0.0f;
-    for (int c = 0; c < 32; ++c) acc += q_s[g * 32 + c];
-    out[L.sig_off() + g] = acc;
-  }
-}
-
 // ---------------------------------------------------------------------------
 struct SplitParams {
   const uint32_t* k_code;
@@ -103,8 +54,11 @@ struct SplitParams {
   const uint32_t* v_sz;
   const void* cidx;
   const uint16_t* psac;
-  const float* prep;
-  float* part;        // [B*H_kv][splits][G][D + 2]
+  const uint16_t* Q;      // bf16 [B][H_q][D]
+  const uint16_t* cent;   // fp16 [H_kv][M][D]
+  const float* P;         // [H_kv][D][r]
+  float scale;            // sm_scale * log2(e)
+  float* part;            // [B*H_kv][splits][G][D + 2]
   int H_kv, H_q, M, r, cap, len, splits, tiles_per_split;
 };
 
@@ -169,14 +123,47 @@ __device__ __forceinline__ f32x2 code_pair(const WordPair& wp, int k) {
   return fsub2(bits, 0x4B0000004B000000ull);
 }
 
-constexpr int kStages = 3;
+constexpr int kStages = 2;
 
+// G consecutive floats to / from shared memory with the widest aligned accesses
+template <int G>
+__device__ __forceinline__ void store_vec(float* dst, const float (&v)[G]) {
+  if constexpr (G % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < G; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+  } else if constexpr (G == 2) {
+    *reinterpret_cast<float2*>(dst) = make_float2(v[0], v[1]);
+  } else {
+    dst[0] = v[0];
+  }
+}
+template <int G>
+__device__ __forceinline__ void load_vec(const float* src, float (&v)[G]) {
+  if constexpr (G % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < G; i += 4) {
+      const float4 x = *reinterpret_cast<const float4*>(src + i);
+      v[i] = x.x; v[i + 1] = x.y; v[i + 2] = x.z; v[i + 3] = x.w;
+    }
+  } else if constexpr (G == 2) {
+    const float2 x = *reinterpret_cast<const float2*>(src);
+    v[0] = x.x; v[1] = x.y;
+  } else {
+    v[0] = src[0];
+  }
+}
+
+// Thread mapping of the split kernel (128 threads, 128-token tiles):
+//   cb = tid % 16: 8-channel block (half of code word cb/2, group cb/4)
+//   ts = tid / 16: token slice, tokens ts, ts+8, ... of the tile
+// In both phases a thread works on its 8 channels of 16 tokens, so the query
+// values of its channels stay in registers. Per-token partial logits go
+// through shared memory to the token's owner thread (tid = token).
 template <int D, int G, bool U16>
 struct DCfg {
   static constexpr int NG = D / 32;
   static constexpr int NW = D / 16;            // code words per token
-  static constexpr int CH = (G >= 8) ? 8 : 16; // channels per thread in the value phase
-  static constexpr int CB = D / CH;            // channel blocks
+  static constexpr int CB = D / 8;             // 8-channel blocks
   static constexpr int TS = kThreads / CB;     // token slices
   static constexpr int IDXB = U16 ? 2 : 1;
   // per-stage byte offsets (all multiples of 16)
@@ -187,30 +174,34 @@ struct DCfg {
   static constexpr int ix_off = vs_off + kTile * NG * 4;
   static constexpr int ps_off = ix_off + kTile * IDXB;
   // tables after the stages
-  static constexpr int qs_bytes = D * G * 4;                  // q' as [D/2][G] pairs
-  static constexpr int pw_bytes = kTile * NG * G * 4;          // p s_v per (token, group, head)
-  static constexpr int red_bytes = (TS * G * D + kThreads * G * NG) * 4;   // final reduction
+  // per-token rows padded by 4 floats so that 8 consecutive tokens start in
+  // distinct 16-byte bank groups (conflict-free 16-byte accesses)
+  static constexpr int PS = CB * G + 4;                        // partial logits [token][cb][G]
+  static constexpr int PWS = NG * G + 4;                       // p s_v [token][group][G]
+  static constexpr int part_bytes = kTile * PS * 4;
+  static constexpr int pw_bytes = kTile * PWS * 4;
+  static constexpr int red_bytes = (TS * G * D + kThreads * G * NG) * 4;  // final reduction
   __host__ __device__ static int stage_bytes(int r) { return (ps_off + kTile * r * 2 + 15) & ~15; }
   __host__ __device__ static int stages_bytes(int r) {
     const int st = kStages * stage_bytes(r);
     return st > red_bytes ? st : red_bytes;
   }
   __host__ __device__ static int tables_bytes(int M, int r) {
-    return qs_bytes + pw_bytes + (G * M + G * r + G * NG + 4 * G + 4) * 4;
+    return part_bytes + pw_bytes + (G * M + G * r + G * NG + 4 * G + 4) * 4;
   }
 };
 
 template <int D, int G, bool U16>
 __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
   using Cfg = DCfg<D, G, U16>;
-  constexpr int NG = Cfg::NG, NW = Cfg::NW, CH = Cfg::CH, CB = Cfg::CB, TS = Cfg::TS;
+  constexpr int NG = Cfg::NG, NW = Cfg::NW, CB = Cfg::CB, TS = Cfg::TS;
   extern __shared__ __align__(16) unsigned char smem[];
   const int r = p.r, M = p.M;
   const int stage = Cfg::stage_bytes(r);
   unsigned char* tables = smem + Cfg::stages_bytes(r);
-  f32x2* qs2 = reinterpret_cast<f32x2*>(tables);                              // [D/2][G]
-  float* pw_s = reinterpret_cast<float*>(tables + Cfg::qs_bytes);               // [kTile][NG][G]
-  float* mus = pw_s + kTile * NG * G;                                           // [G][M]
+  float* part_s = reinterpret_cast<float*>(tables);                             // [kTile][CB][G]
+  float* pw_s = reinterpret_cast<float*>(tables + Cfg::part_bytes);            // [kTile][NG][G]
+  float* mus = reinterpret_cast<float*>(tables + Cfg::part_bytes + Cfg::pw_bytes);  // [G][M]
   float* us = mus + G * M;                                                      // [G][r]
   float* sgs = us + G * r;                                                      // [G][NG]
   float* red = sgs + G * NG;                                                    // [4 warps][G]
@@ -218,7 +209,6 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int split = blockIdx.x, bh = blockIdx.y;
   const int b = bh / p.H_kv, h = bh % p.H_kv;
-  const PrepLayout L(D, M, r);
   const size_t base_slot = size_t(bh) * p.cap;
   const int t_begin = split * p.tiles_per_split * kTile;
   const int t_end = min(p.len, t_begin + p.tiles_per_split * kTile);
@@ -245,22 +235,82 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
     cp_async_commit();
   };
   issue(0);
-  issue(1);
 
-  // query-side tables of the G query heads sharing this KV head
-  const float* prep_h = p.prep + size_t(b * p.H_q + h * G) * L.stride;
-  for (int i = tid; i < G * (D / 2); i += kThreads) {
-    const int g = i % G, c2 = i / G;
-    const float* q = prep_h + size_t(g) * L.stride + L.q_off();
-    qs2[c2 * G + g] = pack2(q[2 * c2], q[2 * c2 + 1]);
+  // ---- query-side tables of the G query heads sharing this KV head, built
+  // while the first tile is in flight (part_s is not used before that tile):
+  // q in log2 units, q . mu_j for every centre, u = q P, per-group sums of q
+  float* qs = part_s;                                    // [G][D]
+  float* pst = part_s + G * D;                           // a chunk of rows of P, [rows][r]
+  for (int i = tid; i < G * D; i += kThreads)
+    qs[i] = bf16_to_f32(p.Q[size_t(b * p.H_q + h * G) * D + i]) * p.scale;
+  for (int i = tid; i < G * r; i += kThreads) us[i] = 0.0f;
+  __syncthreads();
+  {
+    const __half* cent_h = reinterpret_cast<const __half*>(p.cent) + size_t(h) * M * D;
+    for (int j = tid; j < M; j += kThreads) {
+      float acc[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) acc[g] = 0.0f;
+      const uint4* row = reinterpret_cast<const uint4*>(cent_h + size_t(j) * D);
+#pragma unroll 4
+      for (int c8 = 0; c8 < D / 8; ++c8) {
+        const uint4 v = __ldg(row + c8);
+        const __half2* h2 = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 m = __half22float2(h2[k]);
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            acc[g] = fmaf(qs[g * D + c8 * 8 + 2 * k], m.x, acc[g]);
+            acc[g] = fmaf(qs[g * D + c8 * 8 + 2 * k + 1], m.y, acc[g]);
+          }
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) mus[g * M + j] = acc[g];
+    }
+    for (int i = tid; i < G * NG; i += kThreads) {
+      const float* q = qs + (i / NG) * D + (i % NG) * 32;
+      float acc = 0.0f;
+      for (int c = 0; c < 32; ++c) acc += q[c];
+      sgs[i] = acc;
+    }
+    if (r) {
+      const float* Ph = p.P + size_t(h) * D * r;
+      const int rows = min(D, (Cfg::part_bytes / 4 - G * D) / r);   // >= 1 since r <= D
+      for (int c0 = 0; c0 < D; c0 += rows) {
+        const int nr = min(rows, D - c0);
+        for (int i = tid; i < nr * r; i += kThreads) pst[i] = Ph[size_t(c0) * r + i];
+        __syncthreads();
+        for (int i = tid; i < G * r; i += kThreads) {
+          const float* q = qs + (i / r) * D + c0;
+          const float* pc = pst + i % r;
+          float acc = us[i];
+          for (int c = 0; c < nr; ++c) acc = fmaf(q[c], pc[c * r], acc);
+          us[i] = acc;
+        }
+        __syncthreads();
+      }
+    }
   }
-  for (int i = tid; i < G * M; i += kThreads) mus[i] = prep_h[size_t(i / M) * L.stride + L.mu_off() + i % M];
-  for (int i = tid; i < G * r; i += kThreads) us[i] = prep_h[size_t(i / r) * L.stride + L.u_off() + i % r];
-  for (int i = tid; i < G * NG; i += kThreads) sgs[i] = prep_h[size_t(i / NG) * L.stride + L.sig_off() + i % NG];
 
-  // per-thread state; the running max is identical in every thread
+  const int cb = tid % CB, ts = tid / CB;
+  const int word = cb >> 1, sub = (cb & 1) * 4, grp = cb >> 2;   // channel pairs sub..sub+3 of the word
+  // this thread's query values: 8 channels x G heads as channel pairs, each
+  // channel carrying the factor 4^-e that matches its code extraction
+  f32x2 q2[G][4];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float* q = qs + g * D + cb * 8;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int c0 = cb * 8 + 2 * k;
+      q2[g][k] = pack2(ldexpf(q[2 * k], -2 * code_exp(c0 % 16)), ldexpf(q[2 * k + 1], -2 * code_exp((c0 + 1) % 16)));
+    }
+  }
+
   float m_run[G], lsum[G], pz[G][NG];
-  f32x2 oacc[G][CH / 2];
+  f32x2 oacc[G][4];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     m_run[g] = -FLT_MAX;
@@ -268,20 +318,47 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
 #pragma unroll
     for (int k = 0; k < NG; ++k) pz[g][k] = 0.0f;
 #pragma unroll
-    for (int c = 0; c < CH / 2; ++c) oacc[g][c] = 0ull;
+    for (int c = 0; c < 4; ++c) oacc[g][c] = 0ull;
   }
-  const int cb = tid % CB, ts = tid / CB;
-  const int vword = (cb * CH) / 16, vsub = ((cb * CH) % 16) / 2, vgrp = (cb * CH) / 32;
 
   for (int tile = 0; tile < ntiles; ++tile) {
-    cp_async_wait<1>();
+    cp_async_wait<0>();
     __syncthreads();          // tile data ready; every thread is done with tile - 1
-    issue(tile + 2);          // into the stage tile - 1 used
+    issue(tile + 1);          // into the stage tile - 1 used
     const unsigned char* cur = smem + (tile % kStages) * stage;
     const int n = min(kTile, t_end - (t_begin + tile * kTile));
-    const int t = tid;                                 // logit phase: thread = token
 
-    // ---- logits of the G query heads
+    // ---- K: partial dot products of this thread's 8 channels, scaled by s_grp
+    {
+      const uint32_t* kw = reinterpret_cast<const uint32_t*>(cur + Cfg::kc_off);
+      const uint32_t* ksz = reinterpret_cast<const uint32_t*>(cur + Cfg::ks_off);
+#pragma unroll 4
+      for (int k = 0; k < kTile / TS; ++k) {
+        const int t = ts + k * TS;
+        const WordPair wp = word_pair(kw[t * NW + word]);
+        f32x2 dacc[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) dacc[g] = 0ull;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const f32x2 cpair = code_pair(wp, sub + c);
+#pragma unroll
+          for (int g = 0; g < G; ++g) dacc[g] = ffma2(q2[g][c], cpair, dacc[g]);
+        }
+        const float s = __half2float(__ushort_as_half(uint16_t(ksz[t * NG + grp] & 0xffff)));
+        float pd[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float2 d2 = unpack2(dacc[g]);
+          pd[g] = s * (d2.x + d2.y);
+        }
+        store_vec<G>(part_s + t * Cfg::PS + cb * G, pd);
+      }
+    }
+    __syncthreads();
+
+    // ---- logits (thread = token): partials + centre + zero terms + PSAC
+    const int t = tid;
     float lg[G];
     {
       int idx;
@@ -290,43 +367,20 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
       idx = min(idx, M - 1);
 #pragma unroll
       for (int g = 0; g < G; ++g) lg[g] = mus[g * M + idx];
-      const uint32_t* kw = reinterpret_cast<const uint32_t*>(cur + Cfg::kc_off) + t * NW;
+      const float* src = part_s + t * Cfg::PS;
+#pragma unroll
+      for (int c = 0; c < CB; ++c) {
+        float pd[G];
+        load_vec<G>(src + c * G, pd);
+#pragma unroll
+        for (int g = 0; g < G; ++g) lg[g] += pd[g];
+      }
       const uint32_t* ksz = reinterpret_cast<const uint32_t*>(cur + Cfg::ks_off) + t * NG;
 #pragma unroll
-      for (int grp = 0; grp < NG; grp += 2) {          // two groups' chains interleaved
-        const uint4 wv = *reinterpret_cast<const uint4*>(kw + 2 * grp);
-        const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
-        f32x2 dacc[2][G];
+      for (int k = 0; k < NG; ++k) {
+        const float z = __half2float(__ushort_as_half(uint16_t(ksz[k] >> 16)));
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-          for (int g = 0; g < G; ++g) dacc[u][g] = 0ull;
-#pragma unroll
-        for (int ww = 0; ww < 2; ++ww) {
-          const WordPair wp0 = word_pair(words[ww]), wp1 = word_pair(words[2 + ww]);
-          const f32x2* q0 = qs2 + (grp * 2 + ww) * 8 * G;
-          const f32x2* q1 = qs2 + (grp * 2 + 2 + ww) * 8 * G;
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const f32x2 c0 = code_pair(wp0, k), c1 = code_pair(wp1, k);
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-              dacc[0][g] = ffma2(q0[k * G + g], c0, dacc[0][g]);
-              dacc[1][g] = ffma2(q1[k * G + g], c1, dacc[1][g]);
-            }
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const uint32_t sz = ksz[grp + u];
-          const float s = __half2float(__ushort_as_half(uint16_t(sz & 0xffff)));
-          const float z = __half2float(__ushort_as_half(uint16_t(sz >> 16)));
-#pragma unroll
-          for (int g = 0; g < G; ++g) {
-            const float2 d2 = unpack2(dacc[u][g]);
-            lg[g] = fmaf(s, d2.x + d2.y, fmaf(z, sgs[g * NG + grp + u], lg[g]));
-          }
-        }
+        for (int g = 0; g < G; ++g) lg[g] = fmaf(z, sgs[g * NG + k], lg[g]);
       }
       if (r) {
         const __half2* a2 = reinterpret_cast<const __half2*>(cur + Cfg::ps_off) + t * (r / 2);
@@ -368,7 +422,7 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
 #pragma unroll
         for (int k = 0; k < NG; ++k) pz[g][k] *= alpha[g];
 #pragma unroll
-        for (int c = 0; c < CH / 2; ++c) oacc[g][c] = fmul2(oacc[g][c], a2);
+        for (int c = 0; c < 4; ++c) oacc[g][c] = fmul2(oacc[g][c], a2);
       }
     }
     // ---- probabilities; p s_v per (group, head) for the value phase; sum p z_v
@@ -381,39 +435,43 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
         lsum[g] += pr[g];
       }
 #pragma unroll
-      for (int grp = 0; grp < NG; ++grp) {
-        const uint32_t sz = vsz[grp];
-        const float s = (t < n) ? __half2float(__ushort_as_half(uint16_t(sz & 0xffff))) : 0.0f;
-        const float z = (t < n) ? __half2float(__ushort_as_half(uint16_t(sz >> 16))) : 0.0f;
-        float* dst = pw_s + (t * NG + grp) * G;
+      for (int k = 0; k < NG; ++k) {
+        const uint32_t sz = vsz[k];
+        const float sv = (t < n) ? __half2float(__ushort_as_half(uint16_t(sz & 0xffff))) : 0.0f;
+        const float zv = (t < n) ? __half2float(__ushort_as_half(uint16_t(sz >> 16))) : 0.0f;
+        float pw[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          dst[g] = pr[g] * s;
-          pz[g][grp] = fmaf(pr[g], z, pz[g][grp]);
+          pw[g] = pr[g] * sv;
+          pz[g][k] = fmaf(pr[g], zv, pz[g][k]);
         }
+        store_vec<G>(pw_s + t * Cfg::PWS + k * G, pw);
       }
     }
     __syncthreads();
 
-    // ---- values: thread = (channel block, token slice)
+    // ---- values: this thread's 8 channels over its 16 tokens
     {
       const uint32_t* vw = reinterpret_cast<const uint32_t*>(cur + Cfg::vc_off);
-      for (int tt = ts; tt < n; tt += TS) {
-        const WordPair wp = word_pair(vw[tt * NW + vword]);
-        const float* pws = pw_s + (tt * NG + vgrp) * G;
+#pragma unroll 4
+      for (int k = 0; k < kTile / TS; ++k) {
+        const int tt = ts + k * TS;
+        const WordPair wp = word_pair(vw[tt * NW + word]);
+        float pv[G];
+        load_vec<G>(pw_s + tt * Cfg::PWS + grp * G, pv);
         f32x2 pw[G];
 #pragma unroll
-        for (int g = 0; g < G; ++g) pw[g] = pack2(pws[g], pws[g]);
+        for (int g = 0; g < G; ++g) pw[g] = pack2(pv[g], pv[g]);   // {p s_v, p s_v}
 #pragma unroll
-        for (int k = 0; k < CH / 2; ++k) {
-          const f32x2 cpair = code_pair(wp, vsub + k);
+        for (int c = 0; c < 4; ++c) {
+          const f32x2 cpair = code_pair(wp, sub + c);
 #pragma unroll
-          for (int g = 0; g < G; ++g) oacc[g][k] = ffma2(pw[g], cpair, oacc[g][k]);
+          for (int g = 0; g < G; ++g) oacc[g][c] = ffma2(pw[g], cpair, oacc[g][c]);
         }
       }
     }
     // no barrier here: the next tile's first barrier orders these reads before
-    // the copy into this stage and before the next writes of pw_s
+    // the copy into this stage and the next writes of part_s / pw_s
   }
   cp_async_wait<0>();
   __syncthreads();
@@ -424,11 +482,11 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
 #pragma unroll
   for (int g = 0; g < G; ++g) {
 #pragma unroll
-    for (int k = 0; k < CH / 2; ++k) {
-      const float2 v = unpack2(oacc[g][k]);
-      const int c = cb * CH + 2 * k;
-      rbuf[(ts * G + g) * D + c] = ldexpf(v.x, -2 * code_exp(c % 16));
-      rbuf[(ts * G + g) * D + c + 1] = ldexpf(v.y, -2 * code_exp((c + 1) % 16));
+    for (int c = 0; c < 4; ++c) {
+      const float2 v = unpack2(oacc[g][c]);
+      const int ch = cb * 8 + 2 * c;
+      rbuf[(ts * G + g) * D + ch] = ldexpf(v.x, -2 * code_exp(ch % 16));
+      rbuf[(ts * G + g) * D + ch + 1] = ldexpf(v.y, -2 * code_exp((ch + 1) % 16));
     }
 #pragma unroll
     for (int k = 0; k < NG; ++k) zbuf[(tid * G + g) * NG + k] = pz[g][k];
@@ -448,7 +506,10 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
     dst[g * (D + 2) + c] = o + z;
   }
   if (tid < G) {
-    dst[tid * (D + 2) + D] = m_run[tid];
+    float mr = m_run[0];
+#pragma unroll
+    for (int g = 1; g < G; ++g) if (tid == g) mr = m_run[g];
+    dst[tid * (D + 2) + D] = mr;
     dst[tid * (D + 2) + D + 1] = red[tid] + red[G + tid] + red[2 * G + tid] + red[3 * G + tid];
   }
 }
@@ -563,27 +624,19 @@ void plan_splits(const kv2_cache& c, int H_q, int len, int* splits, int* tiles_p
 size_t decode_workspace_bytes(const kv2_cache& c, int H_q, int len) {
   int splits, tps;
   plan_splits(c, H_q, len, &splits, &tps);
-  const PrepLayout L(c.d, c.M, c.r);
-  const size_t prep = size_t(c.B) * H_q * L.stride * 4;
-  const size_t part = size_t(c.B) * c.H_kv * splits * (H_q / c.H_kv) * (c.d + 2) * 4;
-  return ((prep + 255) & ~size_t(255)) + part;
+  return size_t(c.B) * c.H_kv * splits * (H_q / c.H_kv) * (c.d + 2) * 4;
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   const kv2_cache& c = *a.c;
   int splits, tps;
   plan_splits(c, a.H_q, a.len, &splits, &tps);
-  const PrepLayout L(c.d, c.M, c.r);
-  float* prep = static_cast<float*>(a.ws);
-  const size_t prep_bytes = (size_t(c.B) * a.H_q * L.stride * 4 + 255) & ~size_t(255);
-  float* part = reinterpret_cast<float*>(static_cast<char*>(a.ws) + prep_bytes);
-  decode_prep<<<c.B * a.H_q, 128, 0, s>>>(a.Q, c.centroids, c.P, a.H_q, c.H_kv, c.d, c.M, c.r,
-                                          a.sm_scale * kLog2e, prep);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  SplitParams sp{c.k_code, c.v_code, c.k_sz, c.v_sz, c.cidx, c.psac, prep, part,
-                 c.H_kv, a.H_q, c.M, c.r, c.capacity, a.len, splits, tps};
+  float* part = static_cast<float*>(a.ws);
+  SplitParams sp{c.k_code, c.v_code, c.k_sz, c.v_sz, c.cidx, c.psac,
+                 static_cast<const uint16_t*>(a.Q), static_cast<const uint16_t*>(c.centroids), c.P,
+                 a.sm_scale * kLog2e, part, c.H_kv, a.H_q, c.M, c.r, c.capacity, a.len, splits, tps};
   const int G = a.H_q / c.H_kv;
+  cudaError_t e;
   if (c.d == 64) e = (c.M > 256) ? launch_g<64, true>(G, sp, c.B, s) : launch_g<64, false>(G, sp, c.B, s);
   else e = (c.M > 256) ? launch_g<128, true>(G, sp, c.B, s) : launch_g<128, false>(G, sp, c.B, s);
   if (e != cudaSuccess) return e;

@@ -43,9 +43,8 @@ struct QCfg {
   static constexpr size_t mu_bytes = size_t(D) * MP * 2;
   static constexpr size_t warp_wk_bytes = size_t(D) * KPT * 4;   // w*k [D][KPT], later e [KPT][D]
   __host__ __device__ static size_t warp_bytes(int C) { return (warp_wk_bytes + size_t(KPT) * 8 + size_t(KPT) * C * 2 + 15) & ~size_t(15); }
-  static size_t smem(int C) {
-    return mu_bytes + size_t(MP) * 4 + size_t(D) * 4 + size_t(kWarps) * warp_bytes(C);
-  }
+  __host__ __device__ static size_t head_bytes(int r) { return mu_bytes + size_t(MP) * 4 + size_t(D) * 4 + size_t(D) * r * 4; }
+  static size_t smem(int C, int r) { return head_bytes(r) + size_t(kWarps) * warp_bytes(C); }
 };
 
 template <int D, int CPL, int KPT>
@@ -57,8 +56,9 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
   __half* mu_s = reinterpret_cast<__half*>(smem);                            // [D][MP]
   float* nrm_s = reinterpret_cast<float*>(smem + Cfg::mu_bytes);              // [MP]
   float* w_s = nrm_s + MP;                                                    // [D]
+  float* P_s = w_s + D;                                                       // [D][r]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  unsigned char* wbase = reinterpret_cast<unsigned char*>(w_s + D) + size_t(warp) * Cfg::warp_bytes(a.C);
+  unsigned char* wbase = smem + Cfg::head_bytes(a.r) + size_t(warp) * Cfg::warp_bytes(a.C);
   float* wk_w = reinterpret_cast<float*>(wbase);                              // [D][KPT]
   float* e_w = wk_w;                                                          // [KPT][D] after ranking
   unsigned long long* best_w = reinterpret_cast<unsigned long long*>(wbase + Cfg::warp_wk_bytes);  // [KPT]
@@ -79,8 +79,10 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
     return (size_t(b) * a.H + h) * a.cap + size_t(a.pos + t);
   };
 
-  // ---- once per CTA: centroid table (fp16, transposed, lane-interleaved), w, norms
+  // ---- once per CTA: centroid table (fp16, transposed, lane-interleaved), w,
+  // the PSAC basis, norms
   for (int i = tid; i < D; i += kThreads) w_s[i] = a.w[size_t(h) * D + i];
+  for (int i = tid; i < D * a.r; i += kThreads) P_s[i] = a.P[size_t(h) * D * a.r + i];
   for (int idx = tid; idx < MP * (D / 8); idx += kThreads) {
     const int j = idx % MP, c8 = idx / MP;
     uint4 v = make_uint4(0, 0, 0, 0);
@@ -94,9 +96,10 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
   for (int j = tid; j < MP; j += kThreads) {
     float acc = 0.0f;
     if (j < M) {
-      const __half* row = cent + size_t(j) * D;
+      const __half* col = mu_s + (j % 32) * CPL + j / 32;     // centroid j in the staged table
+#pragma unroll 8
       for (int c = 0; c < D; ++c) {
-        const float m = __half2float(row[c]);
+        const float m = __half2float(col[c * MP]);
         acc = __fmaf_rn(__fmul_rn(w_s[c], m), m, acc);
       }
     }
@@ -105,16 +108,19 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
   __syncthreads();
 
   for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    const int k0 = tile * KT + warp * KPT;
-    const int nk = min(KPT, rows_total - k0);
+    // key k of this warp is row tile*KT + k*kWarps + warp, so that a short
+    // append spreads over all warps
+    const int rem = rows_total - tile * KT - warp;
+    const int nk = rem > 0 ? min(KPT, (rem + kWarps - 1) / kWarps) : 0;
     if (nk <= 0) continue;                       // warp-uniform
+    auto row_of = [&](int k) { return tile * KT + k * kWarps + warp; };
 
     // ---- w*k for this warp's keys, transposed to [D][KPT]
     for (int idx = lane; idx < KPT * (D / 8); idx += 32) {
       const int k = idx % KPT, c8 = idx / KPT;
       float f[8];
       if (k < nk) {
-        const uint4 v = *reinterpret_cast<const uint4*>(key_ptr(a.K, k0 + k) + c8 * 8);
+        const uint4 v = *reinterpret_cast<const uint4*>(key_ptr(a.K, row_of(k)) + c8 * 8);
         const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -215,7 +221,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
         const int k = task / C, i = task - k * C;
         const int j = cand_w[k * C + i];
         const int col = (j % 32) * CPL + j / 32;
-        const uint16_t* krow = key_ptr(a.K, k0 + k);
+        const uint16_t* krow = key_ptr(a.K, row_of(k));
         float E = 0.0f;
 #pragma unroll 1
         for (int g = 0; g < NG; ++g) {
@@ -247,7 +253,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
       const int which = task / (nk * NG);   // 0: keys, 1: values
       const int kg = task - which * nk * NG;
       const int k = kg / NG, g = kg - k * NG;
-      const int row = k0 + k;
+      const int row = row_of(k);
       const size_t slot = slot_of(row);
       float x[kGroup];
       int j = 0;
@@ -304,11 +310,12 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
     // ---- PSAC coefficients a_i = sum_c P_ci e_c (ascending c)
     for (int task = lane; task < nk * a.r; task += 32) {
       const int k = task / a.r, i = task - k * a.r;
-      const float* Pcol = a.P + size_t(h) * D * a.r + i;
+      const float* Pcol = P_s + i;
       const float* e = e_w + k * D;
       float acc = 0.0f;
-      for (int c = 0; c < D; ++c) acc = __fmaf_rn(__ldg(Pcol + size_t(c) * a.r), e[c], acc);
-      a.psac[slot_of(k0 + k) * a.r + i] = f16_rn(acc);
+#pragma unroll 8
+      for (int c = 0; c < D; ++c) acc = __fmaf_rn(Pcol[c * a.r], e[c], acc);
+      a.psac[slot_of(row_of(k)) * a.r + i] = f16_rn(acc);
     }
     __syncwarp();    // e_w / wk_w and cand_w are reused by this warp's next tile
   }
@@ -317,7 +324,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
 template <int D, int CPL, int KPT>
 cudaError_t launch_cfg(const QuantizeArgs& a, cudaStream_t s) {
   using Cfg = QCfg<D, CPL, KPT>;
-  const size_t smem = Cfg::smem(a.C);
+  const size_t smem = Cfg::smem(a.C, a.r);
   auto kern = quantize_kernel<D, CPL, KPT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;

@@ -141,9 +141,9 @@ kv2_status kv2_quantize_append(const kv2_cache* cache, const uint16_t* K, const 
                                int n_new, int pos, int candidates, void* stream);
 
 /*
- * Workspace for kv2_attention_decode, in bytes (per-query-head centroid
- * logits qmu[M], q P, and the split-K partials). Returns 0 for unsupported
- * shapes.
+ * Workspace for kv2_attention_decode, in bytes: the split-K partials (per
+ * query head and split, d output sums, the running maximum and the softmax
+ * denominator, fp32). Returns 0 for unsupported shapes.
  */
 size_t kv2_decode_workspace_size(const kv2_cache* cache, int H_q, int len);
 

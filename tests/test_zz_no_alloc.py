@@ -63,7 +63,7 @@ def test_noalloc_matches_workspace_decode_twice(T, length, ov):
 
 def test_noalloc_rejects_shapes_beyond_the_array():
     import bit_kv_cache_centroid_b200 as kv2
-    s = wl.spec("tiny", d=128, H_q=64, H_kv=64, M=512, r=16, B=64, T=16)
+    s = wl.spec("tiny", d=128, H_q=64, H_kv=64, M=512, r=16, B=512, T=16)
     c = kv2.Cache(s.B, s.H_kv, s.d, s.M, s.r, 32, torch.zeros(s.H_kv, s.M, s.d, dtype=torch.int16))
     Q = torch.zeros(s.B, s.H_q, s.d, dtype=torch.int16, device="cuda")
     assert kv2.kv2_decode_workspace_size(c, s.H_q, 16) > 8 << 20
