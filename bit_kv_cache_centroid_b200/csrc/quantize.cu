@@ -149,10 +149,15 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
 #pragma unroll 2
       for (int c = 0; c < D; ++c) {
         float wk[KPT];
+        if constexpr (KPT % 4 == 0) {
 #pragma unroll
-        for (int k = 0; k < KPT; k += 4) {
-          const float4 v = *reinterpret_cast<const float4*>(wk_w + c * KPT + k);
-          wk[k] = v.x; wk[k + 1] = v.y; wk[k + 2] = v.z; wk[k + 3] = v.w;
+          for (int k = 0; k < KPT; k += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(wk_w + c * KPT + k);
+            wk[k] = v.x; wk[k + 1] = v.y; wk[k + 2] = v.z; wk[k + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < KPT; ++k) wk[k] = wk_w[c * KPT + k];
         }
         float m[CPL];
         if constexpr (CPL >= 8) {
@@ -346,6 +351,13 @@ cudaError_t launch_cfg(const QuantizeArgs& a, cudaStream_t s) {
 template <int D>
 cudaError_t launch_d(const QuantizeArgs& a, cudaStream_t s) {
   const int mp = (a.M + 31) / 32;
+  if (a.B * a.n_new <= 8 * kWarps) {            // short appends: one key per warp and tile
+    if (mp <= 1) return launch_cfg<D, 1, 1>(a, s);
+    if (mp <= 2) return launch_cfg<D, 2, 1>(a, s);
+    if (mp <= 4) return launch_cfg<D, 4, 1>(a, s);
+    if (mp <= 8) return launch_cfg<D, 8, 1>(a, s);
+    return launch_cfg<D, 16, 1>(a, s);
+  }
   if (mp <= 1) return launch_cfg<D, 1, 16>(a, s);
   if (mp <= 2) return launch_cfg<D, 2, 16>(a, s);
   if (mp <= 4) return launch_cfg<D, 4, 16>(a, s);

@@ -65,6 +65,9 @@ def test_tiny_bit_exact(orc):
     (100, 3, 0, 1, 65, 16),      # M not a multiple of 32, no PSAC
     (256, 256, 8, 1, 40, 0),     # candidates = M: brute-force choice
     (33, 1, 16, 2, 70, 3),       # candidates = 1
+    (64, 4, 8, 8, 1, 4095),      # decode append: one token per sequence (short-append kernel)
+    (512, 8, 16, 4, 16, 9),      # 64 keys per head: the largest short append, u16 ids
+    (32, 2, 8, 3, 5, 1),         # 15 keys: warps with and without a key
 ])
 def test_mid_sizes_bit_exact(orc, M, C, r, B, n_tok, pos):
     s = wl.spec("tiny", d=128, H_q=4, H_kv=2, M=M, r=r, B=B, T=n_tok, n_new=1, n_hist=64, Nq=0)
@@ -77,6 +80,13 @@ def test_nearest_centre_mode(orc):
     s = wl.spec("tiny", d=64, M=16, r=8)
     ref, got = _run(orc, s, C=1, unit_w=True)
     _compare(ref, got, what="qvg")
+
+
+def test_short_append_d64_bit_exact(orc):
+    """d = 64 through the short-append kernel (3 sequences x 2 tokens)."""
+    s = wl.spec("tiny", d=64, H_q=4, H_kv=2, M=48, r=8, B=3, T=2, n_new=1, n_hist=64, Nq=0)
+    ref, got = _run(orc, s, pos=21, n_tok=2, C=4)
+    _compare(ref, got, what="short d64")
 
 
 def test_video_keys_bit_exact(orc):
