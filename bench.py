@@ -34,6 +34,10 @@ sys.path.insert(0, ROOT)
 import workloads as wl  # noqa: E402
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (read + write) of one decode_split launch on the LLM decode
+# workload, from the ncu capture summarised in profiles/decode_split_llm_decode.md;
+# None whenever the kernel has changed since that capture.
+DECODE_SPLIT_TRAFFIC = 242_363_904
 BYTES_PER_TOKEN_HEAD = lambda d, r, M: 2 * (d // 16) * 4 + 2 * (d // 32) * 4 + (1 if M <= 256 else 2) + 2 * r
 
 
@@ -219,8 +223,8 @@ def run_gpu(args, rank, world):
                    "global_batch": s.B * world, "seq_len": length, "parallelism": f"replicas x{world}",
                    "l2": "packed cache 237 MB > 126 MB L2 (no flush)"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
-                     "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": None,
-                     "kernel": "kv2_attention_decode (prep + split-K + combine)",
+                     "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": DECODE_SPLIT_TRAFFIC,
+                     "kernel": "kv2_attention_decode (decode_split + decode_combine)",
                      "peak_source": src, "decode_ms": round(dec_ms, 5)},
         "e2e": {"value": round(bytes_step / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
