@@ -13,23 +13,38 @@
 //             + (q P) . a_t                      (all scaled by sm_scale * log2 e)
 //   out     = sum_t softmax_t * (code_t s_t + z_t)
 //
-// Three kernels:
-//   decode_split  grid (splits, B*H_kv): first the query-side tables of the G
-//                 query heads sharing the KV head (q scaled, with a per-channel
-//                 power-of-4 factor matching the code extraction; q.mu_j for
-//                 every centre; u = qP; per-group sums of q), built while the
-//                 first tile is in flight; then it streams 128-token tiles of
-//                 every packed stream with cp.async (double-buffered), one
-//                 thread per token for the logits of the G query heads (so
-//                 each byte is read once per KV head), online softmax, values
-//                 accumulated as sum_t (p_t s_t) code_t + sum_t p_t z_t;
+// Two kernels:
+//   decode_split  grid (splits, B*H_kv), 4 warps. Prologue: the query-side
+//                 tables of the G query heads sharing the KV head (q in log2
+//                 units, q.mu_j for every centre, u = qP, per-group sums of q),
+//                 built while the first tile is in flight. Then 128-token tiles
+//                 of every packed stream arrive by cp.async (double-buffered)
+//                 and each tile takes three phases:
+//                   q.k   the sums  sum_{c in g} q_c code_c  on the tensor cores
+//                         (mma.sync m16n8k16, fp16 operands, fp32 accumulate):
+//                         A = codes (tokens x channels), B = q; one accumulator
+//                         per channel group, scaled by the token's s_g;
+//                   owner one thread per token adds the centre, zero and PSAC
+//                         terms, runs the online softmax and writes p_t s_t,g;
+//                   p.v   sum_t (p_t s_t,g) code_t,c on the tensor cores:
+//                         A = codes (channels x tokens), B = p s.
+//                 The fp32 operands q and p s enter the tensor cores as two fp16
+//                 halves (hi = fp16(x), lo = fp16(x - hi), about 22 significant
+//                 bits) placed in separate columns of the n8 tile, so G <= 4
+//                 heads fill one tile and 8 heads two; the two column sums are
+//                 added in fp32. q is scaled by a power of two per CTA so that
+//                 its halves stay normal fp16 numbers.
 //   decode_combine log-sum-exp merge of the splits.
-// Codes become floats without integer->float conversions: for channel i of a
-// 32-bit code word, (word & (3 << 2i)) | 0x4B000000 is the float 2^23 + code*4^i;
-// subtracting 2^23 leaves code*4^i exactly, and q carries the factor 4^-i
-// (channels 10..15 use the word shifted right by 12, so the exponent stays
-// below 10). Two channels are extracted at once into an fp32 pair with 64-bit
-// logic on a duplicated word, then consumed by packed f32x2 arithmetic.
+//
+// Codes become fp16 operands with three integer/half instructions per pair
+// and no conversions: for a code sitting at bits 2i..2i+1 (i <= 3) of a 16-bit
+// half, (half & (3 << 2i)) | 0x6400 is the fp16 number 1024 + code * 4^i, and
+// one fp16 fma with 4^-i and -1024 * 4^-i gives the code exactly. For q.k a
+// quad of lanes takes the 16 channels of a code word as the pairs
+// (tig, 8+tig) of the word and (4+tig, 12+tig) of the word shifted right by 8
+// (tig = lane % 4), a fixed permutation of the contraction index that q's
+// operand follows. For p.v a byte permute puts the byte holding channel c of
+// two tokens into the two halves.
 #include <cfloat>
 
 #include "common.cuh"
@@ -39,14 +54,11 @@ namespace kv2 {
 namespace {
 
 constexpr int kTile = 128;        // tokens per tile
-constexpr int kThreads = 128;     // one thread per token in the logit phase
+constexpr int kThreads = 128;     // one thread per token in the owner phase
+constexpr int kWarps = kThreads / 32;
+constexpr int kStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 
-// power-of-4 exponent carried by channel i (0..15) of a code word: channels
-// 0..9 are read in place, channels 10..15 from the word shifted right by 12
-__host__ __device__ constexpr int code_exp(int i) { return i < 10 ? i : i - 6; }
-
-// ---------------------------------------------------------------------------
 struct SplitParams {
   const uint32_t* k_code;
   const uint32_t* v_code;
@@ -70,73 +82,40 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
 
-// Packed fp32 pairs (Blackwell f32x2 arithmetic): one instruction, two lanes.
-typedef unsigned long long f32x2;
-__device__ __forceinline__ f32x2 pack2u(uint32_t lo, uint32_t hi) {
-  f32x2 r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
-  return r;
-}
-__device__ __forceinline__ f32x2 pack2(float lo, float hi) {
-  f32x2 r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ float2 unpack2(f32x2 v) {
-  float2 r;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
-  return r;
-}
-__device__ __forceinline__ f32x2 ffma2(f32x2 a, f32x2 b, f32x2 c) {
-  f32x2 d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+// d = a * b + c on two fp16 lanes
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
 }
-__device__ __forceinline__ f32x2 fsub2(f32x2 a, f32x2 b) {
-  f32x2 d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
+// two codes (at the bits of `mask` in each half of x) -> two exact fp16 codes
+__device__ __forceinline__ uint32_t unpack_codes(uint32_t x, uint32_t mask, uint32_t scale, uint32_t offset) {
+  return hfma2((x & mask) | 0x64006400u, scale, offset);
 }
-__device__ __forceinline__ f32x2 fmul2(f32x2 a, f32x2 b) {
-  f32x2 d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
+// d += A B, m16n8k16, fp16 operands, fp32 accumulators
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-
-// {w, w} and {w >> 12, w >> 12}: the two 64-bit sources of a code word's pairs
-struct WordPair {
-  f32x2 lo, hi;
-};
-__device__ __forceinline__ WordPair word_pair(uint32_t w) {
-  const uint32_t wh = w >> 12;
-  return WordPair{pack2u(w, w), pack2u(wh, wh)};
+// four transposed 8x8 fp16 tiles; lane i gives the address of row i % 8 of tile i / 8
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], const void* row) {
+  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(row));
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(s));
 }
-// codes of channels (2k, 2k+1) of a code word as {code*4^e(2k), code*4^e(2k+1)}
-__device__ __forceinline__ f32x2 code_pair(const WordPair& wp, int k) {
-  const int c0 = 2 * k, c1 = 2 * k + 1;
-  const f32x2 src = (c0 < 10) ? wp.lo : wp.hi;            // pairs never straddle channel 10
-  const unsigned long long mask =
-      (static_cast<unsigned long long>(3u << (2 * code_exp(c1))) << 32) | (3u << (2 * code_exp(c0)));
-  f32x2 bits;
-  asm("{\n\t.reg .b64 t;\n\tand.b64 t, %1, %2;\n\tor.b64 %0, t, 0x4B0000004B000000;\n\t}\n"
-      : "=l"(bits) : "l"(src), "l"(mask));
-  return fsub2(bits, 0x4B0000004B000000ull);
+// x = hi + lo with hi = fp16(x), lo = fp16(x - hi)
+__device__ __forceinline__ uint16_t f16_hi(float x) { return __half_as_ushort(__float2half_rn(x)); }
+__device__ __forceinline__ uint16_t f16_lo(float x) {
+  return __half_as_ushort(__float2half_rn(x - __half2float(__float2half_rn(x))));
+}
+__device__ __forceinline__ uint32_t pack_h2(uint16_t lo_half, uint16_t hi_half) {
+  return uint32_t(lo_half) | (uint32_t(hi_half) << 16);
 }
 
-constexpr int kStages = 2;
-
-// G consecutive floats to / from shared memory with the widest aligned accesses
-template <int G>
-__device__ __forceinline__ void store_vec(float* dst, const float (&v)[G]) {
-  if constexpr (G % 4 == 0) {
-#pragma unroll
-    for (int i = 0; i < G; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-  } else if constexpr (G == 2) {
-    *reinterpret_cast<float2*>(dst) = make_float2(v[0], v[1]);
-  } else {
-    dst[0] = v[0];
-  }
-}
+// G consecutive floats from shared memory with the widest aligned loads
 template <int G>
 __device__ __forceinline__ void load_vec(const float* src, float (&v)[G]) {
   if constexpr (G % 4 == 0) {
@@ -153,19 +132,68 @@ __device__ __forceinline__ void load_vec(const float* src, float (&v)[G]) {
   }
 }
 
-// Thread mapping of the split kernel (128 threads, 128-token tiles):
-//   cb = tid % 16: 8-channel block (half of code word cb/2, group cb/4)
-//   ts = tid / 16: token slice, tokens ts, ts+8, ... of the tile
-// In both phases a thread works on its 8 channels of 16 tokens, so the query
-// values of its channels stay in registers. Per-token partial logits go
-// through shared memory to the token's owner thread (tid = token).
+// Column n of an n8 operand tile holds, for G <= 4, the hi half of head n
+// (n < G) or the lo half of head n - G (G <= n < 2G), other columns zero; for
+// G = 8, tile 0 holds the hi halves and tile 1 the lo halves of heads 0..7.
+template <int G>
+struct Cols {
+  static constexpr int NT = (G == 8) ? 2 : 1;
+  __device__ static int head(int n) { return (G == 8) ? n : (n < G ? n : n - G); }
+  __device__ static bool used(int n) { return (G == 8) || n < 2 * G; }
+  __device__ static bool is_lo(int nt, int n) { return (G == 8) ? nt == 1 : n >= G; }
+};
+
+// Adds the hi and lo column sums of a fragment (c0..c3 = rows r, r, r+8, r+8
+// and columns 2 tig, 2 tig + 1 of each n8 tile) and calls f(row_sel, head,
+// value) once per (row, head) on the lane that holds the sum. Every lane of
+// the warp must call it (it shuffles).
+template <int G, int NT, typename F>
+__device__ __forceinline__ void combine_hi_lo(const float (&c)[NT][4], int tig, F&& f) {
+  if constexpr (G == 8) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f(i >> 1, 2 * tig + (i & 1), c[0][i] + c[NT - 1][i]);
+  } else if constexpr (G == 4) {
+    float v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = c[0][i] + __shfl_xor_sync(0xffffffffu, c[0][i], 2);
+    if (tig < 2) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) f(i >> 1, 2 * tig + (i & 1), v[i]);
+    }
+  } else if constexpr (G == 2) {
+    float v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = c[0][i] + __shfl_xor_sync(0xffffffffu, c[0][i], 1);
+    if (tig == 0) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) f(i >> 1, i & 1, v[i]);
+    }
+  } else {
+    if (tig == 0) {
+      f(0, 0, c[0][0] + c[0][1]);
+      f(1, 0, c[0][2] + c[0][3]);
+    }
+  }
+}
+
+// Shared memory of the split kernel:
+//   stages  kStages x raw tile copies (codes, scale/zero words, ids, PSAC)
+//           (reused at the end for the final reduction)
+//   lg      [kTile][LS] fp32   q.k sums per token and head
+//   wt      [NG][kTile][NCOL] fp16   p s_v per group, token and column
+//   tables  q.mu [G][M], u [G][r], group sums [G][NG], reduction slots
+// lg and wt also hold the prologue's scratch (q and rows of P).
 template <int D, int G, bool U16>
 struct DCfg {
   static constexpr int NG = D / 32;
-  static constexpr int NW = D / 16;            // code words per token
-  static constexpr int CB = D / 8;             // 8-channel blocks
-  static constexpr int TS = kThreads / CB;     // token slices
+  static constexpr int NW = D / 16;            // code words per token = q.k k-steps
+  static constexpr int NT = Cols<G>::NT;
+  static constexpr int NCOL = 8 * NT;
+  static constexpr int MTK = kTile / 16 / kWarps;   // token m-tiles per warp in q.k
+  static constexpr int MTV = NW / kWarps;           // channel m-tiles (words) per warp in p.v
+  static_assert(MTV >= 1 && MTV <= 2, "one channel group per warp in p.v");
   static constexpr int IDXB = U16 ? 2 : 1;
+  static constexpr int LS = G < 4 ? 4 : G;
   // per-stage byte offsets (all multiples of 16)
   static constexpr int kc_off = 0;
   static constexpr int vc_off = kc_off + kTile * NW * 4;
@@ -173,40 +201,39 @@ struct DCfg {
   static constexpr int vs_off = ks_off + kTile * NG * 4;
   static constexpr int ix_off = vs_off + kTile * NG * 4;
   static constexpr int ps_off = ix_off + kTile * IDXB;
-  // tables after the stages
-  // per-token rows padded by 4 floats so that 8 consecutive tokens start in
-  // distinct 16-byte bank groups (conflict-free 16-byte accesses)
-  static constexpr int PS = CB * G + 4;                        // partial logits [token][cb][G]
-  static constexpr int PWS = NG * G + 4;                       // p s_v [token][group][G]
-  static constexpr int part_bytes = kTile * PS * 4;
-  static constexpr int pw_bytes = kTile * PWS * 4;
-  static constexpr int red_bytes = (TS * G * D + kThreads * G * NG) * 4;  // final reduction
+  static constexpr int lg_bytes = kTile * LS * 4;
+  static constexpr int wt_bytes = NG * kTile * NCOL * 2;
+  static constexpr int scratch_floats = (lg_bytes + wt_bytes) / 4;
+  static constexpr int red_bytes = (G * D + kThreads * G * NG) * 4;   // final reduction
   __host__ __device__ static int stage_bytes(int r) { return (ps_off + kTile * r * 2 + 15) & ~15; }
   __host__ __device__ static int stages_bytes(int r) {
     const int st = kStages * stage_bytes(r);
     return st > red_bytes ? st : red_bytes;
   }
   __host__ __device__ static int tables_bytes(int M, int r) {
-    return part_bytes + pw_bytes + (G * M + G * r + G * NG + 4 * G + 4) * 4;
+    return lg_bytes + wt_bytes + (G * M + G * r + G * NG + 4 * G + 4) * 4;
   }
 };
 
 template <int D, int G, bool U16>
 __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
   using Cfg = DCfg<D, G, U16>;
-  constexpr int NG = Cfg::NG, NW = Cfg::NW, CB = Cfg::CB, TS = Cfg::TS;
+  using CL = Cols<G>;
+  constexpr int NG = Cfg::NG, NW = Cfg::NW, NT = Cfg::NT, NCOL = Cfg::NCOL;
+  constexpr int MTK = Cfg::MTK, MTV = Cfg::MTV, LS = Cfg::LS;
   extern __shared__ __align__(16) unsigned char smem[];
   const int r = p.r, M = p.M;
   const int stage = Cfg::stage_bytes(r);
   unsigned char* tables = smem + Cfg::stages_bytes(r);
-  float* part_s = reinterpret_cast<float*>(tables);                             // [kTile][CB][G]
-  float* pw_s = reinterpret_cast<float*>(tables + Cfg::part_bytes);            // [kTile][NG][G]
-  float* mus = reinterpret_cast<float*>(tables + Cfg::part_bytes + Cfg::pw_bytes);  // [G][M]
-  float* us = mus + G * M;                                                      // [G][r]
-  float* sgs = us + G * r;                                                      // [G][NG]
-  float* red = sgs + G * NG;                                                    // [4 warps][G]
+  float* lg_s = reinterpret_cast<float*>(tables);                                  // [kTile][LS]
+  uint16_t* wt_s = reinterpret_cast<uint16_t*>(tables + Cfg::lg_bytes);            // [NG][kTile][NCOL]
+  float* mus = reinterpret_cast<float*>(tables + Cfg::lg_bytes + Cfg::wt_bytes);   // [G][M]
+  float* us = mus + G * M;                                                         // [G][r]
+  float* sgs = us + G * r;                                                         // [G][NG]
+  float* red = sgs + G * NG;                                                       // [kWarps][G], [kWarps]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gid = lane >> 2, tig = lane & 3;
   const int split = blockIdx.x, bh = blockIdx.y;
   const int b = bh / p.H_kv, h = bh % p.H_kv;
   const size_t base_slot = size_t(bh) * p.cap;
@@ -237,10 +264,10 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
   issue(0);
 
   // ---- query-side tables of the G query heads sharing this KV head, built
-  // while the first tile is in flight (part_s is not used before that tile):
+  // while the first tile is in flight (lg and wt are not used before it):
   // q in log2 units, q . mu_j for every centre, u = q P, per-group sums of q
-  float* qs = part_s;                                    // [G][D]
-  float* pst = part_s + G * D;                           // a chunk of rows of P, [rows][r]
+  float* qs = lg_s;                                      // [G][D]
+  float* pst = lg_s + G * D;                             // a chunk of rows of P, [rows][r]
   for (int i = tid; i < G * D; i += kThreads)
     qs[i] = bf16_to_f32(p.Q[size_t(b * p.H_q + h * G) * D + i]) * p.scale;
   for (int i = tid; i < G * r; i += kThreads) us[i] = 0.0f;
@@ -277,7 +304,7 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
     }
     if (r) {
       const float* Ph = p.P + size_t(h) * D * r;
-      const int rows = min(D, (Cfg::part_bytes / 4 - G * D) / r);   // >= 1 since r <= D
+      const int rows = min(D, (Cfg::scratch_floats - G * D) / r);   // >= 1 since r <= D
       for (int c0 = 0; c0 < D; c0 += rows) {
         const int nr = min(rows, D - c0);
         for (int i = tid; i < nr * r; i += kThreads) pst[i] = Ph[size_t(c0) * r + i];
@@ -293,33 +320,66 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
       }
     }
   }
+  // power-of-two scale of q for the tensor cores: max |q| 2^eq below 2^14
+  float qmax = 0.0f;
+  for (int i = tid; i < G * D; i += kThreads) qmax = fmaxf(qmax, fabsf(qs[i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, o));
+  if (lane == 0) red[kWarps * G + warp] = qmax;
+  __syncthreads();
+  qmax = fmaxf(fmaxf(red[kWarps * G], red[kWarps * G + 1]), fmaxf(red[kWarps * G + 2], red[kWarps * G + 3]));
+  int qexp = 0;
+  frexpf(qmax, &qexp);
+  const int eq = (qmax > 0.0f) ? 14 - qexp : 0;
+  const float qmul = ldexpf(1.0f, eq), qinv = ldexpf(1.0f, -eq);
 
-  const int cb = tid % CB, ts = tid / CB;
-  const int word = cb >> 1, sub = (cb & 1) * 4, grp = cb >> 2;   // channel pairs sub..sub+3 of the word
-  // this thread's query values: 8 channels x G heads as channel pairs, each
-  // channel carrying the factor 4^-e that matches its code extraction
-  f32x2 q2[G][4];
+  // B operand of q.k for every k-step: column gid of each n8 tile, rows
+  // (channels) tig, 8+tig | 4+tig, 12+tig of the k-step's code word
+  uint32_t bq[NT][NW][2];
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const float* q = qs + g * D + cb * 8;
+  for (int nt = 0; nt < NT; ++nt) {
+    const bool used = CL::used(gid), lo = CL::is_lo(nt, gid);
+    const float* qh = qs + min(CL::head(gid), G - 1) * D;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int c0 = cb * 8 + 2 * k;
-      q2[g][k] = pack2(ldexpf(q[2 * k], -2 * code_exp(c0 % 16)), ldexpf(q[2 * k + 1], -2 * code_exp((c0 + 1) % 16)));
+    for (int ks = 0; ks < NW; ++ks) {
+      const int c = 16 * ks + tig;
+      const float x[4] = {qh[c] * qmul, qh[c + 8] * qmul, qh[c + 4] * qmul, qh[c + 12] * qmul};
+      uint16_t hv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) hv[i] = used ? (lo ? f16_lo(x[i]) : f16_hi(x[i])) : uint16_t(0);
+      bq[nt][ks][0] = pack_h2(hv[0], hv[1]);
+      bq[nt][ks][1] = pack_h2(hv[2], hv[3]);
     }
   }
+  // code unpacking constants (fp16 4^-i and -1024 * 4^-i in both halves)
+  const uint32_t mk = (3u << (2 * tig)) | (3u << (16 + 2 * tig));
+  const uint32_t sck = 0x3C003C00u - 0x08000800u * uint32_t(tig);
+  const uint32_t ofk = 0xE400E400u - 0x08000800u * uint32_t(tig);
+  const int cv = gid & 3;
+  const uint32_t mv = (3u << (2 * cv)) | (3u << (16 + 2 * cv));
+  const uint32_t scv = 0x3C003C00u - 0x08000800u * uint32_t(cv);
+  const uint32_t ofv = 0xE400E400u - 0x08000800u * uint32_t(cv);
+  const uint32_t selv0 = uint32_t(gid >> 2) | (uint32_t(4 + (gid >> 2)) << 8);       // channel gid
+  const uint32_t selv1 = uint32_t(2 + (gid >> 2)) | (uint32_t(6 + (gid >> 2)) << 8);  // channel gid + 8
+  // heads of this lane's two accumulator columns in p.v
+  const int hc0 = min(CL::head(2 * tig), G - 1), hc1 = min(CL::head(2 * tig + 1), G - 1);
 
   float m_run[G], lsum[G], pz[G][NG];
-  f32x2 oacc[G][4];
+  float oacc[MTV][NT][4];     // p.v sums scaled by 2^ev_acc
+  int ev_acc = 0;
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     m_run[g] = -FLT_MAX;
     lsum[g] = 0.0f;
 #pragma unroll
     for (int k = 0; k < NG; ++k) pz[g][k] = 0.0f;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) oacc[g][c] = 0ull;
   }
+#pragma unroll
+  for (int mt = 0; mt < MTV; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) oacc[mt][nt][i] = 0.0f;
 
   for (int tile = 0; tile < ntiles; ++tile) {
     cp_async_wait<0>();
@@ -328,53 +388,67 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
     const unsigned char* cur = smem + (tile % kStages) * stage;
     const int n = min(kTile, t_end - (t_begin + tile * kTile));
 
-    // ---- K: partial dot products of this thread's 8 channels, scaled by s_grp
+    // ---- q.k on the tensor cores: warp w takes tokens 16 MTK w .. 16 MTK (w + 1) - 1
     {
       const uint32_t* kw = reinterpret_cast<const uint32_t*>(cur + Cfg::kc_off);
       const uint32_t* ksz = reinterpret_cast<const uint32_t*>(cur + Cfg::ks_off);
-#pragma unroll 4
-      for (int k = 0; k < kTile / TS; ++k) {
-        const int t = ts + k * TS;
-        const WordPair wp = word_pair(kw[t * NW + word]);
-        f32x2 dacc[G];
 #pragma unroll
-        for (int g = 0; g < G; ++g) dacc[g] = 0ull;
+      for (int mt = 0; mt < MTK; ++mt) {
+        const int t0 = (warp * MTK + mt) * 16 + gid, t1 = t0 + 8;
+        uint32_t w0[NW], w1[NW];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const f32x2 cpair = code_pair(wp, sub + c);
-#pragma unroll
-          for (int g = 0; g < G; ++g) dacc[g] = ffma2(q2[g][c], cpair, dacc[g]);
+        for (int i = 0; i < NW; i += 4) {
+          const uint4 x0 = *reinterpret_cast<const uint4*>(kw + t0 * NW + i);
+          const uint4 x1 = *reinterpret_cast<const uint4*>(kw + t1 * NW + i);
+          w0[i] = x0.x; w0[i + 1] = x0.y; w0[i + 2] = x0.z; w0[i + 3] = x0.w;
+          w1[i] = x1.x; w1[i + 1] = x1.y; w1[i + 2] = x1.z; w1[i + 3] = x1.w;
         }
-        const float s = __half2float(__ushort_as_half(uint16_t(ksz[t * NG + grp] & 0xffff)));
-        float pd[G];
+        float L[NT][4];
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float2 d2 = unpack2(dacc[g]);
-          pd[g] = s * (d2.x + d2.y);
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) L[nt][i] = 0.0f;
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+          float C[NT][4];
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) C[nt][i] = 0.0f;
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            const int ks = 2 * g + kk;
+            const uint32_t a[4] = {unpack_codes(w0[ks], mk, sck, ofk), unpack_codes(w1[ks], mk, sck, ofk),
+                                   unpack_codes(w0[ks] >> 8, mk, sck, ofk), unpack_codes(w1[ks] >> 8, mk, sck, ofk)};
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma16816(C[nt], a, bq[nt][ks][0], bq[nt][ks][1]);
+          }
+          const float s0 = __half2float(__ushort_as_half(uint16_t(ksz[t0 * NG + g] & 0xffff))) * qinv;
+          const float s1 = __half2float(__ushort_as_half(uint16_t(ksz[t1 * NG + g] & 0xffff))) * qinv;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            L[nt][0] = fmaf(s0, C[nt][0], L[nt][0]);
+            L[nt][1] = fmaf(s0, C[nt][1], L[nt][1]);
+            L[nt][2] = fmaf(s1, C[nt][2], L[nt][2]);
+            L[nt][3] = fmaf(s1, C[nt][3], L[nt][3]);
+          }
         }
-        store_vec<G>(part_s + t * Cfg::PS + cb * G, pd);
+        combine_hi_lo<G, NT>(L, tig, [&](int rs, int g, float v) { lg_s[(rs ? t1 : t0) * LS + g] = v; });
       }
     }
     __syncthreads();
 
-    // ---- logits (thread = token): partials + centre + zero terms + PSAC
+    // ---- owner phase (thread = token): centre, zero and PSAC terms
     const int t = tid;
     float lg[G];
     {
+      load_vec<G>(lg_s + t * LS, lg);
       int idx;
       if constexpr (U16) idx = reinterpret_cast<const uint16_t*>(cur + Cfg::ix_off)[t];
       else idx = cur[Cfg::ix_off + t];
       idx = min(idx, M - 1);
 #pragma unroll
-      for (int g = 0; g < G; ++g) lg[g] = mus[g * M + idx];
-      const float* src = part_s + t * Cfg::PS;
-#pragma unroll
-      for (int c = 0; c < CB; ++c) {
-        float pd[G];
-        load_vec<G>(src + c * G, pd);
-#pragma unroll
-        for (int g = 0; g < G; ++g) lg[g] += pd[g];
-      }
+      for (int g = 0; g < G; ++g) lg[g] += mus[g * M + idx];
       const uint32_t* ksz = reinterpret_cast<const uint32_t*>(cur + Cfg::ks_off) + t * NG;
 #pragma unroll
       for (int k = 0; k < NG; ++k) {
@@ -395,7 +469,17 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
         for (int g = 0; g < G; ++g) lg[g] = -FLT_MAX;
       }
     }
-    // ---- tile max per head (block-wide), new running max
+    uint32_t vszr[NG];
+    float smax = 0.0f;                               // largest value scale of the token
+    {
+      const uint32_t* vsz = reinterpret_cast<const uint32_t*>(cur + Cfg::vs_off) + t * NG;
+#pragma unroll
+      for (int k = 0; k < NG; ++k) {
+        vszr[k] = (t < n) ? vsz[k] : 0u;
+        smax = fmaxf(smax, __half2float(__ushort_as_half(uint16_t(vszr[k] & 0xffff))));
+      }
+    }
+    // ---- tile max per head and of the value scales (block-wide)
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       float m = lg[g];
@@ -403,7 +487,20 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
       for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
       if (lane == 0) red[warp * G + g] = m;
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, o));
+    if (lane == 0) red[kWarps * G + warp] = smax;
     __syncthreads();
+    // p s_v enters p.v scaled by 2^ev (largest value below 2^14), so that its
+    // fp16 hi and lo halves stay normal numbers
+    int ev = ev_acc;
+    {
+      const float st = fmaxf(fmaxf(red[kWarps * G], red[kWarps * G + 1]),
+                             fmaxf(red[kWarps * G + 2], red[kWarps * G + 3]));
+      int se = 0;
+      frexpf(st, &se);
+      if (st > 0.0f) ev = 14 - se;
+    }
     float alpha[G];
     bool rescale = false;
 #pragma unroll
@@ -414,20 +511,29 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
       rescale |= (m_new != m_run[g]);
       m_run[g] = m_new;
     }
-    if (rescale) {                                   // uniform across the CTA
+    if (rescale || ev != ev_acc) {                   // uniform across the CTA
+      const float f = ldexpf(1.0f, ev - ev_acc);
+      float ac0 = f, ac1 = f;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        const f32x2 a2 = pack2(alpha[g], alpha[g]);
         lsum[g] *= alpha[g];
 #pragma unroll
         for (int k = 0; k < NG; ++k) pz[g][k] *= alpha[g];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) oacc[g][c] = fmul2(oacc[g][c], a2);
+        if (g == hc0) ac0 = alpha[g] * f;
+        if (g == hc1) ac1 = alpha[g] * f;
       }
+      ev_acc = ev;
+#pragma unroll
+      for (int mt = 0; mt < MTV; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          oacc[mt][nt][0] *= ac0; oacc[mt][nt][1] *= ac1;
+          oacc[mt][nt][2] *= ac0; oacc[mt][nt][3] *= ac1;
+        }
     }
-    // ---- probabilities; p s_v per (group, head) for the value phase; sum p z_v
+    // ---- probabilities; p s_v as (hi, lo) fp16 columns per group; sum p z_v
     {
-      const uint32_t* vsz = reinterpret_cast<const uint32_t*>(cur + Cfg::vs_off) + t * NG;
+      const float vmul = ldexpf(1.0f, ev);
       float pr[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
@@ -436,58 +542,111 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
       }
 #pragma unroll
       for (int k = 0; k < NG; ++k) {
-        const uint32_t sz = vsz[k];
-        const float sv = (t < n) ? __half2float(__ushort_as_half(uint16_t(sz & 0xffff))) : 0.0f;
-        const float zv = (t < n) ? __half2float(__ushort_as_half(uint16_t(sz >> 16))) : 0.0f;
-        float pw[G];
+        const uint32_t sz = vszr[k];                 // 0 for t >= n
+        const float sv = __half2float(__ushort_as_half(uint16_t(sz & 0xffff))) * vmul;
+        const float zv = __half2float(__ushort_as_half(uint16_t(sz >> 16)));
+        float w[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          pw[g] = pr[g] * sv;
+          w[g] = pr[g] * sv;
           pz[g][k] = fmaf(pr[g], zv, pz[g][k]);
         }
-        store_vec<G>(pw_s + t * Cfg::PWS + k * G, pw);
+        uint32_t hw[NCOL / 2];
+#pragma unroll
+        for (int c2 = 0; c2 < NCOL / 2; ++c2) {
+          uint16_t hv[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int col = 2 * c2 + e, nt = col / 8, nn = col % 8;
+            hv[e] = 0;
+            if (CL::used(nn)) {
+              const float x = w[min(CL::head(nn), G - 1)];
+              hv[e] = CL::is_lo(nt, nn) ? f16_lo(x) : f16_hi(x);
+            }
+          }
+          hw[c2] = pack_h2(hv[0], hv[1]);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(wt_s + (size_t(k) * kTile + t) * NCOL);
+#pragma unroll
+        for (int q4 = 0; q4 < NT; ++q4) dst[q4] = make_uint4(hw[4 * q4], hw[4 * q4 + 1], hw[4 * q4 + 2], hw[4 * q4 + 3]);
       }
     }
     __syncthreads();
 
-    // ---- values: this thread's 8 channels over its 16 tokens
+    // ---- p.v on the tensor cores: warp w takes code words (16-channel
+    // m-tiles) MTV w .. MTV (w + 1) - 1, all in channel group MTV w / 2. The
+    // tile's sums start from zero and join the running sums in fp32 (the
+    // tensor cores' accumulation truncates, and carried over a whole split
+    // its bias would show through the cancellation of code and zero terms).
     {
+      float tacc[MTV][NT][4];
+#pragma unroll
+      for (int mt = 0; mt < MTV; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) tacc[mt][nt][i] = 0.0f;
       const uint32_t* vw = reinterpret_cast<const uint32_t*>(cur + Cfg::vc_off);
-#pragma unroll 4
-      for (int k = 0; k < kTile / TS; ++k) {
-        const int tt = ts + k * TS;
-        const WordPair wp = word_pair(vw[tt * NW + word]);
-        float pv[G];
-        load_vec<G>(pw_s + tt * Cfg::PWS + grp * G, pv);
-        f32x2 pw[G];
+      const int wi0 = warp * MTV;
+      const uint16_t* wt_g = wt_s + size_t(wi0 / 2) * kTile * NCOL;
 #pragma unroll
-        for (int g = 0; g < G; ++g) pw[g] = pack2(pv[g], pv[g]);   // {p s_v, p s_v}
+      for (int ks2 = 0; ks2 < kTile / 32; ++ks2) {
+        uint32_t bw[NT][4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const f32x2 cpair = code_pair(wp, sub + c);
+        for (int nt = 0; nt < NT; ++nt) ldmatrix_x4_trans(bw[nt], wt_g + (32 * ks2 + lane) * NCOL + 8 * nt);
 #pragma unroll
-          for (int g = 0; g < G; ++g) oacc[g][c] = ffma2(pw[g], cpair, oacc[g][c]);
+        for (int kk = 0; kk < 2; ++kk) {
+          const int ta = 32 * ks2 + 16 * kk + 2 * tig;
+          uint32_t wa0[MTV], wb0[MTV], wa1[MTV], wb1[MTV];
+          if constexpr (MTV == 2) {
+            const uint2 x0 = *reinterpret_cast<const uint2*>(vw + ta * NW + wi0);
+            const uint2 x1 = *reinterpret_cast<const uint2*>(vw + (ta + 1) * NW + wi0);
+            const uint2 x2 = *reinterpret_cast<const uint2*>(vw + (ta + 8) * NW + wi0);
+            const uint2 x3 = *reinterpret_cast<const uint2*>(vw + (ta + 9) * NW + wi0);
+            wa0[0] = x0.x; wa0[1] = x0.y; wb0[0] = x1.x; wb0[1] = x1.y;
+            wa1[0] = x2.x; wa1[1] = x2.y; wb1[0] = x3.x; wb1[1] = x3.y;
+          } else {
+            wa0[0] = vw[ta * NW + wi0];
+            wb0[0] = vw[(ta + 1) * NW + wi0];
+            wa1[0] = vw[(ta + 8) * NW + wi0];
+            wb1[0] = vw[(ta + 9) * NW + wi0];
+          }
+#pragma unroll
+          for (int mt = 0; mt < MTV; ++mt) {
+            const uint32_t a[4] = {unpack_codes(__byte_perm(wa0[mt], wb0[mt], selv0), mv, scv, ofv),
+                                   unpack_codes(__byte_perm(wa0[mt], wb0[mt], selv1), mv, scv, ofv),
+                                   unpack_codes(__byte_perm(wa1[mt], wb1[mt], selv0), mv, scv, ofv),
+                                   unpack_codes(__byte_perm(wa1[mt], wb1[mt], selv1), mv, scv, ofv)};
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma16816(tacc[mt][nt], a, bw[nt][2 * kk], bw[nt][2 * kk + 1]);
+          }
         }
       }
+#pragma unroll
+      for (int mt = 0; mt < MTV; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) oacc[mt][nt][i] += tacc[mt][nt][i];
     }
     // no barrier here: the next tile's first barrier orders these reads before
-    // the copy into this stage and the next writes of part_s / pw_s
+    // the copy into this stage and the next writes of lg / wt
   }
   cp_async_wait<0>();
   __syncthreads();
 
-  // ---- reduce: value partials over token slices, p z_v and p sums over threads
-  float* rbuf = reinterpret_cast<float*>(smem);            // [TS][G][D], then [kThreads][G][NG]
-  float* zbuf = rbuf + TS * G * D;
+  // ---- reduce: p.v sums (one lane per channel and head), p z_v and p sums
+  // over the owner threads
+  float* ofin = reinterpret_cast<float*>(smem);            // [G][D]
+  float* zbuf = ofin + G * D;                               // [kThreads][G][NG]
+  const float vinv = ldexpf(1.0f, -ev_acc);
+#pragma unroll
+  for (int mt = 0; mt < MTV; ++mt) {
+    const int c0 = (warp * MTV + mt) * 16 + gid;
+    combine_hi_lo<G, NT>(oacc[mt], tig, [&](int rs, int g, float v) { ofin[g * D + c0 + 8 * rs] = v * vinv; });
+  }
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const float2 v = unpack2(oacc[g][c]);
-      const int ch = cb * 8 + 2 * c;
-      rbuf[(ts * G + g) * D + ch] = ldexpf(v.x, -2 * code_exp(ch % 16));
-      rbuf[(ts * G + g) * D + ch + 1] = ldexpf(v.y, -2 * code_exp((ch + 1) % 16));
-    }
 #pragma unroll
     for (int k = 0; k < NG; ++k) zbuf[(tid * G + g) * NG + k] = pz[g][k];
     float l = lsum[g];
@@ -499,11 +658,9 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
   float* dst = p.part + (size_t(bh) * p.splits + split) * G * (D + 2);
   for (int i = tid; i < G * D; i += kThreads) {
     const int g = i / D, c = i % D;
-    float o = 0.0f;
-    for (int k = 0; k < TS; ++k) o += rbuf[(k * G + g) * D + c];
     float z = 0.0f;
     for (int k = 0; k < kThreads; ++k) z += zbuf[(k * G + g) * NG + c / 32];
-    dst[g * (D + 2) + c] = o + z;
+    dst[g * (D + 2) + c] = ofin[i] + z;
   }
   if (tid < G) {
     float mr = m_run[0];
