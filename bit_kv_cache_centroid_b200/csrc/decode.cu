@@ -100,6 +100,28 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+// d = A B (accumulators start at zero)
+__device__ __forceinline__ void mma16816_zc(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};\n"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
+}
+// order-preserving map of floats (no NaN) to signed integers, and back
+__device__ __forceinline__ int f2ord(float x) {
+  const int i = __float_as_int(x);
+  return i ^ ((i >> 31) & 0x7fffffff);
+}
+__device__ __forceinline__ float ord2f(int k) { return __int_as_float(k ^ ((k >> 31) & 0x7fffffff)); }
+// two fp32 values as fp16 pairs hi = fp16(x), lo = fp16(x - hi)
+__device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(x0, x1);
+  const float2 hf = __half22float2(h);
+  const __half2 l = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
 // four transposed 8x8 fp16 tiles; lane i gives the address of row i % 8 of tile i / 8
 __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], const void* row) {
   const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(row));
@@ -181,7 +203,8 @@ __device__ __forceinline__ void combine_hi_lo(const float (&c)[NT][4], int tig, 
 //           (reused at the end for the final reduction)
 //   lg      [kTile][LS] fp32   q.k sums per token and head
 //   wt      [NG][kTile][NCOL] fp16   p s_v per group, token and column
-//   tables  q.mu [G][M], u [G][r], group sums [G][NG], reduction slots
+//   tables  q.mu [G][M], u [G][r], group sums [G][NG], reduction slots,
+//           B fragments of the zero-point / PSAC k-steps [XK][NT][32 lanes]
 // lg and wt also hold the prologue's scratch (q and rows of P).
 template <int D, int G, bool U16>
 struct DCfg {
@@ -210,8 +233,13 @@ struct DCfg {
     const int st = kStages * stage_bytes(r);
     return st > red_bytes ? st : red_bytes;
   }
+  // k-steps of the zero-point and PSAC terms (columns z_0..z_NG-1, a_0..a_r-1)
+  __host__ __device__ static int xk(int r) { return (NG + r + 15) / 16; }
+  __host__ __device__ static int small_floats(int M, int r) {
+    return (G * M + G * r + G * NG + kWarps * G + 2 * kWarps + 3) & ~3;
+  }
   __host__ __device__ static int tables_bytes(int M, int r) {
-    return lg_bytes + wt_bytes + (G * M + G * r + G * NG + 4 * G + 4) * 4;
+    return lg_bytes + wt_bytes + small_floats(M, r) * 4 + xk(r) * NT * 32 * 8;
   }
 };
 
@@ -230,7 +258,9 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
   float* mus = reinterpret_cast<float*>(tables + Cfg::lg_bytes + Cfg::wt_bytes);   // [G][M]
   float* us = mus + G * M;                                                         // [G][r]
   float* sgs = us + G * r;                                                         // [G][NG]
-  float* red = sgs + G * NG;                                                       // [kWarps][G], [kWarps]
+  float* red = sgs + G * NG;                                                       // [kWarps][G], [2][kWarps]
+  uint2* baux = reinterpret_cast<uint2*>(mus + Cfg::small_floats(M, r));           // [XK][NT][32]
+  const int XK = Cfg::xk(r);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gid = lane >> 2, tig = lane & 3;
@@ -320,18 +350,52 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
       }
     }
   }
-  // power-of-two scale of q for the tensor cores: max |q| 2^eq below 2^14
-  float qmax = 0.0f;
+  __syncthreads();           // sgs and us are complete
+  // power-of-two scales for the tensor cores: max |q| 2^eq and
+  // max(|sigma|, |u|) 2^ea below 2^14
+  float qmax = 0.0f, amax = 0.0f;
   for (int i = tid; i < G * D; i += kThreads) qmax = fmaxf(qmax, fabsf(qs[i]));
+  for (int i = tid; i < G * NG; i += kThreads) amax = fmaxf(amax, fabsf(sgs[i]));
+  for (int i = tid; i < G * r; i += kThreads) amax = fmaxf(amax, fabsf(us[i]));
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, o));
-  if (lane == 0) red[kWarps * G + warp] = qmax;
+  for (int o = 16; o > 0; o >>= 1) {
+    qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, o));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  }
+  if (lane == 0) {
+    red[kWarps * G + warp] = qmax;
+    red[kWarps * G + kWarps + warp] = amax;
+  }
   __syncthreads();
-  qmax = fmaxf(fmaxf(red[kWarps * G], red[kWarps * G + 1]), fmaxf(red[kWarps * G + 2], red[kWarps * G + 3]));
-  int qexp = 0;
+  const float* rq = red + kWarps * G;
+  qmax = fmaxf(fmaxf(rq[0], rq[1]), fmaxf(rq[2], rq[3]));
+  amax = fmaxf(fmaxf(rq[4], rq[5]), fmaxf(rq[6], rq[7]));
+  int qexp = 0, aexp = 0;
   frexpf(qmax, &qexp);
+  frexpf(amax, &aexp);
   const int eq = (qmax > 0.0f) ? 14 - qexp : 0;
+  const int ea = (amax > 0.0f) ? 14 - aexp : 0;
   const float qmul = ldexpf(1.0f, eq), qinv = ldexpf(1.0f, -eq);
+  const float amul = ldexpf(1.0f, ea), ainv = ldexpf(1.0f, -ea);
+  // B fragments of the zero-point / PSAC k-steps: aux column c is sigma_c
+  // (c < NG) or u_(c-NG) (c - NG < r), zero beyond
+  for (int i = tid; i < XK * NT * 32; i += kThreads) {
+    const int x = i / (NT * 32), nt = (i / 32) % NT, l = i % 32;
+    const int n = l >> 2, tg = l & 3;
+    const bool used = CL::used(n), lo = CL::is_lo(nt, n);
+    const int hd = min(CL::head(n), G - 1);
+    uint16_t hv[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int c = 16 * x + 2 * tg + (e & 1) + 8 * (e >> 1);
+      float v = 0.0f;
+      if (c < NG) v = sgs[hd * NG + c];
+      else if (c - NG < r) v = us[hd * r + c - NG];
+      v *= amul;
+      hv[e] = used ? (lo ? f16_lo(v) : f16_hi(v)) : uint16_t(0);
+    }
+    baux[i] = make_uint2(pack_h2(hv[0], hv[1]), pack_h2(hv[2], hv[3]));
+  }
 
   // B operand of q.k for every k-step: column gid of each n8 tile, rows
   // (channels) tig, 8+tig | 4+tig, 12+tig of the k-step's code word
@@ -412,16 +476,15 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
         for (int g = 0; g < NG; ++g) {
           float C[NT][4];
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) C[nt][i] = 0.0f;
-#pragma unroll
           for (int kk = 0; kk < 2; ++kk) {
             const int ks = 2 * g + kk;
             const uint32_t a[4] = {unpack_codes(w0[ks], mk, sck, ofk), unpack_codes(w1[ks], mk, sck, ofk),
                                    unpack_codes(w0[ks] >> 8, mk, sck, ofk), unpack_codes(w1[ks] >> 8, mk, sck, ofk)};
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma16816(C[nt], a, bq[nt][ks][0], bq[nt][ks][1]);
+            for (int nt = 0; nt < NT; ++nt) {
+              if (kk == 0) mma16816_zc(C[nt], a, bq[nt][ks][0], bq[nt][ks][1]);
+              else mma16816(C[nt], a, bq[nt][ks][0], bq[nt][ks][1]);
+            }
           }
           const float s0 = __half2float(__ushort_as_half(uint16_t(ksz[t0 * NG + g] & 0xffff))) * qinv;
           const float s1 = __half2float(__ushort_as_half(uint16_t(ksz[t1 * NG + g] & 0xffff))) * qinv;
@@ -433,12 +496,44 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
             L[nt][3] = fmaf(s1, C[nt][3], L[nt][3]);
           }
         }
+        // zero-point and PSAC terms, sum_g z_g sigma_g + sum_i a_i u_i, as XK
+        // more k-steps over the columns (z_0 .. z_NG-1, a_0 .. a_r-1) of the
+        // token's scale/zero words and PSAC coefficients (exact fp16 values)
+        {
+          const uint32_t* kz0 = ksz + t0 * NG;
+          const uint32_t* kz1 = ksz + t1 * NG;
+          const uint32_t* ps0 = reinterpret_cast<const uint32_t*>(cur + Cfg::ps_off) + t0 * (r / 2);
+          const uint32_t* ps1 = reinterpret_cast<const uint32_t*>(cur + Cfg::ps_off) + t1 * (r / 2);
+          auto aux_pair = [&](const uint32_t* kz, const uint32_t* ps, int c) -> uint32_t {
+            if (c < NG) return __byte_perm(kz[c], kz[c + 1], 0x7632);   // z_c, z_c+1
+            return (c - NG < r) ? ps[(c - NG) >> 1] : 0u;               // a pair
+          };
+          float Ca[NT][4];
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) Ca[nt][i] = 0.0f;
+          for (int x = 0; x < XK; ++x) {
+            const int c = 16 * x + 2 * tig;
+            const uint32_t a[4] = {aux_pair(kz0, ps0, c), aux_pair(kz1, ps1, c),
+                                   aux_pair(kz0, ps0, c + 8), aux_pair(kz1, ps1, c + 8)};
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              const uint2 bb = baux[(x * NT + nt) * 32 + lane];
+              mma16816(Ca[nt], a, bb.x, bb.y);
+            }
+          }
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) L[nt][i] = fmaf(Ca[nt][i], ainv, L[nt][i]);
+        }
         combine_hi_lo<G, NT>(L, tig, [&](int rs, int g, float v) { lg_s[(rs ? t1 : t0) * LS + g] = v; });
       }
     }
     __syncthreads();
 
-    // ---- owner phase (thread = token): centre, zero and PSAC terms
+    // ---- owner phase (thread = token): the centre term, online softmax
     const int t = tid;
     float lg[G];
     {
@@ -449,21 +544,6 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
       idx = min(idx, M - 1);
 #pragma unroll
       for (int g = 0; g < G; ++g) lg[g] += mus[g * M + idx];
-      const uint32_t* ksz = reinterpret_cast<const uint32_t*>(cur + Cfg::ks_off) + t * NG;
-#pragma unroll
-      for (int k = 0; k < NG; ++k) {
-        const float z = __half2float(__ushort_as_half(uint16_t(ksz[k] >> 16)));
-#pragma unroll
-        for (int g = 0; g < G; ++g) lg[g] = fmaf(z, sgs[g * NG + k], lg[g]);
-      }
-      if (r) {
-        const __half2* a2 = reinterpret_cast<const __half2*>(cur + Cfg::ps_off) + t * (r / 2);
-        for (int k = 0; k < r / 2; ++k) {
-          const float2 a = __half22float2(a2[k]);
-#pragma unroll
-          for (int g = 0; g < G; ++g) lg[g] = fmaf(us[g * r + 2 * k], a.x, fmaf(us[g * r + 2 * k + 1], a.y, lg[g]));
-        }
-      }
       if (t >= n) {
 #pragma unroll
         for (int g = 0; g < G; ++g) lg[g] = -FLT_MAX;
@@ -476,27 +556,28 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
 #pragma unroll
       for (int k = 0; k < NG; ++k) {
         vszr[k] = (t < n) ? vsz[k] : 0u;
-        smax = fmaxf(smax, __half2float(__ushort_as_half(uint16_t(vszr[k] & 0xffff))));
+        smax = fmaxf(smax, fabsf(__half2float(__ushort_as_half(uint16_t(vszr[k] & 0xffff)))));
       }
     }
     // ---- tile max per head and of the value scales (block-wide)
+    // (warp maxima by integer reductions of order-preserving keys)
+    int* redi = reinterpret_cast<int*>(red);
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      float m = lg[g];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      if (lane == 0) red[warp * G + g] = m;
+      const int m = __reduce_max_sync(0xffffffffu, f2ord(lg[g]));
+      if (lane == 0) redi[warp * G + g] = m;
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, o));
-    if (lane == 0) red[kWarps * G + warp] = smax;
+    {
+      const int m = __reduce_max_sync(0xffffffffu, __float_as_int(smax));   // smax >= 0
+      if (lane == 0) redi[kWarps * G + warp] = m;
+    }
     __syncthreads();
     // p s_v enters p.v scaled by 2^ev (largest value below 2^14), so that its
     // fp16 hi and lo halves stay normal numbers
     int ev = ev_acc;
     {
-      const float st = fmaxf(fmaxf(red[kWarps * G], red[kWarps * G + 1]),
-                             fmaxf(red[kWarps * G + 2], red[kWarps * G + 3]));
+      const float st = __int_as_float(max(max(redi[kWarps * G], redi[kWarps * G + 1]),
+                                           max(redi[kWarps * G + 2], redi[kWarps * G + 3])));
       int se = 0;
       frexpf(st, &se);
       if (st > 0.0f) ev = 14 - se;
@@ -505,7 +586,7 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
     bool rescale = false;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      const float tmax = fmaxf(fmaxf(red[g], red[G + g]), fmaxf(red[2 * G + g], red[3 * G + g]));
+      const float tmax = ord2f(max(max(redi[g], redi[G + g]), max(redi[2 * G + g], redi[3 * G + g])));
       const float m_new = fmaxf(m_run[g], tmax);
       alpha[g] = exp2f(m_run[g] - m_new);
       rescale |= (m_new != m_run[g]);
@@ -551,20 +632,19 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
           w[g] = pr[g] * sv;
           pz[g][k] = fmaf(pr[g], zv, pz[g][k]);
         }
+        // columns as described for Cols: hi halves of the G heads, then lo halves
         uint32_t hw[NCOL / 2];
+        if constexpr (G >= 4) {
 #pragma unroll
-        for (int c2 = 0; c2 < NCOL / 2; ++c2) {
-          uint16_t hv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = 2 * c2 + e, nt = col / 8, nn = col % 8;
-            hv[e] = 0;
-            if (CL::used(nn)) {
-              const float x = w[min(CL::head(nn), G - 1)];
-              hv[e] = CL::is_lo(nt, nn) ? f16_lo(x) : f16_hi(x);
-            }
-          }
-          hw[c2] = pack_h2(hv[0], hv[1]);
+          for (int j = 0; j < G / 2; ++j) split_pair(w[2 * j], w[2 * j + 1], hw[j], hw[G / 2 + j]);
+        } else if constexpr (G == 2) {
+          split_pair(w[0], w[1], hw[0], hw[1]);
+          hw[2] = hw[3] = 0u;
+        } else {
+          uint32_t hi, lo;
+          split_pair(w[0], 0.0f, hi, lo);
+          hw[0] = (hi & 0xffffu) | (lo << 16);
+          hw[1] = hw[2] = hw[3] = 0u;
         }
         uint4* dst = reinterpret_cast<uint4*>(wt_s + (size_t(k) * kTile + t) * NCOL);
 #pragma unroll
