@@ -142,7 +142,7 @@ def run_gpu(args, rank, world):
     length = s.T + 1
     scale = 1.0 / math.sqrt(s.d)
     out = torch.empty((s.B, s.H_q, s.d), dtype=torch.bfloat16, device="cuda")
-    ws = torch.empty(kv2.kv2_decode_workspace_size(cache, s.H_q, length), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(kv2.kv2_decode_workspace_size(cache, s.H_q, length), dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
     def step():

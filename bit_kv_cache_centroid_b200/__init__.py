@@ -208,7 +208,8 @@ def kv2_attention_decode(cache: Cache, length: int, Q: torch.Tensor, sm_scale: f
         out = torch.empty((B, H_q, dd), dtype=torch.float32 if out_dtype == KV2_OUT_F32 else torch.bfloat16,
                           device=Q.device)
     if ws is None:
-        ws = torch.empty(max(kv2_decode_workspace_size(cache, H_q, length), 16), dtype=torch.uint8,
+        # zeroed: the first word is the sticky error word of device-side waits
+        ws = torch.zeros(max(kv2_decode_workspace_size(cache, H_q, length), 16), dtype=torch.uint8,
                          device=Q.device)
     d = cache.desc()
     _check(_get_lib().kv2_attention_decode(ctypes.byref(d), length, _ptr(Q), H_q, float(sm_scale), _ptr(out),

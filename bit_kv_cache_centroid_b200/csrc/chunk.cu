@@ -37,6 +37,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "mbarrier.cuh"
 
 namespace kv2 {
 namespace {
@@ -69,9 +70,6 @@ constexpr uint32_t kTmemCols = 512;
 // ---------------------------------------------------------------------------
 // PTX wrappers (sm_100a)
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
 
 // UMMA shared-memory matrix descriptor: start, leading / stride byte offsets,
 // version 1 (Blackwell), layout (0 = no swizzle, 2 = 128-byte swizzle).
@@ -119,30 +117,6 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
 __device__ __forceinline__ void fence_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-// try_wait suspends the calling thread (it issues nothing) until the phase
-// completes or a hardware time limit passes; either way control comes back.
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t phase) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
-      "selp.b32 %0, 1, 0, P1;\n\t}\n"
-      : "=r"(done)
-      : "r"(bar), "r"(phase)
-      : "memory");
-  return done != 0;
-}
-// Bounded wait: until the phase completes or `budget` SM clock cycles pass.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase, unsigned long long budget) {
-  const unsigned long long t0 = clock64();
-  while (!mbar_try(bar, phase)) {
-    if (clock64() - t0 > budget) return false;
-  }
-  return true;
-}
 
 // Bounded wait that also gives up as soon as another role raised the abort
 // flag; a wait that runs out raises it.
@@ -657,11 +631,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
   }
 }
 
-unsigned long long env_budget() {
-  const char* e = std::getenv("KV2_WAIT_BUDGET_CYCLES");
-  return e ? std::strtoull(e, nullptr, 10) : (1ull << 31);   // ~1 s at 2 GHz
-}
-
 }  // namespace
 
 size_t chunk_workspace_bytes(const kv2_cache&, int, int) { return 256; }
@@ -676,9 +645,8 @@ cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t s) {
   p.B = c.B; p.H_kv = c.H_kv; p.H_q = a.H_q; p.M = c.M; p.r = c.r; p.cap = c.capacity;
   p.len = a.len; p.Nq = a.Nq; p.F = a.frame_tokens; p.out_dtype = a.out_dtype;
   p.scale_log2 = a.sm_scale * 1.4426950408889634f;
-  p.budget = env_budget();
-  const char* ft = std::getenv("KV2_FORCE_WAIT_TIMEOUT");
-  p.force_timeout = (ft && ft[0] == '1') ? 1 : 0;
+  p.budget = env_wait_budget();
+  p.force_timeout = env_force_timeout();
   if (p.force_timeout) p.budget = 1u << 20;
   cudaError_t e = cudaMemsetAsync(a.ws, 0, sizeof(int), s);
   if (e != cudaSuccess) return e;

@@ -49,6 +49,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "mbarrier.cuh"
 
 namespace kv2 {
 namespace {
@@ -56,7 +57,7 @@ namespace {
 constexpr int kTile = 128;        // tokens per tile
 constexpr int kThreads = 128;     // one thread per token in the owner phase
 constexpr int kWarps = kThreads / 32;
-constexpr int kStages = 2;
+constexpr int kStages = 3;        // tiles in shared memory (two copies ahead of the one in use)
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct SplitParams {
@@ -71,16 +72,11 @@ struct SplitParams {
   const float* P;         // [H_kv][D][r]
   float scale;            // sm_scale * log2(e)
   float* part;            // [B*H_kv][splits][G][D + 2]
+  int* err;               // sticky error word: 1 after a wait ran out of its budget
+  unsigned long long budget;   // SM clock cycles a wait may take
+  int force_timeout;      // wait on copies that are never issued (tests)
   int H_kv, H_q, M, r, cap, len, splits, tiles_per_split;
 };
-
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
 
 // d = a * b + c on two fp16 lanes
 __device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
@@ -199,7 +195,8 @@ __device__ __forceinline__ void combine_hi_lo(const float (&c)[NT][4], int tig, 
 }
 
 // Shared memory of the split kernel:
-//   stages  kStages x raw tile copies (codes, scale/zero words, ids, PSAC)
+//   stages  kStages x raw tile copies (codes, scale/zero words, ids, PSAC),
+//           filled by bulk copies that complete on one barrier per stage
 //           (reused at the end for the final reduction)
 //   lg      [kTile][LS] fp32   q.k sums per token and head
 //   wt      [NG][kTile][NCOL] fp16   p s_v per group, token and column
@@ -227,7 +224,7 @@ struct DCfg {
   static constexpr int lg_bytes = kTile * LS * 4;
   static constexpr int wt_bytes = NG * kTile * NCOL * 2;
   static constexpr int scratch_floats = (lg_bytes + wt_bytes) / 4;
-  static constexpr int red_bytes = (G * D + kThreads * G * NG) * 4;   // final reduction
+  static constexpr int red_bytes = (G * D + kWarps * G * NG) * 4;    // final reduction
   __host__ __device__ static int stage_bytes(int r) { return (ps_off + kTile * r * 2 + 15) & ~15; }
   __host__ __device__ static int stages_bytes(int r) {
     const int st = kStages * stage_bytes(r);
@@ -238,9 +235,11 @@ struct DCfg {
   __host__ __device__ static int small_floats(int M, int r) {
     return (G * M + G * r + G * NG + kWarps * G + 2 * kWarps + 3) & ~3;
   }
-  __host__ __device__ static int tables_bytes(int M, int r) {
+  // one full-barrier per stage, after the other tables
+  __host__ __device__ static int bar_off(int M, int r) {
     return lg_bytes + wt_bytes + small_floats(M, r) * 4 + xk(r) * NT * 32 * 8;
   }
+  __host__ __device__ static int tables_bytes(int M, int r) { return bar_off(M, r) + kStages * 8 + 8; }
 };
 
 template <int D, int G, bool U16>
@@ -271,27 +270,32 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
   const int t_end = min(p.len, t_begin + p.tiles_per_split * kTile);
   const int ntiles = (t_end > t_begin) ? (t_end - t_begin + kTile - 1) / kTile : 0;
 
+  // tile copies: thread 0 issues one bulk copy per stream into the tile's
+  // stage; they complete on the stage's barrier
+  const uint32_t bar0 = smem_u32(tables + Cfg::bar_off(M, r));
+  int issued = 0;                                        // tiles issued (thread 0)
   auto issue = [&](int tile) {
-    if (tile < ntiles) {
-      unsigned char* dst = smem + (tile % kStages) * stage;
-      const int t0 = t_begin + tile * kTile;
-      const int n16 = (min(kTile, t_end - t0) + 15) & ~15;   // within capacity (cap % 16 == 0)
-      const size_t s0 = base_slot + t0;
-      auto copy = [&](int off, const void* src, int bytes_per_tok) {
-        const int chunks = n16 * bytes_per_tok / 16;
-        const char* g = static_cast<const char*>(src) + s0 * bytes_per_tok;
-        for (int i = tid; i < chunks; i += kThreads) cp_async16(dst + off + i * 16, g + i * 16);
-      };
-      copy(Cfg::kc_off, p.k_code, NW * 4);
-      copy(Cfg::vc_off, p.v_code, NW * 4);
-      copy(Cfg::ks_off, p.k_sz, NG * 4);
-      copy(Cfg::vs_off, p.v_sz, NG * 4);
-      copy(Cfg::ix_off, p.cidx, Cfg::IDXB);
-      if (r) copy(Cfg::ps_off, p.psac, r * 2);
-    }
-    cp_async_commit();
+    if (tile >= ntiles || p.force_timeout) return;
+    const int st = tile % kStages;
+    const uint32_t dst = smem_u32(smem + st * stage);
+    const uint32_t bar = bar0 + 8 * st;
+    const int t0 = t_begin + tile * kTile;
+    const int n16 = (min(kTile, t_end - t0) + 15) & ~15;   // within capacity (cap % 16 == 0)
+    const size_t s0 = base_slot + t0;                      // a multiple of 16
+    mbar_arrive_expect_tx(bar, uint32_t(n16) * uint32_t(2 * NW * 4 + 2 * NG * 4 + Cfg::IDXB + 2 * r));
+    bulk_g2s(dst + Cfg::kc_off, p.k_code + s0 * NW, n16 * NW * 4, bar);
+    bulk_g2s(dst + Cfg::vc_off, p.v_code + s0 * NW, n16 * NW * 4, bar);
+    bulk_g2s(dst + Cfg::ks_off, p.k_sz + s0 * NG, n16 * NG * 4, bar);
+    bulk_g2s(dst + Cfg::vs_off, p.v_sz + s0 * NG, n16 * NG * 4, bar);
+    bulk_g2s(dst + Cfg::ix_off, static_cast<const unsigned char*>(p.cidx) + s0 * Cfg::IDXB, n16 * Cfg::IDXB, bar);
+    if (r) bulk_g2s(dst + Cfg::ps_off, p.psac + s0 * r, n16 * r * 2, bar);
+    issued = tile + 1;
   };
-  issue(0);
+  if (tid == 0) {
+    for (int i = 0; i < kStages; ++i) mbar_init(bar0 + 8 * i, 1);
+    mbar_init_fence();
+    for (int i = 0; i < kStages - 1; ++i) issue(i);
+  }
 
   // ---- query-side tables of the G query heads sharing this KV head, built
   // while the first tile is in flight (lg and wt are not used before it):
@@ -445,11 +449,18 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) oacc[mt][nt][i] = 0.0f;
 
-  for (int tile = 0; tile < ntiles; ++tile) {
-    cp_async_wait<0>();
-    __syncthreads();          // tile data ready; every thread is done with tile - 1
-    issue(tile + 1);          // into the stage tile - 1 used
-    const unsigned char* cur = smem + (tile % kStages) * stage;
+  bool aborted = false;
+  int tile = 0;
+  for (; tile < ntiles; ++tile) {
+    const int st = tile % kStages;
+    const bool ok = mbar_wait(bar0 + 8 * st, (tile / kStages) & 1, p.budget);
+    // (the barrier also tells that every thread is done with tile - 1)
+    if (__syncthreads_or(!ok)) {
+      aborted = true;
+      break;
+    }
+    if (tid == 0) issue(tile + kStages - 1);   // into the stage tile - 1 used
+    const unsigned char* cur = smem + st * stage;
     const int n = min(kTile, t_end - (t_begin + tile * kTile));
 
     // ---- q.k on the tensor cores: warp w takes tokens 16 MTK w .. 16 MTK (w + 1) - 1
@@ -712,13 +723,26 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
     // no barrier here: the next tile's first barrier orders these reads before
     // the copy into this stage and the next writes of lg / wt
   }
-  cp_async_wait<0>();
+  if (aborted) {
+    // a tile's copies did not arrive within the budget: report it, let the
+    // copies still in flight land (bounded), and poison this split's output
+    if (tid == 0) {
+      atomicExch(p.err, 1);
+      for (int j = tile; j < issued; ++j) mbar_wait(bar0 + 8 * (j % kStages), (j / kStages) & 1, p.budget);
+    }
+    float* dst = p.part + (size_t(bh) * p.splits + split) * G * (D + 2);
+    for (int i = tid; i < G * (D + 2); i += kThreads) {
+      const int c = i % (D + 2);
+      dst[i] = (c == D + 1) ? 1.0f : (c == D ? 0.0f : __int_as_float(0x7fc00000));
+    }
+    return;
+  }
   __syncthreads();
 
-  // ---- reduce: p.v sums (one lane per channel and head), p z_v and p sums
-  // over the owner threads
+  // ---- reduce: p.v sums (one lane per channel and head); p z_v and p sums
+  // over the owner threads (warp shuffles, then the 4 warps' partials)
   float* ofin = reinterpret_cast<float*>(smem);            // [G][D]
-  float* zbuf = ofin + G * D;                               // [kThreads][G][NG]
+  float* zred = ofin + G * D;                               // [kWarps][G][NG]
   const float vinv = ldexpf(1.0f, -ev_acc);
 #pragma unroll
   for (int mt = 0; mt < MTV; ++mt) {
@@ -728,7 +752,12 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
 #pragma unroll
   for (int g = 0; g < G; ++g) {
 #pragma unroll
-    for (int k = 0; k < NG; ++k) zbuf[(tid * G + g) * NG + k] = pz[g][k];
+    for (int k = 0; k < NG; ++k) {
+      float z = pz[g][k];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+      if (lane == 0) zred[(warp * G + g) * NG + k] = z;
+    }
     float l = lsum[g];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
@@ -737,10 +766,11 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
   __syncthreads();
   float* dst = p.part + (size_t(bh) * p.splits + split) * G * (D + 2);
   for (int i = tid; i < G * D; i += kThreads) {
-    const int g = i / D, c = i % D;
+    const int g = i / D, k = (i % D) / 32;
     float z = 0.0f;
-    for (int k = 0; k < kThreads; ++k) z += zbuf[(k * G + g) * NG + c / 32];
-    dst[g * (D + 2) + c] = ofin[i] + z;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) z += zred[(w * G + g) * NG + k];
+    dst[g * (D + 2) + i % D] = ofin[i] + z;
   }
   if (tid < G) {
     float mr = m_run[0];
@@ -858,20 +888,27 @@ void plan_splits(const kv2_cache& c, int H_q, int len, int* splits, int* tiles_p
 
 }  // namespace
 
+// workspace: a 256-byte header (word 0: the sticky error word), then the
+// split partials
+constexpr size_t kWsHeader = 256;
+
 size_t decode_workspace_bytes(const kv2_cache& c, int H_q, int len) {
   int splits, tps;
   plan_splits(c, H_q, len, &splits, &tps);
-  return size_t(c.B) * c.H_kv * splits * (H_q / c.H_kv) * (c.d + 2) * 4;
+  return kWsHeader + size_t(c.B) * c.H_kv * splits * (H_q / c.H_kv) * (c.d + 2) * 4;
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   const kv2_cache& c = *a.c;
   int splits, tps;
   plan_splits(c, a.H_q, a.len, &splits, &tps);
-  float* part = static_cast<float*>(a.ws);
+  float* part = reinterpret_cast<float*>(static_cast<char*>(a.ws) + kWsHeader);
+  const int force = env_force_timeout();
   SplitParams sp{c.k_code, c.v_code, c.k_sz, c.v_sz, c.cidx, c.psac,
                  static_cast<const uint16_t*>(a.Q), static_cast<const uint16_t*>(c.centroids), c.P,
-                 a.sm_scale * kLog2e, part, c.H_kv, a.H_q, c.M, c.r, c.capacity, a.len, splits, tps};
+                 a.sm_scale * kLog2e, part, static_cast<int*>(a.ws),
+                 force ? (1ull << 20) : env_wait_budget(), force,
+                 c.H_kv, a.H_q, c.M, c.r, c.capacity, a.len, splits, tps};
   const int G = a.H_q / c.H_kv;
   cudaError_t e;
   if (c.d == 64) e = (c.M > 256) ? launch_g<64, true>(G, sp, c.B, s) : launch_g<64, false>(G, sp, c.B, s);

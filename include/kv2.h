@@ -141,9 +141,10 @@ kv2_status kv2_quantize_append(const kv2_cache* cache, const uint16_t* K, const 
                                int n_new, int pos, int candidates, void* stream);
 
 /*
- * Workspace for kv2_attention_decode, in bytes: the split-K partials (per
- * query head and split, d output sums, the running maximum and the softmax
- * denominator, fp32). Returns 0 for unsupported shapes.
+ * Workspace for kv2_attention_decode, in bytes: a 256-byte header whose
+ * first 32-bit word is the sticky error word (below), then the split-K
+ * partials (per query head and split, d output sums, the running maximum and
+ * the softmax denominator, fp32). Returns 0 for unsupported shapes.
  */
 size_t kv2_decode_workspace_size(const kv2_cache* cache, int H_q, int len);
 
@@ -156,7 +157,13 @@ size_t kv2_decode_workspace_size(const kv2_cache* cache, int H_q, int len);
  * merge. fp32 arithmetic throughout.
  * Q   : bf16 [B][H_q][d]; out: [B][H_q][d], fp32 (KV2_OUT_F32) or bf16
  *       (KV2_OUT_BF16, round to nearest even). len = 0 writes zeros.
- * ws  : device workspace of kv2_decode_workspace_size(cache, H_q, len) bytes.
+ * ws  : device workspace of kv2_decode_workspace_size(cache, H_q, len) bytes,
+ *       zeroed by the caller before its first use. Its first 32-bit word is
+ *       a sticky error word: the kernel sets it to 1 when one of its waits
+ *       for the cache tiles it copies into shared memory runs out of its
+ *       budget (KV2_WAIT_BUDGET_CYCLES SM cycles, default 2^31); the outputs
+ *       of the affected (batch, KV head) are then NaN. The library never
+ *       clears it. Errors of the launch itself are returned as KV2_ERR_CUDA.
  */
 kv2_status kv2_attention_decode(const kv2_cache* cache, int len, const uint16_t* Q, int H_q,
                                 float sm_scale, void* out, int out_dtype,
@@ -178,6 +185,8 @@ kv2_status kv2_attention_decode(const kv2_cache* cache, int len, const uint16_t*
  *    stream capture.
  *  - All calls share the array and it keeps the last call's contents: calls
  *    that overlap on the GPU race on it and must be serialized by the caller.
+ *  - The array starts zeroed, so its error word (see kv2_attention_decode)
+ *    is sticky for the life of the process.
  *  - No cudaMalloc, cudaFree or other allocating call is made.
  */
 kv2_status kv2_attention_decode_noalloc(const kv2_cache* cache, int len, const uint16_t* Q,

@@ -130,3 +130,33 @@ def test_long_horizon_decode_full_size_sampled(orc):
                          pc.centroids[heads])
     ref = orc.decode(sub, P[heads], s.T, Q[:, heads], scale)
     assert_attention_close(out[:, heads], ref, what="long-horizon decode")
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(orc):
+    """Copies that are never issued: every wait on a tile runs out of its
+    budget, the kernel sets the workspace's error word, writes NaN for the
+    affected heads and returns; the next normal call on the same context is
+    correct (the error word stays set until the caller clears it)."""
+    import os
+    import bit_kv_cache_centroid_b200 as kv2
+    s = wl.spec("tiny", d=128, H_q=8, H_kv=2, M=64, r=8, T=600, B=1)
+    pc = wl.random_packed_cache(s, T=600, seed=9)
+    P = _basis(s, 4)
+    rng = np.random.default_rng(5)
+    Q = to_dev(wl.bf16_bits(rng.standard_normal((1, s.H_q, s.d)).astype(np.float32)), torch.int16)
+    gc = gpu_cache_like(pc)
+    gc.P.copy_(torch.from_numpy(P))
+    ws = torch.zeros(kv2.kv2_decode_workspace_size(gc, s.H_q, 600), dtype=torch.uint8, device="cuda")
+    os.environ["KV2_FORCE_WAIT_TIMEOUT"] = "1"
+    try:
+        bad = kv2.kv2_attention_decode(gc, 600, Q, 0.1, ws=ws)
+    finally:
+        del os.environ["KV2_FORCE_WAIT_TIMEOUT"]
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 1
+    assert torch.isnan(bad).all()
+    ws.zero_()
+    good = kv2.kv2_attention_decode(gc, 600, Q, 0.1, ws=ws).cpu().numpy()
+    assert int(ws[:4].view(torch.int32).item()) == 0
+    ref = orc.decode(pc, P, 600, Q.cpu().numpy().view(np.uint16), 0.1)
+    assert_attention_close(good, ref, what="after timeout")
