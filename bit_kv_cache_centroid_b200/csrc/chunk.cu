@@ -462,8 +462,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
     // ================= producer: packed tiles -> operand tiles =================
     // The packed fields of cached tile j+1 are loaded while tile j is
     // dequantized; the centroid half-row is fetched as soon as its id is known.
+    // lanes 8q..8q+7 of a producer warp take 8 consecutive rows and one half:
+    // their 16-byte stores then fall on 8 distinct swizzled bank groups
     const int pt = tid - kProdWarp0 * 32;
-    const int row = pt >> 1, half = pt & 1;
+    const int row = (pt >> 5) * 16 + (pt & 7) + 8 * ((pt >> 4) & 1), half = (pt >> 3) & 1;
     const size_t slot0 = (size_t(b) * p.H_kv + h) * p.cap;
     const uint4* cent4 = reinterpret_cast<const uint4*>(p.cent) + size_t(h) * p.M * (kD / 8) + half * 8;
     RawHalf raw;
