@@ -212,10 +212,41 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Code of bit position 2j of a 16-bit code field as a float times 4^j, exact:
-// (w & (3 << 2j)) | 0x4B000000 is the float 2^23 + code * 4^j.
-__device__ __forceinline__ float code_x4j(uint32_t w, int j) {
-  return __uint_as_float((w & (3u << (2 * j))) | 0x4B000000u) - 8388608.0f;
+// Packed fp32 pairs (Blackwell f32x2 arithmetic: one instruction, two lanes,
+// each rounded as its scalar counterpart)
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 pk2(float a, float b) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float2 up2(f32x2 v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ f32x2 ffma2(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f32x2 fadd2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// codes at bit positions 4i and 4i+2 of a 16-bit code field as the float pair
+// {code * 4^(2i), code * 4^(2i+1)}, exact ((w & m) | 0x4B000000 is 2^23 + code * 4^j)
+__device__ __forceinline__ f32x2 code_pair_x4j(uint32_t w, int i) {
+  const unsigned long long ww = (static_cast<unsigned long long>(w) << 32) | w;
+  const unsigned long long m =
+      (static_cast<unsigned long long>(3u << (4 * i + 2)) << 32) | static_cast<unsigned long long>(3u << (4 * i));
+  f32x2 bits;
+  asm("{\n\t.reg .b64 t;\n\tand.b64 t, %1, %2;\n\tor.b64 %0, t, 0x4B0000004B000000;\n\t}\n"
+      : "=l"(bits) : "l"(ww), "l"(m));
+  f32x2 d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(bits), "l"(0x4B0000004B000000ull));
+  return d;
 }
 
 struct ChunkParams {
@@ -280,12 +311,14 @@ __device__ void dequant_cache_half(const RawHalf& r, const uint4 (&m4)[8], int r
     const float vs = __half2float(__ushort_as_half(uint16_t(vsz[g] & 0xffff)));
     const float kz = __half2float(__ushort_as_half(uint16_t(ksz[g] >> 16)));
     const float vz = __half2float(__ushort_as_half(uint16_t(vsz[g] >> 16)));
-    float ksc[8], vsc[8];
+    f32x2 ksc[4], vsc[4];                           // {s 4^-2i, s 4^-(2i+1)}
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      ksc[j] = ks * __uint_as_float(uint32_t(127 - 2 * j) << 23);
-      vsc[j] = vs * __uint_as_float(uint32_t(127 - 2 * j) << 23);
+    for (int i = 0; i < 4; ++i) {
+      const float e0 = __uint_as_float(uint32_t(127 - 4 * i) << 23), e1 = __uint_as_float(uint32_t(125 - 4 * i) << 23);
+      ksc[i] = pk2(ks * e0, ks * e1);
+      vsc[i] = pk2(vs * e0, vs * e1);
     }
+    const f32x2 kz2 = pk2(kz, kz), vz2 = pk2(vz, vz);
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {                // 8 channels per chunk
       const int c16 = half * 8 + g * 4 + cc;         // chunk index within the row
@@ -297,11 +330,10 @@ __device__ void dequant_cache_half(const RawHalf& r, const uint4 (&m4)[8], int r
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float2 m = __half22float2(mh[i]);
-        const float k0f = __fadd_rn(__fmaf_rn(code_x4j(kword, 2 * i), ksc[2 * i], kz), m.x);
-        const float k1f = __fadd_rn(__fmaf_rn(code_x4j(kword, 2 * i + 1), ksc[2 * i + 1], kz), m.y);
-        kb[i] = pack_bf16(k0f, k1f);
-        vb[i] = pack_f16(__fmaf_rn(code_x4j(vword, 2 * i), vsc[2 * i], vz),
-                         __fmaf_rn(code_x4j(vword, 2 * i + 1), vsc[2 * i + 1], vz));
+        const float2 kf = up2(fadd2(ffma2(code_pair_x4j(kword, i), ksc[i], kz2), pk2(m.x, m.y)));
+        const float2 vf = up2(ffma2(code_pair_x4j(vword, i), vsc[i], vz2));
+        kb[i] = pack_bf16(kf.x, kf.y);
+        vb[i] = pack_f16(vf.x, vf.y);
       }
       *reinterpret_cast<uint4*>(stage + ST_K + sw128_off(row, c16)) = make_uint4(kb[0], kb[1], kb[2], kb[3]);
       *reinterpret_cast<uint4*>(stage + ST_V + sw128_off(row, c16)) = make_uint4(vb[0], vb[1], vb[2], vb[3]);
@@ -548,9 +580,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
                              fmaxf(fmaxf(mpart[4], mpart[5]), fmaxf(mpart[6], mpart[7])));
       const float m_new = fmaxf(m_run, mt * p.scale_log2);
       const float alpha = (m_new == -INFINITY) ? 1.0f : ex2(m_run - m_new);
-      float spart[8];
+      f32x2 spart[4];                                   // 8 partial sums as 4 pairs
 #pragma unroll
-      for (int i = 0; i < 8; ++i) spart[i] = 0.0f;
+      for (int i = 0; i < 4; ++i) spart[i] = 0ull;
+      const f32x2 sc2 = pk2(p.scale_log2, p.scale_log2), nm2 = pk2(-m_new, -m_new);
 #pragma unroll 1
       for (int c0 = 0; c0 < kKeys; c0 += 32) {
         float v[32];
@@ -559,25 +592,25 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
         if (full) {
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
-            const float p0 = ex2(fmaf(v[i], p.scale_log2, -m_new));
-            const float p1 = ex2(fmaf(v[i + 1], p.scale_log2, -m_new));
-            spart[i & 7] += p0;
-            spart[(i + 1) & 7] += p1;
+            const float2 x = up2(ffma2(pk2(v[i], v[i + 1]), sc2, nm2));
+            const float p0 = ex2(x.x), p1 = ex2(x.y);
+            spart[(i >> 1) & 3] = fadd2(spart[(i >> 1) & 3], pk2(p0, p1));
             pw[i / 2] = pack_f16(p0, p1);
           }
         } else {
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
-            const float p0 = (c0 + i < lim) ? ex2(fmaf(v[i], p.scale_log2, -m_new)) : 0.0f;
-            const float p1 = (c0 + i + 1 < lim) ? ex2(fmaf(v[i + 1], p.scale_log2, -m_new)) : 0.0f;
-            spart[i & 7] += p0;
-            spart[(i + 1) & 7] += p1;
+            const float2 x = up2(ffma2(pk2(v[i], v[i + 1]), sc2, nm2));
+            const float p0 = (c0 + i < lim) ? ex2(x.x) : 0.0f;
+            const float p1 = (c0 + i + 1 < lim) ? ex2(x.y) : 0.0f;
+            spart[(i >> 1) & 3] = fadd2(spart[(i >> 1) & 3], pk2(p0, p1));
             pw[i / 2] = pack_f16(p0, p1);
           }
         }
         tmem_st16(tS + c0 / 2, pw);       // P over S columns already read
       }
-      const float lsum = ((spart[0] + spart[1]) + (spart[2] + spart[3])) + ((spart[4] + spart[5]) + (spart[6] + spart[7]));
+      const float2 s01 = up2(fadd2(spart[0], spart[1])), s23 = up2(fadd2(spart[2], spart[3]));
+      const float lsum = (s01.x + s23.x) + (s01.y + s23.y);
       l_run = l_run * alpha + lsum;
       m_run = m_new;
       if (__any_sync(0xffffffffu, j > 0 && alpha != 1.0f)) {   // warp-wide TMEM access
