@@ -220,6 +220,124 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
     }
     __syncwarp();
 
+    if constexpr (KPT == 1) {
+      // One key per warp: the remaining phases run across the lanes (lane =
+      // channel within a group, or (candidate, group)), with the same
+      // arithmetic per decision as the general path below.
+      const int row = row_of(0);
+      const uint16_t* krow = key_ptr(a.K, row);
+      const uint16_t* vrow = key_ptr(a.V, row);
+      float kx[NG], vx[NG];                            // channel g * 32 + lane
+#pragma unroll
+      for (int g = 0; g < NG; ++g) {
+        kx[g] = __uint_as_float(uint32_t(krow[g * kGroup + lane]) << 16);
+        vx[g] = __uint_as_float(uint32_t(vrow[g * kGroup + lane]) << 16);
+      }
+      // ---- perturbation estimate: lane (candidate i, group g) takes the
+      // group's scale; E_i = fmaf chain over ascending g of (W_g s_g) s_g;
+      // least (E, rank)
+      int rank = 0;
+      if (C > 1) {
+        uint32_t best_e = 0xFFFFFFFFu, best_i = 0xFFFFFFFFu;
+        for (int i0 = 0; i0 < C; i0 += 32 / NG) {
+          const int i = i0 + lane / NG, g = lane % NG;
+          float sg = 0.0f;
+          if (i < C) {
+            const int j = cand_w[i];
+            const int col = (j % 32) * CPL + j / 32;
+            const uint16_t* kseg = krow + g * kGroup;
+            float mn = FLT_MAX, mx = -FLT_MAX;
+#pragma unroll
+            for (int c = 0; c < kGroup; c += 8) {
+              const uint4 kv = *reinterpret_cast<const uint4*>(kseg + c);
+              const uint32_t ku[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const float m0 = __half2float(mu_s[(g * kGroup + c + 2 * q) * MP + col]);
+                const float m1 = __half2float(mu_s[(g * kGroup + c + 2 * q + 1) * MP + col]);
+                const float x0 = __fsub_rn(__uint_as_float(ku[q] << 16), m0);
+                const float x1 = __fsub_rn(__uint_as_float(ku[q] & 0xffff0000u), m1);
+                mn = fminf(mn, fminf(x0, x1));
+                mx = fmaxf(mx, fmaxf(x0, x1));
+              }
+            }
+            sg = group_params(mn, mx).s;
+          }
+          float E = 0.0f;
+#pragma unroll
+          for (int gg = 0; gg < NG; ++gg) {
+            const float sgg = __shfl_sync(0xffffffffu, sg, (lane / NG) * NG + gg);
+            E = __fmaf_rn(__fmul_rn(a.Wg[size_t(h) * NG + gg], sgg), sgg, E);
+          }
+          const bool mine = (g == 0) && (i < C);
+          const uint32_t eo = mine ? float_order(E) : 0xFFFFFFFFu;
+          const uint32_t emin = __reduce_min_sync(0xffffffffu, eo);
+          const uint32_t imin = __reduce_min_sync(0xffffffffu, (mine && eo == emin) ? uint32_t(i) : 0xFFFFFFFFu);
+          if (emin < best_e || (emin == best_e && imin < best_i)) { best_e = emin; best_i = imin; }
+        }
+        rank = int(best_i);
+      }
+      // ---- K residual and V codecs, lane = channel of the group
+      const int jc = cand_w[rank];
+      const int colc = (jc % 32) * CPL + jc / 32;
+      const size_t slot = slot_of(row);
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+          const int c = g * kGroup + lane;
+          const float x = (which == 0) ? __fsub_rn(kx[g], __half2float(mu_s[c * MP + colc])) : vx[g];
+          float mn = x, mx = x;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          }
+          const GroupParams gp = group_params(mn, mx);
+          const uint32_t q = group_code(x, gp);
+          const uint32_t bits = q << (2 * (lane & 15));
+          const uint32_t w0 = __reduce_or_sync(0xffffffffu, lane < 16 ? bits : 0u);
+          const uint32_t w1 = __reduce_or_sync(0xffffffffu, lane >= 16 ? bits : 0u);
+          if (lane == 0) {
+            uint32_t* code = (which == 0 ? a.k_code : a.v_code) + slot * (D / 16) + g * 2;
+            *reinterpret_cast<uint2*>(code) = make_uint2(w0, w1);
+            (which == 0 ? a.k_sz : a.v_sz)[slot * NG + g] = uint32_t(gp.s_bits) | (uint32_t(gp.z_bits) << 16);
+            if (which == 0 && g == 0) {
+              if (M <= 256) static_cast<uint8_t*>(a.cidx)[slot] = uint8_t(jc);
+              else static_cast<uint16_t*>(a.cidx)[slot] = uint16_t(jc);
+            }
+          }
+          if (which == 0) e_w[c] = __fsub_rn(x, group_dequant(q, gp));
+        }
+      }
+      __syncwarp();
+      // ---- PSAC coefficients a_i = sum_c P_ci e_c: lane partial sums over
+      // channels lane, lane + 32, ..., then a warp tree (fp32; the fp16 result
+      // is within one ulp of the ascending-c chain)
+      for (int i0 = 0; i0 < a.r; i0 += 8) {
+        float acc[8];
+#pragma unroll
+        for (int ii = 0; ii < 8; ++ii) acc[ii] = 0.0f;
+#pragma unroll
+        for (int kc = 0; kc < D / 32; ++kc) {
+          const int c = lane + 32 * kc;
+          const float e = e_w[c];
+          const float* Pr = P_s + c * a.r + i0;
+#pragma unroll
+          for (int ii = 0; ii < 8; ++ii)
+            if (i0 + ii < a.r) acc[ii] = __fmaf_rn(Pr[ii], e, acc[ii]);
+        }
+        float mine = 0.0f;
+#pragma unroll
+        for (int ii = 0; ii < 8; ++ii) {
+          float v = acc[ii];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          if (lane == ii) mine = v;
+        }
+        if (lane < 8 && i0 + lane < a.r) a.psac[slot * a.r + i0 + lane] = f16_rn(mine);
+      }
+    } else {
     // ---- perturbation estimate per (key, candidate); least (E, rank) per key
     if (C > 1) {
       for (int task = lane; task < nk * C; task += 32) {
@@ -321,6 +439,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
 #pragma unroll 8
       for (int c = 0; c < D; ++c) acc = __fmaf_rn(Pcol[c * a.r], e[c], acc);
       a.psac[slot_of(row_of(k)) * a.r + i] = f16_rn(acc);
+    }
     }
     __syncwarp();    // e_w / wk_w and cand_w are reused by this warp's next tile
   }
