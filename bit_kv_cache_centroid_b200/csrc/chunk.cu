@@ -205,6 +205,13 @@ __device__ __forceinline__ uint32_t pack_f16(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// max of three floats in one instruction
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // 2^x on the MUFU unit (relative error ~2^-22; P is rounded to fp16 after)
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -569,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
         tmem_ld32(tS + c0, v);
         if (full) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) mpart[i & 7] = fmaxf(mpart[i & 7], v[i]);
+          for (int i = 0; i < 32; i += 2) mpart[(i >> 1) & 7] = fmax3(mpart[(i >> 1) & 7], v[i], v[i + 1]);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i)
