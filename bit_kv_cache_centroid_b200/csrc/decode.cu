@@ -118,6 +118,18 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uin
   hi = *reinterpret_cast<const uint32_t*>(&h);
   lo = *reinterpret_cast<const uint32_t*>(&l);
 }
+// d = A B, m16n8k32, A unsigned 8-bit, B signed 8-bit, exact int32 sums
+__device__ __forceinline__ void mma16832_u8s8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};\n"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0));
+}
+// exact float of an integer |x| < 2^22 (magic-number conversion)
+__device__ __forceinline__ float small_int_to_float(int x) {
+  return __int_as_float(0x4B400000 + x) - 12582912.0f;
+}
 // four transposed 8x8 fp16 tiles; lane i gives the address of row i % 8 of tile i / 8
 __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], const void* row) {
   const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(row));
@@ -355,7 +367,7 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
     }
   }
   __syncthreads();           // sgs and us are complete
-  // power-of-two scales for the tensor cores: max |q| 2^eq and
+  // scales for the tensor cores: max |q| 2^eq below 2^15 and
   // max(|sigma|, |u|) 2^ea below 2^14
   float qmax = 0.0f, amax = 0.0f;
   for (int i = tid; i < G * D; i += kThreads) qmax = fmaxf(qmax, fabsf(qs[i]));
@@ -377,17 +389,20 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
   int qexp = 0, aexp = 0;
   frexpf(qmax, &qexp);
   frexpf(amax, &aexp);
-  const int eq = (qmax > 0.0f) ? 14 - qexp : 0;
+  const int eq = (qmax > 0.0f) ? 15 - qexp : 0;
   const int ea = (amax > 0.0f) ? 14 - aexp : 0;
-  const float qmul = ldexpf(1.0f, eq), qinv = ldexpf(1.0f, -eq);
+  // q enters q.k as the integer rint(q qmul), |.| <= 127 * 256 (two signed
+  // 8-bit digits); qinv = 1 / qmul rounded to fp32
+  const float qmul = ldexpf(127.0f / 128.0f, eq), qinv = 1.0f / qmul;
   const float amul = ldexpf(1.0f, ea), ainv = ldexpf(1.0f, -ea);
   // B fragments of the zero-point / PSAC k-steps: aux column c is sigma_c
   // (c < NG) or u_(c-NG) (c - NG < r), zero beyond
   for (int i = tid; i < XK * NT * 32; i += kThreads) {
     const int x = i / (NT * 32), nt = (i / 32) % NT, l = i % 32;
     const int n = l >> 2, tg = l & 3;
-    const bool used = CL::used(n), lo = CL::is_lo(nt, n);
-    const int hd = min(CL::head(n), G - 1);
+    const int hq = 4 * nt + n / 2;                        // q.k column convention
+    const bool used = hq < G, lo = (n & 1) != 0;
+    const int hd = min(hq, G - 1);
     uint16_t hv[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -401,28 +416,36 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
     baux[i] = make_uint2(pack_h2(hv[0], hv[1]), pack_h2(hv[2], hv[3]));
   }
 
-  // B operand of q.k for every k-step: column gid of each n8 tile, rows
-  // (channels) tig, 8+tig | 4+tig, 12+tig of the k-step's code word
-  uint32_t bq[NT][NW][2];
+  // B operand of q.k (8-bit, one k-step of 32 per channel group): column n
+  // of n8 tile nt is head 4 nt + n / 2, digit n % 2 of q 2^eq rounded to an
+  // integer q_int = d0 + 256 d1 (d0 in [-128, 127], |q_int| <= 127 * 256); row
+  // 4 tig + i (i < 4) of the group's k-step is channel tig + 4 i of its first
+  // code word, row 16 + 4 tig + i channel tig + 4 i of its second
+  uint32_t bq8[NT][NG][2];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    const bool used = CL::used(gid), lo = CL::is_lo(nt, gid);
-    const float* qh = qs + min(CL::head(gid), G - 1) * D;
+    const int hd = 4 * nt + gid / 2, dg = gid & 1;
 #pragma unroll
-    for (int ks = 0; ks < NW; ++ks) {
-      const int c = 16 * ks + tig;
-      const float x[4] = {qh[c] * qmul, qh[c + 8] * qmul, qh[c + 4] * qmul, qh[c + 12] * qmul};
-      uint16_t hv[4];
+    for (int g = 0; g < NG; ++g) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) hv[i] = used ? (lo ? f16_lo(x[i]) : f16_hi(x[i])) : uint16_t(0);
-      bq[nt][ks][0] = pack_h2(hv[0], hv[1]);
-      bq[nt][ks][1] = pack_h2(hv[2], hv[3]);
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          int qd = 0;
+          if (hd < G) {
+            const int c = 32 * g + 16 * hf + tig + 4 * i;
+            const int qi = __float2int_rn(qs[hd * D + c] * qmul);
+            const int d1 = (qi + 128) >> 8;
+            qd = dg ? d1 : qi - 256 * d1;
+          }
+          word |= (uint32_t(qd) & 0xffu) << (8 * i);
+        }
+        bq8[nt][g][hf] = word;
+      }
     }
   }
-  // code unpacking constants (fp16 4^-i and -1024 * 4^-i in both halves)
-  const uint32_t mk = (3u << (2 * tig)) | (3u << (16 + 2 * tig));
-  const uint32_t sck = 0x3C003C00u - 0x08000800u * uint32_t(tig);
-  const uint32_t ofk = 0xE400E400u - 0x08000800u * uint32_t(tig);
+  // p.v code unpacking constants (fp16 4^-i and -1024 * 4^-i in both halves)
   const int cv = gid & 3;
   const uint32_t mv = (3u << (2 * cv)) | (3u << (16 + 2 * cv));
   const uint32_t scv = 0x3C003C00u - 0x08000800u * uint32_t(cv);
@@ -478,33 +501,25 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
           w0[i] = x0.x; w0[i + 1] = x0.y; w0[i + 2] = x0.z; w0[i + 3] = x0.w;
           w1[i] = x1.x; w1[i + 1] = x1.y; w1[i + 2] = x1.z; w1[i + 3] = x1.w;
         }
-        float L[NT][4];
+        // sum_{c in g} code_c q_int,c per group: one 8-bit k-step (exact
+        // int32), scaled by the token's s_g 2^-eq; this lane's column pair is
+        // head 4 nt + tig (both digits)
+        const uint32_t m8 = 0x03030303u;
+        float L[NT][2];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) L[nt][i] = 0.0f;
+        for (int nt = 0; nt < NT; ++nt) L[nt][0] = L[nt][1] = 0.0f;
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
-          float C[NT][4];
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk) {
-            const int ks = 2 * g + kk;
-            const uint32_t a[4] = {unpack_codes(w0[ks], mk, sck, ofk), unpack_codes(w1[ks], mk, sck, ofk),
-                                   unpack_codes(w0[ks] >> 8, mk, sck, ofk), unpack_codes(w1[ks] >> 8, mk, sck, ofk)};
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-              if (kk == 0) mma16816_zc(C[nt], a, bq[nt][ks][0], bq[nt][ks][1]);
-              else mma16816(C[nt], a, bq[nt][ks][0], bq[nt][ks][1]);
-            }
-          }
+          const uint32_t a[4] = {(w0[2 * g] >> (2 * tig)) & m8, (w1[2 * g] >> (2 * tig)) & m8,
+                                 (w0[2 * g + 1] >> (2 * tig)) & m8, (w1[2 * g + 1] >> (2 * tig)) & m8};
           const float s0 = __half2float(__ushort_as_half(uint16_t(ksz[t0 * NG + g] & 0xffff))) * qinv;
           const float s1 = __half2float(__ushort_as_half(uint16_t(ksz[t1 * NG + g] & 0xffff))) * qinv;
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            L[nt][0] = fmaf(s0, C[nt][0], L[nt][0]);
-            L[nt][1] = fmaf(s0, C[nt][1], L[nt][1]);
-            L[nt][2] = fmaf(s1, C[nt][2], L[nt][2]);
-            L[nt][3] = fmaf(s1, C[nt][3], L[nt][3]);
+            int C[4];
+            mma16832_u8s8(C, a, bq8[nt][g][0], bq8[nt][g][1]);
+            L[nt][0] = fmaf(s0, small_int_to_float(C[0] + 256 * C[1]), L[nt][0]);
+            L[nt][1] = fmaf(s1, small_int_to_float(C[2] + 256 * C[3]), L[nt][1]);
           }
         }
         // zero-point and PSAC terms, sum_g z_g sigma_g + sum_i a_i u_i, as XK
@@ -534,12 +549,16 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
               mma16816(Ca[nt], a, bb.x, bb.y);
             }
           }
+          // (columns 2 tig, 2 tig + 1: hi and lo part of head 4 nt + tig)
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) L[nt][i] = fmaf(Ca[nt][i], ainv, L[nt][i]);
+          for (int nt = 0; nt < NT; ++nt) {
+            const int hd = 4 * nt + tig;
+            if (hd < G) {
+              lg_s[t0 * LS + hd] = fmaf(Ca[nt][0] + Ca[nt][1], ainv, L[nt][0]);
+              lg_s[t1 * LS + hd] = fmaf(Ca[nt][2] + Ca[nt][3], ainv, L[nt][1]);
+            }
+          }
         }
-        combine_hi_lo<G, NT>(L, tig, [&](int rs, int g, float v) { lg_s[(rs ? t1 : t0) * LS + g] = v; });
       }
     }
     __syncthreads();
