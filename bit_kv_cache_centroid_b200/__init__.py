@@ -65,6 +65,9 @@ def _load():
     L.kv2_attention_decode.argtypes = [ctypes.POINTER(kv2_cache), I, P, I, ctypes.c_float, P, I, P, S, P]
     L.kv2_attention_decode_noalloc.restype = I
     L.kv2_attention_decode_noalloc.argtypes = [ctypes.POINTER(kv2_cache), I, P, I, ctypes.c_float, P, I, P]
+    L.kv2_append_attention_decode.restype = I
+    L.kv2_append_attention_decode.argtypes = [ctypes.POINTER(kv2_cache), P, P, I, I, I, P, I, ctypes.c_float, P, I,
+                                              P, S, P]
     L.kv2_chunk_workspace_size.restype = S
     L.kv2_chunk_workspace_size.argtypes = [ctypes.POINTER(kv2_cache), I, I]
     L.kv2_attention_chunk.restype = I
@@ -93,8 +96,8 @@ def __getattr__(name):
 
 EXPORTS = ["kv2_status_string", "kv2_last_error", "kv2_version", "kv2_fit_workspace_size",
            "kv2_fit_psac_basis", "kv2_quantize_append", "kv2_decode_workspace_size",
-           "kv2_attention_decode", "kv2_attention_decode_noalloc", "kv2_chunk_workspace_size",
-           "kv2_attention_chunk"]
+           "kv2_attention_decode", "kv2_attention_decode_noalloc", "kv2_append_attention_decode",
+           "kv2_chunk_workspace_size", "kv2_attention_chunk"]
 
 
 def _check(status: int):
@@ -214,6 +217,25 @@ def kv2_attention_decode(cache: Cache, length: int, Q: torch.Tensor, sm_scale: f
     d = cache.desc()
     _check(_get_lib().kv2_attention_decode(ctypes.byref(d), length, _ptr(Q), H_q, float(sm_scale), _ptr(out),
                                     out_dtype, _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def kv2_append_attention_decode(cache: Cache, K_new: torch.Tensor, V_new: torch.Tensor, pos: int, candidates: int,
+                                Q: torch.Tensor, sm_scale: float, out_dtype: int = KV2_OUT_F32, out=None, ws=None,
+                                stream=None):
+    """Append K_new, V_new (bf16 [B][n_new][H_kv][d]) at slot pos, then decode Q over pos + n_new tokens."""
+    B, H_q, dd = Q.shape
+    n_new = K_new.shape[1]
+    if out is None:
+        out = torch.empty((B, H_q, dd), dtype=torch.float32 if out_dtype == KV2_OUT_F32 else torch.bfloat16,
+                          device=Q.device)
+    if ws is None:
+        ws = torch.zeros(max(kv2_decode_workspace_size(cache, H_q, pos + n_new), 16), dtype=torch.uint8,
+                         device=Q.device)
+    d = cache.desc()
+    _check(_get_lib().kv2_append_attention_decode(ctypes.byref(d), _ptr(K_new), _ptr(V_new), n_new, pos, candidates,
+                                                  _ptr(Q), H_q, float(sm_scale), _ptr(out), out_dtype, _ptr(ws),
+                                                  ws.numel(), _stream(stream)))
     return out
 
 

@@ -109,22 +109,54 @@ kv2_status kv2_fit_psac_basis(const uint16_t* Qhist, int n, int H_q, int H_kv, i
   return cuda_status(kv2::launch_fit(a, static_cast<cudaStream_t>(stream)), "fit launch");
 }
 
-kv2_status kv2_quantize_append(const kv2_cache* c, const uint16_t* K, const uint16_t* V, int n_new,
-                               int pos, int candidates, void* stream) {
-  kv2_status st = check_cache(c, true, true);
-  if (st != KV2_OK) return st;
+namespace {
+
+// argument checks of a quantize/append call (the cache already checked)
+kv2_status check_quantize(const kv2_cache* c, const uint16_t* K, const uint16_t* V, int n_new, int pos,
+                          int candidates) {
   if (n_new < 0) return fail(KV2_ERR_INVALID_ARG, "quantize: n_new=%d < 0", n_new);
   if (pos < 0 || pos > c->capacity - n_new)
     return fail(KV2_ERR_CAPACITY, "quantize: slots [%d, %d) exceed capacity %d", pos, pos + n_new, c->capacity);
   if (candidates < 1 || candidates > c->M)
     return fail(KV2_ERR_INVALID_ARG, "quantize: candidates=%d outside 1..M=%d", candidates, c->M);
-  if (n_new == 0) return ok();
-  if (!K || !V || !aligned16(K) || !aligned16(V))
+  if (n_new > 0 && (!K || !V || !aligned16(K) || !aligned16(V)))
     return fail(KV2_ERR_INVALID_ARG, "quantize: K / V NULL or not 16-byte aligned");
-  kv2::QuantizeArgs a{K, V, c->B, c->H_kv, c->d, c->M, c->r, c->capacity, n_new, pos, candidates,
-                      c->centroids, c->P, c->w, c->Wg, c->k_code, c->v_code, c->k_sz, c->v_sz,
-                      c->cidx, c->psac};
-  return cuda_status(kv2::launch_quantize(a, static_cast<cudaStream_t>(stream)), "quantize launch");
+  return KV2_OK;
+}
+
+kv2::QuantizeArgs quantize_args(const kv2_cache* c, const uint16_t* K, const uint16_t* V, int n_new, int pos,
+                                int candidates) {
+  return kv2::QuantizeArgs{K, V, c->B, c->H_kv, c->d, c->M, c->r, c->capacity, n_new, pos, candidates,
+                           c->centroids, c->P, c->w, c->Wg, c->k_code, c->v_code, c->k_sz, c->v_sz,
+                           c->cidx, c->psac};
+}
+
+// argument checks of a decode call (the cache already checked)
+kv2_status check_decode(const kv2_cache* c, int len, const uint16_t* Q, int H_q, void* out, int out_dtype,
+                        void* ws, size_t ws_bytes) {
+  if (H_q <= 0 || H_q % c->H_kv) return fail(KV2_ERR_UNSUPPORTED, "decode: H_q=%d not a multiple of H_kv=%d", H_q, c->H_kv);
+  const int G = H_q / c->H_kv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return fail(KV2_ERR_UNSUPPORTED, "decode: H_q/H_kv=%d (supported 1, 2, 4, 8)", G);
+  if (len < 0 || len > c->capacity) return fail(KV2_ERR_CAPACITY, "decode: len=%d outside 0..capacity=%d", len, c->capacity);
+  if (out_dtype != KV2_OUT_F32 && out_dtype != KV2_OUT_BF16) return fail(KV2_ERR_INVALID_ARG, "decode: out_dtype=%d", out_dtype);
+  if (!Q || !out || !ws || !aligned16(Q) || !aligned16(out) || !aligned16(ws))
+    return fail(KV2_ERR_INVALID_ARG, "decode: Q / out / ws NULL or not 16-byte aligned");
+  const size_t need = kv2::decode_workspace_bytes(*c, H_q, len);
+  if (ws_bytes < need) return fail(KV2_ERR_WORKSPACE, "decode: workspace %zu < %zu bytes", ws_bytes, need);
+  return KV2_OK;
+}
+
+}  // namespace
+
+kv2_status kv2_quantize_append(const kv2_cache* c, const uint16_t* K, const uint16_t* V, int n_new,
+                               int pos, int candidates, void* stream) {
+  kv2_status st = check_cache(c, true, true);
+  if (st != KV2_OK) return st;
+  st = check_quantize(c, K, V, n_new, pos, candidates);
+  if (st != KV2_OK) return st;
+  if (n_new == 0) return ok();
+  return cuda_status(kv2::launch_quantize(quantize_args(c, K, V, n_new, pos, candidates),
+                                          static_cast<cudaStream_t>(stream)), "quantize launch");
 }
 
 size_t kv2_decode_workspace_size(const kv2_cache* c, int H_q, int len) {
@@ -137,17 +169,32 @@ kv2_status kv2_attention_decode(const kv2_cache* c, int len, const uint16_t* Q, 
                                 void* out, int out_dtype, void* ws, size_t ws_bytes, void* stream) {
   kv2_status st = check_cache(c, true, false);
   if (st != KV2_OK) return st;
-  if (H_q <= 0 || H_q % c->H_kv) return fail(KV2_ERR_UNSUPPORTED, "decode: H_q=%d not a multiple of H_kv=%d", H_q, c->H_kv);
-  const int G = H_q / c->H_kv;
-  if (G != 1 && G != 2 && G != 4 && G != 8) return fail(KV2_ERR_UNSUPPORTED, "decode: H_q/H_kv=%d (supported 1, 2, 4, 8)", G);
-  if (len < 0 || len > c->capacity) return fail(KV2_ERR_CAPACITY, "decode: len=%d outside 0..capacity=%d", len, c->capacity);
-  if (out_dtype != KV2_OUT_F32 && out_dtype != KV2_OUT_BF16) return fail(KV2_ERR_INVALID_ARG, "decode: out_dtype=%d", out_dtype);
-  if (!Q || !out || !ws || !aligned16(Q) || !aligned16(out) || !aligned16(ws))
-    return fail(KV2_ERR_INVALID_ARG, "decode: Q / out / ws NULL or not 16-byte aligned");
-  const size_t need = kv2::decode_workspace_bytes(*c, H_q, len);
-  if (ws_bytes < need) return fail(KV2_ERR_WORKSPACE, "decode: workspace %zu < %zu bytes", ws_bytes, need);
+  st = check_decode(c, len, Q, H_q, out, out_dtype, ws, ws_bytes);
+  if (st != KV2_OK) return st;
   kv2::DecodeArgs a{c, len, H_q, Q, sm_scale, out, out_dtype, ws, ws_bytes};
   return cuda_status(kv2::launch_decode(a, static_cast<cudaStream_t>(stream)), "decode launch");
+}
+
+kv2_status kv2_append_attention_decode(const kv2_cache* c, const uint16_t* K_new, const uint16_t* V_new,
+                                       int n_new, int pos, int candidates, const uint16_t* Q, int H_q,
+                                       float sm_scale, void* out, int out_dtype, void* ws, size_t ws_bytes,
+                                       void* stream) {
+  kv2_status st = check_cache(c, true, true);
+  if (st != KV2_OK) return st;
+  st = check_quantize(c, K_new, V_new, n_new, pos, candidates);
+  if (st != KV2_OK) return st;
+  const int len = pos + n_new;
+  st = check_decode(c, len, Q, H_q, out, out_dtype, ws, ws_bytes);
+  if (st != KV2_OK) return st;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  kv2::DecodeArgs a{c, len, H_q, Q, sm_scale, out, out_dtype, ws, ws_bytes};
+  if (n_new > 0) {
+    st = cuda_status(kv2::launch_quantize(quantize_args(c, K_new, V_new, n_new, pos, candidates), s),
+                     "quantize launch");
+    if (st != KV2_OK) return st;
+    a.wait_from = pos;
+  }
+  return cuda_status(kv2::launch_decode(a, s), "decode launch");
 }
 
 size_t kv2_chunk_workspace_size(const kv2_cache* c, int H_q, int Nq) {

@@ -75,6 +75,7 @@ struct SplitParams {
   int* err;               // sticky error word: 1 after a wait ran out of its budget
   unsigned long long budget;   // SM clock cycles a wait may take
   int force_timeout;      // wait on copies that are never issued (tests)
+  int wait_from;          // first slot the preceding (primary) kernel writes
   int H_kv, H_q, M, r, cap, len, splits, tiles_per_split;
 };
 
@@ -278,6 +279,7 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
   // stage; they complete on the stage's barrier
   const uint32_t bar0 = smem_u32(tables + Cfg::bar_off(M, r));
   int issued = 0;                                        // tiles issued (thread 0)
+  bool dep_done = false;                                 // primary grid waited for (thread 0)
   auto issue = [&](int tile) {
     if (tile >= ntiles || p.force_timeout) return;
     const int st = tile % kStages;
@@ -285,6 +287,12 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
     const uint32_t bar = bar0 + 8 * st;
     const int t0 = t_begin + tile * kTile;
     const int n16 = (min(kTile, t_end - t0) + 15) & ~15;   // within capacity (cap % 16 == 0)
+    if (!dep_done && t0 + n16 > p.wait_from) {
+      // the tile reaches slots the primary kernel writes: wait for its grid
+      // to complete (and its writes to be visible) before copying
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      dep_done = true;
+    }
     const size_t s0 = base_slot + t0;                      // a multiple of 16
     mbar_arrive_expect_tx(bar, uint32_t(n16) * uint32_t(2 * NW * 4 + 2 * NG * 4 + Cfg::IDXB + 2 * r));
     bulk_g2s(dst + Cfg::kc_off, p.k_code + s0 * NW, n16 * NW * 4, bar);
@@ -833,8 +841,22 @@ cudaError_t launch_split(const SplitParams& sp, int B, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(sp.splits, B * sp.H_kv);
-  kern<<<grid, kThreads, smem, s>>>(sp);
-  return cudaGetLastError();
+  if (sp.wait_from == INT32_MAX) {
+    kern<<<grid, kThreads, smem, s>>>(sp);
+    return cudaGetLastError();
+  }
+  // programmatic dependent of the kernel before it on the stream
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, sp);
 }
 
 template <int D, bool U16>
@@ -918,7 +940,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   SplitParams sp{c.k_code, c.v_code, c.k_sz, c.v_sz, c.cidx, c.psac,
                  static_cast<const uint16_t*>(a.Q), static_cast<const uint16_t*>(c.centroids), c.P,
                  a.sm_scale * kLog2e, part, static_cast<int*>(a.ws),
-                 force ? (1ull << 20) : env_wait_budget(), force,
+                 force ? (1ull << 20) : env_wait_budget(), force, a.wait_from,
                  c.H_kv, a.H_q, c.M, c.r, c.capacity, a.len, splits, tps};
   const int G = a.H_q / c.H_kv;
   cudaError_t e;

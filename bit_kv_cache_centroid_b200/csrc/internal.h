@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <climits>
 
 #include <cuda_runtime.h>
 
@@ -42,6 +43,11 @@ struct DecodeArgs {
   int out_dtype;
   void* ws;
   size_t ws_bytes;
+  // Slots at or after wait_from are written by the kernel just before on the
+  // stream; the decode then starts as its programmatic dependent and waits
+  // for it only before copying a tile that reaches such a slot. INT32_MAX:
+  // ordinary stream order.
+  int wait_from = INT32_MAX;
 };
 size_t decode_workspace_bytes(const kv2_cache& c, int H_q, int len);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);

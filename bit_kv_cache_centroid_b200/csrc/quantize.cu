@@ -64,6 +64,9 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
   unsigned long long* best_w = reinterpret_cast<unsigned long long*>(wbase + Cfg::warp_wk_bytes);  // [KPT]
   uint16_t* cand_w = reinterpret_cast<uint16_t*>(best_w + KPT);              // [KPT][C]
 
+  // a decode launched as this kernel's programmatic dependent may start now;
+  // it waits for this grid before reading the slots written here
+  asm volatile("griddepcontrol.launch_dependents;");
   const int h = blockIdx.y;
   const int rows_total = a.B * a.n_new;
   const int ntiles = (rows_total + KT - 1) / KT;

@@ -194,6 +194,29 @@ kv2_status kv2_attention_decode_noalloc(const kv2_cache* cache, int len, const u
                                         void* stream);
 
 /*
+ * kv2_append_attention_decode — one decode step of a serving loop: appends
+ * the n_new new tokens of every sequence at slots [pos, pos + n_new) exactly
+ * as kv2_quantize_append does, then attends exactly as kv2_attention_decode
+ * does over len = pos + n_new cached tokens ("QuantWM: Training-Free 2-bit KV
+ * Cache Quantization for Stable Video World Models", "1. QSAC" and "2. PSAC":
+ * new Keys are quantized as they enter the cache and attention reads the
+ * packed cache). The results are those of the two calls in sequence, bit for
+ * bit. The two kernels overlap: the attention kernel is launched as the
+ * programmatic dependent of the append kernel and waits for it only before
+ * copying a tile that reaches slot pos, so the append's latency hides behind
+ * the attention over the older tokens. The pages have no counterpart; it is a
+ * convenience of this library.
+ * K_new, V_new: bf16 [B][n_new][H_kv][d] (device); n_new = 0 only attends.
+ * Q, H_q, sm_scale, out, out_dtype, ws, ws_bytes: as kv2_attention_decode,
+ *   with ws of kv2_decode_workspace_size(cache, H_q, pos + n_new) bytes.
+ * Errors: those of both calls, checked before anything is launched.
+ */
+kv2_status kv2_append_attention_decode(const kv2_cache* cache, const uint16_t* K_new,
+                                       const uint16_t* V_new, int n_new, int pos, int candidates,
+                                       const uint16_t* Q, int H_q, float sm_scale, void* out,
+                                       int out_dtype, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Workspace for kv2_attention_chunk, in bytes (fp16 q P per query). Returns 0
  * for unsupported shapes.
  */

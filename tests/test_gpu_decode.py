@@ -160,3 +160,47 @@ def test_bounded_wait_reports_timeout_and_context_survives(orc):
     assert int(ws[:4].view(torch.int32).item()) == 0
     ref = orc.decode(pc, P, 600, Q.cpu().numpy().view(np.uint16), 0.1)
     assert_attention_close(good, ref, what="after timeout")
+
+
+@pytest.mark.parametrize("B,H_q,H_kv,M,r,T,n_new", [
+    (8, 32, 8, 64, 8, 3000, 1),       # decode step: one token per sequence, tile boundary inside a split
+    (2, 8, 2, 512, 16, 700, 5),       # several tokens, u16 ids, rank 16
+    (1, 4, 4, 64, 8, 127, 1),         # appended token in the first (only) tile
+])
+def test_append_attention_decode_equals_the_two_calls(orc, B, H_q, H_kv, M, r, T, n_new):
+    """kv2_append_attention_decode (append kernel, then the decode kernel as its
+    programmatic dependent) leaves the same packed bytes and returns the same
+    outputs, bit for bit, as kv2_quantize_append followed by
+    kv2_attention_decode; the outputs also match the oracle."""
+    import bit_kv_cache_centroid_b200 as kv2
+    s = wl.spec("tiny", d=128, H_q=H_q, H_kv=H_kv, M=M, r=r, T=T + n_new, B=B)
+    pc = wl.random_packed_cache(s, T=T + n_new, seed=T)
+    P = _basis(s, 6)
+    rng = np.random.default_rng(T + 1)
+    Kn = wl.bf16_bits(rng.standard_normal((B, n_new, H_kv, 128)).astype(np.float32))
+    Vn = wl.bf16_bits(rng.standard_normal((B, n_new, H_kv, 128)).astype(np.float32))
+    Q = to_dev(wl.bf16_bits(rng.standard_normal((B, H_q, 128)).astype(np.float32)), torch.int16)
+    w = np.abs(rng.standard_normal((H_kv, 128))).astype(np.float32) + 0.1
+    Wg = w.reshape(H_kv, 4, 32).sum(-1).astype(np.float32)
+    scale = 1.0 / np.sqrt(128)
+    outs, caches = [], []
+    for fused in (False, True):
+        gc = gpu_cache_like(pc)
+        gc.set_fit(torch.from_numpy(P), torch.from_numpy(w), torch.from_numpy(Wg))
+        Kd, Vd = to_dev(Kn, torch.int16), to_dev(Vn, torch.int16)
+        if fused:
+            o = kv2.kv2_append_attention_decode(gc, Kd, Vd, T, 4, Q, scale)
+        else:
+            kv2.kv2_quantize_append(gc, Kd, Vd, T, 4)
+            o = kv2.kv2_attention_decode(gc, T + n_new, Q, scale)
+        torch.cuda.synchronize()
+        outs.append(o.cpu().numpy())
+        caches.append(gc.to_host())
+    for name in ("k_code", "v_code", "k_sz", "v_sz", "cidx", "psac"):
+        np.testing.assert_array_equal(caches[0][name], caches[1][name], err_msg=name)
+    np.testing.assert_array_equal(outs[0], outs[1])
+    host = wl.PackedCache(B, H_kv, 128, M, r, pc.capacity,
+                          caches[1]["k_code"], caches[1]["v_code"], caches[1]["k_sz"], caches[1]["v_sz"],
+                          caches[1]["cidx"], caches[1]["psac"], pc.centroids)
+    ref = orc.decode(host, P, T + n_new, Q.cpu().numpy().view(np.uint16), scale)
+    assert_attention_close(outs[1], ref, what=f"append+decode B{B} T{T} n{n_new}")
