@@ -51,6 +51,21 @@ __device__ __forceinline__ uint32_t group_code(float x, const GroupParams& p) {
   return static_cast<uint32_t>(c);
 }
 
+// The same code as group_code, with the quotient taken as (x - z) * inv_s
+// (inv_s = 1/s correctly rounded): that product is within 2.5 ulp of the
+// correctly rounded quotient, so their rint agrees unless the product lies
+// within 2^-18 of a half-integer (the quotient is below 4, where 3 ulp is
+// under 2^-20); those rare cases take the correctly rounded division.
+__device__ __forceinline__ uint32_t group_code_recip(float x, const GroupParams& p, float inv_s) {
+  if (p.s == 0.0f) return 0u;
+  const float d = __fsub_rn(x, p.z);
+  const float qa = __fmul_rn(d, inv_s);
+  float c = rintf(qa);
+  if (fabsf(__fsub_rn(__fsub_rn(qa, floorf(qa)), 0.5f)) < 0x1p-18f) c = rintf(__fdiv_rn(d, p.s));
+  c = fminf(fmaxf(c, 0.0f), 3.0f);
+  return static_cast<uint32_t>(c);
+}
+
 __device__ __forceinline__ float group_dequant(uint32_t code, const GroupParams& p) {
   return __fmaf_rn(static_cast<float>(code), p.s, p.z);
 }

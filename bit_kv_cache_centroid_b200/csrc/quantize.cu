@@ -297,7 +297,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
           }
           const GroupParams gp = group_params(mn, mx);
-          const uint32_t q = group_code(x, gp);
+          const uint32_t q = group_code_recip(x, gp, __frcp_rn(gp.s));
           const uint32_t bits = q << (2 * (lane & 15));
           const uint32_t w0 = __reduce_or_sync(0xffffffffu, lane < 16 ? bits : 0u);
           const uint32_t w1 = __reduce_or_sync(0xffffffffu, lane >= 16 ? bits : 0u);
@@ -416,10 +416,11 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
 #pragma unroll
       for (int c = 1; c < kGroup; ++c) { mn = fminf(mn, x[c]); mx = fmaxf(mx, x[c]); }
       const GroupParams p = group_params(mn, mx);
+      const float inv_s = __frcp_rn(p.s);
       uint32_t w0 = 0, w1 = 0;
 #pragma unroll
       for (int c = 0; c < kGroup; ++c) {
-        const uint32_t q = group_code(x[c], p);
+        const uint32_t q = group_code_recip(x[c], p, inv_s);
         if (c < 16) w0 |= q << (2 * c); else w1 |= q << (2 * (c - 16));
         if (which == 0) e_w[k * D + g * kGroup + c] = __fsub_rn(x[c], group_dequant(q, p));
       }
