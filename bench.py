@@ -286,6 +286,7 @@ def extras(torch, kv2, args, pk):
                        "hbm_frac": round((rd + wr) / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
                        "ranking_TFMAps": round(fma / (ms * 1e-3) / 1e12, 3)}
     out["chunk"] = chunk_section(torch, kv2, args, pk)
+    out["long_horizon"] = long_horizon_section(torch, kv2, args, pk)
     a.record()
     for _ in range(3):
         kv2.kv2_fit_psac_basis(Qh, s.H_kv, s.r)
@@ -346,6 +347,60 @@ def chunk_section(torch, kv2, args, pk):
             "ms": round(ms, 3), "tflop": round(fl / 1e12, 4), "TFLOPs": round(tf, 1),
             "tensor_frac": round(tf / pk["bf16_tflops"], 4), "peak_tflops": pk["bf16_tflops"],
             "timeout_flag": int(ws[:4].view(torch.int32).item())}
+
+
+def long_horizon_section(torch, kv2, args, pk):
+    """Long-horizon world memory: 187,200 cached tokens (120 latent frames,
+    frames 30/60/90 revisiting frame 0), 40 heads (MHA), d=128, M=512 (u16
+    ids), r=16: decode with one query per head, and a 4,680-query chunk."""
+    s = wl.spec("long_horizon")
+    pc = wl.random_packed_cache(s, T=s.T, revisit_every=30)
+    cache = kv2.Cache(s.B, s.H_kv, s.d, s.M, s.r, pc.capacity, torch.from_numpy(pc.centroids.view(np.int16)))
+    cache.load_packed(pc)
+    del pc
+    rng = np.random.default_rng(5)
+    P = np.zeros((s.H_kv, s.d, s.r), np.float32)
+    for h in range(s.H_kv):
+        q, _ = np.linalg.qr(rng.standard_normal((s.d, s.d)))
+        P[h] = q[:, :s.r]
+    cache.P.copy_(torch.from_numpy(P))
+    dev = lambda x: torch.from_numpy(wl.bf16_bits(x).view(np.int16)).cuda()
+    scale = 1.0 / math.sqrt(s.d)
+
+    def timed(fn, n):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(n):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    Qd = dev(rng.standard_normal((s.B, s.H_q, s.d)).astype(np.float32))
+    outd = torch.empty((s.B, s.H_q, s.d), dtype=torch.bfloat16, device="cuda")
+    wsd = torch.zeros(kv2.kv2_decode_workspace_size(cache, s.H_q, s.T), dtype=torch.uint8, device="cuda")
+    dms = timed(lambda: kv2.kv2_attention_decode(cache, s.T, Qd, scale, out_dtype=kv2.KV2_OUT_BF16,
+                                                 out=outd, ws=wsd), 20)
+    dbytes = s.T * s.B * s.H_kv * BYTES_PER_TOKEN_HEAD(s.d, s.r, s.M)
+    dgbs = dbytes / (dms * 1e-3) / 1e9
+    Q = dev(rng.standard_normal((1, s.Nq, s.H_q, s.d)).astype(np.float32))
+    Ks = dev(rng.standard_normal((1, s.Nq, s.H_kv, s.d)).astype(np.float32))
+    Vs = dev(rng.standard_normal((1, s.Nq, s.H_kv, s.d)).astype(np.float32))
+    outc = torch.empty((1, s.Nq, s.H_q, s.d), dtype=torch.bfloat16, device="cuda")
+    wsc = torch.zeros(kv2.kv2_chunk_workspace_size(cache, s.H_q, s.Nq), dtype=torch.uint8, device="cuda")
+    cms = timed(lambda: kv2.kv2_attention_chunk(cache, s.T, Q, Ks, Vs, s.frame_tokens, scale,
+                                                out_dtype=kv2.KV2_OUT_BF16, out=outc, ws=wsc), 3)
+    fl = chunk_flops(s, s.T)
+    tf = fl / (cms * 1e-3) / 1e12
+    return {"workload": "long_horizon: 187,200 cached tokens, 40 heads (MHA), d=128, M=512, r=16, bf16 out",
+            "decode": {"ms": round(dms, 4), "bytes": dbytes, "GBps": round(dgbs, 1),
+                       "hbm_frac": round(dgbs / pk["hbm_gbs"], 4)},
+            "chunk": {"queries": s.Nq, "ms": round(cms, 3), "tflop": round(fl / 1e12, 4), "TFLOPs": round(tf, 1),
+                      "tensor_frac": round(tf / pk["bf16_tflops"], 4),
+                      "timeout_flag": int(wsc[:4].view(torch.int32).item())}}
 
 
 # ----------------------------------------------------------------------------
