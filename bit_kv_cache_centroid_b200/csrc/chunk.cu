@@ -46,6 +46,9 @@ constexpr int kRows = 128;        // queries per query tile (= TMEM lanes)
 constexpr int kKeys = 128;        // keys per tile
 constexpr int kD = 128;
 constexpr int kThreads = 544;     // 17 warps
+// floats per partial output row of a key-range piece: kD sums, the running
+// maximum, the running sum, padded so every row starts on 16 bytes
+constexpr int kPartRow = kD + 4;
 constexpr int kProdWarp0 = 8, kProdThreads = 256, kMmaWarp = 16;
 
 // shared-memory map (offsets from a 1024-byte aligned base)
@@ -274,6 +277,11 @@ struct ChunkParams {
   float scale_log2;
   unsigned long long budget;
   int force_timeout;
+  // work decomposition: QP query-tile pairs per (batch, head); the first
+  // n_full units run whole, each later unit as `pieces` ranges of key tiles
+  // whose partial results (part) are merged by chunk_merge
+  int QP, n_full, pieces;
+  float* part;            // [split units][pieces][2][kRows][kPartRow]
 };
 
 // ---------------------------------------------------------------------------
@@ -385,7 +393,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
   volatile int* abort = reinterpret_cast<volatile int*>(smem + OFF_BAR + B_ABORT);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qt = blockIdx.x, hq = blockIdx.y, b = blockIdx.z;
+  // work item: a whole unit (pair of query tiles of one (batch, head)), or,
+  // for the units of the last wave, one of p.pieces ranges of its key tiles
+  int unit = blockIdx.x, piece = -1;
+  if (unit >= p.n_full) {
+    const int e = unit - p.n_full;
+    unit = p.n_full + e / p.pieces;
+    piece = e % p.pieces;
+  }
+  const int qt = unit % p.QP, hq = (unit / p.QP) % p.H_q, b = unit / (p.QP * p.H_q);
   const int G = p.H_q / p.H_kv, h = hq / G;
   const int q0 = qt * 2 * kRows;
 
@@ -449,20 +465,24 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
   const int self_len = min(p.Nq, (last_q / p.F + 1) * p.F);
   const int n_self = (self_len + kKeys - 1) / kKeys;
   const int n_tiles = n_cache + n_self;
+  const int jA = piece < 0 ? 0 : piece * n_tiles / p.pieces;          // key tiles [jA, jB)
+  const int jB = piece < 0 ? n_tiles : (piece + 1) * n_tiles / p.pieces;
+  const int nloc = jB - jA;
 
   if (warp == kMmaWarp) {
     // ================= MMA issue (one thread) =================
-    for (int j = 0; j < n_tiles; ++j) {
-      const int s = j & 1;
-      const uint32_t use = uint32_t(j >> 1);
+    for (int jj = 0; jj < nloc; ++jj) {
+      const int j = jA + jj;
+      const int s = jj & 1;
+      const uint32_t use = uint32_t(jj >> 1);
       const bool cache = j < n_cache;
-      if (p.force_timeout && j == 0 && !mbar_wait_or_abort(bar + B_NEVER, 0, p.budget, abort)) break;
+      if (p.force_timeout && jj == 0 && !mbar_wait_or_abort(bar + B_NEVER, 0, p.budget, abort)) break;
       if (!mbar_wait_or_abort(bar + B_KV_FULL + 8 * s, use & 1, p.budget, abort)) break;
       fence_after_sync();
       const uint32_t st = sb + OFF_STAGE + s * STAGE_BYTES;
       bool ok = true;
       for (int x = 0; x < 2 && ok; ++x) {
-        if (j > 0 && !mbar_wait_or_abort(bar + B_O_DONE + 8 * x, (j - 1) & 1, p.budget, abort)) { ok = false; break; }
+        if (jj > 0 && !mbar_wait_or_abort(bar + B_O_DONE + 8 * x, (jj - 1) & 1, p.budget, abort)) { ok = false; break; }
         fence_after_sync();
         if (lane == 0) {
           const uint32_t tS = tmem + x * kKeys;
@@ -482,14 +502,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
       }
       if (!ok) break;
       for (int x = 0; x < 2 && ok; ++x) {
-        if (!mbar_wait_or_abort(bar + B_P_FULL + 8 * x, j & 1, p.budget, abort)) { ok = false; break; }
+        if (!mbar_wait_or_abort(bar + B_P_FULL + 8 * x, jj & 1, p.budget, abort)) { ok = false; break; }
         fence_after_sync();
         if (lane == 0) {
           const uint32_t tP = tmem + x * kKeys, tO = tmem + 2 * kKeys + x * kD;
 #pragma unroll
           for (int kk = 0; kk < kKeys / 16; ++kk)
             mma_f16_tmem_a(tO, tP + kk * 8, make_sdesc(st + ST_V + kk * 2048, 16384, 1024, kLayoutSW128), IDESC_PV,
-                           (j > 0 || kk > 0));
+                           (jj > 0 || kk > 0));
           mma_commit(bar + B_O_DONE + 8 * x);
           if (x == 1) mma_commit(bar + B_KV_EMPTY + 8 * s);   // stage free once every MMA on it is done
         }
@@ -508,11 +528,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
     const size_t slot0 = (size_t(b) * p.H_kv + h) * p.cap;
     const uint4* cent4 = reinterpret_cast<const uint4*>(p.cent) + size_t(h) * p.M * (kD / 8) + half * 8;
     RawHalf raw;
-    bool raw_ok = (n_cache > 0) && row < min(kKeys, p.len);
-    if (raw_ok) load_raw_half(p, slot0 + row, half, raw);
-    for (int j = 0; j < n_tiles; ++j) {
-      const int s = j & 1;
-      const uint32_t use = uint32_t(j >> 1);
+    bool raw_ok = nloc > 0 && jA < n_cache && row < min(kKeys, p.len - jA * kKeys);
+    if (raw_ok) load_raw_half(p, slot0 + size_t(jA) * kKeys + row, half, raw);
+    for (int jj = 0; jj < nloc; ++jj) {
+      const int j = jA + jj;
+      const int s = jj & 1;
+      const uint32_t use = uint32_t(jj >> 1);
       const bool cache = j < n_cache;
       const int k0 = cache ? j * kKeys : (j - n_cache) * kKeys;
       const int kvalid = cache ? min(kKeys, p.len - k0) : min(kKeys, self_len - k0);
@@ -524,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
       }
       RawHalf next;
       const int jn = j + 1;
-      const bool next_ok = jn < n_cache && row < min(kKeys, p.len - jn * kKeys);
+      const bool next_ok = jn < jB && jn < n_cache && row < min(kKeys, p.len - jn * kKeys);
       if (next_ok) load_raw_half(p, slot0 + size_t(jn) * kKeys + row, half, next);
       if (use >= 1 && !mbar_wait_or_abort(bar + B_KV_EMPTY + 8 * s, (use - 1) & 1, p.budget, abort)) break;
       uint8_t* stage = smem + OFF_STAGE + s * STAGE_BYTES;
@@ -558,8 +579,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
     const int my_self_lim = min(self_len, (min(qi, p.Nq - 1) / p.F + 1) * p.F);
     float m_run = -INFINITY, l_run = 0.0f;
     bool done = true;
-    for (int j = 0; j < n_tiles; ++j) {
-      if (!mbar_wait_or_abort(bar + B_S_FULL + 8 * x, j & 1, p.budget, abort)) { done = false; break; }
+    for (int jj = 0; jj < nloc; ++jj) {
+      const int j = jA + jj;
+      if (!mbar_wait_or_abort(bar + B_S_FULL + 8 * x, jj & 1, p.budget, abort)) { done = false; break; }
       fence_after_sync();
       const bool cache = j < n_cache;
       const int k0 = cache ? j * kKeys : (j - n_cache) * kKeys;
@@ -620,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
       const float lsum = (s01.x + s23.x) + (s01.y + s23.y);
       l_run = l_run * alpha + lsum;
       m_run = m_new;
-      if (__any_sync(0xffffffffu, j > 0 && alpha != 1.0f)) {   // warp-wide TMEM access
+      if (__any_sync(0xffffffffu, jj > 0 && alpha != 1.0f)) {   // warp-wide TMEM access
 #pragma unroll 1
         for (int c0 = 0; c0 < kD; c0 += 32) {
           float v[32];
@@ -633,7 +655,34 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
       fence_before_sync();
       mbar_arrive(bar + B_P_FULL + 8 * x);
     }
-    if (done && mbar_wait_or_abort(bar + B_O_DONE + 8 * x, (n_tiles - 1) & 1, p.budget, abort)) {
+    if (piece >= 0) {
+      // a piece: unnormalised output rows, running maximum and sum for the merge
+      float* part = p.part + ((size_t(unit - p.n_full) * p.pieces + piece) * 2 + x) * kRows * kPartRow +
+                    size_t(row) * kPartRow;
+      const bool have = done && nloc > 0 &&
+                        mbar_wait_or_abort(bar + B_O_DONE + 8 * x, (nloc - 1) & 1, p.budget, abort);
+      if (have) {
+        fence_after_sync();
+#pragma unroll 1
+        for (int c0 = 0; c0 < kD; c0 += 32) {
+          float v[32];
+          tmem_ld32(tO + c0, v);          // every lane: warp-wide TMEM load
+          float4* dst = reinterpret_cast<float4*>(part + c0);
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) dst[i / 4] = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        }
+        part[kD] = m_run;
+        part[kD + 1] = l_run;
+      } else if (nloc == 0 && done) {
+        for (int c = 0; c < kD; ++c) part[c] = 0.0f;
+        part[kD] = -INFINITY;
+        part[kD + 1] = 0.0f;
+      } else {                             // the pipeline gave up: poison the merged rows
+        for (int c = 0; c < kD; ++c) part[c] = __int_as_float(0x7fc00000);
+        part[kD] = 0.0f;
+        part[kD + 1] = 1.0f;
+      }
+    } else if (done && mbar_wait_or_abort(bar + B_O_DONE + 8 * x, (n_tiles - 1) & 1, p.budget, abort)) {
       fence_after_sync();
       const float inv = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
       const size_t obase = ((size_t(b) * p.Nq + min(qi, p.Nq - 1)) * p.H_q + hq) * kD;
@@ -673,9 +722,77 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
   }
 }
 
+// Merges the pieces of each split unit: log-sum-exp of the partial rows
+// (one block per query row of the unit, one thread per channel).
+__global__ void chunk_merge(const float* __restrict__ part, int n_full, int pieces, int QP, int H_q, int Nq,
+                            void* out, int out_dtype) {
+  const int su = blockIdx.x / (2 * kRows), r2 = blockIdx.x % (2 * kRows);
+  const int unit = n_full + su;
+  const int qt = unit % QP, hq = (unit / QP) % H_q, b = unit / (QP * H_q);
+  const int qi = qt * 2 * kRows + r2;
+  if (qi >= Nq) return;
+  const int c = threadIdx.x;
+  const size_t stride = size_t(2) * kRows * kPartRow;      // between pieces
+  const float* base = part + (size_t(su) * pieces * 2 + r2 / kRows) * kRows * kPartRow + size_t(r2 % kRows) * kPartRow;
+  float m = -INFINITY;
+  for (int pc = 0; pc < pieces; ++pc) {
+    const float* pr = base + pc * stride;
+    if (pr[kD + 1] > 0.0f) m = fmaxf(m, pr[kD]);
+  }
+  float o = 0.0f, l = 0.0f;
+  for (int pc = 0; pc < pieces; ++pc) {
+    const float* pr = base + pc * stride;
+    const float lp = pr[kD + 1];
+    if (!(lp > 0.0f)) continue;
+    const float f = exp2f(pr[kD] - m);
+    o = fmaf(f, pr[c], o);
+    l = fmaf(f, lp, l);
+  }
+  const float v = (l > 0.0f) ? o / l : 0.0f;
+  const size_t oi = ((size_t(b) * Nq + qi) * H_q + hq) * kD + c;
+  if (out_dtype == KV2_OUT_F32) static_cast<float*>(out)[oi] = v;
+  else static_cast<__nv_bfloat16*>(out)[oi] = __float2bfloat16_rn(v);
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// Units beyond the last whole wave are split into ranges of key tiles so the
+// last wave fills the GPU: split = units mod SMs, pieces = SMs / split (at
+// most max_pieces); no split when that leaves fewer than 2 pieces.
+struct ChunkPlan {
+  int QP, n_units, split, pieces;
+};
+ChunkPlan plan_chunk(int B, int H_q, int Nq, int max_pieces) {
+  ChunkPlan pl{};
+  pl.QP = (Nq + 2 * kRows - 1) / (2 * kRows);
+  pl.n_units = pl.QP * H_q * B;
+  const int sms = sm_count();
+  pl.split = 0;
+  pl.pieces = 1;
+  const int rem = pl.n_units % sms;
+  if (pl.n_units > sms && rem > 0) {
+    const int k = min(sms / rem, max_pieces);
+    if (k >= 2) {
+      pl.split = rem;
+      pl.pieces = k;
+    }
+  }
+  return pl;
+}
+
+constexpr size_t kChunkWsHeader = 256;
+
 }  // namespace
 
-size_t chunk_workspace_bytes(const kv2_cache&, int, int) { return 256; }
+size_t chunk_workspace_bytes(const kv2_cache& c, int H_q, int Nq) {
+  const ChunkPlan pl = plan_chunk(c.B, H_q, Nq, 1 << 20);
+  return kChunkWsHeader + size_t(pl.split) * pl.pieces * 2 * kRows * kPartRow * 4;
+}
 
 cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t s) {
   const kv2_cache& c = *a.c;
@@ -690,12 +807,24 @@ cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t s) {
   p.budget = env_wait_budget();
   p.force_timeout = env_force_timeout();
   if (p.force_timeout) p.budget = 1u << 20;
+  // every unit has at least n_cache + 1 key tiles: pieces never come out empty
+  const int n_cache = (a.len + kKeys - 1) / kKeys;
+  const ChunkPlan pl = plan_chunk(c.B, a.H_q, a.Nq, n_cache + 1);
+  p.QP = pl.QP;
+  p.n_full = pl.n_units - pl.split;
+  p.pieces = pl.pieces;
+  p.part = reinterpret_cast<float*>(static_cast<char*>(a.ws) + kChunkWsHeader);
   cudaError_t e = cudaMemsetAsync(a.ws, 0, sizeof(int), s);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(chunk_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SMEM_ALLOC));
   if (e != cudaSuccess) return e;
-  dim3 grid((a.Nq + 2 * kRows - 1) / (2 * kRows), a.H_q, c.B);
-  chunk_attn_kernel<<<grid, kThreads, SMEM_ALLOC, s>>>(p);
+  const int items = p.n_full + pl.split * pl.pieces;
+  if (items == 0) return cudaSuccess;
+  chunk_attn_kernel<<<items, kThreads, SMEM_ALLOC, s>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || pl.split == 0) return e;
+  chunk_merge<<<pl.split * 2 * kRows, kD, 0, s>>>(p.part, p.n_full, pl.pieces, pl.QP, a.H_q, a.Nq, a.out,
+                                                   a.out_dtype);
   return cudaGetLastError();
 }
 

@@ -126,6 +126,9 @@ def test_video_chunk_full_size_sampled(orc):
     Vs = _dense(rng, (1, s.Nq, s.H_kv, 128))
     picks = [0, 127, 128, 1559, 1560, 3119, 3120, 4600, s.Nq - 1] + list(rng.integers(0, s.Nq, 15))
     rows = np.array([(0, int(i), int(rng.integers(0, s.H_q))) for i in picks], np.int32)
+    # the last heads' units run as key-range pieces on a 148-SM GPU: sample them too
+    rows = np.concatenate([rows, np.array([(0, int(i), s.H_q - 1) for i in (0, 2000, 4607, s.Nq - 1)] +
+                                          [(0, 4620, s.H_q - 2)], np.int32)])
     got, ref = _run(orc, pc, P, s.T, Q, Ks, Vs, s.frame_tokens, rows=rows)
     assert_attention_close(got, ref, what="video chunk full size")
 
@@ -145,6 +148,23 @@ def test_long_horizon_chunk_full_size_sampled(orc):
     rows = np.array([(0, i, (7 * k) % s.H_q) for k, i in enumerate(picks)], np.int32)
     got, ref = _run(orc, pc, P, s.T, Q, Ks, Vs, s.frame_tokens, rows=rows)
     assert_attention_close(got, ref, what="long-horizon chunk full size")
+
+
+def test_last_wave_split_into_key_ranges(orc):
+    """150 units (75 heads x 2 query-tile pairs) on a 148-SM GPU: the last
+    wave's 2 units run as ranges of key tiles whose partial results are merged;
+    every row of the split head and rows of whole units match the oracle."""
+    s = wl.spec("tiny", d=128, H_q=75, H_kv=75, M=32, r=8, T=1024, B=1)
+    pc = wl.random_packed_cache(s, T=1024, seed=11)
+    P = _basis(s, 9)
+    rng = np.random.default_rng(21)
+    Nq, F = 300, 100
+    Q = _dense(rng, (1, Nq, 75, 128))
+    Ks = _dense(rng, (1, Nq, 75, 128))
+    Vs = _dense(rng, (1, Nq, 75, 128))
+    rows = [(0, i, 74) for i in range(Nq)] + [(0, i, h) for i, h in ((0, 0), (299, 3), (150, 40), (257, 73))]
+    got, ref = _run(orc, pc, P, 1024, Q, Ks, Vs, F, rows=np.array(rows, np.int32))
+    assert_attention_close(got, ref, what="split last wave")
 
 
 def test_bounded_wait_reports_timeout_and_context_survives(orc):
