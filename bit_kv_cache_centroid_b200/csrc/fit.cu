@@ -78,25 +78,30 @@ __device__ __forceinline__ void pair_of(int round, int i, int D, int* p, int* q)
   *q = a < b ? b : a;
 }
 
-__global__ void __launch_bounds__(256) fit_jacobi(const double* __restrict__ S_all,
-                                                  double* __restrict__ Vt_all, int D, int r,
-                                                  float* __restrict__ P, float* __restrict__ w,
-                                                  float* __restrict__ Wg, float* __restrict__ energy) {
+constexpr int kJacobiThreads = 512;
+
+__global__ void __launch_bounds__(kJacobiThreads) fit_jacobi(const double* __restrict__ S_all,
+                                                             double* __restrict__ Vt_all, int D, int r,
+                                                             float* __restrict__ P, float* __restrict__ w,
+                                                             float* __restrict__ Wg, float* __restrict__ energy) {
+  constexpr int NT = kJacobiThreads;
   extern __shared__ __align__(16) unsigned char smem[];
   double* A = reinterpret_cast<double*>(smem);             // [D][D]
   double* cs = A + D * D;                                  // [D/2]
   double* sn = cs + D / 2;                                 // [D/2]
-  double* red = sn + D / 2;                                // [256]
-  int* order = reinterpret_cast<int*>(red + 256);          // [D]
+  double* red = sn + D / 2;                                // [NT]
+  int* order = reinterpret_cast<int*>(red + NT);           // [D]
+  int* pp = order + D;                                     // [D/2] this round's pairs
+  int* qq = pp + D / 2;                                    // [D/2]
   const int h = blockIdx.x, tid = threadIdx.x;
   const double* S = S_all + size_t(h) * D * D;
   double* Vt = Vt_all + size_t(h) * D * D;
-  for (int i = tid; i < D * D; i += 256) {
+  for (int i = tid; i < D * D; i += NT) {
     A[i] = S[i];
     Vt[i] = (i / D == i % D) ? 1.0 : 0.0;
   }
   // sensitivity weights from the diagonal
-  for (int c = tid; c < D; c += 256) w[size_t(h) * D + c] = float(S[size_t(c) * D + c]);
+  for (int c = tid; c < D; c += NT) w[size_t(h) * D + c] = float(S[size_t(c) * D + c]);
   __syncthreads();
   if (tid < D / 32) {
     float acc = 0.0f;
@@ -105,10 +110,10 @@ __global__ void __launch_bounds__(256) fit_jacobi(const double* __restrict__ S_a
   }
   // total squared norm (convergence reference)
   double tot = 0.0;
-  for (int i = tid; i < D * D; i += 256) tot += A[i] * A[i];
+  for (int i = tid; i < D * D; i += NT) tot += A[i] * A[i];
   red[tid] = tot;
   __syncthreads();
-  for (int s = 128; s > 0; s >>= 1) {
+  for (int s = NT / 2; s > 0; s >>= 1) {
     if (tid < s) red[tid] += red[tid + s];
     __syncthreads();
   }
@@ -118,13 +123,13 @@ __global__ void __launch_bounds__(256) fit_jacobi(const double* __restrict__ S_a
   const int npairs = D / 2;
   for (int sweep = 0; sweep < 40; ++sweep) {
     double off = 0.0;
-    for (int i = tid; i < D * D; i += 256) {
+    for (int i = tid; i < D * D; i += NT) {
       const int a = i / D, b = i % D;
       if (a != b) off += A[i] * A[i];
     }
     red[tid] = off;
     __syncthreads();
-    for (int s = 128; s > 0; s >>= 1) {
+    for (int s = NT / 2; s > 0; s >>= 1) {
       if (tid < s) red[tid] += red[tid + s];
       __syncthreads();
     }
@@ -145,13 +150,14 @@ __global__ void __launch_bounds__(256) fit_jacobi(const double* __restrict__ S_a
         }
         cs[tid] = c;
         sn[tid] = s;
+        pp[tid] = p;
+        qq[tid] = q;
       }
       __syncthreads();
       // rows p, q of A and of Vt (J^T applied from the left; Vt rows = V columns)
-      for (int i = tid; i < npairs * D; i += 256) {
-        const int pi = i / D, k = i % D;
-        int p, q;
-        pair_of(round, pi, D, &p, &q);
+      for (int i = tid; i < npairs * D; i += NT) {
+        const int pi = i / D, k = i - pi * D;
+        const int p = pp[pi], q = qq[pi];
         const double c = cs[pi], s = sn[pi];
         const double apk = A[p * D + k], aqk = A[q * D + k];
         A[p * D + k] = c * apk - s * aqk;
@@ -162,10 +168,9 @@ __global__ void __launch_bounds__(256) fit_jacobi(const double* __restrict__ S_a
       }
       __syncthreads();
       // columns p, q of A (J applied from the right)
-      for (int i = tid; i < npairs * D; i += 256) {
-        const int pi = i % npairs, k = i / npairs;
-        int p, q;
-        pair_of(round, pi, D, &p, &q);
+      for (int i = tid; i < npairs * D; i += NT) {
+        const int k = i / npairs, pi = i - k * npairs;
+        const int p = pp[pi], q = qq[pi];
         const double c = cs[pi], s = sn[pi];
         const double akp = A[k * D + p], akq = A[k * D + q];
         A[k * D + p] = c * akp - s * akq;
@@ -175,7 +180,7 @@ __global__ void __launch_bounds__(256) fit_jacobi(const double* __restrict__ S_a
     }
   }
   // order eigenvalues descending (ties: lower index first)
-  for (int i = tid; i < D; i += 256) {
+  for (int i = tid; i < D; i += NT) {
     const double li = A[i * D + i];
     int rank = 0;
     for (int j = 0; j < D; ++j) {
@@ -191,7 +196,7 @@ __global__ void __launch_bounds__(256) fit_jacobi(const double* __restrict__ S_a
     for (int i = 0; i < r; ++i) top += A[order[i] * D + order[i]];
     energy[h] = float(all > 0.0 ? top / all : 0.0);
   }
-  for (int i = tid; i < r; i += 256) {
+  for (int i = tid; i < r; i += NT) {
     const double* v = Vt + size_t(order[i]) * D;
     int arg = 0;
     for (int c = 1; c < D; ++c)
@@ -213,10 +218,10 @@ cudaError_t launch_fit(const FitArgs& a, cudaStream_t s) {
   fit_gram<<<g1, 256, 0, s>>>(a.Qhist, a.n, a.H_q, a.H_kv, D, S);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t smem = size_t(D) * D * 8 + size_t(D) * 8 + 256 * 8 + size_t(D) * 4;
+  const size_t smem = size_t(D) * D * 8 + size_t(D) * 8 + kJacobiThreads * 8 + size_t(D) * 4 + size_t(D) * 4;
   e = cudaFuncSetAttribute(fit_jacobi, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  fit_jacobi<<<a.H_kv, 256, smem, s>>>(S, Vt, D, a.r, a.P, a.w, a.Wg, a.energy);
+  fit_jacobi<<<a.H_kv, kJacobiThreads, smem, s>>>(S, Vt, D, a.r, a.P, a.w, a.Wg, a.energy);
   return cudaGetLastError();
 }
 
