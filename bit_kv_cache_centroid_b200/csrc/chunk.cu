@@ -222,29 +222,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Packed fp32 pairs (Blackwell f32x2 arithmetic: one instruction, two lanes,
-// each rounded as its scalar counterpart)
-typedef unsigned long long f32x2;
-__device__ __forceinline__ f32x2 pk2(float a, float b) {
-  f32x2 r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ float2 up2(f32x2 v) {
-  float2 r;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
-  return r;
-}
-__device__ __forceinline__ f32x2 ffma2(f32x2 a, f32x2 b, f32x2 c) {
-  f32x2 d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ f32x2 fadd2(f32x2 a, f32x2 b) {
-  f32x2 d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
 // codes at bit positions 4i and 4i+2 of a 16-bit code field as the float pair
 // {code * 4^(2i), code * 4^(2i+1)}, exact ((w & m) | 0x4B000000 is 2^23 + code * 4^j)
 __device__ __forceinline__ f32x2 code_pair_x4j(uint32_t w, int i) {

@@ -185,10 +185,36 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
         } else {
           m[0] = __half2float(mu_base[c * MP]);
         }
+        // the same fmaf per (key, centre), two at a time (fma.rn.f32x2 rounds
+        // each lane as fmaf): pairs of centres when CPL >= KPT, else of keys
+        if constexpr (CPL >= 2 && CPL >= KPT) {
 #pragma unroll
-        for (int k = 0; k < KPT; ++k)
+          for (int k = 0; k < KPT; ++k) {
+            const f32x2 w2 = pk2(wk[k], wk[k]);
 #pragma unroll
-          for (int j = 0; j < CPL; ++j) acc[k][j] = __fmaf_rn(wk[k], m[j], acc[k][j]);
+            for (int j = 0; j < CPL; j += 2) {
+              const float2 r = up2(ffma2(w2, pk2(m[j], m[j + 1]), pk2(acc[k][j], acc[k][j + 1])));
+              acc[k][j] = r.x;
+              acc[k][j + 1] = r.y;
+            }
+          }
+        } else if constexpr (KPT >= 2) {
+#pragma unroll
+          for (int j = 0; j < CPL; ++j) {
+            const f32x2 m2 = pk2(m[j], m[j]);
+#pragma unroll
+            for (int k = 0; k < KPT; k += 2) {
+              const float2 r = up2(ffma2(pk2(wk[k], wk[k + 1]), m2, pk2(acc[k][j], acc[k + 1][j])));
+              acc[k][j] = r.x;
+              acc[k + 1][j] = r.y;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < KPT; ++k)
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) acc[k][j] = __fmaf_rn(wk[k], m[j], acc[k][j]);
+        }
       }
 #pragma unroll
       for (int j = 0; j < CPL; ++j) {
