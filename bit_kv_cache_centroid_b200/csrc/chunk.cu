@@ -208,13 +208,6 @@ __device__ __forceinline__ uint32_t pack_f16(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// max of three floats in one instruction
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-
 // 2^x on the MUFU unit (relative error ~2^-22; P is rounded to fp16 after)
 __device__ __forceinline__ float ex2(float x) {
   float y;

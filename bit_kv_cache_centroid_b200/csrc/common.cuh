@@ -66,6 +66,18 @@ __device__ __forceinline__ uint32_t group_code_recip(float x, const GroupParams&
   return static_cast<uint32_t>(c);
 }
 
+// min / max of three floats in one instruction
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Packed fp32 pairs (Blackwell f32x2 arithmetic: one instruction, two lanes,
 // each rounded as its scalar counterpart)
 typedef unsigned long long f32x2;

@@ -286,8 +286,8 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
                 const float m1 = __half2float(mu_s[(g * kGroup + c + 2 * q + 1) * MP + col]);
                 const float x0 = __fsub_rn(__uint_as_float(ku[q] << 16), m0);
                 const float x1 = __fsub_rn(__uint_as_float(ku[q] & 0xffff0000u), m1);
-                mn = fminf(mn, fminf(x0, x1));
-                mx = fmaxf(mx, fmaxf(x0, x1));
+                mn = fmin3(mn, x0, x1);
+                mx = fmax3(mx, x0, x1);
               }
             }
             sg = group_params(mn, mx).s;
@@ -388,8 +388,8 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
               const float m1 = __half2float(mu_s[(c + 2 * q + 1) * MP + col]);
               const float x0 = __fsub_rn(__uint_as_float(ku[q] << 16), m0);
               const float x1 = __fsub_rn(__uint_as_float(ku[q] & 0xffff0000u), m1);
-              mn = fminf(mn, fminf(x0, x1));
-              mx = fmaxf(mx, fmaxf(x0, x1));
+              mn = fmin3(mn, x0, x1);
+              mx = fmax3(mx, x0, x1);
             }
           }
           const GroupParams p = group_params(mn, mx);
@@ -440,7 +440,9 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
       }
       float mn = x[0], mx = x[0];
 #pragma unroll
-      for (int c = 1; c < kGroup; ++c) { mn = fminf(mn, x[c]); mx = fmaxf(mx, x[c]); }
+      for (int c = 1; c + 1 < kGroup; c += 2) { mn = fmin3(mn, x[c], x[c + 1]); mx = fmax3(mx, x[c], x[c + 1]); }
+      mn = fminf(mn, x[kGroup - 1]);
+      mx = fmaxf(mx, x[kGroup - 1]);
       const GroupParams p = group_params(mn, mx);
       const float inv_s = __frcp_rn(p.s);
       uint32_t w0 = 0, w1 = 0;
