@@ -161,6 +161,25 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// the same load without its wait: the registers are defined only after a
+// later tmem_wait_ld (or tmem_anchor, placed after that wait) on them
+__device__ __forceinline__ void tmem_ld32_issue(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+// waits for every load issued before; ties r to the wait so no use of r moves above it
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]) :: "memory");
+}
+// no instruction: orders later uses of r after the preceding (volatile) wait
+__device__ __forceinline__ void tmem_anchor(uint32_t (&r)[32]) {
+  asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
@@ -174,7 +193,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])),
       "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
       : "memory");
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
@@ -184,7 +202,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
       "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
       "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // byte offset of 16-byte chunk `c16` (0..15) of row `row` in a [2][128][128 B]
@@ -563,16 +580,24 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
 #pragma unroll
       for (int i = 0; i < 8; ++i) mpart[i] = -INFINITY;
 #pragma unroll 1
-      for (int c0 = 0; c0 < kKeys; c0 += 32) {
-        float v[32];
-        tmem_ld32(tS + c0, v);
+      for (int c0 = 0; c0 < kKeys; c0 += 64) {      // 64 columns per wait
+        uint32_t ra[32], rb[32];
+        tmem_ld32_issue(tS + c0, ra);
+        tmem_ld32_issue(tS + c0 + 32, rb);
+        tmem_wait_ld(ra);
+        tmem_anchor(rb);
         if (full) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) mpart[(i >> 1) & 7] = fmax3(mpart[(i >> 1) & 7], v[i], v[i + 1]);
+          for (int i = 0; i < 32; i += 2) {
+            mpart[(i >> 1) & 7] = fmax3(mpart[(i >> 1) & 7], __uint_as_float(ra[i]), __uint_as_float(ra[i + 1]));
+            mpart[(i >> 1) & 7] = fmax3(mpart[(i >> 1) & 7], __uint_as_float(rb[i]), __uint_as_float(rb[i + 1]));
+          }
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (c0 + i < lim) mpart[i & 7] = fmaxf(mpart[i & 7], v[i]);
+          for (int i = 0; i < 32; ++i) {
+            if (c0 + i < lim) mpart[i & 7] = fmaxf(mpart[i & 7], __uint_as_float(ra[i]));
+            if (c0 + 32 + i < lim) mpart[i & 7] = fmaxf(mpart[i & 7], __uint_as_float(rb[i]));
+          }
         }
       }
       const float mt = fmaxf(fmaxf(fmaxf(mpart[0], mpart[1]), fmaxf(mpart[2], mpart[3])),
@@ -606,8 +631,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
             pw[i / 2] = pack_f16(p0, p1);
           }
         }
-        tmem_st16(tS + c0 / 2, pw);       // P over S columns already read
+        tmem_st16(tS + c0 / 2, pw);       // P over S columns already read (no wait: later loads read other columns)
       }
+      tmem_wait_st();
       const float2 s01 = up2(fadd2(spart[0], spart[1])), s23 = up2(fadd2(spart[2], spart[3]));
       const float lsum = (s01.x + s23.x) + (s01.y + s23.y);
       l_run = l_run * alpha + lsum;
@@ -621,6 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
           for (int i = 0; i < 32; ++i) v[i] *= alpha;
           tmem_st32(tO + c0, v);
         }
+        tmem_wait_st();
       }
       fence_before_sync();
       mbar_arrive(bar + B_P_FULL + 8 * x);
