@@ -225,12 +225,6 @@ __device__ __forceinline__ uint32_t pack_f16(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// 2^x on the MUFU unit (relative error ~2^-22; P is rounded to fp16 after)
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 
 // codes at bit positions 4i and 4i+2 of a 16-bit code field as the float pair
 // {code * 4^(2i), code * 4^(2i+1)}, exact ((w & m) | 0x4B000000 is 2^23 + code * 4^j)
@@ -280,7 +274,6 @@ struct ChunkParams {
 struct RawHalf {
   uint4 kw, vw;       // 4 code words each
   uint2 ksz, vsz;     // 2 groups: fp16 scale | fp16 zero << 16
-  uint4 a0, a1;       // PSAC coefficients (half 0 only)
   int idx;            // centroid id
 };
 
@@ -291,15 +284,21 @@ __device__ __forceinline__ void load_raw_half(const ChunkParams& p, size_t slot,
   r.vsz = *reinterpret_cast<const uint2*>(p.v_sz + slot * 4 + half * 2);
   r.idx = (p.M <= 256) ? int(static_cast<const uint8_t*>(p.cidx)[slot])
                        : int(static_cast<const uint16_t*>(p.cidx)[slot]);
-  r.a0 = make_uint4(0, 0, 0, 0);
-  r.a1 = make_uint4(0, 0, 0, 0);
-  if (half == 0 && p.r >= 8) r.a0 = *reinterpret_cast<const uint4*>(p.psac + slot * p.r);
-  if (half == 0 && p.r >= 16) r.a1 = *reinterpret_cast<const uint4*>(p.psac + slot * p.r + 8);
+}
+
+// the PSAC row of a cached token (fp16, zero-padded to 16 coefficients);
+// loaded with the centroid half-row, not with the prefetched fields
+__device__ __forceinline__ void load_psac(const ChunkParams& p, size_t slot, uint4& a0, uint4& a1) {
+  a0 = make_uint4(0, 0, 0, 0);
+  a1 = make_uint4(0, 0, 0, 0);
+  if (p.r >= 8) a0 = *reinterpret_cast<const uint4*>(p.psac + slot * p.r);
+  if (p.r >= 16) a1 = *reinterpret_cast<const uint4*>(p.psac + slot * p.r + 8);
 }
 
 // half a Khat (bf16) row and half a Vhat (fp16) row from the packed fields and
 // the centroid half-row m4; half 0 also writes the PSAC row
-__device__ void dequant_cache_half(const RawHalf& r, const uint4 (&m4)[8], int row, int half, uint8_t* stage) {
+__device__ void dequant_cache_half(const RawHalf& r, const uint4 (&m4)[8], const uint4& a0, const uint4& a1, int row,
+                                   int half, uint8_t* stage) {
   const uint32_t kw[4] = {r.kw.x, r.kw.y, r.kw.z, r.kw.w};
   const uint32_t vw[4] = {r.vw.x, r.vw.y, r.vw.z, r.vw.w};
   const uint32_t ksz[2] = {r.ksz.x, r.ksz.y};
@@ -342,8 +341,8 @@ __device__ void dequant_cache_half(const RawHalf& r, const uint4 (&m4)[8], int r
     }
   }
   if (half == 0) {
-    *reinterpret_cast<uint4*>(stage + ST_A + nosw_off(row, 0)) = r.a0;
-    *reinterpret_cast<uint4*>(stage + ST_A + nosw_off(row, 1)) = r.a1;
+    *reinterpret_cast<uint4*>(stage + ST_A + nosw_off(row, 0)) = a0;
+    *reinterpret_cast<uint4*>(stage + ST_A + nosw_off(row, 1)) = a1;
   }
 }
 
@@ -524,11 +523,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
       const bool cache = j < n_cache;
       const int k0 = cache ? j * kKeys : (j - n_cache) * kKeys;
       const int kvalid = cache ? min(kKeys, p.len - k0) : min(kKeys, self_len - k0);
-      uint4 m4[8];
+      uint4 m4[8], a0, a1;
       if (cache && raw_ok) {
         const uint4* mu = cent4 + size_t(min(raw.idx, p.M - 1)) * (kD / 8);
 #pragma unroll
         for (int c = 0; c < 8; ++c) m4[c] = __ldg(mu + c);
+        if (half == 0) load_psac(p, slot0 + size_t(j) * kKeys + row, a0, a1);
       }
       RawHalf next;
       const int jn = j + 1;
@@ -538,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
       uint8_t* stage = smem + OFF_STAGE + s * STAGE_BYTES;
       if (row < kvalid) {
         if (cache) {
-          dequant_cache_half(raw, m4, row, half, stage);
+          dequant_cache_half(raw, m4, a0, a1, row, half, stage);
         } else {
           const size_t srow = (size_t(b) * p.Nq + k0 + row) * p.H_kv + h;
           copy_self_half(p.Ks + srow * kD, p.Vs + srow * kD, row, half, stage);
