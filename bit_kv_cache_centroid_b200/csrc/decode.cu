@@ -79,16 +79,6 @@ struct SplitParams {
   int H_kv, H_q, M, r, cap, len, splits, tiles_per_split;
 };
 
-// d = a * b + c on two fp16 lanes
-__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-// two codes (at the bits of `mask` in each half of x) -> two exact fp16 codes
-__device__ __forceinline__ uint32_t unpack_codes(uint32_t x, uint32_t mask, uint32_t scale, uint32_t offset) {
-  return hfma2((x & mask) | 0x64006400u, scale, offset);
-}
 // d += A B, m16n8k16, fp16 operands, fp32 accumulators
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -103,14 +93,6 @@ __device__ __forceinline__ int f2ord(float x) {
   return i ^ ((i >> 31) & 0x7fffffff);
 }
 __device__ __forceinline__ float ord2f(int k) { return __int_as_float(k ^ ((k >> 31) & 0x7fffffff)); }
-// two fp32 values as fp16 pairs hi = fp16(x), lo = fp16(x - hi)
-__device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uint32_t& lo) {
-  const __half2 h = __floats2half2_rn(x0, x1);
-  const float2 hf = __half22float2(h);
-  const __half2 l = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
-  hi = *reinterpret_cast<const uint32_t*>(&h);
-  lo = *reinterpret_cast<const uint32_t*>(&l);
-}
 // d = A B, m16n8k32, A unsigned 8-bit, B signed 8-bit, exact int32 sums
 __device__ __forceinline__ void mma16832_u8s8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -445,25 +427,30 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
       }
     }
   }
-  // p.v code unpacking constants (fp16 4^-i and -1024 * 4^-i in both halves)
+  // p.v code mask: this lane's channels sit at bits 2 cv..2 cv + 1 of a byte,
+  // and the masked half is the fp16 subnormal code * 4^cv * 2^-24 (exact)
   const int cv = gid & 3;
   const uint32_t mv = (3u << (2 * cv)) | (3u << (16 + 2 * cv));
-  const uint32_t scv = 0x3C003C00u - 0x08000800u * uint32_t(cv);
-  const uint32_t ofv = 0xE400E400u - 0x08000800u * uint32_t(cv);
   const uint32_t selv0 = uint32_t(gid >> 2) | (uint32_t(4 + (gid >> 2)) << 8);       // channel gid
   const uint32_t selv1 = uint32_t(2 + (gid >> 2)) | (uint32_t(6 + (gid >> 2)) << 8);  // channel gid + 8
   // heads of this lane's two accumulator columns in p.v
   const int hc0 = min(CL::head(2 * tig), G - 1), hc1 = min(CL::head(2 * tig + 1), G - 1);
 
-  float m_run[G], lsum[G], pz[G][NG];
-  float oacc[MTV][NT][4];     // p.v sums scaled by 2^ev_acc
+  // per-thread running sums over the tokens it owns, heads in pairs (2j, 2j+1)
+  constexpr int GP = (G + 1) / 2;
+  float m_run[G], m_thr[G];   // running maximum and the bound m_run + 8 that forces a refresh
+  f32x2 lsum2[GP], pz2[GP][NG];
+  float oacc[MTV][NT][4];     // p.v sums scaled by 2^ev_acc 2^-24 4^cv
   int ev_acc = 0;
+  uint32_t s_thr = 0;         // fp16 bits of 2^(6 - ev_acc): |s_v| at or above it forces a refresh
+  float vmul = 1.0f;          // 2^ev_acc
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    m_run[g] = -FLT_MAX;
-    lsum[g] = 0.0f;
+  for (int g = 0; g < G; ++g) m_run[g] = m_thr[g] = -FLT_MAX;
 #pragma unroll
-    for (int k = 0; k < NG; ++k) pz[g][k] = 0.0f;
+  for (int j = 0; j < GP; ++j) {
+    lsum2[j] = 0ull;
+#pragma unroll
+    for (int k = 0; k < NG; ++k) pz2[j][k] = 0ull;
   }
 #pragma unroll
   for (int mt = 0; mt < MTV; ++mt)
@@ -502,8 +489,8 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
           w1[i] = x1.x; w1[i + 1] = x1.y; w1[i + 2] = x1.z; w1[i + 3] = x1.w;
         }
         // sum_{c in g} code_c q_int,c per group: one 8-bit k-step (exact
-        // int32), scaled by the token's s_g 2^-eq; this lane's column pair is
-        // head 4 nt + tig (both digits)
+        // int32), scaled by the token's s_g (and once at the end by 1 / qmul);
+        // this lane's column pair is head 4 nt + tig (both digits)
         const uint32_t m8 = 0x03030303u;
         float L[NT][2];
 #pragma unroll
@@ -512,8 +499,8 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
         for (int g = 0; g < NG; ++g) {
           const uint32_t a[4] = {(w0[2 * g] >> (2 * tig)) & m8, (w1[2 * g] >> (2 * tig)) & m8,
                                  (w0[2 * g + 1] >> (2 * tig)) & m8, (w1[2 * g + 1] >> (2 * tig)) & m8};
-          const float s0 = __half2float(__ushort_as_half(uint16_t(ksz[t0 * NG + g] & 0xffff))) * qinv;
-          const float s1 = __half2float(__ushort_as_half(uint16_t(ksz[t1 * NG + g] & 0xffff))) * qinv;
+          const float s0 = __half2float(__ushort_as_half(uint16_t(ksz[t0 * NG + g] & 0xffff)));
+          const float s1 = __half2float(__ushort_as_half(uint16_t(ksz[t1 * NG + g] & 0xffff)));
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
             int C[4];
@@ -554,8 +541,8 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
           for (int nt = 0; nt < NT; ++nt) {
             const int hd = 4 * nt + tig;
             if (hd < G) {
-              lg_s[t0 * LS + hd] = fmaf(Ca[nt][0] + Ca[nt][1], ainv, L[nt][0]);
-              lg_s[t1 * LS + hd] = fmaf(Ca[nt][2] + Ca[nt][3], ainv, L[nt][1]);
+              lg_s[t0 * LS + hd] = fmaf(L[nt][0], qinv, (Ca[nt][0] + Ca[nt][1]) * ainv);
+              lg_s[t1 * LS + hd] = fmaf(L[nt][1], qinv, (Ca[nt][2] + Ca[nt][3]) * ainv);
             }
           }
         }
@@ -573,108 +560,124 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
       else idx = cur[Cfg::ix_off + t];
       idx = min(idx, M - 1);
 #pragma unroll
-      for (int g = 0; g < G; ++g) lg[g] += mus[g * M + idx];
-      if (t >= n) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) lg[g] = -FLT_MAX;
-      }
+      for (int g = 0; g < G; ++g) lg[g] = (t < n) ? lg[g] + mus[g * M + idx] : -FLT_MAX;
     }
     uint32_t vszr[NG];
-    float smax = 0.0f;                               // largest value scale of the token
+    uint32_t smaxb = 0;                              // largest |s_v| of the token, fp16 bits
     {
       const uint32_t* vsz = reinterpret_cast<const uint32_t*>(cur + Cfg::vs_off) + t * NG;
 #pragma unroll
       for (int k = 0; k < NG; ++k) {
         vszr[k] = (t < n) ? vsz[k] : 0u;
-        smax = fmaxf(smax, fabsf(__half2float(__ushort_as_half(uint16_t(vszr[k] & 0xffff)))));
+        smaxb = max(smaxb, vszr[k] & 0x7fffu);
       }
     }
-    // ---- tile max per head and of the value scales (block-wide)
-    // (warp maxima by integer reductions of order-preserving keys)
-    int* redi = reinterpret_cast<int*>(red);
+    // Probabilities are taken against the running maximum, which may trail
+    // the true one (p <= 2^8), and p s_v enters p.v scaled by 2^ev_acc with
+    // |s_v| 2^ev_acc < 2^6, so p s_v 2^ev_acc < 2^14 keeps its fp16 halves
+    // normal. The first tile, and a tile that breaks either bound, refresh
+    // both from the block-wide tile maxima and rescale the running sums; the
+    // exponents stay consistent because the partial sums and the running
+    // maximum always move together.
+    bool need = (tile == 0) || smaxb >= s_thr;
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const int m = __reduce_max_sync(0xffffffffu, f2ord(lg[g]));
-      if (lane == 0) redi[warp * G + g] = m;
-    }
-    {
-      const int m = __reduce_max_sync(0xffffffffu, __float_as_int(smax));   // smax >= 0
-      if (lane == 0) redi[kWarps * G + warp] = m;
-    }
-    __syncthreads();
-    // p s_v enters p.v scaled by 2^ev (largest value below 2^14), so that its
-    // fp16 hi and lo halves stay normal numbers
-    int ev = ev_acc;
-    {
-      const float st = __int_as_float(max(max(redi[kWarps * G], redi[kWarps * G + 1]),
-                                           max(redi[kWarps * G + 2], redi[kWarps * G + 3])));
-      int se = 0;
-      frexpf(st, &se);
-      if (st > 0.0f) ev = 14 - se;
-    }
-    float alpha[G];
-    bool rescale = false;
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float tmax = ord2f(max(max(redi[g], redi[G + g]), max(redi[2 * G + g], redi[3 * G + g])));
-      const float m_new = fmaxf(m_run[g], tmax);
-      alpha[g] = exp2f(m_run[g] - m_new);
-      rescale |= (m_new != m_run[g]);
-      m_run[g] = m_new;
-    }
-    if (rescale || ev != ev_acc) {                   // uniform across the CTA
-      const float f = ldexpf(1.0f, ev - ev_acc);
-      float ac0 = f, ac1 = f;
+    for (int g = 0; g < G; ++g) need |= lg[g] > m_thr[g];
+    if (__syncthreads_or(need)) {
+      // (warp maxima by integer reductions of order-preserving keys)
+      int* redi = reinterpret_cast<int*>(red);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        lsum[g] *= alpha[g];
-#pragma unroll
-        for (int k = 0; k < NG; ++k) pz[g][k] *= alpha[g];
-        if (g == hc0) ac0 = alpha[g] * f;
-        if (g == hc1) ac1 = alpha[g] * f;
+        const int m = __reduce_max_sync(0xffffffffu, f2ord(lg[g]));
+        if (lane == 0) redi[warp * G + g] = m;
       }
-      ev_acc = ev;
+      {
+        const int m = __reduce_max_sync(0xffffffffu, int(min(smaxb, 0x7bffu)));   // finite fp16
+        if (lane == 0) redi[kWarps * G + warp] = m;
+      }
+      __syncthreads();
+      int ev = ev_acc;
+      {
+        const int sb = max(max(redi[kWarps * G], redi[kWarps * G + 1]), max(redi[kWarps * G + 2], redi[kWarps * G + 3]));
+        const float st = __half2float(__ushort_as_half(uint16_t(sb)));
+        int se = 0;
+        frexpf(st, &se);                             // st < 2^se
+        if (st > 0.0f) ev = 6 - se;
+      }
+      float alpha[G];
+      bool rescale = false;
 #pragma unroll
-      for (int mt = 0; mt < MTV; ++mt)
+      for (int g = 0; g < G; ++g) {
+        const float tmax = ord2f(max(max(redi[g], redi[G + g]), max(redi[2 * G + g], redi[3 * G + g])));
+        const float m_new = fmaxf(m_run[g], tmax);
+        alpha[g] = ex2(m_run[g] - m_new);
+        rescale |= (m_new != m_run[g]);
+        m_run[g] = m_new;
+        m_thr[g] = m_new + 8.0f;
+      }
+      if (rescale || ev != ev_acc) {                 // uniform across the CTA
+        const float f = ldexpf(1.0f, ev - ev_acc);
+        float ac0 = f, ac1 = f;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          oacc[mt][nt][0] *= ac0; oacc[mt][nt][1] *= ac1;
-          oacc[mt][nt][2] *= ac0; oacc[mt][nt][3] *= ac1;
+        for (int j = 0; j < GP; ++j) {
+          const f32x2 a2 = pk2(alpha[2 * j], alpha[min(2 * j + 1, G - 1)]);
+          lsum2[j] = fmul2(lsum2[j], a2);
+#pragma unroll
+          for (int k = 0; k < NG; ++k) pz2[j][k] = fmul2(pz2[j][k], a2);
         }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          if (g == hc0) ac0 = alpha[g] * f;
+          if (g == hc1) ac1 = alpha[g] * f;
+        }
+        ev_acc = ev;
+        vmul = ldexpf(1.0f, ev);
+        const int e = 6 - ev;                        // s_thr = fp16 bits of 2^e
+        s_thr = (e > 15) ? 0x8000u : (e >= -14) ? uint32_t(e + 15) << 10 : (e >= -24) ? 1u << (e + 24) : 0u;
+#pragma unroll
+        for (int mt = 0; mt < MTV; ++mt)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            oacc[mt][nt][0] *= ac0; oacc[mt][nt][1] *= ac1;
+            oacc[mt][nt][2] *= ac0; oacc[mt][nt][3] *= ac1;
+          }
+      }
     }
     // ---- probabilities; p s_v as (hi, lo) fp16 columns per group; sum p z_v
     {
-      const float vmul = ldexpf(1.0f, ev);
-      float pr[G];
+      f32x2 pr2[GP];
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        pr[g] = (t < n) ? exp2f(lg[g] - m_run[g]) : 0.0f;
-        lsum[g] += pr[g];
+      for (int j = 0; j < GP; ++j) {
+        const float p0 = ex2(lg[2 * j] - m_run[2 * j]);                      // 0 for t >= n
+        const int g1 = min(2 * j + 1, G - 1);
+        const float p1 = (2 * j + 1 < G) ? ex2(lg[g1] - m_run[g1]) : 0.0f;
+        pr2[j] = pk2(p0, p1);
+        lsum2[j] = fadd2(lsum2[j], pr2[j]);
       }
 #pragma unroll
       for (int k = 0; k < NG; ++k) {
         const uint32_t sz = vszr[k];                 // 0 for t >= n
         const float sv = __half2float(__ushort_as_half(uint16_t(sz & 0xffff))) * vmul;
         const float zv = __half2float(__ushort_as_half(uint16_t(sz >> 16)));
-        float w[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          w[g] = pr[g] * sv;
-          pz[g][k] = fmaf(pr[g], zv, pz[g][k]);
-        }
+        const f32x2 sv2 = pk2(sv, sv), zv2 = pk2(zv, zv);
         // columns as described for Cols: hi halves of the G heads, then lo halves
         uint32_t hw[NCOL / 2];
-        if constexpr (G >= 4) {
 #pragma unroll
-          for (int j = 0; j < G / 2; ++j) split_pair(w[2 * j], w[2 * j + 1], hw[j], hw[G / 2 + j]);
-        } else if constexpr (G == 2) {
-          split_pair(w[0], w[1], hw[0], hw[1]);
-          hw[2] = hw[3] = 0u;
-        } else {
-          uint32_t hi, lo;
-          split_pair(w[0], 0.0f, hi, lo);
-          hw[0] = (hi & 0xffffu) | (lo << 16);
-          hw[1] = hw[2] = hw[3] = 0u;
+        for (int i = 0; i < NCOL / 2; ++i) hw[i] = 0u;
+#pragma unroll
+        for (int j = 0; j < GP; ++j) {
+          pz2[j][k] = ffma2(pr2[j], zv2, pz2[j][k]);
+          const float2 w = up2(fmul2(pr2[j], sv2));
+          const __half2 hi = __floats2half2_rn(w.x, w.y);
+          const float2 hf = __half22float2(hi);
+          const float2 d = up2(fsub2(pk2(w.x, w.y), pk2(hf.x, hf.y)));
+          const __half2 lo = __floats2half2_rn(d.x, d.y);
+          const uint32_t hb = *reinterpret_cast<const uint32_t*>(&hi), lb = *reinterpret_cast<const uint32_t*>(&lo);
+          if constexpr (G == 1) {
+            hw[0] = (hb & 0xffffu) | (lb << 16);
+          } else {
+            hw[j] = hb;
+            hw[(G >= 4 ? G / 2 : 1) + j] = lb;
+          }
         }
         uint4* dst = reinterpret_cast<uint4*>(wt_s + (size_t(k) * kTile + t) * NCOL);
 #pragma unroll
@@ -723,10 +726,8 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
           }
 #pragma unroll
           for (int mt = 0; mt < MTV; ++mt) {
-            const uint32_t a[4] = {unpack_codes(__byte_perm(wa0[mt], wb0[mt], selv0), mv, scv, ofv),
-                                   unpack_codes(__byte_perm(wa0[mt], wb0[mt], selv1), mv, scv, ofv),
-                                   unpack_codes(__byte_perm(wa1[mt], wb1[mt], selv0), mv, scv, ofv),
-                                   unpack_codes(__byte_perm(wa1[mt], wb1[mt], selv1), mv, scv, ofv)};
+            const uint32_t a[4] = {__byte_perm(wa0[mt], wb0[mt], selv0) & mv, __byte_perm(wa0[mt], wb0[mt], selv1) & mv,
+                                   __byte_perm(wa1[mt], wb1[mt], selv0) & mv, __byte_perm(wa1[mt], wb1[mt], selv1) & mv};
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) mma16816(tacc[mt][nt], a, bw[nt][2 * kk], bw[nt][2 * kk + 1]);
           }
@@ -762,7 +763,7 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
   // over the owner threads (warp shuffles, then the 4 warps' partials)
   float* ofin = reinterpret_cast<float*>(smem);            // [G][D]
   float* zred = ofin + G * D;                               // [kWarps][G][NG]
-  const float vinv = ldexpf(1.0f, -ev_acc);
+  const float vinv = ldexpf(1.0f, 24 - 2 * cv - ev_acc);   // undoes 2^ev_acc and the codes' 4^cv 2^-24
 #pragma unroll
   for (int mt = 0; mt < MTV; ++mt) {
     const int c0 = (warp * MTV + mt) * 16 + gid;
@@ -772,12 +773,14 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
   for (int g = 0; g < G; ++g) {
 #pragma unroll
     for (int k = 0; k < NG; ++k) {
-      float z = pz[g][k];
+      const float2 zz = up2(pz2[g / 2][k]);
+      float z = (g & 1) ? zz.y : zz.x;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
       if (lane == 0) zred[(warp * G + g) * NG + k] = z;
     }
-    float l = lsum[g];
+    const float2 ll = up2(lsum2[g / 2]);
+    float l = (g & 1) ? ll.y : ll.x;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
     if (lane == 0) red[warp * G + g] = l;
