@@ -18,33 +18,30 @@
 //                 tables of the G query heads sharing the KV head (q in log2
 //                 units, q.mu_j for every centre, u = qP, per-group sums of q),
 //                 built while the first tile is in flight. Then 128-token tiles
-//                 of every packed stream arrive by cp.async (double-buffered)
-//                 and each tile takes three phases:
-//                   q.k   the sums  sum_{c in g} q_c code_c  on the tensor cores
-//                         (mma.sync m16n8k16, fp16 operands, fp32 accumulate):
-//                         A = codes (tokens x channels), B = q; one accumulator
-//                         per channel group, scaled by the token's s_g;
-//                   owner one thread per token adds the centre, zero and PSAC
-//                         terms, runs the online softmax and writes p_t s_t,g;
-//                   p.v   sum_t (p_t s_t,g) code_t,c on the tensor cores:
-//                         A = codes (channels x tokens), B = p s.
-//                 The fp32 operands q and p s enter the tensor cores as two fp16
-//                 halves (hi = fp16(x), lo = fp16(x - hi), about 22 significant
-//                 bits) placed in separate columns of the n8 tile, so G <= 4
-//                 heads fill one tile and 8 heads two; the two column sums are
-//                 added in fp32. q is scaled by a power of two per CTA so that
-//                 its halves stay normal fp16 numbers.
+//                 of every packed stream arrive by 1-D bulk copies (three
+//                 stages, one barrier each) and each tile takes three phases:
+//                   q.k   the sums  sum_{c in g} q_c code_c  as 8-bit integer
+//                         MMAs (mma.sync m16n8k32, A = codes as u8, B = q as
+//                         two signed 8-bit digits, exact int32), scaled by the
+//                         token's s_g; the zero-point and PSAC terms as fp16
+//                         k-steps (A = the token's z_g and a_i, B = hi/lo
+//                         halves of the query's group sums and qP);
+//                   owner one thread per token adds the centre term, runs the
+//                         online softmax and writes p_t s_t,g;
+//                   p.v   sum_t (p_t s_t,g) code_t,c on the tensor cores
+//                         (mma.sync m16n8k16): A = codes (channels x tokens),
+//                         B = p s as fp16 hi = fp16(x), lo = fp16(x - hi)
+//                         (about 22 significant bits) in separate columns of
+//                         the n8 tile, so G <= 4 heads fill one tile and 8
+//                         heads two; the two column sums are added in fp32.
 //   decode_combine log-sum-exp merge of the splits.
 //
-// Codes become fp16 operands with three integer/half instructions per pair
-// and no conversions: for a code sitting at bits 2i..2i+1 (i <= 3) of a 16-bit
-// half, (half & (3 << 2i)) | 0x6400 is the fp16 number 1024 + code * 4^i, and
-// one fp16 fma with 4^-i and -1024 * 4^-i gives the code exactly. For q.k a
-// quad of lanes takes the 16 channels of a code word as the pairs
-// (tig, 8+tig) of the word and (4+tig, 12+tig) of the word shifted right by 8
-// (tig = lane % 4), a fixed permutation of the contraction index that q's
-// operand follows. For p.v a byte permute puts the byte holding channel c of
-// two tokens into the two halves.
+// Codes become operands with one or two integer instructions per register.
+// q.k: (word >> 2 tig) & 0x03030303 puts four codes in the bytes of an 8-bit
+// operand (tig = lane % 4). p.v: a byte permute puts the byte holding channel
+// c of two tokens into the two halves; masking the code's two bits
+// (at bits 2i..2i+1, i <= 3) leaves the fp16 subnormal code * 4^i * 2^-24,
+// exact, and the constant factor is undone once when the sums are read out.
 #include <cfloat>
 
 #include "common.cuh"
@@ -100,10 +97,6 @@ __device__ __forceinline__ void mma16832_u8s8(int (&d)[4], const uint32_t (&a)[4
       "{%10,%10,%10,%10};\n"
       : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0));
-}
-// exact float of an integer |x| < 2^22 (magic-number conversion)
-__device__ __forceinline__ float small_int_to_float(int x) {
-  return __int_as_float(0x4B400000 + x) - 12582912.0f;
 }
 // four transposed 8x8 fp16 tiles; lane i gives the address of row i % 8 of tile i / 8
 __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], const void* row) {
@@ -488,9 +481,27 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
           w0[i] = x0.x; w0[i + 1] = x0.y; w0[i + 2] = x0.z; w0[i + 3] = x0.w;
           w1[i] = x1.x; w1[i + 1] = x1.y; w1[i + 2] = x1.z; w1[i + 3] = x1.w;
         }
+        // the two tokens' scale/zero words (all groups)
+        uint32_t sz0[NG], sz1[NG];
+        if constexpr (NG % 4 == 0) {
+#pragma unroll
+          for (int g = 0; g < NG; g += 4) {
+            const uint4 y0 = *reinterpret_cast<const uint4*>(ksz + t0 * NG + g);
+            const uint4 y1 = *reinterpret_cast<const uint4*>(ksz + t1 * NG + g);
+            sz0[g] = y0.x; sz0[g + 1] = y0.y; sz0[g + 2] = y0.z; sz0[g + 3] = y0.w;
+            sz1[g] = y1.x; sz1[g + 1] = y1.y; sz1[g + 2] = y1.z; sz1[g + 3] = y1.w;
+          }
+        } else {
+#pragma unroll
+          for (int g = 0; g < NG; ++g) {
+            sz0[g] = ksz[t0 * NG + g];
+            sz1[g] = ksz[t1 * NG + g];
+          }
+        }
         // sum_{c in g} code_c q_int,c per group: one 8-bit k-step (exact
-        // int32), scaled by the token's s_g (and once at the end by 1 / qmul);
-        // this lane's column pair is head 4 nt + tig (both digits)
+        // int32, |.| < 2^22, so its conversion is exact), scaled by the
+        // token's s_g (and once at the end by 1 / qmul); this lane's column
+        // pair is head 4 nt + tig (both digits)
         const uint32_t m8 = 0x03030303u;
         float L[NT][2];
 #pragma unroll
@@ -499,14 +510,14 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
         for (int g = 0; g < NG; ++g) {
           const uint32_t a[4] = {(w0[2 * g] >> (2 * tig)) & m8, (w1[2 * g] >> (2 * tig)) & m8,
                                  (w0[2 * g + 1] >> (2 * tig)) & m8, (w1[2 * g + 1] >> (2 * tig)) & m8};
-          const float s0 = __half2float(__ushort_as_half(uint16_t(ksz[t0 * NG + g] & 0xffff)));
-          const float s1 = __half2float(__ushort_as_half(uint16_t(ksz[t1 * NG + g] & 0xffff)));
+          const float s0 = __half2float(__ushort_as_half(uint16_t(sz0[g] & 0xffff)));
+          const float s1 = __half2float(__ushort_as_half(uint16_t(sz1[g] & 0xffff)));
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
             int C[4];
             mma16832_u8s8(C, a, bq8[nt][g][0], bq8[nt][g][1]);
-            L[nt][0] = fmaf(s0, small_int_to_float(C[0] + 256 * C[1]), L[nt][0]);
-            L[nt][1] = fmaf(s1, small_int_to_float(C[2] + 256 * C[3]), L[nt][1]);
+            L[nt][0] = fmaf(s0, __int2float_rn(C[0] + 256 * C[1]), L[nt][0]);
+            L[nt][1] = fmaf(s1, __int2float_rn(C[2] + 256 * C[3]), L[nt][1]);
           }
         }
         // zero-point and PSAC terms, sum_g z_g sigma_g + sum_i a_i u_i, as XK

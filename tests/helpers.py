@@ -1,6 +1,8 @@
 """Shared helpers of the parity tests (no method arithmetic here)."""
 from __future__ import annotations
 
+import os
+
 import numpy as np
 
 import workloads as wl
@@ -20,6 +22,8 @@ def assert_attention_close(got, ref, max_abs=2e-3, rel=1e-3, what=""):
     err = np.abs(got - ref).max() if got.size else 0.0
     r = rel_l2(got, ref) if got.size else 0.0
     assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    if os.environ.get("KV2_TEST_REPORT"):
+        print(f"[attention error] {what}: max-abs {err:.3e} rel-L2 {r:.3e}")
     assert err <= max_abs and r <= rel, f"{what}: max-abs {err:.3e} rel-L2 {r:.3e}"
     return err, r
 
