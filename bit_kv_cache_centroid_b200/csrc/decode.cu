@@ -36,12 +36,13 @@
 //                         heads two; the two column sums are added in fp32.
 //   decode_combine log-sum-exp merge of the splits.
 //
-// Codes become operands with one or two integer instructions per register.
-// q.k: (word >> 2 tig) & 0x03030303 puts four codes in the bytes of an 8-bit
-// operand (tig = lane % 4). p.v: a byte permute puts the byte holding channel
-// c of two tokens into the two halves; masking the code's two bits
-// (at bits 2i..2i+1, i <= 3) leaves the fp16 subnormal code * 4^i * 2^-24,
-// exact, and the constant factor is undone once when the sums are read out.
+// Codes become operands with few integer/half instructions and no
+// conversions. q.k: (word >> 2 tig) & 0x03030303 puts four codes in the bytes
+// of an 8-bit operand (tig = lane % 4). p.v: a byte permute puts the byte
+// holding channel c of two tokens into the two halves, and for a code at bits
+// 2i..2i+1 (i <= 3) of a half, (half & (3 << 2i)) | 0x6400 is the fp16 number
+// 1024 + code * 4^i; one fp16 fma with 4^-i and -1024 * 4^-i gives the code
+// exactly.
 #include <cfloat>
 
 #include "common.cuh"
@@ -76,6 +77,20 @@ struct SplitParams {
   int H_kv, H_q, M, r, cap, len, splits, tiles_per_split;
 };
 
+// d = a * b + c on two fp16 lanes
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+// two codes (at the bits of `mask` in each half of x) -> two exact fp16 codes:
+// (half & mask) | 0x6400 is the fp16 number 1024 + code * 4^i, and one fp16
+// fma with 4^-i and -1024 * 4^-i leaves the code. (Reading the masked bits as
+// fp16 subnormals, code * 4^i * 2^-24, would save the fma, but mma.sync then
+// measured about 9x the error of this form against the oracle.)
+__device__ __forceinline__ uint32_t unpack_codes(uint32_t x, uint32_t mask, uint32_t scale, uint32_t offset) {
+  return hfma2((x & mask) | 0x64006400u, scale, offset);
+}
 // d += A B, m16n8k16, fp16 operands, fp32 accumulators
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -420,10 +435,12 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
       }
     }
   }
-  // p.v code mask: this lane's channels sit at bits 2 cv..2 cv + 1 of a byte,
-  // and the masked half is the fp16 subnormal code * 4^cv * 2^-24 (exact)
+  // p.v code unpacking constants: this lane's channels sit at bits
+  // 2 cv..2 cv + 1 of a byte (fp16 4^-cv and -1024 * 4^-cv in both halves)
   const int cv = gid & 3;
   const uint32_t mv = (3u << (2 * cv)) | (3u << (16 + 2 * cv));
+  const uint32_t scv = 0x3C003C00u - 0x08000800u * uint32_t(cv);
+  const uint32_t ofv = 0xE400E400u - 0x08000800u * uint32_t(cv);
   const uint32_t selv0 = uint32_t(gid >> 2) | (uint32_t(4 + (gid >> 2)) << 8);       // channel gid
   const uint32_t selv1 = uint32_t(2 + (gid >> 2)) | (uint32_t(6 + (gid >> 2)) << 8);  // channel gid + 8
   // heads of this lane's two accumulator columns in p.v
@@ -433,7 +450,7 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
   constexpr int GP = (G + 1) / 2;
   float m_run[G], m_thr[G];   // running maximum and the bound m_run + 8 that forces a refresh
   f32x2 lsum2[GP], pz2[GP][NG];
-  float oacc[MTV][NT][4];     // p.v sums scaled by 2^ev_acc 2^-24 4^cv
+  float oacc[MTV][NT][4];     // p.v sums scaled by 2^ev_acc
   int ev_acc = 0;
   uint32_t s_thr = 0;         // fp16 bits of 2^(6 - ev_acc): |s_v| at or above it forces a refresh
   float vmul = 1.0f;          // 2^ev_acc
@@ -454,112 +471,178 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
 
   bool aborted = false;
   int tile = 0;
-  for (; tile < ntiles; ++tile) {
+  // Iteration `tile` runs the q.k of tile `tile` and the p.v of tile
+  // `tile - 1` (independent work in one barrier interval), then the owner
+  // phase of tile `tile`; one more iteration finishes the last p.v.
+  for (; tile <= ntiles; ++tile) {
+    const bool have = tile < ntiles;
     const int st = tile % kStages;
-    const bool ok = mbar_wait(bar0 + 8 * st, (tile / kStages) & 1, p.budget);
-    // (the barrier also tells that every thread is done with tile - 1)
+    const bool ok = !have || mbar_wait(bar0 + 8 * st, (tile / kStages) & 1, p.budget);
+    // (the barrier also orders the owner phase of tile - 1 before its p.v)
     if (__syncthreads_or(!ok)) {
       aborted = true;
       break;
     }
-    if (tid == 0) issue(tile + kStages - 1);   // into the stage tile - 1 used
     const unsigned char* cur = smem + st * stage;
-    const int n = min(kTile, t_end - (t_begin + tile * kTile));
+    const unsigned char* prv = smem + ((tile + kStages - 1) % kStages) * stage;
+    const int n = have ? min(kTile, t_end - (t_begin + tile * kTile)) : 0;
 
-    // ---- q.k on the tensor cores: warp w takes tokens 16 MTK w .. 16 MTK (w + 1) - 1
-    {
-      const uint32_t* kw = reinterpret_cast<const uint32_t*>(cur + Cfg::kc_off);
-      const uint32_t* ksz = reinterpret_cast<const uint32_t*>(cur + Cfg::ks_off);
+    if (have) {
+      // ---- q.k on the tensor cores: warp w takes tokens 16 MTK w .. 16 MTK (w + 1) - 1
+      {
+        const uint32_t* kw = reinterpret_cast<const uint32_t*>(cur + Cfg::kc_off);
+        const uint32_t* ksz = reinterpret_cast<const uint32_t*>(cur + Cfg::ks_off);
 #pragma unroll
-      for (int mt = 0; mt < MTK; ++mt) {
-        const int t0 = (warp * MTK + mt) * 16 + gid, t1 = t0 + 8;
-        uint32_t w0[NW], w1[NW];
+        for (int mt = 0; mt < MTK; ++mt) {
+          const int t0 = (warp * MTK + mt) * 16 + gid, t1 = t0 + 8;
+          uint32_t w0[NW], w1[NW];
 #pragma unroll
-        for (int i = 0; i < NW; i += 4) {
-          const uint4 x0 = *reinterpret_cast<const uint4*>(kw + t0 * NW + i);
-          const uint4 x1 = *reinterpret_cast<const uint4*>(kw + t1 * NW + i);
-          w0[i] = x0.x; w0[i + 1] = x0.y; w0[i + 2] = x0.z; w0[i + 3] = x0.w;
-          w1[i] = x1.x; w1[i + 1] = x1.y; w1[i + 2] = x1.z; w1[i + 3] = x1.w;
-        }
-        // the two tokens' scale/zero words (all groups)
-        uint32_t sz0[NG], sz1[NG];
-        if constexpr (NG % 4 == 0) {
-#pragma unroll
-          for (int g = 0; g < NG; g += 4) {
-            const uint4 y0 = *reinterpret_cast<const uint4*>(ksz + t0 * NG + g);
-            const uint4 y1 = *reinterpret_cast<const uint4*>(ksz + t1 * NG + g);
-            sz0[g] = y0.x; sz0[g + 1] = y0.y; sz0[g + 2] = y0.z; sz0[g + 3] = y0.w;
-            sz1[g] = y1.x; sz1[g + 1] = y1.y; sz1[g + 2] = y1.z; sz1[g + 3] = y1.w;
+          for (int i = 0; i < NW; i += 4) {
+            const uint4 x0 = *reinterpret_cast<const uint4*>(kw + t0 * NW + i);
+            const uint4 x1 = *reinterpret_cast<const uint4*>(kw + t1 * NW + i);
+            w0[i] = x0.x; w0[i + 1] = x0.y; w0[i + 2] = x0.z; w0[i + 3] = x0.w;
+            w1[i] = x1.x; w1[i + 1] = x1.y; w1[i + 2] = x1.z; w1[i + 3] = x1.w;
           }
-        } else {
+          // the two tokens' scale/zero words (all groups)
+          uint32_t sz0[NG], sz1[NG];
+          if constexpr (NG % 4 == 0) {
 #pragma unroll
-          for (int g = 0; g < NG; ++g) {
-            sz0[g] = ksz[t0 * NG + g];
-            sz1[g] = ksz[t1 * NG + g];
-          }
-        }
-        // sum_{c in g} code_c q_int,c per group: one 8-bit k-step (exact
-        // int32, |.| < 2^22, so its conversion is exact), scaled by the
-        // token's s_g (and once at the end by 1 / qmul); this lane's column
-        // pair is head 4 nt + tig (both digits)
-        const uint32_t m8 = 0x03030303u;
-        float L[NT][2];
+            for (int g = 0; g < NG; g += 4) {
+              const uint4 y0 = *reinterpret_cast<const uint4*>(ksz + t0 * NG + g);
+              const uint4 y1 = *reinterpret_cast<const uint4*>(ksz + t1 * NG + g);
+              sz0[g] = y0.x; sz0[g + 1] = y0.y; sz0[g + 2] = y0.z; sz0[g + 3] = y0.w;
+              sz1[g] = y1.x; sz1[g + 1] = y1.y; sz1[g + 2] = y1.z; sz1[g + 3] = y1.w;
+            }
+          } else {
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) L[nt][0] = L[nt][1] = 0.0f;
-#pragma unroll
-        for (int g = 0; g < NG; ++g) {
-          const uint32_t a[4] = {(w0[2 * g] >> (2 * tig)) & m8, (w1[2 * g] >> (2 * tig)) & m8,
-                                 (w0[2 * g + 1] >> (2 * tig)) & m8, (w1[2 * g + 1] >> (2 * tig)) & m8};
-          const float s0 = __half2float(__ushort_as_half(uint16_t(sz0[g] & 0xffff)));
-          const float s1 = __half2float(__ushort_as_half(uint16_t(sz1[g] & 0xffff)));
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            int C[4];
-            mma16832_u8s8(C, a, bq8[nt][g][0], bq8[nt][g][1]);
-            L[nt][0] = fmaf(s0, __int2float_rn(C[0] + 256 * C[1]), L[nt][0]);
-            L[nt][1] = fmaf(s1, __int2float_rn(C[2] + 256 * C[3]), L[nt][1]);
-          }
-        }
-        // zero-point and PSAC terms, sum_g z_g sigma_g + sum_i a_i u_i, as XK
-        // more k-steps over the columns (z_0 .. z_NG-1, a_0 .. a_r-1) of the
-        // token's scale/zero words and PSAC coefficients (exact fp16 values)
-        {
-          const uint32_t* kz0 = ksz + t0 * NG;
-          const uint32_t* kz1 = ksz + t1 * NG;
-          const uint32_t* ps0 = reinterpret_cast<const uint32_t*>(cur + Cfg::ps_off) + t0 * (r / 2);
-          const uint32_t* ps1 = reinterpret_cast<const uint32_t*>(cur + Cfg::ps_off) + t1 * (r / 2);
-          auto aux_pair = [&](const uint32_t* kz, const uint32_t* ps, int c) -> uint32_t {
-            if (c < NG) return __byte_perm(kz[c], kz[c + 1], 0x7632);   // z_c, z_c+1
-            return (c - NG < r) ? ps[(c - NG) >> 1] : 0u;               // a pair
-          };
-          float Ca[NT][4];
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) Ca[nt][i] = 0.0f;
-          for (int x = 0; x < XK; ++x) {
-            const int c = 16 * x + 2 * tig;
-            const uint32_t a[4] = {aux_pair(kz0, ps0, c), aux_pair(kz1, ps1, c),
-                                   aux_pair(kz0, ps0, c + 8), aux_pair(kz1, ps1, c + 8)};
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-              const uint2 bb = baux[(x * NT + nt) * 32 + lane];
-              mma16816(Ca[nt], a, bb.x, bb.y);
+            for (int g = 0; g < NG; ++g) {
+              sz0[g] = ksz[t0 * NG + g];
+              sz1[g] = ksz[t1 * NG + g];
             }
           }
-          // (columns 2 tig, 2 tig + 1: hi and lo part of head 4 nt + tig)
+          // sum_{c in g} code_c q_int,c per group: one 8-bit k-step (exact
+          // int32, |.| < 2^22, so its conversion is exact), scaled by the
+          // token's s_g (and once at the end by 1 / qmul); this lane's column
+          // pair is head 4 nt + tig (both digits)
+          const uint32_t m8 = 0x03030303u;
+          float L[NT][2];
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const int hd = 4 * nt + tig;
-            if (hd < G) {
-              lg_s[t0 * LS + hd] = fmaf(L[nt][0], qinv, (Ca[nt][0] + Ca[nt][1]) * ainv);
-              lg_s[t1 * LS + hd] = fmaf(L[nt][1], qinv, (Ca[nt][2] + Ca[nt][3]) * ainv);
+          for (int nt = 0; nt < NT; ++nt) L[nt][0] = L[nt][1] = 0.0f;
+#pragma unroll
+          for (int g = 0; g < NG; ++g) {
+            const uint32_t a[4] = {(w0[2 * g] >> (2 * tig)) & m8, (w1[2 * g] >> (2 * tig)) & m8,
+                                   (w0[2 * g + 1] >> (2 * tig)) & m8, (w1[2 * g + 1] >> (2 * tig)) & m8};
+            const float s0 = __half2float(__ushort_as_half(uint16_t(sz0[g] & 0xffff)));
+            const float s1 = __half2float(__ushort_as_half(uint16_t(sz1[g] & 0xffff)));
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              int C[4];
+              mma16832_u8s8(C, a, bq8[nt][g][0], bq8[nt][g][1]);
+              L[nt][0] = fmaf(s0, __int2float_rn(C[0] + 256 * C[1]), L[nt][0]);
+              L[nt][1] = fmaf(s1, __int2float_rn(C[2] + 256 * C[3]), L[nt][1]);
+            }
+          }
+          // zero-point and PSAC terms, sum_g z_g sigma_g + sum_i a_i u_i, as XK
+          // more k-steps over the columns (z_0 .. z_NG-1, a_0 .. a_r-1) of the
+          // token's scale/zero words and PSAC coefficients (exact fp16 values)
+          {
+            const uint32_t* kz0 = ksz + t0 * NG;
+            const uint32_t* kz1 = ksz + t1 * NG;
+            const uint32_t* ps0 = reinterpret_cast<const uint32_t*>(cur + Cfg::ps_off) + t0 * (r / 2);
+            const uint32_t* ps1 = reinterpret_cast<const uint32_t*>(cur + Cfg::ps_off) + t1 * (r / 2);
+            auto aux_pair = [&](const uint32_t* kz, const uint32_t* ps, int c) -> uint32_t {
+              if (c < NG) return __byte_perm(kz[c], kz[c + 1], 0x7632);   // z_c, z_c+1
+              return (c - NG < r) ? ps[(c - NG) >> 1] : 0u;               // a pair
+            };
+            float Ca[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+              for (int i = 0; i < 4; ++i) Ca[nt][i] = 0.0f;
+            for (int x = 0; x < XK; ++x) {
+              const int c = 16 * x + 2 * tig;
+              const uint32_t a[4] = {aux_pair(kz0, ps0, c), aux_pair(kz1, ps1, c),
+                                     aux_pair(kz0, ps0, c + 8), aux_pair(kz1, ps1, c + 8)};
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) {
+                const uint2 bb = baux[(x * NT + nt) * 32 + lane];
+                mma16816(Ca[nt], a, bb.x, bb.y);
+              }
+            }
+            // (columns 2 tig, 2 tig + 1: hi and lo part of head 4 nt + tig)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              const int hd = 4 * nt + tig;
+              if (hd < G) {
+                lg_s[t0 * LS + hd] = fmaf(L[nt][0], qinv, (Ca[nt][0] + Ca[nt][1]) * ainv);
+                lg_s[t1 * LS + hd] = fmaf(L[nt][1], qinv, (Ca[nt][2] + Ca[nt][3]) * ainv);
+              }
             }
           }
         }
       }
     }
-    __syncthreads();
+    if (tile > 0) {
+      // ---- p.v on the tensor cores: warp w takes code words (16-channel
+      // m-tiles) MTV w .. MTV (w + 1) - 1, all in channel group MTV w / 2. The
+      // tile's sums start from zero and join the running sums in fp32 (the
+      // tensor cores' accumulation truncates, and carried over a whole split
+      // its bias would show through the cancellation of code and zero terms).
+      {
+        float tacc[MTV][NT][4];
+#pragma unroll
+        for (int mt = 0; mt < MTV; ++mt)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) tacc[mt][nt][i] = 0.0f;
+        const uint32_t* vw = reinterpret_cast<const uint32_t*>(prv + Cfg::vc_off);
+        const int wi0 = warp * MTV;
+        const uint16_t* wt_g = wt_s + size_t(wi0 / 2) * kTile * NCOL;
+#pragma unroll
+        for (int ks2 = 0; ks2 < kTile / 32; ++ks2) {
+          uint32_t bw[NT][4];
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) ldmatrix_x4_trans(bw[nt], wt_g + (32 * ks2 + lane) * NCOL + 8 * nt);
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            const int ta = 32 * ks2 + 16 * kk + 2 * tig;
+            uint32_t wa0[MTV], wb0[MTV], wa1[MTV], wb1[MTV];
+            if constexpr (MTV == 2) {
+              const uint2 x0 = *reinterpret_cast<const uint2*>(vw + ta * NW + wi0);
+              const uint2 x1 = *reinterpret_cast<const uint2*>(vw + (ta + 1) * NW + wi0);
+              const uint2 x2 = *reinterpret_cast<const uint2*>(vw + (ta + 8) * NW + wi0);
+              const uint2 x3 = *reinterpret_cast<const uint2*>(vw + (ta + 9) * NW + wi0);
+              wa0[0] = x0.x; wa0[1] = x0.y; wb0[0] = x1.x; wb0[1] = x1.y;
+              wa1[0] = x2.x; wa1[1] = x2.y; wb1[0] = x3.x; wb1[1] = x3.y;
+            } else {
+              wa0[0] = vw[ta * NW + wi0];
+              wb0[0] = vw[(ta + 1) * NW + wi0];
+              wa1[0] = vw[(ta + 8) * NW + wi0];
+              wb1[0] = vw[(ta + 9) * NW + wi0];
+            }
+#pragma unroll
+            for (int mt = 0; mt < MTV; ++mt) {
+              const uint32_t a[4] = {unpack_codes(__byte_perm(wa0[mt], wb0[mt], selv0), mv, scv, ofv),
+                                     unpack_codes(__byte_perm(wa0[mt], wb0[mt], selv1), mv, scv, ofv),
+                                     unpack_codes(__byte_perm(wa1[mt], wb1[mt], selv0), mv, scv, ofv),
+                                     unpack_codes(__byte_perm(wa1[mt], wb1[mt], selv1), mv, scv, ofv)};
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) mma16816(tacc[mt][nt], a, bw[nt][2 * kk], bw[nt][2 * kk + 1]);
+            }
+          }
+        }
+#pragma unroll
+        for (int mt = 0; mt < MTV; ++mt)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) oacc[mt][nt][i] += tacc[mt][nt][i];
+      }
+    }
+    if (!have) break;
+    __syncthreads();   // lg complete; the p.v of tile - 1 is done with its stage and wt
+    if (tid == 0) issue(tile + kStages - 1);   // into the stage of tile - 1
 
     // ---- owner phase (thread = token): the centre term, online softmax
     const int t = tid;
@@ -695,64 +778,8 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
         for (int q4 = 0; q4 < NT; ++q4) dst[q4] = make_uint4(hw[4 * q4], hw[4 * q4 + 1], hw[4 * q4 + 2], hw[4 * q4 + 3]);
       }
     }
-    __syncthreads();
-
-    // ---- p.v on the tensor cores: warp w takes code words (16-channel
-    // m-tiles) MTV w .. MTV (w + 1) - 1, all in channel group MTV w / 2. The
-    // tile's sums start from zero and join the running sums in fp32 (the
-    // tensor cores' accumulation truncates, and carried over a whole split
-    // its bias would show through the cancellation of code and zero terms).
-    {
-      float tacc[MTV][NT][4];
-#pragma unroll
-      for (int mt = 0; mt < MTV; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) tacc[mt][nt][i] = 0.0f;
-      const uint32_t* vw = reinterpret_cast<const uint32_t*>(cur + Cfg::vc_off);
-      const int wi0 = warp * MTV;
-      const uint16_t* wt_g = wt_s + size_t(wi0 / 2) * kTile * NCOL;
-#pragma unroll
-      for (int ks2 = 0; ks2 < kTile / 32; ++ks2) {
-        uint32_t bw[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) ldmatrix_x4_trans(bw[nt], wt_g + (32 * ks2 + lane) * NCOL + 8 * nt);
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-          const int ta = 32 * ks2 + 16 * kk + 2 * tig;
-          uint32_t wa0[MTV], wb0[MTV], wa1[MTV], wb1[MTV];
-          if constexpr (MTV == 2) {
-            const uint2 x0 = *reinterpret_cast<const uint2*>(vw + ta * NW + wi0);
-            const uint2 x1 = *reinterpret_cast<const uint2*>(vw + (ta + 1) * NW + wi0);
-            const uint2 x2 = *reinterpret_cast<const uint2*>(vw + (ta + 8) * NW + wi0);
-            const uint2 x3 = *reinterpret_cast<const uint2*>(vw + (ta + 9) * NW + wi0);
-            wa0[0] = x0.x; wa0[1] = x0.y; wb0[0] = x1.x; wb0[1] = x1.y;
-            wa1[0] = x2.x; wa1[1] = x2.y; wb1[0] = x3.x; wb1[1] = x3.y;
-          } else {
-            wa0[0] = vw[ta * NW + wi0];
-            wb0[0] = vw[(ta + 1) * NW + wi0];
-            wa1[0] = vw[(ta + 8) * NW + wi0];
-            wb1[0] = vw[(ta + 9) * NW + wi0];
-          }
-#pragma unroll
-          for (int mt = 0; mt < MTV; ++mt) {
-            const uint32_t a[4] = {__byte_perm(wa0[mt], wb0[mt], selv0) & mv, __byte_perm(wa0[mt], wb0[mt], selv1) & mv,
-                                   __byte_perm(wa1[mt], wb1[mt], selv0) & mv, __byte_perm(wa1[mt], wb1[mt], selv1) & mv};
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma16816(tacc[mt][nt], a, bw[nt][2 * kk], bw[nt][2 * kk + 1]);
-          }
-        }
-      }
-#pragma unroll
-      for (int mt = 0; mt < MTV; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) oacc[mt][nt][i] += tacc[mt][nt][i];
-    }
-    // no barrier here: the next tile's first barrier orders these reads before
-    // the copy into this stage and the next writes of lg / wt
+    // no barrier here: the next iteration's first barrier orders the writes
+    // of wt before the p.v that reads them
   }
   if (aborted) {
     // a tile's copies did not arrive within the budget: report it, let the
@@ -774,7 +801,7 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
   // over the owner threads (warp shuffles, then the 4 warps' partials)
   float* ofin = reinterpret_cast<float*>(smem);            // [G][D]
   float* zred = ofin + G * D;                               // [kWarps][G][NG]
-  const float vinv = ldexpf(1.0f, 24 - 2 * cv - ev_acc);   // undoes 2^ev_acc and the codes' 4^cv 2^-24
+  const float vinv = ldexpf(1.0f, -ev_acc);
 #pragma unroll
   for (int mt = 0; mt < MTV; ++mt) {
     const int c0 = (warp * MTV + mt) * 16 + gid;
