@@ -781,6 +781,9 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
     // no barrier here: the next iteration's first barrier orders the writes
     // of wt before the p.v that reads them
   }
+  // the merge kernel (this grid's programmatic dependent) may be scheduled
+  // now; it waits for this grid's completion before reading the partials
+  asm volatile("griddepcontrol.launch_dependents;");
   if (aborted) {
     // a tile's copies did not arrive within the budget: report it, let the
     // copies still in flight land (bounded), and poison this split's output
@@ -844,29 +847,46 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
 // ---------------------------------------------------------------------------
 __global__ void decode_combine(const float* __restrict__ part, int H_q, int H_kv, int D,
                                int splits, void* out, int out_dtype) {
+  // launched as the split kernel's programmatic dependent: its partials are
+  // complete and visible after this wait
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int bq = blockIdx.x;
   const int b = bq / H_q, hq = bq % H_q;
   const int G = H_q / H_kv, h = hq / G, g = hq % G;
   const float* base = part + (size_t(b * H_kv + h) * splits) * G * (D + 2) + g * (D + 2);
   const size_t sstride = size_t(G) * (D + 2);
+  const int c = threadIdx.x, lane = c & 31;          // one thread per channel (blockDim = D)
+  // lane s of every warp reads split s (32 at a time): the overall maximum
   float m = -FLT_MAX;
-  for (int s = 0; s < splits; ++s) {
-    const float l = base[s * sstride + D + 1];
-    if (l > 0.0f) m = fmaxf(m, base[s * sstride + D]);
+  for (int s0 = 0; s0 < splits; s0 += 32) {
+    const int sp = s0 + lane;
+    if (sp < splits && base[sp * sstride + D + 1] > 0.0f) m = fmaxf(m, base[sp * sstride + D]);
   }
-  for (int c = threadIdx.x; c < D; c += blockDim.x) {
-    float o = 0.0f, l = 0.0f;
-    for (int s = 0; s < splits; ++s) {
-      const float ls = base[s * sstride + D + 1];
-      if (!(ls > 0.0f)) continue;
-      const float f = exp2f(base[s * sstride + D] - m);
-      o = fmaf(f, base[s * sstride + c], o);
-      l = fmaf(f, ls, l);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  // weights 2^(m_s - m) per split (0 for an empty split), shared by shuffles;
+  // the channel sums' loads are independent of one another
+  float o = 0.0f, l = 0.0f;
+  for (int s0 = 0; s0 < splits; s0 += 32) {
+    const int sp = s0 + lane;
+    float f = 0.0f;
+    if (sp < splits) {
+      const float ls = base[sp * sstride + D + 1];
+      if (ls > 0.0f) {
+        f = exp2f(base[sp * sstride + D] - m);
+        l = fmaf(f, ls, l);
+      }
     }
-    const float v = (l > 0.0f) ? o / l : 0.0f;
-    if (out_dtype == KV2_OUT_F32) static_cast<float*>(out)[size_t(bq) * D + c] = v;
-    else static_cast<__nv_bfloat16*>(out)[size_t(bq) * D + c] = __float2bfloat16_rn(v);
+    const int ns = min(32, splits - s0);
+    const float* col = base + size_t(s0) * sstride + c;
+#pragma unroll 8
+    for (int j = 0; j < ns; ++j) o = fmaf(__shfl_sync(0xffffffffu, f, j), col[j * sstride], o);
   }
+#pragma unroll
+  for (int k = 16; k > 0; k >>= 1) l += __shfl_xor_sync(0xffffffffu, l, k);
+  const float v = (l > 0.0f) ? o / l : 0.0f;
+  if (out_dtype == KV2_OUT_F32) static_cast<float*>(out)[size_t(bq) * D + c] = v;
+  else static_cast<__nv_bfloat16*>(out)[size_t(bq) * D + c] = __float2bfloat16_rn(v);
 }
 
 template <int D, int G, bool U16>
@@ -988,8 +1008,19 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   if (c.d == 64) e = (c.M > 256) ? launch_g<64, true>(G, sp, c.B, s) : launch_g<64, false>(G, sp, c.B, s);
   else e = (c.M > 256) ? launch_g<128, true>(G, sp, c.B, s) : launch_g<128, false>(G, sp, c.B, s);
   if (e != cudaSuccess) return e;
-  decode_combine<<<c.B * a.H_q, 128, 0, s>>>(part, a.H_q, c.H_kv, c.d, splits, a.out, a.out_dtype);
-  return cudaGetLastError();
+  // the merge runs as the split kernel's programmatic dependent (its launch
+  // overlaps the split kernel's last CTAs)
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(c.B * a.H_q);
+  cfg.blockDim = dim3(c.d);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_combine, static_cast<const float*>(part), a.H_q, c.H_kv, c.d, splits,
+                            a.out, a.out_dtype);
 }
 
 }  // namespace kv2
