@@ -484,6 +484,12 @@ cudaError_t launch_cfg(const QuantizeArgs& a, cudaStream_t s) {
   auto kern = quantize_kernel<D, CPL, KPT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
+  // the SM's shared-memory split as large as the attention kernels': an SM
+  // changes its split only when idle, so with a smaller one the attention
+  // CTAs launched beside this kernel (as its programmatic dependents) could
+  // not start on its SMs until it exits
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, int(cudaSharedmemCarveoutMaxShared));
+  if (e != cudaSuccess) return e;
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem) != cudaSuccess || per_sm < 1)
     per_sm = 1;
