@@ -8,10 +8,12 @@
 // block-causal by latent frame. Thousands of queries per call make Q K^T and
 // P V dense contractions, so they run on tcgen05.mma:
 //
-//   S  = Q . Khat^T           bf16 x bf16, Khat = bf16(fmaf(code, s, z) + mu[idx])
+//   S  = Q . Khat^T           fp16 x fp16, Khat = fp16(code s + fp16(z + mu[idx]))
+//                             (Q scaled per row by a power of two, undone in
+//                             the softmax)
 //      + U . A^T              fp16 x fp16, U = fp16(q P), A = the stored fp16
 //                             PSAC coefficients (K = 16 extra contraction columns)
-//   O += P . Vhat             fp16 x fp16, Vhat = fp16(fmaf(code, s, z)), P = fp16
+//   O += P . Vhat             fp16 x fp16, Vhat = fp16(code s + z), P = fp16
 //
 // One CTA (17 warps) serves two 128-query tiles of one (batch, query head);
 // every dequantized key/value tile feeds both. Warp roles:
@@ -19,8 +21,8 @@
 //                   S from TMEM, online softmax, P written back into the S
 //                   columns as fp16 pairs, O rescaled in TMEM when a row max grows;
 //   warps 8-15      producer (two threads per key row, 64 channels each):
-//                   packed key/value tiles -> 128-byte-swizzled bf16 Khat /
-//                   fp16 Vhat / fp16 PSAC tiles in a 2-stage ring;
+//                   packed key/value tiles -> 128-byte-swizzled fp16 Khat /
+//                   Vhat and PSAC tiles in a 2-stage ring (fp16x2 arithmetic);
 //   warp 16         issues the MMAs (one thread) and owns the TMEM allocation.
 // TMEM (512 columns): S0, S1, O0, O1. The PV MMA reads P straight from TMEM.
 // mbarriers: kv_full/kv_empty (ring), s_full, p_full, o_done (per query tile).
@@ -87,7 +89,7 @@ constexpr uint32_t kLayoutNone = 0, kLayoutSW128 = 2;
 constexpr uint32_t make_idesc(uint32_t a_fmt, uint32_t b_fmt, uint32_t b_mn_major, uint32_t N, uint32_t M) {
   return (1u << 4) | (a_fmt << 7) | (b_fmt << 10) | (b_mn_major << 16) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
-constexpr uint32_t IDESC_QK = make_idesc(1, 1, 0, kKeys, kRows);
+constexpr uint32_t IDESC_QK = make_idesc(0, 0, 0, kKeys, kRows);
 constexpr uint32_t IDESC_UA = make_idesc(0, 0, 0, kKeys, kRows);
 constexpr uint32_t IDESC_PV = make_idesc(0, 0, 1, kD, kRows);
 
@@ -226,18 +228,35 @@ __device__ __forceinline__ uint32_t pack_f16(float a, float b) {
 }
 
 
-// codes at bit positions 4i and 4i+2 of a 16-bit code field as the float pair
-// {code * 4^(2i), code * 4^(2i+1)}, exact ((w & m) | 0x4B000000 is 2^23 + code * 4^j)
-__device__ __forceinline__ f32x2 code_pair_x4j(uint32_t w, int i) {
-  const unsigned long long ww = (static_cast<unsigned long long>(w) << 32) | w;
-  const unsigned long long m =
-      (static_cast<unsigned long long>(3u << (4 * i + 2)) << 32) | static_cast<unsigned long long>(3u << (4 * i));
-  f32x2 bits;
-  asm("{\n\t.reg .b64 t;\n\tand.b64 t, %1, %2;\n\tor.b64 %0, t, 0x4B0000004B000000;\n\t}\n"
-      : "=l"(bits) : "l"(ww), "l"(m));
-  f32x2 d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(bits), "l"(0x4B0000004B000000ull));
+// d = a * b + c on two fp16 lanes; d = a + b
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
+}
+__device__ __forceinline__ uint32_t hadd2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// The codes of channels 2i, 2i+1 of an 8-channel chunk sit at bits 4i and
+// 4i+2 of its 16-bit code field. With the field in both halves of x (and x
+// shifted right by 8 for i >= 2), (x & mask) | 0x6400 puts the fp16 numbers
+// 1024 + code * 16^i' in the low half and 1024 + 4 code * 16^i' in the high
+// half (i' = i mod 2, bits within the fp16 mantissa); one fp16 fma with the
+// exact constants below leaves the two codes (exact small integers).
+__device__ __forceinline__ uint32_t code_pair_f16(uint32_t x, uint32_t x8, int i) {
+  const uint32_t src = (i < 2) ? x : x8;
+  const int ip = i & 1;
+  const uint32_t mask = (3u << (4 * ip)) | (3u << (16 + 4 * ip + 2));
+  const uint32_t scale = ip ? 0x24002C00u : 0x34003C00u;    // {1/16, 1/64} : {1, 1/4}
+  const uint32_t offset = ip ? 0xCC00D400u : 0xDC00E400u;   // {-64, -16} : {-1024, -256}
+  return hfma2((src & mask) | 0x64006400u, scale, offset);
+}
+// the 16-bit code field `lc & 1` of word w in both halves of a word
+__device__ __forceinline__ uint32_t field_both(uint32_t w, int lc) {
+  return __byte_perm(w, 0u, (lc & 1) ? 0x3232u : 0x1010u);
 }
 
 struct ChunkParams {
@@ -295,46 +314,31 @@ __device__ __forceinline__ void load_psac(const ChunkParams& p, size_t slot, uin
   if (p.r >= 16) a1 = *reinterpret_cast<const uint4*>(p.psac + slot * p.r + 8);
 }
 
-// half a Khat (bf16) row and half a Vhat (fp16) row from the packed fields and
-// the centroid half-row m4; half 0 also writes the PSAC row
+// half a Khat row and half a Vhat row (both fp16) from the packed fields and
+// the centroid half-row m4; half 0 also writes the PSAC row. In fp16
+// arithmetic: Khat = fma(code, s, z + mu), Vhat = fma(code, s, z), codes exact.
 __device__ void dequant_cache_half(const RawHalf& r, const uint4 (&m4)[8], const uint4& a0, const uint4& a1, int row,
                                    int half, uint8_t* stage) {
   const uint32_t kw[4] = {r.kw.x, r.kw.y, r.kw.z, r.kw.w};
   const uint32_t vw[4] = {r.vw.x, r.vw.y, r.vw.z, r.vw.w};
   const uint32_t ksz[2] = {r.ksz.x, r.ksz.y};
   const uint32_t vsz[2] = {r.vsz.x, r.vsz.y};
-  // fmaf(code, s, z) with the code read as code * 4^j: the scale carries 4^-j
-  // (exact power-of-two scaling), so the product and its single rounding are
-  // those of fmaf(code, s, z).
 #pragma unroll
   for (int g = 0; g < 2; ++g) {
-    const float ks = __half2float(__ushort_as_half(uint16_t(ksz[g] & 0xffff)));
-    const float vs = __half2float(__ushort_as_half(uint16_t(vsz[g] & 0xffff)));
-    const float kz = __half2float(__ushort_as_half(uint16_t(ksz[g] >> 16)));
-    const float vz = __half2float(__ushort_as_half(uint16_t(vsz[g] >> 16)));
-    f32x2 ksc[4], vsc[4];                           // {s 4^-2i, s 4^-(2i+1)}
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float e0 = __uint_as_float(uint32_t(127 - 4 * i) << 23), e1 = __uint_as_float(uint32_t(125 - 4 * i) << 23);
-      ksc[i] = pk2(ks * e0, ks * e1);
-      vsc[i] = pk2(vs * e0, vs * e1);
-    }
-    const f32x2 kz2 = pk2(kz, kz), vz2 = pk2(vz, vz);
+    const uint32_t ks2 = __byte_perm(ksz[g], 0u, 0x1010u), kz2 = __byte_perm(ksz[g], 0u, 0x3232u);
+    const uint32_t vs2 = __byte_perm(vsz[g], 0u, 0x1010u), vz2 = __byte_perm(vsz[g], 0u, 0x3232u);
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {                // 8 channels per chunk
       const int c16 = half * 8 + g * 4 + cc;         // chunk index within the row
       const int lc = g * 4 + cc;                      // chunk index within this half
-      const __half2* mh = reinterpret_cast<const __half2*>(&m4[lc]);
-      const uint32_t kword = (kw[lc >> 1] >> ((lc & 1) * 16)) & 0xffffu;
-      const uint32_t vword = (vw[lc >> 1] >> ((lc & 1) * 16)) & 0xffffu;
+      const uint32_t mu[4] = {m4[lc].x, m4[lc].y, m4[lc].z, m4[lc].w};
+      const uint32_t kx = field_both(kw[lc >> 1], lc), vx = field_both(vw[lc >> 1], lc);
+      const uint32_t kx8 = kx >> 8, vx8 = vx >> 8;
       uint32_t kb[4], vb[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float2 m = __half22float2(mh[i]);
-        const float2 kf = up2(fadd2(ffma2(code_pair_x4j(kword, i), ksc[i], kz2), pk2(m.x, m.y)));
-        const float2 vf = up2(ffma2(code_pair_x4j(vword, i), vsc[i], vz2));
-        kb[i] = pack_bf16(kf.x, kf.y);
-        vb[i] = pack_f16(vf.x, vf.y);
+        kb[i] = hfma2(code_pair_f16(kx, kx8, i), ks2, hadd2(kz2, mu[i]));
+        vb[i] = hfma2(code_pair_f16(vx, vx8, i), vs2, vz2);
       }
       *reinterpret_cast<uint4*>(stage + ST_K + sw128_off(row, c16)) = make_uint4(kb[0], kb[1], kb[2], kb[3]);
       *reinterpret_cast<uint4*>(stage + ST_V + sw128_off(row, c16)) = make_uint4(vb[0], vb[1], vb[2], vb[3]);
@@ -346,20 +350,24 @@ __device__ void dequant_cache_half(const RawHalf& r, const uint4 (&m4)[8], const
   }
 }
 
-// chunk token -> half a Khat row (bf16 copy) and half a Vhat row (bf16 -> fp16)
+// eight bf16 values -> eight fp16 values (round to nearest even)
+__device__ __forceinline__ uint4 bf16x8_to_f16(const uint4& v) {
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) o[i] = pack_f16(__uint_as_float(u[i] << 16), __uint_as_float(u[i] & 0xffff0000u));
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// chunk token -> half a Khat row and half a Vhat row (bf16 -> fp16)
 __device__ void copy_self_half(const uint16_t* krow, const uint16_t* vrow, int row, int half, uint8_t* stage) {
   const uint4* k4 = reinterpret_cast<const uint4*>(krow) + half * 8;
   const uint4* v4 = reinterpret_cast<const uint4*>(vrow) + half * 8;
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     const int c16 = half * 8 + c;
-    *reinterpret_cast<uint4*>(stage + ST_K + sw128_off(row, c16)) = __ldg(k4 + c);
-    const uint4 v = __ldg(v4 + c);
-    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) o[i] = pack_f16(__uint_as_float(u[i] << 16), __uint_as_float(u[i] & 0xffff0000u));
-    *reinterpret_cast<uint4*>(stage + ST_V + sw128_off(row, c16)) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(stage + ST_K + sw128_off(row, c16)) = bf16x8_to_f16(__ldg(k4 + c));
+    *reinterpret_cast<uint4*>(stage + ST_V + sw128_off(row, c16)) = bf16x8_to_f16(__ldg(v4 + c));
   }
 }
 
@@ -406,21 +414,27 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
   }
   if (warp == kMmaWarp) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
 
-  // ---- Q tiles (bf16, SW128 K-major) and U = fp16(q P) (no swizzle, K = 16)
+  // ---- Q tiles (fp16, SW128 K-major) and U = fp16(q P) (no swizzle, K = 16),
+  // each row scaled by 2^qexp with max(|q|, |u|) 2^qexp below 2^15: fp16 range
+  // whatever the bf16 input (the bf16 -> fp16 conversion of q exact); the
+  // softmax thread of the row undoes the factor in its score scale
+  int qexp = 0;
   if (warp < 8) {
     const int x = warp >> 2, row = tid - x * kRows;
     const int qi = q0 + x * kRows + row;
     const bool q_ok = qi < p.Nq;
     uint8_t* qtile = smem + (x ? OFF_Q1 : OFF_Q0);
+    const uint4* src = reinterpret_cast<const uint4*>(p.Q + ((size_t(b) * p.Nq + min(qi, p.Nq - 1)) * p.H_q + hq) * kD);
+    uint32_t amax = 0;                                // largest |q| of the row, as bf16 bits in both halves
     float u[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) u[j] = 0.0f;
-    const uint4* src = reinterpret_cast<const uint4*>(p.Q + ((size_t(b) * p.Nq + min(qi, p.Nq - 1)) * p.H_q + hq) * kD);
     const float* Ph = p.P + size_t(h) * kD * p.r;
 #pragma unroll 1
     for (int c16 = 0; c16 < 16; ++c16) {
       const uint4 v = q_ok ? __ldg(src + c16) : make_uint4(0, 0, 0, 0);
-      *reinterpret_cast<uint4*>(qtile + sw128_off(row, c16)) = v;
+      amax = __vmaxu2(amax, __vmaxu2(__vmaxu2(v.x & 0x7fff7fffu, v.y & 0x7fff7fffu),
+                                     __vmaxu2(v.z & 0x7fff7fffu, v.w & 0x7fff7fffu)));
       if (p.r > 0) {
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -433,9 +447,28 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
         }
       }
     }
+    float rmax = __uint_as_float(max(amax & 0xffffu, amax >> 16) << 16);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) rmax = fmaxf(rmax, fabsf(u[j]));
+    if (rmax > 0.0f && rmax < 1e30f) {
+      int e = 0;
+      frexpf(rmax, &e);                               // rmax < 2^e
+      qexp = min(max(15 - e, -64), 64);
+    }
+    const float qmul = ldexpf(1.0f, qexp);
+#pragma unroll 1
+    for (int c16 = 0; c16 < 16; ++c16) {
+      const uint4 v = q_ok ? __ldg(src + c16) : make_uint4(0, 0, 0, 0);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      uint32_t hq4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        hq4[i] = pack_f16(__uint_as_float(w[i] << 16) * qmul, __uint_as_float(w[i] & 0xffff0000u) * qmul);
+      *reinterpret_cast<uint4*>(qtile + sw128_off(row, c16)) = make_uint4(hq4[0], hq4[1], hq4[2], hq4[3]);
+    }
     uint32_t uw[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) uw[j] = pack_f16(u[2 * j], u[2 * j + 1]);
+    for (int j = 0; j < 8; ++j) uw[j] = pack_f16(u[2 * j] * qmul, u[2 * j + 1] * qmul);
     uint8_t* utile = smem + (x ? OFF_U1 : OFF_U0);
     *reinterpret_cast<uint4*>(utile + nosw_off(row, 0)) = make_uint4(uw[0], uw[1], uw[2], uw[3]);
     *reinterpret_cast<uint4*>(utile + nosw_off(row, 1)) = make_uint4(uw[4], uw[5], uw[6], uw[7]);
@@ -564,6 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + x * kKeys + lane_base, tO = tmem + 2 * kKeys + x * kD + lane_base;
     const int my_self_lim = min(self_len, (min(qi, p.Nq - 1) / p.F + 1) * p.F);
+    const float sc_row = p.scale_log2 * ldexpf(1.0f, -qexp);   // the row's Q carries 2^qexp
     float m_run = -INFINITY, l_run = 0.0f;
     bool done = true;
     for (int jj = 0; jj < nloc; ++jj) {
@@ -602,12 +636,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
       }
       const float mt = fmaxf(fmaxf(fmaxf(mpart[0], mpart[1]), fmaxf(mpart[2], mpart[3])),
                              fmaxf(fmaxf(mpart[4], mpart[5]), fmaxf(mpart[6], mpart[7])));
-      const float m_new = fmaxf(m_run, mt * p.scale_log2);
+      const float m_new = fmaxf(m_run, mt * sc_row);
       const float alpha = (m_new == -INFINITY) ? 1.0f : ex2(m_run - m_new);
       f32x2 spart[4];                                   // 8 partial sums as 4 pairs
 #pragma unroll
       for (int i = 0; i < 4; ++i) spart[i] = 0ull;
-      const f32x2 sc2 = pk2(p.scale_log2, p.scale_log2), nm2 = pk2(-m_new, -m_new);
+      const f32x2 sc2 = pk2(sc_row, sc_row), nm2 = pk2(-m_new, -m_new);
 #pragma unroll 1
       for (int c0 = 0; c0 < kKeys; c0 += 32) {
         float v[32];

@@ -115,6 +115,13 @@ float or_f32_from_bf16(uint16_t b)
     return f;
 }
 
+/* fp16 nearest-even rounding of an exact (double) value: one rounding, as an
+ * fp16 add or fused multiply-add performs it */
+static double f16_round(double x)
+{
+    return (double)or_f32_from_f16(f16_encode_exact(round_to_format(x, 10, -14, F16_MAX, RND_NEAREST_EVEN)));
+}
+
 uint16_t or_bf16_from_f32(float x)
 {
     if (isnan(x)) return 0x7fc0u;
@@ -491,7 +498,9 @@ static void dequant_exact(const or_cache* c, size_t slot, double* kh, double* vh
     }
 }
 
-/* operand-precision dequantized rows (chunk kernel precision) */
+/* operand-precision dequantized rows (chunk kernel precision): fp16
+ * arithmetic with one rounding per operation, Khat = fp16(code s + fp16(z + mu)),
+ * Vhat = fp16(code s + z) */
 static void dequant_operand(const or_cache* c, size_t slot, double* kh, double* vh)
 {
     int d = c->d, ng = d / GROUP;
@@ -501,15 +510,12 @@ static void dequant_operand(const or_cache* c, size_t slot, double* kh, double* 
     int h = (int)((slot / (size_t)c->cap) % (size_t)c->Hkv);
     for (int g = 0; g < ng; ++g) {
         uint32_t ks = c->k_sz[slot * ng + g], vs = c->v_sz[slot * ng + g];
-        float s = or_f32_from_f16((uint16_t)(ks & 0xffff)), z = or_f32_from_f16((uint16_t)(ks >> 16));
-        float sv = or_f32_from_f16((uint16_t)(vs & 0xffff)), zv = or_f32_from_f16((uint16_t)(vs >> 16));
+        double s = or_f32_from_f16((uint16_t)(ks & 0xffff)), z = or_f32_from_f16((uint16_t)(ks >> 16));
+        double sv = or_f32_from_f16((uint16_t)(vs & 0xffff)), zv = or_f32_from_f16((uint16_t)(vs >> 16));
         for (int ch = g * GROUP; ch < (g + 1) * GROUP; ++ch) {
-            float m = or_f32_from_f16(c->cent[((size_t)h * c->M + j) * d + ch]);
-            float kd = fmaf((float)code_at(kw, ch), s, z);
-            float k32 = kd + m;
-            kh[ch] = or_f32_from_bf16(or_bf16_from_f32(k32));
-            float vd = fmaf((float)code_at(vw, ch), sv, zv);
-            vh[ch] = or_f32_from_f16(or_f16_from_f32(vd, RND_NEAREST_EVEN));
+            double m = or_f32_from_f16(c->cent[((size_t)h * c->M + j) * d + ch]);
+            kh[ch] = f16_round((double)code_at(kw, ch) * s + f16_round(z + m));
+            vh[ch] = f16_round((double)code_at(vw, ch) * sv + zv);
         }
     }
 }
@@ -612,7 +618,7 @@ int or_chunk(int B, int Hkv, int d, int M, int r, int cap,
             const uint16_t* vr = Vself + (((size_t)b * Nq + j) * Hkv + h) * d;
             double acc = 0.0;
             for (int ch = 0; ch < d; ++ch) {
-                acc += q[ch] * (double)or_f32_from_bf16(kr[ch]);
+                acc += q[ch] * f16_round(or_f32_from_bf16(kr[ch]));
                 vals[n * d + ch] = or_f32_from_f16(or_f16_from_f32(or_f32_from_bf16(vr[ch]), RND_NEAREST_EVEN));
             }
             logit[n] = acc * sm_scale;

@@ -1,6 +1,7 @@
 """GPU parity of kv2_attention_chunk (tcgen05) against the fp64 oracle on the
-same packed cache and the kernel's operand precision (bf16 keys = bf16 of
-centre + residual, fp16 values, fp16 q P): max-abs 2e-3 and relative L2 1e-3
+same packed cache and the kernel's operand precision (fp16 keys =
+fp16(code s + fp16(z + centre)), fp16 values = fp16(code s + z), fp16 q P,
+self keys and values rounded to fp16): max-abs 2e-3 and relative L2 1e-3
 on the fp32 output, and the bf16 output against the bf16 rounding of the
 oracle. Also: the block-causal frame mask, empty cache, ragged tiles, and the
 bounded device-side wait that reports a timeout instead of hanging."""

@@ -175,7 +175,7 @@ def test_chunk_mask_and_dense_self_attention(orc):
 
 
 def test_chunk_cache_part_equals_decode_when_exact(orc):
-    """Cache values chosen so the chunk's bf16/fp16 operands are exact, and self
+    """Cache values chosen so the chunk's fp16 operands are exact, and self
     keys that no query can select: the chunk call reduces to decode."""
     s = wl.spec("tiny", T=48, Nq=8, frame_tokens=4, r=8)
     pc = wl.random_packed_cache(s, T=48)
