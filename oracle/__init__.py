@@ -72,8 +72,9 @@ def _declare(L):
     L.or_chunk.argtypes = ([_I] * 6 + [_P] * 8 + [_I, _P, _I, _I, _P, _P, _I,
                                                   ctypes.c_double, _P, _I, _P])
     L.or_decode_logits.argtypes = [_I] * 7 + [_P] * 6 + [_I, _P, _P]
+    L.or_fit_centroids.argtypes = [_I] * 5 + [_P, _P, _P, _I, _P, _P]
     for f in (L.or_codec_group, L.or_fit, L.or_quantize, L.or_decode, L.or_chunk,
-              L.or_decode_logits):
+              L.or_decode_logits, L.or_fit_centroids):
         f.restype = _I if f is not L.or_codec_group else None
 
 
@@ -178,6 +179,22 @@ def quantize(pc, K: np.ndarray, V: np.ndarray, pos: int, C: int, P: np.ndarray,
     if rc:
         raise ValueError("or_quantize: bad arguments")
     return dbg
+
+
+def fit_centroids(X: np.ndarray, M: int, C: int, w: np.ndarray, Wg: np.ndarray,
+                  centroids: np.ndarray, iters: int):
+    """QSAC-aware centre fitting (reading in ``kv2_oracle.c``): X bf16 bits
+    [n][H_kv][d], initial centres fp16 bits [H_kv][M][d] -> (fitted centres
+    fp16 bits [H_kv][M][d], last assignment int32 [n][H_kv])."""
+    X = _c(X, np.uint16)
+    n, Hkv, d = X.shape
+    cent = np.array(_c(centroids, np.uint16), copy=True)
+    assign = np.full((max(n, 1), Hkv), -1, np.int32)
+    rc = lib().or_fit_centroids(n, Hkv, d, M, C, _ptr(X), _ptr(_c(w, np.float32)), _ptr(_c(Wg, np.float32)),
+                                iters, _ptr(cent), _ptr(assign))
+    if rc:
+        raise ValueError("or_fit_centroids: bad arguments")
+    return cent, assign[:n]
 
 
 def _cache_args(pc):

@@ -312,6 +312,76 @@ int or_fit(const uint16_t* Qh, int n, int Hq, int Hkv, int d, int r,
 /* library: [B][Hkv][cap][...].                                              */
 /* ------------------------------------------------------------------------ */
 
+/* QSAC decision for one key k (fp32 [d]) of KV head h: returns the chosen
+ * centre and leaves its residual k - mu_j in xbest. mu [M][d], nrm [M] as
+ * above; scratch: score [M], cand [C], used [M], x [d]. Optional debug
+ * outputs (candidate ids, scores, E per candidate) when non-NULL. */
+static int qsac_choose(const float* k, const float* wh, const float* Wgh, const float* mu, const float* nrm,
+                       int M, int C, int d, float* wk, float* score, int* cand, char* used, float* x,
+                       float* xbest, int32_t* cand_out, float* score_out, float* E_out)
+{
+    int ng = d / GROUP;
+    for (int c = 0; c < d; ++c) wk[c] = wh[c] * k[c];
+    /* ranking */
+    for (int j = 0; j < M; ++j) {
+        float dot = 0.0f;
+        const float* m = mu + (size_t)j * d;
+        for (int c = 0; c < d; ++c) dot = fmaf(wk[c], m[c], dot);
+        score[j] = fmaf(-2.0f, dot, nrm[j]);
+    }
+    memset(used, 0, (size_t)M);
+    for (int i = 0; i < C; ++i) {
+        int best = -1;
+        for (int j = 0; j < M; ++j) {
+            if (used[j]) continue;
+            if (best < 0 || score[j] < score[best]) best = j;
+        }
+        used[best] = 1;
+        cand[i] = best;
+        if (cand_out) cand_out[i] = best;
+        if (score_out) score_out[i] = score[best];
+    }
+    /* choice by estimated perturbation */
+    int chosen = -1;
+    float bestE = 0.0f;
+    for (int i = 0; i < C; ++i) {
+        int j = cand[i];
+        const float* m = mu + (size_t)j * d;
+        for (int c = 0; c < d; ++c) x[c] = k[c] - m[c];
+        float E = 0.0f;
+        for (int g = 0; g < ng; ++g) {
+            uint16_t sb, zb;
+            codec_params(x + g * GROUP, GROUP, &sb, &zb);
+            float s = or_f32_from_f16(sb);
+            float ws = Wgh[g] * s;
+            E = fmaf(ws, s, E);
+        }
+        if (E_out) E_out[i] = E;
+        if (chosen < 0 || E < bestE) {
+            chosen = j;
+            bestE = E;
+            memcpy(xbest, x, (size_t)d * sizeof(float));
+        }
+    }
+    return chosen;
+}
+
+/* the centres of KV head h as fp32 and their weighted norms
+ * nrm_j = sum_c (w_c mu_jc) mu_jc (fp32 fmaf chain over ascending c) */
+static void qsac_tables(const uint16_t* cent, const float* wh, int h, int M, int d, float* mu, float* nrm)
+{
+    for (int j = 0; j < M; ++j) {
+        float acc = 0.0f;
+        for (int c = 0; c < d; ++c) {
+            float m = or_f32_from_f16(cent[((size_t)h * M + j) * d + c]);
+            mu[(size_t)j * d + c] = m;
+            float wm = wh[c] * m;
+            acc = fmaf(wm, m, acc);
+        }
+        nrm[j] = acc;
+    }
+}
+
 static uint32_t pack_word(const uint32_t* codes16)
 {
     uint32_t w = 0;
@@ -361,66 +431,16 @@ int or_quantize(int B, int Hkv, int d, int M, int r, int cap,
     char* used = (char*)malloc((size_t)M);
     for (int h = 0; h < Hkv; ++h) {
         const float* wh = w + (size_t)h * d;
-        for (int j = 0; j < M; ++j) {
-            float acc = 0.0f;
-            for (int c = 0; c < d; ++c) {
-                float m = or_f32_from_f16(cent[((size_t)h * M + j) * d + c]);
-                mu[(size_t)j * d + c] = m;
-                float wm = wh[c] * m;
-                acc = fmaf(wm, m, acc);
-            }
-            nrm[j] = acc;
-        }
+        qsac_tables(cent, wh, h, M, d, mu, nrm);
         for (int b = 0; b < B; ++b) {
             for (int t = 0; t < n_new; ++t) {
                 size_t in = (((size_t)b * n_new + t) * Hkv + h) * d;
                 size_t slot = ((size_t)b * Hkv + h) * cap + (size_t)(pos + t);
                 size_t dbg = (((size_t)b * n_new + t) * Hkv + h);
-                for (int c = 0; c < d; ++c) {
-                    k[c] = or_f32_from_bf16(K[in + c]);
-                    wk[c] = wh[c] * k[c];
-                }
-                /* ranking */
-                for (int j = 0; j < M; ++j) {
-                    float dot = 0.0f;
-                    const float* m = mu + (size_t)j * d;
-                    for (int c = 0; c < d; ++c) dot = fmaf(wk[c], m[c], dot);
-                    score[j] = fmaf(-2.0f, dot, nrm[j]);
-                }
-                memset(used, 0, (size_t)M);
-                for (int i = 0; i < C; ++i) {
-                    int best = -1;
-                    for (int j = 0; j < M; ++j) {
-                        if (used[j]) continue;
-                        if (best < 0 || score[j] < score[best]) best = j;
-                    }
-                    used[best] = 1;
-                    cand[i] = best;
-                    if (cand_out) cand_out[dbg * C + i] = best;
-                    if (score_out) score_out[dbg * C + i] = score[best];
-                }
-                /* choice by estimated perturbation */
-                int chosen = -1;
-                float bestE = 0.0f;
-                for (int i = 0; i < C; ++i) {
-                    int j = cand[i];
-                    const float* m = mu + (size_t)j * d;
-                    for (int c = 0; c < d; ++c) x[c] = k[c] - m[c];
-                    float E = 0.0f;
-                    for (int g = 0; g < ng; ++g) {
-                        uint16_t sb, zb;
-                        codec_params(x + g * GROUP, GROUP, &sb, &zb);
-                        float s = or_f32_from_f16(sb);
-                        float ws = Wg[(size_t)h * ng + g] * s;
-                        E = fmaf(ws, s, E);
-                    }
-                    if (E_out) E_out[dbg * C + i] = E;
-                    if (chosen < 0 || E < bestE) {
-                        chosen = j;
-                        bestE = E;
-                        memcpy(xbest, x, (size_t)d * sizeof(float));
-                    }
-                }
+                for (int c = 0; c < d; ++c) k[c] = or_f32_from_bf16(K[in + c]);
+                int chosen = qsac_choose(k, wh, Wg + (size_t)h * ng, mu, nrm, M, C, d, wk, score, cand, used, x,
+                                         xbest, cand_out ? cand_out + dbg * C : NULL,
+                                         score_out ? score_out + dbg * C : NULL, E_out ? E_out + dbg * C : NULL);
                 /* residual codes, scales, zeros */
                 quantize_row(xbest, d, cw, szr, deq);
                 memcpy(k_code + slot * nw, cw, (size_t)nw * 4);
@@ -450,14 +470,85 @@ int or_quantize(int B, int Hkv, int d, int M, int r, int cap,
 }
 
 /* ------------------------------------------------------------------------ */
+/* QSAC-aware centre fitting.                                                 */
+/*   Article "1. QSAC" names the clustering (QSAC picks INT2-friendly Key     */
+/*   centres) but not its loop. Reading taken: Lloyd iterations whose          */
+/*   assignment step is the QSAC decision above (rank by the weighted          */
+/*   distance, keep C candidates, choose the least estimated perturbation) and */
+/*   whose update step moves every centre to the mean of the keys assigned to  */
+/*   it; a centre with no key keeps its value. The mean: the keys' sum in      */
+/*   64-bit fixed point (units of 2^-24, each bf16 value truncated toward 0    */
+/*   to a whole number of units: exact for |k| >= 2^-17), divided by the count */
+/*   in fp64 (one rounding), scaled by 2^-24 (exact), rounded to fp16 (nearest */
+/*   even). Exact, order-free sums make the update independent of summation   */
+/*   order. Valid while n * max|k| < 2^39.                                      */
+/* X bf16 [n][Hkv][d]; cent fp16 [Hkv][M][d] (in: initial centres, out: the   */
+/* fitted ones); assign [n][Hkv] (out, may be NULL): the last assignment.      */
+/* ------------------------------------------------------------------------ */
+
+int or_fit_centroids(int n, int Hkv, int d, int M, int C, const uint16_t* X, const float* w,
+                     const float* Wg, int iters, uint16_t* cent, int32_t* assign)
+{
+    if (d % GROUP || C < 1 || C > M || n < 0 || iters < 0) return 1;
+    int ng = d / GROUP;
+    float* mu = (float*)malloc((size_t)M * d * sizeof(float));
+    float* nrm = (float*)malloc((size_t)M * sizeof(float));
+    float* score = (float*)malloc((size_t)M * sizeof(float));
+    int* cand = (int*)malloc((size_t)C * sizeof(int));
+    float* k = (float*)malloc((size_t)d * sizeof(float));
+    float* wk = (float*)malloc((size_t)d * sizeof(float));
+    float* x = (float*)malloc((size_t)d * sizeof(float));
+    float* xbest = (float*)malloc((size_t)d * sizeof(float));
+    char* used = (char*)malloc((size_t)M);
+    int* a = (int*)malloc(((size_t)n + 1) * sizeof(int));
+    int64_t* sum = (int64_t*)malloc((size_t)M * d * sizeof(int64_t));
+    int64_t* cnt = (int64_t*)malloc((size_t)M * sizeof(int64_t));
+    for (int it = 0; it < iters; ++it) {
+        for (int h = 0; h < Hkv; ++h) {
+            const float* wh = w + (size_t)h * d;
+            qsac_tables(cent, wh, h, M, d, mu, nrm);
+            /* assignment */
+            for (int t = 0; t < n; ++t) {
+                const uint16_t* xr = X + ((size_t)t * Hkv + h) * d;
+                for (int c = 0; c < d; ++c) k[c] = or_f32_from_bf16(xr[c]);
+                a[t] = qsac_choose(k, wh, Wg + (size_t)h * ng, mu, nrm, M, C, d, wk, score, cand, used, x, xbest,
+                                   NULL, NULL, NULL);
+                if (assign) assign[(size_t)t * Hkv + h] = a[t];
+            }
+            /* update */
+            memset(sum, 0, (size_t)M * d * sizeof(int64_t));
+            memset(cnt, 0, (size_t)M * sizeof(int64_t));
+            for (int t = 0; t < n; ++t) {
+                const uint16_t* xr = X + ((size_t)t * Hkv + h) * d;
+                cnt[a[t]] += 1;
+                for (int c = 0; c < d; ++c)
+                    sum[(size_t)a[t] * d + c] += (int64_t)ldexp((double)or_f32_from_bf16(xr[c]), 24);
+            }
+            for (int j = 0; j < M; ++j) {
+                if (cnt[j] == 0) continue;
+                for (int c = 0; c < d; ++c) {
+                    double q = (double)sum[(size_t)j * d + c] / (double)cnt[j];
+                    cent[((size_t)h * M + j) * d + c] =
+                        f16_encode_exact(round_to_format(ldexp(q, -24), 10, -14, F16_MAX, RND_NEAREST_EVEN));
+                }
+            }
+        }
+    }
+    free(mu); free(nrm); free(score); free(cand); free(k); free(wk); free(x); free(xbest); free(used);
+    free(a); free(sum); free(cnt);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Attention over the packed cache (fp64).                                    */
 /*   logit_t = scale * (q . khat_t + (q P) . a_t), khat_t = mu_idx + deq_t:    */
 /*   the PSAC term is the Key compensation of article "2. PSAC" applied to the */
 /*   score, q.(khat + P a) = q.khat + (qP).a. Softmax in two passes.           */
 /*   Decode: dequantized values are exact (mu + code s + z in fp64), matching   */
-/*   a kernel that never rounds them. Chunk: the kernel's operand precision:   */
-/*   khat = bf16(fp32(fmaf(code, s, z) + mu)), vhat = fp16(fmaf(code, s, z)),  */
-/*   u = qP as fp16, self keys bf16, self values as fp16.                      */
+/*   a kernel that never rounds them. Chunk: the kernel's operand precision,   */
+/*   fp16 arithmetic with one rounding per operation:                          */
+/*   khat = fp16(code s + fp16(z + mu)), vhat = fp16(code s + z), u = qP as    */
+/*   fp16, self keys and values rounded from bf16 to fp16.                     */
 /* ------------------------------------------------------------------------ */
 
 typedef struct {
