@@ -5,7 +5,7 @@ pointers (``tensor.data_ptr()``) and the current CUDA stream. PyTorch is used
 for device memory and streams only. If ``libkv2.so`` is missing or fails to
 load, importing the binding raises: there is no CPU fallback.
 
-Names follow the C ABI: ``kv2_fit_psac_basis``, ``kv2_quantize_append``,
+Names follow the C ABI: ``kv2_fit_psac_basis``, ``kv2_fit_centroids``, ``kv2_quantize_append``,
 ``kv2_attention_decode``, ``kv2_attention_chunk`` and the workspace-size
 queries. ``Cache`` owns the device buffers of one packed cache and builds the
 ``kv2_cache`` descriptor.
@@ -57,6 +57,10 @@ def _load():
     L.kv2_fit_workspace_size.argtypes = [I, I]
     L.kv2_fit_psac_basis.restype = I
     L.kv2_fit_psac_basis.argtypes = [P, I, I, I, I, I, P, P, P, P, P, S, P]
+    L.kv2_fit_centroids_workspace_size.restype = S
+    L.kv2_fit_centroids_workspace_size.argtypes = [I, I, I]
+    L.kv2_fit_centroids.restype = I
+    L.kv2_fit_centroids.argtypes = [P, I, I, I, I, I, P, P, I, P, P, P, S, P]
     L.kv2_quantize_append.restype = I
     L.kv2_quantize_append.argtypes = [ctypes.POINTER(kv2_cache), P, P, I, I, I, P]
     L.kv2_decode_workspace_size.restype = S
@@ -95,7 +99,8 @@ def __getattr__(name):
 
 
 EXPORTS = ["kv2_status_string", "kv2_last_error", "kv2_version", "kv2_fit_workspace_size",
-           "kv2_fit_psac_basis", "kv2_quantize_append", "kv2_decode_workspace_size",
+           "kv2_fit_psac_basis", "kv2_fit_centroids_workspace_size", "kv2_fit_centroids",
+           "kv2_quantize_append", "kv2_decode_workspace_size",
            "kv2_attention_decode", "kv2_attention_decode_noalloc", "kv2_append_attention_decode",
            "kv2_chunk_workspace_size", "kv2_attention_chunk"]
 
@@ -187,6 +192,25 @@ def kv2_fit_psac_basis(Qhist: torch.Tensor, H_kv: int, r: int, P=None, w=None, W
     _check(_get_lib().kv2_fit_psac_basis(_ptr(Qhist), n, H_q, H_kv, d, r, _ptr(P), _ptr(w), _ptr(Wg),
                                   _ptr(energy), _ptr(ws), ws.numel(), _stream(stream)))
     return P[:, :, :r], w, Wg, energy
+
+
+def kv2_fit_centroids_workspace_size(H_kv: int, d: int, M: int) -> int:
+    return int(_get_lib().kv2_fit_centroids_workspace_size(H_kv, d, M))
+
+
+def kv2_fit_centroids(X: torch.Tensor, centroids: torch.Tensor, candidates: int, w: torch.Tensor,
+                      Wg: torch.Tensor, iters: int, assign=None, ws=None, stream=None):
+    """X bf16 [n][H_kv][d] sample keys, centroids fp16 [H_kv][M][d] (device;
+    updated in place) -> (centroids, assign int32 [n][H_kv])."""
+    n, H_kv, d = X.shape
+    M = centroids.shape[1]
+    dev = X.device
+    assign = torch.empty((max(n, 1), H_kv), dtype=torch.int32, device=dev) if assign is None else assign
+    need = kv2_fit_centroids_workspace_size(H_kv, d, M)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev) if ws is None else ws
+    _check(_get_lib().kv2_fit_centroids(_ptr(X), n, H_kv, d, M, candidates, _ptr(w), _ptr(Wg), iters,
+                                        _ptr(centroids), _ptr(assign), _ptr(ws), ws.numel(), _stream(stream)))
+    return centroids, assign[:n]
 
 
 def kv2_quantize_append(cache: Cache, K: torch.Tensor, V: torch.Tensor, pos: int,

@@ -109,6 +109,31 @@ kv2_status kv2_fit_psac_basis(const uint16_t* Qhist, int n, int H_q, int H_kv, i
   return cuda_status(kv2::launch_fit(a, static_cast<cudaStream_t>(stream)), "fit launch");
 }
 
+size_t kv2_fit_centroids_workspace_size(int H_kv, int d, int M) {
+  if (H_kv <= 0 || (d != 64 && d != 128) || M < 1 || M > 512) return 0;
+  return kv2::fit_centroids_workspace_bytes(H_kv, d, M);
+}
+
+kv2_status kv2_fit_centroids(const uint16_t* X, int n, int H_kv, int d, int M, int candidates, const float* w,
+                             const float* Wg, int iters, uint16_t* centroids, int32_t* assign, void* ws,
+                             size_t ws_bytes, void* stream) {
+  if (H_kv <= 0 || n < 0 || n > 65536) return fail(KV2_ERR_INVALID_ARG, "fit_centroids: H_kv=%d, n=%d", H_kv, n);
+  if (d != 64 && d != 128) return fail(KV2_ERR_UNSUPPORTED, "fit_centroids: head dim d=%d (supported: 64, 128)", d);
+  if (M < 1 || M > 512) return fail(KV2_ERR_UNSUPPORTED, "fit_centroids: M=%d outside 1..512", M);
+  if (candidates < 1 || candidates > M)
+    return fail(KV2_ERR_INVALID_ARG, "fit_centroids: candidates=%d outside 1..M=%d", candidates, M);
+  if (iters < 0) return fail(KV2_ERR_INVALID_ARG, "fit_centroids: iters=%d < 0", iters);
+  if (iters == 0 || n == 0) return KV2_OK;
+  if (!X || !w || !Wg || !centroids || !assign || !ws)
+    return fail(KV2_ERR_INVALID_ARG, "fit_centroids: NULL pointer");
+  if (!aligned16(X) || !aligned16(centroids) || !aligned16(ws))
+    return fail(KV2_ERR_INVALID_ARG, "fit_centroids: misaligned pointer");
+  const size_t need = kv2::fit_centroids_workspace_bytes(H_kv, d, M);
+  if (ws_bytes < need) return fail(KV2_ERR_WORKSPACE, "fit_centroids: workspace %zu < %zu bytes", ws_bytes, need);
+  kv2::FitCentroidsArgs a{X, n, H_kv, d, M, candidates, iters, w, Wg, centroids, assign, ws};
+  return cuda_status(kv2::launch_fit_centroids(a, static_cast<cudaStream_t>(stream)), "fit_centroids launch");
+}
+
 namespace {
 
 // argument checks of a quantize/append call (the cache already checked)

@@ -30,8 +30,25 @@ struct QuantizeArgs {
   uint32_t* v_sz;
   void* cidx;
   uint16_t* psac;
+  // assignment only (centre fitting): when set, the chosen centre of row
+  // (b * n_new + t) and head h goes to assign[row * H + h] and nothing is
+  // packed (V, P and the cache streams are not read or written)
+  int32_t* assign = nullptr;
 };
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s);
+
+// QSAC-aware centre fitting (Lloyd iterations with the QSAC assignment).
+struct FitCentroidsArgs {
+  const uint16_t* X;   // bf16 [n][H][D] sample keys
+  int n, H, D, M, C, iters;
+  const float* w;      // [H][D]
+  const float* Wg;     // [H][D/32]
+  uint16_t* cent;      // fp16 [H][M][D], initial centres in, fitted centres out
+  int32_t* assign;     // [n][H]: the last assignment
+  void* ws;            // fit_centroids_workspace_bytes(H, D, M)
+};
+size_t fit_centroids_workspace_bytes(int H, int D, int M);
+cudaError_t launch_fit_centroids(const FitCentroidsArgs& a, cudaStream_t s);
 
 // Decode attention.
 struct DecodeArgs {

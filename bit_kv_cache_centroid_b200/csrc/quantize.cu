@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
 #pragma unroll
       for (int g = 0; g < NG; ++g) {
         kx[g] = __uint_as_float(uint32_t(krow[g * kGroup + lane]) << 16);
-        vx[g] = __uint_as_float(uint32_t(vrow[g * kGroup + lane]) << 16);
+        vx[g] = a.assign ? 0.0f : __uint_as_float(uint32_t(vrow[g * kGroup + lane]) << 16);
       }
       // ---- perturbation estimate: lane (candidate i, group g) takes the
       // group's scale; E_i = fmaf chain over ascending g of (W_g s_g) s_g;
@@ -306,8 +306,11 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
         }
         rank = int(best_i);
       }
-      // ---- K residual and V codecs, lane = channel of the group
       const int jc = cand_w[rank];
+      if (a.assign) {
+        if (lane == 0) a.assign[size_t(row) * a.H + h] = jc;
+      } else {
+      // ---- K residual and V codecs, lane = channel of the group
       const int colc = (jc % 32) * CPL + jc / 32;
       const size_t slot = slot_of(row);
 #pragma unroll
@@ -366,6 +369,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
         }
         if (lane < 8 && i0 + lane < a.r) a.psac[slot * a.r + i0 + lane] = f16_rn(mine);
       }
+      }
     } else {
     // ---- perturbation estimate per (key, candidate); least (E, rank) per key
     if (C > 1) {
@@ -400,6 +404,12 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
       __syncwarp();
     }
 
+    if (a.assign) {
+      for (int k = lane; k < nk; k += 32) {
+        const int rank = (C > 1) ? int(best_w[k] & 0xffffffffu) : 0;
+        a.assign[size_t(row_of(k)) * a.H + h] = cand_w[k * C + rank];
+      }
+    } else {
     // ---- K residual and V codecs per (key, group)
     for (int task = lane; task < nk * NG * 2; task += 32) {
       const int which = task / (nk * NG);   // 0: keys, 1: values
@@ -471,6 +481,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
 #pragma unroll 8
       for (int c = 0; c < D; ++c) acc = __fmaf_rn(Pcol[c * a.r], e[c], acc);
       a.psac[slot_of(row_of(k)) * a.r + i] = f16_rn(acc);
+    }
     }
     }
     __syncwarp();    // e_w / wk_w and cand_w are reused by this warp's next tile

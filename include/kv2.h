@@ -118,6 +118,38 @@ kv2_status kv2_fit_psac_basis(const uint16_t* Qhist, int n, int H_q, int H_kv, i
                               void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Workspace for kv2_fit_centroids, in bytes: (H_kv*M*d + H_kv*M)*8 (64-bit
+ * integer sums and counts). Returns 0 for unsupported shapes.
+ */
+size_t kv2_fit_centroids_workspace_size(int H_kv, int d, int M);
+
+/*
+ * kv2_fit_centroids — Key centres for the QSAC assignment (article "1. QSAC":
+ * the clustering picks INT2-friendly centres). The pages do not print the
+ * loop; it is read as Lloyd iterations whose assignment step is the QSAC
+ * decision of kv2_quantize_append (same ranking, candidates and choice,
+ * bit for bit) and whose update step moves every centre to the mean of the
+ * keys assigned to it; a centre that no key chooses keeps its value.
+ * Mean: each bf16 key value as a whole number of 2^-24 units (truncated
+ * toward zero), summed in 64-bit integers (exact, order-free), divided by
+ * the count in fp64, times 2^-24, rounded to fp16 (nearest even).
+ * X        : bf16 [n][H_kv][d] sample keys (read-only), n <= 65536,
+ *            |k| < 2^23 (so the 64-bit sums cannot overflow).
+ * w, Wg    : the sensitivities of kv2_fit_psac_basis (read-only).
+ * centroids: fp16 [H_kv][M][d], initial centres in, fitted centres out.
+ * assign   : int32 [n][H_kv] out: the assignment of the last iteration.
+ * iters >= 0 iterations (0 leaves everything unchanged); candidates 1..M.
+ * ws       : device workspace of kv2_fit_centroids_workspace_size bytes.
+ * All pointers are device memory owned by the caller; asynchronous on stream.
+ * Errors: KV2_ERR_INVALID_ARG (NULL / misaligned pointers, n out of range,
+ * candidates outside 1..M, iters < 0), KV2_ERR_UNSUPPORTED (d not 64/128,
+ * M outside 1..512), KV2_ERR_WORKSPACE.
+ */
+kv2_status kv2_fit_centroids(const uint16_t* X, int n, int H_kv, int d, int M, int candidates,
+                             const float* w, const float* Wg, int iters, uint16_t* centroids,
+                             int32_t* assign, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * kv2_quantize_append — QSAC centroid assignment, INT2 residual/value
  * packing and PSAC coefficients for n_new new tokens of every (batch, KV
  * head), written to slots [pos, pos + n_new) (article "1. QSAC", "2. PSAC").
