@@ -290,6 +290,23 @@ def extras(torch, kv2, args, pk):
                        "GBps": round((rd + wr) / (ms * 1e-3) / 1e9, 2),
                        "hbm_frac": round((rd + wr) / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
                        "ranking_TFMAps": round(fma / (ms * 1e-3) / 1e12, 3)}
+    # QSAC-aware centre fitting on the chunk's new keys (5 iterations)
+    X = K[0]
+    cent0 = torch.from_numpy(w.centroids.view(np.int16)).to(dev)
+    cent = cent0.clone()
+    kv2.kv2_fit_centroids(X, cent, s.C, wt, Wg, 1)
+    torch.cuda.synchronize()
+    iters = 5
+    cent.copy_(cent0)
+    a.record()
+    kv2.kv2_fit_centroids(X, cent, s.C, wt, Wg, iters)
+    b.record()
+    torch.cuda.synchronize()
+    it_ms = a.elapsed_time(b) / iters
+    nk = X.shape[0] * X.shape[1]
+    out["fit_centroids"] = {"workload": f"{X.shape[0]} keys x {X.shape[1]} heads, d={s.d}, M={s.M}, C={s.C}, "
+                                        f"{iters} iterations", "ms_per_iteration": round(it_ms, 4),
+                            "ranking_TFMAps": round(nk * s.M * s.d / (it_ms * 1e-3) / 1e12, 3)}
     out["chunk"] = chunk_section(torch, kv2, args, pk)
     out["long_horizon"] = long_horizon_section(torch, kv2, args, pk)
     a.record()
