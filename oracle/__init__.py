@@ -67,11 +67,11 @@ def _declare(L):
     L.or_f32_from_bf16.restype = ctypes.c_float
     L.or_codec_group.argtypes = [_P, _I, _P, _P, _P, _P]
     L.or_fit.argtypes = [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P]
-    L.or_quantize.argtypes = [_I] * 6 + [_P, _P, _I, _I, _I, _P, _P, _P, _P] + [_P] * 6 + [_P] * 3
-    L.or_decode.argtypes = [_I] * 6 + [_P] * 8 + [_I, _P, _I, ctypes.c_double, _P]
-    L.or_chunk.argtypes = ([_I] * 6 + [_P] * 8 + [_I, _P, _I, _I, _P, _P, _I,
+    L.or_quantize.argtypes = [_I] * 6 + [_P, _P, _I, _I, _I, _P, _P, _P, _P] + [_P] * 6 + [_I, _P] + [_P] * 3
+    L.or_decode.argtypes = [_I] * 6 + [_P] * 6 + [_I, _P] + [_P] * 2 + [_I, _P, _I, ctypes.c_double, _P]
+    L.or_chunk.argtypes = ([_I] * 6 + [_P] * 6 + [_I, _P] + [_P] * 2 + [_I, _P, _I, _I, _P, _P, _I,
                                                   ctypes.c_double, _P, _I, _P])
-    L.or_decode_logits.argtypes = [_I] * 7 + [_P] * 6 + [_I, _P, _P]
+    L.or_decode_logits.argtypes = [_I] * 7 + [_P] * 4 + [_I, _P] + [_P] * 2 + [_I, _P, _P]
     L.or_fit_centroids.argtypes = [_I] * 5 + [_P, _P, _P, _I, _P, _P]
     for f in (L.or_codec_group, L.or_fit, L.or_quantize, L.or_decode, L.or_chunk,
               L.or_decode_logits, L.or_fit_centroids):
@@ -163,7 +163,6 @@ def quantize(pc, K: np.ndarray, V: np.ndarray, pos: int, C: int, P: np.ndarray,
     w = _c(w, np.float32)
     Wg = _c(Wg, np.float32)
     r = pc.r
-    psac = pc.psac if r else np.zeros(1, np.uint16)
     dbg = None
     if debug:
         dbg = QuantDebug(np.zeros((B, n_new, Hkv, C), np.int32),
@@ -173,7 +172,7 @@ def quantize(pc, K: np.ndarray, V: np.ndarray, pos: int, C: int, P: np.ndarray,
         B, Hkv, d, pc.M, r, pc.capacity, _ptr(K), _ptr(V), n_new, pos, C,
         _ptr(_c(pc.centroids, np.uint16)), _ptr(P), _ptr(w), _ptr(Wg),
         _ptr(pc.k_code), _ptr(pc.v_code), _ptr(pc.k_sz), _ptr(pc.v_sz),
-        _ptr(pc.cidx), _ptr(psac),
+        _ptr(pc.cidx), *_psac_args(pc),
         _ptr(dbg.cand) if dbg else None, _ptr(dbg.score) if dbg else None,
         _ptr(dbg.E) if dbg else None)
     if rc:
@@ -197,13 +196,21 @@ def fit_centroids(X: np.ndarray, M: int, C: int, w: np.ndarray, Wg: np.ndarray,
     return cent, assign[:n]
 
 
-def _cache_args(pc):
+def _psac_args(pc):
+    """(coefficients, format, per-token scales) of a packed cache: format 0 =
+    fp16 [r], 1 = int8 [r] with one fp16 scale per token."""
+    fmt = getattr(pc, "psac_fmt", 0)
     psac = pc.psac if pc.r else np.zeros(1, np.uint16)
+    sc = pc.psac_scale if (fmt == 1 and pc.r) else np.zeros(1, np.uint16)
+    return _ptr(psac), fmt, _ptr(sc)
+
+
+def _cache_args(pc):
     P = getattr(pc, "P", None)
     if P is None or pc.r == 0:
         P = np.zeros(1, np.float32)
     return (_ptr(pc.k_code), _ptr(pc.v_code), _ptr(pc.k_sz), _ptr(pc.v_sz),
-            _ptr(pc.cidx), _ptr(psac), _ptr(_c(pc.centroids, np.uint16)),
+            _ptr(pc.cidx), *_psac_args(pc), _ptr(_c(pc.centroids, np.uint16)),
             _ptr(_c(P, np.float32)))
 
 
@@ -245,9 +252,8 @@ def decode_logits(pc, P: np.ndarray, b: int, h: int, length: int, q: np.ndarray)
     q = _c(q, np.float64)
     pc.P = P
     out = np.zeros(length, np.float64)
-    psac = pc.psac if pc.r else np.zeros(1, np.uint16)
     Pp = _c(P, np.float32) if pc.r else np.zeros(1, np.float32)
     lib().or_decode_logits(pc.H_kv, pc.d, pc.M, pc.r, pc.capacity, b, h,
-                           _ptr(pc.k_code), _ptr(pc.k_sz), _ptr(pc.cidx), _ptr(psac),
+                           _ptr(pc.k_code), _ptr(pc.k_sz), _ptr(pc.cidx), *_psac_args(pc),
                            _ptr(_c(pc.centroids, np.uint16)), _ptr(Pp), length, _ptr(q), _ptr(out))
     return out

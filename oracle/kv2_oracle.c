@@ -382,6 +382,25 @@ static void qsac_tables(const uint16_t* cent, const float* wh, int h, int M, int
     }
 }
 
+/* INT8 PSAC coefficients with one fp16 scale per token (the compensation
+ * information stored compactly, article "2. PSAC" and the compression count
+ * of the evaluation). Reading taken: symmetric, scale = fp16 round-up of the
+ * fp32 quotient max|a| / 127, so every |a / scale| <= 127; code =
+ * clamp(round-half-even(a / scale), -127, 127) (fp32 division), 0 when the
+ * scale is 0; the coefficient read back is code * scale. */
+static void psac_int8(const float* a, int r, float amax, int8_t* q, uint16_t* scale_bits)
+{
+    uint16_t sb = or_f16_from_f32(amax / 127.0f, RND_UP);
+    float s = or_f32_from_f16(sb);
+    *scale_bits = sb;
+    for (int i = 0; i < r; ++i) {
+        float v = (s > 0.0f) ? rintf(a[i] / s) : 0.0f;
+        if (v > 127.0f) v = 127.0f;
+        if (v < -127.0f) v = -127.0f;
+        q[i] = (int8_t)v;
+    }
+}
+
 static uint32_t pack_word(const uint32_t* codes16)
 {
     uint32_t w = 0;
@@ -412,10 +431,10 @@ int or_quantize(int B, int Hkv, int d, int M, int r, int cap,
                 const uint16_t* K, const uint16_t* V, int n_new, int pos, int C,
                 const uint16_t* cent, const float* P, const float* w, const float* Wg,
                 uint32_t* k_code, uint32_t* v_code, uint32_t* k_sz, uint32_t* v_sz,
-                void* cidx, uint16_t* psac,
+                void* cidx, uint16_t* psac, int psac_fmt, uint16_t* psac_scale,
                 int32_t* cand_out, float* score_out, float* E_out)
 {
-    if (d % GROUP || C < 1 || C > M || pos < 0 || pos + n_new > cap) return 1;
+    if (d % GROUP || C < 1 || C > M || pos < 0 || pos + n_new > cap || (psac_fmt != 0 && psac_fmt != 1)) return 1;
     int ng = d / GROUP, nw = d / 16;
     float* mu = (float*)malloc((size_t)M * d * sizeof(float));
     float* nrm = (float*)malloc((size_t)M * sizeof(float));
@@ -429,6 +448,7 @@ int or_quantize(int B, int Hkv, int d, int M, int r, int cap,
     uint32_t* cw = (uint32_t*)malloc((size_t)nw * sizeof(uint32_t));
     uint32_t* szr = (uint32_t*)malloc((size_t)ng * sizeof(uint32_t));
     char* used = (char*)malloc((size_t)M);
+    float* acoef = (float*)malloc(((size_t)r + 1) * sizeof(float));
     for (int h = 0; h < Hkv; ++h) {
         const float* wh = w + (size_t)h * d;
         qsac_tables(cent, wh, h, M, d, mu, nrm);
@@ -448,14 +468,19 @@ int or_quantize(int B, int Hkv, int d, int M, int r, int cap,
                 if (M <= 256) ((uint8_t*)cidx)[slot] = (uint8_t)chosen;
                 else ((uint16_t*)cidx)[slot] = (uint16_t)chosen;
                 /* PSAC coefficients of the key's quantization error */
+                float amax = 0.0f;
                 for (int i = 0; i < r; ++i) {
                     float a = 0.0f;
                     for (int c = 0; c < d; ++c) {
                         float e = xbest[c] - deq[c];
                         a = fmaf(P[((size_t)h * d + c) * r + i], e, a);
                     }
-                    psac[slot * (size_t)r + i] = or_f16_from_f32(a, RND_NEAREST_EVEN);
+                    acoef[i] = a;
+                    if (fabsf(a) > amax) amax = fabsf(a);
+                    if (psac_fmt == 0) psac[slot * (size_t)r + i] = or_f16_from_f32(a, RND_NEAREST_EVEN);
                 }
+                if (psac_fmt == 1 && r > 0) psac_int8(acoef, r, amax, (int8_t*)psac + slot * (size_t)r,
+                                                      psac_scale + slot);
                 /* values: same codec, no centre */
                 for (int c = 0; c < d; ++c) x[c] = or_f32_from_bf16(V[in + c]);
                 quantize_row(x, d, cw, szr, NULL);
@@ -465,7 +490,7 @@ int or_quantize(int B, int Hkv, int d, int M, int r, int cap,
         }
     }
     free(mu); free(nrm); free(score); free(cand); free(k); free(wk); free(x);
-    free(deq); free(xbest); free(cw); free(szr); free(used);
+    free(deq); free(xbest); free(cw); free(szr); free(used); free(acoef);
     return 0;
 }
 
@@ -557,7 +582,18 @@ typedef struct {
     const void* cidx;
     const uint16_t *psac, *cent;
     const float* P;
+    int psac_fmt;                 /* 0: fp16 [r]; 1: int8 [r] + fp16 scale per token */
+    const uint16_t* psac_scale;
 } or_cache;
+
+/* PSAC coefficient i of a cached token, exact: the stored fp16 value, or
+ * code * scale for the int8 format */
+static double psac_value(const or_cache* c, size_t slot, int i)
+{
+    if (c->psac_fmt == 0) return (double)or_f32_from_f16(c->psac[slot * (size_t)c->r + i]);
+    int8_t q = ((const int8_t*)c->psac)[slot * (size_t)c->r + i];
+    return (double)q * (double)or_f32_from_f16(c->psac_scale[slot]);
+}
 
 static int cache_idx(const or_cache* c, size_t slot)
 {
@@ -629,11 +665,11 @@ static void softmax_combine(const double* logit, const double* vals, int n, int 
 int or_decode(int B, int Hkv, int d, int M, int r, int cap,
               const uint32_t* k_code, const uint32_t* v_code, const uint32_t* k_sz,
               const uint32_t* v_sz, const void* cidx, const uint16_t* psac,
-              const uint16_t* cent, const float* P,
+              int psac_fmt, const uint16_t* psac_scale, const uint16_t* cent, const float* P,
               int len, const uint16_t* Q, int Hq, double sm_scale, double* out)
 {
     if (Hq % Hkv || len < 0 || len > cap) return 1;
-    or_cache c = {B, Hkv, d, M, r, cap, k_code, v_code, k_sz, v_sz, cidx, psac, cent, P};
+    or_cache c = {B, Hkv, d, M, r, cap, k_code, v_code, k_sz, v_sz, cidx, psac, cent, P, psac_fmt, psac_scale};
     int G = Hq / Hkv;
     double* logit = (double*)malloc(((size_t)len + 1) * sizeof(double));
     double* vals = (double*)malloc(((size_t)len + 1) * d * sizeof(double));
@@ -655,7 +691,7 @@ int or_decode(int B, int Hkv, int d, int M, int r, int cap,
                 double acc = 0.0;
                 for (int ch = 0; ch < d; ++ch) acc += q[ch] * kh[ch];
                 for (int i = 0; i < r; ++i)
-                    acc += u[i] * (double)or_f32_from_f16(psac[slot * r + i]);
+                    acc += u[i] * psac_value(&c, slot, i);
                 logit[t] = acc * sm_scale;
             }
             softmax_combine(logit, vals, len, d, out + ((size_t)b * Hq + hq) * d);
@@ -671,12 +707,12 @@ int or_decode(int B, int Hkv, int d, int M, int r, int cap,
 int or_chunk(int B, int Hkv, int d, int M, int r, int cap,
              const uint32_t* k_code, const uint32_t* v_code, const uint32_t* k_sz,
              const uint32_t* v_sz, const void* cidx, const uint16_t* psac,
-             const uint16_t* cent, const float* P, int len,
+             int psac_fmt, const uint16_t* psac_scale, const uint16_t* cent, const float* P, int len,
              const uint16_t* Q, int Hq, int Nq, const uint16_t* Kself, const uint16_t* Vself,
              int frame_tokens, double sm_scale, const int32_t* rows, int nrows, double* out)
 {
     if (Hq % Hkv || len < 0 || len > cap || frame_tokens <= 0) return 1;
-    or_cache c = {B, Hkv, d, M, r, cap, k_code, v_code, k_sz, v_sz, cidx, psac, cent, P};
+    or_cache c = {B, Hkv, d, M, r, cap, k_code, v_code, k_sz, v_sz, cidx, psac, cent, P, psac_fmt, psac_scale};
     int G = Hq / Hkv;
     size_t nmax = (size_t)len + (size_t)Nq + 1;
     double* logit = (double*)malloc(nmax * sizeof(double));
@@ -700,7 +736,7 @@ int or_chunk(int B, int Hkv, int d, int M, int r, int cap,
             dequant_operand(&c, slot, kh, vals + n * d);
             double acc = 0.0;
             for (int ch = 0; ch < d; ++ch) acc += q[ch] * kh[ch];
-            for (int a = 0; a < r; ++a) acc += u[a] * (double)or_f32_from_f16(psac[slot * r + a]);
+            for (int a = 0; a < r; ++a) acc += u[a] * f16_round(psac_value(&c, slot, a));
             logit[n] = acc * sm_scale;
         }
         int fi = i / frame_tokens;
@@ -724,10 +760,10 @@ int or_chunk(int B, int Hkv, int d, int M, int r, int cap,
  * PSAC and centroid closed forms. q fp64 [d]; out [len]. */
 int or_decode_logits(int Hkv, int d, int M, int r, int cap, int b, int h,
                      const uint32_t* k_code, const uint32_t* k_sz, const void* cidx,
-                     const uint16_t* psac, const uint16_t* cent, const float* P,
-                     int len, const double* q, double* out)
+                     const uint16_t* psac, int psac_fmt, const uint16_t* psac_scale,
+                     const uint16_t* cent, const float* P, int len, const double* q, double* out)
 {
-    or_cache c = {b + 1, Hkv, d, M, r, cap, k_code, k_code, k_sz, k_sz, cidx, psac, cent, P};
+    or_cache c = {b + 1, Hkv, d, M, r, cap, k_code, k_code, k_sz, k_sz, cidx, psac, cent, P, psac_fmt, psac_scale};
     double* kh = (double*)malloc((size_t)d * sizeof(double));
     double* vh = (double*)malloc((size_t)d * sizeof(double));
     double* u = (double*)malloc(((size_t)r + 1) * sizeof(double));
@@ -740,7 +776,7 @@ int or_decode_logits(int Hkv, int d, int M, int r, int cap, int b, int h,
         dequant_exact(&c, slot, kh, vh);
         double acc = 0.0;
         for (int ch = 0; ch < d; ++ch) acc += q[ch] * kh[ch];
-        for (int i = 0; i < r; ++i) acc += u[i] * (double)or_f32_from_f16(psac[slot * r + i]);
+        for (int i = 0; i < r; ++i) acc += u[i] * psac_value(&c, slot, i);
         out[t] = acc;
     }
     free(kh); free(vh); free(u);

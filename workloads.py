@@ -319,7 +319,9 @@ class PackedCache:
     """Host copy of a packed cache, in the library's layout:
     k_code/v_code u32 [B][H_kv][cap][d/16], k_sz/v_sz u32 [B][H_kv][cap][d/32]
     (low half fp16 scale, high half fp16 zero), cidx u8/u16 [B][H_kv][cap],
-    psac fp16 bits [B][H_kv][cap][r], centroids fp16 bits [H_kv][M][d]."""
+    psac fp16 bits [B][H_kv][cap][r] (format 0) or int8 codes [B][H_kv][cap][r]
+    with fp16 scale bits psac_scale [B][H_kv][cap] (format 1), centroids fp16
+    bits [H_kv][M][d]."""
     B: int
     H_kv: int
     d: int
@@ -333,9 +335,11 @@ class PackedCache:
     cidx: np.ndarray
     psac: np.ndarray
     centroids: np.ndarray
+    psac_fmt: int = 0
+    psac_scale: np.ndarray | None = None
 
     @staticmethod
-    def empty(B, H_kv, d, M, r, capacity, centroids):
+    def empty(B, H_kv, d, M, r, capacity, centroids, psac_fmt: int = 0):
         cap = (capacity + 15) // 16 * 16          # the library wants capacity % 16 == 0
         return PackedCache(
             B, H_kv, d, M, r, cap,
@@ -344,18 +348,21 @@ class PackedCache:
             np.zeros((B, H_kv, cap, d // GROUP), np.uint32),
             np.zeros((B, H_kv, cap, d // GROUP), np.uint32),
             np.zeros((B, H_kv, cap), np.uint8 if M <= 256 else np.uint16),
-            np.zeros((B, H_kv, cap, max(r, 1)), np.uint16),
-            centroids)
+            np.zeros((B, H_kv, cap, max(r, 1)), np.int8 if psac_fmt == 1 else np.uint16),
+            centroids, psac_fmt,
+            np.zeros((B, H_kv, cap), np.uint16) if psac_fmt == 1 else None)
 
 
 def random_packed_cache(s: Spec, T: int | None = None, seed: int | None = None,
                         centroids: np.ndarray | None = None,
-                        revisit_every: int = 0) -> PackedCache:
+                        revisit_every: int = 0, psac_fmt: int = 0) -> PackedCache:
     """A packed cache of T tokens filled with seeded random fields shaped like
     quantizer output: every u32 code word uniform (so each 2-bit code is
     uniform on 0..3), per-group fp16 scales log-normal around the spread of a
     unit-variance residual, zeros near -1.5 scale, centroid ids uniform, PSAC
-    coefficients ~ N(0, (0.05 scale)^2). With ``revisit_every`` = n > 0 the
+    coefficients ~ N(0, (0.05 scale)^2) (format 1: int8 codes uniform on
+    -127..127 with fp16 per-token scales of 0.15 scale / 127). With
+    ``revisit_every`` = n > 0 the
     tokens of frame n, 2n, ... repeat frame 0 with 10% of code words redrawn,
     so that retrieval targets recur (long-horizon workload)."""
     T = s.T if T is None else T
@@ -363,7 +370,7 @@ def random_packed_cache(s: Spec, T: int | None = None, seed: int | None = None,
     cap = (max(s.capacity, T) + 15) // 16 * 16
     if centroids is None:
         centroids = f16_bits(rng.standard_normal((s.H_kv, s.M, s.d)).astype(np.float32))
-    pc = PackedCache.empty(s.B, s.H_kv, s.d, s.M, s.r, cap, centroids)
+    pc = PackedCache.empty(s.B, s.H_kv, s.d, s.M, s.r, cap, centroids, psac_fmt)
     sh = (s.B, s.H_kv, T)
     ng = s.d // GROUP
     pc.k_code[:, :, :T] = rng.integers(0, 2 ** 32, sh + (s.d // 16,), dtype=np.uint32)
@@ -375,13 +382,18 @@ def random_packed_cache(s: Spec, T: int | None = None, seed: int | None = None,
     pc.cidx[:, :, :T] = rng.integers(0, s.M, sh).astype(pc.cidx.dtype)
     if s.r:
         sc = f16_values((pc.k_sz[:, :, :T] & 0xFFFF).astype(np.uint16)).mean(-1, keepdims=True)
-        pc.psac[:, :, :T] = f16_bits(0.05 * sc * rng.standard_normal(sh + (s.r,)))
+        if psac_fmt == 1:
+            pc.psac[:, :, :T] = rng.integers(-127, 128, sh + (s.r,)).astype(np.int8)
+            pc.psac_scale[:, :, :T] = f16_bits(0.15 * sc[..., 0] / 127.0)
+        else:
+            pc.psac[:, :, :T] = f16_bits(0.05 * sc * rng.standard_normal(sh + (s.r,)))
     if revisit_every and s.frame_tokens > 1:
         F = s.frame_tokens
         for f in range(revisit_every, T // F, revisit_every):
             dst = slice(f * F, (f + 1) * F)
-            for arr in (pc.k_code, pc.v_code, pc.k_sz, pc.v_sz, pc.cidx, pc.psac):
-                arr[:, :, dst] = arr[:, :, 0:F]
+            for arr in (pc.k_code, pc.v_code, pc.k_sz, pc.v_sz, pc.cidx, pc.psac, pc.psac_scale):
+                if arr is not None:
+                    arr[:, :, dst] = arr[:, :, 0:F]
             redraw = rng.random((s.B, s.H_kv, F)) < 0.1
             fresh = rng.integers(0, 2 ** 32, (s.B, s.H_kv, F, s.d // 16), dtype=np.uint32)
             pc.k_code[:, :, dst] = np.where(redraw[..., None], fresh, pc.k_code[:, :, dst])
