@@ -41,7 +41,8 @@ class kv2_cache(ctypes.Structure):
                 ("k_sz", ctypes.c_void_p), ("v_sz", ctypes.c_void_p),
                 ("cidx", ctypes.c_void_p), ("psac", ctypes.c_void_p),
                 ("centroids", ctypes.c_void_p), ("P", ctypes.c_void_p),
-                ("w", ctypes.c_void_p), ("Wg", ctypes.c_void_p)]
+                ("w", ctypes.c_void_p), ("Wg", ctypes.c_void_p),
+                ("psac_fmt", ctypes.c_int32), ("psac_scale", ctypes.c_void_p)]
 
 
 def _load():
@@ -123,10 +124,11 @@ class Cache:
     """Device buffers of one packed cache (layout of include/kv2.h) plus the
     read-only centroid table and fitted statistics it points to."""
 
-    def __init__(self, B, H_kv, d, M, r, capacity, centroids, device="cuda"):
+    def __init__(self, B, H_kv, d, M, r, capacity, centroids, device="cuda", psac_fmt=0):
         if capacity % 16:
             raise ValueError("capacity must be a multiple of 16")
         self.B, self.H_kv, self.d, self.M, self.r, self.capacity = B, H_kv, d, M, r, capacity
+        self.psac_fmt = psac_fmt
         sh = (B, H_kv, capacity)
         u32 = torch.int32
         self.k_code = torch.zeros(sh + (d // 16,), dtype=u32, device=device)
@@ -134,7 +136,9 @@ class Cache:
         self.k_sz = torch.zeros(sh + (d // GROUP,), dtype=u32, device=device)
         self.v_sz = torch.zeros(sh + (d // GROUP,), dtype=u32, device=device)
         self.cidx = torch.zeros(sh, dtype=torch.uint8 if M <= 256 else torch.int16, device=device)
-        self.psac = torch.zeros(sh + (max(r, 1),), dtype=torch.int16, device=device)
+        self.psac = torch.zeros(sh + (max(r, 1),), dtype=torch.int8 if psac_fmt == 1 else torch.int16,
+                                device=device)
+        self.psac_scale = torch.zeros(sh, dtype=torch.int16, device=device) if psac_fmt == 1 else None
         self.centroids = torch.as_tensor(centroids).to(device=device, dtype=torch.int16).contiguous()
         self.P = torch.zeros((H_kv, d, max(r, 1)), dtype=torch.float32, device=device)
         self.w = torch.ones((H_kv, d), dtype=torch.float32, device=device)
@@ -146,7 +150,8 @@ class Cache:
                          self.k_code.data_ptr(), self.v_code.data_ptr(), self.k_sz.data_ptr(),
                          self.v_sz.data_ptr(), self.cidx.data_ptr(),
                          self.psac.data_ptr() if self.r else 0, self.centroids.data_ptr(),
-                         self.P.data_ptr(), self.w.data_ptr(), self.Wg.data_ptr())
+                         self.P.data_ptr(), self.w.data_ptr(), self.Wg.data_ptr(), self.psac_fmt,
+                         self.psac_scale.data_ptr() if self.psac_scale is not None else 0)
 
     def set_fit(self, P, w, Wg):
         if self.r:
@@ -160,13 +165,19 @@ class Cache:
             getattr(self, name).copy_(torch.from_numpy(getattr(pc, name).view("int32")))
         self.cidx.copy_(torch.from_numpy(pc.cidx.view("uint8" if self.M <= 256 else "int16")))
         if self.r:
-            self.psac.copy_(torch.from_numpy(pc.psac.view("int16")))
+            self.psac.copy_(torch.from_numpy(pc.psac.view("int8" if self.psac_fmt == 1 else "int16")))
+            if self.psac_fmt == 1:
+                self.psac_scale.copy_(torch.from_numpy(pc.psac_scale.view("int16")))
 
     def to_host(self):
         """Host numpy copies of the packed streams (library layout)."""
         out = {n: getattr(self, n).cpu().numpy().view("uint32") for n in ("k_code", "v_code", "k_sz", "v_sz")}
         out["cidx"] = self.cidx.cpu().numpy().view("uint8" if self.M <= 256 else "uint16")
-        out["psac"] = self.psac.cpu().numpy().view("uint16")[..., :self.r]
+        if self.psac_fmt == 1:
+            out["psac"] = self.psac.cpu().numpy()[..., :self.r]
+            out["psac_scale"] = self.psac_scale.cpu().numpy().view("uint16")
+        else:
+            out["psac"] = self.psac.cpu().numpy().view("uint16")[..., :self.r]
         return out
 
 

@@ -41,6 +41,7 @@ kv2_status check_cache(const kv2_cache* c, bool need_cache_streams, bool need_fi
   if (c->M > kv2::kMaxCentroids) return fail(KV2_ERR_UNSUPPORTED, "M=%d centroids (max 512)", c->M);
   if (c->r > c->d || (c->r & 1)) return fail(KV2_ERR_UNSUPPORTED, "PSAC rank r=%d (even, <= d)", c->r);
   if (c->capacity % 16) return fail(KV2_ERR_UNSUPPORTED, "capacity %d is not a multiple of 16", c->capacity);
+  if (c->psac_fmt != 0 && c->psac_fmt != 1) return fail(KV2_ERR_INVALID_ARG, "psac_fmt=%d (0: fp16, 1: int8)", c->psac_fmt);
   if (!c->centroids || !aligned16(c->centroids))
     return fail(KV2_ERR_INVALID_ARG, "centroids must be a non-NULL 16-byte aligned pointer");
   if (need_cache_streams) {
@@ -49,6 +50,8 @@ kv2_status check_cache(const kv2_cache* c, bool need_cache_streams, bool need_fi
       if (!p || !aligned16(p)) return fail(KV2_ERR_INVALID_ARG, "cache stream pointer NULL or not 16-byte aligned");
     if (c->r && (!c->psac || !aligned16(c->psac)))
       return fail(KV2_ERR_INVALID_ARG, "psac pointer NULL or not 16-byte aligned");
+    if (c->psac_fmt == 1 && c->r && (!c->psac_scale || !aligned16(c->psac_scale)))
+      return fail(KV2_ERR_INVALID_ARG, "psac_scale pointer NULL or not 16-byte aligned (int8 PSAC format)");
   }
   if (need_fit) {
     if (!c->w || !c->Wg || !aligned16(c->w) || !aligned16(c->Wg))
@@ -87,7 +90,7 @@ const char* kv2_status_string(kv2_status s) {
 
 const char* kv2_last_error(void) { return g_last_error; }
 
-int kv2_version(void) { return 100; }
+int kv2_version(void) { return 101; }
 
 size_t kv2_fit_workspace_size(int H_kv, int d) {
   if (H_kv <= 0 || (d != 64 && d != 128)) return 0;
@@ -151,9 +154,12 @@ kv2_status check_quantize(const kv2_cache* c, const uint16_t* K, const uint16_t*
 
 kv2::QuantizeArgs quantize_args(const kv2_cache* c, const uint16_t* K, const uint16_t* V, int n_new, int pos,
                                 int candidates) {
-  return kv2::QuantizeArgs{K, V, c->B, c->H_kv, c->d, c->M, c->r, c->capacity, n_new, pos, candidates,
-                           c->centroids, c->P, c->w, c->Wg, c->k_code, c->v_code, c->k_sz, c->v_sz,
-                           c->cidx, c->psac};
+  kv2::QuantizeArgs a{K, V, c->B, c->H_kv, c->d, c->M, c->r, c->capacity, n_new, pos, candidates,
+                      c->centroids, c->P, c->w, c->Wg, c->k_code, c->v_code, c->k_sz, c->v_sz,
+                      c->cidx, c->psac};
+  a.psac_fmt = c->psac_fmt;
+  a.psac_scale = c->psac_scale;
+  return a;
 }
 
 // argument checks of a decode call (the cache already checked)

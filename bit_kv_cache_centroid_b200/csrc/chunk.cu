@@ -282,6 +282,8 @@ struct ChunkParams {
   // whose partial results (part) are merged by chunk_merge
   int QP, n_full, pieces;
   float* part;            // [split units][pieces][2][kRows][kPartRow]
+  int psac_fmt;           // 0: fp16 coefficients; 1: int8 codes + fp16 scale per token
+  const uint16_t* psac_scale;
 };
 
 // ---------------------------------------------------------------------------
@@ -310,6 +312,30 @@ __device__ __forceinline__ void load_raw_half(const ChunkParams& p, size_t slot,
 __device__ __forceinline__ void load_psac(const ChunkParams& p, size_t slot, uint4& a0, uint4& a1) {
   a0 = make_uint4(0, 0, 0, 0);
   a1 = make_uint4(0, 0, 0, 0);
+  if (p.psac_fmt == 1) {
+    // int8 codes (r = 8 or 16) and the token's scale: fp16(code * scale)
+    if (p.r == 0) return;
+    const float sc = __half2float(__ushort_as_half(p.psac_scale[slot]));
+    const int8_t* q8 = reinterpret_cast<const int8_t*>(p.psac) + slot * p.r;
+    uint32_t w[4];
+    const uint2 lo = *reinterpret_cast<const uint2*>(q8);
+    w[0] = lo.x; w[1] = lo.y;
+    if (p.r >= 16) {
+      const uint2 hi = *reinterpret_cast<const uint2*>(q8 + 8);
+      w[2] = hi.x; w[3] = hi.y;
+    } else {
+      w[2] = w[3] = 0u;
+    }
+    uint32_t h[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t two = (w[i >> 1] >> (16 * (i & 1))) & 0xffffu;
+      h[i] = pack_f16(float(int8_t(two & 0xff)) * sc, float(int8_t(two >> 8)) * sc);
+    }
+    a0 = make_uint4(h[0], h[1], h[2], h[3]);
+    a1 = make_uint4(h[4], h[5], h[6], h[7]);
+    return;
+  }
   if (p.r >= 8) a0 = *reinterpret_cast<const uint4*>(p.psac + slot * p.r);
   if (p.r >= 16) a1 = *reinterpret_cast<const uint4*>(p.psac + slot * p.r + 8);
 }
@@ -830,6 +856,7 @@ cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t s) {
   ChunkParams p{};
   p.k_code = c.k_code; p.v_code = c.v_code; p.k_sz = c.k_sz; p.v_sz = c.v_sz;
   p.cidx = c.cidx; p.psac = c.psac; p.cent = c.centroids; p.P = c.P;
+  p.psac_fmt = c.psac_fmt; p.psac_scale = c.psac_scale;
   p.Q = a.Q; p.Ks = a.Kself; p.Vs = a.Vself; p.out = a.out;
   p.err = static_cast<int*>(a.ws);
   p.B = c.B; p.H_kv = c.H_kv; p.H_q = a.H_q; p.M = c.M; p.r = c.r; p.cap = c.capacity;

@@ -118,6 +118,21 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// INT8 PSAC coefficients of one token: scale = fp16 round-up of the fp32
+// quotient max|a| / 127, code = clamp(round-half-even(a / scale), -127, 127)
+// (0 when the scale is 0); the coefficient read back is code * scale
+__device__ __forceinline__ void psac_int8(const float* a, int r, int8_t* q, uint16_t* scale_bits) {
+  float amax = 0.0f;
+  for (int i = 0; i < r; ++i) amax = fmaxf(amax, fabsf(a[i]));
+  const uint16_t sb = f16_ru(__fdiv_rn(amax, 127.0f));
+  const float s = f16_to_f32(sb);
+  for (int i = 0; i < r; ++i) {
+    const float v = (s > 0.0f) ? rintf(__fdiv_rn(a[i], s)) : 0.0f;
+    q[i] = static_cast<int8_t>(fminf(fmaxf(v, -127.0f), 127.0f));
+  }
+  *scale_bits = sb;
+}
+
 __device__ __forceinline__ float group_dequant(uint32_t code, const GroupParams& p) {
   return __fmaf_rn(static_cast<float>(code), p.s, p.z);
 }

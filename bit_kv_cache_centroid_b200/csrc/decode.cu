@@ -75,6 +75,8 @@ struct SplitParams {
   int force_timeout;      // wait on copies that are never issued (tests)
   int wait_from;          // first slot the preceding (primary) kernel writes
   int H_kv, H_q, M, r, cap, len, splits, tiles_per_split;
+  int psac_fmt;                 // 0: fp16 coefficients; 1: int8 codes + fp16 scale per token
+  const uint16_t* psac_scale;
 };
 
 // d = a * b + c on two fp16 lanes
@@ -284,13 +286,20 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
       dep_done = true;
     }
     const size_t s0 = base_slot + t0;                      // a multiple of 16
-    mbar_arrive_expect_tx(bar, uint32_t(n16) * uint32_t(2 * NW * 4 + 2 * NG * 4 + Cfg::IDXB + 2 * r));
+    const int ps_bytes = (p.psac_fmt == 1) ? (r ? r + 2 : 0) : 2 * r;   // per token
+    mbar_arrive_expect_tx(bar, uint32_t(n16) * uint32_t(2 * NW * 4 + 2 * NG * 4 + Cfg::IDXB + ps_bytes));
     bulk_g2s(dst + Cfg::kc_off, p.k_code + s0 * NW, n16 * NW * 4, bar);
     bulk_g2s(dst + Cfg::vc_off, p.v_code + s0 * NW, n16 * NW * 4, bar);
     bulk_g2s(dst + Cfg::ks_off, p.k_sz + s0 * NG, n16 * NG * 4, bar);
     bulk_g2s(dst + Cfg::vs_off, p.v_sz + s0 * NG, n16 * NG * 4, bar);
     bulk_g2s(dst + Cfg::ix_off, static_cast<const unsigned char*>(p.cidx) + s0 * Cfg::IDXB, n16 * Cfg::IDXB, bar);
-    if (r) bulk_g2s(dst + Cfg::ps_off, p.psac + s0 * r, n16 * r * 2, bar);
+    if (r && p.psac_fmt == 1) {
+      // int8 codes [kTile][r], then the fp16 scales [kTile], in the PSAC region
+      bulk_g2s(dst + Cfg::ps_off, reinterpret_cast<const int8_t*>(p.psac) + s0 * r, n16 * r, bar);
+      bulk_g2s(dst + Cfg::ps_off + kTile * r, p.psac_scale + s0, n16 * 2, bar);
+    } else if (r) {
+      bulk_g2s(dst + Cfg::ps_off, p.psac + s0 * r, n16 * r * 2, bar);
+    }
     issued = tile + 1;
   };
   if (tid == 0) {
@@ -550,9 +559,22 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
             const uint32_t* kz1 = ksz + t1 * NG;
             const uint32_t* ps0 = reinterpret_cast<const uint32_t*>(cur + Cfg::ps_off) + t0 * (r / 2);
             const uint32_t* ps1 = reinterpret_cast<const uint32_t*>(cur + Cfg::ps_off) + t1 * (r / 2);
-            auto aux_pair = [&](const uint32_t* kz, const uint32_t* ps, int c) -> uint32_t {
+            const bool q8 = p.psac_fmt == 1;
+            float sc0 = 0.0f, sc1 = 0.0f;              // int8 format: the tokens' scales
+            if (q8 && r) {
+              const uint16_t* scl = reinterpret_cast<const uint16_t*>(cur + Cfg::ps_off + kTile * r);
+              sc0 = __half2float(__ushort_as_half(scl[t0]));
+              sc1 = __half2float(__ushort_as_half(scl[t1]));
+            }
+            auto aux_pair = [&](const uint32_t* kz, const uint32_t* ps, int t, float sc, int c) -> uint32_t {
               if (c < NG) return __byte_perm(kz[c], kz[c + 1], 0x7632);   // z_c, z_c+1
-              return (c - NG < r) ? ps[(c - NG) >> 1] : 0u;               // a pair
+              if (c - NG >= r) return 0u;
+              if (!q8) return ps[(c - NG) >> 1];                            // an fp16 pair
+              // int8 pair: fp16(code * scale) of coefficients c - NG, c - NG + 1
+              const uint16_t two = reinterpret_cast<const uint16_t*>(cur + Cfg::ps_off)[(t * r + c - NG) >> 1];
+              const float a0 = float(int8_t(two & 0xff)) * sc, a1 = float(int8_t(two >> 8)) * sc;
+              const __half2 hv = __floats2half2_rn(a0, a1);
+              return *reinterpret_cast<const uint32_t*>(&hv);
             };
             float Ca[NT][4];
 #pragma unroll
@@ -561,8 +583,8 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
               for (int i = 0; i < 4; ++i) Ca[nt][i] = 0.0f;
             for (int x = 0; x < XK; ++x) {
               const int c = 16 * x + 2 * tig;
-              const uint32_t a[4] = {aux_pair(kz0, ps0, c), aux_pair(kz1, ps1, c),
-                                     aux_pair(kz0, ps0, c + 8), aux_pair(kz1, ps1, c + 8)};
+              const uint32_t a[4] = {aux_pair(kz0, ps0, t0, sc0, c), aux_pair(kz1, ps1, t1, sc1, c),
+                                     aux_pair(kz0, ps0, t0, sc0, c + 8), aux_pair(kz1, ps1, t1, sc1, c + 8)};
 #pragma unroll
               for (int nt = 0; nt < NT; ++nt) {
                 const uint2 bb = baux[(x * NT + nt) * 32 + lane];
@@ -1002,7 +1024,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
                  static_cast<const uint16_t*>(a.Q), static_cast<const uint16_t*>(c.centroids), c.P,
                  a.sm_scale * kLog2e, part, static_cast<int*>(a.ws),
                  force ? (1ull << 20) : env_wait_budget(), force, a.wait_from,
-                 c.H_kv, a.H_q, c.M, c.r, c.capacity, a.len, splits, tps};
+                 c.H_kv, a.H_q, c.M, c.r, c.capacity, a.len, splits, tps, c.psac_fmt, c.psac_scale};
   const int G = a.H_q / c.H_kv;
   cudaError_t e;
   if (c.d == 64) e = (c.M > 256) ? launch_g<64, true>(G, sp, c.B, s) : launch_g<64, false>(G, sp, c.B, s);

@@ -34,6 +34,10 @@ struct QuantizeArgs {
   // (b * n_new + t) and head h goes to assign[row * H + h] and nothing is
   // packed (V, P and the cache streams are not read or written)
   int32_t* assign = nullptr;
+  // PSAC storage: 0 = fp16 coefficients in psac; 1 = int8 codes in psac and
+  // one fp16 scale per token in psac_scale
+  int psac_fmt = 0;
+  uint16_t* psac_scale = nullptr;
 };
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s);
 

@@ -42,9 +42,12 @@ struct QCfg {
   static constexpr int KT = kWarps * KPT;        // keys per tile
   static constexpr size_t mu_bytes = size_t(D) * MP * 2;
   static constexpr size_t warp_wk_bytes = size_t(D) * KPT * 4;   // w*k [D][KPT], later e [KPT][D]
-  __host__ __device__ static size_t warp_bytes(int C) { return (warp_wk_bytes + size_t(KPT) * 8 + size_t(KPT) * C * 2 + 15) & ~size_t(15); }
+  // per warp: w*k / e, best (E, rank) per key, candidates, and (int8 PSAC
+  // format only, r8 = r) the fp32 coefficients [KPT][r8] before quantization
+  __host__ __device__ static size_t cand_end(int C) { return (warp_wk_bytes + size_t(KPT) * 8 + size_t(KPT) * C * 2 + 15) & ~size_t(15); }
+  __host__ __device__ static size_t warp_bytes(int C, int r8) { return (cand_end(C) + size_t(KPT) * r8 * 4 + 15) & ~size_t(15); }
   __host__ __device__ static size_t head_bytes(int r) { return mu_bytes + size_t(MP) * 4 + size_t(D) * 4 + size_t(D) * r * 4; }
-  static size_t smem(int C, int r) { return head_bytes(r) + size_t(kWarps) * warp_bytes(C); }
+  static size_t smem(int C, int r, int r8) { return head_bytes(r) + size_t(kWarps) * warp_bytes(C, r8); }
 };
 
 template <int D, int CPL, int KPT>
@@ -58,11 +61,13 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
   float* w_s = nrm_s + MP;                                                    // [D]
   float* P_s = w_s + D;                                                       // [D][r]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  unsigned char* wbase = smem + Cfg::head_bytes(a.r) + size_t(warp) * Cfg::warp_bytes(a.C);
+  const int r8 = (a.psac_fmt == 1) ? a.r : 0;
+  unsigned char* wbase = smem + Cfg::head_bytes(a.r) + size_t(warp) * Cfg::warp_bytes(a.C, r8);
   float* wk_w = reinterpret_cast<float*>(wbase);                              // [D][KPT]
   float* e_w = wk_w;                                                          // [KPT][D] after ranking
   unsigned long long* best_w = reinterpret_cast<unsigned long long*>(wbase + Cfg::warp_wk_bytes);  // [KPT]
   uint16_t* cand_w = reinterpret_cast<uint16_t*>(best_w + KPT);              // [KPT][C]
+  float* psa_w = reinterpret_cast<float*>(wbase + Cfg::cand_end(a.C));         // [KPT][r8]
 
   // a decode launched as this kernel's programmatic dependent may start now;
   // it waits for this grid before reading the slots written here
@@ -367,7 +372,14 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
           for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
           if (lane == ii) mine = v;
         }
-        if (lane < 8 && i0 + lane < a.r) a.psac[slot * a.r + i0 + lane] = f16_rn(mine);
+        if (lane < 8 && i0 + lane < a.r) {
+          if (r8) psa_w[i0 + lane] = mine;
+          else a.psac[slot * a.r + i0 + lane] = f16_rn(mine);
+        }
+      }
+      if (r8) {
+        __syncwarp();
+        if (lane == 0) psac_int8(psa_w, a.r, reinterpret_cast<int8_t*>(a.psac) + slot * a.r, a.psac_scale + slot);
       }
       }
     } else {
@@ -480,7 +492,15 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
       float acc = 0.0f;
 #pragma unroll 8
       for (int c = 0; c < D; ++c) acc = __fmaf_rn(Pcol[c * a.r], e[c], acc);
-      a.psac[slot_of(row_of(k)) * a.r + i] = f16_rn(acc);
+      if (r8) psa_w[k * a.r + i] = acc;
+      else a.psac[slot_of(row_of(k)) * a.r + i] = f16_rn(acc);
+    }
+    if (r8) {
+      __syncwarp();
+      for (int k = lane; k < nk; k += 32) {
+        const size_t slot = slot_of(row_of(k));
+        psac_int8(psa_w + k * a.r, a.r, reinterpret_cast<int8_t*>(a.psac) + slot * a.r, a.psac_scale + slot);
+      }
     }
     }
     }
@@ -491,7 +511,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
 template <int D, int CPL, int KPT>
 cudaError_t launch_cfg(const QuantizeArgs& a, cudaStream_t s) {
   using Cfg = QCfg<D, CPL, KPT>;
-  const size_t smem = Cfg::smem(a.C, a.r);
+  const size_t smem = Cfg::smem(a.C, a.r, a.psac_fmt == 1 ? a.r : 0);
   auto kern = quantize_kernel<D, CPL, KPT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;

@@ -61,7 +61,11 @@ enum { KV2_OUT_F32 = 0, KV2_OUT_BF16 = 1 };
  *                    low half = fp16 scale s, high half = fp16 zero z; the
  *                    dequantized value of code q is fmaf(q, s, z)
  *   cidx           : centroid id per token, uint8 (M <= 256) or uint16 [B][H_kv][capacity]
- *   psac           : fp16 [B][H_kv][capacity][r] PSAC coefficients a = P^T e
+ *   psac           : PSAC coefficients a = P^T e, [B][H_kv][capacity][r]:
+ *                    fp16 (psac_fmt 0), or int8 codes (psac_fmt 1) whose
+ *                    coefficient is code * psac_scale[slot]
+ *   psac_scale     : fp16 [B][H_kv][capacity], one scale per token (psac_fmt 1
+ *                    only; NULL otherwise)
  *   centroids      : fp16 [H_kv][M][d] (read-only; shared by the batch)
  *   P, w, Wg       : fp32 [H_kv][d][r] basis, [H_kv][d] channel sensitivities,
  *                    [H_kv][d/32] group sensitivities, as written by
@@ -81,6 +85,8 @@ typedef struct kv2_cache {
   const float* P;
   const float* w;
   const float* Wg;
+  int32_t psac_fmt;      /* 0: fp16 coefficients; 1: int8 codes + fp16 scale per token */
+  uint16_t* psac_scale;
 } kv2_cache;
 
 /* Human-readable name of a status. Never NULL. */

@@ -69,10 +69,10 @@ def to_dev(x, dtype=None):
     return t.cuda()
 
 
-def host_cache(s: wl.Spec, centroids, capacity=None):
+def host_cache(s: wl.Spec, centroids, capacity=None, psac_fmt=0):
     cap = s.capacity if capacity is None else capacity
     cap = (cap + 15) // 16 * 16
-    return wl.PackedCache.empty(s.B, s.H_kv, s.d, s.M, s.r, cap, centroids)
+    return wl.PackedCache.empty(s.B, s.H_kv, s.d, s.M, s.r, cap, centroids, psac_fmt)
 
 
 def gpu_cache_like(pc, fit=None):
@@ -81,7 +81,7 @@ def gpu_cache_like(pc, fit=None):
     import torch
     import bit_kv_cache_centroid_b200 as kv2
     c = kv2.Cache(pc.B, pc.H_kv, pc.d, pc.M, pc.r, pc.capacity,
-                  torch.from_numpy(pc.centroids.view(np.int16)))
+                  torch.from_numpy(pc.centroids.view(np.int16)), psac_fmt=getattr(pc, "psac_fmt", 0))
     c.load_packed(pc)
     if fit is not None:
         c.set_fit(torch.from_numpy(fit.P), torch.from_numpy(fit.w), torch.from_numpy(fit.Wg))

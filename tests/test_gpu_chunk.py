@@ -191,3 +191,21 @@ def test_bounded_wait_reports_timeout_and_context_survives(orc):
     got, ref = _run(orc, pc, P, 128, Q, Ks, Vs, 64, ws=ws)
     assert int(ws[:4].view(torch.int32).item()) == 0
     assert_attention_close(got, ref, what="after timeout")
+
+
+@pytest.mark.parametrize("M,r,T,length,Nq,F", [
+    (256, 8, 700, 613, 300, 100),
+    (512, 16, 400, 257, 130, 65),
+])
+def test_int8_psac_caches(orc, M, r, T, length, Nq, F):
+    """Int8 PSAC coefficients with per-token fp16 scales; the kernel's PSAC
+    operand is fp16(code * scale), as the oracle takes it."""
+    s = wl.spec("tiny", d=128, H_q=4, H_kv=2, M=M, r=r, T=T, B=1)
+    pc = wl.random_packed_cache(s, T=T, seed=M + r + 11, psac_fmt=1)
+    P = _basis(s, 7)
+    rng = np.random.default_rng(Nq + F + 1)
+    Q = _dense(rng, (1, Nq, 4, 128), 1.5)
+    Ks = _dense(rng, (1, Nq, 2, 128), 1.5)
+    Vs = _dense(rng, (1, Nq, 2, 128))
+    got, ref = _run(orc, pc, P, length, Q, Ks, Vs, F)
+    assert_attention_close(got, ref, what=f"chunk int8 psac M{M} r{r}")

@@ -204,3 +204,31 @@ def test_append_attention_decode_equals_the_two_calls(orc, B, H_q, H_kv, M, r, T
                           caches[1]["cidx"], caches[1]["psac"], pc.centroids)
     ref = orc.decode(host, P, T + n_new, Q.cpu().numpy().view(np.uint16), scale)
     assert_attention_close(outs[1], ref, what=f"append+decode B{B} T{T} n{n_new}")
+
+
+@pytest.mark.parametrize("d,G,M,r,T,length", [
+    (128, 4, 64, 8, 1200, 1100),       # LLM-like table, rank 8
+    (128, 1, 512, 16, 2100, 2049),     # MHA, u16 ids, rank 16
+    (64, 4, 16, 8, 900, 899),          # d = 64
+])
+def test_int8_psac_caches(orc, d, G, M, r, T, length):
+    """Int8 PSAC coefficients with per-token fp16 scales (the oracle reads
+    them back exactly as code * scale)."""
+    s = wl.spec("tiny", d=d, H_kv=2, H_q=2 * G, M=M, r=r, T=T, B=2)
+    pc = wl.random_packed_cache(s, T=T, seed=d + G + M + r + 7, psac_fmt=1)
+    P = _basis(s, 4)
+    rng = np.random.default_rng(T + 1)
+    Q = wl.bf16_bits(rng.standard_normal((s.B, s.H_q, d)).astype(np.float32) * 1.5)
+    got, ref = _decode_both(orc, pc, P, length, Q, 1.0 / np.sqrt(d))
+    assert_attention_close(got, ref, what=f"int8 psac d{d} G{G} M{M} r{r} len{length}")
+
+
+def test_int8_psac_oracle_quantized_cache(orc):
+    """Keys appended by the oracle's quantizer in the int8 PSAC format."""
+    w = wl.make("tiny")
+    s = w.spec
+    f = orc.fit(w.Qhist, s.H_kv, s.r)
+    pc = host_cache(s, w.centroids, psac_fmt=1)
+    orc.quantize(pc, w.K[:, :s.T], w.V[:, :s.T], 0, s.C, f.P, f.w, f.Wg)
+    got, ref = _decode_both(orc, pc, f.P, s.T, w.Qdec, 1.0 / np.sqrt(s.d))
+    assert_attention_close(got, ref, what="int8 psac oracle-quantized")

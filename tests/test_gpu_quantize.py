@@ -131,3 +131,45 @@ def test_capacity_overflow_rejected():
     with pytest.raises(kv2.Kv2Error) as e:
         kv2.kv2_quantize_append(c, K, K, 30, 1)
     assert e.value.status == 3
+
+
+def _run_int8(orc, s, pos, n_tok, C):
+    """The same append in the int8 PSAC format on both sides."""
+    w = wl.make(s.name, **{k: getattr(s, k) for k in ("B", "H_q", "H_kv", "d", "M", "r", "T", "n_new", "n_hist", "Nq")})
+    s = w.spec
+    f = orc.fit(w.Qhist, s.H_kv, s.r)
+    cap = (pos + n_tok + 15) // 16 * 16 + 16
+    ref = host_cache(s, w.centroids, capacity=cap, psac_fmt=1)
+    K = np.ascontiguousarray(w.K[:, :n_tok])
+    V = np.ascontiguousarray(w.V[:, :n_tok])
+    orc.quantize(ref, K, V, pos, C, f.P, f.w, f.Wg)
+    import bit_kv_cache_centroid_b200 as kv2
+    gc = gpu_cache_like(host_cache(s, w.centroids, capacity=cap, psac_fmt=1), fit=f)
+    kv2.kv2_quantize_append(gc, to_dev(K, torch.int16), to_dev(V, torch.int16), pos, C)
+    torch.cuda.synchronize()
+    return ref, gc.to_host()
+
+
+@pytest.mark.parametrize("M,C,r,B,n_tok,pos,exact", [
+    (64, 4, 8, 2, 203, 5, True),      # 8 keys per warp: coefficients from the same fp32 chain
+    (512, 8, 16, 1, 77, 0, True),     # rank 16, u16 ids
+    (64, 4, 8, 8, 1, 4095, False),    # one key per warp (the coefficients' sum order differs)
+    (256, 8, 16, 3, 5, 1, False),
+])
+def test_int8_psac(orc, M, C, r, B, n_tok, pos, exact):
+    """INT8 PSAC format: codes, ids and packed fields as in the fp16 format;
+    the per-token scale and int8 codes bit-exact where the kernel sums the
+    coefficients in the oracle's order, else within 1 fp16 ulp and +-1."""
+    s = wl.spec("tiny", d=128, H_q=4, H_kv=2, M=M, r=r, B=B, T=n_tok, n_new=1, n_hist=64, Nq=0)
+    ref, got = _run_int8(orc, s, pos, n_tok, C)
+    sl = (slice(None), slice(None), slice(pos, pos + n_tok))
+    for name in ("k_code", "v_code", "cidx"):
+        np.testing.assert_array_equal(got[name][sl], getattr(ref, name)[sl], err_msg=name)
+    gq = got["psac"][sl].astype(np.int32)
+    rq = ref.psac[sl][..., :r].astype(np.int32)
+    dsc = f16_ulp_diff(got["psac_scale"][sl], ref.psac_scale[sl])
+    if exact:
+        assert np.array_equal(gq, rq) and dsc.max() == 0
+    else:
+        assert np.abs(gq - rq).max() <= 1 and dsc.max() <= 1
+    assert np.abs(gq).max() <= 127
