@@ -40,7 +40,8 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # workload, from the ncu capture summarised in profiles/decode_split_llm_decode.md;
 # None whenever the kernel has changed since that capture.
 DECODE_SPLIT_TRAFFIC = 242_194_944
-BYTES_PER_TOKEN_HEAD = lambda d, r, M: 2 * (d // 16) * 4 + 2 * (d // 32) * 4 + (1 if M <= 256 else 2) + 2 * r
+BYTES_PER_TOKEN_HEAD = lambda d, r, M, psac_fmt=0: (2 * (d // 16) * 4 + 2 * (d // 32) * 4 + (1 if M <= 256 else 2)
+                                                    + (2 * r if psac_fmt == 0 else (r + 2 if r else 0)))
 
 
 def peaks():
@@ -250,10 +251,43 @@ def run_gpu(args, rank, world):
         "clocks": clk.summary(),
     }
     if not args.skip_extras and rank == 0:
+        result["int8_psac_decode"] = int8_psac_decode(torch, kv2, args, pk, w, s, Q, scale, out)
         result.update(extras(torch, kv2, args, pk))
     if rank == 0 and not args.no_cpu:
         result["cpu_baseline"] = cpu_baseline(args, budget_s=args.cpu_seconds)
     return result
+
+
+def int8_psac_decode(torch, kv2, args, pk, w, s, Q, scale, out):
+    """The LLM decode workload with the PSAC coefficients stored as int8
+    codes and one fp16 scale per token (decode alone, same timing as above)."""
+    dev = torch.device("cuda")
+    P, wt, Wg, en = kv2.kv2_fit_psac_basis(torch.from_numpy(w.Qhist.view(np.int16)).to(dev), s.H_kv, s.r)
+    cache = kv2.Cache(s.B, s.H_kv, s.d, s.M, s.r, s.capacity, torch.from_numpy(w.centroids.view(np.int16)),
+                      psac_fmt=1)
+    cache.set_fit(P, wt, Wg)
+    K = torch.from_numpy(np.ascontiguousarray(w.K[:, :s.T + 1]).view(np.int16)).to(dev)
+    V = torch.from_numpy(np.ascontiguousarray(w.V[:, :s.T + 1]).view(np.int16)).to(dev)
+    kv2.kv2_quantize_append(cache, K, V, 0, s.C)
+    del K, V
+    length = s.T + 1
+    ws = torch.zeros(kv2.kv2_decode_workspace_size(cache, s.H_q, length), dtype=torch.uint8, device=dev)
+    f = lambda: kv2.kv2_attention_decode(cache, length, Q, scale, out_dtype=kv2.KV2_OUT_BF16, out=out, ws=ws)
+    for _ in range(3):
+        f()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        f()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / args.steps
+    per = BYTES_PER_TOKEN_HEAD(s.d, s.r, s.M, 1)
+    gbs = length * s.B * s.H_kv * per / (ms * 1e-3) / 1e9
+    return {"workload": "llm_decode with int8 PSAC coefficients + fp16 scale per token",
+            "bytes_per_token_head": per, "ms": round(ms, 5), "GBps": round(gbs, 1),
+            "hbm_frac": round(gbs / pk["hbm_gbs"], 4)}
 
 
 def extras(torch, kv2, args, pk):
