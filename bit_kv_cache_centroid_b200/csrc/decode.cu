@@ -239,7 +239,9 @@ struct DCfg {
   __host__ __device__ static int tables_bytes(int M, int r) { return bar_off(M, r) + kStages * 8 + 8; }
 };
 
-template <int D, int G, bool U16>
+// Q8: the PSAC coefficients are int8 codes with a per-token fp16 scale
+// (cache format 1), else fp16 (format 0)
+template <int D, int G, bool U16, bool Q8>
 __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
   using Cfg = DCfg<D, G, U16>;
   using CL = Cols<G>;
@@ -286,14 +288,14 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
       dep_done = true;
     }
     const size_t s0 = base_slot + t0;                      // a multiple of 16
-    const int ps_bytes = (p.psac_fmt == 1) ? (r ? r + 2 : 0) : 2 * r;   // per token
+    const int ps_bytes = Q8 ? (r ? r + 2 : 0) : 2 * r;   // per token
     mbar_arrive_expect_tx(bar, uint32_t(n16) * uint32_t(2 * NW * 4 + 2 * NG * 4 + Cfg::IDXB + ps_bytes));
     bulk_g2s(dst + Cfg::kc_off, p.k_code + s0 * NW, n16 * NW * 4, bar);
     bulk_g2s(dst + Cfg::vc_off, p.v_code + s0 * NW, n16 * NW * 4, bar);
     bulk_g2s(dst + Cfg::ks_off, p.k_sz + s0 * NG, n16 * NG * 4, bar);
     bulk_g2s(dst + Cfg::vs_off, p.v_sz + s0 * NG, n16 * NG * 4, bar);
     bulk_g2s(dst + Cfg::ix_off, static_cast<const unsigned char*>(p.cidx) + s0 * Cfg::IDXB, n16 * Cfg::IDXB, bar);
-    if (r && p.psac_fmt == 1) {
+    if (Q8 && r) {
       // int8 codes [kTile][r], then the fp16 scales [kTile], in the PSAC region
       bulk_g2s(dst + Cfg::ps_off, reinterpret_cast<const int8_t*>(p.psac) + s0 * r, n16 * r, bar);
       bulk_g2s(dst + Cfg::ps_off + kTile * r, p.psac_scale + s0, n16 * 2, bar);
@@ -559,7 +561,7 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
             const uint32_t* kz1 = ksz + t1 * NG;
             const uint32_t* ps0 = reinterpret_cast<const uint32_t*>(cur + Cfg::ps_off) + t0 * (r / 2);
             const uint32_t* ps1 = reinterpret_cast<const uint32_t*>(cur + Cfg::ps_off) + t1 * (r / 2);
-            const bool q8 = p.psac_fmt == 1;
+            constexpr bool q8 = Q8;
             float sc0 = 0.0f, sc1 = 0.0f;              // int8 format: the tokens' scales
             if (q8 && r) {
               const uint16_t* scl = reinterpret_cast<const uint16_t*>(cur + Cfg::ps_off + kTile * r);
@@ -920,7 +922,7 @@ size_t split_smem(int M, int r) {
 template <int D, int G, bool U16>
 cudaError_t launch_split(const SplitParams& sp, int B, cudaStream_t s) {
   const size_t smem = split_smem<D, G, U16>(sp.M, sp.r);
-  auto kern = decode_split<D, G, U16>;
+  auto kern = sp.psac_fmt == 1 ? decode_split<D, G, U16, true> : decode_split<D, G, U16, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(sp.splits, B * sp.H_kv);
@@ -957,7 +959,7 @@ cudaError_t launch_g(int G, const SplitParams& sp, int B, cudaStream_t s) {
 template <int D, int G, bool U16>
 int ctas_per_sm_t(int M, int r) {
   const size_t smem = split_smem<D, G, U16>(M, r);
-  auto kern = decode_split<D, G, U16>;
+  auto kern = decode_split<D, G, U16, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess) return 4;
   int n = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, smem) != cudaSuccess || n <= 0) return 4;
