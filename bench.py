@@ -132,6 +132,30 @@ def setup_decode(torch, kv2, s: wl.Spec):
     return w, cache, new_k, new_v, Q, Qh
 
 
+METRIC = "2-bit KV attention: packed-cache GB/s (% of HBM peak); quantize tokens/s"
+
+
+def decode_config(world: int) -> dict:
+    """The workload both arms report (the LLM decode step, weak scaling over
+    independent replicas)."""
+    s = wl.spec("llm_decode")
+    return {"workload": "llm_decode: B=8, H_q=32, H_kv=8, d=128, T=32768 cached, M=64, C=4, r=8, "
+                        "bf16 out; step = append 1 token/seq + decode",
+            "global_batch": s.B * world, "seq_len": s.T + 1, "parallelism": f"replicas x{world}",
+            "l2": "packed cache 237 MB > 126 MB L2 (no flush)"}
+
+
+def max_over_ranks(value: float, device: str = "cuda") -> float:
+    """The largest of the ranks' values (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_gpu(args, rank, world):
     import torch
     import bit_kv_cache_centroid_b200 as kv2
@@ -170,11 +194,7 @@ def run_gpu(args, rank, world):
         t1.record(stream)
         torch.cuda.synchronize()
         time.sleep(0.2)
-    total_ms = t0.elapsed_time(t1)
-    if dist:
-        tt = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(t0.elapsed_time(t1))
     ms_step = total_ms / args.steps
 
     # the two parts on their own (breakdown; the decode alone feeds the roofline)
@@ -231,14 +251,11 @@ def run_gpu(args, rank, world):
     pk, src = peaks()
     achieved = bytes_step / (dec_ms * 1e-3) / 1e9
     result = {
-        "metric": "2-bit KV attention: packed-cache GB/s (% of HBM peak); quantize tokens/s",
+        "metric": METRIC,
         "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "u2+f32", "data": "synthetic",
-        "config": {"workload": "llm_decode: B=8, H_q=32, H_kv=8, d=128, T=32768 cached, M=64, C=4, r=8, "
-                               "bf16 out; step = append 1 token/seq + decode",
-                   "global_batch": s.B * world, "seq_len": length, "parallelism": f"replicas x{world}",
-                   "l2": "packed cache 237 MB > 126 MB L2 (no flush)"},
+        "config": decode_config(world),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
                      "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": DECODE_SPLIT_TRAFFIC,
                      "kernel": "kv2_attention_decode (decode_split + decode_combine)",
@@ -488,16 +505,15 @@ def cpu_baseline(args, budget_s=15.0):
             "seconds": round(t, 2)}
 
 
-def run_reference(args):
+def run_reference(args, world: int = 1):
     r = cpu_baseline(args, budget_s=max(2.0, args.cpu_seconds / max(args.steps, 1)))
     ms = (r["seconds"] * 1e3)
     return {"impl": "reference",
-            "metric": "2-bit KV attention: packed-cache GB/s (% of HBM peak); quantize tokens/s",
-            "value": r["value"], "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "metric": METRIC,
+            "value": r["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "llm_decode: B=8, H_q=32, H_kv=8, d=128, T=32768 cached, M=64, C=4, r=8",
-                       "global_batch": 8, "seq_len": 32769, "parallelism": "none (CPU oracle)"},
+            "config": decode_config(world),
             "cpu_baseline": r,
             "e2e": {"value": r["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -518,8 +534,9 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":
+        # the CPU oracle on the host: rank 0 alone works and prints
         if rank == 0:
-            print(json.dumps(run_reference(args)), flush=True)
+            print(json.dumps(run_reference(args, world)), flush=True)
         return
     if world > 1:
         import datetime
