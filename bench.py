@@ -307,6 +307,31 @@ def int8_psac_decode(torch, kv2, args, pk, w, s, Q, scale, out):
             "hbm_frac": round(gbs / pk["hbm_gbs"], 4)}
 
 
+def retrieval_shift(torch, kv2, w, s, wt, Wg, P):
+    """How often Key quantization moves a query's most-attended token: the
+    quantize workload's keys (cached frame + new tokens, video statistics)
+    quantized with QSAC (C candidates, fitted weights, PSAC rank r) and with
+    the nearest centre (C = 1, unit weights, no PSAC), against the exact keys,
+    for 128 history queries per head."""
+    dev = torch.device("cuda")
+    n = w.K.shape[1]
+    Kd = torch.from_numpy(np.ascontiguousarray(w.K).view(np.int16)).to(dev)
+    Vd = torch.from_numpy(np.ascontiguousarray(w.V).view(np.int16)).to(dev)
+    Qr = torch.from_numpy(np.ascontiguousarray(w.Qhist[None, :128]).view(np.int16)).to(dev)
+    dense = kv2.kv2_dense_top1(Kd, Qr)
+    cap = (n + 15) // 16 * 16
+    res = {"tokens": n, "queries": int(Qr.shape[1] * Qr.shape[2])}
+    for name, C, r in (("qsac_psac", s.C, s.r), ("nearest_centre", 1, 0)):
+        cache = kv2.Cache(1, s.H_kv, s.d, s.M, r, cap, torch.from_numpy(w.centroids.view(np.int16)))
+        if r:
+            cache.set_fit(P, wt, Wg)
+        kv2.kv2_quantize_append(cache, Kd, Vd, 0, C)
+        top = kv2.kv2_decode_top1(cache, n, Qr)
+        res[name] = round(float((top != dense).float().mean().item()), 4)
+    torch.cuda.synchronize()
+    return res
+
+
 def extras(torch, kv2, args, pk):
     """Quantize/append throughput and fit time (same JSON line)."""
     out = {}
@@ -341,6 +366,7 @@ def extras(torch, kv2, args, pk):
                        "GBps": round((rd + wr) / (ms * 1e-3) / 1e9, 2),
                        "hbm_frac": round((rd + wr) / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
                        "ranking_TFMAps": round(fma / (ms * 1e-3) / 1e12, 3)}
+    out["retrieval_shift"] = retrieval_shift(torch, kv2, w, s, wt, Wg, P)
     # QSAC-aware centre fitting on the chunk's new keys (5 iterations)
     X = K[0]
     cent0 = torch.from_numpy(w.centroids.view(np.int16)).to(dev)

@@ -62,6 +62,12 @@ def _load():
     L.kv2_fit_centroids_workspace_size.argtypes = [I, I, I]
     L.kv2_fit_centroids.restype = I
     L.kv2_fit_centroids.argtypes = [P, I, I, I, I, I, P, P, I, P, P, P, S, P]
+    L.kv2_top1_workspace_size.restype = S
+    L.kv2_top1_workspace_size.argtypes = [I, I, I, I]
+    L.kv2_decode_top1.restype = I
+    L.kv2_decode_top1.argtypes = [P, I, P, I, I, P, P, S, P]
+    L.kv2_dense_top1.restype = I
+    L.kv2_dense_top1.argtypes = [P, I, I, I, I, P, I, I, P, P, S, P]
     L.kv2_quantize_append.restype = I
     L.kv2_quantize_append.argtypes = [ctypes.POINTER(kv2_cache), P, P, I, I, I, P]
     L.kv2_decode_workspace_size.restype = S
@@ -101,6 +107,7 @@ def __getattr__(name):
 
 EXPORTS = ["kv2_status_string", "kv2_last_error", "kv2_version", "kv2_fit_workspace_size",
            "kv2_fit_psac_basis", "kv2_fit_centroids_workspace_size", "kv2_fit_centroids",
+           "kv2_top1_workspace_size", "kv2_decode_top1", "kv2_dense_top1",
            "kv2_quantize_append", "kv2_decode_workspace_size",
            "kv2_attention_decode", "kv2_attention_decode_noalloc", "kv2_append_attention_decode",
            "kv2_chunk_workspace_size", "kv2_attention_chunk"]
@@ -222,6 +229,38 @@ def kv2_fit_centroids(X: torch.Tensor, centroids: torch.Tensor, candidates: int,
     _check(_get_lib().kv2_fit_centroids(_ptr(X), n, H_kv, d, M, candidates, _ptr(w), _ptr(Wg), iters,
                                         _ptr(centroids), _ptr(assign), _ptr(ws), ws.numel(), _stream(stream)))
     return centroids, assign[:n]
+
+
+def kv2_top1_workspace_size(B: int, nq: int, H_q: int, length: int) -> int:
+    return int(_get_lib().kv2_top1_workspace_size(B, nq, H_q, length))
+
+
+def kv2_decode_top1(cache: Cache, length: int, Q: torch.Tensor, top1=None, ws=None, stream=None):
+    """Q bf16 [B][nq][H_q][d] (or [B][H_q][d]) -> int32 of Q's leading shape:
+    the cached token with the largest logit."""
+    Q4 = Q if Q.dim() == 4 else Q.unsqueeze(1)
+    B, nq, H_q, _ = Q4.shape
+    top1 = torch.empty((B, nq, H_q), dtype=torch.int32, device=Q.device) if top1 is None else top1
+    need = max(kv2_top1_workspace_size(B, nq, H_q, length), 16)
+    ws = torch.empty(need, dtype=torch.uint8, device=Q.device) if ws is None else ws
+    d = cache.desc()
+    _check(_get_lib().kv2_decode_top1(ctypes.byref(d), length, _ptr(Q4), nq, H_q, _ptr(top1), _ptr(ws),
+                                      ws.numel(), _stream(stream)))
+    return top1 if Q.dim() == 4 else top1[:, 0]
+
+
+def kv2_dense_top1(K: torch.Tensor, Q: torch.Tensor, top1=None, ws=None, stream=None):
+    """K bf16 [B][len][H_kv][d], Q bf16 [B][nq][H_q][d] (or [B][H_q][d]) ->
+    int32: the key with the largest q . k."""
+    B, length, H_kv, d = K.shape
+    Q4 = Q if Q.dim() == 4 else Q.unsqueeze(1)
+    nq, H_q = Q4.shape[1], Q4.shape[2]
+    top1 = torch.empty((B, nq, H_q), dtype=torch.int32, device=Q.device) if top1 is None else top1
+    need = max(kv2_top1_workspace_size(B, nq, H_q, length), 16)
+    ws = torch.empty(need, dtype=torch.uint8, device=Q.device) if ws is None else ws
+    _check(_get_lib().kv2_dense_top1(_ptr(K), B, length, H_kv, d, _ptr(Q4), nq, H_q, _ptr(top1), _ptr(ws),
+                                     ws.numel(), _stream(stream)))
+    return top1 if Q.dim() == 4 else top1[:, 0]
 
 
 def kv2_quantize_append(cache: Cache, K: torch.Tensor, V: torch.Tensor, pos: int,

@@ -14,7 +14,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OBJDIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libkv2.so")
-SOURCES = ["api.cu", "quantize.cu", "decode.cu", "decode_noalloc.cu", "fit.cu", "chunk.cu", "fit_centroids.cu"]
+SOURCES = ["api.cu", "quantize.cu", "decode.cu", "decode_noalloc.cu", "fit.cu", "chunk.cu", "fit_centroids.cu", "top1.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]

@@ -112,6 +112,38 @@ kv2_status kv2_fit_psac_basis(const uint16_t* Qhist, int n, int H_q, int H_kv, i
   return cuda_status(kv2::launch_fit(a, static_cast<cudaStream_t>(stream)), "fit launch");
 }
 
+size_t kv2_top1_workspace_size(int B, int nq, int H_q, int len) {
+  if (B <= 0 || nq <= 0 || H_q <= 0 || len < 0) return 0;
+  return kv2::top1_workspace_bytes(B, nq, H_q, len);
+}
+
+kv2_status kv2_decode_top1(const kv2_cache* c, int len, const uint16_t* Q, int nq, int H_q, int32_t* top1,
+                           void* ws, size_t ws_bytes, void* stream) {
+  kv2_status st = check_cache(c, true, false);
+  if (st != KV2_OK) return st;
+  if (H_q <= 0 || H_q % c->H_kv) return fail(KV2_ERR_UNSUPPORTED, "top1: H_q=%d not a multiple of H_kv=%d", H_q, c->H_kv);
+  if (len < 0 || len > c->capacity) return fail(KV2_ERR_CAPACITY, "top1: len=%d outside 0..capacity=%d", len, c->capacity);
+  if (nq <= 0) return fail(KV2_ERR_INVALID_ARG, "top1: nq=%d", nq);
+  if (!Q || !top1 || !ws || !aligned16(ws)) return fail(KV2_ERR_INVALID_ARG, "top1: NULL or misaligned pointer");
+  const size_t need = kv2::top1_workspace_bytes(c->B, nq, H_q, len);
+  if (ws_bytes < need) return fail(KV2_ERR_WORKSPACE, "top1: workspace %zu < %zu bytes", ws_bytes, need);
+  kv2::Top1Args a{c, Q, nullptr, c->B, nq, H_q, c->H_kv, c->d, len, top1, ws};
+  return cuda_status(kv2::launch_top1(a, static_cast<cudaStream_t>(stream)), "top1 launch");
+}
+
+kv2_status kv2_dense_top1(const uint16_t* K, int B, int len, int H_kv, int d, const uint16_t* Q, int nq, int H_q,
+                          int32_t* top1, void* ws, size_t ws_bytes, void* stream) {
+  if (B <= 0 || nq <= 0 || H_kv <= 0 || len < 0 || d <= 0 || d > 1024)
+    return fail(KV2_ERR_INVALID_ARG, "dense_top1: B=%d H_kv=%d len=%d d=%d", B, H_kv, len, d);
+  if (H_q <= 0 || H_q % H_kv) return fail(KV2_ERR_UNSUPPORTED, "dense_top1: H_q=%d not a multiple of H_kv=%d", H_q, H_kv);
+  if ((len && !K) || !Q || !top1 || !ws || !aligned16(ws))
+    return fail(KV2_ERR_INVALID_ARG, "dense_top1: NULL or misaligned pointer");
+  const size_t need = kv2::top1_workspace_bytes(B, nq, H_q, len);
+  if (ws_bytes < need) return fail(KV2_ERR_WORKSPACE, "dense_top1: workspace %zu < %zu bytes", ws_bytes, need);
+  kv2::Top1Args a{nullptr, Q, K, B, nq, H_q, H_kv, d, len, top1, ws};
+  return cuda_status(kv2::launch_top1(a, static_cast<cudaStream_t>(stream)), "dense_top1 launch");
+}
+
 size_t kv2_fit_centroids_workspace_size(int H_kv, int d, int M) {
   if (H_kv <= 0 || (d != 64 && d != 128) || M < 1 || M > 512) return 0;
   return kv2::fit_centroids_workspace_bytes(H_kv, d, M);

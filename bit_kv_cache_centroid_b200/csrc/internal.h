@@ -52,6 +52,19 @@ struct FitCentroidsArgs {
   void* ws;            // fit_centroids_workspace_bytes(H, D, M)
 };
 size_t fit_centroids_workspace_bytes(int H, int D, int M);
+
+// Most-attended token per query (retrieval analysis): over the packed cache
+// (c set, K null) or over dense bf16 keys K [B][len][H_kv][d] (c null).
+struct Top1Args {
+  const kv2_cache* c;
+  const uint16_t* Q;   // bf16 [B][nq][H_q][d]
+  const uint16_t* K;
+  int B, nq, H_q, H_kv, d, len;
+  int32_t* top1;       // [B][nq][H_q]
+  void* ws;            // top1_workspace_bytes(B, nq, H_q, len)
+};
+size_t top1_workspace_bytes(int B, int nq, int H_q, int len);
+cudaError_t launch_top1(const Top1Args& a, cudaStream_t s);
 cudaError_t launch_fit_centroids(const FitCentroidsArgs& a, cudaStream_t s);
 
 // Decode attention.

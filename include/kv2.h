@@ -156,6 +156,35 @@ kv2_status kv2_fit_centroids(const uint16_t* X, int n, int H_kv, int d, int M, i
                              int32_t* assign, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Workspace for kv2_decode_top1 / kv2_dense_top1, in bytes:
+ * B*nq*H_q*ceil(len/4096)*8. Returns 0 for invalid sizes.
+ */
+size_t kv2_top1_workspace_size(int B, int nq, int H_q, int len);
+
+/*
+ * kv2_decode_top1 — the most-attended cached token of each query: the index
+ * of the largest logit q . khat_t + (q P) . a_t over tokens [0, len) of the
+ * packed cache (the logit decode uses, before scaling), computed in fp32 with
+ * the channels in order; ties go to the lower index; -1 when len = 0. With
+ * kv2_dense_top1 on the original keys it measures the retrieval shift that
+ * Key quantization causes (article introduction and Table 1: which
+ * temporal-spatial tokens a Query selects). Not on the attention hot path.
+ * Q: bf16 [B][nq][H_q][d] (nq queries per sequence); top1: int32
+ * [B][nq][H_q] (device, written); ws: kv2_top1_workspace_size(B, nq, H_q, len)
+ * bytes.
+ */
+kv2_status kv2_decode_top1(const kv2_cache* cache, int len, const uint16_t* Q, int nq, int H_q, int32_t* top1,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * kv2_dense_top1 — the same over dense bf16 keys K [B][len][H_kv][d]:
+ * the index of the largest q . k_t (fp32, channels in order, ties to the
+ * lower index).
+ */
+kv2_status kv2_dense_top1(const uint16_t* K, int B, int len, int H_kv, int d, const uint16_t* Q, int nq, int H_q,
+                          int32_t* top1, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * kv2_quantize_append — QSAC centroid assignment, INT2 residual/value
  * packing and PSAC coefficients for n_new new tokens of every (batch, KV
  * head), written to slots [pos, pos + n_new) (article "1. QSAC", "2. PSAC").

@@ -257,3 +257,40 @@ def decode_logits(pc, P: np.ndarray, b: int, h: int, length: int, q: np.ndarray)
                            _ptr(pc.k_code), _ptr(pc.k_sz), _ptr(pc.cidx), *_psac_args(pc),
                            _ptr(_c(pc.centroids, np.uint16)), _ptr(Pp), length, _ptr(q), _ptr(out))
     return out
+
+
+def bf16_f64(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> their exact values in fp64."""
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def decode_top1(pc, P: np.ndarray, length: int, Q: np.ndarray):
+    """Most-attended cached token per query: argmax over t < length of the
+    fp64 logit q . khat_t + (q P) . a_t (first index among equal maxima), and
+    the logits themselves. Q bf16 [B][nq][H_q][d] -> (int [B][nq][H_q],
+    fp64 [B][nq][H_q][length])."""
+    Q = _c(Q, np.uint16)
+    B, nq, Hq, d = Q.shape
+    G = Hq // pc.H_kv
+    lg = np.zeros((B, nq, Hq, max(length, 1)), np.float64)
+    for b in range(B):
+        for i in range(nq):
+            for hq in range(Hq):
+                q = bf16_f64(Q[b, i, hq])
+                if length:
+                    lg[b, i, hq, :length] = decode_logits(pc, P, b, hq // G, length, q)
+    top = np.argmax(lg[..., :length], axis=-1) if length else np.full((B, nq, Hq), -1)
+    return top, lg[..., :length]
+
+
+def dense_top1(K: np.ndarray, Q: np.ndarray):
+    """Most-attended key per query over dense bf16 keys K [B][len][H_kv][d]:
+    argmax of the fp64 q . k (first index among equal maxima), and the logits."""
+    K = bf16_f64(_c(K, np.uint16))
+    Qv = bf16_f64(_c(Q, np.uint16))
+    B, n, Hkv, d = K.shape
+    G = Qv.shape[2] // Hkv
+    Kg = np.repeat(K, G, axis=2)                       # [B][len][H_q][d]
+    lg = np.einsum("bihd,bthd->biht", Qv, Kg)
+    return np.argmax(lg, axis=-1), lg
+
