@@ -67,11 +67,12 @@ def _declare(L):
     L.or_f32_from_bf16.restype = ctypes.c_float
     L.or_codec_group.argtypes = [_P, _I, _P, _P, _P, _P]
     L.or_fit.argtypes = [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P]
-    L.or_quantize.argtypes = [_I] * 6 + [_P, _P, _I, _I, _I, _P, _P, _P, _P] + [_P] * 6 + [_I, _P] + [_P] * 3
-    L.or_decode.argtypes = [_I] * 6 + [_P] * 6 + [_I, _P] + [_P] * 2 + [_I, _P, _I, ctypes.c_double, _P]
-    L.or_chunk.argtypes = ([_I] * 6 + [_P] * 6 + [_I, _P] + [_P] * 2 + [_I, _P, _I, _I, _P, _P, _I,
+    L.or_quantize.argtypes = ([_I] * 6 + [_P, _P, _I, _I, _I, _P, _P, _P, _P] + [_P] * 6 + [_I, _P, _P, _I]
+                              + [_P] * 3)
+    L.or_decode.argtypes = [_I] * 6 + [_P] * 6 + [_I, _P, _P, _I] + [_P] * 2 + [_I, _P, _I, ctypes.c_double, _P]
+    L.or_chunk.argtypes = ([_I] * 6 + [_P] * 6 + [_I, _P, _P, _I] + [_P] * 2 + [_I, _P, _I, _I, _P, _P, _I,
                                                   ctypes.c_double, _P, _I, _P])
-    L.or_decode_logits.argtypes = [_I] * 7 + [_P] * 4 + [_I, _P] + [_P] * 2 + [_I, _P, _P]
+    L.or_decode_logits.argtypes = [_I] * 7 + [_P] * 4 + [_I, _P, _P, _I] + [_P] * 2 + [_I, _P, _P]
     L.or_fit_centroids.argtypes = [_I] * 5 + [_P, _P, _P, _I, _P, _P]
     for f in (L.or_codec_group, L.or_fit, L.or_quantize, L.or_decode, L.or_chunk,
               L.or_decode_logits, L.or_fit_centroids):
@@ -197,12 +198,16 @@ def fit_centroids(X: np.ndarray, M: int, C: int, w: np.ndarray, Wg: np.ndarray,
 
 
 def _psac_args(pc):
-    """(coefficients, format, per-token scales) of a packed cache: format 0 =
-    fp16 [r], 1 = int8 [r] with one fp16 scale per token."""
+    """(coefficients, format, per-token scales, block table, page tokens) of
+    a packed cache: format 0 = fp16 [r], 1 = int8 [r] with one fp16 scale per
+    token; a paged cache holds its streams as a pool of pages addressed
+    through the block table [B][capacity / page]."""
     fmt = getattr(pc, "psac_fmt", 0)
     psac = pc.psac if pc.r else np.zeros(1, np.uint16)
     sc = pc.psac_scale if (fmt == 1 and pc.r) else np.zeros(1, np.uint16)
-    return _ptr(psac), fmt, _ptr(sc)
+    table = getattr(pc, "table", None)
+    return (_ptr(psac), fmt, _ptr(sc), _ptr(_c(table, np.int32)) if table is not None else None,
+            int(getattr(pc, "page", 0)))
 
 
 def _cache_args(pc):

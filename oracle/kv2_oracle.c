@@ -382,6 +382,16 @@ static void qsac_tables(const uint16_t* cent, const float* wh, int h, int M, int
     }
 }
 
+/* Slot of token t of (sequence b, KV head h): contiguous streams
+ * [B][Hkv][cap], or a pool of pages [pages][Hkv][page] addressed through the
+ * block table (a page holds `page` consecutive tokens of one sequence). */
+static size_t slot_at(int Hkv, int cap, const int32_t* table, int page, int b, int h, int t)
+{
+    if (!table) return ((size_t)b * Hkv + h) * cap + (size_t)t;
+    int32_t pg = table[(size_t)b * (cap / page) + t / page];
+    return ((size_t)pg * Hkv + h) * page + (size_t)(t % page);
+}
+
 /* INT8 PSAC coefficients with one fp16 scale per token (the compensation
  * information stored compactly, article "2. PSAC" and the compression count
  * of the evaluation). Reading taken: symmetric, scale = fp16 round-up of the
@@ -432,9 +442,11 @@ int or_quantize(int B, int Hkv, int d, int M, int r, int cap,
                 const uint16_t* cent, const float* P, const float* w, const float* Wg,
                 uint32_t* k_code, uint32_t* v_code, uint32_t* k_sz, uint32_t* v_sz,
                 void* cidx, uint16_t* psac, int psac_fmt, uint16_t* psac_scale,
+                const int32_t* table, int page,
                 int32_t* cand_out, float* score_out, float* E_out)
 {
-    if (d % GROUP || C < 1 || C > M || pos < 0 || pos + n_new > cap || (psac_fmt != 0 && psac_fmt != 1)) return 1;
+    if (d % GROUP || C < 1 || C > M || pos < 0 || pos + n_new > cap || (psac_fmt != 0 && psac_fmt != 1) ||
+        (table && (page <= 0 || cap % page))) return 1;
     int ng = d / GROUP, nw = d / 16;
     float* mu = (float*)malloc((size_t)M * d * sizeof(float));
     float* nrm = (float*)malloc((size_t)M * sizeof(float));
@@ -455,7 +467,7 @@ int or_quantize(int B, int Hkv, int d, int M, int r, int cap,
         for (int b = 0; b < B; ++b) {
             for (int t = 0; t < n_new; ++t) {
                 size_t in = (((size_t)b * n_new + t) * Hkv + h) * d;
-                size_t slot = ((size_t)b * Hkv + h) * cap + (size_t)(pos + t);
+                size_t slot = slot_at(Hkv, cap, table, page, b, h, pos + t);
                 size_t dbg = (((size_t)b * n_new + t) * Hkv + h);
                 for (int c = 0; c < d; ++c) k[c] = or_f32_from_bf16(K[in + c]);
                 int chosen = qsac_choose(k, wh, Wg + (size_t)h * ng, mu, nrm, M, C, d, wk, score, cand, used, x,
@@ -584,7 +596,10 @@ typedef struct {
     const float* P;
     int psac_fmt;                 /* 0: fp16 [r]; 1: int8 [r] + fp16 scale per token */
     const uint16_t* psac_scale;
+    const int32_t* table;         /* paged: page ids [B][cap / page]; NULL: contiguous */
+    int page;                     /* tokens per page (paged) */
 } or_cache;
+
 
 /* PSAC coefficient i of a cached token, exact: the stored fp16 value, or
  * code * scale for the int8 format */
@@ -612,7 +627,7 @@ static void dequant_exact(const or_cache* c, size_t slot, double* kh, double* vh
     const uint32_t* kw = c->k_code + slot * (d / 16);
     const uint32_t* vw = c->v_code + slot * (d / 16);
     int j = cache_idx(c, slot);
-    int h = (int)((slot / (size_t)c->cap) % (size_t)c->Hkv);
+    int h = (int)((slot / (size_t)(c->table ? c->page : c->cap)) % (size_t)c->Hkv);
     for (int g = 0; g < ng; ++g) {
         uint32_t ks = c->k_sz[slot * ng + g], vs = c->v_sz[slot * ng + g];
         double s = or_f32_from_f16((uint16_t)(ks & 0xffff)), z = or_f32_from_f16((uint16_t)(ks >> 16));
@@ -634,7 +649,7 @@ static void dequant_operand(const or_cache* c, size_t slot, double* kh, double* 
     const uint32_t* kw = c->k_code + slot * (d / 16);
     const uint32_t* vw = c->v_code + slot * (d / 16);
     int j = cache_idx(c, slot);
-    int h = (int)((slot / (size_t)c->cap) % (size_t)c->Hkv);
+    int h = (int)((slot / (size_t)(c->table ? c->page : c->cap)) % (size_t)c->Hkv);
     for (int g = 0; g < ng; ++g) {
         uint32_t ks = c->k_sz[slot * ng + g], vs = c->v_sz[slot * ng + g];
         double s = or_f32_from_f16((uint16_t)(ks & 0xffff)), z = or_f32_from_f16((uint16_t)(ks >> 16));
@@ -665,11 +680,13 @@ static void softmax_combine(const double* logit, const double* vals, int n, int 
 int or_decode(int B, int Hkv, int d, int M, int r, int cap,
               const uint32_t* k_code, const uint32_t* v_code, const uint32_t* k_sz,
               const uint32_t* v_sz, const void* cidx, const uint16_t* psac,
-              int psac_fmt, const uint16_t* psac_scale, const uint16_t* cent, const float* P,
+              int psac_fmt, const uint16_t* psac_scale, const int32_t* table, int page,
+              const uint16_t* cent, const float* P,
               int len, const uint16_t* Q, int Hq, double sm_scale, double* out)
 {
     if (Hq % Hkv || len < 0 || len > cap) return 1;
-    or_cache c = {B, Hkv, d, M, r, cap, k_code, v_code, k_sz, v_sz, cidx, psac, cent, P, psac_fmt, psac_scale};
+    or_cache c = {B, Hkv, d, M, r, cap, k_code, v_code, k_sz, v_sz, cidx, psac, cent, P, psac_fmt, psac_scale,
+                  table, page};
     int G = Hq / Hkv;
     double* logit = (double*)malloc(((size_t)len + 1) * sizeof(double));
     double* vals = (double*)malloc(((size_t)len + 1) * d * sizeof(double));
@@ -686,7 +703,7 @@ int or_decode(int B, int Hkv, int d, int M, int r, int cap,
                 for (int ch = 0; ch < d; ++ch) u[i] += q[ch] * (double)P[((size_t)h * d + ch) * r + i];
             }
             for (int t = 0; t < len; ++t) {
-                size_t slot = ((size_t)b * Hkv + h) * cap + t;
+                size_t slot = slot_at(Hkv, cap, table, page, b, h, t);
                 dequant_exact(&c, slot, kh, vals + (size_t)t * d);
                 double acc = 0.0;
                 for (int ch = 0; ch < d; ++ch) acc += q[ch] * kh[ch];
@@ -707,12 +724,14 @@ int or_decode(int B, int Hkv, int d, int M, int r, int cap,
 int or_chunk(int B, int Hkv, int d, int M, int r, int cap,
              const uint32_t* k_code, const uint32_t* v_code, const uint32_t* k_sz,
              const uint32_t* v_sz, const void* cidx, const uint16_t* psac,
-             int psac_fmt, const uint16_t* psac_scale, const uint16_t* cent, const float* P, int len,
+             int psac_fmt, const uint16_t* psac_scale, const int32_t* table, int page,
+             const uint16_t* cent, const float* P, int len,
              const uint16_t* Q, int Hq, int Nq, const uint16_t* Kself, const uint16_t* Vself,
              int frame_tokens, double sm_scale, const int32_t* rows, int nrows, double* out)
 {
     if (Hq % Hkv || len < 0 || len > cap || frame_tokens <= 0) return 1;
-    or_cache c = {B, Hkv, d, M, r, cap, k_code, v_code, k_sz, v_sz, cidx, psac, cent, P, psac_fmt, psac_scale};
+    or_cache c = {B, Hkv, d, M, r, cap, k_code, v_code, k_sz, v_sz, cidx, psac, cent, P, psac_fmt, psac_scale,
+                  table, page};
     int G = Hq / Hkv;
     size_t nmax = (size_t)len + (size_t)Nq + 1;
     double* logit = (double*)malloc(nmax * sizeof(double));
@@ -732,7 +751,7 @@ int or_chunk(int B, int Hkv, int d, int M, int r, int cap,
         }
         size_t n = 0;
         for (int t = 0; t < len; ++t, ++n) {
-            size_t slot = ((size_t)b * Hkv + h) * cap + t;
+            size_t slot = slot_at(Hkv, cap, table, page, b, h, t);
             dequant_operand(&c, slot, kh, vals + n * d);
             double acc = 0.0;
             for (int ch = 0; ch < d; ++ch) acc += q[ch] * kh[ch];
@@ -761,9 +780,11 @@ int or_chunk(int B, int Hkv, int d, int M, int r, int cap,
 int or_decode_logits(int Hkv, int d, int M, int r, int cap, int b, int h,
                      const uint32_t* k_code, const uint32_t* k_sz, const void* cidx,
                      const uint16_t* psac, int psac_fmt, const uint16_t* psac_scale,
+                     const int32_t* table, int page,
                      const uint16_t* cent, const float* P, int len, const double* q, double* out)
 {
-    or_cache c = {b + 1, Hkv, d, M, r, cap, k_code, k_code, k_sz, k_sz, cidx, psac, cent, P, psac_fmt, psac_scale};
+    or_cache c = {b + 1, Hkv, d, M, r, cap, k_code, k_code, k_sz, k_sz, cidx, psac, cent, P, psac_fmt, psac_scale,
+                  table, page};
     double* kh = (double*)malloc((size_t)d * sizeof(double));
     double* vh = (double*)malloc((size_t)d * sizeof(double));
     double* u = (double*)malloc(((size_t)r + 1) * sizeof(double));
@@ -772,7 +793,7 @@ int or_decode_logits(int Hkv, int d, int M, int r, int cap, int b, int h,
         for (int ch = 0; ch < d; ++ch) u[i] += q[ch] * (double)P[((size_t)h * d + ch) * r + i];
     }
     for (int t = 0; t < len; ++t) {
-        size_t slot = ((size_t)b * Hkv + h) * cap + t;
+        size_t slot = slot_at(Hkv, cap, table, page, b, h, t);
         dequant_exact(&c, slot, kh, vh);
         double acc = 0.0;
         for (int ch = 0; ch < d; ++ch) acc += q[ch] * kh[ch];

@@ -337,6 +337,8 @@ class PackedCache:
     centroids: np.ndarray
     psac_fmt: int = 0
     psac_scale: np.ndarray | None = None
+    table: np.ndarray | None = None    # paged: page ids [B][capacity / page]
+    page: int = 0                       # tokens per page (paged)
 
     @staticmethod
     def empty(B, H_kv, d, M, r, capacity, centroids, psac_fmt: int = 0):
@@ -351,6 +353,30 @@ class PackedCache:
             np.zeros((B, H_kv, cap, max(r, 1)), np.int8 if psac_fmt == 1 else np.uint16),
             centroids, psac_fmt,
             np.zeros((B, H_kv, cap), np.uint16) if psac_fmt == 1 else None)
+
+
+def to_paged(pc: PackedCache, page: int, n_pages: int, seed: int = 0) -> PackedCache:
+    """The same packed cache stored as a pool of n_pages pages of `page`
+    tokens (streams [n_pages][H_kv][page][...]) in a seeded random order,
+    addressed through a block table [B][capacity / page]; pages not in the
+    table hold random bytes."""
+    assert pc.capacity % page == 0
+    pps = pc.capacity // page
+    assert n_pages >= pc.B * pps
+    rng = np.random.default_rng(seed)
+    table = rng.permutation(n_pages)[:pc.B * pps].astype(np.int32).reshape(pc.B, pps)
+
+    def pool(a):
+        if a is None:
+            return None
+        out = rng.integers(0, 255, (n_pages, pc.H_kv, page) + a.shape[3:]).astype(a.dtype)
+        for b in range(pc.B):
+            for i in range(pps):
+                out[table[b, i]] = a[b, :, i * page:(i + 1) * page]
+        return out
+    return PackedCache(pc.B, pc.H_kv, pc.d, pc.M, pc.r, pc.capacity, pool(pc.k_code), pool(pc.v_code),
+                       pool(pc.k_sz), pool(pc.v_sz), pool(pc.cidx), pool(pc.psac), pc.centroids,
+                       pc.psac_fmt, pool(pc.psac_scale), table, page)
 
 
 def random_packed_cache(s: Spec, T: int | None = None, seed: int | None = None,
