@@ -15,6 +15,7 @@ from __future__ import annotations
 import ctypes
 import os
 
+import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -42,7 +43,8 @@ class kv2_cache(ctypes.Structure):
                 ("cidx", ctypes.c_void_p), ("psac", ctypes.c_void_p),
                 ("centroids", ctypes.c_void_p), ("P", ctypes.c_void_p),
                 ("w", ctypes.c_void_p), ("Wg", ctypes.c_void_p),
-                ("psac_fmt", ctypes.c_int32), ("psac_scale", ctypes.c_void_p)]
+                ("psac_fmt", ctypes.c_int32), ("psac_scale", ctypes.c_void_p),
+                ("block_table", ctypes.c_void_p), ("page_tokens", ctypes.c_int32)]
 
 
 def _load():
@@ -131,12 +133,25 @@ class Cache:
     """Device buffers of one packed cache (layout of include/kv2.h) plus the
     read-only centroid table and fitted statistics it points to."""
 
-    def __init__(self, B, H_kv, d, M, r, capacity, centroids, device="cuda", psac_fmt=0):
+    def __init__(self, B, H_kv, d, M, r, capacity, centroids, device="cuda", psac_fmt=0,
+                 page_tokens=0, num_pages=0):
+        """page_tokens > 0: a paged cache, its streams a pool of num_pages pages
+        of page_tokens tokens; block_table [B][capacity / page_tokens] (int32,
+        device) maps each sequence's pages (initially pages in order)."""
         if capacity % 16:
             raise ValueError("capacity must be a multiple of 16")
         self.B, self.H_kv, self.d, self.M, self.r, self.capacity = B, H_kv, d, M, r, capacity
         self.psac_fmt = psac_fmt
-        sh = (B, H_kv, capacity)
+        self.page_tokens = page_tokens
+        if page_tokens:
+            pps = capacity // page_tokens
+            num_pages = num_pages or B * pps
+            sh = (num_pages, H_kv, page_tokens)
+            self.block_table = torch.arange(B * pps, dtype=torch.int32, device=device).remainder(num_pages) \
+                .view(B, pps).contiguous()
+        else:
+            sh = (B, H_kv, capacity)
+            self.block_table = None
         u32 = torch.int32
         self.k_code = torch.zeros(sh + (d // 16,), dtype=u32, device=device)
         self.v_code = torch.zeros(sh + (d // 16,), dtype=u32, device=device)
@@ -158,7 +173,9 @@ class Cache:
                          self.v_sz.data_ptr(), self.cidx.data_ptr(),
                          self.psac.data_ptr() if self.r else 0, self.centroids.data_ptr(),
                          self.P.data_ptr(), self.w.data_ptr(), self.Wg.data_ptr(), self.psac_fmt,
-                         self.psac_scale.data_ptr() if self.psac_scale is not None else 0)
+                         self.psac_scale.data_ptr() if self.psac_scale is not None else 0,
+                         self.block_table.data_ptr() if self.block_table is not None else 0,
+                         self.page_tokens)
 
     def set_fit(self, P, w, Wg):
         if self.r:
@@ -175,6 +192,8 @@ class Cache:
             self.psac.copy_(torch.from_numpy(pc.psac.view("int8" if self.psac_fmt == 1 else "int16")))
             if self.psac_fmt == 1:
                 self.psac_scale.copy_(torch.from_numpy(pc.psac_scale.view("int16")))
+        if self.block_table is not None and getattr(pc, "table", None) is not None:
+            self.block_table.copy_(torch.from_numpy(np.ascontiguousarray(pc.table, dtype=np.int32)))
 
     def to_host(self):
         """Host numpy copies of the packed streams (library layout)."""

@@ -42,6 +42,9 @@ kv2_status check_cache(const kv2_cache* c, bool need_cache_streams, bool need_fi
   if (c->r > c->d || (c->r & 1)) return fail(KV2_ERR_UNSUPPORTED, "PSAC rank r=%d (even, <= d)", c->r);
   if (c->capacity % 16) return fail(KV2_ERR_UNSUPPORTED, "capacity %d is not a multiple of 16", c->capacity);
   if (c->psac_fmt != 0 && c->psac_fmt != 1) return fail(KV2_ERR_INVALID_ARG, "psac_fmt=%d (0: fp16, 1: int8)", c->psac_fmt);
+  if (c->block_table && (c->page_tokens < 128 || c->page_tokens % 128 || c->capacity % c->page_tokens))
+    return fail(KV2_ERR_UNSUPPORTED, "paged cache: page_tokens=%d (a multiple of 128 dividing capacity %d)",
+                c->page_tokens, c->capacity);
   if (!c->centroids || !aligned16(c->centroids))
     return fail(KV2_ERR_INVALID_ARG, "centroids must be a non-NULL 16-byte aligned pointer");
   if (need_cache_streams) {
@@ -191,6 +194,8 @@ kv2::QuantizeArgs quantize_args(const kv2_cache* c, const uint16_t* K, const uin
                       c->cidx, c->psac};
   a.psac_fmt = c->psac_fmt;
   a.psac_scale = c->psac_scale;
+  a.table = c->block_table;
+  a.page = c->page_tokens;
   return a;
 }
 

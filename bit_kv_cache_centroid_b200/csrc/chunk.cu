@@ -284,6 +284,8 @@ struct ChunkParams {
   float* part;            // [split units][pieces][2][kRows][kPartRow]
   int psac_fmt;           // 0: fp16 coefficients; 1: int8 codes + fp16 scale per token
   const uint16_t* psac_scale;
+  const int32_t* table;   // paged cache: block table [B][cap / page] (null: contiguous)
+  int page;
 };
 
 // ---------------------------------------------------------------------------
@@ -570,11 +572,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
     // their 16-byte stores then fall on 8 distinct swizzled bank groups
     const int pt = tid - kProdWarp0 * 32;
     const int row = (pt >> 5) * 16 + (pt & 7) + 8 * ((pt >> 4) & 1), half = (pt >> 3) & 1;
-    const size_t slot0 = (size_t(b) * p.H_kv + h) * p.cap;
+    auto slot_of = [&](int t) { return cache_slot(p.table, p.page, p.H_kv, p.cap, b, h, t); };
     const uint4* cent4 = reinterpret_cast<const uint4*>(p.cent) + size_t(h) * p.M * (kD / 8) + half * 8;
     RawHalf raw;
     bool raw_ok = nloc > 0 && jA < n_cache && row < min(kKeys, p.len - jA * kKeys);
-    if (raw_ok) load_raw_half(p, slot0 + size_t(jA) * kKeys + row, half, raw);
+    if (raw_ok) load_raw_half(p, slot_of(jA * kKeys + row), half, raw);
     for (int jj = 0; jj < nloc; ++jj) {
       const int j = jA + jj;
       const int s = jj & 1;
@@ -587,12 +589,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
         const uint4* mu = cent4 + size_t(min(raw.idx, p.M - 1)) * (kD / 8);
 #pragma unroll
         for (int c = 0; c < 8; ++c) m4[c] = __ldg(mu + c);
-        if (half == 0) load_psac(p, slot0 + size_t(j) * kKeys + row, a0, a1);
+        if (half == 0) load_psac(p, slot_of(j * kKeys + row), a0, a1);
       }
       RawHalf next;
       const int jn = j + 1;
       const bool next_ok = jn < jB && jn < n_cache && row < min(kKeys, p.len - jn * kKeys);
-      if (next_ok) load_raw_half(p, slot0 + size_t(jn) * kKeys + row, half, next);
+      if (next_ok) load_raw_half(p, slot_of(jn * kKeys + row), half, next);
       if (use >= 1 && !mbar_wait_or_abort(bar + B_KV_EMPTY + 8 * s, (use - 1) & 1, p.budget, abort)) break;
       uint8_t* stage = smem + OFF_STAGE + s * STAGE_BYTES;
       if (row < kvalid) {
@@ -857,6 +859,7 @@ cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t s) {
   p.k_code = c.k_code; p.v_code = c.v_code; p.k_sz = c.k_sz; p.v_sz = c.v_sz;
   p.cidx = c.cidx; p.psac = c.psac; p.cent = c.centroids; p.P = c.P;
   p.psac_fmt = c.psac_fmt; p.psac_scale = c.psac_scale;
+  p.table = c.block_table; p.page = c.page_tokens;
   p.Q = a.Q; p.Ks = a.Kself; p.Vs = a.Vself; p.out = a.out;
   p.err = static_cast<int*>(a.ws);
   p.B = c.B; p.H_kv = c.H_kv; p.H_q = a.H_q; p.M = c.M; p.r = c.r; p.cap = c.capacity;

@@ -118,6 +118,17 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// Slot of token t of (sequence b, KV head h): contiguous streams
+// [B][H_kv][cap], or a pool of pages [pages][H_kv][page] addressed through the
+// block table [B][cap / page] (a page holds `page` consecutive tokens of one
+// sequence; page is a multiple of 128, so a 128-token tile never leaves it)
+__device__ __forceinline__ size_t cache_slot(const int32_t* table, int page, int H_kv, int cap, int b, int h,
+                                             int t) {
+  if (!table) return (size_t(b) * H_kv + h) * cap + t;
+  const int pg = table[size_t(b) * (cap / page) + t / page];
+  return (size_t(pg) * H_kv + h) * page + (t % page);
+}
+
 // INT8 PSAC coefficients of one token: scale = fp16 round-up of the fp32
 // quotient max|a| / 127, code = clamp(round-half-even(a / scale), -127, 127)
 // (0 when the scale is 0); the coefficient read back is code * scale

@@ -77,6 +77,8 @@ struct SplitParams {
   int H_kv, H_q, M, r, cap, len, splits, tiles_per_split;
   int psac_fmt;                 // 0: fp16 coefficients; 1: int8 codes + fp16 scale per token
   const uint16_t* psac_scale;
+  const int32_t* table;         // paged cache: block table [B][cap / page] (null: contiguous)
+  int page;
 };
 
 // d = a * b + c on two fp16 lanes
@@ -287,7 +289,8 @@ __global__ void __launch_bounds__(kThreads) decode_split(SplitParams p) {
       asm volatile("griddepcontrol.wait;" ::: "memory");
       dep_done = true;
     }
-    const size_t s0 = base_slot + t0;                      // a multiple of 16
+    // (a multiple of 16; a tile never leaves its page)
+    const size_t s0 = p.table ? cache_slot(p.table, p.page, p.H_kv, p.cap, b, h, t0) : base_slot + t0;
     const int ps_bytes = Q8 ? (r ? r + 2 : 0) : 2 * r;   // per token
     mbar_arrive_expect_tx(bar, uint32_t(n16) * uint32_t(2 * NW * 4 + 2 * NG * 4 + Cfg::IDXB + ps_bytes));
     bulk_g2s(dst + Cfg::kc_off, p.k_code + s0 * NW, n16 * NW * 4, bar);
@@ -1026,7 +1029,8 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
                  static_cast<const uint16_t*>(a.Q), static_cast<const uint16_t*>(c.centroids), c.P,
                  a.sm_scale * kLog2e, part, static_cast<int*>(a.ws),
                  force ? (1ull << 20) : env_wait_budget(), force, a.wait_from,
-                 c.H_kv, a.H_q, c.M, c.r, c.capacity, a.len, splits, tps, c.psac_fmt, c.psac_scale};
+                 c.H_kv, a.H_q, c.M, c.r, c.capacity, a.len, splits, tps, c.psac_fmt, c.psac_scale,
+                 c.block_table, c.page_tokens};
   const int G = a.H_q / c.H_kv;
   cudaError_t e;
   if (c.d == 64) e = (c.M > 256) ? launch_g<64, true>(G, sp, c.B, s) : launch_g<64, false>(G, sp, c.B, s);

@@ -38,6 +38,9 @@ struct QuantizeArgs {
   // one fp16 scale per token in psac_scale
   int psac_fmt = 0;
   uint16_t* psac_scale = nullptr;
+  // paged cache: block table [B][cap / page] (null: contiguous streams)
+  const int32_t* table = nullptr;
+  int page = 0;
 };
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s);
 

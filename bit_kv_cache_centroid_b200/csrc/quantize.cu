@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
   };
   auto slot_of = [&](int row) {
     const int b = row / a.n_new, t = row - b * a.n_new;
-    return (size_t(b) * a.H + h) * a.cap + size_t(a.pos + t);
+    return cache_slot(a.table, a.page, a.H, a.cap, b, h, a.pos + t);
   };
 
   // ---- once per CTA: centroid table (fp16, transposed, lane-interleaved), w,

@@ -35,6 +35,8 @@ struct Top1Params {
   const uint16_t* psac_scale;
   const uint16_t* cent;
   const float* P;
+  const int32_t* table;     // paged cache: block table (null: contiguous)
+  int page;
   int B, nq, H_q, H_kv, d, M, r, cap, len, psac_fmt, splits;
   unsigned long long* part;  // [B*nq*H_q][splits]: (order key of the logit << 32) | ~index
 };
@@ -68,7 +70,7 @@ __global__ void __launch_bounds__(kTopThreads) top1_split(Top1Params p) {
       const uint16_t* kr = p.K + ((size_t(b) * p.len + t) * p.H_kv + h) * p.d;
       for (int c = 0; c < p.d; ++c) acc = fmaf(q[c], bf16_to_f32(kr[c]), acc);
     } else {
-      const size_t slot = (size_t(b) * p.H_kv + h) * p.cap + t;
+      const size_t slot = cache_slot(p.table, p.page, p.H_kv, p.cap, b, h, t);
       const int j = (p.M <= 256) ? int(static_cast<const uint8_t*>(p.cidx)[slot])
                                  : int(static_cast<const uint16_t*>(p.cidx)[slot]);
       const uint16_t* mu = p.cent + (size_t(h) * p.M + min(j, p.M - 1)) * p.d;
@@ -142,6 +144,8 @@ cudaError_t launch_top1(const Top1Args& a, cudaStream_t s) {
     p.r = c.r;
     p.cap = c.capacity;
     p.psac_fmt = c.psac_fmt;
+    p.table = c.block_table;
+    p.page = c.page_tokens;
   }
   p.splits = a.len > 0 ? (a.len + kTokensPerCta - 1) / kTokensPerCta : 1;
   p.part = static_cast<unsigned long long*>(a.ws);

@@ -66,6 +66,11 @@ enum { KV2_OUT_F32 = 0, KV2_OUT_BF16 = 1 };
  *                    coefficient is code * psac_scale[slot]
  *   psac_scale     : fp16 [B][H_kv][capacity], one scale per token (psac_fmt 1
  *                    only; NULL otherwise)
+ * Paged cache (block_table set): every stream above is instead a pool of pages
+ * [pages][H_kv][page_tokens][...]; token t of sequence b lives in page
+ * block_table[b][t / page_tokens] at offset t % page_tokens. capacity is the
+ * logical length per sequence (a multiple of page_tokens); the pool may hold
+ * any number of pages, shared by the sequences through their tables.
  *   centroids      : fp16 [H_kv][M][d] (read-only; shared by the batch)
  *   P, w, Wg       : fp32 [H_kv][d][r] basis, [H_kv][d] channel sensitivities,
  *                    [H_kv][d/32] group sensitivities, as written by
@@ -87,6 +92,8 @@ typedef struct kv2_cache {
   const float* Wg;
   int32_t psac_fmt;      /* 0: fp16 coefficients; 1: int8 codes + fp16 scale per token */
   uint16_t* psac_scale;
+  const int32_t* block_table;  /* paged cache: page ids [B][capacity / page_tokens]; NULL: contiguous */
+  int32_t page_tokens;         /* tokens per page (a multiple of 128) when block_table is set */
 } kv2_cache;
 
 /* Human-readable name of a status. Never NULL. */

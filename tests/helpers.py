@@ -80,8 +80,10 @@ def gpu_cache_like(pc, fit=None):
     contents copied in, and (optionally) the fitted statistics."""
     import torch
     import bit_kv_cache_centroid_b200 as kv2
+    paged = getattr(pc, "table", None) is not None
     c = kv2.Cache(pc.B, pc.H_kv, pc.d, pc.M, pc.r, pc.capacity,
-                  torch.from_numpy(pc.centroids.view(np.int16)), psac_fmt=getattr(pc, "psac_fmt", 0))
+                  torch.from_numpy(pc.centroids.view(np.int16)), psac_fmt=getattr(pc, "psac_fmt", 0),
+                  page_tokens=pc.page if paged else 0, num_pages=pc.k_code.shape[0] if paged else 0)
     c.load_packed(pc)
     if fit is not None:
         c.set_fit(torch.from_numpy(fit.P), torch.from_numpy(fit.w), torch.from_numpy(fit.Wg))
