@@ -75,3 +75,41 @@ def test_unsupported_shapes_are_rejected(lib):
     assert lib.kv2_attention_chunk(ctypes.byref(d), 0, ctypes.c_void_p(16), 2, 4, ctypes.c_void_p(16),
                                    ctypes.c_void_p(16), 4, ctypes.c_float(1.0), ctypes.c_void_p(16), 0,
                                    ctypes.c_void_p(16), 1 << 20, None) == 2
+
+
+def _desc(**kw):
+    """A cache descriptor with fake (never dereferenced) aligned pointers."""
+    import bit_kv_cache_centroid_b200 as kv2
+    base = dict(B=1, H_kv=2, d=128, M=64, r=8, capacity=256, k_code=0x1000, v_code=0x2000, k_sz=0x3000,
+                v_sz=0x4000, cidx=0x5000, psac=0x6000, centroids=0x7000, P=0x8000, w=0x9000, Wg=0xA000,
+                psac_fmt=0, psac_scale=0, block_table=0, page_tokens=0)
+    base.update(kw)
+    return kv2.kv2_cache(**base)
+
+
+def test_argument_checks_of_the_later_entry_points(lib):
+    """Checks that return before any device work (no GPU needed)."""
+    P = ctypes.c_void_p
+    lib.kv2_last_error.restype = ctypes.c_char_p
+    lib.kv2_fit_centroids_workspace_size.restype = ctypes.c_size_t
+    lib.kv2_top1_workspace_size.restype = ctypes.c_size_t
+    # workspace sizes: (H*M*d + H*M) 64-bit words; B*nq*H_q*ceil(len/4096) words
+    assert lib.kv2_fit_centroids_workspace_size(2, 128, 64) == (2 * 64 * 128 + 2 * 64) * 8
+    assert lib.kv2_fit_centroids_workspace_size(2, 96, 64) == 0
+    assert lib.kv2_top1_workspace_size(2, 3, 4, 5000) == 2 * 3 * 4 * 2 * 8
+    # centre fitting: candidates outside 1..M, unsupported d, a no-op call
+    args = lambda C, d, iters: (P(0x1000), 16, 2, d, 64, C, P(0x2000), P(0x3000), iters, P(0x4000), P(0x5000),
+                                P(0x6000), ctypes.c_size_t(1 << 20), None)
+    assert lib.kv2_fit_centroids(*args(65, 128, 1)) == 1              # KV2_ERR_INVALID_ARG
+    assert b"candidates" in lib.kv2_last_error()
+    assert lib.kv2_fit_centroids(*args(4, 96, 1)) == 2                # KV2_ERR_UNSUPPORTED
+    assert lib.kv2_fit_centroids(*args(4, 128, 0)) == 0               # iters = 0: nothing to do
+    # paged cache: a page size that is not a multiple of 128 is refused
+    bad = _desc(block_table=0xB000, page_tokens=96)
+    top1 = lib.kv2_decode_top1(ctypes.byref(bad), 10, P(0x1000), 1, 2, P(0x2000), P(0x3000),
+                               ctypes.c_size_t(1 << 20), None)
+    assert top1 == 2 and b"page_tokens" in lib.kv2_last_error()
+    # int8 PSAC format without its scale array is refused
+    noscale = _desc(psac_fmt=1)
+    assert lib.kv2_quantize_append(ctypes.byref(noscale), P(0x1000), P(0x2000), 1, 0, 1, None) == 1
+    assert b"psac_scale" in lib.kv2_last_error()
