@@ -66,14 +66,16 @@ def _declare(L):
     L.or_f32_from_bf16.argtypes = [ctypes.c_uint16]
     L.or_f32_from_bf16.restype = ctypes.c_float
     L.or_codec_group.argtypes = [_P, _I, _P, _P, _P, _P]
-    L.or_fit.argtypes = [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P]
+    # the last argument of each is the group size (channels per scale, zero)
+    L.or_fit.argtypes = [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I]
     L.or_quantize.argtypes = ([_I] * 6 + [_P, _P, _I, _I, _I, _P, _P, _P, _P] + [_P] * 6 + [_I, _P, _P, _I]
-                              + [_P] * 3)
-    L.or_decode.argtypes = [_I] * 6 + [_P] * 6 + [_I, _P, _P, _I] + [_P] * 2 + [_I, _P, _I, ctypes.c_double, _P]
+                              + [_P] * 3 + [_I])
+    L.or_decode.argtypes = ([_I] * 6 + [_P] * 6 + [_I, _P, _P, _I] + [_P] * 2
+                            + [_I, _P, _I, ctypes.c_double, _P, _I])
     L.or_chunk.argtypes = ([_I] * 6 + [_P] * 6 + [_I, _P, _P, _I] + [_P] * 2 + [_I, _P, _I, _I, _P, _P, _I,
-                                                  ctypes.c_double, _P, _I, _P])
-    L.or_decode_logits.argtypes = [_I] * 7 + [_P] * 4 + [_I, _P, _P, _I] + [_P] * 2 + [_I, _P, _P]
-    L.or_fit_centroids.argtypes = [_I] * 5 + [_P, _P, _P, _I, _P, _P]
+                                                  ctypes.c_double, _P, _I, _P, _I])
+    L.or_decode_logits.argtypes = [_I] * 7 + [_P] * 4 + [_I, _P, _P, _I] + [_P] * 2 + [_I, _P, _P, _I]
+    L.or_fit_centroids.argtypes = [_I] * 5 + [_P, _P, _P, _I, _P, _P, _I]
     for f in (L.or_codec_group, L.or_fit, L.or_quantize, L.or_decode, L.or_chunk,
               L.or_decode_logits, L.or_fit_centroids):
         f.restype = _I if f is not L.or_codec_group else None
@@ -126,21 +128,22 @@ def codec_group(x: np.ndarray):
 class Fit:
     P: np.ndarray       # fp32 [H_kv][d][r]
     w: np.ndarray       # fp32 [H_kv][d]
-    Wg: np.ndarray      # fp32 [H_kv][d/32]
+    Wg: np.ndarray      # fp32 [H_kv][d/group]
     evals: np.ndarray   # fp64 [H_kv][d], descending
     energy: np.ndarray  # fp64 [H_kv], top-r share of the energy
 
 
-def fit(Qhist: np.ndarray, H_kv: int, r: int) -> Fit:
-    """PSAC basis + sensitivity weights from history queries bf16 [n][H_q][d]."""
+def fit(Qhist: np.ndarray, H_kv: int, r: int, group: int = 32) -> Fit:
+    """PSAC basis + sensitivity weights from history queries bf16 [n][H_q][d];
+    W sums w over groups of ``group`` channels."""
     Qhist = _c(Qhist, np.uint16)
     n, Hq, d = Qhist.shape
     P = np.zeros((H_kv, d, max(r, 1)), np.float32)[:, :, :r].copy()
     w = np.zeros((H_kv, d), np.float32)
-    Wg = np.zeros((H_kv, d // 32), np.float32)
+    Wg = np.zeros((H_kv, max(d // group, 1)), np.float32)
     ev = np.zeros((H_kv, d), np.float64)
     en = np.zeros(H_kv, np.float64)
-    rc = lib().or_fit(_ptr(Qhist), n, Hq, H_kv, d, r, _ptr(P), _ptr(w), _ptr(Wg), _ptr(ev), _ptr(en))
+    rc = lib().or_fit(_ptr(Qhist), n, Hq, H_kv, d, r, _ptr(P), _ptr(w), _ptr(Wg), _ptr(ev), _ptr(en), group)
     if rc:
         raise ValueError("or_fit: bad arguments")
     return Fit(P, w, Wg, ev, en)
@@ -164,6 +167,8 @@ def quantize(pc, K: np.ndarray, V: np.ndarray, pos: int, C: int, P: np.ndarray,
     w = _c(w, np.float32)
     Wg = _c(Wg, np.float32)
     r = pc.r
+    if Wg.shape[-1] != d // pc.group:
+        raise ValueError(f"Wg has {Wg.shape[-1]} groups; the cache's groups of {pc.group} need {d // pc.group}")
     dbg = None
     if debug:
         dbg = QuantDebug(np.zeros((B, n_new, Hkv, C), np.int32),
@@ -175,23 +180,25 @@ def quantize(pc, K: np.ndarray, V: np.ndarray, pos: int, C: int, P: np.ndarray,
         _ptr(pc.k_code), _ptr(pc.v_code), _ptr(pc.k_sz), _ptr(pc.v_sz),
         _ptr(pc.cidx), *_psac_args(pc),
         _ptr(dbg.cand) if dbg else None, _ptr(dbg.score) if dbg else None,
-        _ptr(dbg.E) if dbg else None)
+        _ptr(dbg.E) if dbg else None, pc.group)
     if rc:
         raise ValueError("or_quantize: bad arguments")
     return dbg
 
 
 def fit_centroids(X: np.ndarray, M: int, C: int, w: np.ndarray, Wg: np.ndarray,
-                  centroids: np.ndarray, iters: int):
+                  centroids: np.ndarray, iters: int, group: int = 32):
     """QSAC-aware centre fitting (reading in ``kv2_oracle.c``): X bf16 bits
     [n][H_kv][d], initial centres fp16 bits [H_kv][M][d] -> (fitted centres
     fp16 bits [H_kv][M][d], last assignment int32 [n][H_kv])."""
     X = _c(X, np.uint16)
     n, Hkv, d = X.shape
+    if np.shape(Wg)[-1] != d // group:
+        raise ValueError("Wg does not match the group size")
     cent = np.array(_c(centroids, np.uint16), copy=True)
     assign = np.full((max(n, 1), Hkv), -1, np.int32)
     rc = lib().or_fit_centroids(n, Hkv, d, M, C, _ptr(X), _ptr(_c(w, np.float32)), _ptr(_c(Wg, np.float32)),
-                                iters, _ptr(cent), _ptr(assign))
+                                iters, _ptr(cent), _ptr(assign), group)
     if rc:
         raise ValueError("or_fit_centroids: bad arguments")
     return cent, assign[:n]
@@ -226,7 +233,7 @@ def decode(pc, P: np.ndarray, length: int, Q: np.ndarray, sm_scale: float) -> np
     pc.P = P
     out = np.zeros((B, Hq, d), np.float64)
     rc = lib().or_decode(pc.B, pc.H_kv, pc.d, pc.M, pc.r, pc.capacity, *_cache_args(pc),
-                         length, _ptr(Q), Hq, float(sm_scale), _ptr(out))
+                         length, _ptr(Q), Hq, float(sm_scale), _ptr(out), pc.group)
     if rc:
         raise ValueError("or_decode: bad arguments")
     return out
@@ -246,7 +253,7 @@ def chunk(pc, P: np.ndarray, length: int, Q: np.ndarray, Kself: np.ndarray,
     out = np.zeros((rows.shape[0], d), np.float64)
     rc = lib().or_chunk(pc.B, pc.H_kv, pc.d, pc.M, pc.r, pc.capacity, *_cache_args(pc),
                         length, _ptr(Q), Hq, Nq, _ptr(Kself), _ptr(Vself), frame_tokens,
-                        float(sm_scale), _ptr(rows), rows.shape[0], _ptr(out))
+                        float(sm_scale), _ptr(rows), rows.shape[0], _ptr(out), pc.group)
     if rc:
         raise ValueError("or_chunk: bad arguments")
     return out
@@ -258,9 +265,12 @@ def decode_logits(pc, P: np.ndarray, b: int, h: int, length: int, q: np.ndarray)
     pc.P = P
     out = np.zeros(length, np.float64)
     Pp = _c(P, np.float32) if pc.r else np.zeros(1, np.float32)
-    lib().or_decode_logits(pc.H_kv, pc.d, pc.M, pc.r, pc.capacity, b, h,
-                           _ptr(pc.k_code), _ptr(pc.k_sz), _ptr(pc.cidx), *_psac_args(pc),
-                           _ptr(_c(pc.centroids, np.uint16)), _ptr(Pp), length, _ptr(q), _ptr(out))
+    rc = lib().or_decode_logits(pc.H_kv, pc.d, pc.M, pc.r, pc.capacity, b, h,
+                                _ptr(pc.k_code), _ptr(pc.k_sz), _ptr(pc.cidx), *_psac_args(pc),
+                                _ptr(_c(pc.centroids, np.uint16)), _ptr(Pp), length, _ptr(q), _ptr(out),
+                                pc.group)
+    if rc:
+        raise ValueError("or_decode_logits: bad arguments")
     return out
 
 

@@ -23,15 +23,16 @@
  * QSAC vs brute-force argmin (candidates = M) and vs plain nearest centre
  * (candidates = 1, unit weights); PSAC r = d and r = 0 closed forms; Jacobi vs
  * numpy.linalg.eigh; attention vs a two-pass softmax and a centroid-only closed
- * form. Parity unpinned: whether the perturbation estimate is the authors' exact
+ * form; group sizes 64 and 128 by per-group codec invariants, exact
+ * reconstruction of group-constant residuals, the single-group QSAC choice as
+ * the least residual range, and W over one whole-row group as the trace of
+ * the Gram matrix. Parity unpinned: whether the perturbation estimate is the authors' exact
  * heuristic (the pages print no worked example).
  */
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
-
-#define GROUP 32
 
 /* ------------------------------------------------------------------------ */
 /* IEEE 754 binary16 / bfloat16                                             */
@@ -135,10 +136,13 @@ uint16_t or_bf16_from_f32(float x)
 /* ------------------------------------------------------------------------ */
 /* INT2 group codec                                                          */
 /*   QuantWM article, "1. QSAC": the centre-relative residual is quantized to  */
-/*   2 bits; the cache stores an fp16 scale and an fp16 zero per group of 32    */
-/*   channels (asymmetric INT2). Reading taken: zero = the group minimum       */
-/*   rounded down to fp16, scale = (max - zero)/3 rounded up to fp16, so that  */
-/*   [zero, zero + 3 scale] covers the group; codes round half to even.        */
+/*   2 bits; the cache stores an fp16 scale and an fp16 zero per group of      */
+/*   consecutive channels (asymmetric INT2). The pages fix no group size: the  */
+/*   cache format takes 32 (default), 64 or 128, the larger ones trading       */
+/*   accuracy for the compression the evaluation counts. Reading taken: zero = */
+/*   the group minimum rounded down to fp16, scale = (max - zero)/3 rounded up */
+/*   to fp16, so that [zero, zero + 3 scale] covers the group; codes round     */
+/*   half to even.                                                             */
 /* ------------------------------------------------------------------------ */
 
 static void codec_params(const float* x, int n, uint16_t* s_bits, uint16_t* z_bits)
@@ -236,10 +240,10 @@ static void jacobi_eigen(double* A, double* V, int n)
 }
 
 int or_fit(const uint16_t* Qh, int n, int Hq, int Hkv, int d, int r,
-           float* P, float* w, float* Wg, double* evals, double* energy)
+           float* P, float* w, float* Wg, double* evals, double* energy, int group)
 {
-    if (Hkv <= 0 || Hq % Hkv || d % GROUP || r < 0 || r > d || n <= 0) return 1;
-    int G = Hq / Hkv, ng = d / GROUP;
+    if (Hkv <= 0 || Hq % Hkv || group <= 0 || d % group || r < 0 || r > d || n <= 0) return 1;
+    int G = Hq / Hkv, ng = d / group;
     double* S = (double*)calloc((size_t)d * d, sizeof(double));
     double* Vec = (double*)malloc((size_t)d * d * sizeof(double));
     double* lam = (double*)malloc((size_t)d * sizeof(double));
@@ -259,7 +263,7 @@ int or_fit(const uint16_t* Qh, int n, int Hq, int Hkv, int d, int r,
         for (int c = 0; c < d; ++c) w[(size_t)h * d + c] = (float)S[c * d + c];
         for (int g = 0; g < ng; ++g) {
             float acc = 0.0f;
-            for (int c = g * GROUP; c < (g + 1) * GROUP; ++c) acc = acc + w[(size_t)h * d + c];
+            for (int c = g * group; c < (g + 1) * group; ++c) acc = acc + w[(size_t)h * d + c];
             Wg[(size_t)h * ng + g] = acc;
         }
         jacobi_eigen(S, Vec, d);
@@ -308,8 +312,8 @@ int or_fit(const uint16_t* Qh, int n, int Hq, int Hkv, int d, int r,
 /*   e = residual - dequantized residual, an fp32 fmaf chain over ascending c, */
 /*   stored as fp16 (round to nearest even).                                   */
 /* Layouts: K, V bf16 [B][n_new][Hkv][d]; centroids fp16 [Hkv][M][d];          */
-/* P [Hkv][d][r]; w [Hkv][d]; Wg [Hkv][d/32]; packed streams as in the         */
-/* library: [B][Hkv][cap][...].                                              */
+/* P [Hkv][d][r]; w [Hkv][d]; Wg [Hkv][d/group]; packed streams as in the      */
+/* library: [B][Hkv][cap][...], (scale, zero) per group of `group` channels.  */
 /* ------------------------------------------------------------------------ */
 
 /* QSAC decision for one key k (fp32 [d]) of KV head h: returns the chosen
@@ -317,10 +321,10 @@ int or_fit(const uint16_t* Qh, int n, int Hq, int Hkv, int d, int r,
  * above; scratch: score [M], cand [C], used [M], x [d]. Optional debug
  * outputs (candidate ids, scores, E per candidate) when non-NULL. */
 static int qsac_choose(const float* k, const float* wh, const float* Wgh, const float* mu, const float* nrm,
-                       int M, int C, int d, float* wk, float* score, int* cand, char* used, float* x,
+                       int M, int C, int d, int group, float* wk, float* score, int* cand, char* used, float* x,
                        float* xbest, int32_t* cand_out, float* score_out, float* E_out)
 {
-    int ng = d / GROUP;
+    int ng = d / group;
     for (int c = 0; c < d; ++c) wk[c] = wh[c] * k[c];
     /* ranking */
     for (int j = 0; j < M; ++j) {
@@ -351,7 +355,7 @@ static int qsac_choose(const float* k, const float* wh, const float* Wgh, const 
         float E = 0.0f;
         for (int g = 0; g < ng; ++g) {
             uint16_t sb, zb;
-            codec_params(x + g * GROUP, GROUP, &sb, &zb);
+            codec_params(x + g * group, group, &sb, &zb);
             float s = or_f32_from_f16(sb);
             float ws = Wgh[g] * s;
             E = fmaf(ws, s, E);
@@ -418,22 +422,26 @@ static uint32_t pack_word(const uint32_t* codes16)
     return w;
 }
 
-static void quantize_row(const float* x, int d, uint32_t* code_words, uint32_t* sz, float* deq)
+/* One row of d channels in groups of `group` consecutive channels: each
+ * group's fp16 (scale, zero) into sz[g], then every channel's code under its
+ * own group's parameters, 16 codes per word in channel order. */
+static void quantize_row(const float* x, int d, int group, uint32_t* code_words, uint32_t* sz, float* deq)
 {
     uint32_t codes[16];
-    for (int g = 0; g < d / GROUP; ++g) {
+    for (int g = 0; g < d / group; ++g) {
         uint16_t sb, zb;
-        codec_params(x + g * GROUP, GROUP, &sb, &zb);
-        float s = or_f32_from_f16(sb), z = or_f32_from_f16(zb);
+        codec_params(x + g * group, group, &sb, &zb);
         sz[g] = (uint32_t)sb | ((uint32_t)zb << 16);
-        for (int half = 0; half < 2; ++half) {
-            for (int i = 0; i < 16; ++i) {
-                int c = g * GROUP + half * 16 + i;
-                codes[i] = codec_code(x[c], s, z);
-                if (deq) deq[c] = codec_dequant(codes[i], s, z);
-            }
-            code_words[(g * GROUP + half * 16) / 16] = pack_word(codes);
+    }
+    for (int wd = 0; wd < d / 16; ++wd) {
+        for (int i = 0; i < 16; ++i) {
+            int c = wd * 16 + i;
+            uint32_t p = sz[c / group];
+            float s = or_f32_from_f16((uint16_t)(p & 0xffff)), z = or_f32_from_f16((uint16_t)(p >> 16));
+            codes[i] = codec_code(x[c], s, z);
+            if (deq) deq[c] = codec_dequant(codes[i], s, z);
         }
+        code_words[wd] = pack_word(codes);
     }
 }
 
@@ -443,11 +451,11 @@ int or_quantize(int B, int Hkv, int d, int M, int r, int cap,
                 uint32_t* k_code, uint32_t* v_code, uint32_t* k_sz, uint32_t* v_sz,
                 void* cidx, uint16_t* psac, int psac_fmt, uint16_t* psac_scale,
                 const int32_t* table, int page,
-                int32_t* cand_out, float* score_out, float* E_out)
+                int32_t* cand_out, float* score_out, float* E_out, int group)
 {
-    if (d % GROUP || C < 1 || C > M || pos < 0 || pos + n_new > cap || (psac_fmt != 0 && psac_fmt != 1) ||
+    if (group <= 0 || d % group || d % 16 || C < 1 || C > M || pos < 0 || pos + n_new > cap || (psac_fmt != 0 && psac_fmt != 1) ||
         (table && (page <= 0 || cap % page))) return 1;
-    int ng = d / GROUP, nw = d / 16;
+    int ng = d / group, nw = d / 16;
     float* mu = (float*)malloc((size_t)M * d * sizeof(float));
     float* nrm = (float*)malloc((size_t)M * sizeof(float));
     float* score = (float*)malloc((size_t)M * sizeof(float));
@@ -470,11 +478,11 @@ int or_quantize(int B, int Hkv, int d, int M, int r, int cap,
                 size_t slot = slot_at(Hkv, cap, table, page, b, h, pos + t);
                 size_t dbg = (((size_t)b * n_new + t) * Hkv + h);
                 for (int c = 0; c < d; ++c) k[c] = or_f32_from_bf16(K[in + c]);
-                int chosen = qsac_choose(k, wh, Wg + (size_t)h * ng, mu, nrm, M, C, d, wk, score, cand, used, x,
+                int chosen = qsac_choose(k, wh, Wg + (size_t)h * ng, mu, nrm, M, C, d, group, wk, score, cand, used, x,
                                          xbest, cand_out ? cand_out + dbg * C : NULL,
                                          score_out ? score_out + dbg * C : NULL, E_out ? E_out + dbg * C : NULL);
                 /* residual codes, scales, zeros */
-                quantize_row(xbest, d, cw, szr, deq);
+                quantize_row(xbest, d, group, cw, szr, deq);
                 memcpy(k_code + slot * nw, cw, (size_t)nw * 4);
                 memcpy(k_sz + slot * ng, szr, (size_t)ng * 4);
                 if (M <= 256) ((uint8_t*)cidx)[slot] = (uint8_t)chosen;
@@ -495,7 +503,7 @@ int or_quantize(int B, int Hkv, int d, int M, int r, int cap,
                                                       psac_scale + slot);
                 /* values: same codec, no centre */
                 for (int c = 0; c < d; ++c) x[c] = or_f32_from_bf16(V[in + c]);
-                quantize_row(x, d, cw, szr, NULL);
+                quantize_row(x, d, group, cw, szr, NULL);
                 memcpy(v_code + slot * nw, cw, (size_t)nw * 4);
                 memcpy(v_sz + slot * ng, szr, (size_t)ng * 4);
             }
@@ -524,10 +532,10 @@ int or_quantize(int B, int Hkv, int d, int M, int r, int cap,
 /* ------------------------------------------------------------------------ */
 
 int or_fit_centroids(int n, int Hkv, int d, int M, int C, const uint16_t* X, const float* w,
-                     const float* Wg, int iters, uint16_t* cent, int32_t* assign)
+                     const float* Wg, int iters, uint16_t* cent, int32_t* assign, int group)
 {
-    if (d % GROUP || C < 1 || C > M || n < 0 || iters < 0) return 1;
-    int ng = d / GROUP;
+    if (group <= 0 || d % group || C < 1 || C > M || n < 0 || iters < 0) return 1;
+    int ng = d / group;
     float* mu = (float*)malloc((size_t)M * d * sizeof(float));
     float* nrm = (float*)malloc((size_t)M * sizeof(float));
     float* score = (float*)malloc((size_t)M * sizeof(float));
@@ -548,7 +556,8 @@ int or_fit_centroids(int n, int Hkv, int d, int M, int C, const uint16_t* X, con
             for (int t = 0; t < n; ++t) {
                 const uint16_t* xr = X + ((size_t)t * Hkv + h) * d;
                 for (int c = 0; c < d; ++c) k[c] = or_f32_from_bf16(xr[c]);
-                a[t] = qsac_choose(k, wh, Wg + (size_t)h * ng, mu, nrm, M, C, d, wk, score, cand, used, x, xbest,
+                a[t] = qsac_choose(k, wh, Wg + (size_t)h * ng, mu, nrm, M, C, d, group, wk, score, cand, used, x,
+                                   xbest,
                                    NULL, NULL, NULL);
                 if (assign) assign[(size_t)t * Hkv + h] = a[t];
             }
@@ -598,6 +607,7 @@ typedef struct {
     const uint16_t* psac_scale;
     const int32_t* table;         /* paged: page ids [B][cap / page]; NULL: contiguous */
     int page;                     /* tokens per page (paged) */
+    int group;                    /* channels per (scale, zero) group */
 } or_cache;
 
 
@@ -623,7 +633,7 @@ static uint32_t code_at(const uint32_t* words, int ch)
 /* exact dequantized key/value rows of one token (decode precision) */
 static void dequant_exact(const or_cache* c, size_t slot, double* kh, double* vh)
 {
-    int d = c->d, ng = d / GROUP;
+    int d = c->d, ng = d / c->group;
     const uint32_t* kw = c->k_code + slot * (d / 16);
     const uint32_t* vw = c->v_code + slot * (d / 16);
     int j = cache_idx(c, slot);
@@ -632,7 +642,7 @@ static void dequant_exact(const or_cache* c, size_t slot, double* kh, double* vh
         uint32_t ks = c->k_sz[slot * ng + g], vs = c->v_sz[slot * ng + g];
         double s = or_f32_from_f16((uint16_t)(ks & 0xffff)), z = or_f32_from_f16((uint16_t)(ks >> 16));
         double sv = or_f32_from_f16((uint16_t)(vs & 0xffff)), zv = or_f32_from_f16((uint16_t)(vs >> 16));
-        for (int ch = g * GROUP; ch < (g + 1) * GROUP; ++ch) {
+        for (int ch = g * c->group; ch < (g + 1) * c->group; ++ch) {
             double m = or_f32_from_f16(c->cent[((size_t)h * c->M + j) * d + ch]);
             kh[ch] = m + (double)code_at(kw, ch) * s + z;
             vh[ch] = (double)code_at(vw, ch) * sv + zv;
@@ -645,7 +655,7 @@ static void dequant_exact(const or_cache* c, size_t slot, double* kh, double* vh
  * Vhat = fp16(code s + z) */
 static void dequant_operand(const or_cache* c, size_t slot, double* kh, double* vh)
 {
-    int d = c->d, ng = d / GROUP;
+    int d = c->d, ng = d / c->group;
     const uint32_t* kw = c->k_code + slot * (d / 16);
     const uint32_t* vw = c->v_code + slot * (d / 16);
     int j = cache_idx(c, slot);
@@ -654,7 +664,7 @@ static void dequant_operand(const or_cache* c, size_t slot, double* kh, double* 
         uint32_t ks = c->k_sz[slot * ng + g], vs = c->v_sz[slot * ng + g];
         double s = or_f32_from_f16((uint16_t)(ks & 0xffff)), z = or_f32_from_f16((uint16_t)(ks >> 16));
         double sv = or_f32_from_f16((uint16_t)(vs & 0xffff)), zv = or_f32_from_f16((uint16_t)(vs >> 16));
-        for (int ch = g * GROUP; ch < (g + 1) * GROUP; ++ch) {
+        for (int ch = g * c->group; ch < (g + 1) * c->group; ++ch) {
             double m = or_f32_from_f16(c->cent[((size_t)h * c->M + j) * d + ch]);
             kh[ch] = f16_round((double)code_at(kw, ch) * s + f16_round(z + m));
             vh[ch] = f16_round((double)code_at(vw, ch) * sv + zv);
@@ -682,11 +692,11 @@ int or_decode(int B, int Hkv, int d, int M, int r, int cap,
               const uint32_t* v_sz, const void* cidx, const uint16_t* psac,
               int psac_fmt, const uint16_t* psac_scale, const int32_t* table, int page,
               const uint16_t* cent, const float* P,
-              int len, const uint16_t* Q, int Hq, double sm_scale, double* out)
+              int len, const uint16_t* Q, int Hq, double sm_scale, double* out, int group)
 {
-    if (Hq % Hkv || len < 0 || len > cap) return 1;
+    if (Hq % Hkv || len < 0 || len > cap || group <= 0 || d % group) return 1;
     or_cache c = {B, Hkv, d, M, r, cap, k_code, v_code, k_sz, v_sz, cidx, psac, cent, P, psac_fmt, psac_scale,
-                  table, page};
+                  table, page, group};
     int G = Hq / Hkv;
     double* logit = (double*)malloc(((size_t)len + 1) * sizeof(double));
     double* vals = (double*)malloc(((size_t)len + 1) * d * sizeof(double));
@@ -727,11 +737,11 @@ int or_chunk(int B, int Hkv, int d, int M, int r, int cap,
              int psac_fmt, const uint16_t* psac_scale, const int32_t* table, int page,
              const uint16_t* cent, const float* P, int len,
              const uint16_t* Q, int Hq, int Nq, const uint16_t* Kself, const uint16_t* Vself,
-             int frame_tokens, double sm_scale, const int32_t* rows, int nrows, double* out)
+             int frame_tokens, double sm_scale, const int32_t* rows, int nrows, double* out, int group)
 {
-    if (Hq % Hkv || len < 0 || len > cap || frame_tokens <= 0) return 1;
+    if (Hq % Hkv || len < 0 || len > cap || frame_tokens <= 0 || group <= 0 || d % group) return 1;
     or_cache c = {B, Hkv, d, M, r, cap, k_code, v_code, k_sz, v_sz, cidx, psac, cent, P, psac_fmt, psac_scale,
-                  table, page};
+                  table, page, group};
     int G = Hq / Hkv;
     size_t nmax = (size_t)len + (size_t)Nq + 1;
     double* logit = (double*)malloc(nmax * sizeof(double));
@@ -781,10 +791,11 @@ int or_decode_logits(int Hkv, int d, int M, int r, int cap, int b, int h,
                      const uint32_t* k_code, const uint32_t* k_sz, const void* cidx,
                      const uint16_t* psac, int psac_fmt, const uint16_t* psac_scale,
                      const int32_t* table, int page,
-                     const uint16_t* cent, const float* P, int len, const double* q, double* out)
+                     const uint16_t* cent, const float* P, int len, const double* q, double* out, int group)
 {
+    if (group <= 0 || d % group) return 1;
     or_cache c = {b + 1, Hkv, d, M, r, cap, k_code, k_code, k_sz, k_sz, cidx, psac, cent, P, psac_fmt, psac_scale,
-                  table, page};
+                  table, page, group};
     double* kh = (double*)malloc((size_t)d * sizeof(double));
     double* vh = (double*)malloc((size_t)d * sizeof(double));
     double* u = (double*)malloc(((size_t)r + 1) * sizeof(double));

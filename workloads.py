@@ -29,7 +29,7 @@ from dataclasses import dataclass
 
 import numpy as np
 
-GROUP = 32            # channels per quantization group
+GROUP = 32            # default channels per quantization group (32, 64 or 128)
 GRID = (30, 52)       # latent tokens per 480p frame: 480/16 x 832/16
 FRAME_TOKENS = GRID[0] * GRID[1]
 
@@ -53,6 +53,7 @@ class Spec:
     frame_tokens: int  # tokens per latent frame (chunk mask)
     key_law: str      # "gaussian" | "video" | "long"
     top_energy: float  # share of Query energy in the top-8 directions
+    group: int = GROUP  # channels per (scale, zero) group of the packed cache
 
     @property
     def G(self) -> int:
@@ -317,8 +318,9 @@ def make(name: str, seed: int | None = None, *, with_chunk: bool = True,
 @dataclass
 class PackedCache:
     """Host copy of a packed cache, in the library's layout:
-    k_code/v_code u32 [B][H_kv][cap][d/16], k_sz/v_sz u32 [B][H_kv][cap][d/32]
-    (low half fp16 scale, high half fp16 zero), cidx u8/u16 [B][H_kv][cap],
+    k_code/v_code u32 [B][H_kv][cap][d/16], k_sz/v_sz u32
+    [B][H_kv][cap][d/group] (low half fp16 scale, high half fp16 zero of each
+    group of `group` consecutive channels), cidx u8/u16 [B][H_kv][cap],
     psac fp16 bits [B][H_kv][cap][r] (format 0) or int8 codes [B][H_kv][cap][r]
     with fp16 scale bits psac_scale [B][H_kv][cap] (format 1), centroids fp16
     bits [H_kv][M][d]."""
@@ -339,20 +341,22 @@ class PackedCache:
     psac_scale: np.ndarray | None = None
     table: np.ndarray | None = None    # paged: page ids [B][capacity / page]
     page: int = 0                       # tokens per page (paged)
+    group: int = GROUP                  # channels per (scale, zero) group
 
     @staticmethod
-    def empty(B, H_kv, d, M, r, capacity, centroids, psac_fmt: int = 0):
+    def empty(B, H_kv, d, M, r, capacity, centroids, psac_fmt: int = 0, group: int = GROUP):
         cap = (capacity + 15) // 16 * 16          # the library wants capacity % 16 == 0
+        assert d % group == 0
         return PackedCache(
             B, H_kv, d, M, r, cap,
             np.zeros((B, H_kv, cap, d // 16), np.uint32),
             np.zeros((B, H_kv, cap, d // 16), np.uint32),
-            np.zeros((B, H_kv, cap, d // GROUP), np.uint32),
-            np.zeros((B, H_kv, cap, d // GROUP), np.uint32),
+            np.zeros((B, H_kv, cap, d // group), np.uint32),
+            np.zeros((B, H_kv, cap, d // group), np.uint32),
             np.zeros((B, H_kv, cap), np.uint8 if M <= 256 else np.uint16),
             np.zeros((B, H_kv, cap, max(r, 1)), np.int8 if psac_fmt == 1 else np.uint16),
             centroids, psac_fmt,
-            np.zeros((B, H_kv, cap), np.uint16) if psac_fmt == 1 else None)
+            np.zeros((B, H_kv, cap), np.uint16) if psac_fmt == 1 else None, group=group)
 
 
 def to_paged(pc: PackedCache, page: int, n_pages: int, seed: int = 0) -> PackedCache:
@@ -376,7 +380,7 @@ def to_paged(pc: PackedCache, page: int, n_pages: int, seed: int = 0) -> PackedC
         return out
     return PackedCache(pc.B, pc.H_kv, pc.d, pc.M, pc.r, pc.capacity, pool(pc.k_code), pool(pc.v_code),
                        pool(pc.k_sz), pool(pc.v_sz), pool(pc.cidx), pool(pc.psac), pc.centroids,
-                       pc.psac_fmt, pool(pc.psac_scale), table, page)
+                       pc.psac_fmt, pool(pc.psac_scale), table, page, pc.group)
 
 
 def random_packed_cache(s: Spec, T: int | None = None, seed: int | None = None,
@@ -396,9 +400,9 @@ def random_packed_cache(s: Spec, T: int | None = None, seed: int | None = None,
     cap = (max(s.capacity, T) + 15) // 16 * 16
     if centroids is None:
         centroids = f16_bits(rng.standard_normal((s.H_kv, s.M, s.d)).astype(np.float32))
-    pc = PackedCache.empty(s.B, s.H_kv, s.d, s.M, s.r, cap, centroids, psac_fmt)
+    pc = PackedCache.empty(s.B, s.H_kv, s.d, s.M, s.r, cap, centroids, psac_fmt, s.group)
     sh = (s.B, s.H_kv, T)
-    ng = s.d // GROUP
+    ng = s.d // s.group
     pc.k_code[:, :, :T] = rng.integers(0, 2 ** 32, sh + (s.d // 16,), dtype=np.uint32)
     pc.v_code[:, :, :T] = rng.integers(0, 2 ** 32, sh + (s.d // 16,), dtype=np.uint32)
     for arr, typical in ((pc.k_sz, 0.6), (pc.v_sz, 1.4)):
