@@ -24,7 +24,7 @@ LIB_PATH = os.path.join(_HERE, "libkv2.so")
 KV2_OK = 0
 KV2_OUT_F32 = 0
 KV2_OUT_BF16 = 1
-GROUP = 32
+GROUP = 32          # default channels per (scale, zero) group
 STATUS = {0: "KV2_OK", 1: "KV2_ERR_INVALID_ARG", 2: "KV2_ERR_UNSUPPORTED", 3: "KV2_ERR_CAPACITY",
           4: "KV2_ERR_CUDA", 5: "KV2_ERR_TIMEOUT", 6: "KV2_ERR_WORKSPACE"}
 
@@ -44,7 +44,8 @@ class kv2_cache(ctypes.Structure):
                 ("centroids", ctypes.c_void_p), ("P", ctypes.c_void_p),
                 ("w", ctypes.c_void_p), ("Wg", ctypes.c_void_p),
                 ("psac_fmt", ctypes.c_int32), ("psac_scale", ctypes.c_void_p),
-                ("block_table", ctypes.c_void_p), ("page_tokens", ctypes.c_int32)]
+                ("block_table", ctypes.c_void_p), ("page_tokens", ctypes.c_int32),
+                ("group", ctypes.c_int32)]
 
 
 def _load():
@@ -59,11 +60,11 @@ def _load():
     L.kv2_fit_workspace_size.restype = S
     L.kv2_fit_workspace_size.argtypes = [I, I]
     L.kv2_fit_psac_basis.restype = I
-    L.kv2_fit_psac_basis.argtypes = [P, I, I, I, I, I, P, P, P, P, P, S, P]
+    L.kv2_fit_psac_basis.argtypes = [P, I, I, I, I, I, I, P, P, P, P, P, S, P]
     L.kv2_fit_centroids_workspace_size.restype = S
     L.kv2_fit_centroids_workspace_size.argtypes = [I, I, I]
     L.kv2_fit_centroids.restype = I
-    L.kv2_fit_centroids.argtypes = [P, I, I, I, I, I, P, P, I, P, P, P, S, P]
+    L.kv2_fit_centroids.argtypes = [P, I, I, I, I, I, I, P, P, I, P, P, P, S, P]
     L.kv2_top1_workspace_size.restype = S
     L.kv2_top1_workspace_size.argtypes = [I, I, I, I]
     L.kv2_decode_top1.restype = I
@@ -134,13 +135,17 @@ class Cache:
     read-only centroid table and fitted statistics it points to."""
 
     def __init__(self, B, H_kv, d, M, r, capacity, centroids, device="cuda", psac_fmt=0,
-                 page_tokens=0, num_pages=0):
+                 page_tokens=0, num_pages=0, group=GROUP):
         """page_tokens > 0: a paged cache, its streams a pool of num_pages pages
         of page_tokens tokens; block_table [B][capacity / page_tokens] (int32,
-        device) maps each sequence's pages (initially pages in order)."""
+        device) maps each sequence's pages (initially pages in order). group:
+        channels per (scale, zero) group."""
         if capacity % 16:
             raise ValueError("capacity must be a multiple of 16")
+        if d % group:
+            raise ValueError(f"group {group} does not divide d = {d}")
         self.B, self.H_kv, self.d, self.M, self.r, self.capacity = B, H_kv, d, M, r, capacity
+        self.group = group
         self.psac_fmt = psac_fmt
         self.page_tokens = page_tokens
         if page_tokens:
@@ -155,8 +160,8 @@ class Cache:
         u32 = torch.int32
         self.k_code = torch.zeros(sh + (d // 16,), dtype=u32, device=device)
         self.v_code = torch.zeros(sh + (d // 16,), dtype=u32, device=device)
-        self.k_sz = torch.zeros(sh + (d // GROUP,), dtype=u32, device=device)
-        self.v_sz = torch.zeros(sh + (d // GROUP,), dtype=u32, device=device)
+        self.k_sz = torch.zeros(sh + (d // group,), dtype=u32, device=device)
+        self.v_sz = torch.zeros(sh + (d // group,), dtype=u32, device=device)
         self.cidx = torch.zeros(sh, dtype=torch.uint8 if M <= 256 else torch.int16, device=device)
         self.psac = torch.zeros(sh + (max(r, 1),), dtype=torch.int8 if psac_fmt == 1 else torch.int16,
                                 device=device)
@@ -164,7 +169,7 @@ class Cache:
         self.centroids = torch.as_tensor(centroids).to(device=device, dtype=torch.int16).contiguous()
         self.P = torch.zeros((H_kv, d, max(r, 1)), dtype=torch.float32, device=device)
         self.w = torch.ones((H_kv, d), dtype=torch.float32, device=device)
-        self.Wg = torch.full((H_kv, d // GROUP), float(GROUP), dtype=torch.float32, device=device)
+        self.Wg = torch.full((H_kv, d // group), float(group), dtype=torch.float32, device=device)
         self.energy = torch.zeros(H_kv, dtype=torch.float32, device=device)
 
     def desc(self) -> kv2_cache:
@@ -175,13 +180,13 @@ class Cache:
                          self.P.data_ptr(), self.w.data_ptr(), self.Wg.data_ptr(), self.psac_fmt,
                          self.psac_scale.data_ptr() if self.psac_scale is not None else 0,
                          self.block_table.data_ptr() if self.block_table is not None else 0,
-                         self.page_tokens)
+                         self.page_tokens, self.group)
 
     def set_fit(self, P, w, Wg):
         if self.r:
             self.P.copy_(torch.as_tensor(P).reshape(self.H_kv, self.d, self.r))
         self.w.copy_(torch.as_tensor(w).reshape(self.H_kv, self.d))
-        self.Wg.copy_(torch.as_tensor(Wg).reshape(self.H_kv, self.d // GROUP))
+        self.Wg.copy_(torch.as_tensor(Wg).reshape(self.H_kv, self.d // self.group))
 
     def load_packed(self, pc):
         """Copy a host packed cache (numpy arrays, library layout) in."""
@@ -216,17 +221,18 @@ def kv2_fit_workspace_size(H_kv: int, d: int) -> int:
 
 
 def kv2_fit_psac_basis(Qhist: torch.Tensor, H_kv: int, r: int, P=None, w=None, Wg=None,
-                       energy=None, ws=None, stream=None):
-    """Qhist bf16 [n][H_q][d] (device) -> (P [H_kv][d][r], w [H_kv][d], Wg, energy)."""
+                       energy=None, ws=None, stream=None, group: int = GROUP):
+    """Qhist bf16 [n][H_q][d] (device) -> (P [H_kv][d][r], w [H_kv][d],
+    Wg [H_kv][d/group], energy)."""
     n, H_q, d = Qhist.shape
     dev = Qhist.device
     P = torch.empty((H_kv, d, max(r, 1)), dtype=torch.float32, device=dev) if P is None else P
     w = torch.empty((H_kv, d), dtype=torch.float32, device=dev) if w is None else w
-    Wg = torch.empty((H_kv, d // GROUP), dtype=torch.float32, device=dev) if Wg is None else Wg
+    Wg = torch.empty((H_kv, d // group), dtype=torch.float32, device=dev) if Wg is None else Wg
     energy = torch.empty(H_kv, dtype=torch.float32, device=dev) if energy is None else energy
     need = kv2_fit_workspace_size(H_kv, d)
     ws = torch.empty(need, dtype=torch.uint8, device=dev) if ws is None else ws
-    _check(_get_lib().kv2_fit_psac_basis(_ptr(Qhist), n, H_q, H_kv, d, r, _ptr(P), _ptr(w), _ptr(Wg),
+    _check(_get_lib().kv2_fit_psac_basis(_ptr(Qhist), n, H_q, H_kv, d, r, group, _ptr(P), _ptr(w), _ptr(Wg),
                                   _ptr(energy), _ptr(ws), ws.numel(), _stream(stream)))
     return P[:, :, :r], w, Wg, energy
 
@@ -236,16 +242,17 @@ def kv2_fit_centroids_workspace_size(H_kv: int, d: int, M: int) -> int:
 
 
 def kv2_fit_centroids(X: torch.Tensor, centroids: torch.Tensor, candidates: int, w: torch.Tensor,
-                      Wg: torch.Tensor, iters: int, assign=None, ws=None, stream=None):
+                      Wg: torch.Tensor, iters: int, assign=None, ws=None, stream=None, group: int = GROUP):
     """X bf16 [n][H_kv][d] sample keys, centroids fp16 [H_kv][M][d] (device;
-    updated in place) -> (centroids, assign int32 [n][H_kv])."""
+    updated in place), Wg for groups of ``group`` channels -> (centroids,
+    assign int32 [n][H_kv])."""
     n, H_kv, d = X.shape
     M = centroids.shape[1]
     dev = X.device
     assign = torch.empty((max(n, 1), H_kv), dtype=torch.int32, device=dev) if assign is None else assign
     need = kv2_fit_centroids_workspace_size(H_kv, d, M)
     ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev) if ws is None else ws
-    _check(_get_lib().kv2_fit_centroids(_ptr(X), n, H_kv, d, M, candidates, _ptr(w), _ptr(Wg), iters,
+    _check(_get_lib().kv2_fit_centroids(_ptr(X), n, H_kv, d, M, candidates, group, _ptr(w), _ptr(Wg), iters,
                                         _ptr(centroids), _ptr(assign), _ptr(ws), ws.numel(), _stream(stream)))
     return centroids, assign[:n]
 

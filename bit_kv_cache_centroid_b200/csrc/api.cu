@@ -32,6 +32,17 @@ kv2_status cuda_status(cudaError_t e, const char* what) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Shape and pointer checks common to every call that reads the cache.
+// Channels per (scale, zero) group (0 selects 32). The kernels are
+// instantiated for 32, 64 and 128 channels; this version of the boundary
+// takes 32 only.
+kv2_status check_group(int d, int group) {
+  const int g = group ? group : kv2::kGroup;
+  if (g != 32 && g != 64 && g != 128) return fail(KV2_ERR_UNSUPPORTED, "group=%d (32, 64 or 128)", group);
+  if (g > d) return fail(KV2_ERR_UNSUPPORTED, "group=%d larger than d=%d", g, d);
+  if (g != kv2::kGroup) return fail(KV2_ERR_UNSUPPORTED, "group=%d: this library version takes groups of 32", g);
+  return KV2_OK;
+}
+
 kv2_status check_cache(const kv2_cache* c, bool need_cache_streams, bool need_fit) {
   if (!c) return fail(KV2_ERR_INVALID_ARG, "cache descriptor is NULL");
   if (c->B <= 0 || c->H_kv <= 0 || c->capacity < 0 || c->M <= 0 || c->r < 0)
@@ -40,6 +51,7 @@ kv2_status check_cache(const kv2_cache* c, bool need_cache_streams, bool need_fi
   if (c->d != 64 && c->d != 128) return fail(KV2_ERR_UNSUPPORTED, "head dim d=%d (supported: 64, 128)", c->d);
   if (c->M > kv2::kMaxCentroids) return fail(KV2_ERR_UNSUPPORTED, "M=%d centroids (max 512)", c->M);
   if (c->r > c->d || (c->r & 1)) return fail(KV2_ERR_UNSUPPORTED, "PSAC rank r=%d (even, <= d)", c->r);
+  if (kv2_status st = check_group(c->d, c->group); st != KV2_OK) return st;
   if (c->capacity % 16) return fail(KV2_ERR_UNSUPPORTED, "capacity %d is not a multiple of 16", c->capacity);
   if (c->psac_fmt != 0 && c->psac_fmt != 1) return fail(KV2_ERR_INVALID_ARG, "psac_fmt=%d (0: fp16, 1: int8)", c->psac_fmt);
   if (c->block_table && (c->page_tokens < 128 || c->page_tokens % 128 || c->capacity % c->page_tokens))
@@ -93,25 +105,26 @@ const char* kv2_status_string(kv2_status s) {
 
 const char* kv2_last_error(void) { return g_last_error; }
 
-int kv2_version(void) { return 101; }
+int kv2_version(void) { return 200; }
 
 size_t kv2_fit_workspace_size(int H_kv, int d) {
   if (H_kv <= 0 || (d != 64 && d != 128)) return 0;
   return kv2::fit_workspace_bytes(H_kv, d);
 }
 
-kv2_status kv2_fit_psac_basis(const uint16_t* Qhist, int n, int H_q, int H_kv, int d, int r,
+kv2_status kv2_fit_psac_basis(const uint16_t* Qhist, int n, int H_q, int H_kv, int d, int r, int group,
                               float* P, float* w, float* Wg, float* energy, void* ws,
                               size_t ws_bytes, void* stream) {
   if (n <= 0 || H_q <= 0 || H_kv <= 0 || r < 0) return fail(KV2_ERR_INVALID_ARG, "fit: sizes must be positive");
   if (H_q % H_kv) return fail(KV2_ERR_UNSUPPORTED, "fit: H_q=%d not a multiple of H_kv=%d", H_q, H_kv);
   if (d != 64 && d != 128) return fail(KV2_ERR_UNSUPPORTED, "fit: head dim d=%d (supported: 64, 128)", d);
   if (r > d) return fail(KV2_ERR_UNSUPPORTED, "fit: r=%d > d=%d", r, d);
+  if (kv2_status st = check_group(d, group); st != KV2_OK) return st;
   if (!Qhist || !w || !Wg || !ws || (r && !P)) return fail(KV2_ERR_INVALID_ARG, "fit: NULL pointer");
   if (!aligned16(Qhist) || !aligned16(ws)) return fail(KV2_ERR_INVALID_ARG, "fit: misaligned pointer");
   if (ws_bytes < kv2::fit_workspace_bytes(H_kv, d))
     return fail(KV2_ERR_WORKSPACE, "fit: workspace %zu < %zu bytes", ws_bytes, kv2::fit_workspace_bytes(H_kv, d));
-  kv2::FitArgs a{Qhist, n, H_q, H_kv, d, r, P, w, Wg, energy, ws};
+  kv2::FitArgs a{Qhist, n, H_q, H_kv, d, r, P, w, Wg, energy, ws, group ? group : kv2::kGroup};
   return cuda_status(kv2::launch_fit(a, static_cast<cudaStream_t>(stream)), "fit launch");
 }
 
@@ -152,15 +165,16 @@ size_t kv2_fit_centroids_workspace_size(int H_kv, int d, int M) {
   return kv2::fit_centroids_workspace_bytes(H_kv, d, M);
 }
 
-kv2_status kv2_fit_centroids(const uint16_t* X, int n, int H_kv, int d, int M, int candidates, const float* w,
-                             const float* Wg, int iters, uint16_t* centroids, int32_t* assign, void* ws,
-                             size_t ws_bytes, void* stream) {
+kv2_status kv2_fit_centroids(const uint16_t* X, int n, int H_kv, int d, int M, int candidates, int group,
+                             const float* w, const float* Wg, int iters, uint16_t* centroids, int32_t* assign,
+                             void* ws, size_t ws_bytes, void* stream) {
   if (H_kv <= 0 || n < 0 || n > 65536) return fail(KV2_ERR_INVALID_ARG, "fit_centroids: H_kv=%d, n=%d", H_kv, n);
   if (d != 64 && d != 128) return fail(KV2_ERR_UNSUPPORTED, "fit_centroids: head dim d=%d (supported: 64, 128)", d);
   if (M < 1 || M > 512) return fail(KV2_ERR_UNSUPPORTED, "fit_centroids: M=%d outside 1..512", M);
   if (candidates < 1 || candidates > M)
     return fail(KV2_ERR_INVALID_ARG, "fit_centroids: candidates=%d outside 1..M=%d", candidates, M);
   if (iters < 0) return fail(KV2_ERR_INVALID_ARG, "fit_centroids: iters=%d < 0", iters);
+  if (kv2_status st = check_group(d, group); st != KV2_OK) return st;
   if (iters == 0 || n == 0) return KV2_OK;
   if (!X || !w || !Wg || !centroids || !assign || !ws)
     return fail(KV2_ERR_INVALID_ARG, "fit_centroids: NULL pointer");
@@ -168,7 +182,8 @@ kv2_status kv2_fit_centroids(const uint16_t* X, int n, int H_kv, int d, int M, i
     return fail(KV2_ERR_INVALID_ARG, "fit_centroids: misaligned pointer");
   const size_t need = kv2::fit_centroids_workspace_bytes(H_kv, d, M);
   if (ws_bytes < need) return fail(KV2_ERR_WORKSPACE, "fit_centroids: workspace %zu < %zu bytes", ws_bytes, need);
-  kv2::FitCentroidsArgs a{X, n, H_kv, d, M, candidates, iters, w, Wg, centroids, assign, ws};
+  kv2::FitCentroidsArgs a{X, n, H_kv, d, M, candidates, iters, w, Wg, centroids, assign, ws,
+                          group ? group : kv2::kGroup};
   return cuda_status(kv2::launch_fit_centroids(a, static_cast<cudaStream_t>(stream)), "fit_centroids launch");
 }
 
@@ -196,6 +211,7 @@ kv2::QuantizeArgs quantize_args(const kv2_cache* c, const uint16_t* K, const uin
   a.psac_scale = c->psac_scale;
   a.table = c->block_table;
   a.page = c->page_tokens;
+  a.group = kv2::cache_group(*c);
   return a;
 }
 

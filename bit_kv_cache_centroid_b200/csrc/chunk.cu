@@ -296,15 +296,27 @@ struct ChunkParams {
 // loaded one tile ahead of their use.
 struct RawHalf {
   uint4 kw, vw;       // 4 code words each
-  uint2 ksz, vsz;     // 2 groups: fp16 scale | fp16 zero << 16
+  uint2 ksz, vsz;     // the (fp16 scale | fp16 zero << 16) words of channels
+                      // 64*half .. +31 and 64*half+32 .. +63
   int idx;            // centroid id
 };
 
+// GS: channels per (scale, zero) group (32, 64 or 128): a row holds 128 / GS
+// scale/zero words, and both 32-channel quarters of a half share one word
+// when GS > 32
+template <int GS>
 __device__ __forceinline__ void load_raw_half(const ChunkParams& p, size_t slot, int half, RawHalf& r) {
   r.kw = *reinterpret_cast<const uint4*>(p.k_code + slot * 8 + half * 4);
   r.vw = *reinterpret_cast<const uint4*>(p.v_code + slot * 8 + half * 4);
-  r.ksz = *reinterpret_cast<const uint2*>(p.k_sz + slot * 4 + half * 2);
-  r.vsz = *reinterpret_cast<const uint2*>(p.v_sz + slot * 4 + half * 2);
+  if constexpr (GS == 32) {
+    r.ksz = *reinterpret_cast<const uint2*>(p.k_sz + slot * 4 + half * 2);
+    r.vsz = *reinterpret_cast<const uint2*>(p.v_sz + slot * 4 + half * 2);
+  } else {
+    constexpr int NG = kD / GS;
+    const uint32_t k = p.k_sz[slot * NG + (half * 64) / GS], v = p.v_sz[slot * NG + (half * 64) / GS];
+    r.ksz = make_uint2(k, k);
+    r.vsz = make_uint2(v, v);
+  }
   r.idx = (p.M <= 256) ? int(static_cast<const uint8_t*>(p.cidx)[slot])
                        : int(static_cast<const uint16_t*>(p.cidx)[slot]);
 }
@@ -406,6 +418,7 @@ __device__ __forceinline__ void zero_half(uint8_t* tile, int row, int half) {
 }
 
 // ---------------------------------------------------------------------------
+template <int GS>
 __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -576,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
     const uint4* cent4 = reinterpret_cast<const uint4*>(p.cent) + size_t(h) * p.M * (kD / 8) + half * 8;
     RawHalf raw;
     bool raw_ok = nloc > 0 && jA < n_cache && row < min(kKeys, p.len - jA * kKeys);
-    if (raw_ok) load_raw_half(p, slot_of(jA * kKeys + row), half, raw);
+    if (raw_ok) load_raw_half<GS>(p, slot_of(jA * kKeys + row), half, raw);
     for (int jj = 0; jj < nloc; ++jj) {
       const int j = jA + jj;
       const int s = jj & 1;
@@ -594,7 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
       RawHalf next;
       const int jn = j + 1;
       const bool next_ok = jn < jB && jn < n_cache && row < min(kKeys, p.len - jn * kKeys);
-      if (next_ok) load_raw_half(p, slot_of(jn * kKeys + row), half, next);
+      if (next_ok) load_raw_half<GS>(p, slot_of(jn * kKeys + row), half, next);
       if (use >= 1 && !mbar_wait_or_abort(bar + B_KV_EMPTY + 8 * s, (use - 1) & 1, p.budget, abort)) break;
       uint8_t* stage = smem + OFF_STAGE + s * STAGE_BYTES;
       if (row < kvalid) {
@@ -877,11 +890,13 @@ cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t s) {
   p.part = reinterpret_cast<float*>(static_cast<char*>(a.ws) + kChunkWsHeader);
   cudaError_t e = cudaMemsetAsync(a.ws, 0, sizeof(int), s);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(chunk_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SMEM_ALLOC));
+  const int group = cache_group(c);
+  auto kern = group == 128 ? chunk_attn_kernel<128> : group == 64 ? chunk_attn_kernel<64> : chunk_attn_kernel<32>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SMEM_ALLOC));
   if (e != cudaSuccess) return e;
   const int items = p.n_full + pl.split * pl.pieces;
   if (items == 0) return cudaSuccess;
-  chunk_attn_kernel<<<items, kThreads, SMEM_ALLOC, s>>>(p);
+  kern<<<items, kThreads, SMEM_ALLOC, s>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess || pl.split == 0) return e;
   chunk_merge<<<pl.split * 2 * kRows, kD, 0, s>>>(p.part, p.n_full, pl.pieces, pl.QP, a.H_q, a.Nq, a.out,

@@ -6,7 +6,8 @@
 // components use statistics of already generated Queries. Here:
 //   S_h  = (1/N) sum q q^T over the N = n*G history queries of KV head h's
 //          query-head group (uncentred second moment, fp64);
-//   w    = diag(S) (per-channel sensitivity, fp32), Wg = per-group sums of w;
+//   w    = diag(S) (per-channel sensitivity, fp32), Wg = per-group sums of w
+//          (groups of 32, 64 or 128 consecutive channels);
 //   P    = top-r eigenvectors of S (descending eigenvalues, largest-magnitude
 //          entry positive), energy = top-r share of trace(S).
 // Kernels: fit_gram (fp64 32x32 output tiles), fit_jacobi (one CTA per head:
@@ -83,7 +84,8 @@ constexpr int kJacobiThreads = 512;
 __global__ void __launch_bounds__(kJacobiThreads) fit_jacobi(const double* __restrict__ S_all,
                                                              double* __restrict__ Vt_all, int D, int r,
                                                              float* __restrict__ P, float* __restrict__ w,
-                                                             float* __restrict__ Wg, float* __restrict__ energy) {
+                                                             float* __restrict__ Wg, float* __restrict__ energy,
+                                                             int group) {
   constexpr int NT = kJacobiThreads;
   extern __shared__ __align__(16) unsigned char smem[];
   double* A = reinterpret_cast<double*>(smem);             // [D][D]
@@ -103,10 +105,11 @@ __global__ void __launch_bounds__(kJacobiThreads) fit_jacobi(const double* __res
   // sensitivity weights from the diagonal
   for (int c = tid; c < D; c += NT) w[size_t(h) * D + c] = float(S[size_t(c) * D + c]);
   __syncthreads();
-  if (tid < D / 32) {
+  // group sensitivities: w summed over each group's channels in ascending order
+  if (tid < D / group) {
     float acc = 0.0f;
-    for (int c = tid * 32; c < tid * 32 + 32; ++c) acc = __fadd_rn(acc, w[size_t(h) * D + c]);
-    Wg[size_t(h) * (D / 32) + tid] = acc;
+    for (int c = tid * group; c < tid * group + group; ++c) acc = __fadd_rn(acc, w[size_t(h) * D + c]);
+    Wg[size_t(h) * (D / group) + tid] = acc;
   }
   // total squared norm (convergence reference)
   double tot = 0.0;
@@ -221,7 +224,7 @@ cudaError_t launch_fit(const FitArgs& a, cudaStream_t s) {
   const size_t smem = size_t(D) * D * 8 + size_t(D) * 8 + kJacobiThreads * 8 + size_t(D) * 4 + size_t(D) * 4;
   e = cudaFuncSetAttribute(fit_jacobi, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  fit_jacobi<<<a.H_kv, kJacobiThreads, smem, s>>>(S, Vt, D, a.r, a.P, a.w, a.Wg, a.energy);
+  fit_jacobi<<<a.H_kv, kJacobiThreads, smem, s>>>(S, Vt, D, a.r, a.P, a.w, a.Wg, a.energy, a.group);
   return cudaGetLastError();
 }
 

@@ -103,6 +103,7 @@ cudaError_t launch_fit_centroids(const FitCentroidsArgs& a, cudaStream_t s) {
   q.P = nullptr;
   q.w = a.w;
   q.Wg = a.Wg;
+  q.group = a.group;
   q.assign = a.assign;
   for (int it = 0; it < a.iters; ++it) {
     e = launch_quantize(q, s);

@@ -12,8 +12,11 @@
 
 namespace kv2 {
 
-constexpr int kGroup = 32;          // channels per quantization group
+constexpr int kGroup = 32;          // channels of a sub-group: one code-word pair, one 8-bit q.k k-step
 constexpr int kMaxCentroids = 512;  // centroid ids fit in u16 above 256
+
+// Channels per (scale, zero) group of a cache descriptor (0 selects 32).
+inline int cache_group(const kv2_cache& c) { return c.group ? c.group : kGroup; }
 
 // Arguments of one quantize/append call (validated by the host entry point).
 struct QuantizeArgs {
@@ -23,7 +26,7 @@ struct QuantizeArgs {
   const uint16_t* cent;  // fp16 [H][M][d]
   const float* P;        // [H][d][r]
   const float* w;        // [H][d]
-  const float* Wg;       // [H][d/32]
+  const float* Wg;       // [H][d/group]
   uint32_t* k_code;
   uint32_t* v_code;
   uint32_t* k_sz;
@@ -41,6 +44,7 @@ struct QuantizeArgs {
   // paged cache: block table [B][cap / page] (null: contiguous streams)
   const int32_t* table = nullptr;
   int page = 0;
+  int group = kGroup;  // channels per (scale, zero) group: 32, 64 or 128
 };
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s);
 
@@ -49,10 +53,11 @@ struct FitCentroidsArgs {
   const uint16_t* X;   // bf16 [n][H][D] sample keys
   int n, H, D, M, C, iters;
   const float* w;      // [H][D]
-  const float* Wg;     // [H][D/32]
+  const float* Wg;     // [H][D/group]
   uint16_t* cent;      // fp16 [H][M][D], initial centres in, fitted centres out
   int32_t* assign;     // [n][H]: the last assignment
   void* ws;            // fit_centroids_workspace_bytes(H, D, M)
+  int group = kGroup;  // channels per (scale, zero) group of the QSAC estimate
 };
 size_t fit_centroids_workspace_bytes(int H, int D, int M);
 
@@ -98,6 +103,7 @@ struct FitArgs {
   float* Wg;
   float* energy;
   void* ws;
+  int group = kGroup;     // Wg sums w over groups of this many channels
 };
 size_t fit_workspace_bytes(int H_kv, int d);
 cudaError_t launch_fit(const FitArgs& a, cudaStream_t s);

@@ -50,11 +50,14 @@ struct QCfg {
   static size_t smem(int C, int r, int r8) { return head_bytes(r) + size_t(kWarps) * warp_bytes(C, r8); }
 };
 
-template <int D, int CPL, int KPT>
+// GS: channels per (scale, zero) group (32, 64 or 128); a group is SPG
+// sub-groups of 32 channels (one code-word pair each)
+template <int D, int CPL, int KPT, int GS>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
   using Cfg = QCfg<D, CPL, KPT>;
   constexpr int MP = Cfg::MP, KT = Cfg::KT;
-  constexpr int NG = D / kGroup;
+  constexpr int NG = D / GS, NS = D / kGroup, SPG = GS / kGroup;
+  static_assert(GS % kGroup == 0 && D % GS == 0, "groups of whole 32-channel sub-groups");
   extern __shared__ __align__(16) unsigned char smem[];
   __half* mu_s = reinterpret_cast<__half*>(smem);                            // [D][MP]
   float* nrm_s = reinterpret_cast<float*>(smem + Cfg::mu_bytes);              // [MP]
@@ -261,11 +264,11 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
       const int row = row_of(0);
       const uint16_t* krow = key_ptr(a.K, row);
       const uint16_t* vrow = key_ptr(a.V, row);
-      float kx[NG], vx[NG];                            // channel g * 32 + lane
+      float kx[NS], vx[NS];                            // channel k * 32 + lane of sub-group k
 #pragma unroll
-      for (int g = 0; g < NG; ++g) {
-        kx[g] = __uint_as_float(uint32_t(krow[g * kGroup + lane]) << 16);
-        vx[g] = a.assign ? 0.0f : __uint_as_float(uint32_t(vrow[g * kGroup + lane]) << 16);
+      for (int k = 0; k < NS; ++k) {
+        kx[k] = __uint_as_float(uint32_t(krow[k * kGroup + lane]) << 16);
+        vx[k] = a.assign ? 0.0f : __uint_as_float(uint32_t(vrow[k * kGroup + lane]) << 16);
       }
       // ---- perturbation estimate: lane (candidate i, group g) takes the
       // group's scale; E_i = fmaf chain over ascending g of (W_g s_g) s_g;
@@ -279,16 +282,16 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
           if (i < C) {
             const int j = cand_w[i];
             const int col = (j % 32) * CPL + j / 32;
-            const uint16_t* kseg = krow + g * kGroup;
+            const uint16_t* kseg = krow + g * GS;
             float mn = FLT_MAX, mx = -FLT_MAX;
 #pragma unroll
-            for (int c = 0; c < kGroup; c += 8) {
+            for (int c = 0; c < GS; c += 8) {
               const uint4 kv = *reinterpret_cast<const uint4*>(kseg + c);
               const uint32_t ku[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
-                const float m0 = __half2float(mu_s[(g * kGroup + c + 2 * q) * MP + col]);
-                const float m1 = __half2float(mu_s[(g * kGroup + c + 2 * q + 1) * MP + col]);
+                const float m0 = __half2float(mu_s[(g * GS + c + 2 * q) * MP + col]);
+                const float m1 = __half2float(mu_s[(g * GS + c + 2 * q + 1) * MP + col]);
                 const float x0 = __fsub_rn(__uint_as_float(ku[q] << 16), m0);
                 const float x1 = __fsub_rn(__uint_as_float(ku[q] & 0xffff0000u), m1);
                 mn = fmin3(mn, x0, x1);
@@ -315,36 +318,53 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
       if (a.assign) {
         if (lane == 0) a.assign[size_t(row) * a.H + h] = jc;
       } else {
-      // ---- K residual and V codecs, lane = channel of the group
+      // ---- K residual and V codecs, lane = channel of each 32-channel
+      // sub-group; a group's range spans its SPG sub-groups and the lanes
       const int colc = (jc % 32) * CPL + jc / 32;
       const size_t slot = slot_of(row);
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
-          const int c = g * kGroup + lane;
-          const float x = (which == 0) ? __fsub_rn(kx[g], __half2float(mu_s[c * MP + colc])) : vx[g];
-          float mn = x, mx = x;
+          float x[SPG];
+#pragma unroll
+          for (int u = 0; u < SPG; ++u) {
+            const int k = g * SPG + u, c = k * kGroup + lane;
+            x[u] = (which == 0) ? __fsub_rn(kx[k], __half2float(mu_s[c * MP + colc])) : vx[k];
+          }
+          float mn = x[0], mx = x[0];
+#pragma unroll
+          for (int u = 1; u < SPG; ++u) {
+            mn = fminf(mn, x[u]);
+            mx = fmaxf(mx, x[u]);
+          }
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) {
             mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
           }
           const GroupParams gp = group_params(mn, mx);
-          const uint32_t q = group_code_recip(x, gp, __frcp_rn(gp.s));
-          const uint32_t bits = q << (2 * (lane & 15));
-          const uint32_t w0 = __reduce_or_sync(0xffffffffu, lane < 16 ? bits : 0u);
-          const uint32_t w1 = __reduce_or_sync(0xffffffffu, lane >= 16 ? bits : 0u);
+          const float inv_s = __frcp_rn(gp.s);
+#pragma unroll
+          for (int u = 0; u < SPG; ++u) {
+            const int k = g * SPG + u, c = k * kGroup + lane;
+            const uint32_t q = group_code_recip(x[u], gp, inv_s);
+            const uint32_t bits = q << (2 * (lane & 15));
+            const uint32_t w0 = __reduce_or_sync(0xffffffffu, lane < 16 ? bits : 0u);
+            const uint32_t w1 = __reduce_or_sync(0xffffffffu, lane >= 16 ? bits : 0u);
+            if (lane == 0) {
+              uint32_t* code = (which == 0 ? a.k_code : a.v_code) + slot * (D / 16) + k * 2;
+              *reinterpret_cast<uint2*>(code) = make_uint2(w0, w1);
+            }
+            if (which == 0) e_w[c] = __fsub_rn(x[u], group_dequant(q, gp));
+          }
           if (lane == 0) {
-            uint32_t* code = (which == 0 ? a.k_code : a.v_code) + slot * (D / 16) + g * 2;
-            *reinterpret_cast<uint2*>(code) = make_uint2(w0, w1);
             (which == 0 ? a.k_sz : a.v_sz)[slot * NG + g] = uint32_t(gp.s_bits) | (uint32_t(gp.z_bits) << 16);
             if (which == 0 && g == 0) {
               if (M <= 256) static_cast<uint8_t*>(a.cidx)[slot] = uint8_t(jc);
               else static_cast<uint16_t*>(a.cidx)[slot] = uint16_t(jc);
             }
           }
-          if (which == 0) e_w[c] = __fsub_rn(x, group_dequant(q, gp));
         }
       }
       __syncwarp();
@@ -395,7 +415,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
         for (int g = 0; g < NG; ++g) {
           float mn = FLT_MAX, mx = -FLT_MAX;
 #pragma unroll
-          for (int c = g * kGroup; c < (g + 1) * kGroup; c += 8) {
+          for (int c = g * GS; c < (g + 1) * GS; c += 8) {
             const uint4 kv = *reinterpret_cast<const uint4*>(krow + c);
             const uint32_t ku[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
@@ -422,60 +442,80 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
         a.assign[size_t(row_of(k)) * a.H + h] = cand_w[k * C + rank];
       }
     } else {
-    // ---- K residual and V codecs per (key, group)
+    // ---- K residual and V codecs per (key, group); a group larger than 32
+    // channels takes its range over all its sub-groups first, then codes
+    // them one sub-group at a time (residuals recomputed)
     for (int task = lane; task < nk * NG * 2; task += 32) {
       const int which = task / (nk * NG);   // 0: keys, 1: values
       const int kg = task - which * nk * NG;
       const int k = kg / NG, g = kg - k * NG;
       const int row = row_of(k);
       const size_t slot = slot_of(row);
-      float x[kGroup];
-      int j = 0;
+      int j = 0, col = 0;
       if (which == 0) {
         const int rank = (C > 1) ? int(best_w[k] & 0xffffffffu) : 0;
         j = cand_w[k * C + rank];
-        const int col = (j % 32) * CPL + j / 32;
-        const uint16_t* krow = key_ptr(a.K, row) + g * kGroup;
-#pragma unroll
-        for (int c = 0; c < kGroup; c += 8) {
-          const uint4 kv = *reinterpret_cast<const uint4*>(krow + c);
-          const uint32_t ku[4] = {kv.x, kv.y, kv.z, kv.w};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            x[c + 2 * q] = __fsub_rn(__uint_as_float(ku[q] << 16), __half2float(mu_s[(g * kGroup + c + 2 * q) * MP + col]));
-            x[c + 2 * q + 1] = __fsub_rn(__uint_as_float(ku[q] & 0xffff0000u),
-                                         __half2float(mu_s[(g * kGroup + c + 2 * q + 1) * MP + col]));
-          }
-        }
-      } else {
-        const uint16_t* vrow = key_ptr(a.V, row) + g * kGroup;
-#pragma unroll
-        for (int c = 0; c < kGroup; c += 8) {
-          const uint4 vv = *reinterpret_cast<const uint4*>(vrow + c);
-          const uint32_t vu[4] = {vv.x, vv.y, vv.z, vv.w};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            x[c + 2 * q] = __uint_as_float(vu[q] << 16);
-            x[c + 2 * q + 1] = __uint_as_float(vu[q] & 0xffff0000u);
-          }
-        }
+        col = (j % 32) * CPL + j / 32;
       }
+      // the 32 residuals (keys) or values (which = 1) of channels c0 .. c0 + 31
+      auto load32 = [&](int c0, float (&x)[kGroup]) {
+        if (which == 0) {
+          const uint16_t* krow = key_ptr(a.K, row) + c0;
+#pragma unroll
+          for (int c = 0; c < kGroup; c += 8) {
+            const uint4 kv = *reinterpret_cast<const uint4*>(krow + c);
+            const uint32_t ku[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              x[c + 2 * q] = __fsub_rn(__uint_as_float(ku[q] << 16), __half2float(mu_s[(c0 + c + 2 * q) * MP + col]));
+              x[c + 2 * q + 1] = __fsub_rn(__uint_as_float(ku[q] & 0xffff0000u),
+                                           __half2float(mu_s[(c0 + c + 2 * q + 1) * MP + col]));
+            }
+          }
+        } else {
+          const uint16_t* vrow = key_ptr(a.V, row) + c0;
+#pragma unroll
+          for (int c = 0; c < kGroup; c += 8) {
+            const uint4 vv = *reinterpret_cast<const uint4*>(vrow + c);
+            const uint32_t vu[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              x[c + 2 * q] = __uint_as_float(vu[q] << 16);
+              x[c + 2 * q + 1] = __uint_as_float(vu[q] & 0xffff0000u);
+            }
+          }
+        }
+      };
+      float x[kGroup];
+      load32(g * GS, x);
       float mn = x[0], mx = x[0];
 #pragma unroll
       for (int c = 1; c + 1 < kGroup; c += 2) { mn = fmin3(mn, x[c], x[c + 1]); mx = fmax3(mx, x[c], x[c + 1]); }
       mn = fminf(mn, x[kGroup - 1]);
       mx = fmaxf(mx, x[kGroup - 1]);
+#pragma unroll 1
+      for (int u = 1; u < SPG; ++u) {
+        float y[kGroup];
+        load32(g * GS + u * kGroup, y);
+#pragma unroll
+        for (int c = 0; c + 1 < kGroup; c += 2) { mn = fmin3(mn, y[c], y[c + 1]); mx = fmax3(mx, y[c], y[c + 1]); }
+      }
       const GroupParams p = group_params(mn, mx);
       const float inv_s = __frcp_rn(p.s);
-      uint32_t w0 = 0, w1 = 0;
+#pragma unroll 1
+      for (int u = 0; u < SPG; ++u) {
+        if (u > 0) load32(g * GS + u * kGroup, x);
+        const int c0 = g * GS + u * kGroup;
+        uint32_t w0 = 0, w1 = 0;
 #pragma unroll
-      for (int c = 0; c < kGroup; ++c) {
-        const uint32_t q = group_code_recip(x[c], p, inv_s);
-        if (c < 16) w0 |= q << (2 * c); else w1 |= q << (2 * (c - 16));
-        if (which == 0) e_w[k * D + g * kGroup + c] = __fsub_rn(x[c], group_dequant(q, p));
+        for (int c = 0; c < kGroup; ++c) {
+          const uint32_t q = group_code_recip(x[c], p, inv_s);
+          if (c < 16) w0 |= q << (2 * c); else w1 |= q << (2 * (c - 16));
+          if (which == 0) e_w[k * D + c0 + c] = __fsub_rn(x[c], group_dequant(q, p));
+        }
+        uint32_t* code = (which == 0 ? a.k_code : a.v_code) + slot * (D / 16) + c0 / 16;
+        *reinterpret_cast<uint2*>(code) = make_uint2(w0, w1);
       }
-      uint32_t* code = (which == 0 ? a.k_code : a.v_code) + slot * (D / 16) + g * 2;
-      *reinterpret_cast<uint2*>(code) = make_uint2(w0, w1);
       (which == 0 ? a.k_sz : a.v_sz)[slot * NG + g] = uint32_t(p.s_bits) | (uint32_t(p.z_bits) << 16);
       if (which == 0 && g == 0) {
         if (M <= 256) static_cast<uint8_t*>(a.cidx)[slot] = uint8_t(j);
@@ -508,11 +548,11 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
   }
 }
 
-template <int D, int CPL, int KPT>
+template <int D, int CPL, int KPT, int GS>
 cudaError_t launch_cfg(const QuantizeArgs& a, cudaStream_t s) {
   using Cfg = QCfg<D, CPL, KPT>;
   const size_t smem = Cfg::smem(a.C, a.r, a.psac_fmt == 1 ? a.r : 0);
-  auto kern = quantize_kernel<D, CPL, KPT>;
+  auto kern = quantize_kernel<D, CPL, KPT, GS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   // the SM's shared-memory split as large as the attention kernels': an SM
@@ -536,28 +576,40 @@ cudaError_t launch_cfg(const QuantizeArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-template <int D>
+template <int D, int GS>
 cudaError_t launch_d(const QuantizeArgs& a, cudaStream_t s) {
   const int mp = (a.M + 31) / 32;
   if (a.B * a.n_new <= 8 * kWarps) {            // short appends: one key per warp and tile
-    if (mp <= 1) return launch_cfg<D, 1, 1>(a, s);
-    if (mp <= 2) return launch_cfg<D, 2, 1>(a, s);
-    if (mp <= 4) return launch_cfg<D, 4, 1>(a, s);
-    if (mp <= 8) return launch_cfg<D, 8, 1>(a, s);
-    return launch_cfg<D, 16, 1>(a, s);
+    if (mp <= 1) return launch_cfg<D, 1, 1, GS>(a, s);
+    if (mp <= 2) return launch_cfg<D, 2, 1, GS>(a, s);
+    if (mp <= 4) return launch_cfg<D, 4, 1, GS>(a, s);
+    if (mp <= 8) return launch_cfg<D, 8, 1, GS>(a, s);
+    return launch_cfg<D, 16, 1, GS>(a, s);
   }
-  if (mp <= 1) return launch_cfg<D, 1, 16>(a, s);
-  if (mp <= 2) return launch_cfg<D, 2, 16>(a, s);
-  if (mp <= 4) return launch_cfg<D, 4, 16>(a, s);
-  if (mp <= 8) return launch_cfg<D, 8, 8>(a, s);
-  return launch_cfg<D, 16, 4>(a, s);
+  if (mp <= 1) return launch_cfg<D, 1, 16, GS>(a, s);
+  if (mp <= 2) return launch_cfg<D, 2, 16, GS>(a, s);
+  if (mp <= 4) return launch_cfg<D, 4, 16, GS>(a, s);
+  if (mp <= 8) return launch_cfg<D, 8, 8, GS>(a, s);
+  return launch_cfg<D, 16, 4, GS>(a, s);
 }
 
 }  // namespace
 
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s) {
   if (a.B * a.n_new == 0) return cudaSuccess;
-  return a.d == 64 ? launch_d<64>(a, s) : launch_d<128>(a, s);
+  if (a.d == 64) {
+    switch (a.group) {
+      case 32: return launch_d<64, 32>(a, s);
+      case 64: return launch_d<64, 64>(a, s);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  switch (a.group) {
+    case 32: return launch_d<128, 32>(a, s);
+    case 64: return launch_d<128, 64>(a, s);
+    case 128: return launch_d<128, 128>(a, s);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace kv2

@@ -37,6 +37,7 @@ struct Top1Params {
   const float* P;
   const int32_t* table;     // paged cache: block table (null: contiguous)
   int page;
+  int group;                // channels per (scale, zero) group
   int B, nq, H_q, H_kv, d, M, r, cap, len, psac_fmt, splits;
   unsigned long long* part;  // [B*nq*H_q][splits]: (order key of the logit << 32) | ~index
 };
@@ -75,7 +76,7 @@ __global__ void __launch_bounds__(kTopThreads) top1_split(Top1Params p) {
                                  : int(static_cast<const uint16_t*>(p.cidx)[slot]);
       const uint16_t* mu = p.cent + (size_t(h) * p.M + min(j, p.M - 1)) * p.d;
       for (int c = 0; c < p.d; ++c) {
-        const uint32_t sz = p.k_sz[slot * (p.d / 32) + c / 32];
+        const uint32_t sz = p.k_sz[slot * (p.d / p.group) + c / p.group];
         const float s = f16_to_f32(uint16_t(sz & 0xffff)), z = f16_to_f32(uint16_t(sz >> 16));
         const uint32_t code = (p.k_code[slot * (p.d / 16) + c / 16] >> (2 * (c % 16))) & 3u;
         acc = fmaf(q[c], fmaf(float(code), s, z) + f16_to_f32(mu[c]), acc);
@@ -146,6 +147,7 @@ cudaError_t launch_top1(const Top1Args& a, cudaStream_t s) {
     p.psac_fmt = c.psac_fmt;
     p.table = c.block_table;
     p.page = c.page_tokens;
+    p.group = cache_group(c);
   }
   p.splits = a.len > 0 ? (a.len + kTokensPerCta - 1) / kTokensPerCta : 1;
   p.part = static_cast<unsigned long long*>(a.ws);

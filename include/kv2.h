@@ -21,7 +21,9 @@
  *    enqueued asynchronously; argument errors are returned synchronously
  *    before anything is enqueued; a failed launch returns KV2_ERR_CUDA.
  *  - Supported shapes: head dim d in {64, 128}; quantization groups of 32
- *    channels; 1 <= M <= 512 centroids per KV head (ids stored as u8 when
+ *    channels (the `group` field and argument below; 64 and 128, group <= d,
+ *    are part of the format and return KV2_ERR_UNSUPPORTED from this
+ *    version of the library); 1 <= M <= 512 centroids per KV head (ids stored as u8 when
  *    M <= 256, else u16); 0 <= r <= d PSAC rank (r a multiple of 8 for the
  *    chunk kernel, r <= 16 there); H_q a multiple of H_kv. Anything else
  *    returns KV2_ERR_UNSUPPORTED.
@@ -57,9 +59,10 @@ enum { KV2_OUT_F32 = 0, KV2_OUT_BF16 = 1 };
  * KV head h) every stream is contiguous along tokens, slot = (b*H_kv + h)*capacity + t:
  *   k_code, v_code : uint32 [B][H_kv][capacity][d/16]; channel c of a token is
  *                    in word c/16 at bits 2(c%16)..2(c%16)+1 (INT2 codes 0..3)
- *   k_sz, v_sz     : uint32 [B][H_kv][capacity][d/32]; per 32-channel group,
- *                    low half = fp16 scale s, high half = fp16 zero z; the
- *                    dequantized value of code q is fmaf(q, s, z)
+ *   k_sz, v_sz     : uint32 [B][H_kv][capacity][d/group]; per group of `group`
+ *                    consecutive channels (group g = channels g*group ..
+ *                    g*group + group - 1), low half = fp16 scale s, high half =
+ *                    fp16 zero z; the dequantized value of code q is fmaf(q, s, z)
  *   cidx           : centroid id per token, uint8 (M <= 256) or uint16 [B][H_kv][capacity]
  *   psac           : PSAC coefficients a = P^T e, [B][H_kv][capacity][r]:
  *                    fp16 (psac_fmt 0), or int8 codes (psac_fmt 1) whose
@@ -73,8 +76,12 @@ enum { KV2_OUT_F32 = 0, KV2_OUT_BF16 = 1 };
  * any number of pages, shared by the sequences through their tables.
  *   centroids      : fp16 [H_kv][M][d] (read-only; shared by the batch)
  *   P, w, Wg       : fp32 [H_kv][d][r] basis, [H_kv][d] channel sensitivities,
- *                    [H_kv][d/32] group sensitivities, as written by
- *                    kv2_fit_psac_basis (read-only)
+ *                    [H_kv][d/group] group sensitivities, as written by
+ *                    kv2_fit_psac_basis with the same group (read-only)
+ *   group          : channels per (scale, zero) group: 32 (0 also selects 32),
+ *                    64 or 128. Larger groups store fewer scales and zeros (the
+ *                    compression QuantWM's evaluation counts) at a coarser INT2
+ *                    grid.
  * A key is reconstructed as centroid[cidx] + fmaf(code, s, z) (+ P a for the
  * logit correction), a value as fmaf(code, s, z).
  */
@@ -94,6 +101,7 @@ typedef struct kv2_cache {
   uint16_t* psac_scale;
   const int32_t* block_table;  /* paged cache: page ids [B][capacity / page_tokens]; NULL: contiguous */
   int32_t page_tokens;         /* tokens per page (a multiple of 128) when block_table is set */
+  int32_t group;               /* channels per (scale, zero) group; 0 selects 32 */
 } kv2_cache;
 
 /* Human-readable name of a status. Never NULL. */
@@ -102,7 +110,8 @@ const char* kv2_status_string(kv2_status s);
 /* Detail of the last error returned on the calling host thread ("" if none). */
 const char* kv2_last_error(void);
 
-/* Library ABI version (major*100 + minor). */
+/* Library ABI version (major*100 + minor). 200: the group field of kv2_cache
+ * and the group argument of kv2_fit_psac_basis / kv2_fit_centroids. */
 int kv2_version(void);
 
 /*
@@ -119,15 +128,19 @@ size_t kv2_fit_workspace_size(int H_kv, int d);
  *          statistics pool the n*G vectors of its query heads h*G..h*G+G-1
  *          (G = H_q/H_kv).
  * Outputs (fp32, device): S = (1/(n*G)) sum q q^T (uncentred second moment),
- *   w[h][c] = S_cc; Wg[h][g] = sum of w over group g's 32 channels;
+ *   w[h][c] = S_cc; Wg[h][g] = sum of w over group g's `group` channels
+ *   (ascending channel order, fp32), Wg of [H_kv][d/group];
  *   P[h][c][i] = i-th eigenvector of S by decreasing eigenvalue (i < r), sign
  *   fixed so its largest-magnitude entry is positive; energy[h] (may be NULL)
  *   = share of trace(S) in the top r eigenvalues.
  * Method on the device: fp64 Gram accumulation, cyclic Jacobi in fp64.
+ * group: channels per (scale, zero) group of the cache the statistics serve
+ *   (32, or 0 for 32; 64 and 128 return KV2_ERR_UNSUPPORTED from this
+ *   version).
  * ws: device workspace of kv2_fit_workspace_size(H_kv, d) bytes.
  */
 kv2_status kv2_fit_psac_basis(const uint16_t* Qhist, int n, int H_q, int H_kv, int d,
-                              int r, float* P, float* w, float* Wg, float* energy,
+                              int r, int group, float* P, float* w, float* Wg, float* energy,
                               void* ws, size_t ws_bytes, void* stream);
 
 /*
@@ -148,7 +161,9 @@ size_t kv2_fit_centroids_workspace_size(int H_kv, int d, int M);
  * the count in fp64, times 2^-24, rounded to fp16 (nearest even).
  * X        : bf16 [n][H_kv][d] sample keys (read-only), n <= 65536,
  *            |k| < 2^23 (so the 64-bit sums cannot overflow).
- * w, Wg    : the sensitivities of kv2_fit_psac_basis (read-only).
+ * w, Wg    : the sensitivities of kv2_fit_psac_basis (read-only), Wg for
+ *            groups of `group` channels (32, or 0 for 32; 64 and 128 return
+ *            KV2_ERR_UNSUPPORTED from this version).
  * centroids: fp16 [H_kv][M][d], initial centres in, fitted centres out.
  * assign   : int32 [n][H_kv] out: the assignment of the last iteration.
  * iters >= 0 iterations (0 leaves everything unchanged); candidates 1..M.
@@ -158,7 +173,7 @@ size_t kv2_fit_centroids_workspace_size(int H_kv, int d, int M);
  * candidates outside 1..M, iters < 0), KV2_ERR_UNSUPPORTED (d not 64/128,
  * M outside 1..512), KV2_ERR_WORKSPACE.
  */
-kv2_status kv2_fit_centroids(const uint16_t* X, int n, int H_kv, int d, int M, int candidates,
+kv2_status kv2_fit_centroids(const uint16_t* X, int n, int H_kv, int d, int M, int candidates, int group,
                              const float* w, const float* Wg, int iters, uint16_t* centroids,
                              int32_t* assign, void* ws, size_t ws_bytes, void* stream);
 

@@ -72,7 +72,7 @@ def to_dev(x, dtype=None):
 def host_cache(s: wl.Spec, centroids, capacity=None, psac_fmt=0):
     cap = s.capacity if capacity is None else capacity
     cap = (cap + 15) // 16 * 16
-    return wl.PackedCache.empty(s.B, s.H_kv, s.d, s.M, s.r, cap, centroids, psac_fmt)
+    return wl.PackedCache.empty(s.B, s.H_kv, s.d, s.M, s.r, cap, centroids, psac_fmt, s.group)
 
 
 def gpu_cache_like(pc, fit=None):
@@ -83,7 +83,8 @@ def gpu_cache_like(pc, fit=None):
     paged = getattr(pc, "table", None) is not None
     c = kv2.Cache(pc.B, pc.H_kv, pc.d, pc.M, pc.r, pc.capacity,
                   torch.from_numpy(pc.centroids.view(np.int16)), psac_fmt=getattr(pc, "psac_fmt", 0),
-                  page_tokens=pc.page if paged else 0, num_pages=pc.k_code.shape[0] if paged else 0)
+                  page_tokens=pc.page if paged else 0, num_pages=pc.k_code.shape[0] if paged else 0,
+                  group=getattr(pc, "group", 32))
     c.load_packed(pc)
     if fit is not None:
         c.set_fit(torch.from_numpy(fit.P), torch.from_numpy(fit.w), torch.from_numpy(fit.Wg))

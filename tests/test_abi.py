@@ -82,7 +82,7 @@ def _desc(**kw):
     import bit_kv_cache_centroid_b200 as kv2
     base = dict(B=1, H_kv=2, d=128, M=64, r=8, capacity=256, k_code=0x1000, v_code=0x2000, k_sz=0x3000,
                 v_sz=0x4000, cidx=0x5000, psac=0x6000, centroids=0x7000, P=0x8000, w=0x9000, Wg=0xA000,
-                psac_fmt=0, psac_scale=0, block_table=0, page_tokens=0)
+                psac_fmt=0, psac_scale=0, block_table=0, page_tokens=0, group=0)
     base.update(kw)
     return kv2.kv2_cache(**base)
 
@@ -98,8 +98,8 @@ def test_argument_checks_of_the_later_entry_points(lib):
     assert lib.kv2_fit_centroids_workspace_size(2, 96, 64) == 0
     assert lib.kv2_top1_workspace_size(2, 3, 4, 5000) == 2 * 3 * 4 * 2 * 8
     # centre fitting: candidates outside 1..M, unsupported d, a no-op call
-    args = lambda C, d, iters: (P(0x1000), 16, 2, d, 64, C, P(0x2000), P(0x3000), iters, P(0x4000), P(0x5000),
-                                P(0x6000), ctypes.c_size_t(1 << 20), None)
+    args = lambda C, d, iters: (P(0x1000), 16, 2, d, 64, C, 32, P(0x2000), P(0x3000), iters, P(0x4000),
+                                P(0x5000), P(0x6000), ctypes.c_size_t(1 << 20), None)
     assert lib.kv2_fit_centroids(*args(65, 128, 1)) == 1              # KV2_ERR_INVALID_ARG
     assert b"candidates" in lib.kv2_last_error()
     assert lib.kv2_fit_centroids(*args(4, 96, 1)) == 2                # KV2_ERR_UNSUPPORTED
@@ -113,3 +113,32 @@ def test_argument_checks_of_the_later_entry_points(lib):
     noscale = _desc(psac_fmt=1)
     assert lib.kv2_quantize_append(ctypes.byref(noscale), P(0x1000), P(0x2000), 1, 0, 1, None) == 1
     assert b"psac_scale" in lib.kv2_last_error()
+
+
+def test_group_argument_checks(lib):
+    """Groups of 32 channels (0 selects 32) pass the checks; 64 and 128 are
+    part of the format but refused by this version; other sizes, and a group
+    wider than the head, are refused with their reason."""
+    P = ctypes.c_void_p
+    lib.kv2_last_error.restype = ctypes.c_char_p
+    lib.kv2_version.restype = ctypes.c_int
+    assert lib.kv2_version() >= 200
+    for group, ok in ((0, True), (32, True), (64, False), (128, False), (48, False), (256, False)):
+        d = _desc(group=group)
+        # capacity overflow is reported only after the descriptor passed its checks
+        rc = lib.kv2_quantize_append(ctypes.byref(d), P(0x1000), P(0x2000), 10, 250, 1, None)
+        assert rc == (3 if ok else 2), (group, rc)
+        if not ok:
+            assert b"group" in lib.kv2_last_error()
+    d64 = _desc(d=64, group=128)
+    assert lib.kv2_quantize_append(ctypes.byref(d64), P(0x1000), P(0x2000), 1, 0, 1, None) == 2
+    assert b"larger than d" in lib.kv2_last_error()
+    # the statistics entry points take the group as an argument
+    fit = lambda group: lib.kv2_fit_psac_basis(P(0x1000), 16, 4, 2, 128, 8, group, P(0x2000), P(0x3000),
+                                               P(0x4000), None, P(0x5000), ctypes.c_size_t(16), None)
+    assert fit(64) == 2 and b"group" in lib.kv2_last_error()
+    assert fit(32) == 6                       # past the group check: the workspace is too small
+    cent = lambda group: lib.kv2_fit_centroids(P(0x1000), 16, 2, 128, 64, 4, group, P(0x2000), P(0x3000), 1,
+                                               P(0x4000), P(0x5000), P(0x6000), ctypes.c_size_t(16), None)
+    assert cent(96) == 2 and b"group" in lib.kv2_last_error()
+    assert cent(0) == 6
