@@ -39,9 +39,13 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) of one decode_split launch on the LLM decode
 # workload, from the ncu capture summarised in profiles/decode_split_llm_decode.md;
 # None whenever the kernel has changed since that capture.
-DECODE_SPLIT_TRAFFIC = 240_908_544
-BYTES_PER_TOKEN_HEAD = lambda d, r, M, psac_fmt=0: (2 * (d // 16) * 4 + 2 * (d // 32) * 4 + (1 if M <= 256 else 2)
-                                                    + (2 * r if psac_fmt == 0 else (r + 2 if r else 0)))
+DECODE_SPLIT_TRAFFIC = None
+# packed bytes per (token, KV head): K and V code words, K and V scale/zero
+# words (one per group of `group` channels), the centroid id, the PSAC
+# coefficients (fp16, or int8 codes with one fp16 scale)
+BYTES_PER_TOKEN_HEAD = lambda d, r, M, psac_fmt=0, group=32: (2 * (d // 16) * 4 + 2 * (d // group) * 4
+                                                              + (1 if M <= 256 else 2)
+                                                              + (2 * r if psac_fmt == 0 else (r + 2 if r else 0)))
 
 
 def peaks():
