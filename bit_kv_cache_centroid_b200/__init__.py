@@ -87,6 +87,12 @@ def _load():
     L.kv2_attention_chunk.restype = I
     L.kv2_attention_chunk.argtypes = [ctypes.POINTER(kv2_cache), I, P, I, I, P, P, I,
                                       ctypes.c_float, P, I, P, S, P]
+    L.kv2_page_bytes.restype = S
+    L.kv2_page_bytes.argtypes = [ctypes.POINTER(kv2_cache)]
+    L.kv2_page_store.restype = I
+    L.kv2_page_store.argtypes = [ctypes.POINTER(kv2_cache), I, I, P, P]
+    L.kv2_page_load.restype = I
+    L.kv2_page_load.argtypes = [ctypes.POINTER(kv2_cache), I, I, P, P]
     return L
 
 
@@ -113,7 +119,8 @@ EXPORTS = ["kv2_status_string", "kv2_last_error", "kv2_version", "kv2_fit_worksp
            "kv2_top1_workspace_size", "kv2_decode_top1", "kv2_dense_top1",
            "kv2_quantize_append", "kv2_decode_workspace_size",
            "kv2_attention_decode", "kv2_attention_decode_noalloc", "kv2_append_attention_decode",
-           "kv2_chunk_workspace_size", "kv2_attention_chunk"]
+           "kv2_chunk_workspace_size", "kv2_attention_chunk",
+           "kv2_page_bytes", "kv2_page_store", "kv2_page_load"]
 
 
 def _check(status: int):
@@ -148,9 +155,11 @@ class Cache:
         self.group = group
         self.psac_fmt = psac_fmt
         self.page_tokens = page_tokens
+        self.num_pages = 0
         if page_tokens:
             pps = capacity // page_tokens
             num_pages = num_pages or B * pps
+            self.num_pages = num_pages
             sh = (num_pages, H_kv, page_tokens)
             self.block_table = torch.arange(B * pps, dtype=torch.int32, device=device).remainder(num_pages) \
                 .view(B, pps).contiguous()
@@ -374,3 +383,35 @@ def kv2_attention_chunk(cache: Cache, length: int, Q: torch.Tensor, Kself: torch
                                    frame_tokens, float(sm_scale), _ptr(out), out_dtype, _ptr(ws),
                                    ws.numel(), _stream(stream)))
     return out
+
+
+# ----------------------------------------------------------------------------
+# pages of a paged cache out of HBM and back
+# ----------------------------------------------------------------------------
+
+def kv2_page_bytes(cache: Cache) -> int:
+    """Bytes of one page's host image (0 if the cache is not paged)."""
+    d = cache.desc()
+    return int(_get_lib().kv2_page_bytes(ctypes.byref(d)))
+
+
+def kv2_page_store(cache: Cache, page: int, host=None, stream=None):
+    """Copy page ``page`` of every stream into ``host`` (a CPU uint8 tensor of
+    kv2_page_bytes bytes; page-locked when allocated here) and return it. The
+    copies are asynchronous on the stream: synchronize before reading it."""
+    if host is None:
+        host = torch.empty(kv2_page_bytes(cache), dtype=torch.uint8, pin_memory=True)
+    d = cache.desc()
+    _check(_get_lib().kv2_page_store(ctypes.byref(d), page, cache.num_pages, ctypes.c_void_p(host.data_ptr()),
+                                     _stream(stream)))
+    return host
+
+
+def kv2_page_load(cache: Cache, page: int, host, stream=None):
+    """Copy a page image (from kv2_page_store) into page ``page``; the caller
+    points block-table entries at it."""
+    if host.numel() * host.element_size() < kv2_page_bytes(cache):
+        raise ValueError("host buffer smaller than kv2_page_bytes")
+    d = cache.desc()
+    _check(_get_lib().kv2_page_load(ctypes.byref(d), page, cache.num_pages, ctypes.c_void_p(host.data_ptr()),
+                                    _stream(stream)))

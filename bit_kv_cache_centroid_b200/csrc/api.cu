@@ -312,4 +312,81 @@ kv2_status kv2_attention_chunk(const kv2_cache* c, int len, const uint16_t* Q, i
   return cuda_status(e, "chunk launch");
 }
 
+namespace {
+
+// one stream of a paged cache: device base and bytes per token slot
+struct PageStream {
+  char* base;
+  size_t per_token;
+};
+
+// the streams of a cache in the order of a page's host image; returns how many
+int page_streams(const kv2_cache* c, PageStream (&s)[7]) {
+  const size_t words = size_t(c->d / 16) * 4, groups = size_t(c->d / kv2::cache_group(*c)) * 4;
+  int n = 0;
+  s[n++] = {reinterpret_cast<char*>(c->k_code), words};
+  s[n++] = {reinterpret_cast<char*>(c->v_code), words};
+  s[n++] = {reinterpret_cast<char*>(c->k_sz), groups};
+  s[n++] = {reinterpret_cast<char*>(c->v_sz), groups};
+  s[n++] = {static_cast<char*>(c->cidx), size_t(c->M <= 256 ? 1 : 2)};
+  if (c->r) s[n++] = {reinterpret_cast<char*>(c->psac), size_t(c->psac_fmt == 1 ? c->r : 2 * c->r)};
+  if (c->r && c->psac_fmt == 1) s[n++] = {reinterpret_cast<char*>(c->psac_scale), 2};
+  return n;
+}
+
+size_t page_image_bytes(const kv2_cache* c) {
+  PageStream s[7];
+  const int n = page_streams(c, s);
+  size_t per_token = 0;
+  for (int i = 0; i < n; ++i) per_token += s[i].per_token;
+  return size_t(c->H_kv) * size_t(c->page_tokens) * per_token;
+}
+
+kv2_status check_page(const kv2_cache* c, int page, int num_pages, const void* host) {
+  kv2_status st = check_cache(c, true, false);
+  if (st != KV2_OK) return st;
+  if (!c->block_table) return fail(KV2_ERR_INVALID_ARG, "page: the cache is not paged (block_table is NULL)");
+  if (num_pages <= 0 || page < 0 || page >= num_pages)
+    return fail(KV2_ERR_INVALID_ARG, "page: page %d outside 0..num_pages-1 (num_pages=%d)", page, num_pages);
+  if (!host) return fail(KV2_ERR_INVALID_ARG, "page: host buffer is NULL");
+  return KV2_OK;
+}
+
+// page `page` of every stream (slots page*H_kv*page_tokens .. +H_kv*page_tokens,
+// contiguous in each stream) to or from the host image
+kv2_status page_copy(const kv2_cache* c, int page, char* host, bool store, cudaStream_t stream) {
+  PageStream s[7];
+  const int n = page_streams(c, s);
+  const size_t slots = size_t(c->H_kv) * size_t(c->page_tokens);
+  for (int i = 0; i < n; ++i) {
+    const size_t bytes = slots * s[i].per_token;
+    char* dev = s[i].base + size_t(page) * bytes;
+    const cudaError_t e = store ? cudaMemcpyAsync(host, dev, bytes, cudaMemcpyDeviceToHost, stream)
+                                : cudaMemcpyAsync(dev, host, bytes, cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return cuda_status(e, store ? "page_store copy" : "page_load copy");
+    host += bytes;
+  }
+  return ok();
+}
+
+}  // namespace
+
+size_t kv2_page_bytes(const kv2_cache* c) {
+  if (!c || !c->block_table || check_cache(c, false, false) != KV2_OK) return 0;
+  return page_image_bytes(c);
+}
+
+kv2_status kv2_page_store(const kv2_cache* c, int page, int num_pages, void* host, void* stream) {
+  const kv2_status st = check_page(c, page, num_pages, host);
+  if (st != KV2_OK) return st;
+  return page_copy(c, page, static_cast<char*>(host), true, static_cast<cudaStream_t>(stream));
+}
+
+kv2_status kv2_page_load(const kv2_cache* c, int page, int num_pages, const void* host, void* stream) {
+  const kv2_status st = check_page(c, page, num_pages, host);
+  if (st != KV2_OK) return st;
+  return page_copy(c, page, const_cast<char*>(static_cast<const char*>(host)), false,
+                   static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

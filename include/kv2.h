@@ -317,9 +317,11 @@ size_t kv2_chunk_workspace_size(const kv2_cache* cache, int H_q, int Nq);
  * chunk's own dense keys/values, block-causal by latent frame: query i sees
  * every cached token and the self tokens j with j/frame_tokens <= i/frame_tokens.
  * Tensor cores (tcgen05, accumulators in TMEM): packed key tiles are
- * dequantized to bf16 centroid + residual in shared memory, the PSAC term
- * (qP).a enters as fp16 extra contraction columns, value tiles and
- * probabilities are fp16, accumulation fp32.
+ * dequantized in shared memory to fp16(code*s + fp16(z + centroid)), value
+ * tiles to fp16(code*s + z), the chunk's own keys and values are rounded
+ * from bf16 to fp16, each query row is scaled by a power of two and
+ * converted to fp16, the PSAC term (qP).a enters as fp16 extra contraction
+ * columns, probabilities are fp16, accumulation fp32.
  * Q     : bf16 [B][Nq][H_q][d]; Kself, Vself: bf16 [B][Nq][H_kv][d];
  * out   : [B][Nq][H_q][d] fp32 or bf16. Requires d = 128.
  * ws    : device workspace of kv2_chunk_workspace_size(cache, H_q, Nq) bytes.
@@ -328,6 +330,36 @@ kv2_status kv2_attention_chunk(const kv2_cache* cache, int len, const uint16_t* 
                                int Nq, const uint16_t* Kself, const uint16_t* Vself,
                                int frame_tokens, float sm_scale, void* out, int out_dtype,
                                void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Pages of a paged cache moved out of HBM and back (long-horizon memory:
+ * a sequence's older chunks kept in host memory and brought back when the
+ * caller wants them in the attention window again; which pages to move is
+ * the caller's policy).
+ *
+ * A page holds page_tokens consecutive tokens of every KV head in each
+ * stream: k_code, v_code, k_sz, v_sz, cidx, then psac (r > 0) and
+ * psac_scale (int8 PSAC format, r > 0). Its image in host memory is those
+ * streams' page slices back to back in that order, kv2_page_bytes(cache)
+ * bytes: H_kv * page_tokens * (8*(d/16) + 8*(d/group) + id bytes + PSAC
+ * bytes per token).
+ *
+ * kv2_page_store copies page `page` (0 <= page < num_pages, the pool's page
+ * count) of the cache's device streams into `host`; kv2_page_load copies an
+ * image from `host` into page `page`. To evict, store a page and drop it
+ * from the block table; to retrieve, load the image into a free page and
+ * point the table entry at it (the block table is the caller's device
+ * memory). Both are cudaMemcpyAsync calls on `stream`, one per stream: with
+ * page-locked host memory they are asynchronous, with pageable memory a
+ * store returns after its copies. The page's device bytes are not otherwise
+ * read or written.
+ * Errors: KV2_ERR_INVALID_ARG (cache not paged, page outside 0..num_pages-1,
+ * NULL host buffer), the cache checks of kv2_quantize_append, KV2_ERR_CUDA.
+ * kv2_page_bytes returns 0 for a descriptor that is not a valid paged cache.
+ */
+size_t kv2_page_bytes(const kv2_cache* cache);
+kv2_status kv2_page_store(const kv2_cache* cache, int page, int num_pages, void* host, void* stream);
+kv2_status kv2_page_load(const kv2_cache* cache, int page, int num_pages, const void* host, void* stream);
 
 #ifdef __cplusplus
 }

@@ -142,3 +142,25 @@ def test_group_argument_checks(lib):
                                                P(0x4000), P(0x5000), P(0x6000), ctypes.c_size_t(16), None)
     assert cent(96) == 2 and b"group" in lib.kv2_last_error()
     assert cent(0) == 6
+
+
+def test_page_image_size_and_argument_checks(lib):
+    """A page's host image is H_kv * page_tokens slots of every stream back to
+    back; the store/load checks return before any copy is issued."""
+    P = ctypes.c_void_p
+    lib.kv2_last_error.restype = ctypes.c_char_p
+    lib.kv2_page_bytes.restype = ctypes.c_size_t
+    paged = dict(block_table=0xB000, page_tokens=128)
+    # per token slot: 2 x 8 code words, 2 x 4 scale/zero words, a u8 id, 8 fp16 coefficients
+    assert lib.kv2_page_bytes(ctypes.byref(_desc(**paged))) == 2 * 128 * (32 + 32 + 16 + 16 + 1 + 16)
+    # int8 coefficients with a per-token fp16 scale; u16 ids; no PSAC
+    assert lib.kv2_page_bytes(ctypes.byref(_desc(psac_fmt=1, psac_scale=0xC000, **paged))) == \
+        2 * 128 * (32 + 32 + 16 + 16 + 1 + 8 + 2)
+    assert lib.kv2_page_bytes(ctypes.byref(_desc(M=512, r=0, **paged))) == 2 * 128 * (32 + 32 + 16 + 16 + 2)
+    assert lib.kv2_page_bytes(ctypes.byref(_desc())) == 0                      # not paged
+    store = lambda d, page, n, host: lib.kv2_page_store(ctypes.byref(d), page, n, host, None)
+    assert store(_desc(), 0, 4, P(0x1000)) == 1 and b"not paged" in lib.kv2_last_error()
+    assert store(_desc(**paged), 4, 4, P(0x1000)) == 1 and b"outside" in lib.kv2_last_error()
+    assert store(_desc(**paged), -1, 4, P(0x1000)) == 1
+    assert store(_desc(**paged), 0, 4, None) == 1 and b"NULL" in lib.kv2_last_error()
+    assert lib.kv2_page_load(ctypes.byref(_desc(**paged)), 0, 0, P(0x1000), None) == 1

@@ -99,3 +99,46 @@ def test_append_through_the_block_table(orc):
                     assert np.array_equal(got, hf[name][b, :, lo:hi]), name
     Q = to_dev(w.Qdec, torch.int16)
     assert torch.equal(kv2.kv2_attention_decode(gc, 537, Q, 0.1), kv2.kv2_attention_decode(gp, 537, Q, 0.1))
+
+
+@pytest.mark.parametrize("fmt,M", [(0, 64), (1, 512)])
+def test_evict_and_retrieve_a_page(orc, fmt, M):
+    """Long-horizon memory: a page stored to host memory is the page's slice of
+    every stream back to back; after the page is cleared on the device (its
+    slot reused) the decode changes, and after the image is loaded into a spare
+    page of the pool and the block-table entry points there, decode and top-1
+    are bit-identical to before; the retrieved cache still matches the oracle."""
+    import bit_kv_cache_centroid_b200 as kv2
+    s = wl.spec("tiny", d=128, H_kv=2, H_q=8, M=M, r=8, T=1024, B=2)
+    pc = wl.random_packed_cache(s, T=1024, seed=21 + fmt, psac_fmt=fmt)
+    n_pages = pc.B * pc.capacity // 128 + 4
+    pg = wl.to_paged(pc, 128, n_pages, seed=2)
+    gp = gpu_cache_like(pg)
+    P = _basis(2, 128, 8, 5)
+    gp.P.copy_(torch.from_numpy(P))
+    rng = np.random.default_rng(3)
+    Q = to_dev(wl.bf16_bits(rng.standard_normal((2, 8, 128)).astype(np.float32)), torch.int16)
+    before = kv2.kv2_attention_decode(gp, 1000, Q, 0.09)
+    top_before = kv2.kv2_decode_top1(gp, 1000, Q)
+    src = int(pg.table[1, 2])                       # tokens 256..383 of sequence 1
+    spare = sorted(set(range(n_pages)) - set(pg.table.ravel().tolist()))[0]
+    img = kv2.kv2_page_store(gp, src)
+    torch.cuda.synchronize()
+    names = ["k_code", "v_code", "k_sz", "v_sz", "cidx", "psac"] + (["psac_scale"] if fmt == 1 else [])
+    want = np.concatenate([np.ascontiguousarray(getattr(pg, n)[src]).reshape(-1).view(np.uint8) for n in names])
+    assert img.numel() == kv2.kv2_page_bytes(gp) == want.size
+    assert np.array_equal(img.numpy(), want)
+    for n in names:
+        getattr(gp, n)[src].zero_()
+    assert not torch.equal(kv2.kv2_attention_decode(gp, 1000, Q, 0.09), before)
+    kv2.kv2_page_load(gp, spare, img)
+    gp.block_table[1, 2] = spare
+    after = kv2.kv2_attention_decode(gp, 1000, Q, 0.09)
+    assert torch.equal(after, before)
+    assert torch.equal(kv2.kv2_decode_top1(gp, 1000, Q), top_before)
+    moved = wl.to_paged(pc, 128, n_pages, seed=2)
+    moved.table[1, 2] = spare
+    for n in names:
+        getattr(moved, n)[spare] = getattr(pg, n)[src]
+    ref = orc.decode(moved, P, 1000, Q.cpu().numpy().view(np.uint16), 0.09)
+    assert_attention_close(after.cpu().numpy(), ref, what=f"retrieved page fmt{fmt}")
