@@ -164,3 +164,20 @@ def test_page_image_size_and_argument_checks(lib):
     assert store(_desc(**paged), -1, 4, P(0x1000)) == 1
     assert store(_desc(**paged), 0, 4, None) == 1 and b"NULL" in lib.kv2_last_error()
     assert lib.kv2_page_load(ctypes.byref(_desc(**paged)), 0, 0, P(0x1000), None) == 1
+
+
+def test_plain_c_client(lib, tmp_path):
+    """The header compiles as pedantic C11 and a C program linked against
+    libkv2.so gets the documented results from the host-side checks."""
+    import shutil
+    import subprocess
+    if not shutil.which("gcc"):
+        pytest.skip("gcc not available")
+    libdir = os.path.join(ROOT, "bit_kv_cache_centroid_b200")
+    exe = str(tmp_path / "c_client")
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "host", "c_client.c"), "-o", exe, "-L", libdir, "-l:libkv2.so",
+                    f"-Wl,-rpath,{libdir}"], check=True, capture_output=True)
+    r = subprocess.run([exe], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    assert "c client ok" in r.stdout
