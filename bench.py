@@ -272,20 +272,29 @@ def run_gpu(args, rank, world):
         "clocks": clk.summary(),
     }
     if not args.skip_extras and rank == 0:
-        result["int8_psac_decode"] = int8_psac_decode(torch, kv2, args, pk, w, s, Q, scale, out)
+        result["int8_psac_decode"] = variant_decode(torch, kv2, args, pk, w, s, Q, scale, out, psac_fmt=1)
+        result["group128_decode"] = variant_decode(torch, kv2, args, pk, w, s, Q, scale, out, group=128)
+        result["group128_int8_psac_decode"] = variant_decode(torch, kv2, args, pk, w, s, Q, scale, out,
+                                                             psac_fmt=1, group=128)
         result.update(extras(torch, kv2, args, pk))
     if rank == 0 and not args.no_cpu:
         result["cpu_baseline"] = cpu_baseline(args, budget_s=args.cpu_seconds)
     return result
 
 
-def int8_psac_decode(torch, kv2, args, pk, w, s, Q, scale, out):
-    """The LLM decode workload with the PSAC coefficients stored as int8
-    codes and one fp16 scale per token (decode alone, same timing as above)."""
+def variant_decode(torch, kv2, args, pk, w, s, Q, scale, out, psac_fmt=0, group=32):
+    """The LLM decode workload in another cache format: PSAC coefficients as
+    int8 codes with one fp16 scale per token (psac_fmt 1) and/or one scale and
+    zero per `group` channels (decode alone, same timing as above). A format
+    the library refuses is reported as skipped, with the library's reason."""
     dev = torch.device("cuda")
-    P, wt, Wg, en = kv2.kv2_fit_psac_basis(torch.from_numpy(w.Qhist.view(np.int16)).to(dev), s.H_kv, s.r)
+    try:
+        P, wt, Wg, en = kv2.kv2_fit_psac_basis(torch.from_numpy(w.Qhist.view(np.int16)).to(dev), s.H_kv, s.r,
+                                               group=group)
+    except kv2.Kv2Error as e:
+        return {"skipped": str(e)}
     cache = kv2.Cache(s.B, s.H_kv, s.d, s.M, s.r, s.capacity, torch.from_numpy(w.centroids.view(np.int16)),
-                      psac_fmt=1)
+                      psac_fmt=psac_fmt, group=group)
     cache.set_fit(P, wt, Wg)
     K = torch.from_numpy(np.ascontiguousarray(w.K[:, :s.T + 1]).view(np.int16)).to(dev)
     V = torch.from_numpy(np.ascontiguousarray(w.V[:, :s.T + 1]).view(np.int16)).to(dev)
@@ -304,11 +313,12 @@ def int8_psac_decode(torch, kv2, args, pk, w, s, Q, scale, out):
     b.record()
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / args.steps
-    per = BYTES_PER_TOKEN_HEAD(s.d, s.r, s.M, 1)
+    per = BYTES_PER_TOKEN_HEAD(s.d, s.r, s.M, psac_fmt, group)
     gbs = length * s.B * s.H_kv * per / (ms * 1e-3) / 1e9
-    return {"workload": "llm_decode with int8 PSAC coefficients + fp16 scale per token",
-            "bytes_per_token_head": per, "ms": round(ms, 5), "GBps": round(gbs, 1),
-            "hbm_frac": round(gbs / pk["hbm_gbs"], 4)}
+    fmt = "int8 PSAC coefficients + fp16 scale per token" if psac_fmt == 1 else "fp16 PSAC coefficients"
+    return {"workload": f"llm_decode with {fmt}, scale/zero per {group} channels",
+            "bytes_per_token_head": per, "compression_vs_bf16": round(2 * 2 * s.d / per, 3),
+            "ms": round(ms, 5), "GBps": round(gbs, 1), "hbm_frac": round(gbs / pk["hbm_gbs"], 4)}
 
 
 def retrieval_shift(torch, kv2, w, s, wt, Wg, P):
