@@ -217,10 +217,13 @@ kv2_status kv2_dense_top1(const uint16_t* K, int B, int len, int H_kv, int d, co
  *   whose residual gives the least E_j = sum_g W_g s_g^2 (s_g the group's fp16
  *   scale) is chosen, ties to the better-ranked. C = 1 with w = 1 is the plain
  *   nearest-centre (QVG) assignment.
- * Codec per group of 32 (residual k - mu for keys, v for values): zero =
+ * Codec per group of `group` channels (residual k - mu for keys, v for values): zero =
  *   fp16 round-down of the minimum, scale = fp16 round-up of (max - zero)/3,
  *   code = clamp(round-half-even((x - zero)/scale), 0, 3) (0 when scale = 0).
- * PSAC: a_i = sum_c P_ci (x_c - fmaf(code_c, s, z)), rounded to fp16.
+ * PSAC: a_i = sum_c P_ci (x_c - fmaf(code_c, s, z)), rounded to fp16
+ *   (psac_fmt 0), or (psac_fmt 1) stored as int8 codes with one fp16 scale per
+ *   token: scale = fp16 round-up of max_i |a_i| / 127, code_i =
+ *   clamp(round-half-even(a_i / scale), -127, 127) (0 when the scale is 0).
  * All quantizer decisions are taken in fp32 in the order stated in the oracle
  * and are reproducible bit for bit. Tokens outside [pos, pos+n_new) are never
  * read or written; concurrent calls on overlapping slots race.
