@@ -48,6 +48,17 @@ BYTES_PER_TOKEN_HEAD = lambda d, r, M, psac_fmt=0, group=32: (2 * (d // 16) * 4 
                                                               + (2 * r if psac_fmt == 0 else (r + 2 if r else 0)))
 
 
+def compression(d, r, M, T, psac_fmt=0, group=32):
+    """KV-cache compression against bf16 K+V (4 d bytes per token-head): per
+    token, and with the per-head tables (fp16 centres M x d, the fp32 basis
+    d x r, w and W) counted over T cached tokens, as the method's compression
+    figure accounts for centres, quantization parameters and compensation."""
+    per = BYTES_PER_TOKEN_HEAD(d, r, M, psac_fmt, group)
+    tables = M * d * 2 + d * r * 4 + d * 4 + (d // group) * 4
+    return {"bytes_per_token_head": per, "ratio": round(4 * d / per, 3),
+            "ratio_with_tables": round(4 * d / (per + tables / T), 3)}
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -266,6 +277,7 @@ def run_gpu(args, rank, world):
                      "peak_source": src, "decode_ms": round(dec_ms, 5)},
         "e2e": {"value": round(bytes_step / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
+        "compression": compression(s.d, s.r, s.M, s.T + 1),
         "step_ms": {"append_alone": round(app_ms, 5), "decode_alone": round(dec_ms, 5),
                     "step_overlapped": round(ms_step, 5)},
         "gpu_launches": 3 * args.steps,
@@ -317,7 +329,7 @@ def variant_decode(torch, kv2, args, pk, w, s, Q, scale, out, psac_fmt=0, group=
     gbs = length * s.B * s.H_kv * per / (ms * 1e-3) / 1e9
     fmt = "int8 PSAC coefficients + fp16 scale per token" if psac_fmt == 1 else "fp16 PSAC coefficients"
     return {"workload": f"llm_decode with {fmt}, scale/zero per {group} channels",
-            "bytes_per_token_head": per, "compression_vs_bf16": round(2 * 2 * s.d / per, 3),
+            "bytes_per_token_head": per, "compression": compression(s.d, s.r, s.M, length, psac_fmt, group),
             "ms": round(ms, 5), "GBps": round(gbs, 1), "hbm_frac": round(gbs / pk["hbm_gbs"], 4)}
 
 

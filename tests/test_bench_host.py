@@ -52,3 +52,20 @@ def test_reference_arm_under_torchrun_prints_once():
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["unit"] == "GB/s"
     assert d["config"]["parallelism"] == "replicas x2" and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_compression_closed_forms():
+    """113 B per token-head on the LLM workload (4.53x against 512 B of bf16
+    K+V); its per-head tables (64 fp16 centres, an 8-column fp32 basis, w, W)
+    add 21,008 B over 32,769 tokens (4.505x); 128-channel groups with int8
+    coefficients: 83 B (6.17x)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    c = bench.compression(128, 8, 64, 32769)
+    assert c["bytes_per_token_head"] == 113 and c["ratio"] == 4.531
+    tables = 64 * 128 * 2 + 128 * 8 * 4 + 128 * 4 + 4 * 4
+    assert tables == 21008
+    assert c["ratio_with_tables"] == round(512 / (113 + tables / 32769), 3) == 4.505
+    g = bench.compression(128, 8, 256, 37440, psac_fmt=1, group=128)
+    assert g["bytes_per_token_head"] == 83 and g["ratio"] == 6.169
+    assert bench.compression(128, 16, 512, 187200)["bytes_per_token_head"] == 130
