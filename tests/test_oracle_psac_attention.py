@@ -203,3 +203,43 @@ def test_chunk_cache_part_equals_decode_when_exact(orc):
     for n, (_, i, hq) in enumerate(rows):
         dec = orc.decode(pc, P, 48, Q[:, i], 0.125)[0, hq]
         np.testing.assert_allclose(out[n], dec, rtol=1e-12, atol=1e-12)
+
+
+def test_chunk_operand_rounding_hand_derived(orc):
+    """Two cached tokens whose chunk operands round (fp16 arithmetic, one
+    rounding per operation; derived by hand):
+      K_hat = fp16(code s + fp16(z + mu)): z = 1024, mu = 0.25, s = 0.5.
+        token 0, code 1: fp16(0.5 + fp16(1024.25) = 1024) = fp16(1024.5) =
+        1024 (a tie, to even; the exact key is 1024.75);
+        token 1, code 0: fp16(0 + 1024) = 1024 (exact 1024.25).
+      So the chunk's two logits are equal and token 0 takes weight 1/2 exactly,
+      where decode (exact keys) sees a gap of 0.5 * sm_scale.
+      V_hat = fp16(code s + z) in channel 32 (group 1): token 0 code 1, s = 1,
+        z = 2048: fp16(2049) = 2048 (a tie, to even); token 1: 0.
+      Channel 0 of V: token 0 has zero 1, token 1 zero 0.
+    A self key of -4000 on channel 0 takes no weight (logit -500)."""
+    d = 64
+    f16 = lambda x: int(np.float16(x).view(np.uint16))
+    cent = np.zeros((1, 1, d), np.uint16)
+    cent[0, 0, 0] = f16(0.25)
+    pc = wl.PackedCache.empty(1, 1, d, 1, 0, 16, cent)
+    pc.k_code[0, 0, 0, 0] = 1                          # token 0, channel 0: code 1
+    pc.k_sz[0, 0, :2, 0] = f16(0.5) | (f16(1024.0) << 16)
+    pc.v_code[0, 0, 0, 2] = 1                          # token 0, channel 32: code 1
+    pc.v_sz[0, 0, 0, 0] = f16(0.0) | (f16(1.0) << 16)
+    pc.v_sz[0, 0, 0, 1] = f16(1.0) | (f16(2048.0) << 16)
+    q = np.zeros((1, 1, 1, d), np.float32)
+    q[..., 0] = 1.0
+    Q = wl.bf16_bits(q)
+    Ks = np.zeros((1, 1, 1, d), np.float32)
+    Ks[..., 0] = -4000.0
+    Vs = np.zeros((1, 1, 1, d), np.float32)
+    P = np.zeros((1, d, 0), np.float32)
+    scale = 0.125
+    out = orc.chunk(pc, P, 2, Q, wl.bf16_bits(Ks), wl.bf16_bits(Vs), 1, scale, np.array([(0, 0, 0)], np.int32))[0]
+    assert out[0] == 0.5
+    assert out[32] == 1024.0
+    dec = orc.decode(pc, P, 2, Q[:, 0], scale)[0, 0]
+    p0 = 1.0 / (1.0 + np.exp(-0.5 * scale))          # exact keys 1024.75 and 1024.25
+    np.testing.assert_allclose(dec[0], p0, rtol=1e-14)
+    np.testing.assert_allclose(dec[32], p0 * 2049.0, rtol=1e-14)
