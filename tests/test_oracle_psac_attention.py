@@ -243,3 +243,31 @@ def test_chunk_operand_rounding_hand_derived(orc):
     p0 = 1.0 / (1.0 + np.exp(-0.5 * scale))          # exact keys 1024.75 and 1024.25
     np.testing.assert_allclose(dec[0], p0, rtol=1e-14)
     np.testing.assert_allclose(dec[32], p0 * 2049.0, rtol=1e-14)
+
+
+def test_chunk_psac_query_rounding_hand_derived(orc):
+    """The chunk's PSAC operand u = fp16(q P): with q = e_0 and P[0][0] =
+    fp32(1/3) = 0.3333333432674408, u = 0.333251953125 (fp16 of 1/3, rounded
+    down). Two cached tokens identical but for their coefficient (1 and 0):
+    the chunk weights token 0 by sigmoid(u * scale), decode by
+    sigmoid(fp32(1/3) * scale); the values are 1 and 0 in channel 0."""
+    d = 64
+    f16 = lambda x: int(np.float16(x).view(np.uint16))
+    pc = wl.PackedCache.empty(1, 1, d, 1, 8, 16, np.zeros((1, 1, d), np.uint16))
+    pc.psac[0, 0, 0, 0] = f16(1.0)
+    pc.v_sz[0, 0, 0, 0] = f16(1.0) << 16                 # token 0: values 1 in channels 0..31
+    P = np.zeros((1, d, 8), np.float32)
+    P[0, 0, 0] = np.float32(1.0 / 3.0)
+    q = np.zeros((1, 1, 1, d), np.float32)
+    q[..., 0] = 1.0
+    Q = wl.bf16_bits(q)
+    Ks = np.zeros((1, 1, 1, d), np.float32)
+    Ks[..., 0] = -4000.0
+    scale = 2.0
+    out = orc.chunk(pc, P, 2, Q, wl.bf16_bits(Ks), wl.bf16_bits(np.zeros((1, 1, 1, d), np.float32)), 1, scale,
+                    np.array([(0, 0, 0)], np.int32))[0]
+    u16 = 0.333251953125
+    assert float(np.float16(1.0 / 3.0)) == u16
+    np.testing.assert_allclose(out[0], 1.0 / (1.0 + np.exp(-u16 * scale)), rtol=1e-14)
+    dec = orc.decode(pc, P, 2, Q[:, 0], scale)[0, 0]
+    np.testing.assert_allclose(dec[0], 1.0 / (1.0 + np.exp(-float(np.float32(1.0 / 3.0)) * scale)), rtol=1e-14)
