@@ -106,3 +106,27 @@ def test_unchosen_centre_keeps_its_value_and_noop_cases(orc):
     assert np.array_equal(same, init)
     empty, a0 = orc.fit_centroids(Xb[:0], M, 2, w, Wg, init, iters=2)
     assert np.array_equal(empty, init) and a0.shape == (0, H)
+
+
+def test_fixed_point_mean_truncates_below_one_unit(orc):
+    """The update's mean counts each key value in whole 2^-24 units,
+    truncated toward zero: a lone key of +-0.75 * 2^-24 (bf16-exact) leaves
+    its channel of the centre at 0, where the exact mean would round to
+    +-2^-24; values of whole units average exactly (2^-20 and 2^-23 -> 9
+    units)."""
+    d = 64
+    X = np.zeros((2, 1, d), np.float32)
+    X[0, 0, 0] = 0.75 * 2.0 ** -24
+    X[0, 0, 1] = -0.75 * 2.0 ** -24
+    X[0, 0, 2] = 2.0 ** -20
+    X[1, 0, 2] = 2.0 ** -23
+    Xb = wl.bf16_bits(X)
+    assert np.array_equal(wl.bf16_values(Xb), X)
+    w = np.ones((1, d), np.float32)
+    Wg = np.full((1, d // 32), 32.0, np.float32)
+    cent0 = wl.f16_bits(np.full((1, 1, d), 0.5, np.float32))
+    cent, assign = orc.fit_centroids(Xb, 1, 1, w, Wg, cent0, 1)
+    got = wl.f16_values(cent)[0, 0].astype(np.float64)
+    assert got[0] == 0.0 and got[1] == 0.0
+    assert got[2] == 9 * 2.0 ** -24                    # (16 + 2) / 2 units
+    assert np.all(got[3:] == 0.0) and np.all(assign == 0)
