@@ -26,7 +26,10 @@
  * form; group sizes 64 and 128 by per-group codec invariants, exact
  * reconstruction of group-constant residuals, the single-group QSAC choice as
  * the least residual range, and W over one whole-row group as the trace of
- * the Gram matrix. Parity unpinned: whether the perturbation estimate is the authors' exact
+ * the Gram matrix; 4-element groups exhaustively over a value grid (nearest
+ * level, exact ties to even) and QSAC by brute force; the chunk operands'
+ * fp16 rounding (keys, values, q P) on hand-derived ties; the centre update's
+ * truncation below one 2^-24 unit. Parity unpinned: whether the perturbation estimate is the authors' exact
  * heuristic (the pages print no worked example).
  */
 #include <math.h>
