@@ -223,3 +223,35 @@ def test_fit_centroids_bit_exact(orc, group, M, C, n):
     ref_c, ref_a = orc.fit_centroids(X, M, C, f.w, f.Wg, w.centroids, 2, group=group)
     assert np.array_equal(got_a.cpu().numpy(), ref_a)
     assert np.array_equal(got_c.cpu().numpy().view(np.uint16), ref_c)
+
+
+def test_paged_group128_int8_identical_to_contiguous(orc):
+    """Groups of 128 channels with int8 coefficients in a paged cache (pages
+    shuffled among spare pages): decode bit-identical to the contiguous cache
+    and within tolerance of the oracle; a page round trip through host memory
+    leaves it unchanged."""
+    _need(128)
+    import bit_kv_cache_centroid_b200 as kv2
+    s = wl.spec("tiny", d=128, H_kv=2, H_q=8, M=64, r=8, T=1024, B=2, group=128)
+    pc = wl.random_packed_cache(s, T=1024, seed=31, psac_fmt=1)
+    n_pages = pc.B * pc.capacity // 128 + 3
+    pg = wl.to_paged(pc, 128, n_pages, seed=4)
+    P = _basis(2, 128, 8, 7)
+    gc, gp = gpu_cache_like(pc), gpu_cache_like(pg)
+    for c in (gc, gp):
+        c.P.copy_(torch.from_numpy(P))
+    rng = np.random.default_rng(8)
+    Q = to_dev(wl.bf16_bits(rng.standard_normal((2, 8, 128)).astype(np.float32)), torch.int16)
+    a = kv2.kv2_attention_decode(gc, 1000, Q, 0.09)
+    b = kv2.kv2_attention_decode(gp, 1000, Q, 0.09)
+    assert torch.equal(a, b)
+    assert kv2.kv2_page_bytes(gp) == 2 * 128 * (32 + 32 + 4 + 4 + 1 + 8 + 2)
+    src = int(pg.table[0, 5])
+    img = kv2.kv2_page_store(gp, src)
+    torch.cuda.synchronize()
+    for n in ("k_code", "v_code", "k_sz", "v_sz", "cidx", "psac", "psac_scale"):
+        getattr(gp, n)[src].zero_()
+    kv2.kv2_page_load(gp, src, img)
+    assert torch.equal(kv2.kv2_attention_decode(gp, 1000, Q, 0.09), a)
+    ref = orc.decode(pg, P, 1000, Q.cpu().numpy().view(np.uint16), 0.09)
+    assert_attention_close(b.cpu().numpy(), ref, what="paged group 128 int8")
