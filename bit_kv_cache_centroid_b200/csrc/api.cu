@@ -32,14 +32,11 @@ kv2_status cuda_status(cudaError_t e, const char* what) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Shape and pointer checks common to every call that reads the cache.
-// Channels per (scale, zero) group (0 selects 32). The kernels are
-// instantiated for 32, 64 and 128 channels; this version of the boundary
-// takes 32 only.
+// Channels per (scale, zero) group (0 selects 32): 32, 64 or 128, at most d.
 kv2_status check_group(int d, int group) {
   const int g = group ? group : kv2::kGroup;
   if (g != 32 && g != 64 && g != 128) return fail(KV2_ERR_UNSUPPORTED, "group=%d (32, 64 or 128)", group);
   if (g > d) return fail(KV2_ERR_UNSUPPORTED, "group=%d larger than d=%d", g, d);
-  if (g != kv2::kGroup) return fail(KV2_ERR_UNSUPPORTED, "group=%d: this library version takes groups of 32", g);
   return KV2_OK;
 }
 

@@ -116,14 +116,13 @@ def test_argument_checks_of_the_later_entry_points(lib):
 
 
 def test_group_argument_checks(lib):
-    """Groups of 32 channels (0 selects 32) pass the checks; 64 and 128 are
-    part of the format but refused by this version; other sizes, and a group
-    wider than the head, are refused with their reason."""
+    """Groups of 32, 64 and 128 channels (0 selects 32) pass the checks; other
+    sizes, and a group wider than the head, are refused with their reason."""
     P = ctypes.c_void_p
     lib.kv2_last_error.restype = ctypes.c_char_p
     lib.kv2_version.restype = ctypes.c_int
     assert lib.kv2_version() >= 200
-    for group, ok in ((0, True), (32, True), (64, False), (128, False), (48, False), (256, False)):
+    for group, ok in ((0, True), (32, True), (64, True), (128, True), (48, False), (256, False)):
         d = _desc(group=group)
         # capacity overflow is reported only after the descriptor passed its checks
         rc = lib.kv2_quantize_append(ctypes.byref(d), P(0x1000), P(0x2000), 10, 250, 1, None)
@@ -136,8 +135,8 @@ def test_group_argument_checks(lib):
     # the statistics entry points take the group as an argument
     fit = lambda group: lib.kv2_fit_psac_basis(P(0x1000), 16, 4, 2, 128, 8, group, P(0x2000), P(0x3000),
                                                P(0x4000), None, P(0x5000), ctypes.c_size_t(16), None)
-    assert fit(64) == 2 and b"group" in lib.kv2_last_error()
-    assert fit(32) == 6                       # past the group check: the workspace is too small
+    assert fit(96) == 2 and b"group" in lib.kv2_last_error()
+    assert fit(32) == 6 and fit(64) == 6 and fit(128) == 6                       # past the group check: the workspace is too small
     cent = lambda group: lib.kv2_fit_centroids(P(0x1000), 16, 2, 128, 64, 4, group, P(0x2000), P(0x3000), 1,
                                                P(0x4000), P(0x5000), P(0x6000), ctypes.c_size_t(16), None)
     assert cent(96) == 2 and b"group" in lib.kv2_last_error()
