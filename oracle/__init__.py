@@ -152,7 +152,7 @@ def fit(Qhist: np.ndarray, H_kv: int, r: int, group: int = 32) -> Fit:
 @dataclass
 class QuantDebug:
     cand: np.ndarray    # int32 [B][n_new][H_kv][C]: candidates in rank order
-    score: np.ndarray   # fp32 ranking scores of the candidates
+    score: np.ndarray   # fp32 weighted distances D_j of the candidates
     E: np.ndarray       # fp32 perturbation estimates of the candidates
 
 

@@ -300,17 +300,17 @@ int or_fit(const uint16_t* Qh, int n, int Hq, int Hkv, int d, int r,
 /* ------------------------------------------------------------------------ */
 /* QSAC + INT2 packing + PSAC coefficients for appended tokens.               */
 /*   Ranking (article "1. QSAC": candidates by a Query-sensitivity-weighted    */
-/*   distance): D_j = sum_c w_c (k_c - mu_jc)^2. The key's own weighted norm   */
-/*   sum_c w_c k_c^2 is the same for every j, so the ranking score is          */
-/*       score_j = nrm_j - 2 dot_j,                                            */
-/*       nrm_j = sum_c (w_c mu_jc) mu_jc,   dot_j = sum_c (w_c k_c) mu_jc,     */
-/*   each sum an fp32 fmaf chain over ascending c starting from 0, the         */
-/*   products w_c mu_jc and w_c k_c rounded to fp32 first, and                 */
-/*   score_j = fmaf(-2, dot_j, nrm_j). Candidates: the C smallest (score, j).  */
+/*   distance): the weighted squared distance itself,                          */
+/*       D_j = sum_c w_c (k_c - mu_jc)^2,                                      */
+/*   in fp32 as written: t = k_c - mu_jc (fp32 subtraction), then              */
+/*   acc = fmaf(w_c * t, t, acc) over ascending c from 0 (the product w_c * t  */
+/*   rounded to fp32 first). Candidates: the set of the C smallest (D_j, j),   */
+/*   equal distances to the lower index.                                       */
 /*   Choice (same section: estimated perturbation from the residual group's    */
 /*   dynamic range and its sensitivity): E_j = sum_g (W_g s_g) s_g, an fp32     */
-/*   fmaf chain over ascending g with s_g the group's fp16 scale; the least E  */
-/*   wins, ties to the earlier candidate.                                      */
+/*   fmaf chain over ascending g with s_g the group's fp16 scale; the least    */
+/*   (E_j, j) over the candidate set wins, so the choice depends on the set    */
+/*   alone, not on the order the ranking lists it in.                          */
 /*   PSAC coefficients (article "2. PSAC"): a_i = sum_c P_ci e_c with          */
 /*   e = residual - dequantized residual, an fp32 fmaf chain over ascending c, */
 /*   stored as fp16 (round to nearest even).                                   */
@@ -319,23 +319,29 @@ int or_fit(const uint16_t* Qh, int n, int Hq, int Hkv, int d, int r,
 /* library: [B][Hkv][cap][...], (scale, zero) per group of `group` channels.  */
 /* ------------------------------------------------------------------------ */
 
+/* weighted squared distance of key k to centre m, fp32 in the order above */
+static float qsac_distance(const float* k, const float* m, const float* wh, int d)
+{
+    float acc = 0.0f;
+    for (int c = 0; c < d; ++c) {
+        float t = k[c] - m[c];
+        float wt = wh[c] * t;
+        acc = fmaf(wt, t, acc);
+    }
+    return acc;
+}
+
 /* QSAC decision for one key k (fp32 [d]) of KV head h: returns the chosen
- * centre and leaves its residual k - mu_j in xbest. mu [M][d], nrm [M] as
- * above; scratch: score [M], cand [C], used [M], x [d]. Optional debug
- * outputs (candidate ids, scores, E per candidate) when non-NULL. */
-static int qsac_choose(const float* k, const float* wh, const float* Wgh, const float* mu, const float* nrm,
-                       int M, int C, int d, int group, float* wk, float* score, int* cand, char* used, float* x,
+ * centre and leaves its residual k - mu_j in xbest. mu [M][d]; scratch:
+ * score [M], cand [C], used [M], x [d]. Optional debug outputs (candidate ids
+ * in rank order, their distances D_j, E per candidate) when non-NULL. */
+static int qsac_choose(const float* k, const float* wh, const float* Wgh, const float* mu,
+                       int M, int C, int d, int group, float* score, int* cand, char* used, float* x,
                        float* xbest, int32_t* cand_out, float* score_out, float* E_out)
 {
     int ng = d / group;
-    for (int c = 0; c < d; ++c) wk[c] = wh[c] * k[c];
     /* ranking */
-    for (int j = 0; j < M; ++j) {
-        float dot = 0.0f;
-        const float* m = mu + (size_t)j * d;
-        for (int c = 0; c < d; ++c) dot = fmaf(wk[c], m[c], dot);
-        score[j] = fmaf(-2.0f, dot, nrm[j]);
-    }
+    for (int j = 0; j < M; ++j) score[j] = qsac_distance(k, mu + (size_t)j * d, wh, d);
     memset(used, 0, (size_t)M);
     for (int i = 0; i < C; ++i) {
         int best = -1;
@@ -364,7 +370,7 @@ static int qsac_choose(const float* k, const float* wh, const float* Wgh, const 
             E = fmaf(ws, s, E);
         }
         if (E_out) E_out[i] = E;
-        if (chosen < 0 || E < bestE) {
+        if (chosen < 0 || E < bestE || (E == bestE && j < chosen)) {
             chosen = j;
             bestE = E;
             memcpy(xbest, x, (size_t)d * sizeof(float));
@@ -373,20 +379,10 @@ static int qsac_choose(const float* k, const float* wh, const float* Wgh, const 
     return chosen;
 }
 
-/* the centres of KV head h as fp32 and their weighted norms
- * nrm_j = sum_c (w_c mu_jc) mu_jc (fp32 fmaf chain over ascending c) */
-static void qsac_tables(const uint16_t* cent, const float* wh, int h, int M, int d, float* mu, float* nrm)
+/* the centres of KV head h as fp32 */
+static void qsac_tables(const uint16_t* cent, int h, int M, int d, float* mu)
 {
-    for (int j = 0; j < M; ++j) {
-        float acc = 0.0f;
-        for (int c = 0; c < d; ++c) {
-            float m = or_f32_from_f16(cent[((size_t)h * M + j) * d + c]);
-            mu[(size_t)j * d + c] = m;
-            float wm = wh[c] * m;
-            acc = fmaf(wm, m, acc);
-        }
-        nrm[j] = acc;
-    }
+    for (size_t i = 0; i < (size_t)M * d; ++i) mu[i] = or_f32_from_f16(cent[(size_t)h * M * d + i]);
 }
 
 /* Slot of token t of (sequence b, KV head h): contiguous streams
@@ -460,11 +456,9 @@ int or_quantize(int B, int Hkv, int d, int M, int r, int cap,
         (table && (page <= 0 || cap % page))) return 1;
     int ng = d / group, nw = d / 16;
     float* mu = (float*)malloc((size_t)M * d * sizeof(float));
-    float* nrm = (float*)malloc((size_t)M * sizeof(float));
     float* score = (float*)malloc((size_t)M * sizeof(float));
     int* cand = (int*)malloc((size_t)C * sizeof(int));
     float* k = (float*)malloc((size_t)d * sizeof(float));
-    float* wk = (float*)malloc((size_t)d * sizeof(float));
     float* x = (float*)malloc((size_t)d * sizeof(float));
     float* deq = (float*)malloc((size_t)d * sizeof(float));
     float* xbest = (float*)malloc((size_t)d * sizeof(float));
@@ -474,14 +468,14 @@ int or_quantize(int B, int Hkv, int d, int M, int r, int cap,
     float* acoef = (float*)malloc(((size_t)r + 1) * sizeof(float));
     for (int h = 0; h < Hkv; ++h) {
         const float* wh = w + (size_t)h * d;
-        qsac_tables(cent, wh, h, M, d, mu, nrm);
+        qsac_tables(cent, h, M, d, mu);
         for (int b = 0; b < B; ++b) {
             for (int t = 0; t < n_new; ++t) {
                 size_t in = (((size_t)b * n_new + t) * Hkv + h) * d;
                 size_t slot = slot_at(Hkv, cap, table, page, b, h, pos + t);
                 size_t dbg = (((size_t)b * n_new + t) * Hkv + h);
                 for (int c = 0; c < d; ++c) k[c] = or_f32_from_bf16(K[in + c]);
-                int chosen = qsac_choose(k, wh, Wg + (size_t)h * ng, mu, nrm, M, C, d, group, wk, score, cand, used, x,
+                int chosen = qsac_choose(k, wh, Wg + (size_t)h * ng, mu, M, C, d, group, score, cand, used, x,
                                          xbest, cand_out ? cand_out + dbg * C : NULL,
                                          score_out ? score_out + dbg * C : NULL, E_out ? E_out + dbg * C : NULL);
                 /* residual codes, scales, zeros */
@@ -512,7 +506,7 @@ int or_quantize(int B, int Hkv, int d, int M, int r, int cap,
             }
         }
     }
-    free(mu); free(nrm); free(score); free(cand); free(k); free(wk); free(x);
+    free(mu); free(score); free(cand); free(k); free(x);
     free(deq); free(xbest); free(cw); free(szr); free(used); free(acoef);
     return 0;
 }
@@ -540,11 +534,9 @@ int or_fit_centroids(int n, int Hkv, int d, int M, int C, const uint16_t* X, con
     if (group <= 0 || d % group || C < 1 || C > M || n < 0 || iters < 0) return 1;
     int ng = d / group;
     float* mu = (float*)malloc((size_t)M * d * sizeof(float));
-    float* nrm = (float*)malloc((size_t)M * sizeof(float));
     float* score = (float*)malloc((size_t)M * sizeof(float));
     int* cand = (int*)malloc((size_t)C * sizeof(int));
     float* k = (float*)malloc((size_t)d * sizeof(float));
-    float* wk = (float*)malloc((size_t)d * sizeof(float));
     float* x = (float*)malloc((size_t)d * sizeof(float));
     float* xbest = (float*)malloc((size_t)d * sizeof(float));
     char* used = (char*)malloc((size_t)M);
@@ -554,12 +546,12 @@ int or_fit_centroids(int n, int Hkv, int d, int M, int C, const uint16_t* X, con
     for (int it = 0; it < iters; ++it) {
         for (int h = 0; h < Hkv; ++h) {
             const float* wh = w + (size_t)h * d;
-            qsac_tables(cent, wh, h, M, d, mu, nrm);
+            qsac_tables(cent, h, M, d, mu);
             /* assignment */
             for (int t = 0; t < n; ++t) {
                 const uint16_t* xr = X + ((size_t)t * Hkv + h) * d;
                 for (int c = 0; c < d; ++c) k[c] = or_f32_from_bf16(xr[c]);
-                a[t] = qsac_choose(k, wh, Wg + (size_t)h * ng, mu, nrm, M, C, d, group, wk, score, cand, used, x,
+                a[t] = qsac_choose(k, wh, Wg + (size_t)h * ng, mu, M, C, d, group, score, cand, used, x,
                                    xbest,
                                    NULL, NULL, NULL);
                 if (assign) assign[(size_t)t * Hkv + h] = a[t];
@@ -583,7 +575,7 @@ int or_fit_centroids(int n, int Hkv, int d, int M, int C, const uint16_t* X, con
             }
         }
     }
-    free(mu); free(nrm); free(score); free(cand); free(k); free(wk); free(x); free(xbest); free(used);
+    free(mu); free(score); free(cand); free(k); free(x); free(xbest); free(used);
     free(a); free(sum); free(cnt);
     return 0;
 }
