@@ -27,6 +27,11 @@ __device__ __forceinline__ uint32_t float_order(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Inverse of float_order.
+__device__ __forceinline__ float order_float(uint32_t o) {
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
+}
+
 // INT2 group codec, shared by the quantizer's decision and encoding stages.
 // zero = round-down of the minimum, scale = round-up of (max - zero)/3.
 struct GroupParams {

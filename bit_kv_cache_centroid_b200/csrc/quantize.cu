@@ -7,11 +7,13 @@
 // estimated perturbation of the INT2 residual from its dynamic range and the
 // channels' sensitivity) and section "2. Principal Subspace Attention
 // Compensation (PSAC)" (projection of the Key error on the top Query
-// directions). The fp32 operation order of every decision is the one stated in
-// include/kv2.h and reproduced bit for bit:
-//   ranking  score_j = fmaf(-2, dot_j, nrm_j), dot_j = fmaf chain over c of
-//            (w_c*k_c) * mu_jc, nrm_j = fmaf chain over c of (w_c*mu_jc) * mu_jc;
-//   choice   E_j = fmaf chain over g of (Wg_g*s_g) * s_g;
+// directions). The decisions are those of the definitions below, evaluated in
+// fp32 in the stated order, and reproduced bit for bit:
+//   ranking  D_j = sum_c w_c (k_c - mu_jc)^2: t = k_c - mu_jc, then
+//            acc = fmaf(w_c * t, t, acc) over ascending c; candidates = the set
+//            of the C smallest (D_j, j);
+//   choice   E_j = fmaf chain over g of (Wg_g*s_g) * s_g; the least (E_j, j)
+//            over the candidate set;
 //   PSAC     a_i = fmaf chain over c of P_ci * e_c.
 //
 // Structure: persistent CTAs, each bound to one KV head, stage the head's
@@ -19,12 +21,26 @@
 // (j%32)*CPL + j/32, so lane l of a warp owns centroids l, l+32, ...) and the
 // centroid norms, then loop over tiles of 8*KPT keys. Within a tile every warp
 // runs its own KPT keys through the whole pipeline with warp synchronization
-// only: w*k staging, the ranking product (register tile KPT keys x CPL
-// centres per lane, fp32 FMA on the CUDA cores), top-C by warp-wide integer
+// only: w*k staging, the ranking product, top-C by warp-wide integer
 // min-reductions of order-preserving score keys, the perturbation estimate per
-// candidate, the K-residual and V codecs and the PSAC coefficients. Ranking is
-// the dominant cost (M*d FMAs per key); tensor cores are not used, since they
-// would change the decisions.
+// candidate, the K-residual and V codecs and the PSAC coefficients.
+//
+// Ranking in two steps. The M*d products (the dominant cost) run in the
+// expanded form f_j = nrm_j - 2 dot_j, nrm_j = sum_c (w_c mu_jc) mu_jc,
+// dot_j = sum_c (w_c k_c) mu_jc (register tile KPT keys x CPL centres per
+// lane, one fp32 FMA per product, fma chains over ascending c), which equals
+// D_j - sum_c w_c k_c^2 in exact arithmetic. With Ka = sum_c |w_c| k_c^2 and
+// Na = max_j sum_c |w_c| mu_jc^2, standard error bounds of fma chains give
+// |f_j - (D_j - K)| <= g (Na + 2 sqrt(Ka Na)) (Cauchy-Schwarz bounds
+// sum_c |w_c k_c mu_jc|) and |fp32 D_j - D_j| <= g (sqrt(Ka) + sqrt(Na))^2,
+// g = gamma_{d+3} = (d+3) 2^-24 / (1 - (d+3) 2^-24). So every centre of the
+// exact C smallest has f_j <= c + 2b, where c is the C-th smallest f and
+// b = g (Ka + 2 Na + 4 sqrt(Ka Na)). When no centre outside the fast top C
+// lies under that threshold (nearly always), the fast top C is the exact set;
+// otherwise every centre under it gets its fp32 D_j by the definition and the
+// C smallest (D_j, j) are taken from those. The threshold is computed with
+// g doubled and upward rounding, so it only ever errs towards the exact path.
+// Tensor cores are not used: the exact decisions need the fp32 chains.
 #include <cfloat>
 
 #include "common.cuh"
@@ -42,13 +58,44 @@ struct QCfg {
   static constexpr int KT = kWarps * KPT;        // keys per tile
   static constexpr size_t mu_bytes = size_t(D) * MP * 2;
   static constexpr size_t warp_wk_bytes = size_t(D) * KPT * 4;   // w*k [D][KPT], later e [KPT][D]
-  // per warp: w*k / e, best (E, rank) per key, candidates, and (int8 PSAC
+  // per warp: w*k / e, best (E, centre id) per key, candidates, and (int8 PSAC
   // format only, r8 = r) the fp32 coefficients [KPT][r8] before quantization
   __host__ __device__ static size_t cand_end(int C) { return (warp_wk_bytes + size_t(KPT) * 8 + size_t(KPT) * C * 2 + 15) & ~size_t(15); }
   __host__ __device__ static size_t warp_bytes(int C, int r8) { return (cand_end(C) + size_t(KPT) * r8 * 4 + 15) & ~size_t(15); }
   __host__ __device__ static size_t head_bytes(int r) { return mu_bytes + size_t(MP) * 4 + size_t(D) * 4 + size_t(D) * r * 4; }
   static size_t smem(int C, int r, int r8) { return head_bytes(r) + size_t(kWarps) * warp_bytes(C, r8); }
 };
+
+// Upper end of the fast scores that may belong to a centre of the exact C
+// smallest distances (c: the C-th smallest fast score; bound derived in the
+// file comment, with gamma_{d+3} doubled and every operation rounded up).
+__device__ __forceinline__ float rank_threshold(float c, float ka, float na, int d) {
+  const float g = float(2 * (d + 8)) * 0x1p-24f;
+  const float cross = __fmul_ru(4.0f, __fsqrt_ru(__fmul_ru(ka, na)));
+  const float b = __fmul_ru(g, __fadd_ru(__fadd_ru(ka, __fmul_ru(2.0f, na)), cross));
+  return __fadd_ru(c, __fmul_ru(2.0f, b));
+}
+
+// D_j = sum_c w_c (k_c - mu_jc)^2 by the definition's fp32 order; krow: the
+// key's D bf16 values (16-byte aligned), mu_col: centre j's column of the
+// staged [D][MP] table.
+template <int D, int MP>
+__device__ __forceinline__ float exact_distance(const uint16_t* krow, const __half* mu_col, const float* w_s) {
+  float acc = 0.0f;
+#pragma unroll 2
+  for (int c8 = 0; c8 < D / 8; ++c8) {
+    const uint4 kv = *reinterpret_cast<const uint4*>(krow + c8 * 8);
+    const uint32_t ku[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int c = c8 * 8 + q;
+      const float kc = __uint_as_float((q & 1) ? (ku[q / 2] & 0xffff0000u) : (ku[q / 2] << 16));
+      const float t = __fsub_rn(kc, __half2float(mu_col[c * MP]));
+      acc = __fmaf_rn(__fmul_rn(w_s[c], t), t, acc);
+    }
+  }
+  return acc;
+}
 
 // GS: channels per (scale, zero) group (32, 64 or 128); a group is SPG
 // sub-groups of 32 channels (one code-word pair each)
@@ -58,11 +105,13 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
   constexpr int MP = Cfg::MP, KT = Cfg::KT;
   constexpr int NG = D / GS, NS = D / kGroup, SPG = GS / kGroup;
   static_assert(GS % kGroup == 0 && D % GS == 0, "groups of whole 32-channel sub-groups");
+  static_assert(D * KPT >= 32 * KPT + D / 2, "the w*k buffer holds the exact pass's lists and one key row");
   extern __shared__ __align__(16) unsigned char smem[];
   __half* mu_s = reinterpret_cast<__half*>(smem);                            // [D][MP]
   float* nrm_s = reinterpret_cast<float*>(smem + Cfg::mu_bytes);              // [MP]
   float* w_s = nrm_s + MP;                                                    // [D]
   float* P_s = w_s + D;                                                       // [D][r]
+  __shared__ uint32_t na_bits;   // Na = max_j sum_c |w_c| mu_jc^2 (non-negative: ordered as its bits)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int r8 = (a.psac_fmt == 1) ? a.r : 0;
   unsigned char* wbase = smem + Cfg::head_bytes(a.r) + size_t(warp) * Cfg::warp_bytes(a.C, r8);
@@ -92,6 +141,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
 
   // ---- once per CTA: centroid table (fp16, transposed, lane-interleaved), w,
   // the PSAC basis, norms
+  if (tid == 0) na_bits = 0;
   for (int i = tid; i < D; i += kThreads) w_s[i] = a.w[size_t(h) * D + i];
   for (int i = tid; i < D * a.r; i += kThreads) P_s[i] = a.P[size_t(h) * D * a.r + i];
   for (int idx = tid; idx < MP * (D / 8); idx += kThreads) {
@@ -105,18 +155,22 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
   }
   __syncthreads();
   for (int j = tid; j < MP; j += kThreads) {
-    float acc = 0.0f;
+    float acc = 0.0f, aabs = 0.0f;
     if (j < M) {
       const __half* col = mu_s + (j % 32) * CPL + j / 32;     // centroid j in the staged table
 #pragma unroll 8
       for (int c = 0; c < D; ++c) {
         const float m = __half2float(col[c * MP]);
-        acc = __fmaf_rn(__fmul_rn(w_s[c], m), m, acc);
+        const float wm = __fmul_rn(w_s[c], m);
+        acc = __fmaf_rn(wm, m, acc);
+        aabs = __fmaf_rn(fabsf(wm), fabsf(m), aabs);
       }
     }
     nrm_s[j] = acc;
+    atomicMax(&na_bits, __float_as_uint(aabs));
   }
   __syncthreads();
+  const float na = __uint_as_float(na_bits);
 
   for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
     // key k of this warp is row tile*KT + k*kWarps + warp, so that a short
@@ -126,7 +180,10 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
     if (nk <= 0) continue;                       // warp-uniform
     auto row_of = [&](int k) { return tile * KT + k * kWarps + warp; };
 
-    // ---- w*k for this warp's keys, transposed to [D][KPT]
+    // ---- w*k for this warp's keys, transposed to [D][KPT]; lane l handles
+    // key l % KPT only (32 is a multiple of KPT) and sums its share of
+    // Ka = sum_c |w_c| k_c^2 for the ranking bound
+    float ka = 0.0f;
     for (int idx = lane; idx < KPT * (D / 8); idx += 32) {
       const int k = idx % KPT, c8 = idx / KPT;
       float f[8];
@@ -143,8 +200,14 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
         for (int i = 0; i < 8; ++i) f[i] = 0.0f;
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) wk_w[(c8 * 8 + i) * KPT + k] = __fmul_rn(w_s[c8 * 8 + i], f[i]);
+      for (int i = 0; i < 8; ++i) {
+        const float wk = __fmul_rn(w_s[c8 * 8 + i], f[i]);
+        wk_w[(c8 * 8 + i) * KPT + k] = wk;
+        ka = __fmaf_rn(fabsf(wk), fabsf(f[i]), ka);
+      }
     }
+#pragma unroll
+    for (int o = 16; o >= KPT; o >>= 1) ka += __shfl_xor_sync(0xffffffffu, ka, o);
     if (lane < KPT) best_w[lane] = ~0ull;
     __syncwarp();
 
@@ -234,10 +297,18 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
       }
     }
 
-    // ---- top-C per key: C rounds of a warp-wide min of (score order, id)
+    // ---- top-C per key: C rounds of a warp-wide min of (score order, id);
+    // then the check that no other centre's fast score lies within the
+    // ranking bound of the C-th. A key that fails it (rare) has its centres
+    // under the threshold listed (ids, 32 per key, in this warp's w*k buffer,
+    // free once the ranking products are done) and is decided by the exact
+    // distances after this loop, which keeps the unrolled loop small.
+    int* lists = reinterpret_cast<int*>(wk_w);               // [KPT][32]
+    uint32_t exact_keys = 0, long_lists = 0;                 // bit k: key k needs the exact pass / has > 32
 #pragma unroll
     for (int k = 0; k < KPT; ++k) {
       if (k >= nk) break;
+      uint32_t taken = 0, last = 0;
       for (int i = 0; i < C; ++i) {
         uint32_t best = 0xFFFFFFFFu;
         int bj = 0;
@@ -251,11 +322,74 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
 #pragma unroll
           for (int j = 0; j < CPL; ++j)
             if (j == bj) ord[k][j] = 0xFFFFFFFFu;                // taken
+          taken |= 1u << bj;
         }
         if (lane == 0) cand_w[k * C + i] = uint16_t(wid);
+        last = wmin;
+      }
+      const float thr = rank_threshold(order_float(last), __shfl_sync(0xffffffffu, ka, k), na, D);
+      const uint32_t thr_o = float_order(thr);
+      bool near = false;
+#pragma unroll
+      for (int j = 0; j < CPL; ++j) near |= ord[k][j] <= thr_o;
+      if (__any_sync(0xffffffffu, near)) {
+        lists[k * 32 + lane] = -1;                           // no centre
+        __syncwarp();
+        int n = 0;
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) {
+          const bool in = ((taken >> j) & 1u) || ord[k][j] <= thr_o;
+          const uint32_t m = __ballot_sync(0xffffffffu, in);
+          const int at = n + __popc(m & ((1u << lane) - 1u));
+          if (in && at < 32) lists[k * 32 + at] = j * 32 + lane;
+          n += __popc(m);
+        }
+        exact_keys |= 1u << k;
+        if (n > 32) long_lists |= 1u << k;
       }
     }
     __syncwarp();
+    // ---- the keys whose candidate set the bound left open: fp32 D_j by the
+    // definition, one listed centre per lane, and the C smallest (D_j, j);
+    // with more than 32 centres under the threshold (degenerate tables), C
+    // rounds over every centre instead
+    for (int k = 0; k < nk; ++k) {
+      if (!((exact_keys >> k) & 1u)) continue;                // warp-uniform
+      // the key row (bf16) staged after the lists, so the serial chains
+      // read it from shared memory: D/2 words fit since D * KPT >= 32 * KPT + D/2
+      uint16_t* krow = reinterpret_cast<uint16_t*>(lists + 32 * KPT);
+      if (lane < D / 8)
+        reinterpret_cast<uint4*>(krow)[lane] = reinterpret_cast<const uint4*>(key_ptr(a.K, row_of(k)))[lane];
+      __syncwarp();
+      if (!((long_lists >> k) & 1u)) {
+        const int id = lists[k * 32 + lane];                  // -1: no centre in this slot
+        uint32_t o = 0xFFFFFFFFu;
+        if (id >= 0)
+          o = float_order(__fadd_rn(exact_distance<D, MP>(krow, mu_s + (id % 32) * CPL + id / 32, w_s), 0.0f));
+        for (int i = 0; i < C; ++i) {
+          const uint32_t wmin = __reduce_min_sync(0xffffffffu, o);
+          const uint32_t wid = __reduce_min_sync(0xffffffffu, o == wmin ? uint32_t(id) : 0xFFFFFFFFu);
+          if (uint32_t(id) == wid) o = 0xFFFFFFFFu;
+          if (lane == 0) cand_w[k * C + i] = uint16_t(wid);
+        }
+      } else {
+        uint64_t prev = 0;                                    // (order, id) of the last one taken
+        for (int i = 0; i < C; ++i) {
+          uint64_t best = ~0ull;
+          for (int j = lane; j < M; j += 32) {
+            const uint64_t key = (uint64_t(float_order(__fadd_rn(
+                                      exact_distance<D, MP>(krow, mu_s + (j % 32) * CPL + j / 32, w_s), 0.0f)))
+                                  << 32) | uint32_t(j);
+            if ((i == 0 || key > prev) && key < best) best = key;
+          }
+          const uint32_t hi = __reduce_min_sync(0xffffffffu, uint32_t(best >> 32));
+          const uint32_t lo = __reduce_min_sync(0xffffffffu, uint32_t(best >> 32) == hi ? uint32_t(best) : 0xFFFFFFFFu);
+          prev = (uint64_t(hi) << 32) | lo;
+          if (lane == 0) cand_w[k * C + i] = uint16_t(lo);
+        }
+      }
+      __syncwarp();                                           // krow is rewritten for the next key
+    }
 
     if constexpr (KPT == 1) {
       // One key per warp: the remaining phases run across the lanes (lane =
@@ -272,15 +406,16 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
       }
       // ---- perturbation estimate: lane (candidate i, group g) takes the
       // group's scale; E_i = fmaf chain over ascending g of (W_g s_g) s_g;
-      // least (E, rank)
-      int rank = 0;
+      // least (E, centre id)
+      int jc = cand_w[0];
       if (C > 1) {
-        uint32_t best_e = 0xFFFFFFFFu, best_i = 0xFFFFFFFFu;
+        uint32_t best_e = 0xFFFFFFFFu, best_j = 0xFFFFFFFFu;
         for (int i0 = 0; i0 < C; i0 += 32 / NG) {
           const int i = i0 + lane / NG, g = lane % NG;
           float sg = 0.0f;
+          int j = 0;
           if (i < C) {
-            const int j = cand_w[i];
+            j = cand_w[i];
             const int col = (j % 32) * CPL + j / 32;
             const uint16_t* kseg = krow + g * GS;
             float mn = FLT_MAX, mx = -FLT_MAX;
@@ -309,12 +444,11 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
           const bool mine = (g == 0) && (i < C);
           const uint32_t eo = mine ? float_order(E) : 0xFFFFFFFFu;
           const uint32_t emin = __reduce_min_sync(0xffffffffu, eo);
-          const uint32_t imin = __reduce_min_sync(0xffffffffu, (mine && eo == emin) ? uint32_t(i) : 0xFFFFFFFFu);
-          if (emin < best_e || (emin == best_e && imin < best_i)) { best_e = emin; best_i = imin; }
+          const uint32_t jmin = __reduce_min_sync(0xffffffffu, (mine && eo == emin) ? uint32_t(j) : 0xFFFFFFFFu);
+          if (emin < best_e || (emin == best_e && jmin < best_j)) { best_e = emin; best_j = jmin; }
         }
-        rank = int(best_i);
+        jc = int(best_j);
       }
-      const int jc = cand_w[rank];
       if (a.assign) {
         if (lane == 0) a.assign[size_t(row) * a.H + h] = jc;
       } else {
@@ -403,7 +537,8 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
       }
       }
     } else {
-    // ---- perturbation estimate per (key, candidate); least (E, rank) per key
+    // ---- perturbation estimate per (key, candidate); least (E, centre id)
+    // per key
     if (C > 1) {
       for (int task = lane; task < nk * C; task += 32) {
         const int k = task / C, i = task - k * C;
@@ -431,15 +566,14 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
           const GroupParams p = group_params(mn, mx);
           E = __fmaf_rn(__fmul_rn(a.Wg[size_t(h) * NG + g], p.s), p.s, E);
         }
-        atomicMin(&best_w[k], (static_cast<unsigned long long>(float_order(E)) << 32) | unsigned(i));
+        atomicMin(&best_w[k], (static_cast<unsigned long long>(float_order(E)) << 32) | unsigned(j));
       }
       __syncwarp();
     }
 
     if (a.assign) {
       for (int k = lane; k < nk; k += 32) {
-        const int rank = (C > 1) ? int(best_w[k] & 0xffffffffu) : 0;
-        a.assign[size_t(row_of(k)) * a.H + h] = cand_w[k * C + rank];
+        a.assign[size_t(row_of(k)) * a.H + h] = (C > 1) ? int(best_w[k] & 0xffffffffu) : cand_w[k * C];
       }
     } else {
     // ---- K residual and V codecs per (key, group); a group larger than 32
@@ -453,8 +587,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
       const size_t slot = slot_of(row);
       int j = 0, col = 0;
       if (which == 0) {
-        const int rank = (C > 1) ? int(best_w[k] & 0xffffffffu) : 0;
-        j = cand_w[k * C + rank];
+        j = (C > 1) ? int(best_w[k] & 0xffffffffu) : cand_w[k * C];
         col = (j % 32) * CPL + j / 32;
       }
       // the 32 residuals (keys) or values (which = 1) of channels c0 .. c0 + 31

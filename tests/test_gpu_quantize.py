@@ -96,6 +96,42 @@ def test_video_keys_bit_exact(orc):
     _compare(ref, got, what="video")
 
 
+@pytest.mark.parametrize("B,n_tok,pos", [(1, 300, 0), (8, 1, 77)])
+def test_near_tie_ranking_bit_exact(orc, B, n_tok, pos):
+    """Centre tables built to put near ties at the candidate boundary: centres
+    32..47 repeat 0..15 exactly and 48..63 repeat 16..31 with one channel one
+    fp16 ulp away, and C = 3 is odd, so a key's third and fourth distances are
+    often equal or within fp32 rounding. The kernel's fast ranking then defers
+    to the exact distances; candidates, choice and every packed field must
+    still equal the oracle's (general path with 300 keys, short-append path
+    with one key per sequence)."""
+    import bit_kv_cache_centroid_b200 as kv2
+    s = wl.spec("tiny", d=128, H_q=4, H_kv=2, M=64, r=8, B=B, T=n_tok, n_new=1, n_hist=64, Nq=0)
+    w = wl.make(s.name, **{k: getattr(s, k) for k in ("B", "H_q", "H_kv", "d", "M", "r", "T", "n_new", "n_hist", "Nq")})
+    s = w.spec
+    cent = w.centroids.copy()
+    cent[:, 32:48] = cent[:, 0:16]
+    cent[:, 48:64] = cent[:, 16:32]
+    rng = np.random.default_rng(5)
+    for h in range(s.H_kv):
+        for j in range(48, 64):
+            c = rng.integers(s.d)
+            cent[h, j, c] = np.uint16(cent[h, j, c] + (1 if cent[h, j, c] & 0x7FFF else 0))
+    f = orc.fit(w.Qhist, s.H_kv, s.r)
+    cap = (pos + n_tok + 15) // 16 * 16 + 16
+    ref = host_cache(s, cent, capacity=cap)
+    K = np.ascontiguousarray(w.K[:, :n_tok])
+    V = np.ascontiguousarray(w.V[:, :n_tok])
+    dbg = orc.quantize(ref, K, V, pos, 3, f.P, f.w, f.Wg, debug=True)
+    gc = gpu_cache_like(host_cache(s, cent, capacity=cap), fit=f)
+    kv2.kv2_quantize_append(gc, to_dev(K, torch.int16), to_dev(V, torch.int16), pos, 3)
+    torch.cuda.synchronize()
+    _compare(ref, gc.to_host(), what="near ties")
+    # the construction does put repeated centres among the candidates
+    pairs = np.isin(dbg.cand % 32, dbg.cand[..., :1] % 32).sum(-1) >= 2
+    assert pairs.mean() > 0.3
+
+
 @pytest.mark.slow
 def test_quant_append_full_size_sampled(orc):
     """The full quantize/append workload (4,680 new tokens x 40 heads appended
