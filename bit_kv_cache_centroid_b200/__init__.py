@@ -79,6 +79,8 @@ def _load():
     L.kv2_attention_decode.argtypes = [ctypes.POINTER(kv2_cache), I, P, I, ctypes.c_float, P, I, P, S, P]
     L.kv2_attention_decode_noalloc.restype = I
     L.kv2_attention_decode_noalloc.argtypes = [ctypes.POINTER(kv2_cache), I, P, I, ctypes.c_float, P, I, P]
+    L.kv2_decode_noalloc_error.restype = I
+    L.kv2_decode_noalloc_error.argtypes = [ctypes.POINTER(ctypes.c_int), I, P]
     L.kv2_append_attention_decode.restype = I
     L.kv2_append_attention_decode.argtypes = [ctypes.POINTER(kv2_cache), P, P, I, I, I, P, I, ctypes.c_float, P, I,
                                               P, S, P]
@@ -118,7 +120,8 @@ EXPORTS = ["kv2_status_string", "kv2_last_error", "kv2_version", "kv2_fit_worksp
            "kv2_fit_psac_basis", "kv2_fit_centroids_workspace_size", "kv2_fit_centroids",
            "kv2_top1_workspace_size", "kv2_decode_top1", "kv2_dense_top1",
            "kv2_quantize_append", "kv2_decode_workspace_size",
-           "kv2_attention_decode", "kv2_attention_decode_noalloc", "kv2_append_attention_decode",
+           "kv2_attention_decode", "kv2_attention_decode_noalloc", "kv2_decode_noalloc_error",
+           "kv2_append_attention_decode",
            "kv2_chunk_workspace_size", "kv2_attention_chunk",
            "kv2_page_bytes", "kv2_page_store", "kv2_page_load"]
 
@@ -360,6 +363,15 @@ def kv2_attention_decode_noalloc(cache: Cache, length: int, Q: torch.Tensor, sm_
     _check(_get_lib().kv2_attention_decode_noalloc(ctypes.byref(d), length, _ptr(Q), H_q, float(sm_scale), _ptr(out),
                                             out_dtype, _stream(stream)))
     return out
+
+
+def kv2_decode_noalloc_error(clear: bool = False, stream=None) -> int:
+    """The error word of the fixed scratch array on the current device (1: a
+    decode wait ran out of budget since it was last cleared); zeroes it when
+    ``clear``. Waits for ``stream``."""
+    flag = ctypes.c_int(0)
+    _check(_get_lib().kv2_decode_noalloc_error(ctypes.byref(flag), int(bool(clear)), _stream(stream)))
+    return int(flag.value)
 
 
 def kv2_chunk_workspace_size(cache: Cache, H_q: int, Nq: int) -> int:

@@ -213,21 +213,42 @@ kv2::QuantizeArgs quantize_args(const kv2_cache* c, const uint16_t* K, const uin
 }
 
 // argument checks of a decode call (the cache already checked)
-kv2_status check_decode(const kv2_cache* c, int len, const uint16_t* Q, int H_q, void* out, int out_dtype,
-                        void* ws, size_t ws_bytes) {
+// Decode arguments other than the workspace.
+kv2_status check_decode_args(const kv2_cache* c, int len, const uint16_t* Q, int H_q, void* out, int out_dtype) {
   if (H_q <= 0 || H_q % c->H_kv) return fail(KV2_ERR_UNSUPPORTED, "decode: H_q=%d not a multiple of H_kv=%d", H_q, c->H_kv);
   const int G = H_q / c->H_kv;
   if (G != 1 && G != 2 && G != 4 && G != 8) return fail(KV2_ERR_UNSUPPORTED, "decode: H_q/H_kv=%d (supported 1, 2, 4, 8)", G);
   if (len < 0 || len > c->capacity) return fail(KV2_ERR_CAPACITY, "decode: len=%d outside 0..capacity=%d", len, c->capacity);
   if (out_dtype != KV2_OUT_F32 && out_dtype != KV2_OUT_BF16) return fail(KV2_ERR_INVALID_ARG, "decode: out_dtype=%d", out_dtype);
-  if (!Q || !out || !ws || !aligned16(Q) || !aligned16(out) || !aligned16(ws))
-    return fail(KV2_ERR_INVALID_ARG, "decode: Q / out / ws NULL or not 16-byte aligned");
+  if (!Q || !out || !aligned16(Q) || !aligned16(out))
+    return fail(KV2_ERR_INVALID_ARG, "decode: Q / out NULL or not 16-byte aligned");
+  return KV2_OK;
+}
+
+kv2_status check_decode(const kv2_cache* c, int len, const uint16_t* Q, int H_q, void* out, int out_dtype,
+                        void* ws, size_t ws_bytes) {
+  if (kv2_status st = check_decode_args(c, len, Q, H_q, out, out_dtype); st != KV2_OK) return st;
+  if (!ws || !aligned16(ws)) return fail(KV2_ERR_INVALID_ARG, "decode: ws NULL or not 16-byte aligned");
   const size_t need = kv2::decode_workspace_bytes(*c, H_q, len);
   if (ws_bytes < need) return fail(KV2_ERR_WORKSPACE, "decode: workspace %zu < %zu bytes", ws_bytes, need);
   return KV2_OK;
 }
 
 }  // namespace
+
+}  // extern "C"
+
+namespace kv2 {
+kv2_status validate_decode(const kv2_cache* c, int len, const uint16_t* Q, int H_q, void* out, int out_dtype,
+                           size_t* ws_need) {
+  kv2_status st = check_cache(c, true, false);
+  if (st == KV2_OK) st = check_decode_args(c, len, Q, H_q, out, out_dtype);
+  if (st == KV2_OK) *ws_need = decode_workspace_bytes(*c, H_q, len);
+  return st;
+}
+}  // namespace kv2
+
+extern "C" {
 
 kv2_status kv2_quantize_append(const kv2_cache* c, const uint16_t* K, const uint16_t* V, int n_new,
                                int pos, int candidates, void* stream) {

@@ -127,5 +127,9 @@ cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t s);
 
 // Records the detail returned by kv2_last_error() on this thread; returns st.
 kv2_status set_last_error(kv2_status st, const char* fmt, ...);
+// Every check kv2_attention_decode makes except those of the workspace; on
+// success *ws_need is the workspace size the call needs.
+kv2_status validate_decode(const kv2_cache* c, int len, const uint16_t* Q, int H_q, void* out, int out_dtype,
+                           size_t* ws_need);
 
 }  // namespace kv2

@@ -20,10 +20,9 @@
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream). Work is
  *    enqueued asynchronously; argument errors are returned synchronously
  *    before anything is enqueued; a failed launch returns KV2_ERR_CUDA.
- *  - Supported shapes: head dim d in {64, 128}; quantization groups of 32
- *    channels (the `group` field and argument below; 64 and 128, group <= d,
- *    are part of the format and return KV2_ERR_UNSUPPORTED from this
- *    version of the library); 1 <= M <= 512 centroids per KV head (ids stored as u8 when
+ *  - Supported shapes: head dim d in {64, 128}; quantization groups of 32, 64
+ *    or 128 channels, group <= d (the `group` field and argument below; 0
+ *    selects 32); 1 <= M <= 512 centroids per KV head (ids stored as u8 when
  *    M <= 256, else u16); 0 <= r <= d PSAC rank (r a multiple of 8 for the
  *    chunk kernel, r <= 16 there); H_q a multiple of H_kv. Anything else
  *    returns KV2_ERR_UNSUPPORTED.
@@ -211,12 +210,12 @@ kv2_status kv2_dense_top1(const uint16_t* K, int B, int len, int H_kv, int d, co
  * packing and PSAC coefficients for n_new new tokens of every (batch, KV
  * head), written to slots [pos, pos + n_new) (article "1. QSAC", "2. PSAC").
  * K, V   : bf16 [B][n_new][H_kv][d].
- * candidates (C, 1..M): the C centres of smallest ranking score
- *   score_j = nrm_j - 2 sum_c (w_c k_c) mu_jc   (= weighted squared distance
- *   minus the key's own weighted norm), ties to the lower id, are kept; the one
- *   whose residual gives the least E_j = sum_g W_g s_g^2 (s_g the group's fp16
- *   scale) is chosen, ties to the better-ranked. C = 1 with w = 1 is the plain
- *   nearest-centre (QVG) assignment.
+ * candidates (C, 1..M): the C centres of smallest Query-sensitivity-weighted
+ *   distance D_j = sum_c w_c (k_c - mu_jc)^2 (fp32: t = k_c - mu_jc, then
+ *   fmaf(w_c t, t, acc) over ascending c), ties to the lower id, are kept; of
+ *   those, the one whose residual gives the least E_j = sum_g W_g s_g^2 (s_g
+ *   the group's fp16 scale) is chosen, ties to the lower id. C = 1 with w = 1
+ *   is the plain nearest-centre (QVG) assignment.
  * Codec per group of `group` channels (residual k - mu for keys, v for values): zero =
  *   fp16 round-down of the minimum, scale = fp16 round-up of (max - zero)/3,
  *   code = clamp(round-half-even((x - zero)/scale), 0, 3) (0 when scale = 0).
@@ -224,8 +223,9 @@ kv2_status kv2_dense_top1(const uint16_t* K, int B, int len, int H_kv, int d, co
  *   (psac_fmt 0), or (psac_fmt 1) stored as int8 codes with one fp16 scale per
  *   token: scale = fp16 round-up of max_i |a_i| / 127, code_i =
  *   clamp(round-half-even(a_i / scale), -127, 127) (0 when the scale is 0).
- * All quantizer decisions are taken in fp32 in the order stated in the oracle
- * and are reproducible bit for bit. Tokens outside [pos, pos+n_new) are never
+ * All quantizer decisions are those fp32 definitions, bit for bit (the
+ * kernel ranks by a faster expanded form with a proven error bound and falls
+ * back to D_j itself whenever that bound leaves the candidate set open). Tokens outside [pos, pos+n_new) are never
  * read or written; concurrent calls on overlapping slots race.
  * Errors: KV2_ERR_CAPACITY if pos < 0 or pos + n_new > capacity.
  */
@@ -243,10 +243,20 @@ size_t kv2_decode_workspace_size(const kv2_cache* cache, int H_q, int len);
 /*
  * kv2_attention_decode — one query token per sequence against the first
  * `len` cached tokens of every (batch, KV head), reading the packed cache
- * directly: logit_t = sm_scale * (q.mu[cidx_t] + sum_g (s_g sum_{c in g} q_c
- * code_c + z_g sum_{c in g} q_c) + (qP).a_t); online softmax; values
- * dequantized in registers. Split-K over the sequence, then a log-sum-exp
- * merge. fp32 arithmetic throughout.
+ * directly, as the OmniKVQuant page's abstract describes for its decode
+ * kernel (the 2-bit cache unpacked inside attention, no dense cache built).
+ * Logits follow "2. PSAC" of the QuantWM article (the Key error's projection
+ * on the top Query directions compensates the score):
+ * logit_t = sm_scale * (q.mu[cidx_t] + sum_g (s_g sum_{c in g} q_c code_c +
+ * z_g sum_{c in g} q_c) + (qP).a_t); online softmax; values dequantized in
+ * registers. Split-K over the sequence, then a log-sum-exp merge.
+ * Arithmetic: the code sums sum_{c in g} q_c code_c run as 8-bit integer
+ * tensor-core products (codes exact; q as a 16-bit fixed-point value, two
+ * signed 8-bit digits, rounding at most 2^-16 of its largest component) with
+ * exact int32 sums; the zero-point and PSAC terms and p.v use fp16 tensor-core
+ * operands (stored fp16 values exact, the query's group sums, qP and p*s_v
+ * as fp16 hi/lo pairs, about 22 significant bits); every sum is fp32;
+ * exponentials use the hardware ex2.approx (relative error about 2^-22).
  * Q   : bf16 [B][H_q][d]; out: [B][H_q][d], fp32 (KV2_OUT_F32) or bf16
  *       (KV2_OUT_BF16, round to nearest even). len = 0 writes zeros.
  * ws  : device workspace of kv2_decode_workspace_size(cache, H_q, len) bytes,
@@ -269,21 +279,39 @@ kv2_status kv2_attention_decode(const kv2_cache* cache, int len, const uint16_t*
  * framework that owns the allocator, a serving loop where cudaMalloc would
  * synchronize the device). The paper has no counterpart; it is a convenience
  * of this library.
- *  - Shapes whose kv2_decode_workspace_size exceeds 8 MiB (8388608 bytes) are
- *    rejected with KV2_ERR_WORKSPACE.
+ *  - Every argument is checked first, with the errors of kv2_attention_decode;
+ *    shapes whose kv2_decode_workspace_size exceeds 8 MiB (8388608 bytes) are
+ *    then rejected with KV2_ERR_WORKSPACE.
  *  - Every GPU that loads the library holds the 8 MiB array until exit.
  *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress) and caches it; make that first call before any
- *    stream capture.
+ *    (cudaGetSymbolAddress) and caches it per device ordinal; make that first
+ *    call before any stream capture. The address is that of the device's
+ *    primary context: do not call from another driver context or after
+ *    cudaDeviceReset in the same process.
  *  - All calls share the array and it keeps the last call's contents: calls
  *    that overlap on the GPU race on it and must be serialized by the caller.
- *  - The array starts zeroed, so its error word (see kv2_attention_decode)
- *    is sticky for the life of the process.
+ *  - The array's first 32-bit word is the decode error word of
+ *    kv2_attention_decode: it starts at 0, a decode call sets it to 1 when a
+ *    wait for its cache tiles runs out of budget (those outputs are NaN), and
+ *    no decode call clears it. Read and clear it with kv2_decode_noalloc_error.
  *  - No cudaMalloc, cudaFree or other allocating call is made.
  */
 kv2_status kv2_attention_decode_noalloc(const kv2_cache* cache, int len, const uint16_t* Q,
                                         int H_q, float sm_scale, void* out, int out_dtype,
                                         void* stream);
+
+/*
+ * kv2_decode_noalloc_error — the error word of kv2_attention_decode_noalloc's
+ * fixed array on the current device, for callers that cannot hold a
+ * workspace of their own to inspect. Allocates nothing. Enqueues a 4-byte
+ * device-to-host copy on `stream` and waits for the stream (so it sees every
+ * decode call enqueued there before it), stores the word in *flag (host
+ * memory: 0 = no wait ran out, 1 = at least one did), and when `clear` is
+ * non-zero and the word was set, zeroes it (on `stream`, waited for). The
+ * paper has no counterpart.
+ * Errors: KV2_ERR_INVALID_ARG (flag NULL), KV2_ERR_CUDA.
+ */
+kv2_status kv2_decode_noalloc_error(int* flag, int clear, void* stream);
 
 /*
  * kv2_append_attention_decode — one decode step of a serving loop: appends
@@ -319,6 +347,11 @@ size_t kv2_chunk_workspace_size(const kv2_cache* cache, int H_q, int Nq);
  * model chunk against the whole packed cache (first `len` tokens) plus the
  * chunk's own dense keys/values, block-causal by latent frame: query i sees
  * every cached token and the self tokens j with j/frame_tokens <= i/frame_tokens.
+ * The score is the compensated one of "2. PSAC" in the QuantWM article,
+ * q.(k^ + P a) = q.k^ + (qP).a, over the 2-bit cache unpacked inside the
+ * kernel (the principle the OmniKVQuant page's abstract states); the chunk
+ * shape (thousands of queries per step attending to the whole history) is
+ * that of the article's video world models ("Experimental Validation").
  * Tensor cores (tcgen05, accumulators in TMEM): packed key tiles are
  * dequantized in shared memory to fp16(code*s + fp16(z + centroid)), value
  * tiles to fp16(code*s + z), the chunk's own keys and values are rounded

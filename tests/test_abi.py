@@ -180,3 +180,24 @@ def test_plain_c_client(lib, tmp_path):
     r = subprocess.run([exe], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
     assert "c client ok" in r.stdout
+
+
+def test_noalloc_checks_arguments_before_any_device_work(lib):
+    """The allocation-free decode validates every argument before it looks up
+    its fixed array (which would load the module on the device): on a machine
+    without a GPU, bad calls still get their precise argument errors, and the
+    error-word accessor refuses a NULL flag."""
+    P = ctypes.c_void_p
+    lib.kv2_last_error.restype = ctypes.c_char_p
+    call = lambda desc, length, Q, H_q, out, dtype: lib.kv2_attention_decode_noalloc(
+        ctypes.byref(desc) if desc is not None else None, length, P(Q), H_q, ctypes.c_float(0.1), P(out), dtype, None)
+    assert call(None, 16, 0x1000, 2, 0x2000, 0) == 1 and b"NULL" in lib.kv2_last_error()
+    assert call(_desc(), 16, 0, 2, 0x2000, 0) == 1 and b"Q / out" in lib.kv2_last_error()
+    assert call(_desc(), 16, 0x1008, 2, 0x2000, 0) == 1                     # Q not 16-byte aligned
+    assert call(_desc(), 16, 0x1000, 3, 0x2000, 0) == 2                     # H_q not a multiple of H_kv
+    assert call(_desc(), 300, 0x1000, 2, 0x2000, 0) == 3                    # len beyond capacity
+    assert call(_desc(), 16, 0x1000, 2, 0x2000, 7) == 1                     # out_dtype
+    assert call(_desc(group=48), 16, 0x1000, 2, 0x2000, 0) == 2
+    big = _desc(B=512, H_kv=64, M=512, r=16, capacity=32)
+    assert call(big, 16, 0x1000, 64, 0x2000, 0) == 6 and b"fixed array" in lib.kv2_last_error()
+    assert lib.kv2_decode_noalloc_error(None, 0, None) == 1

@@ -1,12 +1,17 @@
 """kv2_attention_decode_noalloc — decode attention for callers that may not
-allocate device memory (its scratch is a fixed array inside the library).
+allocate device memory (its scratch is a fixed array inside the library), and
+kv2_decode_noalloc_error, which reads and clears that array's error word.
 
 Called through the C ABI and compared with kv2_attention_decode (which takes a
-caller-allocated workspace) on the same cache and queries, twice in a row, so
-that the second call also sees the scratch the first one left behind. The file
-sorts last so that a run stopping at the first failure has run every other test.
+caller-allocated workspace) and with the oracle on the same cache and queries.
+Within one test the shapes change from call to call (many splits, then fewer
+splits with other head counts and head dimension, then the first shape
+again), so that each call runs over scratch another shape left behind. The
+file sorts last so that a run stopping at the first failure has run every
+other test.
 """
 import ctypes
+import os
 
 import numpy as np
 import pytest
@@ -28,8 +33,8 @@ def _setup(T, seed, **ov):
         P[h] = q[:, :s.r]
     gc = gpu_cache_like(pc)
     gc.P.copy_(torch.from_numpy(P))
-    Q = to_dev(wl.bf16_bits(rng.standard_normal((s.B, s.H_q, s.d)).astype(np.float32)), torch.int16)
-    return s, gc, Q
+    Qh = wl.bf16_bits(rng.standard_normal((s.B, s.H_q, s.d)).astype(np.float32))
+    return s, pc, P, gc, Qh, to_dev(Qh, torch.int16)
 
 
 def _noalloc(kv2, gc, length, Q, scale):
@@ -44,21 +49,66 @@ def _noalloc(kv2, gc, length, Q, scale):
     return out
 
 
-@pytest.mark.parametrize("T,length,ov", [
-    (5000, 4999, dict(d=128, H_q=8, H_kv=2, M=64, r=8, B=2)),
-    (3000, 2001, dict(d=128, H_q=4, H_kv=4, M=512, r=16, B=1)),
-])
-def test_noalloc_matches_workspace_decode_twice(T, length, ov):
+def _error_word(kv2, clear):
+    flag = ctypes.c_int(-1)
+    rc = kv2.lib.kv2_decode_noalloc_error(ctypes.byref(flag), int(clear),
+                                          ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0, kv2.lib.kv2_last_error().decode()
+    return flag.value
+
+
+CASES = [
+    (5000, 4999, 21, dict(d=128, H_q=8, H_kv=2, M=64, r=8, B=2)),     # many splits per (batch, head)
+    (3000, 2001, 22, dict(d=128, H_q=4, H_kv=4, M=512, r=16, B=1)),   # u16 ids, rank 16, MHA
+    (700, 650, 23, dict(d=64, H_q=16, H_kv=2, M=32, r=8, B=3)),       # few splits, d = 64, 8 heads per group
+]
+
+
+def test_noalloc_matches_workspace_decode_and_oracle_across_shapes(orc):
+    """Shapes 0, 1, 2, then 0 again, each called twice in a row: both calls
+    equal the workspace decode's output and the oracle's within the attention
+    tolerance."""
     import bit_kv_cache_centroid_b200 as kv2
-    s, gc, Q = _setup(T, 21, **ov)
+    assert _error_word(kv2, clear=False) == 0
+    setups = [_setup(T, seed, **ov) for T, _, seed, ov in CASES]
+    for idx in (0, 1, 2, 0):
+        s, pc, P, gc, Qh, Q = setups[idx]
+        length = CASES[idx][1]
+        scale = 1.0 / np.sqrt(s.d)
+        ref = kv2.kv2_attention_decode(gc, length, Q, scale).cpu().numpy()
+        want = orc.decode(pc, P, length, Qh, scale)
+        for call in ("first", "second"):
+            got = _noalloc(kv2, gc, length, Q, scale)
+            torch.cuda.synchronize()
+            got = got.cpu().numpy()
+            assert_attention_close(got, ref, what=f"case {idx} noalloc {call} call vs workspace decode")
+            assert_attention_close(got, want, what=f"case {idx} noalloc {call} call vs oracle")
+    assert _error_word(kv2, clear=False) == 0
+
+
+def test_noalloc_error_word_reports_a_timeout_and_clears():
+    """Tile copies that are never issued (KV2_FORCE_WAIT_TIMEOUT=1): every wait
+    runs out of its budget, the outputs are NaN and the fixed array's error
+    word reads 1; clearing it reads 0 afterwards, and the next call is correct."""
+    import bit_kv_cache_centroid_b200 as kv2
+    T, length, seed, ov = CASES[0]
+    s, pc, P, gc, Qh, Q = _setup(T, seed, **ov)
     scale = 1.0 / np.sqrt(s.d)
-    ref = kv2.kv2_attention_decode(gc, length, Q, scale)
-    first = _noalloc(kv2, gc, length, Q, scale)
-    second = _noalloc(kv2, gc, length, Q, scale)
+    _error_word(kv2, clear=True)
+    os.environ["KV2_FORCE_WAIT_TIMEOUT"] = "1"
+    try:
+        bad = _noalloc(kv2, gc, length, Q, scale)
+    finally:
+        del os.environ["KV2_FORCE_WAIT_TIMEOUT"]
     torch.cuda.synchronize()
-    r = ref.cpu().numpy()
-    assert_attention_close(first.cpu().numpy(), r, what="noalloc first call")
-    assert_attention_close(second.cpu().numpy(), r, what="noalloc second call")
+    assert torch.isnan(bad).all()
+    assert _error_word(kv2, clear=True) == 1
+    assert _error_word(kv2, clear=False) == 0
+    good = _noalloc(kv2, gc, length, Q, scale)
+    torch.cuda.synchronize()
+    ref = kv2.kv2_attention_decode(gc, length, Q, scale).cpu().numpy()
+    assert_attention_close(good.cpu().numpy(), ref, what="noalloc after a cleared timeout")
+    assert _error_word(kv2, clear=False) == 0
 
 
 def test_noalloc_rejects_shapes_beyond_the_array():
