@@ -36,10 +36,14 @@ sys.path.insert(0, ROOT)
 import workloads as wl  # noqa: E402
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (read + write) of one decode_split launch on the LLM decode
-# workload, from the ncu capture summarised in profiles/decode_split_llm_decode.md;
-# None whenever the kernel has changed since that capture.
+# DRAM bytes (read + write) of one decode launch (split + combine kernels) on
+# the LLM decode workload, from the committed ncu capture of the current
+# kernels; None whenever a kernel has changed since that capture.
 DECODE_SPLIT_TRAFFIC = None
+# fp32 FMA peak of the CUDA cores, derived from the B200's unit counts: 148 SMs
+# x 128 FP32 lanes x one FMA per lane and clock (the packed f32x2 form halves
+# the instructions, not the lane count), at the SM clock in MHz
+FMA_PER_SM_CLOCK = 148 * 128
 # packed bytes per (token, KV head): K and V code words, K and V scale/zero
 # words (one per group of `group` channels), the centroid id, the PSAC
 # coefficients (fp16, or int8 codes with one fp16 scale)
@@ -291,6 +295,10 @@ def run_gpu(args, rank, world):
         result.update(extras(torch, kv2, args, pk))
     if rank == 0 and not args.no_cpu:
         result["cpu_baseline"] = cpu_baseline(args, budget_s=args.cpu_seconds)
+        if "quantize" in result:
+            result["quantize"]["cpu_baseline"] = cpu_quantize()
+        if "chunk" in result:
+            result["chunk"]["cpu_baseline"] = cpu_chunk()
     return result
 
 
@@ -391,7 +399,11 @@ def extras(torch, kv2, args, pk):
                        "token_heads_per_s": round(toks * s.H_kv / (ms * 1e-3), 1),
                        "GBps": round((rd + wr) / (ms * 1e-3) / 1e9, 2),
                        "hbm_frac": round((rd + wr) / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
-                       "ranking_TFMAps": round(fma / (ms * 1e-3) / 1e12, 3)}
+                       "ranking_TFMAps": round(fma / (ms * 1e-3) / 1e12, 3),
+                       "alu_peak_TFMAps": round(FMA_PER_SM_CLOCK * pk.get("sm_max_mhz", 1965.0) * 1e6 / 1e12, 2),
+                       "alu_frac": round(fma / (ms * 1e-3) / (FMA_PER_SM_CLOCK * pk.get("sm_max_mhz", 1965.0) * 1e6),
+                                         4),
+                       "alu_peak_source": "derived: 148 SMs x 128 fp32 lanes x 1 FMA/clock x max SM clock"}
     out["retrieval_shift"] = retrieval_shift(torch, kv2, w, s, wt, Wg, P)
     # QSAC-aware centre fitting on the chunk's new keys (5 iterations)
     X = K[0]
@@ -423,11 +435,13 @@ def extras(torch, kv2, args, pk):
 
 def chunk_flops(s: wl.Spec, length: int) -> float:
     """Algorithmic FLOPs of one chunk call: 4 d per (query, visible key) for
-    Q K^T and P V, plus 2 x 16 per (query, cached key) for the PSAC columns."""
+    Q K^T and P V, plus 2 r per (query, cached key) for the PSAC term (qP).a
+    (the kernel pads the r columns to a multiple of 16; the padding is not
+    counted)."""
     F = s.frame_tokens
     f = np.arange(s.Nq) // F
     self_seen = np.minimum((f + 1) * F, s.Nq).astype(np.float64)
-    per_head = (4.0 * s.d * (length + self_seen) + (2.0 * 16 * length if s.r else 0.0)).sum()
+    per_head = (4.0 * s.d * (length + self_seen) + 2.0 * s.r * length).sum()
     return float(per_head * s.H_q * s.B)
 
 
@@ -532,11 +546,21 @@ def long_horizon_section(torch, kv2, args, pk):
 # CPU: the oracle as it stands
 # ----------------------------------------------------------------------------
 
-def cpu_baseline(args, budget_s=15.0):
-    """Oracle decode (fp64, single thread) on whole sequences of the LLM decode
-    workload until ~budget_s of CPU time; GB/s of packed cache attended."""
-    import oracle
-    oracle.build()
+def host_info() -> dict:
+    """The host the oracle runs on: logical CPUs and the CPU model."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
+
+
+def _llm_oracle_inputs():
     s = wl.spec("llm_decode")
     pc = wl.random_packed_cache(s.with_(B=1), T=s.T + 1)
     rng = np.random.default_rng(5)
@@ -545,6 +569,15 @@ def cpu_baseline(args, budget_s=15.0):
         q, _ = np.linalg.qr(rng.standard_normal((s.d, s.d)))
         P[h] = q[:, :s.r]
     Q = wl.bf16_bits(rng.standard_normal((1, s.H_q, s.d)).astype(np.float32))
+    return s, pc, P, Q
+
+
+def cpu_baseline(args, budget_s=15.0):
+    """Oracle decode (fp64, single thread) on whole sequences of the LLM decode
+    workload until ~budget_s of CPU time; GB/s of packed cache attended."""
+    import oracle
+    oracle.build()
+    s, pc, P, Q = _llm_oracle_inputs()
     seqs, t = 0, 0.0
     while t < budget_s and seqs < 64:
         t0 = time.perf_counter()
@@ -554,20 +587,97 @@ def cpu_baseline(args, budget_s=15.0):
     bytes_ = seqs * (s.T + 1) * s.H_kv * BYTES_PER_TOKEN_HEAD(s.d, s.r, s.M)
     return {"value": round(bytes_ / t / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": f"{seqs} sequence(s) x 8 KV heads x 32 query heads x 32,769 tokens (oracle decode, fp64)",
-            "seconds": round(t, 2)}
+            "seconds": round(t, 2), "host": host_info()}
+
+
+def cpu_quantize(budget_s=8.0):
+    """Oracle quantize/append (single thread, fp32 decisions) on the first new
+    tokens of the quant_append workload, all 40 heads, until ~budget_s."""
+    import oracle
+    oracle.build()
+    s = wl.spec("quant_append")
+    w = wl.make("quant_append", T=wl.FRAME_TOKENS, with_chunk=False)
+    f = oracle.fit(w.Qhist, s.H_kv, s.r)
+    pc = wl.PackedCache.empty(s.B, s.H_kv, s.d, s.M, s.r, (s.capacity + 15) // 16 * 16, w.centroids)
+    done, t, step = 0, 0.0, 16
+    while t < budget_s and done + step <= s.n_new:
+        K = np.ascontiguousarray(w.K_new[:, done:done + step])
+        V = np.ascontiguousarray(w.V_new[:, done:done + step])
+        t0 = time.perf_counter()
+        oracle.quantize(pc, K, V, s.T + done, s.C, f.P, f.w, f.Wg)
+        t += time.perf_counter() - t0
+        done += step
+    return {"value": round(done / t, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{done} of the {s.n_new} new tokens x 40 heads (M=256, C=8, r=8)",
+            "seconds": round(t, 2), "host": host_info()}
+
+
+def cpu_chunk(budget_s=10.0):
+    """Oracle chunk attention (fp64 attention, fp16 operand emulation, single
+    thread) on query rows of one head of the video chunk workload, each over
+    the 37,440 cached tokens plus its visible self part, until ~budget_s; the
+    TFLOP/s of the sample and the full call's time extrapolated from it."""
+    import oracle
+    oracle.build()
+    s = wl.spec("video_chunk")
+    pc = wl.random_packed_cache(s, T=s.T)
+    rng = np.random.default_rng(3)
+    P = np.zeros((s.H_kv, s.d, s.r), np.float32)
+    for h in range(s.H_kv):
+        q, _ = np.linalg.qr(rng.standard_normal((s.d, s.d)))
+        P[h] = q[:, :s.r]
+    Q = wl.bf16_bits(rng.standard_normal((1, s.Nq, s.H_q, s.d)).astype(np.float32))
+    Ks = wl.bf16_bits(rng.standard_normal((1, s.Nq, s.H_kv, s.d)).astype(np.float32))
+    Vs = wl.bf16_bits(rng.standard_normal((1, s.Nq, s.H_kv, s.d)).astype(np.float32))
+    F = s.frame_tokens
+    order = rng.permutation(s.Nq)
+    n, t, flop = 0, 0.0, 0.0
+    while t < budget_s and n < s.Nq:
+        i = int(order[n])
+        t0 = time.perf_counter()
+        oracle.chunk(pc, P, s.T, Q, Ks, Vs, F, 1.0 / math.sqrt(s.d), np.array([[0, i, 0]], np.int32))
+        t += time.perf_counter() - t0
+        seen = min((i // F + 1) * F, s.Nq)
+        flop += 4.0 * s.d * (s.T + seen) + 2.0 * s.r * s.T
+        n += 1
+    full = chunk_flops(s, s.T)
+    return {"value": round(flop / t / 1e12, 8), "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} random query rows of head 0 (of {s.Nq} x {s.H_q}), each over the 37,440 cached "
+                      f"tokens + its visible self tokens",
+            "seconds": round(t, 2), "extrapolated_full_call_s": round(full / (flop / t), 1),
+            "host": host_info()}
 
 
 def run_reference(args, world: int = 1):
-    r = cpu_baseline(args, budget_s=max(2.0, args.cpu_seconds / max(args.steps, 1)))
-    ms = (r["seconds"] * 1e3)
+    """The oracle arm: W untimed and K timed steps, each step the oracle's
+    decode of one of the 8 sequences of the LLM decode workload (all 8 KV heads
+    x 32 query heads x 32,769 tokens, fp64, one host thread); value = packed
+    bytes attended per second over the timed steps."""
+    import oracle
+    oracle.build()
+    s, pc, P, Q = _llm_oracle_inputs()
+    run = lambda: oracle.decode(pc, P, s.T + 1, Q, 1.0 / math.sqrt(s.d))
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    t = time.perf_counter() - t0
+    ms = t * 1e3 / args.steps
+    bytes_step = (s.T + 1) * s.H_kv * BYTES_PER_TOKEN_HEAD(s.d, s.r, s.M)
+    value = round(bytes_step * args.steps / t / 1e9, 4)
+    sample = ("each step: 1 of the 8 sequences of the LLM decode workload (8 KV heads x 32 query heads x "
+              "32,769 tokens, oracle decode, fp64)")
+    r = {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample,
+         "seconds": round(t, 2), "extrapolated_full_step_ms": round(ms * s.B, 1), "host": host_info()}
     return {"impl": "reference",
             "metric": METRIC,
-            "value": r["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic",
             "config": decode_config(world),
             "cpu_baseline": r,
-            "e2e": {"value": r["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
 def main():
