@@ -36,10 +36,10 @@ sys.path.insert(0, ROOT)
 import workloads as wl  # noqa: E402
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (read + write) of one decode launch (split + combine kernels) on
-# the LLM decode workload, from the committed ncu capture of the current
-# kernels; None whenever a kernel has changed since that capture.
-DECODE_SPLIT_TRAFFIC = None
+# DRAM bytes (read + write) of one launch of the split kernel on the LLM
+# decode workload (237,390,336 read + 3,970,560 written, ncu capture of the
+# current kernel); None whenever the kernel changes.
+DECODE_SPLIT_TRAFFIC = 241360896
 # fp32 FMA peak of the CUDA cores, derived from the B200's unit counts: 148 SMs
 # x 128 FP32 lanes x one FMA per lane and clock (the packed f32x2 form halves
 # the instructions, not the lane count), at the SM clock in MHz
@@ -366,9 +366,10 @@ def retrieval_shift(torch, kv2, w, s, wt, Wg, P):
     return res
 
 
-def extras(torch, kv2, args, pk):
-    """Quantize/append throughput and fit time (same JSON line)."""
-    out = {}
+def quantize_section(torch, kv2, args, pk):
+    """Quantize/append throughput: 4,680 new tokens x 40 heads appended at
+    37,440 (M=256, C=8, r=8), after the PSAC basis fit; 3 untimed calls, then
+    the timed ones. Returns the section and what the later sections reuse."""
     s = wl.spec("quant_append")
     w = wl.make("quant_append", T=wl.FRAME_TOKENS, with_chunk=False)
     dev = torch.device("cuda")
@@ -394,16 +395,23 @@ def extras(torch, kv2, args, pk):
     rd = K.numel() * 2 * 2
     wr = toks * s.H_kv * BYTES_PER_TOKEN_HEAD(s.d, s.r, s.M)
     fma = toks * s.H_kv * s.M * s.d
-    out["quantize"] = {"workload": "quant_append: 4680 new tokens x 40 heads, d=128, M=256, C=8, r=8",
-                       "ms": round(ms, 4), "tokens_per_s": round(toks / (ms * 1e-3), 1),
-                       "token_heads_per_s": round(toks * s.H_kv / (ms * 1e-3), 1),
-                       "GBps": round((rd + wr) / (ms * 1e-3) / 1e9, 2),
-                       "hbm_frac": round((rd + wr) / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
-                       "ranking_TFMAps": round(fma / (ms * 1e-3) / 1e12, 3),
-                       "alu_peak_TFMAps": round(FMA_PER_SM_CLOCK * pk.get("sm_max_mhz", 1965.0) * 1e6 / 1e12, 2),
-                       "alu_frac": round(fma / (ms * 1e-3) / (FMA_PER_SM_CLOCK * pk.get("sm_max_mhz", 1965.0) * 1e6),
-                                         4),
-                       "alu_peak_source": "derived: 148 SMs x 128 fp32 lanes x 1 FMA/clock x max SM clock"}
+    sec = {"workload": "quant_append: 4680 new tokens x 40 heads, d=128, M=256, C=8, r=8",
+           "ms": round(ms, 4), "tokens_per_s": round(toks / (ms * 1e-3), 1),
+           "token_heads_per_s": round(toks * s.H_kv / (ms * 1e-3), 1),
+           "GBps": round((rd + wr) / (ms * 1e-3) / 1e9, 2),
+           "hbm_frac": round((rd + wr) / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+           "ranking_TFMAps": round(fma / (ms * 1e-3) / 1e12, 3),
+           "alu_peak_TFMAps": round(FMA_PER_SM_CLOCK * pk.get("sm_max_mhz", 1965.0) * 1e6 / 1e12, 2),
+           "alu_frac": round(fma / (ms * 1e-3) / (FMA_PER_SM_CLOCK * pk.get("sm_max_mhz", 1965.0) * 1e6), 4),
+           "alu_peak_source": "derived: 148 SMs x 128 fp32 lanes x 1 FMA/clock x max SM clock"}
+    return sec, (s, w, K, Qh, P, wt, Wg, a, b)
+
+
+def extras(torch, kv2, args, pk):
+    """Quantize/append throughput and fit time (same JSON line)."""
+    out = {}
+    dev = torch.device("cuda")
+    out["quantize"], (s, w, K, Qh, P, wt, Wg, a, b) = quantize_section(torch, kv2, args, pk)
     out["retrieval_shift"] = retrieval_shift(torch, kv2, w, s, wt, Wg, P)
     # QSAC-aware centre fitting on the chunk's new keys (5 iterations)
     X = K[0]
@@ -709,7 +717,7 @@ def main():
     if args.only == "quantize":
         import torch
         import bit_kv_cache_centroid_b200 as kv2
-        print(json.dumps(extras(torch, kv2, args, peaks()[0])), flush=True)
+        print(json.dumps(quantize_section(torch, kv2, args, peaks()[0])[0]), flush=True)
         return
     if args.only == "chunk":
         import torch
