@@ -5,11 +5,20 @@
 #include <cstdio>
 #include <cstring>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "internal.h"
 
 namespace {
 
 thread_local char g_last_error[512] = "";
+
+// An NVTX range named after the entry point, open for the call (profilers
+// show the library's calls on the host timeline; no cost without a tool).
+struct CallRange {
+  explicit CallRange(const char* name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+};
 
 kv2_status fail(kv2_status st, const char* fmt, ...) {
   va_list ap;
@@ -112,6 +121,7 @@ size_t kv2_fit_workspace_size(int H_kv, int d) {
 kv2_status kv2_fit_psac_basis(const uint16_t* Qhist, int n, int H_q, int H_kv, int d, int r, int group,
                               float* P, float* w, float* Wg, float* energy, void* ws,
                               size_t ws_bytes, void* stream) {
+  const CallRange range_("kv2_fit_psac_basis");
   if (n <= 0 || H_q <= 0 || H_kv <= 0 || r < 0) return fail(KV2_ERR_INVALID_ARG, "fit: sizes must be positive");
   if (H_q % H_kv) return fail(KV2_ERR_UNSUPPORTED, "fit: H_q=%d not a multiple of H_kv=%d", H_q, H_kv);
   if (d != 64 && d != 128) return fail(KV2_ERR_UNSUPPORTED, "fit: head dim d=%d (supported: 64, 128)", d);
@@ -132,6 +142,7 @@ size_t kv2_top1_workspace_size(int B, int nq, int H_q, int len) {
 
 kv2_status kv2_decode_top1(const kv2_cache* c, int len, const uint16_t* Q, int nq, int H_q, int32_t* top1,
                            void* ws, size_t ws_bytes, void* stream) {
+  const CallRange range_("kv2_decode_top1");
   kv2_status st = check_cache(c, true, false);
   if (st != KV2_OK) return st;
   if (H_q <= 0 || H_q % c->H_kv) return fail(KV2_ERR_UNSUPPORTED, "top1: H_q=%d not a multiple of H_kv=%d", H_q, c->H_kv);
@@ -146,6 +157,7 @@ kv2_status kv2_decode_top1(const kv2_cache* c, int len, const uint16_t* Q, int n
 
 kv2_status kv2_dense_top1(const uint16_t* K, int B, int len, int H_kv, int d, const uint16_t* Q, int nq, int H_q,
                           int32_t* top1, void* ws, size_t ws_bytes, void* stream) {
+  const CallRange range_("kv2_dense_top1");
   if (B <= 0 || nq <= 0 || H_kv <= 0 || len < 0 || d <= 0 || d > 1024)
     return fail(KV2_ERR_INVALID_ARG, "dense_top1: B=%d H_kv=%d len=%d d=%d", B, H_kv, len, d);
   if (H_q <= 0 || H_q % H_kv) return fail(KV2_ERR_UNSUPPORTED, "dense_top1: H_q=%d not a multiple of H_kv=%d", H_q, H_kv);
@@ -165,6 +177,7 @@ size_t kv2_fit_centroids_workspace_size(int H_kv, int d, int M) {
 kv2_status kv2_fit_centroids(const uint16_t* X, int n, int H_kv, int d, int M, int candidates, int group,
                              const float* w, const float* Wg, int iters, uint16_t* centroids, int32_t* assign,
                              void* ws, size_t ws_bytes, void* stream) {
+  const CallRange range_("kv2_fit_centroids");
   if (H_kv <= 0 || n < 0 || n > 65536) return fail(KV2_ERR_INVALID_ARG, "fit_centroids: H_kv=%d, n=%d", H_kv, n);
   if (d != 64 && d != 128) return fail(KV2_ERR_UNSUPPORTED, "fit_centroids: head dim d=%d (supported: 64, 128)", d);
   if (M < 1 || M > 512) return fail(KV2_ERR_UNSUPPORTED, "fit_centroids: M=%d outside 1..512", M);
@@ -252,6 +265,7 @@ extern "C" {
 
 kv2_status kv2_quantize_append(const kv2_cache* c, const uint16_t* K, const uint16_t* V, int n_new,
                                int pos, int candidates, void* stream) {
+  const CallRange range_("kv2_quantize_append");
   kv2_status st = check_cache(c, true, true);
   if (st != KV2_OK) return st;
   st = check_quantize(c, K, V, n_new, pos, candidates);
@@ -269,6 +283,7 @@ size_t kv2_decode_workspace_size(const kv2_cache* c, int H_q, int len) {
 
 kv2_status kv2_attention_decode(const kv2_cache* c, int len, const uint16_t* Q, int H_q, float sm_scale,
                                 void* out, int out_dtype, void* ws, size_t ws_bytes, void* stream) {
+  const CallRange range_("kv2_attention_decode");
   kv2_status st = check_cache(c, true, false);
   if (st != KV2_OK) return st;
   st = check_decode(c, len, Q, H_q, out, out_dtype, ws, ws_bytes);
@@ -281,6 +296,7 @@ kv2_status kv2_append_attention_decode(const kv2_cache* c, const uint16_t* K_new
                                        int n_new, int pos, int candidates, const uint16_t* Q, int H_q,
                                        float sm_scale, void* out, int out_dtype, void* ws, size_t ws_bytes,
                                        void* stream) {
+  const CallRange range_("kv2_append_attention_decode");
   kv2_status st = check_cache(c, true, true);
   if (st != KV2_OK) return st;
   st = check_quantize(c, K_new, V_new, n_new, pos, candidates);
@@ -309,6 +325,7 @@ kv2_status kv2_attention_chunk(const kv2_cache* c, int len, const uint16_t* Q, i
                                const uint16_t* Kself, const uint16_t* Vself, int frame_tokens,
                                float sm_scale, void* out, int out_dtype, void* ws, size_t ws_bytes,
                                void* stream) {
+  const CallRange range_("kv2_attention_chunk");
   kv2_status st = check_cache(c, true, false);
   if (st != KV2_OK) return st;
   if (c->d != 128) return fail(KV2_ERR_UNSUPPORTED, "chunk: head dim d=%d (supported: 128)", c->d);
@@ -395,12 +412,14 @@ size_t kv2_page_bytes(const kv2_cache* c) {
 }
 
 kv2_status kv2_page_store(const kv2_cache* c, int page, int num_pages, void* host, void* stream) {
+  const CallRange range_("kv2_page_store");
   const kv2_status st = check_page(c, page, num_pages, host);
   if (st != KV2_OK) return st;
   return page_copy(c, page, static_cast<char*>(host), true, static_cast<cudaStream_t>(stream));
 }
 
 kv2_status kv2_page_load(const kv2_cache* c, int page, int num_pages, const void* host, void* stream) {
+  const CallRange range_("kv2_page_load");
   const kv2_status st = check_page(c, page, num_pages, host);
   if (st != KV2_OK) return st;
   return page_copy(c, page, const_cast<char*>(static_cast<const char*>(host)), false,

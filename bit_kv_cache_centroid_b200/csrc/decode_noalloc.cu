@@ -30,6 +30,8 @@
 // reads it and, on request, clears it.
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "internal.h"
 
 namespace {
@@ -64,6 +66,8 @@ cudaError_t scratch_for_current_device(void** out) {
 extern "C" kv2_status kv2_attention_decode_noalloc(const kv2_cache* cache, int len, const uint16_t* Q,
                                                    int H_q, float sm_scale, void* out, int out_dtype,
                                                    void* stream) {
+  nvtxRangePushA("kv2_attention_decode_noalloc");
+  struct Pop { ~Pop() { nvtxRangePop(); } } pop_;
   // every argument check first, so that a bad call neither loads the module
   // nor touches the device
   size_t need = 0;
