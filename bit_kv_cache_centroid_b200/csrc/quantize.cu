@@ -416,19 +416,20 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
           int j = 0;
           if (i < C) {
             j = cand_w[i];
-            const int col = (j % 32) * CPL + j / 32;
+            const uint4* mseg = reinterpret_cast<const uint4*>(cent + size_t(j) * D + g * GS);   // global, L2
             const uint16_t* kseg = krow + g * GS;
             float mn = FLT_MAX, mx = -FLT_MAX;
 #pragma unroll
             for (int c = 0; c < GS; c += 8) {
               const uint4 kv = *reinterpret_cast<const uint4*>(kseg + c);
+              const uint4 mv = __ldg(mseg + c / 8);
               const uint32_t ku[4] = {kv.x, kv.y, kv.z, kv.w};
+              const uint32_t mu4[4] = {mv.x, mv.y, mv.z, mv.w};
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
-                const float m0 = __half2float(mu_s[(g * GS + c + 2 * q) * MP + col]);
-                const float m1 = __half2float(mu_s[(g * GS + c + 2 * q + 1) * MP + col]);
-                const float x0 = __fsub_rn(__uint_as_float(ku[q] << 16), m0);
-                const float x1 = __fsub_rn(__uint_as_float(ku[q] & 0xffff0000u), m1);
+                const float2 m = __half22float2(*reinterpret_cast<const __half2*>(&mu4[q]));
+                const float x0 = __fsub_rn(__uint_as_float(ku[q] << 16), m.x);
+                const float x1 = __fsub_rn(__uint_as_float(ku[q] & 0xffff0000u), m.y);
                 mn = fmin3(mn, x0, x1);
                 mx = fmax3(mx, x0, x1);
               }
@@ -454,7 +455,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
       } else {
       // ---- K residual and V codecs, lane = channel of each 32-channel
       // sub-group; a group's range spans its SPG sub-groups and the lanes
-      const int colc = (jc % 32) * CPL + jc / 32;
+      const __half* crow = cent + size_t(jc) * D;      // lanes read consecutive channels
       const size_t slot = slot_of(row);
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
@@ -464,7 +465,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
 #pragma unroll
           for (int u = 0; u < SPG; ++u) {
             const int k = g * SPG + u, c = k * kGroup + lane;
-            x[u] = (which == 0) ? __fsub_rn(kx[k], __half2float(mu_s[c * MP + colc])) : vx[k];
+            x[u] = (which == 0) ? __fsub_rn(kx[k], __half2float(crow[c])) : vx[k];
           }
           float mn = x[0], mx = x[0];
 #pragma unroll
@@ -543,7 +544,10 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
       for (int task = lane; task < nk * C; task += 32) {
         const int k = task / C, i = task - k * C;
         const int j = cand_w[k * C + i];
-        const int col = (j % 32) * CPL + j / 32;
+        // the candidate's row of the fp16 centre table in global memory (the
+        // head's table stays in L2): 16-byte reads instead of 2-byte columns
+        // of the transposed shared copy, whose lanes would collide on banks
+        const uint4* mrow = reinterpret_cast<const uint4*>(cent + size_t(j) * D);
         const uint16_t* krow = key_ptr(a.K, row_of(k));
         float E = 0.0f;
 #pragma unroll 1
@@ -552,13 +556,14 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
 #pragma unroll
           for (int c = g * GS; c < (g + 1) * GS; c += 8) {
             const uint4 kv = *reinterpret_cast<const uint4*>(krow + c);
+            const uint4 mv = __ldg(mrow + c / 8);
             const uint32_t ku[4] = {kv.x, kv.y, kv.z, kv.w};
+            const uint32_t mu4[4] = {mv.x, mv.y, mv.z, mv.w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const float m0 = __half2float(mu_s[(c + 2 * q) * MP + col]);
-              const float m1 = __half2float(mu_s[(c + 2 * q + 1) * MP + col]);
-              const float x0 = __fsub_rn(__uint_as_float(ku[q] << 16), m0);
-              const float x1 = __fsub_rn(__uint_as_float(ku[q] & 0xffff0000u), m1);
+              const float2 m = __half22float2(*reinterpret_cast<const __half2*>(&mu4[q]));
+              const float x0 = __fsub_rn(__uint_as_float(ku[q] << 16), m.x);
+              const float x1 = __fsub_rn(__uint_as_float(ku[q] & 0xffff0000u), m.y);
               mn = fmin3(mn, x0, x1);
               mx = fmax3(mx, x0, x1);
             }
@@ -585,11 +590,9 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
       const int k = kg / NG, g = kg - k * NG;
       const int row = row_of(k);
       const size_t slot = slot_of(row);
-      int j = 0, col = 0;
-      if (which == 0) {
-        j = (C > 1) ? int(best_w[k] & 0xffffffffu) : cand_w[k * C];
-        col = (j % 32) * CPL + j / 32;
-      }
+      int j = 0;
+      if (which == 0) j = (C > 1) ? int(best_w[k] & 0xffffffffu) : cand_w[k * C];
+      const uint4* mrow = reinterpret_cast<const uint4*>(cent + size_t(j) * D);   // as in the estimate
       // the 32 residuals (keys) or values (which = 1) of channels c0 .. c0 + 31
       auto load32 = [&](int c0, float (&x)[kGroup]) {
         if (which == 0) {
@@ -597,12 +600,14 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantizeArgs a) {
 #pragma unroll
           for (int c = 0; c < kGroup; c += 8) {
             const uint4 kv = *reinterpret_cast<const uint4*>(krow + c);
+            const uint4 mv = __ldg(mrow + (c0 + c) / 8);
             const uint32_t ku[4] = {kv.x, kv.y, kv.z, kv.w};
+            const uint32_t mu4[4] = {mv.x, mv.y, mv.z, mv.w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              x[c + 2 * q] = __fsub_rn(__uint_as_float(ku[q] << 16), __half2float(mu_s[(c0 + c + 2 * q) * MP + col]));
-              x[c + 2 * q + 1] = __fsub_rn(__uint_as_float(ku[q] & 0xffff0000u),
-                                           __half2float(mu_s[(c0 + c + 2 * q + 1) * MP + col]));
+              const float2 m = __half22float2(*reinterpret_cast<const __half2*>(&mu4[q]));
+              x[c + 2 * q] = __fsub_rn(__uint_as_float(ku[q] << 16), m.x);
+              x[c + 2 * q + 1] = __fsub_rn(__uint_as_float(ku[q] & 0xffff0000u), m.y);
             }
           }
         } else {
