@@ -401,6 +401,18 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
 
   if (warp == kMmaWarp) {
     // ================= MMA issue (one thread) =================
+    // Shared-memory descriptors are built once: an operand's address field
+    // is its address / 16 (14 bits, no carry for any address of the CTA's
+    // shared memory), so a k-step's descriptor is the base plus its offset
+    // / 16 (one 64-bit add instead of the full encoding per MMA).
+    const uint64_t dQ0 = make_sdesc(sb + OFF_Q0, 16, 1024, kLayoutSW128);
+    const uint64_t dQ1 = make_sdesc(sb + OFF_Q1, 16, 1024, kLayoutSW128);
+    const uint64_t dU0 = make_sdesc(sb + OFF_U0, 128, 256, kLayoutNone);
+    const uint64_t dU1 = make_sdesc(sb + OFF_U1, 128, 256, kLayoutNone);
+    const uint64_t dK0 = make_sdesc(sb + OFF_STAGE + ST_K, 16, 1024, kLayoutSW128);
+    const uint64_t dA0 = make_sdesc(sb + OFF_STAGE + ST_A, 128, 256, kLayoutNone);
+    const uint64_t dV0 = make_sdesc(sb + OFF_STAGE + ST_V, 16384, 1024, kLayoutSW128);
+    const uint64_t dStage = uint64_t(STAGE_BYTES >> 4);     // the second stage's offset
     for (int jj = 0; jj < nloc; ++jj) {
       const int j = jA + jj;
       const int s = jj & 1;
@@ -409,23 +421,18 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
       if (p.force_timeout && jj == 0 && !mbar_wait_or_abort(bar + B_NEVER, 0, p.budget, abort)) break;
       if (!mbar_wait_or_abort(bar + B_KV_FULL + 8 * s, use & 1, p.budget, abort)) break;
       fence_after_sync();
-      const uint32_t st = sb + OFF_STAGE + s * STAGE_BYTES;
       bool ok = true;
       for (int x = 0; x < 2 && ok; ++x) {
         if (jj > 0 && !mbar_wait_or_abort(bar + B_O_DONE + 8 * x, (jj - 1) & 1, p.budget, abort)) { ok = false; break; }
         fence_after_sync();
         if (lane == 0) {
           const uint32_t tS = tmem + x * kKeys;
-          const uint32_t qb = sb + (x ? OFF_Q1 : OFF_Q0);
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_f16(tS, make_sdesc(qb + off, 16, 1024, kLayoutSW128),
-                    make_sdesc(st + ST_K + off, 16, 1024, kLayoutSW128), IDESC_QK, kk > 0);
+            const uint64_t off = uint64_t(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+            mma_f16(tS, (x ? dQ1 : dQ0) + off, dK0 + s * dStage + off, IDESC_QK, kk > 0);
           }
-          if (cache && p.r > 0)
-            mma_f16(tS, make_sdesc(sb + (x ? OFF_U1 : OFF_U0), 128, 256, kLayoutNone),
-                    make_sdesc(st + ST_A, 128, 256, kLayoutNone), IDESC_UA, 1);
+          if (cache && p.r > 0) mma_f16(tS, x ? dU1 : dU0, dA0 + s * dStage, IDESC_UA, 1);
           mma_commit(bar + B_S_FULL + 8 * x);
         }
         __syncwarp();
@@ -438,8 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_attn_kernel(ChunkParams p) 
           const uint32_t tP = tmem + x * kKeys, tO = tmem + 2 * kKeys + x * kD;
 #pragma unroll
           for (int kk = 0; kk < kKeys / 16; ++kk)
-            mma_f16_tmem_a(tO, tP + kk * 8, make_sdesc(st + ST_V + kk * 2048, 16384, 1024, kLayoutSW128), IDESC_PV,
-                           (jj > 0 || kk > 0));
+            mma_f16_tmem_a(tO, tP + kk * 8, dV0 + s * dStage + uint64_t(kk * 2048 >> 4), IDESC_PV, (jj > 0 || kk > 0));
           mma_commit(bar + B_O_DONE + 8 * x);
           if (x == 1) mma_commit(bar + B_KV_EMPTY + 8 * s);   // stage free once every MMA on it is done
         }
