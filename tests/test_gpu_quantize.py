@@ -132,6 +132,35 @@ def test_near_tie_ranking_bit_exact(orc, B, n_tok, pos):
     assert pairs.mean() > 0.3
 
 
+@pytest.mark.parametrize("B,n_tok,pos,M,C", [(1, 96, 0, 64, 3), (4, 1, 9, 64, 5), (1, 40, 0, 512, 8)])
+def test_all_centres_tied_bit_exact(orc, B, n_tok, pos, M, C):
+    """Degenerate tables: every centre equal (all distances tie) or two
+    values only, so far more than 32 centres fall within the ranking bound and
+    the kernel takes its every-centre exact pass; the C lowest ids must win
+    exactly as in the oracle (general path, one-key path, 16-bit ids)."""
+    import bit_kv_cache_centroid_b200 as kv2
+    s = wl.spec("tiny", d=128, H_q=2, H_kv=2, M=M, r=8, B=B, T=n_tok, n_new=1, n_hist=64, Nq=0)
+    w = wl.make(s.name, **{k: getattr(s, k) for k in ("B", "H_q", "H_kv", "d", "M", "r", "T", "n_new", "n_hist", "Nq")})
+    s = w.spec
+    cent = w.centroids.copy()
+    cent[0] = cent[0, :1]                       # head 0: every centre the same
+    cent[1, 1::2] = cent[1, 1:2]                # head 1: two distinct centres, each repeated
+    cent[1, 0::2] = cent[1, 0:1]
+    f = orc.fit(w.Qhist, s.H_kv, s.r)
+    cap = (pos + n_tok + 15) // 16 * 16 + 16
+    ref = host_cache(s, cent, capacity=cap)
+    K = np.ascontiguousarray(w.K[:, :n_tok])
+    V = np.ascontiguousarray(w.V[:, :n_tok])
+    orc.quantize(ref, K, V, pos, C, f.P, f.w, f.Wg)
+    gc = gpu_cache_like(host_cache(s, cent, capacity=cap), fit=f)
+    kv2.kv2_quantize_append(gc, to_dev(K, torch.int16), to_dev(V, torch.int16), pos, C)
+    torch.cuda.synchronize()
+    got = gc.to_host()
+    _compare(ref, got, what="tied centres")
+    sl = (slice(None), 0, slice(pos, pos + n_tok))
+    assert np.all(got["cidx"][sl] < C)          # all tie: the C lowest ids are the candidates
+
+
 @pytest.mark.slow
 def test_quant_append_full_size_sampled(orc):
     """The full quantize/append workload (4,680 new tokens x 40 heads appended
