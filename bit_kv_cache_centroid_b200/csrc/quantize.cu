@@ -261,11 +261,17 @@ __global__ void __launch_bounds__(kThreads, CPL >= 16 ? 1 : 2) quantize_kernel(Q
   // a decode launched as this kernel's programmatic dependent may start now;
   // it waits for this grid before reading the slots written here
   asm volatile("griddepcontrol.launch_dependents;");
-  const int h = blockIdx.y;
+  // work: the tiles of every head in one list (head-major); CTA b takes the
+  // b-th of gridDim.x equal runs, so every resident CTA has the same number
+  // of tiles, and stages a head's tables when its run enters that head
   const int rows_total = a.B * a.n_new;
-  const int ntiles = (rows_total + KT - 1) / KT;
+  const int ntiles = (rows_total + KT - 1) / KT;       // per head
+  const long long nwork = static_cast<long long>(ntiles) * a.H;
+  const long long lo = nwork * blockIdx.x / gridDim.x, hi = nwork * (blockIdx.x + 1) / gridDim.x;
   const int M = a.M, C = a.C;
-  const __half* cent = reinterpret_cast<const __half*>(a.cent) + size_t(h) * M * D;
+  int h = -1;
+  const __half* cent = nullptr;
+  float na = 0.0f, mabs = 0.0f;
 
   auto key_ptr = [&](const uint16_t* base, int row) {
     const int b = row / a.n_new, t = row - b * a.n_new;
@@ -276,44 +282,50 @@ __global__ void __launch_bounds__(kThreads, CPL >= 16 ? 1 : 2) quantize_kernel(Q
     return cache_slot(a.table, a.page, a.H, a.cap, b, h, a.pos + t);
   };
 
-  // ---- once per CTA: centroid table (fp16 rows, chunks permuted; zero rows
-  // past M), w, the PSAC basis, norms
-  if (tid == 0) na_bits = mabs_bits = 0;
-  for (int i = tid; i < D; i += kThreads) w_s[i] = a.w[size_t(h) * D + i];
-  for (int i = tid; i < D * a.r; i += kThreads) P_s[i] = a.P[size_t(h) * D * a.r + i];
-  for (int idx = tid; idx < MP * (D / 8); idx += kThreads) {
-    const int j = idx / (D / 8), c8 = idx % (D / 8);
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (j < M) v = *reinterpret_cast<const uint4*>(cent + size_t(j) * D + c8 * 8);
-    *reinterpret_cast<uint4*>(mu_s + mu_index<D>(j, c8)) = v;
-  }
-  __syncthreads();
-  for (int j = tid; j < MP; j += kThreads) {
-    float acc = 0.0f, aabs = 0.0f, mabs = 0.0f;
-    if (j < M) {
-#pragma unroll 2
-      for (int c8 = 0; c8 < D / 8; ++c8) {
-        const uint4 mv = *reinterpret_cast<const uint4*>(mu_s + mu_index<D>(j, c8));
-        const __half* hv = reinterpret_cast<const __half*>(&mv);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float m = __half2float(hv[q]);
-          const float wm = __fmul_rn(w_s[c8 * 8 + q], m);
-          acc = __fmaf_rn(wm, m, acc);
-          aabs = __fmaf_rn(fabsf(wm), fabsf(m), aabs);
-          mabs = __fadd_ru(mabs, fabsf(m));
-        }
+  for (long long wi = lo; wi < hi; ++wi) {
+    const int tile = int(wi % ntiles);
+    if (int(wi / ntiles) != h) {
+      // ---- once per head in the run: centroid table (fp16 rows, chunks
+      // permuted; zero rows past M), w, the PSAC basis, norms
+      h = int(wi / ntiles);
+      cent = reinterpret_cast<const __half*>(a.cent) + size_t(h) * M * D;
+      __syncthreads();                                // the previous head's tables are no longer read
+      if (tid == 0) na_bits = mabs_bits = 0;
+      for (int i = tid; i < D; i += kThreads) w_s[i] = a.w[size_t(h) * D + i];
+      for (int i = tid; i < D * a.r; i += kThreads) P_s[i] = a.P[size_t(h) * D * a.r + i];
+      for (int idx = tid; idx < MP * (D / 8); idx += kThreads) {
+        const int j = idx / (D / 8), c8 = idx % (D / 8);
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (j < M) v = *reinterpret_cast<const uint4*>(cent + size_t(j) * D + c8 * 8);
+        *reinterpret_cast<uint4*>(mu_s + mu_index<D>(j, c8)) = v;
       }
+      __syncthreads();
+      for (int j = tid; j < MP; j += kThreads) {
+        float acc = 0.0f, aabs = 0.0f, asum = 0.0f;
+        if (j < M) {
+#pragma unroll 2
+          for (int c8 = 0; c8 < D / 8; ++c8) {
+            const uint4 mv = *reinterpret_cast<const uint4*>(mu_s + mu_index<D>(j, c8));
+            const __half* hv = reinterpret_cast<const __half*>(&mv);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float m = __half2float(hv[q]);
+              const float wm = __fmul_rn(w_s[c8 * 8 + q], m);
+              acc = __fmaf_rn(wm, m, acc);
+              aabs = __fmaf_rn(fabsf(wm), fabsf(m), aabs);
+              asum = __fadd_ru(asum, fabsf(m));
+            }
+          }
+        }
+        nrm_s[j] = acc;
+        atomicMax(&na_bits, __float_as_uint(aabs));
+        atomicMax(&mabs_bits, __float_as_uint(asum));
+      }
+      __syncthreads();
+      na = __uint_as_float(na_bits);
+      mabs = __uint_as_float(mabs_bits);
     }
-    nrm_s[j] = acc;
-    atomicMax(&na_bits, __float_as_uint(aabs));
-    atomicMax(&mabs_bits, __float_as_uint(mabs));
-  }
-  __syncthreads();
-  const float na = __uint_as_float(na_bits);
-  const float mabs = __uint_as_float(mabs_bits);
 
-  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
     // key k of this warp is row tile*KT + k*kWarps + warp, so that a short
     // append spreads over all warps
     const int rem = rows_total - tile * KT - warp;
@@ -1052,11 +1064,9 @@ cudaError_t launch_cfg(const QuantizeArgs& a, cudaStream_t s) {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int rows = a.B * a.n_new;
-  const int ntiles = (rows + Cfg::KT - 1) / Cfg::KT;
-  int per_head = (sms * per_sm) / a.H;          // persistent CTAs per head: one wave in total
-  per_head = per_head < 1 ? 1 : (per_head > ntiles ? ntiles : per_head);
-  dim3 grid(per_head, a.H);
-  kern<<<grid, kThreads, smem, s>>>(a);
+  const long long nwork = static_cast<long long>((rows + Cfg::KT - 1) / Cfg::KT) * a.H;
+  const long long resident = static_cast<long long>(sms) * per_sm;   // one wave of persistent CTAs
+  kern<<<unsigned(nwork < resident ? nwork : resident), kThreads, smem, s>>>(a);
   return cudaGetLastError();
 }
 
