@@ -522,19 +522,20 @@ __global__ void __launch_bounds__(kThreads, CPL >= 16 ? 1 : 2) quantize_kernel(Q
       }
     }
 
-    // ---- top-C per key: C rounds of a warp-wide min of (score order, id);
-    // then the check that no other centre's fast score lies within the
-    // ranking bound of the C-th. A key that fails it has its centres under
-    // the threshold listed in this warp's w*k buffer (free once the ranking
-    // products are done) and is decided after this loop, which keeps the
-    // unrolled loop small. With several keys per warp and 1 < C < 15 the
-    // list holds (score, id) of the fast top C and of the others under the
-    // threshold, and slot 15 the limit below which a centre is surely in the
-    // exact set (f_j < f_(C+1) - 2b: every centre outside the fast top C has
-    // D_j > D_i); the choice is then made on perturbations (below) and needs
-    // exact distances only when a centre in doubt could win it. Otherwise
-    // (or with more listed centres than fit) the list holds ids, 32 per key,
-    // and the exact distances decide the candidate set.
+    // ---- top-C per key: C rounds of a warp-wide min over the lanes' sorted
+    // lists of packed scores; then the check that no other centre's fast
+    // score lies within the ranking bound of the C-th. A key that fails it
+    // has its centres under the threshold listed in this warp's w*k buffer
+    // (free once the ranking products are done) and is decided after the
+    // perturbations. With several keys per warp and 1 < C < 15 the list
+    // holds (score, id) of the C taken and of the others under the
+    // threshold, and slot 15 the entry count and the limit below which a
+    // taken centre is surely in the exact set (f_i < f_(C+1) - 2b: every
+    // centre outside the taken set has D_j > D_i); the choice is then made on
+    // perturbations and needs exact distances only when a centre in doubt
+    // could win it. Otherwise (or with more listed centres than fit) the
+    // list holds ids, 32 per key, and the exact distances decide the
+    // candidate set.
     int* lists = reinterpret_cast<int*>(wk_w);               // [KPT][32] ids
     unsigned long long* lists64 = reinterpret_cast<unsigned long long*>(wk_w);   // [KPT][16] (score, id)
     // after the lists: the key rows (bf16 [KPT][D], chunks permuted like the
@@ -548,11 +549,9 @@ __global__ void __launch_bounds__(kThreads, CPL >= 16 ? 1 : 2) quantize_kernel(Q
     // the column j (the centre is j * 32 + lane), sorted ascending per key
     constexpr uint32_t JM = CPL - 1;
     uint32_t exact_keys = 0, long_lists = 0, listed = 0;     // bit k: key k's route
-    int ntask[KPT];                                          // perturbations per key
     uint32_t last[KPT];                                      // packed key of the C-th taken
 #pragma unroll
     for (int k = 0; k < KPT; ++k) {
-      ntask[k] = k < nk ? C : 0;
       last[k] = 0;
 #pragma unroll
       for (int j = 0; j < CPL; ++j) ord[k][j] = (ord[k][j] & ~JM) | uint32_t(j);
@@ -583,51 +582,68 @@ __global__ void __launch_bounds__(kThreads, CPL >= 16 ? 1 : 2) quantize_kernel(Q
     // outside it with f_j > max_S f + 2b cannot be in the exact set, and one
     // in S with f_i < min_{j not in S} f_j - 2b surely is. The packed keys
     // bound the true orders from below (key & ~JM) and above (key | JM).
+    uint32_t near_keys = 0;                                  // bit k: a centre outside S under the threshold
 #pragma unroll
     for (int k = 0; k < KPT; ++k) {
       if (k >= nk) break;
-      const float two_b = __shfl_sync(0xffffffffu, two_b_l, k);
-      const uint32_t thr_o = float_order(__fadd_ru(order_float(last[k] | JM), two_b));
-      if (__any_sync(0xffffffffu, ord[k][0] <= thr_o)) {     // the lists are sorted: heads decide
-        if (list_mode) {
-          const uint32_t nxt = __reduce_min_sync(0xffffffffu, ord[k][0]);
-          int n = C;
+      const uint32_t thr_o =
+          float_order(__fadd_ru(order_float(last[k] | JM), __shfl_sync(0xffffffffu, two_b_l, k)));
+      if (__any_sync(0xffffffffu, ord[k][0] <= thr_o)) near_keys |= 1u << k;   // the lists are sorted: heads decide
+    }
+    // the near keys one at a time (rare), from a copy of the key's lists, so
+    // that this code is not repeated per key
+#pragma unroll 1
+    for (int k = 0; k < nk; ++k) {
+      if (!((near_keys >> k) & 1u)) continue;                 // warp-uniform
+      uint32_t cur[CPL], lastk = 0;
 #pragma unroll
-          for (int q = 0; q < CPL; ++q) {
-            const uint32_t v = ord[k][q];
-            const bool in = v <= thr_o;
-            const uint32_t m = __ballot_sync(0xffffffffu, in);
-            const int at = n + __popc(m & ((1u << lane) - 1u));
-            if (in && at < kListLen)
-              lists64[k * 16 + at] = (static_cast<unsigned long long>(v | JM) << 32) | ((v & JM) * 32 + lane);
-            n += __popc(m);
-          }
-          if (n <= kListLen) {
-            if (lane >= n && lane < kListLen) lists64[k * 16 + lane] = ~0ull;
-            if (lane == 0) lists64[k * 16 + kListLen] = float_order(__fsub_rd(order_float(nxt & ~JM), two_b));
-            listed |= 1u << k;
-            ntask[k] = n;
-            continue;
-          }
-          __syncwarp();                                      // the id list below takes these slots
-        }
-        // ids: the C taken, then the others under the threshold
-        const int taken_id = lane < C ? int(cand_w[k * C + lane]) : -1;
-        __syncwarp();
-        lists[k * 32 + lane] = taken_id;
+      for (int kk = 0; kk < KPT; ++kk) {
+        const bool sel = kk == k;
+        lastk = sel ? last[kk] : lastk;
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) cur[j] = sel ? ord[kk][j] : (kk == 0 ? 0u : cur[j]);
+      }
+      const float two_b = __shfl_sync(0xffffffffu, two_b_l, k);
+      const uint32_t thr_o = float_order(__fadd_ru(order_float(lastk | JM), two_b));
+      if (list_mode) {
+        const uint32_t nxt = __reduce_min_sync(0xffffffffu, cur[0]);
         int n = C;
 #pragma unroll
         for (int q = 0; q < CPL; ++q) {
-          const uint32_t v = ord[k][q];
+          const uint32_t v = cur[q];
           const bool in = v <= thr_o;
           const uint32_t m = __ballot_sync(0xffffffffu, in);
           const int at = n + __popc(m & ((1u << lane) - 1u));
-          if (in && at < 32) lists[k * 32 + at] = int((v & JM) * 32 + lane);
+          if (in && at < kListLen)
+            lists64[k * 16 + at] = (static_cast<unsigned long long>(v | JM) << 32) | ((v & JM) * 32 + lane);
           n += __popc(m);
         }
-        exact_keys |= 1u << k;
-        if (n > 32) long_lists |= 1u << k;
+        if (n <= kListLen) {
+          if (lane >= n && lane < kListLen) lists64[k * 16 + lane] = ~0ull;
+          if (lane == 0)       // slot 15: the entry count and the limit
+            lists64[k * 16 + kListLen] = (static_cast<unsigned long long>(n) << 32) |
+                                         float_order(__fsub_rd(order_float(nxt & ~JM), two_b));
+          listed |= 1u << k;
+          continue;
+        }
+        __syncwarp();                                        // the id list below takes these slots
       }
+      // ids: the C taken, then the others under the threshold
+      const int taken_id = lane < C ? int(cand_w[k * C + lane]) : -1;
+      __syncwarp();
+      lists[k * 32 + lane] = taken_id;
+      int n = C;
+#pragma unroll
+      for (int q = 0; q < CPL; ++q) {
+        const uint32_t v = cur[q];
+        const bool in = v <= thr_o;
+        const uint32_t m = __ballot_sync(0xffffffffu, in);
+        const int at = n + __popc(m & ((1u << lane) - 1u));
+        if (in && at < 32) lists[k * 32 + at] = int((v & JM) * 32 + lane);
+        n += __popc(m);
+      }
+      exact_keys |= 1u << k;
+      if (n > 32) long_lists |= 1u << k;
     }
     __syncwarp();
     // ---- the keys whose candidate set the bound left open: fp32 D_j by the
@@ -830,7 +846,8 @@ __global__ void __launch_bounds__(kThreads, CPL >= 16 ? 1 : 2) quantize_kernel(Q
       int off[KPT + 1];
       off[0] = 0;
 #pragma unroll
-      for (int k = 0; k < KPT; ++k) off[k + 1] = off[k] + ntask[k];
+      for (int k = 0; k < KPT; ++k)                     // tasks per key: C, or a listed key's entries
+        off[k + 1] = off[k] + (k >= nk ? 0 : ((listed >> k) & 1u) ? int(lists64[k * 16 + kListLen] >> 32) : C);
       const float* Wg_h = a.Wg + size_t(h) * NG;
       for (int t = lane; t < off[KPT]; t += 32) {
         int k = 0, base = 0;
