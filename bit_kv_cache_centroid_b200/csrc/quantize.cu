@@ -947,12 +947,28 @@ __global__ void __launch_bounds__(kThreads, CPL >= 16 ? 1 : 2) quantize_kernel(Q
         }
         const GroupParams gp = group_params(mn, mx);
         const float inv_s = __frcp_rn(gp.s);
-        uint32_t w0 = 0, w1 = 0;
+        uint32_t w0 = 0, w1 = 0, redo = 0;
 #pragma unroll
         for (int c = 0; c < kGroup; ++c) {
-          const uint32_t q = group_code_recip(x[c], gp, inv_s);
+          bool r;
+          const uint32_t q = group_code_fast(x[c], gp, inv_s, r);
+          redo |= uint32_t(r) << c;
           if (c < 16) w0 |= q << (2 * c); else w1 |= q << (2 * (c - 16));
           ev[t][c] = __fsub_rn(x[c], group_dequant(q, gp));
+        }
+        // the rare channels whose code the correctly rounded division decides
+#pragma unroll 1
+        for (; redo; redo &= redo - 1) {
+          const int c = __ffs(redo) - 1, ch = sg * kGroup + c;
+          const float xc = __fsub_rn(
+              __uint_as_float(uint32_t(rows_w[mu_index<D>(k, ch / 8) + ch % 8]) << 16),
+              __half2float(mu_s[mu_index<D>(j, ch / 8) + ch % 8]));
+          const uint32_t q = group_code(xc, gp);
+          if (c < 16) w0 = (w0 & ~(3u << (2 * c))) | (q << (2 * c));
+          else w1 = (w1 & ~(3u << (2 * (c - 16)))) | (q << (2 * (c - 16)));
+          const float e = __fsub_rn(xc, group_dequant(q, gp));
+#pragma unroll
+          for (int cc = 0; cc < kGroup; ++cc) ev[t][cc] = cc == c ? e : ev[t][cc];
         }
         if (live) {
           const size_t slot = slot_of(row_of(k));
@@ -1042,11 +1058,21 @@ __global__ void __launch_bounds__(256) value_codec_kernel(QuantizeArgs a) {
   }
   const GroupParams gp = group_params(mn, mx);
   const float inv_s = __frcp_rn(gp.s);
-  uint32_t w0 = 0, w1 = 0;
+  uint32_t w0 = 0, w1 = 0, redo = 0;
 #pragma unroll
   for (int c = 0; c < kGroup; ++c) {
-    const uint32_t q = group_code_recip(x[c], gp, inv_s);
+    bool r;
+    const uint32_t q = group_code_fast(x[c], gp, inv_s, r);
+    redo |= uint32_t(r) << c;
     if (c < 16) w0 |= q << (2 * c); else w1 |= q << (2 * (c - 16));
+  }
+  // the rare channels whose code the correctly rounded division decides
+#pragma unroll 1
+  for (; redo; redo &= redo - 1) {
+    const int c = __ffs(redo) - 1;
+    const uint32_t q = group_code(__uint_as_float(uint32_t(vrow[c]) << 16), gp);
+    if (c < 16) w0 = (w0 & ~(3u << (2 * c))) | (q << (2 * c));
+    else w1 = (w1 & ~(3u << (2 * (c - 16)))) | (q << (2 * (c - 16)));
   }
   if (live) {
     const size_t slot = cache_slot(a.table, a.page, a.H, a.cap, b, h, a.pos + tok);

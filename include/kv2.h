@@ -223,10 +223,15 @@ kv2_status kv2_dense_top1(const uint16_t* K, int B, int len, int H_kv, int d, co
  *   (psac_fmt 0), or (psac_fmt 1) stored as int8 codes with one fp16 scale per
  *   token: scale = fp16 round-up of max_i |a_i| / 127, code_i =
  *   clamp(round-half-even(a_i / scale), -127, 127) (0 when the scale is 0).
- * All quantizer decisions are those fp32 definitions, bit for bit (the
- * kernel ranks by a faster expanded form with a proven error bound and falls
- * back to D_j itself whenever that bound leaves the candidate set open). Tokens outside [pos, pos+n_new) are never
- * read or written; concurrent calls on overlapping slots race.
+ * All quantizer decisions are those fp32 definitions, bit for bit. The
+ * kernel ranks by a faster expanded form with an error bound; with more than
+ * 64 rows per head its dot products run on the tensor cores, and that bound
+ * then assumes the tensor cores' fp32 accumulation errs by at most 2^-12 of
+ * the summed product magnitudes (128x the largest error measured on B200).
+ * When the bound leaves the candidate set open, the choice comes from the
+ * perturbations of every centre that may be in the set if they decide it,
+ * else from D_j itself. Tokens outside [pos, pos+n_new) are never read or
+ * written; concurrent calls on overlapping slots race.
  * Errors: KV2_ERR_CAPACITY if pos < 0 or pos + n_new > capacity.
  */
 kv2_status kv2_quantize_append(const kv2_cache* cache, const uint16_t* K, const uint16_t* V,
