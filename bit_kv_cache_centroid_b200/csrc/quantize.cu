@@ -175,6 +175,40 @@ __device__ __forceinline__ void sort_asc(uint32_t (&v)[N]) {
       }
 }
 
+// perturbation() of two (key row, centre) pairs with their chains interleaved
+template <int D, int GS>
+__device__ __forceinline__ void perturbation2(const uint16_t* rows, const int (&kr)[2], const int (&j)[2],
+                                              const __half* mu_s, const float* Wg, float (&E)[2]) {
+  E[0] = E[1] = 0.0f;
+#pragma unroll 1
+  for (int g = 0; g < D / GS; ++g) {
+    float mn[2] = {FLT_MAX, FLT_MAX}, mx[2] = {-FLT_MAX, -FLT_MAX};
+#pragma unroll
+    for (int c = g * GS; c < (g + 1) * GS; c += 8) {
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const uint4 kv = *reinterpret_cast<const uint4*>(rows + mu_index<D>(kr[u], c / 8));
+        const uint4 mv = *reinterpret_cast<const uint4*>(mu_s + mu_index<D>(j[u], c / 8));
+        const uint32_t ku[4] = {kv.x, kv.y, kv.z, kv.w};
+        const uint32_t mu4[4] = {mv.x, mv.y, mv.z, mv.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 m = __half22float2(*reinterpret_cast<const __half2*>(&mu4[q]));
+          const float x0 = __fsub_rn(__uint_as_float(ku[q] << 16), m.x);
+          const float x1 = __fsub_rn(__uint_as_float(ku[q] & 0xffff0000u), m.y);
+          mn[u] = fmin3(mn[u], x0, x1);
+          mx[u] = fmax3(mx[u], x0, x1);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const GroupParams p = group_params(mn[u], mx[u]);
+      E[u] = __fmaf_rn(__fmul_rn(Wg[g], p.s), p.s, E[u]);
+    }
+  }
+}
+
 // warp-wide minimum of 64-bit keys (every lane gets it)
 __device__ __forceinline__ unsigned long long warp_min64(unsigned long long v) {
   const uint32_t hi = __reduce_min_sync(0xffffffffu, uint32_t(v >> 32));
@@ -849,22 +883,36 @@ __global__ void __launch_bounds__(kThreads, CPL >= 16 ? 1 : 2) quantize_kernel(Q
       for (int k = 0; k < KPT; ++k)                     // tasks per key: C, or a listed key's entries
         off[k + 1] = off[k] + (k >= nk ? 0 : ((listed >> k) & 1u) ? int(lists64[k * 16 + kListLen] >> 32) : C);
       const float* Wg_h = a.Wg + size_t(h) * NG;
-      for (int t = lane; t < off[KPT]; t += 32) {
-        int k = 0, base = 0;
+      // two tasks per lane at a time (t and t + 32), their chains independent;
+      // the trip count is the same for every lane (the loop holds a
+      // __syncwarp), lanes past the last task compute a copy and store nothing
+      for (int t0 = 0; t0 < off[KPT]; t0 += 64) {
+        int kt[2], et[2], jt[2];
 #pragma unroll
-        for (int kk = 1; kk < KPT; ++kk)
-          if (t >= off[kk]) { k = kk; base = off[kk]; }
-        const int e = t - base;
-        if ((listed >> k) & 1u) {
-          const unsigned long long ent = lists64[k * 16 + e];
-          const int j = int(uint32_t(ent) & 0xffffu);
-          const bool sure = uint32_t(ent >> 32) < uint32_t(lists64[k * 16 + kListLen]);
-          const float E = perturbation<D, GS>(rows_w, k, mu_s, j, Wg_h);
-          lists64[k * 16 + e] = (static_cast<unsigned long long>(float_order(E)) << 32) | (sure ? 0x80000000u : 0u) | uint32_t(j);
-        } else {
-          const int j = cand_w[k * C + e];
-          const float E = perturbation<D, GS>(rows_w, k, mu_s, j, Wg_h);
-          atomicMin(&best_w[k], (static_cast<unsigned long long>(float_order(E)) << 32) | unsigned(j));
+        for (int u = 0; u < 2; ++u) {
+          const int t = min(t0 + lane + 32 * u, off[KPT] - 1);
+          int k = 0, base = 0;
+#pragma unroll
+          for (int kk = 1; kk < KPT; ++kk)
+            if (t >= off[kk]) { k = kk; base = off[kk]; }
+          kt[u] = k;
+          et[u] = t - base;
+          jt[u] = ((listed >> k) & 1u) ? int(uint32_t(lists64[k * 16 + et[u]]) & 0xffffu) : int(cand_w[k * C + et[u]]);
+        }
+        float E[2];
+        perturbation2<D, GS>(rows_w, kt, jt, mu_s, Wg_h, E);
+        __syncwarp();                                   // list entries are read before any is rewritten
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (t0 + lane + 32 * u >= off[KPT]) break;
+          const int k = kt[u], e = et[u], j = jt[u];
+          if ((listed >> k) & 1u) {
+            const unsigned long long ent = lists64[k * 16 + e];
+            const bool sure = uint32_t(ent >> 32) < uint32_t(lists64[k * 16 + kListLen]);
+            lists64[k * 16 + e] = (static_cast<unsigned long long>(float_order(E[u])) << 32) | (sure ? 0x80000000u : 0u) | uint32_t(j);
+          } else {
+            atomicMin(&best_w[k], (static_cast<unsigned long long>(float_order(E[u])) << 32) | unsigned(j));
+          }
         }
       }
       __syncwarp();
