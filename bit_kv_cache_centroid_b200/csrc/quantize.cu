@@ -580,31 +580,31 @@ __global__ void __launch_bounds__(kThreads, CPL >= 16 ? 1 : 2) quantize_kernel(Q
     uint16_t* rows_w = reinterpret_cast<uint16_t*>(reinterpret_cast<unsigned char*>(wk_w) + KPT * 128);
     const bool list_mode = KPT > 1 && C > 1 && C < kListLen;
     // a lane's scores as packed keys: the order with its low bits replaced by
-    // the column j (the centre is j * 32 + lane), sorted ascending per key
-    constexpr uint32_t JM = CPL - 1;
+    // the centre id j * 32 + lane (so every key is unique and carries its
+    // centre), sorted ascending per key
+    constexpr uint32_t JM = CPL * 32 - 1;
     uint32_t exact_keys = 0, long_lists = 0, listed = 0;     // bit k: key k's route
     uint32_t last[KPT];                                      // packed key of the C-th taken
 #pragma unroll
     for (int k = 0; k < KPT; ++k) {
       last[k] = 0;
 #pragma unroll
-      for (int j = 0; j < CPL; ++j) ord[k][j] = (ord[k][j] & ~JM) | uint32_t(j);
+      for (int j = 0; j < CPL; ++j) ord[k][j] = (ord[k][j] & ~JM) | uint32_t(j * 32 + lane);
       sort_asc<CPL>(ord[k]);
     }
     // C rounds, the keys interleaved and without branches (so that the
     // reductions of different keys overlap): the least head over the lanes
-    // is taken (lowest lane among equal keys) and its lane's list moves up
+    // is taken and its lane's list moves up
     for (int i = 0; i < C; ++i) {
 #pragma unroll
       for (int k = 0; k < KPT; ++k) {
         const uint32_t head = ord[k][0];
         const uint32_t wmin = __reduce_min_sync(0xffffffffu, head);
-        const uint32_t win = __reduce_min_sync(0xffffffffu, head == wmin ? uint32_t(lane) : 32u);
-        const bool up = uint32_t(lane) == win;
+        const bool up = head == wmin;
 #pragma unroll
         for (int j = 0; j + 1 < CPL; ++j) ord[k][j] = up ? ord[k][j + 1] : ord[k][j];
         ord[k][CPL - 1] = up ? 0xFFFFFFFFu : ord[k][CPL - 1];
-        const uint32_t id = (wmin & JM) * 32 + win;
+        const uint32_t id = wmin & JM;
         last[k] = wmin;
         const bool w0 = lane == 0 && k < nk;
         if (w0) cand_w[k * C + i] = uint16_t(id);
@@ -649,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, CPL >= 16 ? 1 : 2) quantize_kernel(Q
           const uint32_t m = __ballot_sync(0xffffffffu, in);
           const int at = n + __popc(m & ((1u << lane) - 1u));
           if (in && at < kListLen)
-            lists64[k * 16 + at] = (static_cast<unsigned long long>(v | JM) << 32) | ((v & JM) * 32 + lane);
+            lists64[k * 16 + at] = (static_cast<unsigned long long>(v | JM) << 32) | (v & JM);
           n += __popc(m);
         }
         if (n <= kListLen) {
@@ -673,7 +673,7 @@ __global__ void __launch_bounds__(kThreads, CPL >= 16 ? 1 : 2) quantize_kernel(Q
         const bool in = v <= thr_o;
         const uint32_t m = __ballot_sync(0xffffffffu, in);
         const int at = n + __popc(m & ((1u << lane) - 1u));
-        if (in && at < 32) lists[k * 32 + at] = int((v & JM) * 32 + lane);
+        if (in && at < 32) lists[k * 32 + at] = int(v & JM);
         n += __popc(m);
       }
       exact_keys |= 1u << k;
