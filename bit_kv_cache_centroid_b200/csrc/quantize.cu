@@ -1069,7 +1069,10 @@ __global__ void __launch_bounds__(kThreads, CPL >= 16 ? 1 : 2) quantize_kernel(Q
 // per 32-channel sub-group of one (row, head); the SPG threads of a group are
 // consecutive lanes and share its range by shuffles (every thread takes part,
 // those past the end with their stores off). Same arithmetic as the one-key
-// path: group_params, then group_code_recip per channel.
+// path: group_params, then group_code_recip per channel. Launched as the key
+// kernel's programmatic dependent (its blocks take the SMs the key kernel's
+// CTAs leave); before it ends it waits for the key grid, so that whatever
+// the stream runs next finds both kernels' writes.
 template <int D, int GS>
 __global__ void __launch_bounds__(256) value_codec_kernel(QuantizeArgs a) {
   constexpr int NS = D / kGroup, SPG = GS / kGroup, NG = D / GS;
@@ -1127,16 +1130,11 @@ __global__ void __launch_bounds__(256) value_codec_kernel(QuantizeArgs a) {
     *reinterpret_cast<uint2*>(a.v_code + slot * (D / 16) + sg * 2) = make_uint2(w0, w1);
     if (sg % SPG == 0) a.v_sz[slot * NG + sg / SPG] = uint32_t(gp.s_bits) | (uint32_t(gp.z_bits) << 16);
   }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 template <int D, int CPL, int KPT, int GS>
 cudaError_t launch_cfg(const QuantizeArgs& a, cudaStream_t s) {
-  if (KPT > 1 && !a.assign) {                  // values first; the key kernel below ends the chain
-    const long long threads = static_cast<long long>(a.B) * a.n_new * a.H * (D / kGroup);
-    value_codec_kernel<D, GS><<<unsigned((threads + 255) / 256), 256, 0, s>>>(a);
-    const cudaError_t ev = cudaGetLastError();
-    if (ev != cudaSuccess) return ev;
-  }
   using Cfg = QCfg<D, CPL, KPT>;
   const size_t smem = Cfg::smem(a.C, a.r, a.psac_fmt == 1 ? a.r : 0);
   auto kern = quantize_kernel<D, CPL, KPT, GS>;
@@ -1158,7 +1156,20 @@ cudaError_t launch_cfg(const QuantizeArgs& a, cudaStream_t s) {
   const long long nwork = static_cast<long long>((rows + Cfg::KT - 1) / Cfg::KT) * a.H;
   const long long resident = static_cast<long long>(sms) * per_sm;   // one wave of persistent CTAs
   kern<<<unsigned(nwork < resident ? nwork : resident), kThreads, smem, s>>>(a);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e != cudaSuccess || KPT == 1 || a.assign) return e;
+  // the values of a multi-key append: the key kernel's programmatic dependent
+  const long long threads = static_cast<long long>(a.B) * a.n_new * a.H * (D / kGroup);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(unsigned((threads + 255) / 256));
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, value_codec_kernel<D, GS>, a);
 }
 
 template <int D, int GS>

@@ -166,6 +166,7 @@ def test_bounded_wait_reports_timeout_and_context_survives(orc):
     (8, 32, 8, 64, 8, 3000, 1),       # decode step: one token per sequence, tile boundary inside a split
     (2, 8, 2, 512, 16, 700, 5),       # several tokens, u16 ids, rank 16
     (1, 4, 4, 64, 8, 127, 1),         # appended token in the first (only) tile
+    (2, 8, 2, 64, 8, 700, 100),       # a long append: key kernel, value kernel, then decode
 ])
 def test_append_attention_decode_equals_the_two_calls(orc, B, H_q, H_kv, M, r, T, n_new):
     """kv2_append_attention_decode (append kernel, then the decode kernel as its
