@@ -71,17 +71,6 @@ __device__ __forceinline__ uint32_t group_code_recip(float x, const GroupParams&
   return static_cast<uint32_t>(c);
 }
 
-// group_code_recip without its rare branch: `redo` is set when the product
-// lies within 2^-18 of a half-integer, where group_code (the correctly
-// rounded division) must decide instead; the caller redoes those channels
-// out of line, which keeps unrolled loops over many channels small.
-__device__ __forceinline__ uint32_t group_code_fast(float x, const GroupParams& p, float inv_s, bool& redo) {
-  const float qa = __fmul_rn(__fsub_rn(x, p.z), inv_s);
-  redo = p.s != 0.0f && fabsf(__fsub_rn(__fsub_rn(qa, floorf(qa)), 0.5f)) < 0x1p-18f;
-  const float c = fminf(fmaxf(rintf(qa), 0.0f), 3.0f);
-  return p.s == 0.0f ? 0u : static_cast<uint32_t>(c);
-}
-
 // min / max of three floats in one instruction
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;

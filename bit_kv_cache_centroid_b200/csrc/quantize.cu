@@ -209,6 +209,38 @@ __device__ __forceinline__ void perturbation2(const uint16_t* rows, const int (&
   }
 }
 
+// Codes of the 32 values x of one sub-group with the group's (s, z): the
+// quotient (x - z) * inv_s rounded to the nearest integer and clamped to
+// 0..3, two channels per packed instruction (each lane rounded as its scalar
+// form); bit c of `redo` flags a quotient within 2^-18 of a half-integer
+// (|q - rint(q)| > 1/2 - 2^-18), whose code the correctly rounded division
+// must decide. With E, also the residual errors x - (code * s + z). A group
+// of scale 0 holds x = z only (z is the rounded-down minimum and s the
+// rounded-up range / 3): its codes are 0 and its errors x - z whatever the
+// quotient gave.
+template <bool E>
+__device__ __forceinline__ void code32(const float (&x)[kGroup], const GroupParams& gp, float inv_s,
+                                       uint32_t& w0, uint32_t& w1, uint32_t& redo, float (&ev)[kGroup]) {
+  const f32x2 z2 = pk2(gp.z, gp.z), is2 = pk2(inv_s, inv_s), s2 = pk2(gp.s, gp.s);
+  w0 = w1 = redo = 0;
+#pragma unroll
+  for (int c = 0; c < kGroup; c += 2) {
+    const float2 qa = up2(fmul2(fsub2(pk2(x[c], x[c + 1]), z2), is2));
+    const float r0 = rintf(qa.x), r1 = rintf(qa.y);
+    redo |= (uint32_t(fabsf(__fsub_rn(qa.x, r0)) > 0.5f - 0x1p-18f) << c) |
+            (uint32_t(fabsf(__fsub_rn(qa.y, r1)) > 0.5f - 0x1p-18f) << (c + 1));
+    const float c0 = fminf(fmaxf(r0, 0.0f), 3.0f), c1 = fminf(fmaxf(r1, 0.0f), 3.0f);
+    const uint32_t q = uint32_t(c0) | (uint32_t(c1) << 2);
+    if (c < 16) w0 |= q << (2 * c); else w1 |= q << (2 * (c - 16));
+    if constexpr (E) {
+      const float2 e = up2(fsub2(pk2(x[c], x[c + 1]), ffma2(pk2(c0, c1), s2, z2)));
+      ev[c] = e.x;
+      ev[c + 1] = e.y;
+    }
+  }
+  if (gp.s == 0.0f) w0 = w1 = redo = 0;
+}
+
 // warp-wide minimum of 64-bit keys (every lane gets it)
 __device__ __forceinline__ unsigned long long warp_min64(unsigned long long v) {
   const uint32_t hi = __reduce_min_sync(0xffffffffu, uint32_t(v >> 32));
@@ -532,8 +564,7 @@ __global__ void __launch_bounds__(kThreads, CPL >= 16 ? 1 : 2) quantize_kernel(Q
               for (int i = 0; i < 4; ++i) {
                 const int key = nt * 8 + 2 * t + (i & 1), cl = mh * 16 + g + 8 * (i >> 1), cj = q * 32 + cl;
                 if (key < KPT)
-                  tb[cl * TBS + key] = (cj < M) ? float_order(__fadd_rn(
-                                                      __fmaf_rn(bk[nt][i & 1], acc[2 * sl + mh][nt][i], nrm_s[cj]), 0.0f))
+                  tb[cl * TBS + key] = (cj < M) ? float_order(__fmaf_rn(bk[nt][i & 1], acc[2 * sl + mh][nt][i], nrm_s[cj]))
                                                 : 0xFFFFFFFFu;
               }
           __syncwarp();
@@ -995,15 +1026,8 @@ __global__ void __launch_bounds__(kThreads, CPL >= 16 ? 1 : 2) quantize_kernel(Q
         }
         const GroupParams gp = group_params(mn, mx);
         const float inv_s = __frcp_rn(gp.s);
-        uint32_t w0 = 0, w1 = 0, redo = 0;
-#pragma unroll
-        for (int c = 0; c < kGroup; ++c) {
-          bool r;
-          const uint32_t q = group_code_fast(x[c], gp, inv_s, r);
-          redo |= uint32_t(r) << c;
-          if (c < 16) w0 |= q << (2 * c); else w1 |= q << (2 * (c - 16));
-          ev[t][c] = __fsub_rn(x[c], group_dequant(q, gp));
-        }
+        uint32_t w0, w1, redo;
+        code32<true>(x, gp, inv_s, w0, w1, redo, ev[t]);
         // the rare channels whose code the correctly rounded division decides
 #pragma unroll 1
         for (; redo; redo &= redo - 1) {
@@ -1109,14 +1133,9 @@ __global__ void __launch_bounds__(256) value_codec_kernel(QuantizeArgs a) {
   }
   const GroupParams gp = group_params(mn, mx);
   const float inv_s = __frcp_rn(gp.s);
-  uint32_t w0 = 0, w1 = 0, redo = 0;
-#pragma unroll
-  for (int c = 0; c < kGroup; ++c) {
-    bool r;
-    const uint32_t q = group_code_fast(x[c], gp, inv_s, r);
-    redo |= uint32_t(r) << c;
-    if (c < 16) w0 |= q << (2 * c); else w1 |= q << (2 * (c - 16));
-  }
+  uint32_t w0, w1, redo;
+  float unused[kGroup];
+  code32<false>(x, gp, inv_s, w0, w1, redo, unused);
   // the rare channels whose code the correctly rounded division decides
 #pragma unroll 1
   for (; redo; redo &= redo - 1) {
