@@ -194,10 +194,10 @@ __device__ __forceinline__ void perturbation2(const uint16_t* rows, const int (&
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const float2 m = __half22float2(*reinterpret_cast<const __half2*>(&mu4[q]));
-          const float x0 = __fsub_rn(__uint_as_float(ku[q] << 16), m.x);
-          const float x1 = __fsub_rn(__uint_as_float(ku[q] & 0xffff0000u), m.y);
-          mn[u] = fmin3(mn[u], x0, x1);
-          mx[u] = fmax3(mx[u], x0, x1);
+          const float2 xx = up2(fsub2(pk2(__uint_as_float(ku[q] << 16), __uint_as_float(ku[q] & 0xffff0000u)),
+                                      pk2(m.x, m.y)));
+          mn[u] = fmin3(mn[u], xx.x, xx.y);
+          mx[u] = fmax3(mx[u], xx.x, xx.y);
         }
       }
     }
@@ -1010,8 +1010,10 @@ __global__ void __launch_bounds__(kThreads, CPL >= 16 ? 1 : 2) quantize_kernel(Q
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const float2 m = __half22float2(*reinterpret_cast<const __half2*>(&mu4[q]));
-            x[c8 * 8 + 2 * q] = __fsub_rn(__uint_as_float(ku[q] << 16), m.x);
-            x[c8 * 8 + 2 * q + 1] = __fsub_rn(__uint_as_float(ku[q] & 0xffff0000u), m.y);
+            const float2 xx = up2(fsub2(pk2(__uint_as_float(ku[q] << 16), __uint_as_float(ku[q] & 0xffff0000u)),
+                                        pk2(m.x, m.y)));
+            x[c8 * 8 + 2 * q] = xx.x;
+            x[c8 * 8 + 2 * q + 1] = xx.y;
           }
         }
         float mn = x[0], mx = x[0];
