@@ -403,7 +403,10 @@ def quantize_section(torch, kv2, args, pk):
            "ranking_TFMAps": round(fma / (ms * 1e-3) / 1e12, 3),
            "alu_peak_TFMAps": round(FMA_PER_SM_CLOCK * pk.get("sm_max_mhz", 1965.0) * 1e6 / 1e12, 2),
            "alu_frac": round(fma / (ms * 1e-3) / (FMA_PER_SM_CLOCK * pk.get("sm_max_mhz", 1965.0) * 1e6), 4),
-           "alu_peak_source": "derived: 148 SMs x 128 fp32 lanes x 1 FMA/clock x max SM clock"}
+           "alu_peak_source": "derived: 148 SMs x 128 fp32 lanes x 1 FMA/clock x max SM clock",
+           "bound": "latency",
+           "note": "alu_frac is the ranking rate against the fp32 FMA peak; the ranking products run on the "
+                   "tensor cores (mma.sync) and the kernel is latency-bound at 16 warps per SM"}
     return sec, (s, w, K, Qh, P, wt, Wg, a, b)
 
 
