@@ -16,15 +16,18 @@
 //            over the candidate set;
 //   PSAC     a_i = fmaf chain over c of P_ci * e_c.
 //
-// Structure: persistent CTAs, each bound to one KV head, stage the head's
-// centroid table once (fp16 rows [M][d], the 16-byte chunks of row j permuted
-// by chunk ^ (j % 8) so that eight rows read at one logical chunk hit eight
-// different bank groups) and the centroid norms, then loop over tiles of
-// 8*KPT keys. Within a tile every warp runs its own KPT keys through the whole
-// pipeline with warp synchronization only: w*k staging, the ranking products,
-// top-C by warp-wide integer min-reductions of order-preserving score keys
-// (lane l owning centres l, l+32, ...), the perturbation estimate per
-// candidate, the K-residual and V codecs and the PSAC coefficients.
+// Structure: one wave of persistent CTAs, each taking an equal run of the
+// head-major list of key tiles (8*KPT keys of one head) and staging a head's
+// centroid table (fp16 rows [M][d], the 16-byte chunks of row j permuted by
+// chunk ^ (j % 8) so that eight rows read at one logical chunk hit eight
+// different bank groups) and norms when its run enters that head. Within a
+// tile every warp runs its own KPT keys through the whole pipeline with warp
+// synchronization only: w*k staging, the ranking products, top-C (lane l
+// owns centres l, l+32, ...; each lane's scores become packed keys, the order
+// with the centre id in its low bits, sorted per key; C rounds of one
+// warp-wide integer minimum), the perturbation estimates, the K-residual
+// codec and the PSAC coefficients. Warps with one key also code the values;
+// the values of multi-key appends are coded by value_codec_kernel.
 //
 // Ranking in two steps. The M*d products (the dominant cost) run in the
 // expanded form f_j = nrm_j - 2 dot_j, nrm_j = sum_c (w_c mu_jc) mu_jc,
@@ -36,11 +39,19 @@
 // g = gamma_{d+3} = (d+3) 2^-24 / (1 - (d+3) 2^-24). So every centre of the
 // exact C smallest has f_j <= c + 2b, where c is the C-th smallest f and
 // b = g (Ka + 2 Na + 4 sqrt(Ka Na)) + 2 e_dot (e_dot: the dot products' own
-// error beyond an fp32 chain, below). When no centre outside the fast top C
-// lies under that threshold (nearly always), the fast top C is the exact set;
-// otherwise every centre under it gets its fp32 D_j by the definition and the
-// C smallest (D_j, j) are taken from those. The threshold is computed with
-// g doubled and upward rounding, so it only ever errs towards the exact path.
+// error beyond an fp32 chain, below). The packed keys bound each true score
+// from both sides, so any C centres S taken by them work: when no centre
+// outside S lies under max_S f + 2b, S is the exact set (nearly always).
+// Otherwise, with several keys per warp and 1 < C < 15, the key is listed:
+// S and the centres under that threshold, a taken centre i marked sure when
+// f_i < min_{j not in S} f_j - 2b (then D_i is below every D_j outside S).
+// The perturbation E of every listed centre is estimated; the least (E, id)
+// among the sure ones is the choice when it beats every doubtful one,
+// whichever doubtful centres are in the exact set; otherwise (and with one
+// key per warp, C = 1, C >= 15 or a longer list) the listed centres get their
+// fp32 D_j by the definition and the C smallest (D_j, j) decide the set. The
+// bounds are computed with g doubled and upward rounding, so they only ever
+// err towards the exact path.
 //
 // Warps with several keys (KPT > 1) take the dot products on the tensor cores
 // (mma.sync m16n8k16, fp16 operands, fp32 accumulation): A = 16 centres x 16
@@ -55,7 +66,8 @@
 // aligns each k16 block's products to the largest and truncates ("Numerical
 // behavior of NVIDIA tensor cores", Fasi, Higham, Mikaitis and Pranesh, PeerJ
 // Computer Science, 2021) bounds a chain of 16 such blocks by about 2^-13.8 S,
-// and the largest error measured on this path's hardware is far below both.
+// and the largest error measured on this path's hardware (2^-19.1 of S,
+// tests/test_gpu_tc_accumulation.py) is far below both.
 // So e_dot = (2^-12 + 2^-18) sqrt(Ka Na) + 2^-24 2^-e sum_c |mu_jc|. A warp
 // with one key (short appends) runs the products as fp32 FMAs (e_dot = 0).
 #include <cfloat>
