@@ -69,7 +69,8 @@ def test_tiny_bit_exact(orc):
     (512, 8, 16, 4, 16, 9),      # 64 keys per head: the largest short append, u16 ids
     (32, 2, 8, 3, 5, 1),         # 15 keys: warps with and without a key
     (256, 16, 8, 1, 150, 0),     # multi-key warps, C >= 15: near keys take the 32-entry id lists
-    (128, 128, 8, 1, 100, 0),    # multi-key warps, C = M: lists past 32 entries, the all-centre fallback
+    (128, 128, 8, 1, 100, 0),    # multi-key warps, C = M: every centre a candidate
+    (256, 40, 8, 1, 100, 0),     # multi-key warps, C > 32: near keys take the all-centre exact fallback
 ])
 def test_mid_sizes_bit_exact(orc, M, C, r, B, n_tok, pos):
     s = wl.spec("tiny", d=128, H_q=4, H_kv=2, M=M, r=r, B=B, T=n_tok, n_new=1, n_hist=64, Nq=0)
