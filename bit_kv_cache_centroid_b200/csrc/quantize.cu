@@ -260,7 +260,7 @@ __device__ __forceinline__ unsigned long long warp_min64(unsigned long long v) {
   return (static_cast<unsigned long long>(hi) << 32) | lo;
 }
 
-constexpr int kListLen = 15;   // listed centres per key in the decision by perturbations (slot 15: the limit)
+constexpr int kListLen = 15;   // listed centres per key in the decision by perturbations (slot 15: count and limit)
 
 // D_j = sum_c w_c (k_c - mu_jc)^2 by the definition's fp32 order; the key:
 // row kr of `rows` (bf16, chunks permuted like the centre table), mu_s: the
